@@ -1,0 +1,436 @@
+"""Pins of the CPU oracle against things other than itself: hand-worked values
+(tests/golden, each cited), library routines (torch float8, scipy), closed
+forms, invariants and brute force.  No GPU needed."""
+import itertools
+import math
+import os
+from collections import OrderedDict
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def _bf16_bits(a):
+    return synth.to_bf16(np.asarray(a, dtype=np.float32))
+
+
+def _bf16_val(b):
+    return synth.bf16_to_f32(np.asarray(b, dtype=np.uint16)).astype(np.float64)
+
+
+# Independent decode used by the tests: E2M1 from the golden table, E4M3 from torch.
+E2M1_GOLDEN = {int(c, 16): float(v) for c, v in _rows("e2m1_table.txt")}
+
+
+def _e4m3_torch(b):
+    return torch.tensor(np.asarray(b, dtype=np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def _dequant_independent(codes, scales, rows, K, ts):
+    codes = np.asarray(codes, dtype=np.uint8).reshape(rows, K // 2)
+    lo, hi = codes & 0xF, codes >> 4
+    nib = np.empty((rows, K), dtype=np.uint8)
+    nib[:, 0::2], nib[:, 1::2] = lo, hi
+    vals = np.vectorize(E2M1_GOLDEN.get)(nib).astype(np.float64)
+    sc = _e4m3_torch(np.asarray(scales).reshape(rows, K // 16))
+    return vals * np.repeat(sc, 16, axis=1) * ts
+
+
+def _matrices_independent(rec, d, F):
+    off = synth.record_layout(d, F)  # the generator's layout: written separately from the oracle's
+    ts = np.frombuffer(rec[off[4]:off[4] + 12].tobytes(), dtype=np.float32).astype(np.float64)
+    w13c, w13s = rec[off[0]:off[0] + F * d], rec[off[1]:off[1] + F * d // 8]
+    W13 = _dequant_independent(w13c, w13s, 2 * F, d, 1.0)
+    W1, W3 = W13[0::2] * ts[0], W13[1::2] * ts[1]
+    W2 = _dequant_independent(rec[off[2]:off[2] + d * F // 2], rec[off[3]:off[3] + d * F // 16],
+                              d, F, ts[2])
+    return W1, W3, W2
+
+
+# ------------------------------------------------------------ formats --
+def test_e2m1_matches_hand_table():
+    for code, val in E2M1_GOLDEN.items():
+        got = oracle.e2m1(code)
+        assert got == val and math.copysign(1, got) == math.copysign(1, val), code
+
+
+def test_e4m3_hand_points():
+    for b, v in _rows("e4m3_points.txt"):
+        assert oracle.e4m3(int(b, 16)) == float(v), b
+
+
+def test_e4m3_exhaustive_vs_torch():
+    ref = _e4m3_torch(np.arange(256))
+    for b in range(256):
+        got = oracle.e4m3(b)
+        if math.isnan(ref[b]):
+            assert math.isnan(got), b
+        else:
+            assert got == ref[b], (b, got, ref[b])
+
+
+def test_nvfp4_worked_example():
+    (cb, sb, ts, ev, od), = _rows("nvfp4_worked_example.txt")
+    d, F = 64, 64
+    off = oracle.record_layout(d, F)
+    rec = np.zeros(off[5], dtype=np.uint8)
+    # element (row 2j=gate_j, K) with j = 3, K = 2i = 20 -> byte 10 of W13 row 6
+    j, i = 3, 10
+    rec[off[0] + (2 * j) * (d // 2) + i] = int(cb, 16)
+    rec[off[1] + (2 * j) * (d // 16) + (2 * i) // 16] = int(sb, 16)
+    rec[off[4]:off[4] + 12] = np.frombuffer(np.array([float(ts)] * 3, np.float32).tobytes(),
+                                            np.uint8)
+    W1 = oracle.dequant_matrix(rec, d, F, 0)
+    assert W1[j, 2 * i] == float(ev) and W1[j, 2 * i + 1] == float(od)
+    assert np.count_nonzero(W1) == 2 and np.count_nonzero(oracle.dequant_matrix(rec, d, F, 1)) == 0
+
+
+def test_record_bytes_golden():
+    for d, F, nb in _rows("record_bytes.txt"):
+        assert oracle.record_layout(int(d), int(F))[5] == int(nb)
+        assert synth.record_bytes(int(d), int(F)) == int(nb)
+
+
+def test_dequant_layout_random_record():
+    rng = np.random.default_rng(1)
+    d, F = 128, 192
+    off = oracle.record_layout(d, F)
+    rec = rng.integers(0, 256, off[5], dtype=np.uint8)
+    for o, n in ((off[1], 2 * F * d // 16), (off[3], d * F // 16)):  # finite scales only
+        s = rec[o:o + n]
+        s[(s & 0x7F) == 0x7F] = 0x38
+    rec[off[4]:off[4] + 12] = np.frombuffer(np.array([0.5, 0.25, 2.0], np.float32).tobytes(),
+                                            np.uint8)
+    W1, W3, W2 = _matrices_independent(rec, d, F)
+    np.testing.assert_array_equal(oracle.dequant_matrix(rec, d, F, 0), W1)
+    np.testing.assert_array_equal(oracle.dequant_matrix(rec, d, F, 1), W3)
+    np.testing.assert_array_equal(oracle.dequant_matrix(rec, d, F, 2), W2)
+
+
+# ------------------------------------------------------------ routing --
+def test_logits_exact_rational():
+    rng = np.random.default_rng(2)
+    E, d = 5, 32
+    Wr = _bf16_bits(rng.normal(0, 0.5, (E, d)))
+    x = _bf16_bits(rng.normal(0, 1, (1, d)))
+    _, _, z, _ = oracle.route(Wr, x, 2)
+    for e in range(E):
+        exact = sum(Fraction(float(a)) * Fraction(float(b))
+                    for a, b in zip(_bf16_val(Wr[e]), _bf16_val(x[0])))
+        assert abs(z[0, e] - float(exact)) <= 1e-15 * max(1.0, abs(float(exact)))
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+def test_topk_bruteforce_subsets(k):
+    rng = np.random.default_rng(10 + k)
+    E, d, T = 16, 64, 24
+    Wr = _bf16_bits(rng.normal(0, 0.1, (E, d)))
+    x = _bf16_bits(rng.normal(0, 1, (T, d)))
+    idx, gates, z, gap = oracle.route(Wr, x, k)
+    for t in range(T):
+        best = max(itertools.combinations(range(E), k), key=lambda s: sum(z[t, list(s)]))
+        assert tuple(idx[t]) == tuple(sorted(best))
+        assert abs(gates[t].sum() - 1.0) < 1e-12
+        # closed form of the renormalised gates: ratios are exp of logit differences
+        for a, b in itertools.combinations(range(k), 2):
+            assert gates[t, a] / gates[t, b] == pytest.approx(
+                math.exp(z[t, idx[t, a]] - z[t, idx[t, b]]), rel=1e-12)
+        zs = np.sort(z[t])[::-1]
+        if k < E:
+            assert gap[t] == zs[k - 1] - zs[k]
+
+
+def test_gates_without_renorm_are_softmax_probabilities():
+    rng = np.random.default_rng(3)
+    E, d = 16, 64
+    Wr = _bf16_bits(rng.normal(0, 0.1, (E, d)))
+    x = _bf16_bits(rng.normal(0, 1, (3, d)))
+    idx, p, z, _ = oracle.route(Wr, x, E, renorm=False)  # k = E: every probability
+    np.testing.assert_array_equal(idx, np.tile(np.arange(E), (3, 1)))
+    np.testing.assert_allclose(p.sum(1), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(p, torch.softmax(torch.tensor(z), dim=1).numpy(), rtol=1e-12)
+
+
+def test_topk_ties_go_to_lower_id():
+    d = 32
+    row = _bf16_bits(np.linspace(-1, 1, d))
+    Wr = np.stack([row * 0, row, row, row, row * 0])  # experts 1,2,3 tie
+    x = _bf16_bits(np.linspace(-1, 1, d)[None])
+    idx, _, _, gap = oracle.route(Wr, x, 2)
+    assert tuple(idx[0]) == (1, 2) and gap[0] == 0.0
+
+
+# --------------------------------------------------------- expert FFN --
+def test_expert_one_hot_input_closed_form():
+    d, F = 128, 256
+    rec = synth.expert_record(0, 5, d, F)
+    W1, W3, W2 = _matrices_independent(rec, d, F)
+    K = 37
+    x = np.zeros(d, dtype=np.uint16)
+    x[K] = _bf16_bits([1.0])[0]
+    y, h = oracle.expert_w4a16(rec, d, F, x)
+    g, u = W1[:, K], W3[:, K]
+    h_ref = g * expit(g) * u
+    np.testing.assert_allclose(h, h_ref, rtol=1e-13, atol=1e-300)
+    np.testing.assert_allclose(y, W2 @ h_ref, rtol=1e-10, atol=1e-14)
+
+
+def test_expert_dense_reference():
+    d, F = 256, 512
+    rec = synth.expert_record(0, 1, d, F)
+    W1, W3, W2 = _matrices_independent(rec, d, F)
+    x = _bf16_bits(np.random.default_rng(4).normal(0, 1, d))
+    xv = _bf16_val(x)
+    y, h = oracle.expert_w4a16(rec, d, F, x)
+    g, u = W1 @ xv, W3 @ xv
+    np.testing.assert_allclose(h, g * expit(g) * u, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(y, W2 @ (g * expit(g) * u), rtol=1e-9, atol=1e-12)
+
+
+def test_silu_special_values():
+    d, F = 64, 64
+    off = oracle.record_layout(d, F)
+    rec = np.zeros(off[5], dtype=np.uint8)
+    rec[off[4]:off[4] + 12] = np.frombuffer(np.array([1, 1, 1], np.float32).tobytes(), np.uint8)
+    x = _bf16_bits(np.ones(d))
+    y, h = oracle.expert_w4a16(rec, d, F, x)  # all-zero codes: silu(0) * 0 = 0
+    assert not h.any() and not y.any()
+
+
+def test_layer_combine_special_cases():
+    s = synth.TINY
+    P = s.L * s.E
+    rb = synth.record_bytes(s.d, s.F)
+    pool = np.concatenate([synth.expert_record(0, e, s.d, s.F) for e in range(s.E)])
+    Wr = synth.router_bf16(0, s.E, s.d)
+    shared = synth.expert_record(0, 0, s.d, s.F, shared=True)
+    x = _bf16_bits(np.random.default_rng(5).normal(0, 1, (3, s.d)))
+    # top-1 with renormalisation: gate 1, y = E_e(x)
+    idx, g, y = oracle.moe_layer(pool, P, 0, s.E, s.d, s.F, 1, Wr, None, x)
+    np.testing.assert_array_equal(g, 1.0)
+    for t in range(3):
+        e = idx[t, 0]
+        np.testing.assert_array_equal(y[t], oracle.expert_w4a16(pool[e * rb:(e + 1) * rb],
+                                                                s.d, s.F, x[t])[0])
+    # the shared expert adds with unit weight
+    _, _, y0 = oracle.moe_layer(pool, P, 0, s.E, s.d, s.F, 2, Wr, None, x)
+    _, _, y1 = oracle.moe_layer(pool, P, 0, s.E, s.d, s.F, 2, Wr, shared, x)
+    for t in range(3):
+        np.testing.assert_allclose(y1[t] - y0[t], oracle.expert_w4a16(shared, s.d, s.F, x[t])[0],
+                                   rtol=1e-9, atol=1e-12)
+    # pool aliasing: record of (layer, e) is (layer*E + e) mod P
+    _, _, ya = oracle.moe_layer(pool[:5 * rb], 5, 0, s.E, s.d, s.F, 1, Wr, None, x)
+    for t in range(3):
+        e = idx[t, 0] % 5
+        np.testing.assert_array_equal(ya[t], oracle.expert_w4a16(pool[e * rb:(e + 1) * rb],
+                                                                 s.d, s.F, x[t])[0])
+
+
+# ------------------------------------------------------------ LRU ------
+def test_lru_hand_trace():
+    rows = _rows("lru_hand_trace.txt")
+    lru = oracle.LRU(1, 16, 4)
+    hits = misses = 0
+    for r in rows:
+        if r[0] == "final":
+            assert list(lru.state()[1]) == [int(v) for v in r[1].split(",")]
+            continue
+        req = [int(v) for v in r[1].split(",")]
+        want = [tuple(int(v) for v in ev.split(":")) for ev in r[2:]]
+        got = lru.batch(0, req)
+        assert got == want, (r, got)
+        hits += sum(g[2] for g in got)
+        misses += sum(1 - g[2] for g in got)
+    assert (misses, hits) == (7, 5)
+
+
+class _DictLRU:
+    """Brute-force LRU for the cross-check: an ordered dict of resident keys."""
+
+    def __init__(self, C):
+        self.C, self.od, self.free = C, OrderedDict(), list(range(C))
+
+    def batch(self, layer, E, experts):
+        out, keys = [], [layer * E + e for e in experts]
+        for key in keys:
+            if key in self.od:
+                self.od.move_to_end(key)
+        for e, key in zip(experts, keys):
+            if key in self.od:
+                out.append((e, self.od[key], 1, -1))
+                continue
+            if self.free:
+                slot, ev = self.free.pop(0), -1
+            else:
+                ev, slot = self.od.popitem(last=False)
+            self.od[key] = slot
+            out.append((e, slot, 0, ev))
+        return out
+
+
+@pytest.mark.parametrize("L,E,C,k", [(1, 16, 4, 2), (3, 8, 5, 3), (4, 32, 40, 4), (2, 64, 64, 10)])
+def test_lru_matches_bruteforce_and_invariants(L, E, C, k):
+    rng = np.random.default_rng(L * 100 + C)
+    lru, ref = oracle.LRU(L, E, C), _DictLRU(C)
+    n_lookups = n_hits = 0
+    for step in range(300):
+        layer = int(rng.integers(L))
+        req = np.sort(rng.choice(E, size=min(k, C, E), replace=False)).astype(np.int32)
+        got = lru.batch(layer, req)
+        assert got == ref.batch(layer, E, [int(v) for v in req])
+        n_lookups += len(got)
+        n_hits += sum(g[2] for g in got)
+        m, owner, stamp, clock = lru.state()
+        res = np.nonzero(owner >= 0)[0]
+        assert len(res) <= C
+        for s in res:
+            assert m[owner[s]] == s  # map/owner bijection
+        assert np.count_nonzero(m >= 0) == len(res)
+        assert clock == n_lookups  # one stamp per lookup
+    assert 0 < n_hits < n_lookups
+
+
+def test_lru_rejects_bad_batches():
+    lru = oracle.LRU(2, 8, 3)
+    for bad in ([3, 1], [1, 1], [9], [0, 1, 2, 3]):
+        with pytest.raises(ValueError):
+            lru.batch(0, bad)
+    with pytest.raises(ValueError):
+        lru.batch(2, [0])
+
+
+# ----------------------------------------------------------- planner --
+def test_planner_golden_cases():
+    for m, bp, bh, thr, mode, q in _rows("planner_cases.txt"):
+        r = oracle.plan_split(int(m), float(bp), float(bh), float(thr))
+        assert (r["mode"], r["q"], r["cpu"]) == (int(mode), int(q), int(m) - int(q))
+
+
+def test_planner_equal_finish_invariant():
+    rng = np.random.default_rng(6)
+    for _ in range(200):
+        m = int(rng.integers(1, 200))
+        bp = float(rng.uniform(5, 60))
+        bh = bp * float(rng.uniform(1.01, 8))
+        r = oracle.plan_split(m, bp, bh, 2.0)
+        qr = r["q_real"]
+        assert qr / bp == pytest.approx((m - qr) / (bh - bp), rel=1e-12)
+        assert qr / bp == pytest.approx(m / bh, rel=1e-12)
+        if bh / bp > 2.0:
+            assert r["q"] == math.floor(qr + 0.5) and r["mode"] == 1
+        else:
+            assert r["q"] == m and r["mode"] == 0
+
+
+# --------------------------------------------------------- quantizer --
+def test_e4m3_rne_vs_torch_including_ties():
+    pos = np.array([oracle.e4m3(b) for b in range(0x7F)])
+    mids = (pos[:-1] + pos[1:]) / 2
+    rng = np.random.default_rng(7)
+    samples = np.concatenate([pos, mids, rng.uniform(0, 448, 4000), rng.uniform(0, 0.02, 2000),
+                              [447.9, 448.0]]).astype(np.float32)
+    ref = torch.tensor(samples).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_rne(float(v)) for v in samples])
+    np.testing.assert_array_equal(got, ref)
+    assert oracle.e4m3_rne(1e6) == 0x7E and oracle.e4m3_rne(449.0) == 0x7E
+
+
+def test_e2m1_rne_midpoints_and_saturation():
+    # midpoint -> value: ties go to the even mantissa
+    for v, want in [(0.25, 0.0), (0.75, 1.0), (1.25, 1.0), (1.75, 2.0), (2.5, 2.0), (3.5, 4.0),
+                    (5.0, 4.0), (7.0, 6.0), (1e9, 6.0), (0.2, 0.0), (0.26, 0.5), (5.01, 6.0)]:
+        assert E2M1_GOLDEN[oracle.e2m1_rne(v)] == want, v
+        assert E2M1_GOLDEN[oracle.e2m1_rne(-v)] == -want, v
+    for c, val in E2M1_GOLDEN.items():  # every representable value maps back to itself
+        assert E2M1_GOLDEN[oracle.e2m1_rne(val)] == val
+
+
+def test_quantizer_round_trip_of_representable_blocks():
+    rng = np.random.default_rng(8)
+    nblk = 64
+    s_t = np.float32(2.0 ** -10)
+    codes = rng.integers(0, 16, (nblk, 16))
+    scales = rng.integers(1, 0x7F, nblk)
+    scales[0] = 0x7E
+    for b in range(nblk):  # every block holds a +-6 so its amax is 6 * scale * s_t
+        codes[b, rng.integers(16)] = 7 if rng.random() < 0.5 else 15
+    x = np.array([[E2M1_GOLDEN[c] * oracle.e4m3(s) * s_t for c in row]
+                  for row, s in zip(codes, scales)], dtype=np.float32).ravel()
+    assert oracle.tensor_scale(x) == s_t
+    qc, qs = oracle.nvfp4_quantize(x, s_t)
+    np.testing.assert_array_equal(qs, scales)
+    lo, hi = qc & 0xF, qc >> 4
+    got = np.empty(x.size, dtype=np.int64)
+    got[0::2], got[1::2] = lo, hi
+    want = codes.ravel().copy()
+    want[np.array([E2M1_GOLDEN[c] for c in want]) == 0.0] = got[
+        np.array([E2M1_GOLDEN[c] for c in want]) == 0.0]  # +-0 may carry either sign
+    np.testing.assert_array_equal(got, want)
+
+
+def test_w4a4_one_hot_row():
+    d, F = 128, 256
+    rec = synth.expert_record(0, 9, d, F)
+    W1, W3, W2 = _matrices_independent(rec, d, F)
+    K = 5
+    x = np.zeros(d, dtype=np.uint16)
+    x[K] = _bf16_bits([1.0])[0]
+    y = oracle.expert_w4a4(rec, d, F, x)
+    s = np.float32(1.0) / np.float32(2688.0)  # one-hot row: quantized x_K = 6 * 448 * s
+    xk = 6.0 * 448.0 * float(s)
+    g, u = W1[:, K] * xk, W3[:, K] * xk
+    h = (g * expit(g) * u).astype(np.float32)
+    sh = oracle.tensor_scale(h)
+    hc, hs = oracle.nvfp4_quantize(h, sh)
+    nib = np.empty(F, dtype=np.int64)
+    nib[0::2], nib[1::2] = hc & 0xF, hc >> 4
+    hq = np.array([E2M1_GOLDEN[c] for c in nib]) * np.repeat(_e4m3_torch(hs), 16) * float(sh)
+    np.testing.assert_allclose(y, W2 @ hq, rtol=1e-9, atol=1e-12)
+    # and the quantized h is within NVFP4's error of h
+    assert np.linalg.norm(hq - h) / np.linalg.norm(h) < 0.15
+
+
+# ----------------------------------------------------- generator sanity --
+def test_generator_weights_dequantize_near_draws():
+    d, F = 256, 512
+    rec = synth.expert_record(0, 2, d, F)
+    for m in range(3):
+        W = oracle.dequant_matrix(rec, d, F, m)
+        M = synth.expert_matrix_f32(0, 2, m, d, F).astype(np.float64)
+        assert np.linalg.norm(W - M) / np.linalg.norm(M) < 0.12
+        assert abs(M.std() - 0.02) < 0.001
+
+
+def test_ar1_statistics():
+    x, _ = synth.decode_hidden_bf16(0, 0, 400, 256)
+    xv = _bf16_val(x)
+    assert abs(xv.var() - 1.0) < 0.1
+    c = np.mean([np.corrcoef(xv[:-1, i], xv[1:, i])[0, 1] for i in range(256)])
+    assert abs(c - 0.9) < 0.03
+
+
+def test_layer_record_index_uses_layer_and_expert():
+    s = synth.TINY
+    L, P = 3, 3 * s.E - 5  # P < L*E: records alias modulo P
+    rb = synth.record_bytes(s.d, s.F)
+    pool = np.concatenate([synth.expert_record(i // s.E, i % s.E, s.d, s.F) for i in range(P)])
+    Wr = synth.router_bf16(2, s.E, s.d)
+    x = _bf16_bits(np.random.default_rng(9).normal(0, 1, (4, s.d)))
+    idx, _, y = oracle.moe_layer(pool, P, 2, s.E, s.d, s.F, 1, Wr, None, x)
+    for t in range(4):
+        r = (2 * s.E + idx[t, 0]) % P
+        np.testing.assert_array_equal(y[t], oracle.expert_w4a16(pool[r * rb:(r + 1) * rb],
+                                                                s.d, s.F, x[t])[0])
