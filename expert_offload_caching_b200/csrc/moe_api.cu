@@ -1,0 +1,667 @@
+// C ABI of the per-layer routed-expert step (declared in include/moe_offload.h).
+//
+// One layer (FreeToken offload backend, florigen.ai "FreeTokenは何をしているのか": experts
+// in host RAM, an LRU cache of expert slots on the GPU, misses sent over PCIe):
+//   compute stream:  route+top-k+lookup kernel -> gate/up and down GEMVs of the
+//                    hit experts and the shared expert (they run while the host
+//                    reads the miss list) -> per miss: wait for its copy event,
+//                    gate/up + down of that expert -> combine.
+//   host:            waits (bounded) for the device's miss list in mapped pinned
+//                    memory, then issues one cudaMemcpyAsync per miss on the copy
+//                    stream (pinned pool -> slot) with an event after each.
+//   copy stream:     the miss records, back to back.
+// A slot is only overwritten after the lookup that evicted it has run, i.e.
+// after every earlier kernel on the compute stream; copies of one slot are
+// ordered on the copy stream.
+#include <atomic>
+#include <chrono>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+#include <immintrin.h>
+
+#include "../../include/moe_offload.h"
+#include "moe_internal.cuh"
+
+using namespace moe;
+
+namespace {
+
+inline int64_t up256(int64_t x) { return (x + 255) / 256 * 256; }
+
+bool dims_valid(const moe_dims *d) {
+    return d && d->L > 0 && d->E > 0 && d->k > 0 && d->k <= d->E && d->d > 0 && d->F > 0 &&
+           d->max_rows > 0 && d->pool_records >= 0;
+}
+bool dims_supported(const moe_dims *d) {
+    return d->d % 64 == 0 && d->F % 64 == 0 && d->k <= kMaxK && d->E <= kMaxE &&
+           d->max_rows <= 4096 && (int64_t)d->L * d->E < (1ll << 31);
+}
+
+RecordLayout layout_of(const moe_dims *d) {
+    RecordLayout r;
+    const int64_t dd = d->d, ff = d->F;
+    r.w13_codes = 0;
+    r.w13_scales = r.w13_codes + up256(2 * ff * dd / 2);
+    r.w2_codes = r.w13_scales + up256(2 * ff * dd / 16);
+    r.w2_scales = r.w2_codes + up256(dd * ff / 2);
+    r.tscales = r.w2_scales + up256(dd * ff / 16);
+    r.bytes = up256(r.tscales + 12);
+    return r;
+}
+
+int decode_rows(const moe_dims *d) { return d->max_rows < kDecodeMaxRows ? d->max_rows : kDecodeMaxRows; }
+int max_jobs(const moe_dims *d, int T) {
+    int64_t n = (int64_t)T * d->k;
+    return (int)(n < d->E ? n : d->E);
+}
+
+// Workspace carve-up; with base == nullptr only sizes are computed.
+struct WsLayout {
+    int64_t z, idx, gates, jobs, n_jobs, ticket, rowrefs, xh, hh, part, xstage, ystage, total;
+};
+WsLayout ws_layout(const moe_dims *d) {
+    WsLayout w;
+    const int64_t T = decode_rows(d), k = d->k, E = d->E, dd = d->d, F = d->F;
+    int64_t o = 0;
+    auto take = [&](int64_t bytes) { int64_t r = o; o += up256(bytes); return r; };
+    w.z = take(T * E * 4);
+    w.idx = take(T * k * 4);
+    w.gates = take(T * k * 4);
+    w.jobs = take((int64_t)max_jobs(d, (int)T) * (int64_t)sizeof(Job));
+    w.n_jobs = take(4);
+    w.ticket = take(4);
+    w.rowrefs = take(T * k * (int64_t)sizeof(RowRef));
+    w.xh = take(T * 2 * dd * 2);
+    w.hh = take(T * (k + 1) * 2 * F * 2);
+    w.part = take(T * (k + 1) * dd * 4);
+    w.xstage = take((int64_t)d->max_rows * dd * 2);
+    w.ystage = take((int64_t)d->max_rows * dd * 4);
+    w.total = o;
+    return w;
+}
+
+struct TableLayout {
+    int64_t hdr, map, owner, stamp, prev, next, total;
+};
+TableLayout table_layout(const moe_dims *d, int64_t C) {
+    TableLayout t;
+    int64_t o = 0;
+    auto take = [&](int64_t bytes) { int64_t r = o; o += up256(bytes); return r; };
+    t.hdr = take(sizeof(TableHdr));
+    t.map = take((int64_t)d->L * d->E * 4);
+    t.owner = take(C * 4);
+    t.stamp = take(C * 8);
+    t.prev = take(C * 4);
+    t.next = take(C * 4);
+    t.total = o;
+    return t;
+}
+
+struct TimedLaunch {
+    int cls;
+    cudaEvent_t a, b;
+    double bytes;
+};
+
+}  // namespace
+
+struct moe_ctx {
+    moe_dims dims;
+    RecordLayout lay;
+    int64_t P = 0;
+    const uint8_t *pool = nullptr;
+    const __nv_bfloat16 *router_w = nullptr;
+    const uint8_t *shared_recs = nullptr;
+    uint8_t *ws = nullptr;
+    WsLayout wl;
+    DecodeWs dws;
+    cudaStream_t cs = nullptr, xs = nullptr;
+    // cache
+    uint8_t *arena = nullptr;
+    int64_t C = 0;
+    Table tab;
+    uint32_t flags = 0;
+    bool configured = false;
+    // miss list page
+    HostPage *page_h = nullptr, *page_d = nullptr;
+    int page_cap = 0;
+    uint32_t seq = 0;
+    std::vector<cudaEvent_t> miss_ev;
+    // state
+    moe_status state = MOE_OK;
+    std::string err;
+    moe_stats stats;
+    int last_T = 0;
+    // timing
+    bool timing = false;
+    std::vector<cudaEvent_t> ev_pool;
+    std::vector<TimedLaunch> pending;
+    // injection and limits
+    int64_t inj_copy_fail_at = 0, inj_drop_publish = 0;
+    double wait_limit = 60.0;
+};
+
+namespace {
+
+moe_status cuda_fail(moe_ctx *c, cudaError_t e, const char *what) {
+    if (c) {
+        c->err = std::string(what) + ": " + cudaGetErrorString(e);
+    }
+    return MOE_ERR_CUDA;
+}
+#define CK(call)                                                    \
+    do {                                                            \
+        cudaError_t e_ = (call);                                    \
+        if (e_ != cudaSuccess) return cuda_fail(ctx, e_, #call);    \
+    } while (0)
+
+cudaEvent_t pool_event(moe_ctx *ctx) {
+    if (!ctx->ev_pool.empty()) {
+        cudaEvent_t e = ctx->ev_pool.back();
+        ctx->ev_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+void time_begin(moe_ctx *ctx, TimedLaunch &tl, int cls) {
+    tl.cls = cls;
+    tl.a = tl.b = nullptr;
+    tl.bytes = 0;
+    if (!ctx->timing) return;
+    tl.a = pool_event(ctx);
+    cudaEventRecord(tl.a, ctx->cs);
+}
+// Returns the index of the pending record, or -1 when timing is off.
+long time_end(moe_ctx *ctx, TimedLaunch &tl, double bytes) {
+    if (!ctx->timing || !tl.a) return -1;
+    tl.b = pool_event(ctx);
+    cudaEventRecord(tl.b, ctx->cs);
+    tl.bytes = bytes;
+    ctx->pending.push_back(tl);
+    return (long)ctx->pending.size() - 1;
+}
+moe_status resolve_timing(moe_ctx *ctx) {
+    if (ctx->pending.empty()) return MOE_OK;
+    CK(cudaStreamSynchronize(ctx->cs));
+    for (auto &t : ctx->pending) {
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, t.a, t.b));
+        ctx->stats.kernel_ms[t.cls] += ms;
+        ctx->stats.kernel_launches[t.cls] += 1;
+        ctx->stats.kernel_bytes[t.cls] += t.bytes;
+        ctx->ev_pool.push_back(t.a);
+        ctx->ev_pool.push_back(t.b);
+    }
+    ctx->pending.clear();
+    return MOE_OK;
+}
+
+int pick_wpt(int K) {
+    int nsteps = (K / 64 + 3) / 4;
+    return nsteps >= 4 ? 4 : (nsteps >= 2 ? 2 : 1);
+}
+
+GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job) {
+    const moe_dims &D = ctx->dims;
+    GemvArgs g;
+    g.mode = mode;
+    g.jobs = ctx->dws.jobs;
+    g.n_jobs = ctx->dws.n_jobs;
+    g.rowrefs = ctx->dws.rowrefs;
+    g.only_job = only_job;
+    g.shared_slot = (only_job < 0 && D.has_shared) ? max_jobs(&D, T) : -1;
+    g.arena = ctx->arena;
+    g.rec_bytes = ctx->lay.bytes;
+    g.shared_rec = D.has_shared ? ctx->shared_recs + (int64_t)layer * ctx->lay.bytes : nullptr;
+    g.T = T;
+    g.k = D.k;
+    g.d = D.d;
+    g.F = D.F;
+    g.lay = ctx->lay;
+    g.act = mode == kGateUp ? ctx->dws.xh : ctx->dws.hh;
+    g.hh_out = ctx->dws.hh;
+    g.part_out = ctx->dws.part;
+    g.wpt = pick_wpt(mode == kGateUp ? D.d : D.F);
+    return g;
+}
+
+double w13_bytes(const moe_ctx *c) { return (double)(c->lay.w2_codes - c->lay.w13_codes) + 8.0; }
+double w2_bytes(const moe_ctx *c) { return (double)(c->lay.tscales - c->lay.w2_codes) + 4.0; }
+
+moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
+                          moe_layer_trace *trace) {
+    const moe_dims &D = ctx->dims;
+    const uint32_t seq = ++ctx->seq;
+    RouteArgs ra;
+    ra.Wr = ctx->router_w + (size_t)layer * D.E * D.d;
+    ra.x = static_cast<const __nv_bfloat16 *>(x);
+    ra.T = T;
+    ra.E = D.E;
+    ra.d = D.d;
+    ra.k = D.k;
+    ra.renorm = D.renormalize;
+    ra.layer = layer;
+    ra.ws = ctx->dws;
+    ra.tab = ctx->tab;
+    ra.page = ctx->page_d;
+    ra.seq = seq;
+    ra.publish = 1;
+    if (ctx->inj_drop_publish > 0) {
+        ra.publish = 0;
+        --ctx->inj_drop_publish;
+    }
+    TimedLaunch tl;
+    time_begin(ctx, tl, MOE_K_ROUTE);
+    CK(launch_route_lookup(ra, ctx->cs));
+    time_end(ctx, tl, (double)D.E * D.d * 2 + (double)T * D.d * 2);
+
+    // hit experts and the shared expert, before the miss list is known
+    const int nj = max_jobs(&D, T);
+    const int grid_y = nj + (D.has_shared ? 1 : 0);
+    TimedLaunch tg, td;
+    time_begin(ctx, tg, MOE_K_GATEUP);
+    CK(launch_gemv(gemv_args(ctx, layer, T, kGateUp, -1), grid_y, ctx->cs));
+    const long ig = time_end(ctx, tg, 0);
+    time_begin(ctx, td, MOE_K_DOWN);
+    CK(launch_gemv(gemv_args(ctx, layer, T, kDown, -1), grid_y, ctx->cs));
+    const long id = time_end(ctx, td, 0);
+
+    // bounded host wait for the device's miss list
+    {
+        auto t0 = std::chrono::steady_clock::now();
+        uint64_t spins = 0;
+        while (ctx->page_h->seq != seq) {
+            _mm_pause();
+            if ((++spins & 4095) == 0) {
+                double el = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+                if (el > ctx->wait_limit) {
+                    ctx->state = MOE_ERR_STATE;
+                    ctx->err = "timed out waiting for the device miss list";
+                    return MOE_ERR_TIMEOUT;
+                }
+            }
+        }
+        std::atomic_thread_fence(std::memory_order_acquire);
+    }
+    const int nev = ctx->page_h->n_events;
+    const HostEvent *ev = ctx->page_h->ev;
+    int n_hit_jobs = 0;
+    for (int j = 0; j < nev; ++j) n_hit_jobs += ev[j].hit;
+    if (ig >= 0 && id >= 0) {  // algorithmic bytes of the two hit launches, now known
+        const int nexp = n_hit_jobs + (D.has_shared ? 1 : 0);
+        ctx->pending[ig].bytes = nexp * w13_bytes(ctx) + (double)T * D.d * 2;
+        ctx->pending[id].bytes = nexp * w2_bytes(ctx) + (double)T * D.F * 4;
+    }
+
+    // misses: one copy per record on the copy stream, an event after each
+    for (int j = 0; j < nev; ++j) {
+        if (ev[j].hit) continue;
+        if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
+            ctx->state = MOE_ERR_STATE;
+            ctx->err = "injected failure of an H2D copy issue";
+            return MOE_ERR_CUDA;
+        }
+        const int64_t rec_idx = ((int64_t)layer * D.E + ev[j].expert) % ctx->P;
+        CK(cudaMemcpyAsync(ctx->arena + (int64_t)ev[j].slot * ctx->lay.bytes,
+                           ctx->pool + rec_idx * ctx->lay.bytes, ctx->lay.bytes,
+                           cudaMemcpyHostToDevice, ctx->xs));
+        CK(cudaEventRecord(ctx->miss_ev[j], ctx->xs));
+        ctx->stats.h2d_copies += 1;
+        ctx->stats.h2d_bytes += ctx->lay.bytes;
+    }
+    for (int j = 0; j < nev; ++j) {
+        if (ev[j].hit) continue;
+        CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[j], 0));
+        TimedLaunch mg, md;
+        time_begin(ctx, mg, MOE_K_GATEUP);
+        CK(launch_gemv(gemv_args(ctx, layer, T, kGateUp, j), 1, ctx->cs));
+        time_end(ctx, mg, w13_bytes(ctx) + (double)T * D.d * 2);
+        time_begin(ctx, md, MOE_K_DOWN);
+        CK(launch_gemv(gemv_args(ctx, layer, T, kDown, j), 1, ctx->cs));
+        time_end(ctx, md, w2_bytes(ctx) + (double)T * D.F * 4);
+    }
+    TimedLaunch tc;
+    time_begin(ctx, tc, MOE_K_COMBINE);
+    CK(launch_combine(ctx->dws.part, ctx->dws.gates, y, T, D.k, D.d, D.has_shared, ctx->cs));
+    time_end(ctx, tc, (double)T * (D.k + 1) * D.d * 4 + (double)T * D.d * 4);
+
+    // trace and counters
+    int64_t hits = 0, evictions = 0;
+    for (int j = 0; j < nev; ++j) {
+        hits += ev[j].hit;
+        evictions += ev[j].evicted >= 0;
+    }
+    ctx->stats.lookups += nev;
+    ctx->stats.hits += hits;
+    ctx->stats.misses += nev - hits;
+    ctx->stats.evictions += evictions;
+    ctx->stats.forward_calls += 1;
+    if (trace) {
+        trace->count = nev;
+        const int n = nev < trace->capacity ? nev : trace->capacity;
+        for (int j = 0; j < n && trace->events; ++j) {
+            moe_cache_event &o = trace->events[j];
+            o.layer = layer;
+            o.expert = ev[j].expert;
+            o.slot = ev[j].slot;
+            o.hit = ev[j].hit;
+            o.evicted_key = ev[j].evicted;
+            o.prefetch = ev[j].prefetch;
+            o.reserved = 0;
+        }
+    }
+    ctx->last_T = T;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_record_bytes(const moe_dims *dims) {
+    if (!dims_valid(dims)) return 0;
+    return (size_t)layout_of(dims).bytes;
+}
+
+moe_status moe_record_layout(const moe_dims *dims, int64_t off[6]) {
+    if (!dims_valid(dims) || !off) return MOE_ERR_ARG;
+    RecordLayout r = layout_of(dims);
+    off[0] = r.w13_codes; off[1] = r.w13_scales; off[2] = r.w2_codes;
+    off[3] = r.w2_scales; off[4] = r.tscales; off[5] = r.bytes;
+    return MOE_OK;
+}
+
+size_t moe_workspace_bytes(const moe_dims *dims) {
+    if (!dims_valid(dims)) return 0;
+    return (size_t)ws_layout(dims).total;
+}
+
+size_t moe_arena_bytes(const moe_dims *dims, int64_t num_slots) {
+    if (!dims_valid(dims) || num_slots <= 0) return 0;
+    return (size_t)(up256(num_slots * layout_of(dims).bytes) + table_layout(dims, num_slots).total);
+}
+
+moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t host_pool_bytes,
+                          const void *router_w, const void *shared_recs, void *workspace,
+                          size_t workspace_bytes, void *compute_stream, void *copy_stream,
+                          moe_ctx **out) {
+    if (!out) return MOE_ERR_ARG;
+    *out = nullptr;
+    if (!dims_valid(dims) || !host_pool || !router_w || !workspace || !compute_stream ||
+        !copy_stream || (dims->has_shared && !shared_recs))
+        return MOE_ERR_ARG;
+    if (!dims_supported(dims)) return MOE_ERR_UNSUPPORTED;
+    const RecordLayout lay = layout_of(dims);
+    const int64_t P = dims->pool_records ? dims->pool_records : (int64_t)dims->L * dims->E;
+    if (P > (int64_t)dims->L * dims->E) return MOE_ERR_ARG;
+    if ((int64_t)host_pool_bytes < P * lay.bytes) return MOE_ERR_ARG;
+    if (workspace_bytes < moe_workspace_bytes(dims)) return MOE_ERR_ARG;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, host_pool) != cudaSuccess || attr.type != cudaMemoryTypeHost) {
+        cudaGetLastError();
+        return MOE_ERR_NOT_PINNED;
+    }
+    moe_ctx *ctx = new moe_ctx();
+    ctx->dims = *dims;
+    ctx->lay = lay;
+    ctx->P = P;
+    ctx->pool = static_cast<const uint8_t *>(host_pool);
+    ctx->router_w = static_cast<const __nv_bfloat16 *>(router_w);
+    ctx->shared_recs = static_cast<const uint8_t *>(shared_recs);
+    ctx->ws = static_cast<uint8_t *>(workspace);
+    ctx->wl = ws_layout(dims);
+    ctx->cs = static_cast<cudaStream_t>(compute_stream);
+    ctx->xs = static_cast<cudaStream_t>(copy_stream);
+    memset(&ctx->stats, 0, sizeof ctx->stats);
+    uint8_t *w = ctx->ws;
+    const WsLayout &L = ctx->wl;
+    ctx->dws.z = reinterpret_cast<float *>(w + L.z);
+    ctx->dws.idx = reinterpret_cast<int32_t *>(w + L.idx);
+    ctx->dws.gates = reinterpret_cast<float *>(w + L.gates);
+    ctx->dws.jobs = reinterpret_cast<Job *>(w + L.jobs);
+    ctx->dws.n_jobs = reinterpret_cast<int32_t *>(w + L.n_jobs);
+    ctx->dws.ticket = reinterpret_cast<uint32_t *>(w + L.ticket);
+    ctx->dws.rowrefs = reinterpret_cast<RowRef *>(w + L.rowrefs);
+    ctx->dws.xh = reinterpret_cast<__half *>(w + L.xh);
+    ctx->dws.hh = reinterpret_cast<__half *>(w + L.hh);
+    ctx->dws.part = reinterpret_cast<float *>(w + L.part);
+
+    ctx->page_cap = 2 * dims->E + 8;
+    const size_t page_bytes = sizeof(HostPage) + sizeof(HostEvent) * ctx->page_cap;
+    moe_status st = MOE_OK;
+    cudaError_t e = cudaHostAlloc(reinterpret_cast<void **>(&ctx->page_h), page_bytes, cudaHostAllocMapped);
+    if (e == cudaSuccess) e = cudaHostGetDevicePointer(reinterpret_cast<void **>(&ctx->page_d), ctx->page_h, 0);
+    if (e == cudaSuccess) {
+        memset((void *)ctx->page_h, 0, page_bytes);
+        ctx->miss_ev.resize(ctx->page_cap, nullptr);
+        for (auto &ev : ctx->miss_ev) {
+            e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+            if (e != cudaSuccess) break;
+        }
+    }
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs);
+    if (e != cudaSuccess) {
+        st = cuda_fail(ctx, e, "moe_layer_init");
+        moe_layer_destroy(ctx);
+        return st;
+    }
+    *out = ctx;
+    return MOE_OK;
+}
+
+moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, size_t arena_bytes,
+                           uint32_t flags) {
+    if (!ctx || !slot_arena || num_slots <= 0) return MOE_ERR_ARG;
+    const moe_dims &D = ctx->dims;
+    const int64_t need = max_jobs(&D, D.max_rows);
+    if (num_slots < need) return MOE_ERR_CAPACITY;
+    if ((flags & MOE_CACHE_PREFETCH_NEXT) && num_slots < 2ll * D.E) return MOE_ERR_CAPACITY;
+    if (num_slots >= (1ll << 31)) return MOE_ERR_ARG;
+    if (arena_bytes < moe_arena_bytes(&D, num_slots)) return MOE_ERR_ARG;
+    const bool reset = (flags & MOE_CACHE_RESET) || !ctx->configured || ctx->arena != slot_arena ||
+                       ctx->C != num_slots;
+    uint8_t *a = static_cast<uint8_t *>(slot_arena);
+    ctx->arena = a;
+    ctx->C = num_slots;
+    const TableLayout tl = table_layout(&D, num_slots);
+    uint8_t *tb = a + up256(num_slots * ctx->lay.bytes);
+    ctx->tab.hdr = reinterpret_cast<TableHdr *>(tb + tl.hdr);
+    ctx->tab.map = reinterpret_cast<int32_t *>(tb + tl.map);
+    ctx->tab.owner = reinterpret_cast<int32_t *>(tb + tl.owner);
+    ctx->tab.stamp = reinterpret_cast<unsigned long long *>(tb + tl.stamp);
+    ctx->tab.prev = reinterpret_cast<int32_t *>(tb + tl.prev);
+    ctx->tab.next = reinterpret_cast<int32_t *>(tb + tl.next);
+    ctx->tab.C = num_slots;
+    ctx->flags = flags & ~MOE_CACHE_RESET;
+    if (reset) {
+        // finish outstanding work of the old state first
+        CK(cudaStreamSynchronize(ctx->xs));
+        CK(cudaStreamSynchronize(ctx->cs));
+        CK(launch_table_reset(ctx->tab, (int64_t)D.L * D.E, ctx->cs));
+        CK(cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs));
+        ctx->pending.clear();
+        memset(&ctx->stats, 0, sizeof ctx->stats);
+        ctx->state = MOE_OK;
+        ctx->err.clear();
+    }
+    ctx->configured = true;
+    return MOE_OK;
+}
+
+moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
+                             moe_layer_trace *trace) {
+    if (!ctx) return MOE_ERR_ARG;
+    if (ctx->state != MOE_OK) return MOE_ERR_STATE;
+    if (!ctx->configured) return MOE_ERR_STATE;
+    const moe_dims &D = ctx->dims;
+    if (layer < 0 || layer >= D.L || T < 1 || T > D.max_rows || !x || !y) return MOE_ERR_ARG;
+    if (T <= kDecodeMaxRows) return forward_decode(ctx, layer, x, T, y, trace);
+    return MOE_ERR_UNSUPPORTED;
+}
+
+moe_status moe_layer_forward_host(moe_ctx *ctx, int32_t layer, const void *x_host, int32_t T,
+                                  float *y_host, moe_layer_trace *trace) {
+    if (!ctx) return MOE_ERR_ARG;
+    if (ctx->state != MOE_OK || !ctx->configured) return MOE_ERR_STATE;
+    const moe_dims &D = ctx->dims;
+    if (layer < 0 || layer >= D.L || T < 1 || T > D.max_rows || !x_host || !y_host) return MOE_ERR_ARG;
+    void *xd = ctx->ws + ctx->wl.xstage;
+    float *yd = reinterpret_cast<float *>(ctx->ws + ctx->wl.ystage);
+    CK(cudaMemcpyAsync(xd, x_host, (size_t)T * D.d * 2, cudaMemcpyHostToDevice, ctx->cs));
+    moe_status st = moe_layer_forward(ctx, layer, xd, T, yd, trace);
+    if (st != MOE_OK) return st;
+    CK(cudaMemcpyAsync(y_host, yd, (size_t)T * D.d * 4, cudaMemcpyDeviceToHost, ctx->cs));
+    return MOE_OK;
+}
+
+moe_status moe_get_routing(moe_ctx *ctx, int32_t *idx, float *gates, int32_t T) {
+    if (!ctx || T < 1 || T != ctx->last_T) return MOE_ERR_ARG;
+    CK(cudaStreamSynchronize(ctx->cs));
+    const size_t n = (size_t)T * ctx->dims.k;
+    if (idx) CK(cudaMemcpy(idx, ctx->dws.idx, n * 4, cudaMemcpyDeviceToHost));
+    if (gates) CK(cudaMemcpy(gates, ctx->dws.gates, n * 4, cudaMemcpyDeviceToHost));
+    return MOE_OK;
+}
+
+moe_status moe_cache_export(moe_ctx *ctx, int32_t *map, int32_t *owner, uint64_t *stamp,
+                            uint64_t *clock) {
+    if (!ctx || !ctx->configured) return MOE_ERR_ARG;
+    CK(cudaStreamSynchronize(ctx->cs));
+    const int64_t nk = (int64_t)ctx->dims.L * ctx->dims.E;
+    if (map) CK(cudaMemcpy(map, ctx->tab.map, nk * 4, cudaMemcpyDeviceToHost));
+    if (owner) CK(cudaMemcpy(owner, ctx->tab.owner, ctx->C * 4, cudaMemcpyDeviceToHost));
+    if (stamp) CK(cudaMemcpy(stamp, ctx->tab.stamp, ctx->C * 8, cudaMemcpyDeviceToHost));
+    if (clock) {
+        TableHdr h;
+        CK(cudaMemcpy(&h, ctx->tab.hdr, sizeof h, cudaMemcpyDeviceToHost));
+        *clock = h.clock;
+    }
+    return MOE_OK;
+}
+
+moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out) {
+    if (!ctx || !out) return MOE_ERR_ARG;
+    moe_status st = resolve_timing(ctx);
+    if (st != MOE_OK) return st;
+    *out = ctx->stats;
+    return MOE_OK;
+}
+
+moe_status moe_set_timing(moe_ctx *ctx, int32_t enable) {
+    if (!ctx) return MOE_ERR_ARG;
+    if (!enable) {
+        moe_status st = resolve_timing(ctx);
+        ctx->timing = false;
+        return st;
+    }
+    ctx->timing = true;
+    return MOE_OK;
+}
+
+moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds) {
+    if (!ctx || !(seconds > 0)) return MOE_ERR_ARG;
+    ctx->wait_limit = seconds;
+    return MOE_OK;
+}
+
+moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
+    if (!ctx || n < 0) return MOE_ERR_ARG;
+    if (what == 0) { ctx->inj_copy_fail_at = 0; ctx->inj_drop_publish = 0; }
+    else if (what == 1) ctx->inj_copy_fail_at = n;
+    else if (what == 2) ctx->inj_drop_publish = n;
+    else return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+moe_status plan_split(int32_t m, double B_P, double B_H, double threshold, double expert_bytes,
+                      moe_split *out) {
+    if (!out || m < 0 || !(B_P > 0) || !(B_H >= 0) || !(expert_bytes > 0)) return MOE_ERR_ARG;
+    const bool faster_host = B_H > B_P;
+    const double q_real = faster_host ? (double)m * B_P / B_H : (double)m;
+    const int32_t mode = (faster_host && B_H / B_P > threshold) ? 1 : 0;
+    int64_t q = mode ? (int64_t)(q_real + 0.5) : m;
+    if (q > m) q = m;
+    out->q = (int32_t)q;
+    out->cpu = m - (int32_t)q;
+    out->mode = mode;
+    out->reserved = 0;
+    out->q_real = q_real;
+    const double t_pcie = q * expert_bytes / B_P;
+    const double t_host = out->cpu > 0 ? out->cpu * expert_bytes / (B_H - B_P) : 0.0;
+    out->t_finish = t_pcie > t_host ? t_pcie : t_host;
+    return MOE_OK;
+}
+
+moe_status moe_measure_h2d(void *dev_buf, const void *host_buf, size_t bytes, size_t chunk_bytes,
+                           int32_t reps, void *stream, double *gbs) {
+    moe_ctx *ctx = nullptr;
+    if (!dev_buf || !host_buf || !bytes || reps < 1 || !stream || !gbs) return MOE_ERR_ARG;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, host_buf) != cudaSuccess || attr.type != cudaMemoryTypeHost) {
+        cudaGetLastError();
+        return MOE_ERR_NOT_PINNED;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t a, b;
+    CK(cudaEventCreate(&a));
+    CK(cudaEventCreate(&b));
+    const size_t chunk = chunk_bytes ? chunk_bytes : bytes;
+    double best = 0.0;
+    for (int r = 0; r < reps; ++r) {
+        CK(cudaEventRecord(a, s));
+        for (size_t o = 0; o < bytes; o += chunk) {
+            const size_t n = bytes - o < chunk ? bytes - o : chunk;
+            CK(cudaMemcpyAsync(static_cast<uint8_t *>(dev_buf) + o,
+                               static_cast<const uint8_t *>(host_buf) + o, n,
+                               cudaMemcpyHostToDevice, s));
+        }
+        CK(cudaEventRecord(b, s));
+        CK(cudaEventSynchronize(b));
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, a, b));
+        const double rate = (double)bytes / (ms * 1e-3) / 1e9;
+        if (rate > best) best = rate;
+    }
+    cudaEventDestroy(a);
+    cudaEventDestroy(b);
+    *gbs = best;
+    return MOE_OK;
+}
+
+const char *moe_status_str(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_NOT_PINNED: return "host pool is not page-locked";
+        case MOE_ERR_CAPACITY: return "cache too small";
+        case MOE_ERR_TIMEOUT: return "timed out waiting for the device";
+        case MOE_ERR_STATE: return "context needs a cache reset";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    }
+    return "unknown status";
+}
+
+const char *moe_last_error(const moe_ctx *ctx) { return ctx ? ctx->err.c_str() : ""; }
+
+void moe_layer_destroy(moe_ctx *ctx) {
+    if (!ctx) return;
+    if (ctx->cs) cudaStreamSynchronize(ctx->cs);
+    if (ctx->xs) cudaStreamSynchronize(ctx->xs);
+    for (auto &t : ctx->pending) {
+        if (t.a) cudaEventDestroy(t.a);
+        if (t.b) cudaEventDestroy(t.b);
+    }
+    for (auto e : ctx->ev_pool) cudaEventDestroy(e);
+    for (auto e : ctx->miss_ev)
+        if (e) cudaEventDestroy(e);
+    if (ctx->page_h) cudaFreeHost(ctx->page_h);
+    delete ctx;
+}
+
+}  // extern "C"

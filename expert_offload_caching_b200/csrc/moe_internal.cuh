@@ -1,0 +1,115 @@
+// Internal definitions shared by the kernels and the C-ABI host code.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+constexpr int kDecodeMaxRows = 32;  // T <= this takes the GEMV (decode) path
+constexpr int kMaxK = 32;
+constexpr int kMaxE = 1024;
+
+// Record sections (byte offsets), computed once per context.
+struct RecordLayout {
+    int64_t w13_codes, w13_scales, w2_codes, w2_scales, tscales, bytes;
+};
+
+// Device cache table, in the slot arena after the slots.  LRU order is kept
+// as a doubly linked list of resident slots (head = least recently used);
+// stamps (the global clock at last use) are kept alongside so the table can be
+// exported and checked against the min-stamp rule.
+struct TableHdr {
+    unsigned long long clock;
+    int32_t next_free;  // slots [next_free, C) have never been filled since the reset
+    int32_t head, tail; // LRU list ends, -1 when empty
+    int32_t pad[11];
+};
+
+struct Table {
+    TableHdr *hdr;
+    int32_t *map;               // [L*E] slot of key or -1
+    int32_t *owner;             // [C] key in slot or -1
+    unsigned long long *stamp;  // [C]
+    int32_t *prev, *next;       // [C] LRU list links
+    int64_t C;
+};
+
+// One distinct expert of a lookup batch, in ascending expert order.
+struct Job {
+    int32_t expert, slot, hit, nrows, row_off, pad[3];
+};
+// A (row, selection position) pair that uses a job's expert.
+struct RowRef {
+    int16_t t, p;
+};
+
+// Miss list published to the host through mapped pinned memory.
+struct HostEvent {
+    int32_t expert, slot, hit, prefetch;
+    int64_t evicted;
+};
+struct HostPage {
+    volatile uint32_t seq;  // written last by the device
+    int32_t n_events;
+    int32_t n_jobs;
+    int32_t n_misses;
+    int32_t pad[4];
+    HostEvent ev[1];        // [capacity]
+};
+
+// Device scratch of the decode path (carved from the caller's workspace).
+struct DecodeWs {
+    float *z;            // [maxT][E] router logits
+    int32_t *idx;        // [maxT][k]
+    float *gates;        // [maxT][k]
+    Job *jobs;           // [max_jobs]
+    int32_t *n_jobs;     // [1]
+    RowRef *rowrefs;     // [maxT*k]
+    __half *xh;          // [maxT][2][d] fp16 hi/lo split of x
+    __half *hh;          // [maxT][k+1][2][F] fp16 hi/lo split of h
+    float *part;         // [maxT][k+1][d] per-selection expert outputs (p = k: shared)
+    uint32_t *ticket;    // last-CTA counter
+};
+
+struct RouteArgs {
+    const __nv_bfloat16 *Wr;  // [E][d] of this layer
+    const __nv_bfloat16 *x;   // [T][d]
+    int T, E, d, k, renorm, layer;
+    DecodeWs ws;
+    Table tab;
+    HostPage *page;          // device alias of the mapped page
+    uint32_t seq;
+    int publish;
+};
+
+enum GemvMode { kGateUp = 0, kDown = 1 };
+
+struct GemvArgs {
+    int mode;
+    const Job *jobs;
+    const int32_t *n_jobs;
+    const RowRef *rowrefs;
+    int only_job;          // >= 0: process just this job; -1: every hit job (+ shared)
+    int shared_slot;       // gridDim.y index of the shared job, -1 if none
+    const uint8_t *arena;
+    int64_t rec_bytes;
+    const uint8_t *shared_rec;
+    int T, k, d, F;
+    RecordLayout lay;
+    const __half *act;     // gate_up: xh; down: hh
+    __half *hh_out;
+    float *part_out;
+    int wpt;               // warps per tile (1, 2 or 4)
+};
+
+// launchers (one per .cu)
+cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
+cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s);
+cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
+                           int has_shared, cudaStream_t s);
+cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
+cudaError_t launch_table_export(Table t, int64_t nkeys, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,237 @@
+/*
+ * moe_offload.h -- C ABI of the per-layer routed-expert step of an
+ * expert-offloading MoE engine (one B200, sm_100a).
+ *
+ * The step, per layer (FreeToken offload backend: experts live in host RAM,
+ * the GPU holds an LRU cache of expert slots and misses stream over PCIe --
+ * florigen.ai "FreeTokenは何をしているのか"; pirouter.ai "32 GB に 65 GB が載る仕組み"):
+ *   1. router logits z = W_r x, softmax, top-k, gates renormalised over the k;
+ *   2. lookup of the selected (layer, expert) pairs in one global LRU cache of
+ *      HBM slots (ai-hardware-zukan "GPUに載らない分をどう間に合わせるか";
+ *      gaming-st.com "技術的背景");
+ *   3. misses: the NVFP4 expert record is copied from the pinned host pool
+ *      into its slot (cudaMemcpyAsync on the copy stream), overlapped with the
+ *      hit experts' compute;
+ *   4. SwiGLU expert FFN over NVFP4 weights (florigen.ai "NVFP4で約135GBまで縮める":
+ *      E2M1 values with block scaling);
+ *   5. y = sum over selected experts in ascending id of g_e * E_e(x) + S(x)
+ *      (S = the layer's shared expert, weight 1, when present).
+ * For prefill chunks, the next layer's experts are streamed in while the
+ * current layer computes (holude.com "長いプロンプトとエージェント処理も意識している").
+ *
+ * Expert record (one contiguous block per (layer, expert); moe_record_layout):
+ *   [0] W13 codes  [2F x d/2] bytes; row 2j = gate_j, row 2j+1 = up_j; E2M1,
+ *                  two per byte, element 2i in the low nibble
+ *   [1] W13 scales [2F x d/16] E4M3 bytes, one per 16 consecutive elements of a row
+ *   [2] W2 codes   [d x F/2] bytes (row = output dim, K = F)
+ *   [3] W2 scales  [d x F/16]
+ *   [4] 3 fp32 tensor scales: gate, up, down
+ *   [5] total size; every section starts on a 256-byte boundary.
+ *   w = e2m1(code) * e4m3(scale) * tensor_scale.
+ *
+ * Conventions: all functions return a moe_status and never throw; pointers
+ * documented as "device" must be device memory of the current CUDA device;
+ * the library never allocates device memory -- the caller passes every
+ * device buffer.  The library owns only its context, a few CUDA events and
+ * one small mapped pinned page for the device-to-host miss list.
+ */
+#ifndef MOE_OFFLOAD_H
+#define MOE_OFFLOAD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_ARG = 1,         /* null pointer, bad size, layer or row count out of range */
+    MOE_ERR_CUDA = 2,        /* a CUDA runtime call failed; moe_last_error() has the text */
+    MOE_ERR_NOT_PINNED = 3,  /* the host pool is not page-locked (cudaHostAlloc/Register) */
+    MOE_ERR_CAPACITY = 4,    /* cache slots fewer than one lookup batch needs */
+    MOE_ERR_TIMEOUT = 5,     /* the host's wait for the device miss list ran out */
+    MOE_ERR_STATE = 6,       /* context unusable until cache_configure(..., MOE_CACHE_RESET) */
+    MOE_ERR_UNSUPPORTED = 7  /* shape outside what the kernels handle (see moe_layer_init) */
+} moe_status;
+
+/* Layer-stack dimensions.  L layers of E routed experts, top-k, hidden width d,
+ * expert FFN width F (SwiGLU: gate and up [F x d], down [d x F]).
+ * has_shared: one always-used shared expert per layer (FreeToken pages: Qwen3.8-Flash-Next
+ * uses 10 routed + 1 shared per token, florigen.ai).  renormalize: gates are
+ * the softmax renormalised over the selected k (1) or the plain softmax probabilities (0).
+ * max_rows: largest T passed to moe_layer_forward.
+ * pool_records: P, the records in the host pool; expert (l, e) is record (l*E + e) mod P;
+ * 0 means P = L*E. */
+typedef struct {
+    int32_t L, E, k, d, F;
+    int32_t has_shared;
+    int32_t renormalize;
+    int32_t max_rows;
+    int64_t pool_records;
+} moe_dims;
+
+typedef struct moe_ctx moe_ctx; /* opaque, library-owned host state */
+
+/* One cache event of a lookup batch. key = layer*E + expert. */
+typedef struct {
+    int32_t layer, expert, slot, hit; /* hit: 1 = hit, 0 = miss (slot newly filled) */
+    int64_t evicted_key;              /* key evicted from slot, -1 if the slot was free */
+    int32_t prefetch;                 /* 1 = entry of a next-layer prefetch batch */
+    int32_t reserved;
+} moe_cache_event;
+
+/* Caller-owned host array that moe_layer_forward fills with the call's cache
+ * events, in batch order (ascending expert id per batch).  count is set to the
+ * number of events; if capacity is smaller, only capacity are written and count
+ * still reports the total. */
+typedef struct {
+    moe_cache_event *events;
+    int32_t capacity;
+    int32_t count;
+} moe_layer_trace;
+
+/* Cumulative counters since the last MOE_CACHE_RESET.
+ * lookups/hits/misses count routed lookups (each distinct (layer, expert) of a
+ * batch once); prefetch_* count next-layer prefetch entries separately. */
+enum { MOE_K_ROUTE = 0, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE, MOE_K_PREFILL_ROUTE,
+       MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_COUNT };
+typedef struct {
+    int64_t lookups, hits, misses, evictions;
+    int64_t prefetch_lookups, prefetch_misses;
+    int64_t h2d_copies, h2d_bytes;
+    int64_t forward_calls;
+    /* with timing on (moe_set_timing): per kernel class, launches, summed device
+     * milliseconds (CUDA events on the launching stream) and algorithmic bytes */
+    int64_t kernel_launches[MOE_K_COUNT];
+    double kernel_ms[MOE_K_COUNT];
+    double kernel_bytes[MOE_K_COUNT];
+} moe_stats;
+
+/* Hybrid split plan (ai-hardware-zukan "GPUに載らない分をどう間に合わせるか";
+ * florigen.ai "CPU/PCIe ratio 1.70x"). */
+typedef struct {
+    int32_t q;        /* misses sent over PCIe */
+    int32_t cpu;      /* misses left to host-side processing (m - q) */
+    int32_t mode;     /* 0 = offload (all over PCIe), 1 = hybrid */
+    int32_t reserved;
+    double q_real;    /* m*B_P/B_H for B_H > B_P, else m */
+    double t_finish;  /* seconds until both sides finish, for experts of expert_bytes */
+} moe_split;
+
+/* cache_configure flags */
+#define MOE_CACHE_RESET 1u          /* empty the cache (cold start), zero the counters */
+#define MOE_CACHE_PREFETCH_NEXT 2u  /* prefill: stream layer l+1's experts during layer l */
+
+/* Bytes of one expert record; 0 if dims are invalid. */
+MOE_API size_t moe_record_bytes(const moe_dims *dims);
+
+/* Section offsets of one record into off[6] (see the layout above). */
+MOE_API moe_status moe_record_layout(const moe_dims *dims, int64_t off[6]);
+
+/* Device workspace bytes moe_layer_init needs for these dims (caller-owned). */
+MOE_API size_t moe_workspace_bytes(const moe_dims *dims);
+
+/* Device bytes of a slot arena of num_slots slots plus its cache table. */
+MOE_API size_t moe_arena_bytes(const moe_dims *dims, int64_t num_slots);
+
+/* Create a context.
+ *   host_pool: P expert records back to back, page-locked host memory
+ *              (else MOE_ERR_NOT_PINNED); read by DMA only; caller-owned, must
+ *              outlive the context; host_pool_bytes >= P * record bytes.
+ *   router_w:  device, bf16 [L][E][d] router weights.
+ *   shared_recs: device, L shared-expert records back to back (has_shared), else NULL.
+ *   workspace: device, >= moe_workspace_bytes(dims), caller-owned.
+ *   compute_stream, copy_stream: cudaStream_t handles (NULL = legacy stream not
+ *              accepted: pass real streams); work is issued on them only.
+ * Shapes handled: d and F multiples of 64, 1 <= k <= 32, k <= E <= 1024,
+ * 1 <= max_rows <= 4096; else MOE_ERR_UNSUPPORTED. */
+MOE_API moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t host_pool_bytes,
+                          const void *router_w, const void *shared_recs, void *workspace,
+                          size_t workspace_bytes, void *compute_stream, void *copy_stream,
+                          moe_ctx **out);
+
+/* Attach the HBM slot arena (device, >= moe_arena_bytes(dims, num_slots),
+ * caller-owned) holding num_slots expert slots and the cache table, and set
+ * flags.  MOE_CACHE_RESET (required the first time and after an error) empties
+ * the cache on the compute stream.  MOE_ERR_CAPACITY if num_slots < k * max_rows
+ * distinct experts could need (min(k*max_rows, E)), or, with
+ * MOE_CACHE_PREFETCH_NEXT, num_slots < 2*E. */
+MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, size_t arena_bytes,
+                           uint32_t flags);
+
+/* One MoE layer on T rows (1 <= T <= max_rows), stream-ordered on compute_stream.
+ *   x: device, bf16 [T][d] hidden states; y: device, fp32 [T][d] output.
+ *   trace: optional host struct filled with the cache events (NULL = none).
+ * Returns after the layer's copies and kernels are issued; y is valid when
+ * compute_stream reaches that point.  The call waits (host side, bounded) for
+ * the device's miss list; on timeout it returns MOE_ERR_TIMEOUT and the
+ * context is in MOE_ERR_STATE until a reset.  T <= 32 takes the decode path
+ * (NVFP4 dequant-GEMV, W4A16); larger T the prefill path (block-scaled NVFP4
+ * grouped GEMM, W4A4 with a per-row fp32 activation scale). */
+MOE_API moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
+                             moe_layer_trace *trace);
+
+/* Same step with HOST buffers: x_host bf16 [T][d] and y_host fp32 [T][d]
+ * (page-locked for asynchronous copies).  The copies run on compute_stream
+ * through the workspace; y_host is valid after compute_stream synchronises. */
+MOE_API moe_status moe_layer_forward_host(moe_ctx *ctx, int32_t layer, const void *x_host, int32_t T,
+                                  float *y_host, moe_layer_trace *trace);
+
+/* Routing of the last forward call: idx int32 [T][k] (ascending per row) and
+ * gates fp32 [T][k], host arrays.  Synchronises compute_stream. */
+MOE_API moe_status moe_get_routing(moe_ctx *ctx, int32_t *idx, float *gates, int32_t T);
+
+/* Copy of the device cache table: map int32 [L*E] (slot or -1), owner int32
+ * [num_slots] (key or -1), stamp uint64 [num_slots], clock.  Any may be NULL.
+ * Synchronises compute_stream. */
+MOE_API moe_status moe_cache_export(moe_ctx *ctx, int32_t *map, int32_t *owner, uint64_t *stamp,
+                            uint64_t *clock);
+
+/* Counters; resolves pending kernel timings (synchronises compute_stream if timing is on). */
+MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
+
+/* Per-kernel-class CUDA-event timing on (1) or off (0). */
+MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
+
+/* Longest host wait for the device miss list, in seconds (default 60). */
+MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
+
+/* Host-side fault injection for tests.  what = 1: the n-th H2D copy issue
+ * (counted from now, 1-based) fails with MOE_ERR_CUDA before it is issued;
+ * what = 2: the next n lookups do not publish their miss list, so the host
+ * wait runs out (MOE_ERR_TIMEOUT); what = 0 clears both. */
+MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
+
+/* Hybrid split: m missing experts, PCIe bandwidth B_P, host expert-processing
+ * bandwidth B_H (bytes/s), auto threshold (2.0 on the pages).  Equal finish
+ * times q/B_P = (m - q)/(B_H - B_P) give q = m*B_P/B_H when B_H > B_P; mode is
+ * hybrid iff B_H/B_P > threshold, and then q = round-half-up(q_real); in offload
+ * mode q = m.  expert_bytes sizes t_finish.  MOE_ERR_ARG for m < 0, B_P <= 0,
+ * B_H < 0 or expert_bytes <= 0.  Pure host function. */
+MOE_API moe_status plan_split(int32_t m, double B_P, double B_H, double threshold, double expert_bytes,
+                      moe_split *out);
+
+/* Pinned host -> device copy bandwidth (the roofline's H2D term; the pages'
+ * "ft bench bw" H2D line, florigen.ai): reps copies of `bytes` from host_buf
+ * (page-locked) to dev_buf on `stream`, timed with CUDA events; best rate in
+ * GB/s (1e9 B/s) into *gbs.  With chunk_bytes > 0 the copy is issued as
+ * back-to-back copies of chunk_bytes each (record-sized copies). */
+MOE_API moe_status moe_measure_h2d(void *dev_buf, const void *host_buf, size_t bytes, size_t chunk_bytes,
+                           int32_t reps, void *stream, double *gbs);
+
+MOE_API const char *moe_status_str(moe_status s);
+MOE_API const char *moe_last_error(const moe_ctx *ctx);
+MOE_API void moe_layer_destroy(moe_ctx *ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_OFFLOAD_H */

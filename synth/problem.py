@@ -1,0 +1,59 @@
+"""Assemble seeded synthetic workloads in host/device memory (inputs only).
+
+A workload is a LayerShape plus:
+  * the pinned host pool of P expert records (record i = routed expert
+    (i // E, i % E)); with ``distinct`` < P only the first ``distinct`` records
+    are generated and record i repeats record i mod distinct (same bytes,
+    same transfer cost; it bounds generation time for 64-156 GB pools);
+  * router weights, bf16 [L, E, d], on the device;
+  * shared-expert records [L] on the device (when the shape has them);
+  * hidden states: decode AR(1) chains or prefill rows, bf16.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (LayerShape, MASTER_SEED, decode_hidden_bf16, expert_record, expert_record_into,
+               record_bytes, replicate_records, router_bf16)
+
+
+def pinned_pool(shape: LayerShape, P: int | None = None, distinct: int | None = None,
+                seed: int = MASTER_SEED) -> torch.Tensor:
+    P = shape.L * shape.E if P is None else P
+    distinct = P if distinct is None else min(distinct, P)
+    rb = record_bytes(shape.d, shape.F)
+    pool = torch.empty(P * rb, dtype=torch.uint8, pin_memory=True)
+    base = pool.data_ptr()
+    for i in range(distinct):
+        expert_record_into(base + i * rb, i // shape.E, i % shape.E, shape.d, shape.F, seed=seed)
+    if distinct < P:
+        replicate_records(base, rb, distinct, P)
+    return pool
+
+
+def router_weights(shape: LayerShape, seed: int = MASTER_SEED) -> np.ndarray:
+    return np.stack([router_bf16(l, shape.E, shape.d, seed=seed) for l in range(shape.L)])
+
+
+def shared_records(shape: LayerShape, seed: int = MASTER_SEED) -> np.ndarray | None:
+    if not shape.shared:
+        return None
+    return np.concatenate([expert_record(l, 0, shape.d, shape.F, shared=True, seed=seed)
+                           for l in range(shape.L)])
+
+
+def to_device(a: np.ndarray | None, device="cuda") -> torch.Tensor | None:
+    if a is None:
+        return None
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def decode_inputs(shape: LayerShape, T: int, streams: int = 1, seed: int = MASTER_SEED,
+                  stream0: int = 0) -> np.ndarray:
+    """bf16 bits [T, L, streams, d]: one AR(1) chain per (stream, layer), no conditioning."""
+    out = np.empty((T, shape.L, streams, shape.d), dtype=np.uint16)
+    for s in range(streams):
+        for l in range(shape.L):
+            out[:, l, s, :] = decode_hidden_bf16(stream0 + s, l, T, shape.d, seed=seed)[0]
+    return out

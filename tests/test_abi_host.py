@@ -1,0 +1,99 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and its pure host functions (layout, sizes, planner, argument checks) agree
+with the oracle and the golden cases."""
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from expert_offload_caching_b200 import abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 18
+    L = abi.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(abi.EXPORTS) <= set(names)
+
+
+@pytest.mark.parametrize("shape", list(synth.SHAPES.values()), ids=lambda s: s.name)
+def test_record_layout_matches_oracle(shape):
+    d = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, shape.shared)
+    assert abi.moe_record_layout(d) == oracle.record_layout(shape.d, shape.F)
+    assert abi.moe_record_bytes(d) == synth.record_bytes(shape.d, shape.F)
+    assert abi.moe_workspace_bytes(d) > 0
+    a1, a2 = abi.moe_arena_bytes(d, 10), abi.moe_arena_bytes(d, 20)
+    assert a2 - a1 >= 10 * abi.moe_record_bytes(d)
+
+
+def _golden_rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def test_plan_split_golden_and_oracle():
+    for m, bp, bh, thr, mode, q in _golden_rows("planner_cases.txt"):
+        r = abi.plan_split(int(m), float(bp), float(bh), float(thr))
+        assert (r.mode, r.q, r.cpu) == (int(mode), int(q), int(m) - int(q))
+    rng = np.random.default_rng(0)
+    for _ in range(300):
+        m = int(rng.integers(0, 300))
+        bp = float(rng.uniform(1, 80))
+        bh = float(rng.uniform(0, 300))
+        eb = float(rng.uniform(1e5, 2e7))
+        r = abi.plan_split(m, bp, bh, 2.0, eb)
+        o = oracle.plan_split(m, bp, bh, 2.0, eb)
+        assert (r.q, r.cpu, r.mode) == (o["q"], o["cpu"], o["mode"])
+        assert r.q_real == pytest.approx(o["q_real"], rel=1e-15)
+        assert r.t_finish == pytest.approx(o["t_finish"], rel=1e-12)
+        if bh > bp:  # equal finish at the real-valued split
+            assert r.q_real / bp == pytest.approx((m - r.q_real) / (bh - bp), rel=1e-12, abs=1e-12)
+
+
+def test_plan_split_rejects_bad_arguments():
+    for args in [(-1, 10.0, 20.0), (3, 0.0, 20.0), (3, 10.0, -1.0), (3, float("nan"), 1.0)]:
+        with pytest.raises(abi.MoeError) as ei:
+            abi.plan_split(*args)
+        assert ei.value.status == abi.MOE_ERR_ARG
+    with pytest.raises(abi.MoeError):
+        abi.plan_split(3, 10.0, 20.0, 2.0, 0.0)
+
+
+def test_init_argument_checks_without_device():
+    good = abi.make_dims(2, 16, 2, 256, 512, max_rows=1)
+    fake = 0x1000  # never dereferenced: argument checks come first
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_layer_init(good, None, 1 << 30, fake, None, fake, 1 << 30, fake, fake)
+    assert ei.value.status == abi.MOE_ERR_ARG
+    bad_shape = abi.make_dims(2, 16, 2, 250, 512, max_rows=1)  # d not a multiple of 64
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_layer_init(bad_shape, fake, 1 << 30, fake, None, fake, 1 << 30, fake, fake)
+    assert ei.value.status == abi.MOE_ERR_UNSUPPORTED
+    too_many_k = abi.make_dims(2, 64, 33, 256, 512, max_rows=1)
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_layer_init(too_many_k, fake, 1 << 30, fake, None, fake, 1 << 30, fake, fake)
+    assert ei.value.status == abi.MOE_ERR_UNSUPPORTED
+    shared_missing = abi.make_dims(2, 16, 2, 256, 512, has_shared=True, max_rows=1)
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_layer_init(shared_missing, fake, 1 << 30, fake, None, fake, 1 << 30, fake, fake)
+    assert ei.value.status == abi.MOE_ERR_ARG
+    assert abi.moe_record_bytes(abi.make_dims(0, 16, 2, 256, 512)) == 0
+    assert abi.moe_status_str(abi.MOE_ERR_TIMEOUT) == "timed out waiting for the device"

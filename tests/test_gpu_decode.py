@@ -1,0 +1,213 @@
+"""Decode path on the GPU against the CPU oracle, through the C ABI.
+
+Bit-exact: expert indices, the cache event sequence (hit/miss, slot,
+evicted key), the table (map, owners, stamps, clock) and slot contents.
+Within 1e-3 relative L2: the layer outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import problem as sp
+from expert_offload_caching_b200 import abi
+from tests.gpu_problem import REL_L2_MAX, DecodeProblem, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+# Several GEMV tiles, ragged K tails (d = 960: 15 chunks of 64; F = 320: 5 chunks),
+# E not a multiple of 32, shared expert, 3 layers.
+MID = synth.LayerShape("mid", L=3, E=40, k=5, d=960, F=320, shared=True, tokens=24, cache_slots=12)
+
+
+def _check_run(pb: DecodeProblem, run, samples=None):
+    idx, gates = pb.oracle_routing()
+    want_events, lru = pb.oracle_trace(idx)
+    assert len(run.events) == len(want_events)
+    for g, w in zip(run.events, want_events):
+        assert g == w, (g, w)
+    m, o, s, c = lru.state()
+    np.testing.assert_array_equal(run.table[0], m)
+    np.testing.assert_array_equal(run.table[1], o)
+    np.testing.assert_array_equal(run.table[2], s)
+    assert run.table[3] == c
+    if run.idx is not None:
+        np.testing.assert_array_equal(run.idx, idx)
+        np.testing.assert_allclose(run.gates, gates, rtol=2e-5, atol=1e-7)
+    pairs = [(t, l) for t in range(pb.T) for l in range(pb.shape.L)] if samples is None else samples
+    y = run.y.cpu().numpy()
+    worst = 0.0
+    for t, l in pairs:
+        e = rel_l2(y[t, l], pb.oracle_y(t, l))
+        worst = max(worst, e)
+        assert e <= REL_L2_MAX, (t, l, e)
+    hits = sum(ev[4] for ev in run.events)
+    assert run.stats.lookups == len(run.events) and run.stats.hits == hits
+    assert run.stats.misses == len(run.events) - hits
+    return worst
+
+
+def test_tiny_decode_full_parity():
+    pb = DecodeProblem(synth.TINY, T=64)
+    run = pb.run(routing=True)
+    worst = _check_run(pb, run)
+    assert worst < 1e-5
+    pb.check_slots(pb._last_stack, run.table[1])
+    assert 0 < run.stats.misses < run.stats.lookups
+
+
+def test_mid_shape_multi_layer_shared_expert():
+    pb = DecodeProblem(MID, T=24)
+    run = pb.run(routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(pb._last_stack, run.table[1])
+
+
+@pytest.mark.parametrize("S", [2, 5, 16])
+def test_batched_decode_rows(S):
+    C = min(S * MID.k, MID.E) + 6
+    pb = DecodeProblem(MID, T=8, streams=S, C=C, stream0=100)
+    run = pb.run(routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(pb._last_stack, run.table[1])
+
+
+def test_all_resident_cache_has_no_misses_after_first_use():
+    pb = DecodeProblem(synth.TINY, T=40, C=synth.TINY.E)
+    run = pb.run()
+    _check_run(pb, run)
+    firsts = {}
+    for ev in run.events:
+        key = ev[2]
+        if key in firsts:
+            assert ev[4] == 1  # resident forever once loaded
+        else:
+            firsts[key] = ev
+            assert ev[4] == 0 and ev[5] == -1
+    assert run.stats.evictions == 0
+
+
+def test_topk_equal_to_E_and_top1():
+    for k in (1, 16):
+        sh = synth.LayerShape(f"tiny-k{k}", L=2, E=16, k=k, d=256, F=512, shared=False,
+                              tokens=6, cache_slots=16)
+        pb = DecodeProblem(sh, T=6)
+        run = pb.run(routing=True)
+        _check_run(pb, run)
+
+
+def test_host_io_path_matches_device_path():
+    pb = DecodeProblem(MID, T=6)
+    a = pb.run()
+    b = pb.run(host_io=True)
+    assert a.events == b.events
+    assert torch.equal(a.y, b.y)
+
+
+def test_cache_persists_across_calls_and_reset_clears_it():
+    pb = DecodeProblem(synth.TINY, T=20)
+    st = pb.stack()
+    r1 = pb.run(stack=st)
+    st.reset()
+    r2 = pb.run(stack=st)
+    assert r1.events == r2.events  # reset = cold start again
+    assert r2.stats.lookups == len(r2.events)  # counters restart at the reset
+
+
+@pytest.mark.parametrize("name,T,samples", [
+    ("gpt-oss-120b-shaped", 512, 6),
+    ("qwen3.8-flash-next-shaped", 256, 6),
+    ("deepseek-v4-flash-shaped", 256, 4),
+])
+def test_full_size_decode_trace_and_sampled_outputs(name, T, samples):
+    """The bench's configurations at full size and full token count: the whole
+    routing and cache trace bit-exact, outputs on sampled (token, layer) pairs.
+    The host pool holds 97 distinct records; expert (l, e) reads record
+    (l*E + e) mod 97 (the C ABI's pool aliasing)."""
+    sh = synth.SHAPES[name]
+    pb = DecodeProblem(sh, T=T, P=97)
+    run = pb.run()
+    rng = np.random.default_rng(1)
+    pairs = [(int(rng.integers(T)), int(rng.integers(sh.L))) for _ in range(samples)]
+    pairs.append((T - 1, sh.L - 1))
+    _check_run(pb, run, samples=pairs)
+    pb.check_slots(pb._last_stack, run.table[1], sample=24)
+    miss_rate = run.stats.misses / run.stats.lookups
+    assert 0.0 < miss_rate < 1.0
+
+
+def test_errors_capacity_and_unpinned_pool():
+    sh = synth.TINY
+    pb = DecodeProblem(sh, T=2)
+    st = pb.stack()
+    with pytest.raises(abi.MoeError) as ei:
+        abi.cache_configure(st.ctx, 1, st.arena, st.arena.numel(), abi.MOE_CACHE_RESET)
+    assert ei.value.status == abi.MOE_ERR_CAPACITY
+    with pytest.raises(abi.MoeError) as ei:  # prefetch needs two layers' worth of slots
+        abi.cache_configure(st.ctx, 4, st.arena, st.arena.numel(),
+                            abi.MOE_CACHE_RESET | abi.MOE_CACHE_PREFETCH_NEXT)
+    assert ei.value.status == abi.MOE_ERR_CAPACITY
+    pageable = np.zeros(pb.pool.numel(), dtype=np.uint8)
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_layer_init(pb.dims(), pageable, pageable.size, st.router_w, None, st.ws,
+                           st.ws.numel(), st.compute, st.copy)
+    assert ei.value.status == abi.MOE_ERR_NOT_PINNED
+    with pytest.raises(abi.MoeError) as ei:
+        st.forward(1, torch.zeros((1, sh.d), dtype=torch.uint16, device="cuda"),
+                   torch.zeros((1, sh.d), device="cuda"))
+    assert ei.value.status == abi.MOE_ERR_ARG
+
+
+def test_injected_timeout_then_reset_recovers():
+    pb = DecodeProblem(synth.TINY, T=10)
+    st = pb.stack()
+    abi.moe_set_wait_limit(st.ctx, 0.2)
+    abi.moe_debug_inject(st.ctx, 2, 1)  # the next lookup does not publish its miss list
+    x = torch.from_numpy(pb.x[0, 0]).cuda()
+    y = torch.zeros((1, pb.shape.d), device="cuda")
+    torch.cuda.synchronize()
+    with pytest.raises(abi.MoeError) as ei:
+        st.forward(0, x, y)
+    assert ei.value.status == abi.MOE_ERR_TIMEOUT
+    with pytest.raises(abi.MoeError) as ei:
+        st.forward(0, x, y)
+    assert ei.value.status == abi.MOE_ERR_STATE
+    st.reset()
+    abi.moe_set_wait_limit(st.ctx, 60.0)
+    run = pb.run(stack=st)
+    _check_run(pb, run)
+
+
+def test_injected_copy_failure_then_reset_recovers():
+    pb = DecodeProblem(synth.TINY, T=10)
+    st = pb.stack()
+    abi.moe_debug_inject(st.ctx, 1, 3)  # the third H2D copy issue fails
+    x = torch.from_numpy(pb.x[:, 0]).cuda()
+    y = torch.zeros((10, 1, pb.shape.d), device="cuda")
+    torch.cuda.synchronize()
+    failed = None
+    for t in range(10):
+        try:
+            st.forward(0, x[t], y[t])
+        except abi.MoeError as e:
+            failed = e
+            break
+    assert failed is not None and failed.status == abi.MOE_ERR_CUDA
+    with pytest.raises(abi.MoeError) as ei:
+        st.forward(0, x[0], y[0])
+    assert ei.value.status == abi.MOE_ERR_STATE
+    st.reset()
+    _check_run(pb, pb.run(stack=st))
+
+
+def test_h2d_measurement():
+    n = 256 << 20
+    h = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    gbs = abi.moe_measure_h2d(d, h, n, 0, 3, s)
+    gbs_rec = abi.moe_measure_h2d(d, h, n, synth.record_bytes(2880, 2880), 3, s)
+    assert 5.0 < gbs < 200.0 and 5.0 < gbs_rec < 200.0
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_measure_h2d(d, np.zeros(16, np.uint8), 16, 0, 1, s)
+    assert ei.value.status == abi.MOE_ERR_NOT_PINNED
