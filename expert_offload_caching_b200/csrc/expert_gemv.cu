@@ -7,40 +7,38 @@
 //   h_j = silu(g_j) * u_j,  g = W1 x, u = W3 x;   y_e = W2 h.
 //   y = sum over selected e (ascending id) of gate_e * y_e + y_shared.
 //
-// Decode is HBM-bound (1 row, weights read once).  The kernel streams each
-// weight row with 128-bit loads (L1 bypass) and keeps the instruction count
-// per byte low enough to stay memory-bound:
-//   * E2M1 codes are decoded in registers with cvt.rn.f16x2.e2m1x2 (2 per op);
-//   * each fp16 value is multiplied by its E4M3 block scale (cvt.rn.f16x2.e4m3x2);
-//     the product of an E2M1 and an E4M3 value is exact in fp16;
+// Decode is HBM-bound (a few rows, weights read once) and latency-bound when
+// one expert is processed alone.  So:
+//   * one CTA per 16-row weight tile; the tile's rows are contiguous in the
+//     record, so the CTA stages the whole tile into shared memory with 16-byte
+//     asynchronous copies (cp.async.cg, L1 bypassed) issued all at once.  No
+//     registers hold data in flight, and with ~26-41 KB per CTA several CTAs
+//     per SM keep ~200 KB per SM of HBM reads outstanding;
+//   * the 4 warps split the tile's K-steps of 256 elements;
+//   * E2M1 codes are decoded in registers with cvt.rn.f16x2.e2m1x2 (2 per op),
+//     then multiplied by the E4M3 block scale (cvt.rn.f16x2.e4m3x2); the
+//     product of an E2M1 and an E4M3 value is exact in fp16;
 //   * the dot products run on the tensor cores (mma.sync m16n8k16, fp16 in,
-//     fp32 accumulate): a warp's tile is 16 weight rows, the 8 mma columns
-//     carry up to 4 activation rows as fp16 (hi, lo) pairs, hi + lo == the
-//     fp32 (or bf16) value, so no precision is lost against fp32 FMAs.
-// Each thread owns one 64-element chunk (32 code bytes, 4 scale bytes) of two
-// tile rows per K-step; the four threads of an mma quad cover 256 consecutive
-// K.  The dot product is order-free, so logical k positions of the mma are
-// mapped onto each thread's own chunk, with the activations loaded at the same
-// positions.  A CTA of 4 warps splits the K-steps of one tile (or serves 2-4
-// tiles when K is short) and reduces in shared memory in a fixed order.
+//     fp32 accumulate): the 8 mma columns carry up to 4 activation rows as fp16
+//     (hi, lo) pairs, hi + lo == the fp32 (or bf16) value, so nothing is lost
+//     against fp32 FMAs.  The dot product is order-free: the mma's logical k
+//     positions are mapped onto each thread's own 64-element chunk, and the
+//     activations are loaded at the same positions;
+//   * K-split partial sums are reduced in shared memory in a fixed order;
+//   * the gate/up launch prefetches the expert's down-projection bytes into
+//     L2 (prefetch.global.L2), so the down launch reads L2;
+//   * the last down launch of a layer also does the combine: its last CTA
+//     (threadfence + ticket, no waiting) sums the partials in ascending id.
 #include "moe_internal.cuh"
 
 namespace moe {
 
 namespace {
 
-__device__ __forceinline__ uint4 ld_stream(const uint8_t *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ uint32_t ld_stream32(const uint8_t *p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
+// Prefetch [p, p + bytes) into L2, one 128-byte line per thread of the CTA.
+__device__ __forceinline__ void prefetch_l2_range(const uint8_t *p, uint32_t bytes) {
+    for (uint32_t o = threadIdx.x * 128u; o < bytes; o += blockDim.x * 128u)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p + o));
 }
 
 // 8 E2M1 codes (one 32-bit word, element 2i in the low nibble of byte i) ->
@@ -58,7 +56,7 @@ __device__ __forceinline__ void e2m1x8_to_f16(uint32_t w, uint32_t (&h)[4]) {
 
 __device__ __forceinline__ __half2 e4m3x2_to_h2(uint32_t v16) {
     uint32_t r;
-    uint16_t s = (uint16_t)v16;
+    const uint16_t s = (uint16_t)v16;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(s));
     return *reinterpret_cast<__half2 *>(&r);
 }
@@ -77,165 +75,222 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-constexpr int kGemvThreads = 128;
+constexpr int kGemvWarps = 4;
 
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+// 16-byte asynchronous copy global -> shared (L1 bypassed), tracked per thread.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// One K-step of one thread: 32 code bytes of each of its two tile rows (from
+// shared memory) and their 4 scale bytes each.  cv = false (the chunk lies past
+// the end of K) feeds zeros.  Every lane of the warp must call this together:
+// mma.sync is a warp-collective (.aligned) instruction.
 template <int NG>
-__global__ void __launch_bounds__(kGemvThreads) expert_gemv_kernel(GemvArgs a) {
+__device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, uint32_t sa, uint32_t sb,
+                                         int c, bool cv, const __half *const (&col)[NG],
+                                         const bool (&colv)[NG], int ngrp, float (&acc)[NG][4]) {
+    const __half2 a01 = e4m3x2_to_h2(sa & 0xffffu), a23 = e4m3x2_to_h2(sa >> 16);
+    const __half2 b01 = e4m3x2_to_h2(sb & 0xffffu), b23 = e4m3x2_to_h2(sb >> 16);
+    const __half2 sAv[4] = {__low2half2(a01), __high2half2(a01), __low2half2(a23), __high2half2(a23)};
+    const __half2 sBv[4] = {__low2half2(b01), __high2half2(b01), __low2half2(b23), __high2half2(b23)};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 qa = cv ? *reinterpret_cast<const uint4 *>(cA + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint4 qb = cv ? *reinterpret_cast<const uint4 *>(cB + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+        const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int w = 4 * h + u;  // 8 codes: elements 8w .. 8w+7 of the chunk
+            uint32_t fa[4], fb[4];
+            e2m1x8_to_f16(wa[u], fa);
+            e2m1x8_to_f16(wb[u], fb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                fa[j] = hmul2u(fa[j], sAv[w >> 1]);
+                fb[j] = hmul2u(fb[j], sBv[w >> 1]);
+            }
+#pragma unroll
+            for (int grp = 0; grp < NG; ++grp) {
+                if (grp < ngrp) {
+                    uint4 bv = make_uint4(0, 0, 0, 0);
+                    if (colv[grp] && cv) bv = __ldg(reinterpret_cast<const uint4 *>(col[grp] + 64 * c + 8 * w));
+                    mma16816(acc[grp], fa[0], fb[0], fa[1], fb[1], bv.x, bv.y);
+                    mma16816(acc[grp], fa[2], fb[2], fa[3], fb[3], bv.z, bv.w);
+                }
+            }
+        }
+    }
+}
+
+// One CTA (4 warps) per 16-row weight tile.  The tile's rows are contiguous in
+// the record; all threads stage it into shared memory with 16-byte cp.async
+// copies (the whole tile in flight at once), then the warps split the K-steps
+// of 256 elements and reduce in shared memory.  Dynamic shared memory: 16*K/2
+// code bytes + K scale bytes.
+template <int NG>
+__global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ float red[kGemvWarps][NG][4][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, q = lane & 3;
     const bool gate_up = a.mode == kGateUp;
 
     // ---- which expert (job) this CTA serves
-    const uint8_t *rec;
-    int nrows, row_off = 0;
-    bool shared = false;
+    const uint8_t *rec = nullptr;
+    int nrows = 0, row_off = 0;
+    bool shared = false, work = true;
     if (a.only_job < 0 && (int)blockIdx.y == a.shared_slot) {
         rec = a.shared_rec;
         nrows = a.T;
         shared = true;
     } else {
         const int jy = a.only_job >= 0 ? a.only_job : (int)blockIdx.y;
-        if (jy >= *a.n_jobs) return;
-        const Job jb = a.jobs[jy];
-        if (a.only_job < 0 && !jb.hit) return;
-        rec = a.arena + (int64_t)jb.slot * a.rec_bytes;
-        nrows = jb.nrows;
-        row_off = jb.row_off;
+        if (jy >= *a.n_jobs) {
+            work = false;
+        } else {
+            const Job jb = a.jobs[jy];
+            if (a.only_job < 0 && !jb.hit) {
+                work = false;
+            } else {
+                rec = a.arena + (int64_t)jb.slot * a.rec_bytes;
+                nrows = jb.nrows;
+                row_off = jb.row_off;
+            }
+        }
     }
 
     const int K = gate_up ? a.d : a.F;
-    const int NCH = K >> 6;
-    const int nsteps = (NCH + 3) >> 2;
     const int tiles = gate_up ? (a.F >> 3) : (a.d >> 4);
-    const int tpc = 4 / a.wpt;
-    const int tile = blockIdx.x * tpc + warp / a.wpt;
-    const int phase = warp % a.wpt;
-    const bool active = tile < tiles;
-
-    const int64_t rowA = gate_up ? 2 * (8 * tile + g) : 16 * tile + g;
-    const int64_t rowB = gate_up ? rowA + 1 : rowA + 8;
-    const uint8_t *codes = rec + (gate_up ? a.lay.w13_codes : a.lay.w2_codes);
-    const uint8_t *scales = rec + (gate_up ? a.lay.w13_scales : a.lay.w2_scales);
-    const uint8_t *cA = codes + rowA * (K >> 1), *cB = codes + rowB * (K >> 1);
-    const uint8_t *sA = scales + rowA * (K >> 4), *sB = scales + rowB * (K >> 4);
-    const float *ts = reinterpret_cast<const float *>(rec + a.lay.tscales);
-
-    __shared__ float red[4][NG][4][32];
-
-    for (int r0 = 0; r0 < nrows; r0 += 4 * NG) {
-        // B-operand column of this thread: mma column n = g carries activation row
-        // r0 + 4*grp + g/2, the hi (g even) or lo (g odd) fp16 part.
-        const __half *col[NG];
-        bool colv[NG];
-        int ngrp = 0;
-#pragma unroll
-        for (int grp = 0; grp < NG; ++grp) {
-            const int r = r0 + 4 * grp + (g >> 1);
-            colv[grp] = active && r < nrows;
-            col[grp] = a.act;
-            if (r0 + 4 * grp < nrows) ngrp = grp + 1;
-            if (colv[grp]) {
-                int t, p;
-                if (shared) { t = r; p = a.k; }
-                else { RowRef rr = a.rowrefs[row_off + r]; t = rr.t; p = rr.p; }
-                col[grp] = gate_up ? a.act + (size_t)t * 2 * a.d + (g & 1) * a.d
-                                   : a.act + (size_t)(t * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
-            }
+    const int tile = blockIdx.x;
+    if (work && tile < tiles) {
+        const int NCH = K >> 6;
+        const int nsteps = (NCH + 3) >> 2;
+        const uint32_t code_bytes = 16u * (uint32_t)(K >> 1), scale_bytes = (uint32_t)K;
+        uint8_t *s_codes = smem, *s_scales = smem + code_bytes;
+        const uint8_t *codes = rec + (gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)tile * code_bytes;
+        const uint8_t *scales = rec + (gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)tile * scale_bytes;
+        // stage the tile: every thread issues its 16-byte pieces, then waits for its own
+        const uint32_t n16c = code_bytes >> 4, n16s = scale_bytes >> 4;
+        for (uint32_t i = threadIdx.x; i < n16c; i += blockDim.x) cp_async16(s_codes + 16 * i, codes + 16 * i);
+        for (uint32_t i = threadIdx.x; i < n16s; i += blockDim.x) cp_async16(s_scales + 16 * i, scales + 16 * i);
+        if (gate_up) {  // this expert's down projection -> L2 for the down launch
+            const uint32_t total = (uint32_t)(a.lay.tscales - a.lay.w2_codes);
+            const uint32_t per = ((total / gridDim.x) + 127u) & ~127u;
+            const uint32_t off = per * blockIdx.x;
+            if (off < total) prefetch_l2_range(rec + a.lay.w2_codes + off, per < total - off ? per : total - off);
         }
-
-        float acc[NG][4];
+        const float *ts = reinterpret_cast<const float *>(rec + a.lay.tscales);
+        // tile-local rows of this thread: gate_up 2g (gate) / 2g+1 (up); down g / g+8
+        const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
+        cp_async_wait_all();
+        __syncthreads();
+        for (int r0 = 0; r0 < nrows; r0 += 4 * NG) {
+            // mma column n = g carries activation row r0 + 4*grp + g/2, the hi (g
+            // even) or lo (g odd) fp16 part.
+            const __half *col[NG];
+            bool colv[NG];
+            int ngrp = 0;
 #pragma unroll
-        for (int grp = 0; grp < NG; ++grp)
+            for (int grp = 0; grp < NG; ++grp) {
+                const int r = r0 + 4 * grp + (g >> 1);
+                colv[grp] = r < nrows;
+                col[grp] = a.act;
+                if (r0 + 4 * grp < nrows) ngrp = grp + 1;
+                if (colv[grp]) {
+                    int t, p;
+                    if (shared) { t = r; p = a.k; }
+                    else { const RowRef rr = a.rowrefs[row_off + r]; t = rr.t; p = rr.p; }
+                    col[grp] = gate_up ? a.act + (size_t)t * 2 * a.d + (g & 1) * a.d
+                                       : a.act + (size_t)(t * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
+                }
+            }
+            float acc[NG][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[grp][j] = 0.f;
-
-        if (active) {
-            for (int s = phase; s < nsteps; s += a.wpt) {
+            for (int grp = 0; grp < NG; ++grp)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[grp][j] = 0.f;
+            for (int s = warp; s < nsteps; s += kGemvWarps) {  // s is uniform across the warp
                 const int c = 4 * s + q;
-                const bool cv = c < NCH;
-                uint4 qa0 = make_uint4(0, 0, 0, 0), qa1 = qa0, qb0 = qa0, qb1 = qa0;
-                uint32_t sca = 0, scb = 0;
-                if (cv) {
-                    qa0 = ld_stream(cA + 32 * c);
-                    qa1 = ld_stream(cA + 32 * c + 16);
-                    qb0 = ld_stream(cB + 32 * c);
-                    qb1 = ld_stream(cB + 32 * c + 16);
-                    sca = ld_stream32(sA + 4 * c);
-                    scb = ld_stream32(sB + 4 * c);
-                }
-                const __half2 a01 = e4m3x2_to_h2(sca & 0xffffu), a23 = e4m3x2_to_h2(sca >> 16);
-                const __half2 b01 = e4m3x2_to_h2(scb & 0xffffu), b23 = e4m3x2_to_h2(scb >> 16);
-                const __half2 sAv[4] = {__low2half2(a01), __high2half2(a01), __low2half2(a23),
-                                        __high2half2(a23)};
-                const __half2 sBv[4] = {__low2half2(b01), __high2half2(b01), __low2half2(b23),
-                                        __high2half2(b23)};
-                const uint32_t wa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
-                const uint32_t wb[8] = {qb0.x, qb0.y, qb0.z, qb0.w, qb1.x, qb1.y, qb1.z, qb1.w};
-#pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    uint32_t fa[4], fb[4];
-                    e2m1x8_to_f16(wa[w], fa);
-                    e2m1x8_to_f16(wb[w], fb);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        fa[j] = hmul2u(fa[j], sAv[w >> 1]);
-                        fb[j] = hmul2u(fb[j], sBv[w >> 1]);
-                    }
-#pragma unroll
-                    for (int grp = 0; grp < NG; ++grp) {
-                        if (grp < ngrp) {
-                            uint4 bv = make_uint4(0, 0, 0, 0);
-                            if (colv[grp] && cv)
-                                bv = __ldg(reinterpret_cast<const uint4 *>(col[grp] + 64 * c + 8 * w));
-                            mma16816(acc[grp], fa[0], fb[0], fa[1], fb[1], bv.x, bv.y);
-                            mma16816(acc[grp], fa[2], fb[2], fa[3], fb[3], bv.z, bv.w);
-                        }
-                    }
-                }
+                const bool cv = c < NCH;  // ragged K tail: some lanes of the quad feed zeros
+                const int cc = cv ? c : 0;
+                const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
+                const uint32_t sb = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rB * (K >> 4) + 4 * c) : 0u;
+                step_mma<NG>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc, sa, sb, cc, cv,
+                             col, colv, ngrp, acc);
             }
-        }
-
-        // ---- reduce the K-split warps of a tile (fixed order), then the epilogue
-        if (a.wpt > 1) {
+            // ---- reduce the warps' partial sums (fixed order), then the epilogue
 #pragma unroll
             for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) red[warp][grp][j][lane] = acc[grp][j];
             __syncthreads();
-            if (phase == 0) {
-                for (int ph = 1; ph < a.wpt; ++ph)
+            if (warp == 0) {
+                for (int w = 1; w < kGemvWarps; ++w)
 #pragma unroll
                     for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) acc[grp][j] += red[warp + ph][grp][j][lane];
+                        for (int j = 0; j < 4; ++j) acc[grp][j] += red[w][grp][j][lane];
+#pragma unroll
+                for (int grp = 0; grp < NG; ++grp) {
+                    const int r = r0 + 4 * grp + q;  // this thread's results: activation row q
+                    if (r >= nrows) continue;
+                    int t, p;
+                    if (shared) { t = r; p = a.k; }
+                    else { const RowRef rr = a.rowrefs[row_off + r]; t = rr.t; p = rr.p; }
+                    const float v0 = acc[grp][0] + acc[grp][1];  // tile row rA
+                    const float v1 = acc[grp][2] + acc[grp][3];  // tile row rB
+                    const size_t sel = (size_t)t * (a.k + 1) + p;
+                    if (gate_up) {
+                        const float gt = ts[0] * v0, up = ts[1] * v1;
+                        const float h = gt / (1.0f + expf(-gt)) * up;
+                        const __half hi = __float2half_rn(h);
+                        const __half lo = __float2half_rn(h - __half2float(hi));
+                        const int j = 8 * tile + g;
+                        a.hh_out[sel * 2 * a.F + j] = hi;
+                        a.hh_out[sel * 2 * a.F + a.F + j] = lo;
+                    } else {
+                        const int i = 16 * tile + g;
+                        a.part_out[sel * a.d + i] = ts[2] * v0;
+                        a.part_out[sel * a.d + i + 8] = ts[2] * v1;
+                    }
+                }
             }
             __syncthreads();
         }
-        if (active && phase == 0) {
-#pragma unroll
-            for (int grp = 0; grp < NG; ++grp) {
-                const int r = r0 + 4 * grp + q;  // this thread's results: activation row q
-                if (r >= nrows) continue;
-                int t, p;
-                if (shared) { t = r; p = a.k; }
-                else { RowRef rr = a.rowrefs[row_off + r]; t = rr.t; p = rr.p; }
-                const float v0 = acc[grp][0] + acc[grp][1];  // tile row g
-                const float v1 = acc[grp][2] + acc[grp][3];  // tile row g + 8
-                const size_t sel = (size_t)t * (a.k + 1) + p;
-                if (gate_up) {
-                    const float gt = ts[0] * v0, up = ts[1] * v1;
-                    const float h = gt / (1.0f + expf(-gt)) * up;
-                    const __half hi = __float2half_rn(h);
-                    const __half lo = __float2half_rn(h - __half2float(hi));
-                    const int j = 8 * tile + g;
-                    a.hh_out[sel * 2 * a.F + j] = hi;
-                    a.hh_out[sel * 2 * a.F + a.F + j] = lo;
-                } else {
-                    const int i = 16 * tile + g;
-                    a.part_out[sel * a.d + i] = ts[2] * v0;
-                    a.part_out[sel * a.d + i + 8] = ts[2] * v1;
+    }
+
+    if (a.combine) {  // the launch's last CTA sums the partials of the layer
+        __shared__ int s_last;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            const unsigned int total = gridDim.x * gridDim.y;
+            s_last = (atomicAdd(a.ticket, 1u) == total - 1);
+        }
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            if (a.combine == 1 || *a.n_misses == 0) {
+                const int n = a.T * a.d;
+                for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                    const int t = i / a.d, c = i - t * a.d;
+                    const float *pr = a.part_out + (size_t)t * (a.k + 1) * a.d + c;
+                    float s = 0.f;
+                    for (int p = 0; p < a.k; ++p) s = fmaf(a.gates[t * a.k + p], pr[(size_t)p * a.d], s);
+                    if (a.shared_rec) s += pr[(size_t)a.k * a.d];
+                    a.y[i] = s;
                 }
             }
+            if (threadIdx.x == 0) *a.ticket = 0u;
         }
     }
 }
@@ -252,17 +307,30 @@ __global__ void combine_kernel(const float *__restrict__ part, const float *__re
     y[i] = acc;
 }
 
+template <int NG>
+cudaError_t launch_ng(const GemvArgs &a, dim3 grid, size_t smem, cudaStream_t s) {
+    static bool configured = false;  // per instantiation: allow > 48 KB of dynamic smem
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<NG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    expert_gemv_kernel<NG><<<grid, kGemvWarps * 32, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s) {
+    const int K = a.mode == kGateUp ? a.d : a.F;
     const int tiles = a.mode == kGateUp ? a.F / 8 : a.d / 16;
-    const int tpc = 4 / a.wpt;
-    dim3 grid((tiles + tpc - 1) / tpc, grid_y);
-    const int rows = a.T;
-    if (rows <= 4) expert_gemv_kernel<1><<<grid, kGemvThreads, 0, s>>>(a);
-    else if (rows <= 8) expert_gemv_kernel<2><<<grid, kGemvThreads, 0, s>>>(a);
-    else expert_gemv_kernel<4><<<grid, kGemvThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    const dim3 grid(tiles, grid_y);
+    const size_t smem = 16 * (size_t)(K / 2) + (size_t)K;
+    if (smem > 96 * 1024) return cudaErrorInvalidValue;
+    if (a.T <= 4) return launch_ng<1>(a, grid, smem, s);
+    if (a.T <= 8) return launch_ng<2>(a, grid, smem, s);
+    return launch_ng<4>(a, grid, smem, s);
 }
 
 cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,

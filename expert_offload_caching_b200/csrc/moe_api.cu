@@ -35,7 +35,8 @@ bool dims_valid(const moe_dims *d) {
            d->max_rows > 0 && d->pool_records >= 0;
 }
 bool dims_supported(const moe_dims *d) {
-    return d->d % 64 == 0 && d->F % 64 == 0 && d->k <= kMaxK && d->E <= kMaxE &&
+    return d->d % 64 == 0 && d->F % 64 == 0 && d->d <= 4096 && d->F <= 4096 && d->k <= kMaxK &&
+           d->E <= kMaxE &&
            d->max_rows <= 4096 && (int64_t)d->L * d->E < (1ll << 31);
 }
 
@@ -59,7 +60,8 @@ int max_jobs(const moe_dims *d, int T) {
 
 // Workspace carve-up; with base == nullptr only sizes are computed.
 struct WsLayout {
-    int64_t z, idx, gates, jobs, n_jobs, ticket, rowrefs, xh, hh, part, xstage, ystage, total;
+    int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, rowrefs, xh, hh, part, xstage,
+        ystage, total;
 };
 WsLayout ws_layout(const moe_dims *d) {
     WsLayout w;
@@ -71,7 +73,9 @@ WsLayout ws_layout(const moe_dims *d) {
     w.gates = take(T * k * 4);
     w.jobs = take((int64_t)max_jobs(d, (int)T) * (int64_t)sizeof(Job));
     w.n_jobs = take(4);
+    w.n_misses = take(4);
     w.ticket = take(4);
+    w.ticket2 = take(4);
     w.rowrefs = take(T * k * (int64_t)sizeof(RowRef));
     w.xh = take(T * 2 * dd * 2);
     w.hh = take(T * (k + 1) * 2 * F * 2);
@@ -201,12 +205,7 @@ moe_status resolve_timing(moe_ctx *ctx) {
     return MOE_OK;
 }
 
-int pick_wpt(int K) {
-    int nsteps = (K / 64 + 3) / 4;
-    return nsteps >= 4 ? 4 : (nsteps >= 2 ? 2 : 1);
-}
-
-GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job) {
+GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int combine = 0) {
     const moe_dims &D = ctx->dims;
     GemvArgs g;
     g.mode = mode;
@@ -226,19 +225,38 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job) {
     g.act = mode == kGateUp ? ctx->dws.xh : ctx->dws.hh;
     g.hh_out = ctx->dws.hh;
     g.part_out = ctx->dws.part;
-    g.wpt = pick_wpt(mode == kGateUp ? D.d : D.F);
+    g.page = ctx->page_d;
+    g.combine = combine;
+    g.n_misses = ctx->dws.n_misses;
+    g.gates = ctx->dws.gates;
+    g.y = nullptr;
+    g.ticket = ctx->dws.ticket2;
     return g;
 }
 
 double w13_bytes(const moe_ctx *c) { return (double)(c->lay.w2_codes - c->lay.w13_codes) + 8.0; }
 double w2_bytes(const moe_ctx *c) { return (double)(c->lay.tscales - c->lay.w2_codes) + 4.0; }
 
+// A kernel reported a failed self-check through the mapped page (error word
+// and a diagnostic record: check code, kernel mode, block, tile, sizes).
+moe_status device_error(moe_ctx *ctx) {
+    const volatile int32_t *dg = ctx->page_h->diag;
+    char buf[256];
+    snprintf(buf, sizeof buf, "device check %d failed: kernel mode %d, block (%d,%d), tile %d, sizes %d %d",
+             (int)ctx->page_h->error, dg[1], dg[2], dg[3], dg[4], dg[5], dg[6]);
+    ctx->err = buf;
+    ctx->state = MOE_ERR_STATE;
+    return MOE_ERR_CUDA;
+}
+
 moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
                           moe_layer_trace *trace) {
     const moe_dims &D = ctx->dims;
+    if (ctx->page_h->error) return device_error(ctx);
     const uint32_t seq = ++ctx->seq;
     RouteArgs ra;
     ra.Wr = ctx->router_w + (size_t)layer * D.E * D.d;
+    ra.Wr_next = layer + 1 < D.L ? ra.Wr + (size_t)D.E * D.d : nullptr;
     ra.x = static_cast<const __nv_bfloat16 *>(x);
     ra.T = T;
     ra.E = D.E;
@@ -268,7 +286,9 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     CK(launch_gemv(gemv_args(ctx, layer, T, kGateUp, -1), grid_y, ctx->cs));
     const long ig = time_end(ctx, tg, 0);
     time_begin(ctx, td, MOE_K_DOWN);
-    CK(launch_gemv(gemv_args(ctx, layer, T, kDown, -1), grid_y, ctx->cs));
+    GemvArgs hd = gemv_args(ctx, layer, T, kDown, -1, 2);  // combines when nothing missed
+    hd.y = y;
+    CK(launch_gemv(hd, grid_y, ctx->cs));
     const long id = time_end(ctx, td, 0);
 
     // bounded host wait for the device's miss list
@@ -288,10 +308,14 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         }
         std::atomic_thread_fence(std::memory_order_acquire);
     }
+    if (ctx->page_h->error) return device_error(ctx);
     const int nev = ctx->page_h->n_events;
     const HostEvent *ev = ctx->page_h->ev;
-    int n_hit_jobs = 0;
-    for (int j = 0; j < nev; ++j) n_hit_jobs += ev[j].hit;
+    int n_hit_jobs = 0, last_miss = -1;
+    for (int j = 0; j < nev; ++j) {
+        n_hit_jobs += ev[j].flags & 1;
+        if (!(ev[j].flags & 1)) last_miss = j;
+    }
     if (ig >= 0 && id >= 0) {  // algorithmic bytes of the two hit launches, now known
         const int nexp = n_hit_jobs + (D.has_shared ? 1 : 0);
         ctx->pending[ig].bytes = nexp * w13_bytes(ctx) + (double)T * D.d * 2;
@@ -300,7 +324,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
 
     // misses: one copy per record on the copy stream, an event after each
     for (int j = 0; j < nev; ++j) {
-        if (ev[j].hit) continue;
+        if (ev[j].flags & 1) continue;
         if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
             ctx->state = MOE_ERR_STATE;
             ctx->err = "injected failure of an H2D copy issue";
@@ -315,25 +339,23 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         ctx->stats.h2d_bytes += ctx->lay.bytes;
     }
     for (int j = 0; j < nev; ++j) {
-        if (ev[j].hit) continue;
+        if (ev[j].flags & 1) continue;
         CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[j], 0));
         TimedLaunch mg, md;
         time_begin(ctx, mg, MOE_K_GATEUP);
         CK(launch_gemv(gemv_args(ctx, layer, T, kGateUp, j), 1, ctx->cs));
         time_end(ctx, mg, w13_bytes(ctx) + (double)T * D.d * 2);
         time_begin(ctx, md, MOE_K_DOWN);
-        CK(launch_gemv(gemv_args(ctx, layer, T, kDown, j), 1, ctx->cs));
+        GemvArgs md_args = gemv_args(ctx, layer, T, kDown, j, j == last_miss ? 1 : 0);
+        md_args.y = y;
+        CK(launch_gemv(md_args, 1, ctx->cs));
         time_end(ctx, md, w2_bytes(ctx) + (double)T * D.F * 4);
     }
-    TimedLaunch tc;
-    time_begin(ctx, tc, MOE_K_COMBINE);
-    CK(launch_combine(ctx->dws.part, ctx->dws.gates, y, T, D.k, D.d, D.has_shared, ctx->cs));
-    time_end(ctx, tc, (double)T * (D.k + 1) * D.d * 4 + (double)T * D.d * 4);
 
     // trace and counters
     int64_t hits = 0, evictions = 0;
     for (int j = 0; j < nev; ++j) {
-        hits += ev[j].hit;
+        hits += ev[j].flags & 1;
         evictions += ev[j].evicted >= 0;
     }
     ctx->stats.lookups += nev;
@@ -349,9 +371,9 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
             o.layer = layer;
             o.expert = ev[j].expert;
             o.slot = ev[j].slot;
-            o.hit = ev[j].hit;
+            o.hit = ev[j].flags & 1;
             o.evicted_key = ev[j].evicted;
-            o.prefetch = ev[j].prefetch;
+            o.prefetch = (ev[j].flags >> 1) & 1;
             o.reserved = 0;
         }
     }
@@ -425,7 +447,9 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     ctx->dws.gates = reinterpret_cast<float *>(w + L.gates);
     ctx->dws.jobs = reinterpret_cast<Job *>(w + L.jobs);
     ctx->dws.n_jobs = reinterpret_cast<int32_t *>(w + L.n_jobs);
+    ctx->dws.n_misses = reinterpret_cast<int32_t *>(w + L.n_misses);
     ctx->dws.ticket = reinterpret_cast<uint32_t *>(w + L.ticket);
+    ctx->dws.ticket2 = reinterpret_cast<uint32_t *>(w + L.ticket2);
     ctx->dws.rowrefs = reinterpret_cast<RowRef *>(w + L.rowrefs);
     ctx->dws.xh = reinterpret_cast<__half *>(w + L.xh);
     ctx->dws.hh = reinterpret_cast<__half *>(w + L.hh);
@@ -445,6 +469,7 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
         }
     }
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket2, 0, 4, ctx->cs);
     if (e != cudaSuccess) {
         st = cuda_fail(ctx, e, "moe_layer_init");
         moe_layer_destroy(ctx);
@@ -484,7 +509,9 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         CK(cudaStreamSynchronize(ctx->cs));
         CK(launch_table_reset(ctx->tab, (int64_t)D.L * D.E, ctx->cs));
         CK(cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs));
+        CK(cudaMemsetAsync(ctx->dws.ticket2, 0, 4, ctx->cs));
         ctx->pending.clear();
+        ctx->page_h->error = 0;
         memset(&ctx->stats, 0, sizeof ctx->stats);
         ctx->state = MOE_OK;
         ctx->err.clear();
@@ -522,6 +549,7 @@ moe_status moe_layer_forward_host(moe_ctx *ctx, int32_t layer, const void *x_hos
 moe_status moe_get_routing(moe_ctx *ctx, int32_t *idx, float *gates, int32_t T) {
     if (!ctx || T < 1 || T != ctx->last_T) return MOE_ERR_ARG;
     CK(cudaStreamSynchronize(ctx->cs));
+    if (ctx->page_h->error) return device_error(ctx);
     const size_t n = (size_t)T * ctx->dims.k;
     if (idx) CK(cudaMemcpy(idx, ctx->dws.idx, n * 4, cudaMemcpyDeviceToHost));
     if (gates) CK(cudaMemcpy(gates, ctx->dws.gates, n * 4, cudaMemcpyDeviceToHost));
@@ -548,6 +576,7 @@ moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out) {
     if (!ctx || !out) return MOE_ERR_ARG;
     moe_status st = resolve_timing(ctx);
     if (st != MOE_OK) return st;
+    if (ctx->page_h->error) return device_error(ctx);
     *out = ctx->stats;
     return MOE_OK;
 }

@@ -45,18 +45,20 @@ struct RowRef {
     int16_t t, p;
 };
 
-// Miss list published to the host through mapped pinned memory.
-struct HostEvent {
-    int32_t expert, slot, hit, prefetch;
-    int64_t evicted;
+// Miss list published to the host through mapped pinned memory: one 16-byte
+// record per lookup entry (one PCIe write each).  flags: bit 0 hit, bit 1 prefetch.
+struct __align__(16) HostEvent {
+    int32_t expert, slot, flags, evicted;  // evicted: key or -1
 };
 struct HostPage {
-    volatile uint32_t seq;  // written last by the device
+    volatile uint32_t seq;    // written last by the device
     int32_t n_events;
     int32_t n_jobs;
     int32_t n_misses;
-    int32_t pad[4];
-    HostEvent ev[1];        // [capacity]
+    volatile int32_t error;   // nonzero: a kernel check failed (see diag)
+    int32_t pad[3];
+    int32_t diag[16];         // where: kernel mode, block, sizes, address low bits
+    HostEvent ev[1];          // [capacity]
 };
 
 // Device scratch of the decode path (carved from the caller's workspace).
@@ -66,15 +68,18 @@ struct DecodeWs {
     float *gates;        // [maxT][k]
     Job *jobs;           // [max_jobs]
     int32_t *n_jobs;     // [1]
+    int32_t *n_misses;   // [1]
     RowRef *rowrefs;     // [maxT*k]
     __half *xh;          // [maxT][2][d] fp16 hi/lo split of x
     __half *hh;          // [maxT][k+1][2][F] fp16 hi/lo split of h
     float *part;         // [maxT][k+1][d] per-selection expert outputs (p = k: shared)
-    uint32_t *ticket;    // last-CTA counter
+    uint32_t *ticket;    // last-CTA counter of the route kernel
+    uint32_t *ticket2;   // last-CTA counter of the combining down launch
 };
 
 struct RouteArgs {
     const __nv_bfloat16 *Wr;  // [E][d] of this layer
+    const __nv_bfloat16 *Wr_next;  // next layer's router (prefetched into L2) or null
     const __nv_bfloat16 *x;   // [T][d]
     int T, E, d, k, renorm, layer;
     DecodeWs ws;
@@ -101,7 +106,14 @@ struct GemvArgs {
     const __half *act;     // gate_up: xh; down: hh
     __half *hh_out;
     float *part_out;
-    int wpt;               // warps per tile (1, 2 or 4)
+    HostPage *page;        // device alias of the mapped page (error word + diagnostics)
+    // combine (down launches only): 1 = always, 2 = only if the lookup had no
+    // miss; performed by the last CTA of the launch
+    int combine;
+    const int32_t *n_misses;
+    const float *gates;
+    float *y;
+    uint32_t *ticket;
 };
 
 // launchers (one per .cu)
@@ -110,6 +122,5 @@ cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s);
 cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
                            int has_shared, cudaStream_t s);
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
-cudaError_t launch_table_export(Table t, int64_t nkeys, cudaStream_t s);
 
 }  // namespace moe

@@ -57,3 +57,41 @@ def decode_inputs(shape: LayerShape, T: int, streams: int = 1, seed: int = MASTE
         for l in range(shape.L):
             out[:, l, s, :] = decode_hidden_bf16(stream0 + s, l, T, shape.d, seed=seed)[0]
     return out
+
+
+class RegisteredPool:
+    """A host pool in ordinary (malloc'd) memory, page-locked with cudaHostRegister.
+
+    Used for pools of tens of GB: it pins exactly the bytes asked for (a
+    cudaHostAlloc through torch's caching host allocator may round the size up).
+    ``tensor`` is a uint8 view; call ``close()`` (or drop the object) to unpin."""
+
+    def __init__(self, shape: LayerShape, P: int | None = None, distinct: int | None = None,
+                 seed: int = MASTER_SEED):
+        P = shape.L * shape.E if P is None else P
+        distinct = P if distinct is None else min(distinct, P)
+        rb = record_bytes(shape.d, shape.F)
+        self.nbytes = P * rb
+        self.array = np.empty(self.nbytes, dtype=np.uint8)
+        base = self.array.ctypes.data
+        for i in range(distinct):
+            expert_record_into(base + i * rb, i // shape.E, i % shape.E, shape.d, shape.F,
+                               seed=seed)
+        if distinct < P:
+            replicate_records(base, rb, distinct, P)
+        rc = torch.cuda.cudart().cudaHostRegister(base, self.nbytes, 0)
+        if int(rc) != 0:
+            raise RuntimeError(f"cudaHostRegister failed ({rc})")
+        self.registered = True
+        self.tensor = torch.from_numpy(self.array)
+
+    def close(self) -> None:
+        if getattr(self, "registered", False):
+            torch.cuda.cudart().cudaHostUnregister(self.array.ctypes.data)
+            self.registered = False
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
