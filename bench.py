@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="override L (small profiling cases)")
     ap.add_argument("--slots", type=int, default=0, help="override the HBM cache slots")
     ap.add_argument("--pool-records", type=int, default=0, help="override the host pool records")
+    ap.add_argument("--warm", action="store_true",
+                    help="warm up on the timed inputs and keep the cache (all-hit runs)")
     return ap.parse_args()
 
 
@@ -228,6 +230,7 @@ def reference_arm(args, shape):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_layer * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "warm_cache": bool(args.warm),
             "config": {"workload": shape.name, "step": "one layer of one token (oracle)"},
             "cpu_baseline": {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
                              "sample": f"{args.steps} layer evaluations (1 token-layer each); "
@@ -280,17 +283,40 @@ def main():
     torch.cuda.synchronize()
 
     # warm-up on other inputs, then a cold cache
-    run_tokens(stack, x_warm[:args.warmup], yw, L)
-    stack.synchronize()
-    stack.reset()
-    if not args.no_kernel_timing:
-        abi.moe_set_timing(stack.ctx, True)
+    if args.warm:
+        run_tokens(stack, x, y, L)
+        stack.synchronize()
+        abi.moe_get_stats(stack.ctx)
+        base = abi.moe_get_stats(stack.ctx)
+    else:
+        run_tokens(stack, x_warm[:args.warmup], yw, L)
+        stack.synchronize()
+        stack.reset()
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
     el = timed(stack, x, y, L, world)
     clk = clocks.stop()
     st = abi.moe_get_stats(stack.ctx)
-    abi.moe_set_timing(stack.ctx, False)
+    if args.warm:  # counters of the timed region only
+        for f in ("lookups", "hits", "misses", "evictions", "h2d_copies", "h2d_bytes", "forward_calls"):
+            setattr(st, f, getattr(st, f) - getattr(base, f))
+        for i in range(8):
+            st.route_phase_us[i] -= base.route_phase_us[i]
+    # the same run again (cold cache again) with CUDA events around every kernel
+    # launch on the compute stream: per-kernel device time for the roofline
+    kst = None
+    if not args.no_kernel_timing:
+        if not args.warm:
+            stack.reset()
+        before = abi.moe_get_stats(stack.ctx)
+        abi.moe_set_timing(stack.ctx, True)
+        timed(stack, x, y, L, world)
+        kst = abi.moe_get_stats(stack.ctx)
+        abi.moe_set_timing(stack.ctx, False)
+        for i in range(abi.MOE_K_COUNT):
+            kst.kernel_launches[i] -= before.kernel_launches[i]
+            kst.kernel_ms[i] -= before.kernel_ms[i]
+            kst.kernel_bytes[i] -= before.kernel_bytes[i]
     el_max = max_over_ranks(el, world)
     tokens_total = sum_over_ranks(float(args.steps), world)
     value = tokens_total / el_max
@@ -302,24 +328,27 @@ def main():
     t_roof = max(hit_bytes / (hbm_peak * 1e9), miss_bytes / (h2d * 1e9))
     t_roof_8tb = max(hit_bytes / 8000e9, miss_bytes / (h2d * 1e9))
 
-    # dominant kernel by device time
-    ms = list(st.kernel_ms)
-    dom = int(np.argmax(ms)) if any(ms) else abi.MOE_K_GATEUP
-    roof = None
-    if st.kernel_launches[dom] > 0 and ms[dom] > 0:
-        achieved = st.kernel_bytes[dom] / (ms[dom] * 1e-3) / 1e9
-        roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "hbm", "achieved": achieved,
-                "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
-                "launches": int(st.kernel_launches[dom]),
-                "avg_launch_us": ms[dom] * 1e3 / st.kernel_launches[dom],
-                "bytes_per_launch": st.kernel_bytes[dom] / st.kernel_launches[dom]}
-    kernels = {abi.KERNEL_NAMES[i]: {"launches": int(st.kernel_launches[i]),
-                                     "ms": round(st.kernel_ms[i], 3),
-                                     "GBps": (st.kernel_bytes[i] / (st.kernel_ms[i] * 1e-3) / 1e9
-                                              if st.kernel_ms[i] > 0 else None)}
-               for i in range(abi.MOE_K_COUNT) if st.kernel_launches[i]}
-    launches = int(st.forward_calls * 4 + 2 * st.misses)
+    # dominant kernel by device time (from the timed pass with per-kernel events)
+    roof, kernels = None, {}
+    if kst is not None:
+        ms = list(kst.kernel_ms)
+        dom = int(np.argmax(ms))
+        if kst.kernel_launches[dom] > 0 and ms[dom] > 0:
+            achieved = kst.kernel_bytes[dom] / (ms[dom] * 1e-3) / 1e9
+            roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "hbm", "achieved": achieved,
+                    "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                    "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
+                    "launches": int(kst.kernel_launches[dom]),
+                    "avg_launch_us": ms[dom] * 1e3 / kst.kernel_launches[dom],
+                    "bytes_per_launch": kst.kernel_bytes[dom] / kst.kernel_launches[dom]}
+        kernels = {abi.KERNEL_NAMES[i]: {"launches": int(kst.kernel_launches[i]),
+                                         "ms": round(kst.kernel_ms[i], 3),
+                                         "GBps": (kst.kernel_bytes[i] / (kst.kernel_ms[i] * 1e-3) / 1e9
+                                                  if kst.kernel_ms[i] > 0 else None)}
+                   for i in range(abi.MOE_K_COUNT) if kst.kernel_launches[i]}
+    route_phases = {n: round(v / max(st.forward_calls, 1), 3)
+                    for n, v in zip(abi.ROUTE_PHASES, st.route_phase_us)}
+    launches = int(st.forward_calls * 3 + 2 * st.misses)  # route, hit gate/up, hit down; 2 per miss
 
     # end to end: host buffers through moe_layer_forward_host
     e2e = None
@@ -341,6 +370,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el_max / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4 x bf16 -> f32 (w4a16)", "data": "synthetic",
+            "warm_cache": bool(args.warm),
             "config": {"workload": f"{shape.name} decode: {L} layers x {E} experts, top-{k}, "
                                    f"d={d}, F={F}, NVFP4 records of {rb} B, batch 1, "
                                    f"{args.steps} tokens, HBM cache {shape.cache_slots} slots "
@@ -358,7 +388,8 @@ def main():
                                "h2d_term_s": miss_bytes / (h2d * 1e9),
                                "bw_hbm_gbs": hbm_peak, "bw_h2d_gbs": h2d,
                                "hit_bytes": hit_bytes, "miss_bytes": miss_bytes},
-            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roof, "kernels": kernels, "route_phase_us_per_call": route_phases,
+            "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk,
         }
         print(json.dumps(line), flush=True)

@@ -16,6 +16,8 @@ MOE_K_ROUTE, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE = 0, 1, 2, 3
 MOE_K_PREFILL_ROUTE, MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_COUNT = 4, 5, 6, 7
 KERNEL_NAMES = ["route_lookup", "gate_up", "down", "combine", "prefill_route", "prefill_gate_up",
                 "prefill_down"]
+ROUTE_PHASES = ["logits", "elect", "topk", "jobs", "table_read", "select_write", "publish",
+                "wait_previous_layer"]
 
 
 class moe_dims(ctypes.Structure):
@@ -43,7 +45,8 @@ class moe_stats(ctypes.Structure):
                 ("h2d_bytes", ctypes.c_int64), ("forward_calls", ctypes.c_int64),
                 ("kernel_launches", ctypes.c_int64 * MOE_K_COUNT),
                 ("kernel_ms", ctypes.c_double * MOE_K_COUNT),
-                ("kernel_bytes", ctypes.c_double * MOE_K_COUNT)]
+                ("kernel_bytes", ctypes.c_double * MOE_K_COUNT),
+                ("route_phase_us", ctypes.c_double * 8)]
 
 
 class moe_split(ctypes.Structure):

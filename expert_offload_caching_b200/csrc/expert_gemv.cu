@@ -75,7 +75,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-constexpr int kGemvWarps = 4;
+constexpr int kMaxSteps = 16;  // K <= 4096: at most 16 K-steps of 256, one per warp
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -131,18 +136,27 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
     }
 }
 
-// One CTA (4 warps) per 16-row weight tile.  The tile's rows are contiguous in
+// One CTA per 16-row weight tile; each warp owns spw consecutive K-steps of 256
+// elements (spw = ceil(K-steps / warps)).  The tile's rows are contiguous in
 // the record; all threads stage it into shared memory with 16-byte cp.async
-// copies (the whole tile in flight at once), then the warps split the K-steps
-// of 256 elements and reduce in shared memory.  Dynamic shared memory: 16*K/2
-// code bytes + K scale bytes.
+// copies (the whole tile in flight at once), each warp computes its steps, and
+// warp 0 sums the warps' partials in a fixed order.  Dynamic shared memory:
+// 16*K/2 code bytes + K scale bytes + the partials (warps x NG x 512 bytes).
+//
+// Launched with programmatic stream serialization: gate/up waits for the
+// route kernel before reading anything (job list, activations); the down
+// projection reads the job list (complete, two launches back), stages its W2
+// tile, and only then waits for gate/up's h.  Both release their dependents
+// early; every dependent waits before writing shared buffers.
 template <int NG>
-__global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ float red[kGemvWarps][NG][4][32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, q = lane & 3;
     const bool gate_up = a.mode == kGateUp;
+
+    if (gate_up) pdl_wait();  // job list and x come from the previous launch
+    pdl_launch_dependents();
 
     // ---- which expert (job) this CTA serves
     const uint8_t *rec = nullptr;
@@ -153,17 +167,20 @@ __global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a
         nrows = a.T;
         shared = true;
     } else {
+        // L2 reads (ld.global.cg): the down launch reads these before its PDL
+        // wait, and an SM's L1 may still hold lines of an older launch
         const int jy = a.only_job >= 0 ? a.only_job : (int)blockIdx.y;
-        if (jy >= *a.n_jobs) {
+        if (jy >= __ldcg(a.n_jobs)) {
             work = false;
         } else {
-            const Job jb = a.jobs[jy];
-            if (a.only_job < 0 && !jb.hit) {
+            const int4 j0 = __ldcg(reinterpret_cast<const int4 *>(&a.jobs[jy]));  // expert, slot, hit, nrows
+            const int row_off_j = __ldcg(&a.jobs[jy].row_off);
+            if (a.only_job < 0 && !j0.z) {
                 work = false;
             } else {
-                rec = a.arena + (int64_t)jb.slot * a.rec_bytes;
-                nrows = jb.nrows;
-                row_off = jb.row_off;
+                rec = a.arena + (int64_t)j0.y * a.rec_bytes;
+                nrows = j0.w;
+                row_off = row_off_j;
             }
         }
     }
@@ -173,9 +190,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a
     const int tile = blockIdx.x;
     if (work && tile < tiles) {
         const int NCH = K >> 6;
+        const int nwarps = (int)(blockDim.x >> 5);
         const int nsteps = (NCH + 3) >> 2;
+        const int spw = (nsteps + nwarps - 1) / nwarps;
         const uint32_t code_bytes = 16u * (uint32_t)(K >> 1), scale_bytes = (uint32_t)K;
         uint8_t *s_codes = smem, *s_scales = smem + code_bytes;
+        float(*red)[NG][4][32] = reinterpret_cast<float(*)[NG][4][32]>(smem + code_bytes + scale_bytes);
         const uint8_t *codes = rec + (gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)tile * code_bytes;
         const uint8_t *scales = rec + (gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)tile * scale_bytes;
         // stage the tile: every thread issues its 16-byte pieces, then waits for its own
@@ -183,7 +203,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a
         for (uint32_t i = threadIdx.x; i < n16c; i += blockDim.x) cp_async16(s_codes + 16 * i, codes + 16 * i);
         for (uint32_t i = threadIdx.x; i < n16s; i += blockDim.x) cp_async16(s_scales + 16 * i, scales + 16 * i);
         if (gate_up) {  // this expert's down projection -> L2 for the down launch
-            const uint32_t total = (uint32_t)(a.lay.tscales - a.lay.w2_codes);
+            const uint32_t total = (uint32_t)(a.lay.bytes - a.lay.w2_codes);
             const uint32_t per = ((total / gridDim.x) + 127u) & ~127u;
             const uint32_t off = per * blockIdx.x;
             if (off < total) prefetch_l2_range(rec + a.lay.w2_codes + off, per < total - off ? per : total - off);
@@ -191,6 +211,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a
         const float *ts = reinterpret_cast<const float *>(rec + a.lay.tscales);
         // tile-local rows of this thread: gate_up 2g (gate) / 2g+1 (up); down g / g+8
         const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
+        if (!gate_up) pdl_wait();  // h comes from the gate/up launch; W2 is already in flight
         cp_async_wait_all();
         __syncthreads();
         for (int r0 = 0; r0 < nrows; r0 += 4 * NG) {
@@ -218,8 +239,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a
             for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[grp][j] = 0.f;
-            for (int s = warp; s < nsteps; s += kGemvWarps) {  // s is uniform across the warp
-                const int c = 4 * s + q;
+            for (int i = 0; i < spw; ++i) {  // this warp's K-steps (uniform across the warp)
+                const int c = 4 * (warp * spw + i) + q;
                 const bool cv = c < NCH;  // ragged K tail: some lanes of the quad feed zeros
                 const int cc = cv ? c : 0;
                 const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
@@ -234,7 +255,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a
                 for (int j = 0; j < 4; ++j) red[warp][grp][j][lane] = acc[grp][j];
             __syncthreads();
             if (warp == 0) {
-                for (int w = 1; w < kGemvWarps; ++w)
+                for (int w = 1; w < nwarps; ++w)
 #pragma unroll
                     for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
@@ -295,20 +316,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) expert_gemv_kernel(GemvArgs a
     }
 }
 
-__global__ void combine_kernel(const float *__restrict__ part, const float *__restrict__ gates,
-                               float *__restrict__ y, int T, int k, int d, int has_shared) {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= T * d) return;
-    const int t = i / d, c = i - t * d;
-    const float *pr = part + (size_t)t * (k + 1) * d + c;
-    float acc = 0.f;
-    for (int p = 0; p < k; ++p) acc = fmaf(gates[t * k + p], pr[(size_t)p * d], acc);
-    if (has_shared) acc += pr[(size_t)k * d];
-    y[i] = acc;
-}
-
 template <int NG>
-cudaError_t launch_ng(const GemvArgs &a, dim3 grid, size_t smem, cudaStream_t s) {
+cudaError_t launch_ng(const GemvArgs &a, dim3 grid, int threads, size_t smem, cudaStream_t s) {
     static bool configured = false;  // per instantiation: allow > 48 KB of dynamic smem
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<NG>,
@@ -316,8 +325,17 @@ cudaError_t launch_ng(const GemvArgs &a, dim3 grid, size_t smem, cudaStream_t s)
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    expert_gemv_kernel<NG><<<grid, kGemvWarps * 32, smem, s>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, expert_gemv_kernel<NG>, a);
 }
 
 }  // namespace
@@ -325,19 +343,16 @@ cudaError_t launch_ng(const GemvArgs &a, dim3 grid, size_t smem, cudaStream_t s)
 cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s) {
     const int K = a.mode == kGateUp ? a.d : a.F;
     const int tiles = a.mode == kGateUp ? a.F / 8 : a.d / 16;
+    const int nsteps = (K / 64 + 3) / 4;
+    if (nsteps < 1 || nsteps > kMaxSteps) return cudaErrorInvalidValue;
+    const int spw = nsteps >= 8 ? 2 : 1;  // 2 K-steps per warp for long rows: smaller CTAs, more per SM
+    const int warps = (nsteps + spw - 1) / spw;
     const dim3 grid(tiles, grid_y);
-    const size_t smem = 16 * (size_t)(K / 2) + (size_t)K;
+    const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
+    const size_t smem = 16 * (size_t)(K / 2) + (size_t)K + (size_t)warps * ng * 4 * 32 * sizeof(float);
     if (smem > 96 * 1024) return cudaErrorInvalidValue;
-    if (a.T <= 4) return launch_ng<1>(a, grid, smem, s);
-    if (a.T <= 8) return launch_ng<2>(a, grid, smem, s);
-    return launch_ng<4>(a, grid, smem, s);
-}
-
-cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
-                           int has_shared, cudaStream_t s) {
-    const int n = T * d;
-    combine_kernel<<<(n + 255) / 256, 256, 0, s>>>(part, gates, y, T, k, d, has_shared);
-    return cudaGetLastError();
+    if (ng == 1) return launch_ng<1>(a, grid, warps * 32, smem, s);
+    return launch_ng<2>(a, grid, warps * 32, smem, s);
 }
 
 }  // namespace moe

@@ -43,12 +43,12 @@ bool dims_supported(const moe_dims *d) {
 RecordLayout layout_of(const moe_dims *d) {
     RecordLayout r;
     const int64_t dd = d->d, ff = d->F;
-    r.w13_codes = 0;
+    r.tscales = 0;  // head: the gate/up half (tensor scales + W13) is a contiguous prefix
+    r.w13_codes = up256(12);
     r.w13_scales = r.w13_codes + up256(2 * ff * dd / 2);
     r.w2_codes = r.w13_scales + up256(2 * ff * dd / 16);
     r.w2_scales = r.w2_codes + up256(dd * ff / 2);
-    r.tscales = r.w2_scales + up256(dd * ff / 16);
-    r.bytes = up256(r.tscales + 12);
+    r.bytes = r.w2_scales + up256(dd * ff / 16);
     return r;
 }
 
@@ -87,7 +87,7 @@ WsLayout ws_layout(const moe_dims *d) {
 }
 
 struct TableLayout {
-    int64_t hdr, map, owner, stamp, prev, next, total;
+    int64_t hdr, map, owner, stamp, total;
 };
 TableLayout table_layout(const moe_dims *d, int64_t C) {
     TableLayout t;
@@ -97,8 +97,6 @@ TableLayout table_layout(const moe_dims *d, int64_t C) {
     t.map = take((int64_t)d->L * d->E * 4);
     t.owner = take(C * 4);
     t.stamp = take(C * 8);
-    t.prev = take(C * 4);
-    t.next = take(C * 4);
     t.total = o;
     return t;
 }
@@ -132,7 +130,7 @@ struct moe_ctx {
     HostPage *page_h = nullptr, *page_d = nullptr;
     int page_cap = 0;
     uint32_t seq = 0;
-    std::vector<cudaEvent_t> miss_ev;
+    std::vector<cudaEvent_t> miss_ev;   // [2 * page_cap]: W13 part, W2 part of miss j
     // state
     moe_status state = MOE_OK;
     std::string err;
@@ -235,7 +233,7 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
 }
 
 double w13_bytes(const moe_ctx *c) { return (double)(c->lay.w2_codes - c->lay.w13_codes) + 8.0; }
-double w2_bytes(const moe_ctx *c) { return (double)(c->lay.tscales - c->lay.w2_codes) + 4.0; }
+double w2_bytes(const moe_ctx *c) { return (double)(c->lay.bytes - c->lay.w2_codes) + 4.0; }
 
 // A kernel reported a failed self-check through the mapped page (error word
 // and a diagnostic record: check code, kernel mode, block, tile, sizes).
@@ -322,7 +320,10 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         ctx->pending[id].bytes = nexp * w2_bytes(ctx) + (double)T * D.F * 4;
     }
 
-    // misses: one copy per record on the copy stream, an event after each
+    // misses: each record in two copies on the copy stream -- the gate/up half
+    // (tensor scales + W13, a prefix of the record) and the down half -- with an
+    // event after each, so a miss's gate/up runs while its down half streams in
+    const int64_t split = ctx->lay.w2_codes;
     for (int j = 0; j < nev; ++j) {
         if (ev[j].flags & 1) continue;
         if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
@@ -331,20 +332,24 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
             return MOE_ERR_CUDA;
         }
         const int64_t rec_idx = ((int64_t)layer * D.E + ev[j].expert) % ctx->P;
-        CK(cudaMemcpyAsync(ctx->arena + (int64_t)ev[j].slot * ctx->lay.bytes,
-                           ctx->pool + rec_idx * ctx->lay.bytes, ctx->lay.bytes,
-                           cudaMemcpyHostToDevice, ctx->xs));
-        CK(cudaEventRecord(ctx->miss_ev[j], ctx->xs));
+        uint8_t *dst = ctx->arena + (int64_t)ev[j].slot * ctx->lay.bytes;
+        const uint8_t *src = ctx->pool + rec_idx * ctx->lay.bytes;
+        CK(cudaMemcpyAsync(dst, src, split, cudaMemcpyHostToDevice, ctx->xs));
+        CK(cudaEventRecord(ctx->miss_ev[2 * j], ctx->xs));
+        CK(cudaMemcpyAsync(dst + split, src + split, ctx->lay.bytes - split, cudaMemcpyHostToDevice,
+                           ctx->xs));
+        CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], ctx->xs));
         ctx->stats.h2d_copies += 1;
         ctx->stats.h2d_bytes += ctx->lay.bytes;
     }
     for (int j = 0; j < nev; ++j) {
         if (ev[j].flags & 1) continue;
-        CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[j], 0));
+        CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j], 0));
         TimedLaunch mg, md;
         time_begin(ctx, mg, MOE_K_GATEUP);
         CK(launch_gemv(gemv_args(ctx, layer, T, kGateUp, j), 1, ctx->cs));
         time_end(ctx, mg, w13_bytes(ctx) + (double)T * D.d * 2);
+        CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j + 1], 0));
         time_begin(ctx, md, MOE_K_DOWN);
         GemvArgs md_args = gemv_args(ctx, layer, T, kDown, j, j == last_miss ? 1 : 0);
         md_args.y = y;
@@ -358,6 +363,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         hits += ev[j].flags & 1;
         evictions += ev[j].evicted >= 0;
     }
+    for (int i = 0; i < 8; ++i) ctx->stats.route_phase_us[i] += ctx->page_h->phase_ns[i] * 1e-3;
     ctx->stats.lookups += nev;
     ctx->stats.hits += hits;
     ctx->stats.misses += nev - hits;
@@ -462,7 +468,7 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     if (e == cudaSuccess) e = cudaHostGetDevicePointer(reinterpret_cast<void **>(&ctx->page_d), ctx->page_h, 0);
     if (e == cudaSuccess) {
         memset((void *)ctx->page_h, 0, page_bytes);
-        ctx->miss_ev.resize(ctx->page_cap, nullptr);
+        ctx->miss_ev.resize(2 * ctx->page_cap, nullptr);
         for (auto &ev : ctx->miss_ev) {
             e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
             if (e != cudaSuccess) break;
@@ -486,7 +492,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
     const int64_t need = max_jobs(&D, D.max_rows);
     if (num_slots < need) return MOE_ERR_CAPACITY;
     if ((flags & MOE_CACHE_PREFETCH_NEXT) && num_slots < 2ll * D.E) return MOE_ERR_CAPACITY;
-    if (num_slots >= (1ll << 31)) return MOE_ERR_ARG;
+    if (num_slots > 65536) return MOE_ERR_UNSUPPORTED;
     if (arena_bytes < moe_arena_bytes(&D, num_slots)) return MOE_ERR_ARG;
     const bool reset = (flags & MOE_CACHE_RESET) || !ctx->configured || ctx->arena != slot_arena ||
                        ctx->C != num_slots;
@@ -499,8 +505,6 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
     ctx->tab.map = reinterpret_cast<int32_t *>(tb + tl.map);
     ctx->tab.owner = reinterpret_cast<int32_t *>(tb + tl.owner);
     ctx->tab.stamp = reinterpret_cast<unsigned long long *>(tb + tl.stamp);
-    ctx->tab.prev = reinterpret_cast<int32_t *>(tb + tl.prev);
-    ctx->tab.next = reinterpret_cast<int32_t *>(tb + tl.next);
     ctx->tab.C = num_slots;
     ctx->flags = flags & ~MOE_CACHE_RESET;
     if (reset) {

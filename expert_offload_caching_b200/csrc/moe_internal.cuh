@@ -16,15 +16,14 @@ struct RecordLayout {
     int64_t w13_codes, w13_scales, w2_codes, w2_scales, tscales, bytes;
 };
 
-// Device cache table, in the slot arena after the slots.  LRU order is kept
-// as a doubly linked list of resident slots (head = least recently used);
-// stamps (the global clock at last use) are kept alongside so the table can be
-// exported and checked against the min-stamp rule.
+// Device cache table, in the slot arena after the slots.  The least recently
+// used slots are the resident slots with the smallest stamps (the global clock
+// at last use; stamps are unique), so victims are found by a parallel scan of
+// the stamps rather than by walking a list.
 struct TableHdr {
     unsigned long long clock;
     int32_t next_free;  // slots [next_free, C) have never been filled since the reset
-    int32_t head, tail; // LRU list ends, -1 when empty
-    int32_t pad[11];
+    int32_t pad[13];
 };
 
 struct Table {
@@ -32,7 +31,6 @@ struct Table {
     int32_t *map;               // [L*E] slot of key or -1
     int32_t *owner;             // [C] key in slot or -1
     unsigned long long *stamp;  // [C]
-    int32_t *prev, *next;       // [C] LRU list links
     int64_t C;
 };
 
@@ -58,6 +56,7 @@ struct HostPage {
     volatile int32_t error;   // nonzero: a kernel check failed (see diag)
     int32_t pad[3];
     int32_t diag[16];         // where: kernel mode, block, sizes, address low bits
+    uint32_t phase_ns[8];     // route kernel, last CTA: ns spent in each phase (globaltimer)
     HostEvent ev[1];          // [capacity]
 };
 
@@ -119,8 +118,6 @@ struct GemvArgs {
 // launchers (one per .cu)
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s);
-cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
-                           int has_shared, cudaStream_t s);
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
 
 }  // namespace moe

@@ -19,14 +19,16 @@
  * For prefill chunks, the next layer's experts are streamed in while the
  * current layer computes (holude.com "長いプロンプトとエージェント処理も意識している").
  *
- * Expert record (one contiguous block per (layer, expert); moe_record_layout):
- *   [0] W13 codes  [2F x d/2] bytes; row 2j = gate_j, row 2j+1 = up_j; E2M1,
- *                  two per byte, element 2i in the low nibble
- *   [1] W13 scales [2F x d/16] E4M3 bytes, one per 16 consecutive elements of a row
- *   [2] W2 codes   [d x F/2] bytes (row = output dim, K = F)
- *   [3] W2 scales  [d x F/16]
- *   [4] 3 fp32 tensor scales: gate, up, down
- *   [5] total size; every section starts on a 256-byte boundary.
+ * Expert record (one contiguous block per (layer, expert); moe_record_layout
+ * returns the offsets off[0..5] of the sections named below):
+ *   off[4] 3 fp32 tensor scales: gate, up, down (at the record head)
+ *   off[0] W13 codes  [2F x d/2] bytes; row 2j = gate_j, row 2j+1 = up_j; E2M1,
+ *                     two per byte, element 2i in the low nibble
+ *   off[1] W13 scales [2F x d/16] E4M3 bytes, one per 16 consecutive elements of a row
+ *   off[2] W2 codes   [d x F/2] bytes (row = output dim, K = F)
+ *   off[3] W2 scales  [d x F/16]
+ *   off[5] total size; every section starts on a 256-byte boundary.  The
+ *   gate/up half (tensor scales + W13) is the prefix [0, off[2]).
  *   w = e2m1(code) * e4m3(scale) * tensor_scale.
  *
  * Conventions: all functions return a moe_status and never throw; pointers
@@ -113,6 +115,12 @@ typedef struct {
     int64_t kernel_launches[MOE_K_COUNT];
     double kernel_ms[MOE_K_COUNT];
     double kernel_bytes[MOE_K_COUNT];
+    /* decode route kernel, summed over calls: microseconds its last CTA spent in
+     * [0] logits + split of x, [1] CTA election, [2] softmax/top-k, [3] job list,
+     * [4] table reads, [5] victim selection + table writes, [6] publishing the
+     * miss list; [7] launch to start (waiting for the previous layer; the
+     * kernel is launched early).  Device %globaltimer. */
+    double route_phase_us[8];
 } moe_stats;
 
 /* Hybrid split plan (ai-hardware-zukan "GPUに載らない分をどう間に合わせるか";
@@ -163,7 +171,9 @@ MOE_API moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, s
  * flags.  MOE_CACHE_RESET (required the first time and after an error) empties
  * the cache on the compute stream.  MOE_ERR_CAPACITY if num_slots < k * max_rows
  * distinct experts could need (min(k*max_rows, E)), or, with
- * MOE_CACHE_PREFETCH_NEXT, num_slots < 2*E. */
+ * MOE_CACHE_PREFETCH_NEXT, num_slots < 2*E; MOE_ERR_UNSUPPORTED above 65536 slots.
+ * Each miss is copied in two parts (the prefix [0, off[2]) holding the tensor
+ * scales and W13, then W2), so the gate/up of a miss overlaps its W2 transfer. */
 MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, size_t arena_bytes,
                            uint32_t flags);
 

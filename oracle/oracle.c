@@ -65,17 +65,18 @@ static double bf16_val(uint16_t b) {
 /* ------------------------------------------------------- record layout -- */
 static int64_t up256(int64_t x) { return (x + 255) / 256 * 256; }
 
-/* Byte offsets: [0] W13 codes [2F x d/2], [1] W13 scales [2F x d/16],
- * [2] W2 codes [d x F/2], [3] W2 scales [d x F/16], [4] 3 fp32 tensor
- * scales (gate, up, down), [5] record size.  W13 row 2j = gate_j, 2j+1 = up_j. */
+/* Byte offsets: [4] 3 fp32 tensor scales (gate, up, down) at the record head,
+ * then [0] W13 codes [2F x d/2], [1] W13 scales [2F x d/16], [2] W2 codes
+ * [d x F/2], [3] W2 scales [d x F/16]; [5] record size.  Every section starts
+ * on a 256-byte boundary.  W13 row 2j = gate_j, 2j+1 = up_j. */
 EXPORT void orc_record_layout(int d, int F, int64_t *off) {
     int64_t w13_rows = 2 * (int64_t)F, w2_rows = d;
-    off[0] = 0;
+    off[4] = 0;
+    off[0] = up256(3 * 4);
     off[1] = off[0] + up256(w13_rows * d / 2);
     off[2] = off[1] + up256(w13_rows * d / 16);
     off[3] = off[2] + up256(w2_rows * F / 2);
-    off[4] = off[3] + up256(w2_rows * F / 16);
-    off[5] = up256(off[4] + 3 * 4);
+    off[5] = off[3] + up256(w2_rows * F / 16);
 }
 
 static float rec_tensor_scale(const uint8_t *rec, const int64_t *off, int which) {

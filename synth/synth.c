@@ -25,13 +25,14 @@
  *   code  = E2M1(x / denom), RNE, saturating to 6   (all codes 0 if value(sb) = 0)
  *
  * Expert record (one contiguous block per (layer, expert)):
+ *   3 fp32 tensor scales (gate, up, down), padded to 256 B
  *   W13 codes  [2F x d/2] bytes, rows interleaved: row 2j = gate_j, 2j+1 = up_j;
  *              two codes per byte, element 2i in the low nibble
  *   W13 scales [2F x d/16] E4M3 bytes
  *   W2 codes   [d x F/2] bytes (row = output dim, K = F)
  *   W2 scales  [d x F/16]
- *   3 fp32 tensor scales (gate, up, down)
  * each section starting on a 256-byte boundary, the whole padded to 256 B.
+ * (The gate/up half -- tensor scales and W13 -- is a contiguous prefix.)
  */
 #include <math.h>
 #include <stdint.h>
@@ -187,12 +188,12 @@ static inline int64_t align256(int64_t x) { return (x + 255) & ~(int64_t)255; }
 /* Section offsets of one record: [w13 codes, w13 scales, w2 codes, w2 scales, tensor scales, total]. */
 EXPORT void synth_record_layout(int32_t d, int32_t F, int64_t *off) {
     int64_t dd = d, ff = F;
-    off[0] = 0;
+    off[4] = 0;                     /* tensor scales at the head */
+    off[0] = align256(12);
     off[1] = off[0] + align256(2 * ff * dd / 2);
     off[2] = off[1] + align256(2 * ff * dd / 16);
     off[3] = off[2] + align256(dd * ff / 2);
-    off[4] = off[3] + align256(dd * ff / 16);
-    off[5] = align256(off[4] + 12);
+    off[5] = off[3] + align256(dd * ff / 16);
 }
 
 /* One expert record from N(0, sigma^2) fp32 draws keyed by (purpose, layer, expert, matrix).

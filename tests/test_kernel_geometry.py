@@ -19,7 +19,7 @@ def test_tile_copies_inside_record_and_aligned(shape):
     assert rb % 256 == 0 and all(o % 256 == 0 for o in off)
     for mode, K, tiles, codes0, scales0, end in (
             ("gate_up", shape.d, shape.F // 8, off[0], off[1], off[2]),
-            ("down", shape.F, shape.d // 16, off[2], off[3], off[4])):
+            ("down", shape.F, shape.d // 16, off[2], off[3], off[5])):
         code_bytes, scale_bytes = 16 * (K // 2), K
         assert code_bytes % 16 == 0 and scale_bytes % 16 == 0
         assert code_bytes + scale_bytes <= 96 * 1024  # dynamic shared memory limit set at launch
@@ -30,8 +30,9 @@ def test_tile_copies_inside_record_and_aligned(shape):
             assert s0 + scale_bytes <= end, (mode, t)
         # shared-memory destinations: codes at 0, scales right after (16-byte multiple)
         assert code_bytes % 16 == 0
+    assert off[4] == 0 and off[0] >= 12  # tensor scales at the head: W13 + scales form a prefix
     # down-projection prefetch ranges issued by the gate/up CTAs
-    total = off[4] - off[2]
+    total = off[5] - off[2]
     grid = shape.F // 8
     per = ((total // grid) + 127) & ~127
     covered = 0
@@ -39,7 +40,7 @@ def test_tile_copies_inside_record_and_aligned(shape):
         o = per * b
         if o < total:
             n = min(per, total - o)
-            assert off[2] + o + n <= off[4]
+            assert off[2] + o + n <= off[5]
             covered += n
     assert covered == total
 
