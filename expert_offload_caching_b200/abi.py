@@ -59,7 +59,7 @@ EXPORTS = ["moe_record_bytes", "moe_record_layout", "moe_workspace_bytes", "moe_
            "moe_layer_init", "cache_configure", "moe_layer_forward", "moe_layer_forward_host",
            "moe_get_routing", "moe_cache_export", "moe_get_stats", "moe_set_timing",
            "moe_set_wait_limit", "moe_debug_inject", "plan_split", "moe_measure_h2d",
-           "moe_status_str", "moe_last_error", "moe_layer_destroy"]
+           "moe_route_noalloc", "moe_status_str", "moe_last_error", "moe_layer_destroy"]
 
 _lib = None
 
@@ -110,6 +110,8 @@ def lib():
         L.plan_split.argtypes = [i32, dbl, dbl, dbl, dbl, ctypes.POINTER(moe_split)]
         L.moe_measure_h2d.restype = ctypes.c_int
         L.moe_measure_h2d.argtypes = [vp, vp, sz, sz, i32, vp, ctypes.POINTER(dbl)]
+        L.moe_route_noalloc.restype = ctypes.c_int
+        L.moe_route_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
         L.moe_status_str.restype = ctypes.c_char_p
         L.moe_status_str.argtypes = [ctypes.c_int]
         L.moe_last_error.restype = ctypes.c_char_p
@@ -243,6 +245,14 @@ def moe_measure_h2d(dev_buf, host_buf, nbytes: int, chunk_bytes: int = 0, reps: 
     _check(lib().moe_measure_h2d(_ptr(dev_buf), _ptr(host_buf), nbytes, chunk_bytes, reps,
                                  _stream(stream), ctypes.byref(gbs)), "moe_measure_h2d")
     return gbs.value
+
+
+def moe_route_noalloc(router_w, x, T: int, E: int, d: int, k: int, renormalize: bool, idx, gates,
+                      stream) -> None:
+    """Routing with no workspace (see include/moe_offload.h): the scratch lives in
+    an array inside the library, so the call allocates nothing."""
+    _check(lib().moe_route_noalloc(_ptr(router_w), _ptr(x), T, E, d, k, int(renormalize),
+                                   _ptr(idx), _ptr(gates), _stream(stream)), "moe_route_noalloc")
 
 
 def moe_status_str(s: int) -> str:

@@ -237,6 +237,28 @@ MOE_API moe_status plan_split(int32_t m, double B_P, double B_H, double threshol
 MOE_API moe_status moe_measure_h2d(void *dev_buf, const void *host_buf, size_t bytes, size_t chunk_bytes,
                            int32_t reps, void *stream, double *gbs);
 
+/* Router logits, softmax and top-k for T rows with no workspace (the routing
+ * part of moe_layer_forward: same selection, gates and ascending id order).
+ * The FreeToken pages have no counterpart: this serves callers that cannot
+ * allocate device memory when they run -- e.g. a host framework that owns the
+ * whole device memory pool and passes only inputs and outputs, or a process
+ * whose memory is planned before start-up -- and so cannot give
+ * moe_layer_init a workspace.  Its scratch (the [T][E] fp32 logits and a CTA
+ * counter, 128 KB + 256 B) lives in an array built into the library, present
+ * on every GPU that loads it until the process exits; the call allocates
+ * nothing.  All calls share that array and it keeps the last call's contents:
+ * each call clears the counter it needs at zero, and calls that overlap on
+ * the GPU race -- serialise them.  The first call on a device looks up the
+ * array's address with that device current; make it before any stream capture.
+ *   router_w: device bf16 [E][d]; x: device bf16 [T][d];
+ *   idx: device int32 [T][k] out (ascending per row); gates: device fp32 [T][k] out;
+ *   stream: cudaStream_t the work is issued on (stream-ordered, returns at once).
+ * Limits: T <= 32, E <= 1024, k <= 32, d a multiple of 64; larger sizes return
+ * MOE_ERR_UNSUPPORTED.  MOE_ERR_ARG for null pointers or k > E. */
+MOE_API moe_status moe_route_noalloc(const void *router_w, const void *x, int32_t T, int32_t E,
+                                     int32_t d, int32_t k, int32_t renormalize, int32_t *idx,
+                                     float *gates, void *stream);
+
 MOE_API const char *moe_status_str(moe_status s);
 MOE_API const char *moe_last_error(const moe_ctx *ctx);
 MOE_API void moe_layer_destroy(moe_ctx *ctx);
