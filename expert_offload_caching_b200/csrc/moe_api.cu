@@ -13,6 +13,7 @@
 // A slot is only overwritten after the lookup that evicted it has run, i.e.
 // after every earlier kernel on the compute stream; copies of one slot are
 // ordered on the copy stream.
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <cstdio>
@@ -52,26 +53,28 @@ RecordLayout layout_of(const moe_dims *d) {
     return r;
 }
 
-int decode_rows(const moe_dims *d) { return d->max_rows < kDecodeMaxRows ? d->max_rows : kDecodeMaxRows; }
 int max_jobs(const moe_dims *d, int T) {
     int64_t n = (int64_t)T * d->k;
     return (int)(n < d->E ? n : d->E);
 }
 
-// Workspace carve-up; with base == nullptr only sizes are computed.
+// Workspace carve-up (offsets from the caller's base).  Row buffers are sized
+// for the largest call (max_rows); the prefill buffers exist when max_rows > 32.
 struct WsLayout {
-    int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, rowrefs, xh, hh, part, xstage,
-        ystage, total;
+    int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, rowrefs, xh, hh, part, cnt, fill,
+        jobidx, h32, xstage, ystage, total;
 };
 WsLayout ws_layout(const moe_dims *d) {
     WsLayout w;
-    const int64_t T = decode_rows(d), k = d->k, E = d->E, dd = d->d, F = d->F;
+    const int64_t T = d->max_rows, k = d->k, E = d->E, dd = d->d, F = d->F;
+    const bool prefill = T > kDecodeMaxRows;
     int64_t o = 0;
     auto take = [&](int64_t bytes) { int64_t r = o; o += up256(bytes); return r; };
     w.z = take(T * E * 4);
     w.idx = take(T * k * 4);
     w.gates = take(T * k * 4);
-    w.jobs = take((int64_t)max_jobs(d, (int)T) * (int64_t)sizeof(Job));
+    const int64_t nj = prefill ? E : max_jobs(d, (int)T);
+    w.jobs = take(nj * (int64_t)sizeof(Job));
     w.n_jobs = take(4);
     w.n_misses = take(4);
     w.ticket = take(4);
@@ -80,8 +83,12 @@ WsLayout ws_layout(const moe_dims *d) {
     w.xh = take(T * 2 * dd * 2);
     w.hh = take(T * (k + 1) * 2 * F * 2);
     w.part = take(T * (k + 1) * dd * 4);
-    w.xstage = take((int64_t)d->max_rows * dd * 2);
-    w.ystage = take((int64_t)d->max_rows * dd * 4);
+    w.cnt = prefill ? take(E * 4) : -1;
+    w.fill = prefill ? take(E * 4) : -1;
+    w.jobidx = prefill ? take(E * 4) : -1;
+    w.h32 = prefill ? take(T * (k + 1) * F * 4) : -1;
+    w.xstage = take(T * dd * 2);
+    w.ystage = take(T * dd * 4);
     w.total = o;
     return w;
 }
@@ -131,6 +138,9 @@ struct moe_ctx {
     int page_cap = 0;
     uint32_t seq = 0;
     std::vector<cudaEvent_t> miss_ev;   // [2 * page_cap]: W13 part, W2 part of miss j
+    cudaEvent_t ev_routed = nullptr;    // prefill: this layer's routed misses copied
+    std::vector<cudaEvent_t> ev_pf;     // [L]: prefetch copies for a layer issued
+    std::vector<char> pf_pending;       // [L]: a prefetch for the layer is not yet waited on
     // state
     moe_status state = MOE_OK;
     std::string err;
@@ -205,7 +215,7 @@ moe_status resolve_timing(moe_ctx *ctx) {
 
 GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int combine = 0) {
     const moe_dims &D = ctx->dims;
-    GemvArgs g;
+    GemvArgs g{};
     g.mode = mode;
     g.jobs = ctx->dws.jobs;
     g.n_jobs = ctx->dws.n_jobs;
@@ -247,14 +257,52 @@ moe_status device_error(moe_ctx *ctx) {
     return MOE_ERR_CUDA;
 }
 
+// Bounded host wait for the device's miss list (sequence number `seq`).
+moe_status wait_miss_list(moe_ctx *ctx, uint32_t seq) {
+    const auto t0 = std::chrono::steady_clock::now();
+    uint64_t spins = 0;
+    while (ctx->page_h->seq != seq) {
+        _mm_pause();
+        if ((++spins & 4095) == 0) {
+            const double el = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+            if (el > ctx->wait_limit) {
+                ctx->state = MOE_ERR_STATE;
+                ctx->err = "timed out waiting for the device miss list";
+                return MOE_ERR_TIMEOUT;
+            }
+        }
+    }
+    std::atomic_thread_fence(std::memory_order_acquire);
+    return MOE_OK;
+}
+
+void fill_trace(moe_ctx *ctx, int32_t layer, int nrouted, int nev, moe_layer_trace *trace) {
+    if (!trace) return;
+    const HostEvent *ev = ctx->page_h->ev;
+    trace->count = nev;
+    const int n = nev < trace->capacity ? nev : trace->capacity;
+    for (int j = 0; j < n && trace->events; ++j) {
+        moe_cache_event &o = trace->events[j];
+        o.layer = j < nrouted ? layer : layer + 1;
+        o.expert = ev[j].expert;
+        o.slot = ev[j].slot;
+        o.hit = ev[j].flags & 1;
+        o.evicted_key = ev[j].evicted;
+        o.prefetch = (ev[j].flags >> 1) & 1;
+        o.reserved = 0;
+    }
+}
+
 moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
                           moe_layer_trace *trace) {
     const moe_dims &D = ctx->dims;
     if (ctx->page_h->error) return device_error(ctx);
     const uint32_t seq = ++ctx->seq;
-    RouteArgs ra;
+    RouteArgs ra{};
     ra.Wr = ctx->router_w + (size_t)layer * D.E * D.d;
     ra.Wr_next = layer + 1 < D.L ? ra.Wr + (size_t)D.E * D.d : nullptr;
+    ra.L = D.L;
+    ra.prefetch = 0;
     ra.x = static_cast<const __nv_bfloat16 *>(x);
     ra.T = T;
     ra.E = D.E;
@@ -270,6 +318,10 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     if (ctx->inj_drop_publish > 0) {
         ra.publish = 0;
         --ctx->inj_drop_publish;
+    }
+    if (ctx->pf_pending[layer]) {  // experts prefetched for this layer by a prefill call
+        CK(cudaStreamWaitEvent(ctx->cs, ctx->ev_pf[layer], 0));
+        ctx->pf_pending[layer] = 0;
     }
     TimedLaunch tl;
     time_begin(ctx, tl, MOE_K_ROUTE);
@@ -291,20 +343,8 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
 
     // bounded host wait for the device's miss list
     {
-        auto t0 = std::chrono::steady_clock::now();
-        uint64_t spins = 0;
-        while (ctx->page_h->seq != seq) {
-            _mm_pause();
-            if ((++spins & 4095) == 0) {
-                double el = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
-                if (el > ctx->wait_limit) {
-                    ctx->state = MOE_ERR_STATE;
-                    ctx->err = "timed out waiting for the device miss list";
-                    return MOE_ERR_TIMEOUT;
-                }
-            }
-        }
-        std::atomic_thread_fence(std::memory_order_acquire);
+        const moe_status ws_ = wait_miss_list(ctx, seq);
+        if (ws_ != MOE_OK) return ws_;
     }
     if (ctx->page_h->error) return device_error(ctx);
     const int nev = ctx->page_h->n_events;
@@ -369,20 +409,128 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     ctx->stats.misses += nev - hits;
     ctx->stats.evictions += evictions;
     ctx->stats.forward_calls += 1;
-    if (trace) {
-        trace->count = nev;
-        const int n = nev < trace->capacity ? nev : trace->capacity;
-        for (int j = 0; j < n && trace->events; ++j) {
-            moe_cache_event &o = trace->events[j];
-            o.layer = layer;
-            o.expert = ev[j].expert;
-            o.slot = ev[j].slot;
-            o.hit = ev[j].flags & 1;
-            o.evicted_key = ev[j].evicted;
-            o.prefetch = (ev[j].flags >> 1) & 1;
-            o.reserved = 0;
-        }
+    fill_trace(ctx, layer, nev, nev, trace);
+    ctx->last_T = T;
+    return MOE_OK;
+}
+
+// One layer of a prefill chunk (T > 32 rows): W4A4 through the expert GEMV,
+// with the next layer's experts prefetched when MOE_CACHE_PREFETCH_NEXT is set.
+moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
+                           moe_layer_trace *trace) {
+    const moe_dims &D = ctx->dims;
+    if (ctx->page_h->error) return device_error(ctx);
+    const uint32_t seq = ++ctx->seq;
+    RouteArgs ra{};
+    ra.Wr = ctx->router_w + (size_t)layer * D.E * D.d;
+    ra.Wr_next = nullptr;
+    ra.L = D.L;
+    ra.prefetch = (ctx->flags & MOE_CACHE_PREFETCH_NEXT) ? 1 : 0;
+    ra.x = static_cast<const __nv_bfloat16 *>(x);
+    ra.T = T;
+    ra.E = D.E;
+    ra.d = D.d;
+    ra.k = D.k;
+    ra.renorm = D.renormalize;
+    ra.layer = layer;
+    ra.ws = ctx->dws;
+    ra.tab = ctx->tab;
+    ra.page = ctx->page_d;
+    ra.seq = seq;
+    ra.publish = 1;
+    if (ctx->inj_drop_publish > 0) {
+        ra.publish = 0;
+        --ctx->inj_drop_publish;
     }
+    CK(cudaMemsetAsync(ctx->dws.cnt, 0, (size_t)D.E * 4, ctx->cs));
+    TimedLaunch tr;
+    time_begin(ctx, tr, MOE_K_PREFILL_ROUTE);
+    CK(launch_prefill_route(ra, ctx->cs));
+    time_end(ctx, tr, (double)D.E * D.d * 2 + (double)T * D.d * 2);
+    CK(launch_prefill_scatter(ra, ctx->cs));
+    CK(launch_quant_x(ra.x, T, D.d, ctx->dws.xh, ctx->cs));
+
+    const moe_status ws_ = wait_miss_list(ctx, seq);
+    if (ws_ != MOE_OK) return ws_;
+    if (ctx->page_h->error) return device_error(ctx);
+    const int nev = ctx->page_h->n_events, n = ctx->page_h->n_jobs;
+    const HostEvent *ev = ctx->page_h->ev;
+
+    // copies on the copy stream: this layer's misses (the layer's compute waits
+    // for them), then the next layer's prefetch misses (its compute waits)
+    auto copy_record = [&](int lyr, const HostEvent &e) -> moe_status {
+        if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
+            ctx->state = MOE_ERR_STATE;
+            ctx->err = "injected failure of an H2D copy issue";
+            return MOE_ERR_CUDA;
+        }
+        const int64_t rec_idx = ((int64_t)lyr * D.E + e.expert) % ctx->P;
+        CK(cudaMemcpyAsync(ctx->arena + (int64_t)e.slot * ctx->lay.bytes, ctx->pool + rec_idx * ctx->lay.bytes,
+                           ctx->lay.bytes, cudaMemcpyHostToDevice, ctx->xs));
+        ctx->stats.h2d_copies += 1;
+        ctx->stats.h2d_bytes += ctx->lay.bytes;
+        return MOE_OK;
+    };
+    int nrm = 0, npm = 0;
+    for (int j = 0; j < n; ++j) {
+        if (ev[j].flags & 1) continue;
+        const moe_status st = copy_record(layer, ev[j]);
+        if (st != MOE_OK) return st;
+        ++nrm;
+    }
+    if (nrm > 0) {
+        CK(cudaEventRecord(ctx->ev_routed, ctx->xs));
+        CK(cudaStreamWaitEvent(ctx->cs, ctx->ev_routed, 0));
+    }
+    if (ctx->pf_pending[layer]) {  // experts prefetched for this layer by the previous call
+        CK(cudaStreamWaitEvent(ctx->cs, ctx->ev_pf[layer], 0));
+        ctx->pf_pending[layer] = 0;
+    }
+    for (int j = n; j < nev; ++j) {
+        if (ev[j].flags & 1) continue;
+        const moe_status st = copy_record(layer + 1, ev[j]);
+        if (st != MOE_OK) return st;
+        ++npm;
+    }
+    if (npm > 0) {
+        CK(cudaEventRecord(ctx->ev_pf[layer + 1], ctx->xs));
+        ctx->pf_pending[layer + 1] = 1;
+    }
+
+    // experts: gate/up (+SwiGLU, fp32 h), h quantized per row, down, combine
+    const int grid_y = n + (D.has_shared ? 1 : 0);
+    GemvArgs gu = gemv_args(ctx, layer, T, kGateUp, -1);
+    gu.all_jobs = 1;
+    gu.h32_out = ctx->dws.h32;
+    gu.shared_slot = D.has_shared ? n : -1;
+    TimedLaunch tg;
+    time_begin(ctx, tg, MOE_K_PREFILL_GATEUP);
+    CK(launch_gemv(gu, grid_y, ctx->cs));
+    time_end(ctx, tg, grid_y * w13_bytes(ctx));
+    CK(launch_quant_h(ctx->dws.h32, T, D.k, D.F, D.has_shared, ctx->dws.hh, ctx->cs));
+    GemvArgs dn = gemv_args(ctx, layer, T, kDown, -1, 0);
+    dn.all_jobs = 1;
+    dn.shared_slot = D.has_shared ? n : -1;
+    TimedLaunch td;
+    time_begin(ctx, td, MOE_K_PREFILL_DOWN);
+    CK(launch_gemv(dn, grid_y, ctx->cs));
+    time_end(ctx, td, grid_y * w2_bytes(ctx));
+    CK(launch_combine(ctx->dws.part, ctx->dws.gates, y, T, D.k, D.d, D.has_shared, ctx->cs));
+
+    int64_t hits = 0, evictions = 0, pf_evict = 0;
+    for (int j = 0; j < n; ++j) {  // (npm: prefetch misses counted above)
+        hits += ev[j].flags & 1;
+        evictions += ev[j].evicted >= 0;
+    }
+    for (int j = n; j < nev; ++j) pf_evict += ev[j].evicted >= 0;
+    ctx->stats.lookups += n;
+    ctx->stats.hits += hits;
+    ctx->stats.misses += n - hits;
+    ctx->stats.evictions += evictions + pf_evict;
+    ctx->stats.prefetch_lookups += nev - n;
+    ctx->stats.prefetch_misses += npm;
+    ctx->stats.forward_calls += 1;
+    fill_trace(ctx, layer, n, nev, trace);
     ctx->last_T = T;
     return MOE_OK;
 }
@@ -460,6 +608,10 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     ctx->dws.xh = reinterpret_cast<__half *>(w + L.xh);
     ctx->dws.hh = reinterpret_cast<__half *>(w + L.hh);
     ctx->dws.part = reinterpret_cast<float *>(w + L.part);
+    ctx->dws.cnt = L.cnt >= 0 ? reinterpret_cast<int32_t *>(w + L.cnt) : nullptr;
+    ctx->dws.fill = L.fill >= 0 ? reinterpret_cast<int32_t *>(w + L.fill) : nullptr;
+    ctx->dws.jobidx = L.jobidx >= 0 ? reinterpret_cast<int32_t *>(w + L.jobidx) : nullptr;
+    ctx->dws.h32 = L.h32 >= 0 ? reinterpret_cast<float *>(w + L.h32) : nullptr;
 
     ctx->page_cap = 2 * dims->E + 8;
     const size_t page_bytes = sizeof(HostPage) + sizeof(HostEvent) * ctx->page_cap;
@@ -470,6 +622,15 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
         memset((void *)ctx->page_h, 0, page_bytes);
         ctx->miss_ev.resize(2 * ctx->page_cap, nullptr);
         for (auto &ev : ctx->miss_ev) {
+            e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+            if (e != cudaSuccess) break;
+        }
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_routed, cudaEventDisableTiming);
+    if (e == cudaSuccess) {
+        ctx->ev_pf.resize(dims->L, nullptr);
+        ctx->pf_pending.assign(dims->L, 0);
+        for (auto &ev : ctx->ev_pf) {
             e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
             if (e != cudaSuccess) break;
         }
@@ -516,6 +677,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         CK(cudaMemsetAsync(ctx->dws.ticket2, 0, 4, ctx->cs));
         ctx->pending.clear();
         ctx->page_h->error = 0;
+        std::fill(ctx->pf_pending.begin(), ctx->pf_pending.end(), 0);
         memset(&ctx->stats, 0, sizeof ctx->stats);
         ctx->state = MOE_OK;
         ctx->err.clear();
@@ -532,7 +694,7 @@ moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t
     const moe_dims &D = ctx->dims;
     if (layer < 0 || layer >= D.L || T < 1 || T > D.max_rows || !x || !y) return MOE_ERR_ARG;
     if (T <= kDecodeMaxRows) return forward_decode(ctx, layer, x, T, y, trace);
-    return MOE_ERR_UNSUPPORTED;
+    return forward_prefill(ctx, layer, x, T, y, trace);
 }
 
 moe_status moe_layer_forward_host(moe_ctx *ctx, int32_t layer, const void *x_host, int32_t T,
@@ -693,6 +855,9 @@ void moe_layer_destroy(moe_ctx *ctx) {
     for (auto e : ctx->ev_pool) cudaEventDestroy(e);
     for (auto e : ctx->miss_ev)
         if (e) cudaEventDestroy(e);
+    for (auto e : ctx->ev_pf)
+        if (e) cudaEventDestroy(e);
+    if (ctx->ev_routed) cudaEventDestroy(ctx->ev_routed);
     if (ctx->page_h) cudaFreeHost(ctx->page_h);
     delete ctx;
 }

@@ -50,11 +50,12 @@ struct __align__(16) HostEvent {
 };
 struct HostPage {
     volatile uint32_t seq;    // written last by the device
-    int32_t n_events;
-    int32_t n_jobs;
-    int32_t n_misses;
+    int32_t n_events;         // routed entries first, then prefetch entries
+    int32_t n_jobs;           // routed entries
+    int32_t n_misses;         // routed misses
     volatile int32_t error;   // nonzero: a kernel check failed (see diag)
-    int32_t pad[3];
+    int32_t n_prefetch_misses;
+    int32_t pad[2];
     int32_t diag[16];         // where: kernel mode, block, sizes, address low bits
     uint32_t phase_ns[8];     // route kernel, last CTA: ns spent in each phase (globaltimer)
     HostEvent ev[1];          // [capacity]
@@ -74,10 +75,17 @@ struct DecodeWs {
     float *part;         // [maxT][k+1][d] per-selection expert outputs (p = k: shared)
     uint32_t *ticket;    // last-CTA counter of the route kernel
     uint32_t *ticket2;   // last-CTA counter of the combining down launch
+    // prefill only (T > 32)
+    int32_t *cnt;        // [E] rows per expert
+    int32_t *fill;       // [E] scatter cursors
+    int32_t *jobidx;     // [E] job of an expert, -1 if unused
+    float *h32;          // [T][k+1][F] fp32 h before its activation quantization
 };
 
 struct RouteArgs {
     const __nv_bfloat16 *Wr;  // [E][d] of this layer
+    int L;                    // layers (prefill prefetches layer + 1 < L)
+    int prefetch;             // prefill: also look up all experts of the next layer
     const __nv_bfloat16 *Wr_next;  // next layer's router (prefetched into L2) or null
     const __nv_bfloat16 *x;   // [T][d]
     int T, E, d, k, renorm, layer;
@@ -96,6 +104,8 @@ struct GemvArgs {
     const int32_t *n_jobs;
     const RowRef *rowrefs;
     int only_job;          // >= 0: process just this job; -1: every hit job (+ shared)
+    int all_jobs;          // with only_job = -1: hit and missed jobs alike (prefill)
+    float *h32_out;        // gate/up: write fp32 h here instead of the fp16 (hi, lo) pair
     int shared_slot;       // gridDim.y index of the shared job, -1 if none
     const uint8_t *arena;
     int64_t rec_bytes;
@@ -119,5 +129,12 @@ struct GemvArgs {
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s);
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
+cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s);
+cudaError_t launch_quant_x(const __nv_bfloat16 *x, int T, int d, __half *xh, cudaStream_t s);
+cudaError_t launch_quant_h(const float *h32, int T, int k, int F, int has_shared, __half *hh,
+                           cudaStream_t s);
+cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
+                           int has_shared, cudaStream_t s);
 
 }  // namespace moe

@@ -142,8 +142,9 @@ __device__ void split_x(const RouteArgs &a) {
     }
 }
 
-// Softmax + top-k of row t by one warp; writes idx/gates of the row in ascending id.
-__device__ void topk_row(const RouteArgs &a, int t) {
+// Softmax + top-k of row t by one warp; writes idx/gates of the row in ascending
+// id and returns the expert selected by this lane (lanes < k), else -1.
+__device__ int topk_row(const RouteArgs &a, int t) {
     const int lane = threadIdx.x & 31;
     const float *z = a.ws.z + (size_t)t * a.E;
     const int nv = (a.E + 31) >> 5;
@@ -198,6 +199,146 @@ __device__ void topk_row(const RouteArgs &a, int t) {
     if (lane < a.k) {
         a.ws.idx[t * a.k + rank] = my_idx;
         a.ws.gates[t * a.k + rank] = g;
+    }
+    return lane < a.k ? my_idx : -1;
+}
+
+constexpr int kLookupMax = kMaxK * kDecodeMaxRows;  // entries of one lookup batch (>= kMaxE)
+
+// Shared memory of one lookup batch.
+struct LookupSmem {
+    int32_t exp[kLookupMax];    // in: the batch's distinct experts, ascending
+    int32_t slot[kLookupMax];   // out: slot of a hit, or -2 - slot for a miss
+    int32_t evict[kLookupMax];  // out: key evicted from the slot, or -1
+    int32_t rank[kLookupMax];
+    int32_t victim[kLookupMax];
+    int32_t old[kLookupMax];
+    uint32_t hitmap[kMaxSlotBits / 32];
+    unsigned long long clock, lastv;
+    int nf, nhit, nmiss;
+    unsigned long long redv[kRouteThreads / 32];
+    int reds[kRouteThreads / 32];
+};
+
+// One lookup batch of `layer` over sm.exp[0..n), run by all threads of the CTA.
+// All table reads happen in one parallel round (the batch's map entries, the
+// header, every slot's stamp); hits get the newest stamps in ascending id;
+// each miss in ascending id takes the lowest never-used slot, else the next
+// least recently used non-hit slot (the smallest stamps, found by block-wide
+// argmin rounds: stamps are unique, so round r takes the minimum above round
+// r-1's).  Same result as the sequential rule.  *t_read: time after the reads.
+__device__ void lookup_batch(const Table &tab, int layer, int E, int n, LookupSmem &sm,
+                             unsigned long long *t_read) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int64_t keybase = (int64_t)layer * E;
+    const int C = (int)tab.C;
+    for (int i = threadIdx.x; i < kMaxSlotBits / 32; i += blockDim.x) sm.hitmap[i] = 0u;
+    for (int j = threadIdx.x; j < n; j += blockDim.x) sm.slot[j] = tab.map[keybase + sm.exp[j]];
+    if (threadIdx.x == 0) { sm.clock = tab.hdr->clock; sm.nf = tab.hdr->next_free; }
+    unsigned long long sv[kStampRegs];  // this thread's slots tid + 256*i
+#pragma unroll
+    for (int i = 0; i < kStampRegs; ++i) {
+        const int sl = threadIdx.x + kRouteThreads * i;
+        sv[i] = sl < C ? tab.stamp[sl] : ~0ull;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && t_read) *t_read = global_ns();
+    for (int j = threadIdx.x; j < n; j += blockDim.x)
+        if (sm.slot[j] >= 0) atomicOr(&sm.hitmap[sm.slot[j] >> 5], 1u << (sm.slot[j] & 31));
+    if (warp == 0) {  // ranks: hits and misses, each in ascending id
+        int hc = 0, mc = 0;
+        for (int j0 = 0; j0 < n; j0 += 32) {
+            const int j = j0 + lane;
+            const bool valid = j < n, hit = valid && sm.slot[j] >= 0;
+            const unsigned hm = __ballot_sync(0xffffffffu, hit);
+            const unsigned mm = __ballot_sync(0xffffffffu, valid && !hit);
+            const unsigned lt = (1u << lane) - 1u;
+            if (valid) sm.rank[j] = hit ? hc + __popc(hm & lt) : mc + __popc(mm & lt);
+            hc += __popc(hm);
+            mc += __popc(mm);
+        }
+        if (lane == 0) { sm.nhit = hc; sm.nmiss = mc; }
+    }
+    __syncthreads();
+    const int nhit = sm.nhit, nmiss = sm.nmiss, nf = sm.nf;
+    const int nfree = C - nf;
+    const int nevict = nmiss > nfree ? nmiss - nfree : 0;
+    unsigned long long last = 0ull;
+    for (int r = 0; r < nevict; ++r) {
+        unsigned long long bv = ~0ull;
+        int bs = -1;
+#pragma unroll
+        for (int i = 0; i < kStampRegs; ++i) {
+            const int sl = threadIdx.x + kRouteThreads * i;
+            if (sl < C && sv[i] > last && sv[i] < bv && !(sm.hitmap[sl >> 5] & (1u << (sl & 31)))) {
+                bv = sv[i];
+                bs = sl;
+            }
+        }
+        for (int sl = threadIdx.x + kRouteThreads * kStampRegs; sl < C; sl += kRouteThreads) {
+            const unsigned long long v = tab.stamp[sl];  // caches beyond the register tile
+            if (v > last && v < bv && !(sm.hitmap[sl >> 5] & (1u << (sl & 31)))) { bv = v; bs = sl; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int os = __shfl_xor_sync(0xffffffffu, bs, o);
+            if (ov < bv) { bv = ov; bs = os; }
+        }
+        if (lane == 0) { sm.redv[warp] = bv; sm.reds[warp] = bs; }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            unsigned long long mv = sm.redv[0];
+            int ms = sm.reds[0];
+            for (int w = 1; w < nw; ++w)
+                if (sm.redv[w] < mv) { mv = sm.redv[w]; ms = sm.reds[w]; }
+            sm.victim[r] = ms;
+            sm.lastv = mv;
+        }
+        __syncthreads();
+        last = sm.lastv;
+    }
+    for (int r = threadIdx.x; r < nevict; r += blockDim.x) sm.old[r] = tab.owner[sm.victim[r]];
+    __syncthreads();
+    const unsigned long long clock = sm.clock;
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        const int s0 = sm.slot[j];
+        if (s0 >= 0) {  // hit: newest stamps in ascending id
+            tab.stamp[s0] = clock + 1 + sm.rank[j];
+            sm.evict[j] = -1;
+        } else {        // miss: a never-used slot, else the next least recently used
+            const int m = sm.rank[j];
+            int sl, ev = -1;
+            if (m < nfree) sl = nf + m;
+            else { sl = sm.victim[m - nfree]; ev = sm.old[m - nfree]; }
+            const int key = (int)(keybase + sm.exp[j]);
+            if (ev >= 0) tab.map[ev] = -1;
+            tab.map[key] = sl;
+            tab.owner[sl] = key;
+            tab.stamp[sl] = clock + 1 + nhit + m;
+            sm.slot[j] = -2 - sl;
+            sm.evict[j] = ev;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        tab.hdr->clock = clock + n;
+        tab.hdr->next_free = nf + (nmiss < nfree ? nmiss : nfree);
+    }
+    __syncthreads();
+}
+
+// Warp 0: one 16-byte record per batch entry at page->ev[base + j].
+__device__ void publish_events(HostPage *page, int base, const LookupSmem &sm, int n, int prefetch) {
+    const int lane = threadIdx.x & 31;
+    for (int j = lane; j < n; j += 32) {
+        const int sj = sm.slot[j];
+        HostEvent he;
+        he.expert = sm.exp[j];
+        he.slot = sj >= 0 ? sj : -2 - sj;
+        he.flags = (sj >= 0 ? 1 : 0) | (prefetch << 1);
+        he.evicted = sm.evict[j];
+        *reinterpret_cast<int4 *>(&page->ev[base + j]) = *reinterpret_cast<int4 *>(&he);
     }
 }
 
@@ -254,12 +395,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     __shared__ uint32_t s_bits[kMaxE / 32];
     __shared__ int s_base[kMaxE / 32];
     __shared__ int s_njobs;
-    __shared__ int32_t s_exp[kMaxK * kDecodeMaxRows];
+    __shared__ LookupSmem sm;
     __shared__ int32_t s_cnt[kMaxK * kDecodeMaxRows];
     __shared__ int32_t s_off[kMaxK * kDecodeMaxRows];
-    __shared__ int32_t s_slot[kMaxK * kDecodeMaxRows];
-    __shared__ int32_t s_evict[kMaxK * kDecodeMaxRows];
     __shared__ int32_t s_idx[kMaxK * kDecodeMaxRows];
+    int32_t *s_exp = sm.exp;
     for (int i = threadIdx.x; i < kMaxE / 32; i += blockDim.x) s_bits[i] = 0u;
     __syncthreads();
     if (threadIdx.x == 0) t_topk = global_ns();
@@ -323,128 +463,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     __syncthreads();
     if (threadIdx.x == 0) t_jobs = global_ns();
 
-    // ---- cache lookup: one batch, ascending id.  All table reads in one round:
-    // the batch's map entries, the header, and every slot's stamp.
-    const int64_t keybase = (int64_t)a.layer * a.E;
-    const int C = (int)a.tab.C;
-    __shared__ unsigned long long s_clock, s_lastv;
-    __shared__ int s_nf, s_nhit, s_nmiss, s_pick;
-    __shared__ unsigned long long s_redv[kRouteThreads / 32];
-    __shared__ int s_reds[kRouteThreads / 32];
-    __shared__ uint32_t s_hitmap[kMaxSlotBits / 32];
-    __shared__ int32_t s_rank[kMaxK * kDecodeMaxRows];
-    __shared__ int32_t s_victim[kMaxK * kDecodeMaxRows];
-    __shared__ int32_t s_old[kMaxK * kDecodeMaxRows];
-    for (int i = threadIdx.x; i < kMaxSlotBits / 32; i += blockDim.x) s_hitmap[i] = 0u;
-    for (int j = threadIdx.x; j < njobs; j += blockDim.x) s_slot[j] = a.tab.map[keybase + s_exp[j]];
-    if (threadIdx.x == 0) { s_clock = a.tab.hdr->clock; s_nf = a.tab.hdr->next_free; }
-    unsigned long long sv[kStampRegs];  // this thread's slots tid + 256*i
-#pragma unroll
-    for (int i = 0; i < kStampRegs; ++i) {
-        const int sl = threadIdx.x + kRouteThreads * i;
-        sv[i] = sl < C ? a.tab.stamp[sl] : ~0ull;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) t_read = global_ns();
-    for (int j = threadIdx.x; j < njobs; j += blockDim.x)
-        if (s_slot[j] >= 0) atomicOr(&s_hitmap[s_slot[j] >> 5], 1u << (s_slot[j] & 31));
-    if (warp == 0) {  // ranks: hits and misses, each in ascending id
-        int hc = 0, mc = 0;
-        for (int j0 = 0; j0 < njobs; j0 += 32) {
-            const int j = j0 + lane;
-            const bool valid = j < njobs, hit = valid && s_slot[j] >= 0;
-            const unsigned hm = __ballot_sync(0xffffffffu, hit);
-            const unsigned mm = __ballot_sync(0xffffffffu, valid && !hit);
-            const unsigned lt = (1u << lane) - 1u;
-            if (valid) s_rank[j] = hit ? hc + __popc(hm & lt) : mc + __popc(mm & lt);
-            hc += __popc(hm);
-            mc += __popc(mm);
-        }
-        if (lane == 0) { s_nhit = hc; s_nmiss = mc; }
-    }
-    __syncthreads();
-    const int nhit = s_nhit, nmiss = s_nmiss, nf = s_nf;
-    const int nfree = C - nf;
-    const int nevict = nmiss > nfree ? nmiss - nfree : 0;
-    // victims: the nevict non-hit slots with the smallest stamps (stamps are
-    // unique, so round r takes the minimum above round r-1's)
-    unsigned long long last = 0ull;
-    for (int r = 0; r < nevict; ++r) {
-        unsigned long long bv = ~0ull;
-        int bs = -1;
-#pragma unroll
-        for (int i = 0; i < kStampRegs; ++i) {
-            const int sl = threadIdx.x + kRouteThreads * i;
-            if (sl < C && sv[i] > last && sv[i] < bv && !(s_hitmap[sl >> 5] & (1u << (sl & 31)))) {
-                bv = sv[i];
-                bs = sl;
-            }
-        }
-        for (int sl = threadIdx.x + kRouteThreads * kStampRegs; sl < C; sl += kRouteThreads) {
-            const unsigned long long v = a.tab.stamp[sl];  // caches beyond the register tile
-            if (v > last && v < bv && !(s_hitmap[sl >> 5] & (1u << (sl & 31)))) { bv = v; bs = sl; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int os = __shfl_xor_sync(0xffffffffu, bs, o);
-            if (ov < bv) { bv = ov; bs = os; }
-        }
-        if (lane == 0) { s_redv[warp] = bv; s_reds[warp] = bs; }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            unsigned long long mv = s_redv[0];
-            int ms = s_reds[0];
-            for (int w = 1; w < nw; ++w)
-                if (s_redv[w] < mv) { mv = s_redv[w]; ms = s_reds[w]; }
-            s_victim[r] = ms;
-            s_lastv = mv;
-        }
-        __syncthreads();
-        last = s_lastv;
-    }
-    for (int r = threadIdx.x; r < nevict; r += blockDim.x) s_old[r] = a.tab.owner[s_victim[r]];
-    __syncthreads();
-    // slots, stamps and table writes (independent per job)
-    const unsigned long long clock = s_clock;
-    for (int j = threadIdx.x; j < njobs; j += blockDim.x) {
-        const int s0 = s_slot[j];
-        if (s0 >= 0) {  // hit: newest stamps in ascending id
-            a.tab.stamp[s0] = clock + 1 + s_rank[j];
-            s_evict[j] = -1;
-        } else {        // miss: a never-used slot, else the next least recently used
-            const int m = s_rank[j];
-            int sl, ev = -1;
-            if (m < nfree) sl = nf + m;
-            else { sl = s_victim[m - nfree]; ev = s_old[m - nfree]; }
-            const int key = (int)(keybase + s_exp[j]);
-            if (ev >= 0) a.tab.map[ev] = -1;
-            a.tab.map[key] = sl;
-            a.tab.owner[sl] = key;
-            a.tab.stamp[sl] = clock + 1 + nhit + m;
-            s_slot[j] = -2 - sl;
-            s_evict[j] = ev;
-        }
-    }
+    // ---- cache lookup: one batch, ascending id
+    lookup_batch(a.tab, a.layer, a.E, njobs, sm, &t_read);
+    const int nmiss = sm.nmiss;
     if (threadIdx.x == 0) {
-        a.tab.hdr->clock = clock + njobs;
-        a.tab.hdr->next_free = nf + (nmiss < nfree ? nmiss : nfree);
         *a.ws.n_misses = nmiss;
+        t_table = global_ns();
     }
-    __syncthreads();
-    if (threadIdx.x == 0) t_table = global_ns();
 
     // ---- publish: one 16-byte record per entry, the counts, phase times, then the flag
     if (warp == 0) {
-        for (int j = lane; j < njobs; j += 32) {
-            const int sj = s_slot[j];
-            HostEvent he;
-            he.expert = s_exp[j];
-            he.slot = sj >= 0 ? sj : -2 - sj;
-            he.flags = sj >= 0 ? 1 : 0;
-            he.evicted = s_evict[j];
-            *reinterpret_cast<int4 *>(&a.page->ev[j]) = *reinterpret_cast<int4 *>(&he);
-        }
+        publish_events(a.page, 0, sm, njobs, 0);
         if (lane == 0) {
             a.page->n_events = njobs;
             a.page->n_jobs = njobs;
@@ -468,7 +497,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     }
     __syncthreads();
     for (int j = threadIdx.x; j < njobs; j += blockDim.x) {
-        const int sj = s_slot[j];
+        const int sj = sm.slot[j];
         Job jb;
         jb.expert = s_exp[j];
         jb.slot = sj >= 0 ? sj : -2 - sj;
@@ -482,6 +511,178 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
         *a.ws.n_jobs = njobs;
         *a.ws.ticket = 0u;
     }
+}
+
+// ------------------------------------------------------------------ prefill --
+// Rows of a prefill chunk (T > 32): logits per (8 rows x 64 experts) CTA with
+// the rows in shared memory; top-k per row with per-expert counts; one CTA for
+// the lookup of the layer's distinct experts and of all experts of the next
+// layer (the prefetch batch, holude.com "長いプロンプトとエージェント処理も意識している":
+// the next layer's experts stream in while the current layer computes); then
+// the rows are scattered into per-expert groups.
+constexpr int kPfRows = 8, kPfExperts = 64;
+
+template <int NV>
+__global__ void __launch_bounds__(kRouteThreads) prefill_logits_kernel(RouteArgs a) {
+    extern __shared__ __align__(16) uint4 xsm[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t0 = blockIdx.x * kPfRows, e0 = blockIdx.y * kPfExperts;
+    const int nr = a.T - t0 < kPfRows ? a.T - t0 : kPfRows;
+    const int nvec = a.d >> 3;
+    const uint4 *xg = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.d);
+    for (int i = threadIdx.x; i < nr * nvec; i += blockDim.x) xsm[i] = __ldg(xg + i);
+    __syncthreads();
+    for (int ee = 0; ee < kPfExperts / (kRouteThreads / 32); ++ee) {
+        const int e = e0 + warp * (kPfExperts / (kRouteThreads / 32)) + ee;
+        if (e >= a.E) break;
+        const uint4 *wrow = reinterpret_cast<const uint4 *>(a.Wr + (size_t)e * a.d);
+        uint4 w[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int v = lane + 32 * i;
+            w[i] = v < nvec ? __ldg(wrow + v) : make_uint4(0, 0, 0, 0);
+        }
+        float acc[kPfRows];
+#pragma unroll
+        for (int r = 0; r < kPfRows; ++r) acc[r] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int v = lane + 32 * i;
+            if (v < nvec) {
+                float wf[8];
+                bf16x8_to_f32(w[i], wf);
+#pragma unroll
+                for (int r = 0; r < kPfRows; ++r) {
+                    if (r < nr) {
+                        float xf[8];
+                        bf16x8_to_f32(xsm[r * nvec + v], xf);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[r] = fmaf(wf[j], xf[j], acc[r]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < kPfRows; ++r) {
+            const float sum = warp_sum(acc[r]);
+            if (lane == 0 && r < nr) a.ws.z[(size_t)(t0 + r) * a.E + e] = sum;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kRouteThreads) prefill_topk_kernel(RouteArgs a) {
+    const int t = blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5);
+    if (t >= a.T) return;
+    const int e = topk_row(a, t);
+    if (e >= 0) atomicAdd(&a.ws.cnt[e], 1);
+}
+
+__global__ void __launch_bounds__(kRouteThreads) prefill_lookup_kernel(RouteArgs a) {
+    __shared__ LookupSmem sm;
+    __shared__ int32_t s_cnt[kMaxE], s_off[kMaxE];
+    __shared__ int s_n, s_nmiss;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp == 0) {  // the layer's distinct experts, ascending, with their row counts
+        int nj = 0;
+        for (int e0 = 0; e0 < a.E; e0 += 32) {
+            const int e = e0 + lane;
+            const int c = e < a.E ? a.ws.cnt[e] : 0;
+            const unsigned m = __ballot_sync(0xffffffffu, c > 0);
+            const int pos = nj + __popc(m & ((1u << lane) - 1u));
+            if (c > 0) { sm.exp[pos] = e; s_cnt[pos] = c; a.ws.jobidx[e] = pos; }
+            else if (e < a.E) a.ws.jobidx[e] = -1;
+            if (e < a.E) a.ws.fill[e] = 0;
+            nj += __popc(m);
+        }
+        int carry = 0;  // exclusive scan of the counts: each group's first row
+        for (int j0 = 0; j0 < nj; j0 += 32) {
+            const int j = j0 + lane;
+            const int c = j < nj ? s_cnt[j] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (j < nj) s_off[j] = carry + incl - c;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) s_n = nj;
+    }
+    __syncthreads();
+    const int n = s_n;
+    lookup_batch(a.tab, a.layer, a.E, n, sm, nullptr);
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        const int sj = sm.slot[j];
+        Job jb;
+        jb.expert = sm.exp[j];
+        jb.slot = sj >= 0 ? sj : -2 - sj;
+        jb.hit = sj >= 0;
+        jb.nrows = s_cnt[j];
+        jb.row_off = s_off[j];
+        jb.pad[0] = jb.pad[1] = jb.pad[2] = 0;
+        a.ws.jobs[j] = jb;
+    }
+    if (warp == 0) publish_events(a.page, 0, sm, n, 0);
+    if (threadIdx.x == 0) {
+        s_nmiss = sm.nmiss;
+        *a.ws.n_jobs = n;
+        *a.ws.n_misses = sm.nmiss;
+    }
+    __syncthreads();  // the routed batch is consumed before the prefetch batch reuses sm
+    int npf = 0, pf_miss = 0;
+    if (a.prefetch && a.layer + 1 < a.L) {
+        for (int e = threadIdx.x; e < a.E; e += blockDim.x) sm.exp[e] = e;
+        __syncthreads();
+        lookup_batch(a.tab, a.layer + 1, a.E, a.E, sm, nullptr);
+        if (warp == 0) publish_events(a.page, n, sm, a.E, 1);
+        npf = a.E;
+        pf_miss = sm.nmiss;
+    }
+    if (warp == 0) {
+        if (lane == 0) {
+            a.page->n_events = n + npf;
+            a.page->n_jobs = n;
+            a.page->n_misses = s_nmiss;
+            a.page->n_prefetch_misses = pf_miss;
+        }
+        __threadfence_system();
+        __syncwarp();
+        if (lane == 0 && a.publish) {
+            __threadfence_system();
+            a.page->seq = a.seq;
+        }
+    }
+}
+
+__global__ void prefill_scatter_kernel(RouteArgs a) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.T * a.k) return;
+    const int e = a.ws.idx[i];
+    const int j = a.ws.jobidx[e];
+    const int pos = a.ws.jobs[j].row_off + atomicAdd(&a.ws.fill[e], 1);
+    a.ws.rowrefs[pos].t = (int16_t)(i / a.k);
+    a.ws.rowrefs[pos].p = (int16_t)(i % a.k);
+}
+
+template <int NV>
+cudaError_t launch_prefill_nv(const RouteArgs &a, cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_logits_kernel<NV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const dim3 grid((a.T + kPfRows - 1) / kPfRows, (a.E + kPfExperts - 1) / kPfExperts);
+    prefill_logits_kernel<NV><<<grid, kRouteThreads, (size_t)kPfRows * a.d * 2, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    prefill_topk_kernel<<<(a.T + kRouteThreads / 32 - 1) / (kRouteThreads / 32), kRouteThreads, 0, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    prefill_lookup_kernel<<<1, kRouteThreads, 0, s>>>(a);
+    return cudaGetLastError();
 }
 
 __global__ void table_reset_kernel(Table t, int64_t nkeys) {
@@ -535,6 +736,25 @@ cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s) {
     if (nv <= 12) return launch_nv<12>(a, grid, s);
     if (nv <= 16) return launch_nv<16>(a, grid, s);
     return cudaErrorInvalidValue;
+}
+
+// Prefill routing: logits, top-k + counts, then the lookup CTA (which
+// publishes the miss and prefetch lists).  The caller zeroes ws.cnt first.
+cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s) {
+    const int nv = ((a.d >> 3) + 31) >> 5;
+    if (nv <= 1) return launch_prefill_nv<1>(a, s);
+    if (nv <= 2) return launch_prefill_nv<2>(a, s);
+    if (nv <= 4) return launch_prefill_nv<4>(a, s);
+    if (nv <= 8) return launch_prefill_nv<8>(a, s);
+    if (nv <= 12) return launch_prefill_nv<12>(a, s);
+    if (nv <= 16) return launch_prefill_nv<16>(a, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s) {
+    const int n = a.T * a.k;
+    prefill_scatter_kernel<<<(n + 255) / 256, 256, 0, s>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s) {

@@ -184,8 +184,14 @@ MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_a
  * compute_stream reaches that point.  The call waits (host side, bounded) for
  * the device's miss list; on timeout it returns MOE_ERR_TIMEOUT and the
  * context is in MOE_ERR_STATE until a reset.  T <= 32 takes the decode path
- * (NVFP4 dequant-GEMV, W4A16); larger T the prefill path (block-scaled NVFP4
- * grouped GEMM, W4A4 with a per-row fp32 activation scale). */
+ * (W4A16: bf16 activations against NVFP4 weights).  Larger T takes the
+ * prefill path: the activations are quantized to NVFP4 per row (E2M1 values,
+ * E4M3 scale per 16, one fp32 scale per row: x per token, h per token and
+ * expert) and multiplied against the NVFP4 weights (W4A4); the lookup batch is
+ * the layer's distinct experts, and with MOE_CACHE_PREFETCH_NEXT a second
+ * batch of all experts of layer + 1 follows, whose misses are copied while
+ * this layer computes (the next call for layer + 1 waits for them).  The trace
+ * lists the routed entries, then the prefetch entries (prefetch = 1, layer + 1). */
 MOE_API moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
                              moe_layer_trace *trace);
 

@@ -304,6 +304,7 @@ EXPORT void orc_expert_w4a4(const uint8_t *rec, int d, int F, const uint16_t *x,
     double tg = rec_tensor_scale(rec, off, 0), tu = rec_tensor_scale(rec, off, 1);
     double td = rec_tensor_scale(rec, off, 2);
     float *hf = (float *)malloc(sizeof(float) * F);
+#pragma omp parallel for schedule(static)
     for (int64_t j = 0; j < F; ++j) {
         double g = 0.0, u = 0.0;
         for (int64_t K = 0; K < d; ++K) {
@@ -315,6 +316,7 @@ EXPORT void orc_expert_w4a4(const uint8_t *rec, int d, int F, const uint16_t *x,
     uint8_t *hc = (uint8_t *)malloc((size_t)F / 2), *hs = (uint8_t *)malloc((size_t)F / 16);
     float sh = orc_tensor_scale_f32(hf, F);
     orc_nvfp4_quantize(hf, F, sh, hc, hs);
+#pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < d; ++i) {
         double acc = 0.0;
         for (int64_t j = 0; j < F; ++j)

@@ -1,0 +1,149 @@
+"""Prefill path on the GPU against the CPU oracle, through the C ABI.
+
+A chunk of T > 32 rows per layer: routing for all rows, one lookup batch of
+the layer's distinct experts (ascending) and, with MOE_CACHE_PREFETCH_NEXT, a
+prefetch batch of all experts of the next layer; experts in W4A4 (per-row
+fp32 activation scales).  Bit-exact: indices, the event sequence (routed and
+prefetch batches), the table, slot contents.  Within 1e-3 relative L2: the
+layer outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from oracle.workloads import conditioned_decode, conditioned_prefill, decode_trace, prefill_trace
+from synth import problem as sp
+from expert_offload_caching_b200 import abi
+from expert_offload_caching_b200.runtime import LayerStack, new_trace, trace_events
+from tests.gpu_problem import REL_L2_MAX, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+PF = synth.LayerShape("pf-mid", L=3, E=40, k=5, d=960, F=320, shared=True, tokens=0, cache_slots=96)
+
+
+class PrefillProblem:
+    def __init__(self, shape, T, P=None, C=None, distinct=None):
+        self.shape, self.T = shape, T
+        self.P = shape.L * shape.E if P is None else P
+        self.C = shape.cache_slots if C is None else C
+        self.rb = synth.record_bytes(shape.d, shape.F)
+        self.Wr = sp.router_weights(shape)
+        self.shared = sp.shared_records(shape)
+        self.pool = sp.pinned_pool(shape, self.P, distinct)
+        self.x = np.stack([conditioned_prefill(self.Wr[l], shape.k, l, T)[0] for l in range(shape.L)])
+
+    def stack(self, prefetch, max_rows=None):
+        sh = self.shape
+        dims = abi.make_dims(sh.L, sh.E, sh.k, sh.d, sh.F, sh.shared, True, max_rows or self.T,
+                             0 if self.P == sh.L * sh.E else self.P)
+        return LayerStack(dims, self.pool, sp.to_device(self.Wr), sp.to_device(self.shared), self.C,
+                          prefetch=prefetch)
+
+    def run(self, st):
+        sh = self.shape
+        xd = torch.from_numpy(self.x).cuda()
+        y = torch.zeros((sh.L, self.T, sh.d), dtype=torch.float32, device="cuda")
+        torch.cuda.synchronize()
+        tr, arr = new_trace(2 * sh.E + 8)
+        events, idx = [], np.empty((sh.L, self.T, sh.k), np.int32)
+        gates = np.empty((sh.L, self.T, sh.k), np.float32)
+        for l in range(sh.L):
+            st.forward(l, xd[l], y[l], tr)
+            events += [(e[5], e[0], e[1], e[2], e[3], e[4]) for e in trace_events(tr, arr)]
+            abi.moe_get_routing(st.ctx, idx[l], gates[l], self.T)
+        st.synchronize()
+        return events, idx, gates, y.cpu().numpy()
+
+    def oracle_y(self, l, rows):
+        sh = self.shape
+        shared = None if self.shared is None else self.shared[l * self.rb:(l + 1) * self.rb]
+        return oracle.moe_layer(self.pool.numpy(), self.P, l, sh.E, sh.d, sh.F, sh.k, self.Wr[l],
+                                shared, self.x[l][rows], w4a4=True)[2]
+
+
+def _check(pb, st, events, idx, gates, y, prefetch, rows=None):
+    sh = pb.shape
+    want_idx = np.stack([oracle.route(pb.Wr[l], pb.x[l], sh.k)[0] for l in range(sh.L)])
+    want_g = np.stack([oracle.route(pb.Wr[l], pb.x[l], sh.k)[1] for l in range(sh.L)])
+    np.testing.assert_array_equal(idx, want_idx)
+    np.testing.assert_allclose(gates, want_g, rtol=2e-5, atol=1e-7)
+    want_ev, lru = prefill_trace(want_idx, sh.L, sh.E, pb.C, prefetch=prefetch)
+    assert len(events) == len(want_ev)
+    for g, w in zip(events, want_ev):
+        assert g == w, (g, w)
+    m = np.empty(sh.L * sh.E, np.int32)
+    o = np.empty(pb.C, np.int32)
+    s = np.empty(pb.C, np.uint64)
+    clock = abi.moe_cache_export(st.ctx, m, o, s)
+    wm, wo, ws, wc = lru.state()
+    np.testing.assert_array_equal(m, wm)
+    np.testing.assert_array_equal(o, wo)
+    np.testing.assert_array_equal(s, ws)
+    assert clock == wc
+    rows = np.arange(pb.T) if rows is None else rows
+    for l in range(sh.L):
+        err = rel_l2(y[l][rows], pb.oracle_y(l, rows))
+        assert err <= REL_L2_MAX, (l, err)
+    return lru
+
+
+@pytest.mark.parametrize("prefetch", [True, False])
+def test_prefill_mid_shape(prefetch):
+    pb = PrefillProblem(PF, T=200)
+    st = pb.stack(prefetch)
+    events, idx, gates, y = pb.run(st)
+    _check(pb, st, events, idx, gates, y, prefetch)
+    stats = abi.moe_get_stats(st.ctx)
+    if prefetch:  # every later layer finds all of its experts prefetched
+        assert stats.prefetch_lookups == (PF.L - 1) * PF.E
+        later = [e for e in events if e[0] == 0 and e[1] > 0]
+        assert later and all(e[4] == 1 for e in later)
+
+
+def test_prefill_then_concurrent_decode_continues_the_cache():
+    """A prefill chunk, then decode steps of 16 rows (one per stream) on the same cache."""
+    sh, T, S, steps = PF, 120, 16, 3
+    pb = PrefillProblem(sh, T=T)
+    st = pb.stack(True, max_rows=T)
+    events, idx, gates, y = pb.run(st)
+    lru = _check(pb, st, events, idx, gates, y, True, rows=np.arange(0, T, 7))
+    xdec = np.empty((steps, sh.L, S, sh.d), np.uint16)
+    for s in range(S):
+        for l in range(sh.L):
+            xdec[:, l, s] = conditioned_decode(pb.Wr[l], sh.k, 50 + s, l, steps)[0]
+    xd = torch.from_numpy(xdec).cuda()
+    yd = torch.zeros((steps, sh.L, S, sh.d), device="cuda")
+    torch.cuda.synchronize()
+    tr, arr = new_trace(2 * sh.E + 8)
+    got = []
+    for t in range(steps):
+        for l in range(sh.L):
+            st.forward(l, xd[t, l], yd[t, l], tr)
+            got += [(t, l, e[1], e[2], e[3], e[4]) for e in trace_events(tr, arr)]
+    st.synchronize()
+    didx = np.stack([[oracle.route(pb.Wr[l], xdec[t, l], sh.k)[0] for l in range(sh.L)]
+                     for t in range(steps)])
+    want, _ = decode_trace(didx, sh.L, sh.E, pb.C, lru=lru)
+    assert got == want
+    ydn = yd.cpu().numpy()
+    shared = [pb.shared[l * pb.rb:(l + 1) * pb.rb] for l in range(sh.L)]
+    for t in range(steps):
+        for l in range(sh.L):
+            want_y = oracle.moe_layer(pb.pool.numpy(), pb.P, l, sh.E, sh.d, sh.F, sh.k, pb.Wr[l],
+                                      shared[l], xdec[t, l])[2]
+            assert rel_l2(ydn[t, l], want_y) <= REL_L2_MAX
+
+
+def test_prefill_full_chunk_qwen_shaped_two_layers():
+    """The 4096-row chunk on Qwen3.8-Flash-Next-shaped layers (512 experts, top-10 + shared,
+    d 2048, F 768, 6144 slots), two layers with prefetch; outputs on sampled rows."""
+    full = synth.QWEN38
+    sh = synth.LayerShape(full.name, L=2, E=full.E, k=full.k, d=full.d, F=full.F, shared=True,
+                          tokens=0, cache_slots=full.cache_slots)
+    pb = PrefillProblem(sh, T=4096, P=97)
+    st = pb.stack(True)
+    events, idx, gates, y = pb.run(st)
+    rows = np.random.default_rng(3).choice(4096, 24, replace=False)
+    _check(pb, st, events, idx, gates, y, True, rows=np.sort(rows))
