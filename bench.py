@@ -35,15 +35,24 @@ from synth import problem as sp  # noqa: E402
 
 METRIC = "MoE decode tok/s at batch 1; % of HBM+H2D roofline; expert miss rate"
 DISTINCT_RECORDS = 32  # generated records; the rest of the pool repeats them (same bytes moved)
+PREFILL_ROWS = 4096     # rows of one prefill chunk
+STREAMS = 16            # concurrent decode streams
+# mode -> (steps, warm-up steps, workload)
+MODE_DEFAULTS = {"decode": (512, 8, "gpt-oss-120b-shaped"),
+                 "prefill": (3, 3, "qwen3.8-flash-next-shaped"),
+                 "concurrent": (128, 4, "qwen3.8-flash-next-shaped")}
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=512)
-    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--mode", default="decode", choices=["decode", "prefill", "concurrent"],
+                    help="decode: batch-1 tokens (default); prefill: 4096-row chunks, cold cache, "
+                         "next-layer prefetch; concurrent: 16 decode streams after one prefill chunk")
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="gpt-oss-120b-shaped", choices=list(synth.SHAPES))
+    ap.add_argument("--config", default=None, choices=list(synth.SHAPES))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-timing", action="store_true")
@@ -52,7 +61,12 @@ def parse():
     ap.add_argument("--pool-records", type=int, default=0, help="override the host pool records")
     ap.add_argument("--warm", action="store_true",
                     help="warm up on the timed inputs and keep the cache (all-hit runs)")
-    return ap.parse_args()
+    a = ap.parse_args()
+    d_steps, d_warm, d_cfg = MODE_DEFAULTS[a.mode]
+    a.steps = d_steps if a.steps is None else a.steps
+    a.warmup = d_warm if a.warmup is None else a.warmup
+    a.config = d_cfg if a.config is None else a.config
+    return a
 
 
 def dist_setup(n):
@@ -143,6 +157,15 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16/fp16 tensor TFLOP/s (burst: the prefill GEMMs run between long copy waits)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured bf16_tflops (burst)"
+    return 1590.0, "fallback bf16 (burst)"
+
+
 def make_inputs(shape, T, stream0):
     return sp.decode_inputs(shape, T, 1, stream0=stream0)
 
@@ -199,7 +222,9 @@ def cpu_baseline(shape, pool_np, P, Wr, shared, x, budget_s=12.0):
 
 
 def reference_arm(args, shape):
-    """The oracle timed on the host cores; each step = one layer of one token."""
+    """The oracle timed on the host cores; each step = one layer of one batch of
+    the mode's rows (decode: 1 row, concurrent: STREAMS rows, prefill: a sample
+    of 64 rows of the chunk, W4A4)."""
     rank = int(os.environ.get("RANK", 0))
     if rank != 0:
         return
@@ -210,12 +235,19 @@ def reference_arm(args, shape):
                            for i in range(P)])
     Wr = sp.router_weights(shape)
     shared = sp.shared_records(shape)
-    x = make_inputs(shape, max(1, (args.steps + args.warmup) // shape.L + 1), 0)
+    R = {"decode": 1, "concurrent": STREAMS, "prefill": 64}[args.mode]
+    n_tok = max(1, (args.steps + args.warmup) // shape.L + 1)
+    if args.mode == "prefill":
+        x = np.stack([np.stack([synth.prefill_rows_fast(l, R, shape.d, seed=synth.MASTER_SEED + t)
+                                for l in range(shape.L)]) for t in range(n_tok)])
+    else:
+        x = sp.decode_inputs(shape, n_tok, R)
 
     def step(i):
         l, t = i % shape.L, i // shape.L
         sh = None if shared is None else shared[l * rb:(l + 1) * rb]
-        oracle.moe_layer(pool, P, l, shape.E, shape.d, shape.F, shape.k, Wr[l], sh, x[t, l])
+        oracle.moe_layer(pool, P, l, shape.E, shape.d, shape.F, shape.k, Wr[l], sh,
+                         np.ascontiguousarray(x[t, l]), w4a4=args.mode == "prefill")
 
     for i in range(args.warmup):
         step(i)
@@ -224,20 +256,55 @@ def reference_arm(args, shape):
         step(args.warmup + i)
     el = time.perf_counter() - t0
     per_layer = el / args.steps
-    tok_s = 1.0 / (per_layer * shape.L)
+    tok_s = R / (per_layer * shape.L)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count()))
-    line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tok/s",
+    metric = {"decode": METRIC,
+              "prefill": "MoE prefill tok/s (4096-row chunk, cold cache, next-layer prefetch); "
+                         "% of HBM+H2D roofline",
+              "concurrent": f"MoE concurrent decode tok/s ({STREAMS} streams, aggregate); "
+                            "% of HBM+H2D roofline; expert miss rate"}[args.mode]
+    line = {"impl": "reference", "metric": metric, "value": tok_s, "unit": "tok/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_layer * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "warm_cache": bool(args.warm),
-            "config": {"workload": shape.name, "step": "one layer of one token (oracle)"},
+            "config": {"workload": f"{shape.name} {args.mode}",
+                       "step": f"one layer of {R} row(s) (oracle)"},
             "cpu_baseline": {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{args.steps} layer evaluations (1 token-layer each); "
-                                       f"tok/s = 1 / (mean layer time x {shape.L} layers)"},
+                             "sample": f"{args.steps} layer evaluations of {R} row(s) each; "
+                                       f"tok/s = {R} / (mean layer time x {shape.L} layers)"},
             "e2e": {"value": tok_s, "unit": "tok/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def open_stack(args, shape, world, max_rows, prefetch=False):
+    """The pinned pool, the layer stack and this box's measured H2D bandwidth."""
+    from expert_offload_caching_b200 import abi
+    from expert_offload_caching_b200.runtime import LayerStack
+    L, E = shape.L, shape.E
+    rb = synth.record_bytes(shape.d, shape.F)
+    # one replica per rank; with several ranks on one host the pools alias so
+    # that the host RAM holds about one full pool in total
+    P = L * E if world == 1 else max(DISTINCT_RECORDS, (L * E) // world)
+    if args.pool_records:
+        P = min(args.pool_records, L * E)
+    pool = sp.RegisteredPool(shape, P, distinct=DISTINCT_RECORDS)
+    Wr = sp.router_weights(shape)
+    shared = sp.shared_records(shape)
+    dims = abi.make_dims(L, E, shape.k, shape.d, shape.F, shape.shared, True, max_rows,
+                         0 if P == L * E else P)
+    stack = LayerStack(dims, pool.tensor, sp.to_device(Wr), sp.to_device(shared),
+                       shape.cache_slots, prefetch=prefetch)
+
+    # H2D bandwidth of this box, measured now (the roofline's PCIe term)
+    nb = 1 << 30
+    hbuf = torch.empty(nb, dtype=torch.uint8, pin_memory=True)
+    dbuf = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    h2d = abi.moe_measure_h2d(dbuf, hbuf, nb, 0, 10, stack.copy)
+    h2d_rec = abi.moe_measure_h2d(dbuf, hbuf, (nb // rb) * rb, rb, 5, stack.copy)
+    del dbuf, hbuf
+    return stack, pool, P, rb, Wr, shared, h2d, h2d_rec
 
 
 def main():
@@ -251,30 +318,16 @@ def main():
         reference_arm(args, shape)
         return
     rank, world, local = dist_setup(args.gpus)
+    {"decode": bench_decode, "prefill": bench_prefill,
+     "concurrent": bench_concurrent}[args.mode](args, shape, rank, world, local)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def bench_decode(args, shape, rank, world, local):
     from expert_offload_caching_b200 import abi
-    from expert_offload_caching_b200.runtime import LayerStack
-
     L, E, k, d, F = shape.L, shape.E, shape.k, shape.d, shape.F
-    rb = synth.record_bytes(d, F)
-    # one replica per rank; with several ranks on one host the pools alias so
-    # that the host RAM holds about one full pool in total
-    P = shape.L * shape.E if world == 1 else max(DISTINCT_RECORDS, (shape.L * shape.E) // world)
-    if args.pool_records:
-        P = min(args.pool_records, shape.L * shape.E)
-    pool = sp.RegisteredPool(shape, P, distinct=DISTINCT_RECORDS)
-    Wr = sp.router_weights(shape)
-    shared = sp.shared_records(shape)
-    dims = abi.make_dims(L, E, k, d, F, shape.shared, True, 1, 0 if P == L * E else P)
-    stack = LayerStack(dims, pool.tensor, sp.to_device(Wr), sp.to_device(shared),
-                       shape.cache_slots)
-
-    # H2D bandwidth of this machine, measured now (the roofline's PCIe term)
-    nb = 1 << 30
-    hbuf = torch.empty(nb, dtype=torch.uint8, pin_memory=True)
-    dbuf = torch.empty(nb, dtype=torch.uint8, device="cuda")
-    h2d = abi.moe_measure_h2d(dbuf, hbuf, nb, 0, 10, stack.copy)
-    h2d_rec = abi.moe_measure_h2d(dbuf, hbuf, (nb // rb) * rb, rb, 5, stack.copy)
-    del dbuf, hbuf
+    stack, pool, P, rb, Wr, shared, h2d, h2d_rec = open_stack(args, shape, world, 1)
 
     x_warm = torch.from_numpy(make_inputs(shape, max(args.warmup, 1), 1000 + rank)).cuda()
     x = torch.from_numpy(make_inputs(shape, args.steps, rank)).cuda()
@@ -395,8 +448,302 @@ def main():
         print(json.dumps(line), flush=True)
     stack.close()
     pool.close()
-    if world > 1:
-        torch.distributed.destroy_process_group()
+
+
+
+def kernel_table(kst):
+    from expert_offload_caching_b200 import abi
+    return {abi.KERNEL_NAMES[i]: {"launches": int(kst.kernel_launches[i]),
+                                  "ms": round(kst.kernel_ms[i], 3),
+                                  "GBps": (kst.kernel_bytes[i] / (kst.kernel_ms[i] * 1e-3) / 1e9
+                                           if kst.kernel_ms[i] > 0 else None)}
+            for i in range(abi.MOE_K_COUNT) if kst.kernel_launches[i]}
+
+
+def stats_combine(a, b, sign):
+    """Field-wise a + sign * b of two moe_stats."""
+    from expert_offload_caching_b200 import abi
+    out = abi.moe_stats()
+    for f in (f[0] for f in abi.moe_stats._fields_):
+        va, vb = getattr(a, f), getattr(b, f)
+        if isinstance(va, (int, float)):
+            setattr(out, f, va + sign * vb)
+        else:
+            arr = getattr(out, f)
+            for i in range(len(arr)):
+                arr[i] = va[i] + sign * vb[i]
+    return out
+
+
+def stats_delta(after, before):
+    """Counters of after minus those of before (same context, no reset in between)."""
+    return stats_combine(after, before, -1)
+
+
+def prefill_rows_device(shape, T, seed):
+    """[L, T, d] bf16 bit patterns of the prefill chunk (i.i.d. N(0, 1) rows per layer)."""
+    x = torch.empty((shape.L, T, shape.d), dtype=torch.int16, device="cuda")
+    for l in range(shape.L):
+        x[l].copy_(torch.from_numpy(synth.prefill_rows_fast(l, T, shape.d, seed=seed).view(np.int16)))
+    return x
+
+
+def run_chunk(stack, x, y, L, host=False):
+    for l in range(L):
+        if host:
+            stack.forward_host(l, x[l], y)
+        else:
+            stack.forward(l, x[l], y)
+
+
+def bench_prefill(args, shape, rank, world, local):
+    """Steps of one prefill chunk (PREFILL_ROWS rows) through all L layers, each
+    from a cold cache with next-layer prefetch.  value = rows / s."""
+    from expert_offload_caching_b200 import abi
+    L, E, k, d, F, T = shape.L, shape.E, shape.k, shape.d, shape.F, PREFILL_ROWS
+    stack, pool, P, rb, Wr, shared, h2d, h2d_rec = open_stack(args, shape, world, T, prefetch=True)
+    xw = prefill_rows_device(shape, T, synth.MASTER_SEED + 1000 + rank)
+    x = prefill_rows_device(shape, T, synth.MASTER_SEED + rank)
+    y = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        stack.reset()
+        run_chunk(stack, xw, y, L)
+    stack.synchronize()
+
+    def one_pass(timing, host=False, xs=x, ys=y):
+        """args.steps cold-cache chunks; device seconds summed over the chunks, counters summed."""
+        total, acc = 0.0, None
+        for _ in range(args.steps):
+            stack.reset()  # synchronises the previous chunk, empties the cache, zeroes counters
+            abi.moe_set_timing(stack.ctx, timing)
+            barrier(world)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stack.compute)
+            run_chunk(stack, xs, ys, L, host)
+            e1.record(stack.compute)
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1) * 1e-3
+            st = abi.moe_get_stats(stack.ctx)
+            abi.moe_set_timing(stack.ctx, False)
+            acc = st if acc is None else stats_combine(acc, st, 1)
+        barrier(world)
+        return total, acc
+
+    clocks = ClockSampler(local if world > 1 else 0)
+    clocks.start()
+    el, st = one_pass(False)
+    clk = clocks.stop()
+    kst = None if args.no_kernel_timing else one_pass(True)[1]
+    el_max = max_over_ranks(el, world)
+    rows_total = sum_over_ranks(float(args.steps * T), world)
+    value = rows_total / el_max
+
+    hbm_peak, peak_kind = measured_peaks()
+    # HBM: every distinct routed expert of a layer (and the shared one) is read at least once
+    hit_bytes = (st.lookups + (st.forward_calls if shape.shared else 0)) * rb
+    miss_bytes = st.h2d_bytes  # routed misses + next-layer prefetch misses
+    t_roof = max(hit_bytes / (hbm_peak * 1e9), miss_bytes / (h2d * 1e9))
+    # expert FLOPs: every row x (k routed + shared) experts x (gate, up, down)
+    sel = T * (k + (1 if shape.shared else 0))
+    flops_gu = 2.0 * sel * 2 * F * d * args.steps * L
+    flops_dn = 2.0 * sel * d * F * args.steps * L
+    roof, kernels = None, {}
+    if kst is not None:
+        kernels = kernel_table(kst)
+        tpeak, tkind = measured_tensor_peak()
+        i_gu, i_dn = abi.KERNEL_NAMES.index("prefill_gate_up"), abi.KERNEL_NAMES.index("prefill_down")
+        dom, fl = (i_gu, flops_gu) if kst.kernel_ms[i_gu] >= kst.kernel_ms[i_dn] else (i_dn, flops_dn)
+        if kst.kernel_launches[dom] and kst.kernel_ms[dom] > 0:
+            achieved = fl / (kst.kernel_ms[dom] * 1e-3) / 1e12
+            roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "tensor", "achieved": achieved,
+                    "peak": tpeak, "unit": "TFLOP/s", "frac": achieved / tpeak,
+                    "peak_kind": tkind, "traffic": None,
+                    "launches": int(kst.kernel_launches[dom]),
+                    "avg_launch_us": kst.kernel_ms[dom] * 1e3 / kst.kernel_launches[dom],
+                    "flops_per_launch": fl / kst.kernel_launches[dom],
+                    "note": "legacy mma.sync f16 (hi/lo activation pairs), fp32 accumulation"}
+        for name, f in (("prefill_gate_up", flops_gu), ("prefill_down", flops_dn)):
+            i = abi.KERNEL_NAMES.index(name)
+            if kst.kernel_ms[i] > 0 and name in kernels:
+                kernels[name]["TFLOPs"] = f / (kst.kernel_ms[i] * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        yh = torch.empty((T, d), dtype=torch.float32).pin_memory()
+        el2, _ = one_pass(False, host=True, xs=xh, ys=yh)
+        e2e = {"value": rows_total / max_over_ranks(el2, world), "unit": "tok/s",
+               "h2d_bytes_per_step": L * T * d * 2, "d2h_bytes_per_step": L * T * d * 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_rows(shape, pool.array, P, Wr, shared, x, rows=64, w4a4=True)
+    if rank == 0:
+        # route, scatter, quant x, gate/up, quant h, down, combine per layer
+        launches = int(st.forward_calls * 7)
+        line = {
+            "metric": "MoE prefill tok/s (4096-row chunk, cold cache, next-layer prefetch); "
+                      "% of HBM+H2D roofline",
+            "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el_max / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4 x nvfp4 -> f32 (w4a4)", "data": "synthetic",
+            "config": {"workload": f"{shape.name} prefill: {T}-row chunk of i.i.d. N(0,1) bf16 rows "
+                                   f"through {L} layers x {E} experts, top-{k}"
+                                   f"{' + shared' if shape.shared else ''}, d={d}, F={F}, NVFP4 "
+                                   f"records of {rb} B, cold cache of {shape.cache_slots} slots per "
+                                   f"chunk, next-layer prefetch on",
+                       "l2": "inputs larger than L2 (each chunk moves "
+                             f"{miss_bytes / max(args.steps, 1) / 1e9:.1f} GB over PCIe)",
+                       "cold_cache": True, "parallelism": f"replicas x{world}",
+                       "pool_distinct_records": DISTINCT_RECORDS},
+            "miss_rate": st.misses / max(st.lookups, 1),
+            "prefetch_miss_rate": st.prefetch_misses / max(st.prefetch_lookups, 1),
+            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec,
+            "layer_roofline": {"t_roof_s": t_roof, "t_measured_s": el, "frac": t_roof / el,
+                               "hbm_term_s": hit_bytes / (hbm_peak * 1e9),
+                               "h2d_term_s": miss_bytes / (h2d * 1e9),
+                               "bw_hbm_gbs": hbm_peak, "bw_h2d_gbs": h2d,
+                               "hit_bytes": hit_bytes, "miss_bytes": miss_bytes,
+                               "h2d_achieved_gbs": miss_bytes / el / 1e9},
+            "expert_tflop": (flops_gu + flops_dn) / 1e12,
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    stack.close()
+    pool.close()
+
+
+def bench_concurrent(args, shape, rank, world, local):
+    """STREAMS decode streams at batch STREAMS after one (untimed) prefill chunk
+    on the same cache: each step is one token of every stream through all L layers."""
+    from expert_offload_caching_b200 import abi
+    L, E, k, d, F, S = shape.L, shape.E, shape.k, shape.d, shape.F, STREAMS
+    stack, pool, P, rb, Wr, shared, h2d, h2d_rec = open_stack(args, shape, world, PREFILL_ROWS,
+                                                              prefetch=True)
+    xp = prefill_rows_device(shape, PREFILL_ROWS, synth.MASTER_SEED + rank)
+    yp = torch.empty((PREFILL_ROWS, d), dtype=torch.float32, device="cuda")
+    x_warm = torch.from_numpy(sp.decode_inputs(shape, max(args.warmup, 1), S,
+                                               stream0=1000 + S * rank)).cuda()
+    x = torch.from_numpy(sp.decode_inputs(shape, args.steps, S, stream0=S * rank)).cuda()
+    y = torch.empty((args.steps, L, S, d), dtype=torch.float32, device="cuda")
+    yw = torch.empty((x_warm.shape[0], L, S, d), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    run_tokens(stack, x_warm[:args.warmup], yw, L)
+
+    def prefilled():
+        stack.reset()
+        run_chunk(stack, xp, yp, L)
+        stack.synchronize()
+        return abi.moe_get_stats(stack.ctx)
+
+    base = prefilled()
+    clocks = ClockSampler(local if world > 1 else 0)
+    clocks.start()
+    el = timed(stack, x, y, L, world)
+    clk = clocks.stop()
+    st = stats_delta(abi.moe_get_stats(stack.ctx), base)
+    kst = None
+    if not args.no_kernel_timing:
+        b2 = prefilled()
+        abi.moe_set_timing(stack.ctx, True)
+        timed(stack, x, y, L, world)
+        abi.moe_set_timing(stack.ctx, False)
+        kst = stats_delta(abi.moe_get_stats(stack.ctx), b2)
+    el_max = max_over_ranks(el, world)
+    tokens_total = sum_over_ranks(float(args.steps * S), world)
+    value = tokens_total / el_max
+
+    hbm_peak, peak_kind = measured_peaks()
+    hit_bytes = (st.hits + (st.forward_calls if shape.shared else 0)) * rb
+    miss_bytes = st.misses * rb
+    t_roof = max(hit_bytes / (hbm_peak * 1e9), miss_bytes / (h2d * 1e9))
+    roof, kernels = None, {}
+    if kst is not None:
+        kernels = kernel_table(kst)
+        ms = list(kst.kernel_ms)
+        dom = int(np.argmax(ms))
+        if kst.kernel_launches[dom] > 0 and ms[dom] > 0:
+            achieved = kst.kernel_bytes[dom] / (ms[dom] * 1e-3) / 1e9
+            roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "hbm", "achieved": achieved,
+                    "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                    "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
+                    "launches": int(kst.kernel_launches[dom]),
+                    "avg_launch_us": ms[dom] * 1e3 / kst.kernel_launches[dom],
+                    "bytes_per_launch": kst.kernel_bytes[dom] / kst.kernel_launches[dom]}
+
+    e2e = None
+    if not args.no_e2e:
+        prefilled()
+        xh = x.cpu().pin_memory()
+        yh = torch.empty((args.steps, L, S, d), dtype=torch.float32).pin_memory()
+        el2 = timed(stack, xh, yh, L, world, host=True)
+        e2e = {"value": tokens_total / max_over_ranks(el2, world), "unit": "tok/s",
+               "h2d_bytes_per_step": L * S * d * 2, "d2h_bytes_per_step": L * S * d * 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_rows(shape, pool.array, P, Wr, shared, x[0], rows=S, w4a4=False)
+    if rank == 0:
+        line = {
+            "metric": f"MoE concurrent decode tok/s ({S} streams, aggregate); "
+                      "% of HBM+H2D roofline; expert miss rate",
+            "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el_max / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4 x bf16 -> f32 (w4a16)", "data": "synthetic",
+            "per_stream_tok_s": value / (S * world),
+            "config": {"workload": f"{shape.name} concurrent decode: {S} AR(1) streams x "
+                                   f"{args.steps} tokens at batch {S}, after one {PREFILL_ROWS}-row "
+                                   f"prefill chunk on the same cache; {L} layers x {E} experts, "
+                                   f"top-{k}{' + shared' if shape.shared else ''}, d={d}, F={F}, "
+                                   f"cache {shape.cache_slots} slots",
+                       "l2": "inputs larger than L2 (each step reads the union of the streams' "
+                             "experts over all layers)",
+                       "cold_cache": False, "parallelism": f"replicas x{world}",
+                       "pool_distinct_records": DISTINCT_RECORDS},
+            "miss_rate": st.misses / max(st.lookups, 1),
+            "experts_per_layer_step": st.lookups / max(st.forward_calls, 1),
+            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec,
+            "layer_roofline": {"t_roof_s": t_roof, "t_measured_s": el, "frac": t_roof / el,
+                               "hbm_term_s": hit_bytes / (hbm_peak * 1e9),
+                               "h2d_term_s": miss_bytes / (h2d * 1e9),
+                               "bw_hbm_gbs": hbm_peak, "bw_h2d_gbs": h2d,
+                               "hit_bytes": hit_bytes, "miss_bytes": miss_bytes},
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(st.forward_calls * 3 + 2 * st.misses), "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    stack.close()
+    pool.close()
+
+
+def cpu_baseline_rows(shape, pool_np, P, Wr, shared, x, rows, w4a4, budget_s=12.0):
+    """The oracle on this host's cores over batches of `rows` rows, layer after
+    layer, until about budget_s seconds have passed; tok/s = rows per whole pass
+    of all layers.  x: device or host [L, >=rows, d] bf16 bits."""
+    import oracle
+    L, E = shape.L, shape.E
+    rb = synth.record_bytes(shape.d, shape.F)
+    xs = x[:, :rows].cpu().numpy().view(np.uint16) if hasattr(x, "cpu") else x[:, :rows]
+    t0 = time.perf_counter()
+    layers = 0
+    while True:
+        l = layers % L
+        sh = None if shared is None else shared[l * rb:(l + 1) * rb]
+        oracle.moe_layer(pool_np, P, l, E, shape.d, shape.F, shape.k, Wr[l], sh,
+                         np.ascontiguousarray(xs[l]), w4a4=w4a4)
+        layers += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count()))
+    return {"value": rows * layers / L / el, "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"{layers} layer evaluation(s) of {rows} rows (first rows of the timed "
+                      f"input), {el:.1f} s of CPU work; tok/s = rows x layers / {L} / s"}
 
 
 if __name__ == "__main__":

@@ -58,6 +58,7 @@ def lib():
         L.synth_expert_record.argtypes = [u64, i32, i32, i32, i32, i32, dbl, vp]
         L.synth_expert_matrix_f32.argtypes = [u64, i32, i32, i32, i32, i32, i32, dbl, vp]
         L.synth_replicate_records.argtypes = [vp, i64, i64, i64]
+        L.synth_prefill_rows_bf16.argtypes = [u64, i32, i32, i32, vp]
         _lib = L
     return _lib
 
@@ -205,6 +206,13 @@ def prefill_rows_bf16(layer: int, T: int, d: int, *, seed: int = MASTER_SEED,
                 raise RuntimeError("input conditioning did not converge")
         out[t] = xb
     return out, redraws
+
+
+def prefill_rows_fast(layer: int, T: int, d: int, *, seed: int = MASTER_SEED) -> np.ndarray:
+    """The rows of prefill_rows_bf16 with no conditioning (attempt 0 everywhere), in C."""
+    out = np.empty((T, d), dtype=np.uint16)
+    lib().synth_prefill_rows_bf16(seed, layer, T, d, _p(out))
+    return out
 
 
 # The workloads (shapes of the models on the FreeToken pages; cache sizes as fractions of

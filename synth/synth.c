@@ -236,3 +236,14 @@ EXPORT void synth_replicate_records(uint8_t *buf, int64_t record_bytes, int64_t 
     for (int64_t i = n_src; i < n_dst; ++i)
         memcpy(buf + i * record_bytes, buf + (i % n_src) * record_bytes, (size_t)record_bytes);
 }
+
+/* T prefill rows of one layer (i.i.d. N(0,1), attempt 0), bf16 [T x d]. */
+EXPORT void synth_prefill_rows_bf16(uint64_t seed, int32_t layer, int32_t T, int32_t d,
+                                    uint16_t *out) {
+#pragma omp parallel for schedule(static)
+    for (int32_t t = 0; t < T; ++t) {
+        uint64_t key = synth_key(seed, 4, 0, (uint64_t)layer, (uint64_t)t, 0);
+        for (int32_t i = 0; i < d; ++i)
+            out[(int64_t)t * d + i] = f32_to_bf16_rne((float)normal01(key, (uint64_t)i));
+    }
+}
