@@ -9,9 +9,10 @@
 //   sb = E4M3(r), saturating; denom = value(sb) * s_t; code = E2M1(v / denom),
 //   saturating; all codes 0 when value(sb) = 0.
 // The conversions are the hardware RNE ones (cvt.rn.satfinite.{e4m3x2,e2m1x2}.f32).
-// The expert GEMV consumes each quantized row as its exact dequantized value
-// e2m1 * e4m3 * s_t, split into an fp16 (hi, lo) pair, so the products with
-// the NVFP4 weights are those of the W4A4 definition up to fp32 rounding.
+// The rows are written in expert-grouped order (a token's x once per expert
+// that it selected, then once more for the shared expert) as NVFP4 codes,
+// block scales and row scales: the operands of the block-scaled tensor-core
+// GEMMs, which apply s_t in their epilogue.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -29,33 +30,17 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(s));
     return __low2float(*reinterpret_cast<__half2 *>(&r));
 }
-// E2M1 RNE codes of (v0, v1) and their values.
-__device__ __forceinline__ float2 e2m1_round_pair(float v0, float v1) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 c;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 c, %2, %1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
-        : "=r"(r)
-        : "f"(v0), "f"(v1));
-    return __half22float2(*reinterpret_cast<__half2 *>(&r));
-}
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 
-__device__ __forceinline__ void store_hilo(__half *hi_row, __half *lo_row, int i, float v) {
-    const __half hi = __float2half_rn(v);
-    hi_row[i] = hi;
-    lo_row[i] = __float2half_rn(v - __half2float(hi));
-}
-
 // One warp quantizes one row of n values (n a multiple of 16) and writes the
-// dequantized row as an fp16 (hi, lo) pair.
+// NVFP4 encoding itself: codes (two per byte, even element in the low nibble),
+// one E4M3 scale per 16 values and the row's fp32 scale s_t.
 template <typename LoadFn>
-__device__ void quant_row(LoadFn load, int n, __half *hi_row, __half *lo_row) {
+__device__ void quant_row_codes(LoadFn load, int n, uint8_t *codes, uint8_t *scales, float *st) {
     const int lane = threadIdx.x & 31;
     float amax = 0.f;
     for (int i = lane; i < n; i += 32) amax = fmaxf(amax, fabsf(load(i)));
@@ -70,38 +55,50 @@ __device__ void quant_row(LoadFn load, int n, __half *hi_row, __half *lo_row) {
             v[j] = load(16 * b + j);
             bmax = fmaxf(bmax, fabsf(v[j]));
         }
-        const float sval = e4m3_value(e4m3_code(bmax / six_st));
+        const uint32_t sc = e4m3_code(bmax / six_st);
+        const float sval = e4m3_value(sc);
         const float denom = sval * s_t;
+        uint32_t word[2] = {0u, 0u};
+        if (sval != 0.f) {
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-            float2 q = make_float2(0.f, 0.f);
-            if (sval != 0.f) q = e2m1_round_pair(v[j] / denom, v[j + 1] / denom);
-            store_hilo(hi_row, lo_row, 16 * b + j, q.x * sval * s_t);
-            store_hilo(hi_row, lo_row, 16 * b + j + 1, q.y * sval * s_t);
+            for (int j = 0; j < 16; j += 2) {
+                uint16_t c;
+                asm("{\n\t.reg .b8 c8;\n\t"
+                    "cvt.rn.satfinite.e2m1x2.f32 c8, %2, %1;\n\t"
+                    "cvt.u16.u8 %0, c8;\n\t}"
+                    : "=h"(c)
+                    : "f"(v[j] / denom), "f"(v[j + 1] / denom));
+                word[j >> 3] |= (uint32_t)(c & 0xffu) << (4 * (j & 7));
+            }
         }
+        *reinterpret_cast<uint2 *>(codes + 8 * b) = make_uint2(word[0], word[1]);
+        scales[b] = (uint8_t)sc;
     }
+    if (lane == 0) *st = s_t;
 }
 
-// x rows (bf16 [T][d]) -> xh [T][2][d]; one warp per row.
-__global__ void quant_x_kernel(const __nv_bfloat16 *__restrict__ x, int T, int d, __half *xh) {
-    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (t >= T) return;
+// Grouped rows of x for the tensor-core GEMMs: row g < T*k is token
+// rowrefs[g].t, row T*k + t (shared expert) is token t; one warp per row.
+__global__ void quant_x_grouped_kernel(const __nv_bfloat16 *__restrict__ x, int T, int k, int d,
+                                       int has_shared, const RowRef *__restrict__ rowrefs,
+                                       uint8_t *codes, uint8_t *scales, float *st) {
+    const int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int tk = T * k;
+    if (g >= tk + (has_shared ? T : 0)) return;
+    const int t = g < tk ? rowrefs[g].t : g - tk;
     const __nv_bfloat16 *row = x + (size_t)t * d;
-    quant_row([&](int i) { return __bfloat162float(row[i]); }, d, xh + (size_t)t * 2 * d,
-              xh + (size_t)t * 2 * d + d);
+    quant_row_codes([&](int i) { return __bfloat162float(row[i]); }, d, codes + (size_t)g * (d / 2),
+                    scales + (size_t)g * (d / 16), st + g);
 }
 
-// h rows (fp32 [T][k+1][F]) -> hh [T][k+1][2][F] for the selections that exist
-// (p < k, and p = k when there is a shared expert); one warp per row.
-__global__ void quant_h_kernel(const float *__restrict__ h32, int T, int k, int F, int has_shared,
-                               __half *hh) {
-    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int per_t = k + (has_shared ? 1 : 0);
-    if (w >= T * per_t) return;
-    const int t = w / per_t, p = w - t * per_t;
-    const size_t sel = (size_t)t * (k + 1) + p;
-    const float *row = h32 + sel * F;
-    quant_row([&](int i) { return row[i]; }, F, hh + sel * 2 * F, hh + sel * 2 * F + F);
+// Grouped h rows (fp32 [rows][F]) -> NVFP4 codes, scales, row scales; one warp per row.
+__global__ void quant_h_grouped_kernel(const float *__restrict__ h32, int rows, int F, uint8_t *codes,
+                                       uint8_t *scales, float *st) {
+    const int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (g >= rows) return;
+    const float *row = h32 + (size_t)g * F;
+    quant_row_codes([&](int i) { return row[i]; }, F, codes + (size_t)g * (F / 2),
+                    scales + (size_t)g * (F / 16), st + g);
 }
 
 // y[t] = sum over p < k of gates[t][p] * part[t][p] (+ part[t][k], the shared expert)
@@ -119,18 +116,21 @@ __global__ void combine_kernel(const float *__restrict__ part, const float *__re
 
 }  // namespace
 
-cudaError_t launch_quant_x(const __nv_bfloat16 *x, int T, int d, __half *xh, cudaStream_t s) {
+cudaError_t launch_quant_x_grouped(const __nv_bfloat16 *x, int T, int k, int d, int has_shared,
+                                   const RowRef *rowrefs, uint8_t *codes, uint8_t *scales, float *st,
+                                   cudaStream_t s) {
+    const int rows = T * k + (has_shared ? T : 0);
     const int warps_per_cta = 8;
-    quant_x_kernel<<<(T + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(x, T, d, xh);
+    quant_x_grouped_kernel<<<(rows + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(
+        x, T, k, d, has_shared, rowrefs, codes, scales, st);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quant_h(const float *h32, int T, int k, int F, int has_shared, __half *hh,
-                           cudaStream_t s) {
-    const int rows = T * (k + (has_shared ? 1 : 0));
+cudaError_t launch_quant_h_grouped(const float *h32, int rows, int F, uint8_t *codes, uint8_t *scales,
+                                   float *st, cudaStream_t s) {
     const int warps_per_cta = 8;
-    quant_h_kernel<<<(rows + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(
-        h32, T, k, F, has_shared, hh);
+    quant_h_grouped_kernel<<<(rows + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(
+        h32, rows, F, codes, scales, st);
     return cudaGetLastError();
 }
 

@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
         } else {
             const int4 j0 = __ldcg(reinterpret_cast<const int4 *>(&a.jobs[jy]));  // expert, slot, hit, nrows
             const int row_off_j = __ldcg(&a.jobs[jy].row_off);
-            if (a.only_job < 0 && !j0.z && !a.all_jobs) {
+            if (a.only_job < 0 && !j0.z) {
                 work = false;
             } else {
                 rec = a.arena + (int64_t)j0.y * a.rec_bytes;
@@ -274,14 +274,10 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
                         const float gt = ts[0] * v0, up = ts[1] * v1;
                         const float h = gt / (1.0f + expf(-gt)) * up;
                         const int j = 8 * tile + g;
-                        if (a.h32_out) {  // prefill: h is quantized to NVFP4 before the down projection
-                            a.h32_out[sel * a.F + j] = h;
-                        } else {
-                            const __half hi = __float2half_rn(h);
-                            const __half lo = __float2half_rn(h - __half2float(hi));
-                            a.hh_out[sel * 2 * a.F + j] = hi;
-                            a.hh_out[sel * 2 * a.F + a.F + j] = lo;
-                        }
+                        const __half hi = __float2half_rn(h);
+                        const __half lo = __float2half_rn(h - __half2float(hi));
+                        a.hh_out[sel * 2 * a.F + j] = hi;
+                        a.hh_out[sel * 2 * a.F + a.F + j] = lo;
                     } else {
                         const int i = 16 * tile + g;
                         a.part_out[sel * a.d + i] = ts[2] * v0;

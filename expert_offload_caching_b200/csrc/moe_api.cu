@@ -38,7 +38,9 @@ bool dims_valid(const moe_dims *d) {
 bool dims_supported(const moe_dims *d) {
     return d->d % 64 == 0 && d->F % 64 == 0 && d->d <= 4096 && d->F <= 4096 && d->k <= kMaxK &&
            d->E <= kMaxE &&
-           d->max_rows <= 4096 && (int64_t)d->L * d->E < (1ll << 31);
+           d->max_rows <= 4096 && (int64_t)d->L * d->E < (1ll << 31) &&
+           // prefill GEMM operands: TMA boxes of 128 bytes of a row
+           (d->max_rows <= kDecodeMaxRows || (d->d >= 256 && d->F >= 256));
 }
 
 RecordLayout layout_of(const moe_dims *d) {
@@ -62,12 +64,17 @@ int max_jobs(const moe_dims *d, int T) {
 // for the largest call (max_rows); the prefill buffers exist when max_rows > 32.
 struct WsLayout {
     int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, rowrefs, xh, hh, part, cnt, fill,
-        jobidx, h32, xstage, ystage, total;
+        jobidx, h32, xq, xq_scales, xq_st, hq, hq_scales, hq_st, pairs, n_pairs, xstage, ystage, total;
 };
+int pairs_capacity(const moe_dims *d) {
+    return grouped_pairs_cap(d->E, d->max_rows, d->k, d->has_shared ? 1 : 0);
+}
 WsLayout ws_layout(const moe_dims *d) {
     WsLayout w;
     const int64_t T = d->max_rows, k = d->k, E = d->E, dd = d->d, F = d->F;
     const bool prefill = T > kDecodeMaxRows;
+    const int64_t Td = prefill ? kDecodeMaxRows : T;  // rows of the decode-only buffers
+    const int64_t R = T * (k + 1);                     // grouped prefill rows (routed + shared)
     int64_t o = 0;
     auto take = [&](int64_t bytes) { int64_t r = o; o += up256(bytes); return r; };
     w.z = take(T * E * 4);
@@ -80,13 +87,21 @@ WsLayout ws_layout(const moe_dims *d) {
     w.ticket = take(4);
     w.ticket2 = take(4);
     w.rowrefs = take(T * k * (int64_t)sizeof(RowRef));
-    w.xh = take(T * 2 * dd * 2);
-    w.hh = take(T * (k + 1) * 2 * F * 2);
+    w.xh = take(Td * 2 * dd * 2);
+    w.hh = take(Td * (k + 1) * 2 * F * 2);
     w.part = take(T * (k + 1) * dd * 4);
     w.cnt = prefill ? take(E * 4) : -1;
     w.fill = prefill ? take(E * 4) : -1;
     w.jobidx = prefill ? take(E * 4) : -1;
-    w.h32 = prefill ? take(T * (k + 1) * F * 4) : -1;
+    w.h32 = prefill ? take(R * F * 4) : -1;
+    w.xq = prefill ? take(R * dd / 2) : -1;
+    w.xq_scales = prefill ? take(R * dd / 16) : -1;
+    w.xq_st = prefill ? take(R * 4) : -1;
+    w.hq = prefill ? take(R * F / 2) : -1;
+    w.hq_scales = prefill ? take(R * F / 16) : -1;
+    w.hq_st = prefill ? take(R * 4) : -1;
+    w.pairs = prefill ? take((int64_t)pairs_capacity(d) * 8) : -1;
+    w.n_pairs = prefill ? take(4) : -1;
     w.xstage = take(T * dd * 2);
     w.ystage = take(T * dd * 4);
     w.total = o;
@@ -141,6 +156,9 @@ struct moe_ctx {
     cudaEvent_t ev_routed = nullptr;    // prefill: this layer's routed misses copied
     std::vector<cudaEvent_t> ev_pf;     // [L]: prefetch copies for a layer issued
     std::vector<char> pf_pending;       // [L]: a prefetch for the layer is not yet waited on
+    // prefill GEMM operand descriptors (activation and shared maps at init,
+    // arena maps at cache_configure)
+    GroupedGemmMaps maps;
     // state
     moe_status state = MOE_OK;
     std::string err;
@@ -448,7 +466,10 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     CK(launch_prefill_route(ra, ctx->cs));
     time_end(ctx, tr, (double)D.E * D.d * 2 + (double)T * D.d * 2);
     CK(launch_prefill_scatter(ra, ctx->cs));
-    CK(launch_quant_x(ra.x, T, D.d, ctx->dws.xh, ctx->cs));
+    CK(launch_tile_plan(ctx->dws.jobs, ctx->dws.n_jobs, T, D.has_shared, ctx->dws.pairs, ctx->dws.n_pairs,
+                        ctx->cs));
+    CK(launch_quant_x_grouped(ra.x, T, D.k, D.d, D.has_shared, ctx->dws.rowrefs, ctx->dws.xq,
+                              ctx->dws.xq_scales, ctx->dws.xq_st, ctx->cs));
 
     const moe_status ws_ = wait_miss_list(ctx, seq);
     if (ws_ != MOE_OK) return ws_;
@@ -458,17 +479,35 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
 
     // copies on the copy stream: this layer's misses (the layer's compute waits
     // for them), then the next layer's prefetch misses (its compute waits)
-    auto copy_record = [&](int lyr, const HostEvent &e) -> moe_status {
+    // Records whose pool indices and slots are both consecutive (a cold cache
+    // hands out free slots in ascending order, and entries come in ascending
+    // expert order) go in one copy.
+    int64_t run_src = -1, run_dst = -1, run_n = 0;
+    auto flush_run = [&]() -> moe_status {
+        if (run_n == 0) return MOE_OK;
         if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
             ctx->state = MOE_ERR_STATE;
             ctx->err = "injected failure of an H2D copy issue";
             return MOE_ERR_CUDA;
         }
-        const int64_t rec_idx = ((int64_t)lyr * D.E + e.expert) % ctx->P;
-        CK(cudaMemcpyAsync(ctx->arena + (int64_t)e.slot * ctx->lay.bytes, ctx->pool + rec_idx * ctx->lay.bytes,
-                           ctx->lay.bytes, cudaMemcpyHostToDevice, ctx->xs));
+        CK(cudaMemcpyAsync(ctx->arena + run_dst * ctx->lay.bytes, ctx->pool + run_src * ctx->lay.bytes,
+                           run_n * ctx->lay.bytes, cudaMemcpyHostToDevice, ctx->xs));
         ctx->stats.h2d_copies += 1;
-        ctx->stats.h2d_bytes += ctx->lay.bytes;
+        ctx->stats.h2d_bytes += run_n * ctx->lay.bytes;
+        run_n = 0;
+        return MOE_OK;
+    };
+    auto copy_record = [&](int lyr, const HostEvent &e) -> moe_status {
+        const int64_t rec_idx = ((int64_t)lyr * D.E + e.expert) % ctx->P;
+        if (run_n > 0 && rec_idx == run_src + run_n && e.slot == run_dst + run_n) {
+            ++run_n;
+            return MOE_OK;
+        }
+        const moe_status st = flush_run();
+        if (st != MOE_OK) return st;
+        run_src = rec_idx;
+        run_dst = e.slot;
+        run_n = 1;
         return MOE_OK;
     };
     int nrm = 0, npm = 0;
@@ -479,6 +518,8 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
         ++nrm;
     }
     if (nrm > 0) {
+        const moe_status st = flush_run();
+        if (st != MOE_OK) return st;
         CK(cudaEventRecord(ctx->ev_routed, ctx->xs));
         CK(cudaStreamWaitEvent(ctx->cs, ctx->ev_routed, 0));
     }
@@ -493,27 +534,53 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
         ++npm;
     }
     if (npm > 0) {
+        const moe_status st = flush_run();
+        if (st != MOE_OK) return st;
         CK(cudaEventRecord(ctx->ev_pf[layer + 1], ctx->xs));
         ctx->pf_pending[layer + 1] = 1;
     }
 
-    // experts: gate/up (+SwiGLU, fp32 h), h quantized per row, down, combine
+    // experts: grouped tensor-core GEMMs -- gate/up (+SwiGLU, fp32 h), h
+    // quantized per row, down -- then the gate-weighted combine
     const int grid_y = n + (D.has_shared ? 1 : 0);
-    GemvArgs gu = gemv_args(ctx, layer, T, kGateUp, -1);
-    gu.all_jobs = 1;
-    gu.h32_out = ctx->dws.h32;
-    gu.shared_slot = D.has_shared ? n : -1;
+    const int cap = grouped_pairs_cap(n, T, D.k, D.has_shared);
+    GroupedGemmArgs gu{};
+    gu.mode = kGateUp;
+    gu.jobs = ctx->dws.jobs;
+    gu.n_jobs = ctx->dws.n_jobs;
+    gu.pairs = ctx->dws.pairs;
+    gu.n_pairs = ctx->dws.n_pairs;
+    gu.m_tiles = (2 * D.F + 127) / 128;
+    gu.layer = layer;
+    gu.T = T;
+    gu.k = D.k;
+    gu.d = D.d;
+    gu.F = D.F;
+    gu.arena = ctx->arena;
+    gu.rec_bytes = ctx->lay.bytes;
+    gu.shared_rec = D.has_shared ? ctx->shared_recs : nullptr;
+    gu.lay = ctx->lay;
+    gu.act_scales = ctx->dws.xq_scales;
+    gu.act_st = ctx->dws.xq_st;
+    gu.rowrefs = ctx->dws.rowrefs;
+    gu.h32 = ctx->dws.h32;
+    gu.part = ctx->dws.part;
+    gu.page = ctx->page_d;
     TimedLaunch tg;
     time_begin(ctx, tg, MOE_K_PREFILL_GATEUP);
-    CK(launch_gemv(gu, grid_y, ctx->cs));
+    CK(launch_grouped_gemm(ctx->maps, gu, cap, ctx->cs));
     time_end(ctx, tg, grid_y * w13_bytes(ctx));
-    CK(launch_quant_h(ctx->dws.h32, T, D.k, D.F, D.has_shared, ctx->dws.hh, ctx->cs));
-    GemvArgs dn = gemv_args(ctx, layer, T, kDown, -1, 0);
-    dn.all_jobs = 1;
-    dn.shared_slot = D.has_shared ? n : -1;
+    const int grouped_rows = T * D.k + (D.has_shared ? T : 0);
+    CK(launch_quant_h_grouped(ctx->dws.h32, grouped_rows, D.F, ctx->dws.hq, ctx->dws.hq_scales,
+                              ctx->dws.hq_st, ctx->cs));
+    GroupedGemmArgs dn = gu;
+    dn.mode = kDown;
+    dn.m_tiles = (D.d + 127) / 128;
+    dn.act_scales = ctx->dws.hq_scales;
+    dn.act_st = ctx->dws.hq_st;
     TimedLaunch td;
     time_begin(ctx, td, MOE_K_PREFILL_DOWN);
-    CK(launch_gemv(dn, grid_y, ctx->cs));
+    CK(launch_grouped_gemm(ctx->maps, dn, cap, ctx->cs));
     time_end(ctx, td, grid_y * w2_bytes(ctx));
     CK(launch_combine(ctx->dws.part, ctx->dws.gates, y, T, D.k, D.d, D.has_shared, ctx->cs));
 
@@ -612,6 +679,29 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     ctx->dws.fill = L.fill >= 0 ? reinterpret_cast<int32_t *>(w + L.fill) : nullptr;
     ctx->dws.jobidx = L.jobidx >= 0 ? reinterpret_cast<int32_t *>(w + L.jobidx) : nullptr;
     ctx->dws.h32 = L.h32 >= 0 ? reinterpret_cast<float *>(w + L.h32) : nullptr;
+    if (L.xq >= 0) {
+        ctx->dws.xq = w + L.xq;
+        ctx->dws.xq_scales = w + L.xq_scales;
+        ctx->dws.xq_st = reinterpret_cast<float *>(w + L.xq_st);
+        ctx->dws.hq = w + L.hq;
+        ctx->dws.hq_scales = w + L.hq_scales;
+        ctx->dws.hq_st = reinterpret_cast<float *>(w + L.hq_st);
+        ctx->dws.pairs = reinterpret_cast<int2 *>(w + L.pairs);
+        ctx->dws.n_pairs = reinterpret_cast<int32_t *>(w + L.n_pairs);
+        const int64_t R = (int64_t)dims->max_rows * (dims->k + 1);
+        bool ok = make_operand_map(&ctx->maps.xq, ctx->dws.xq, dims->d / 2, R, 0, 0) &&
+                  make_operand_map(&ctx->maps.hq, ctx->dws.hq, dims->F / 2, R, 0, 0);
+        if (ok && dims->has_shared) {
+            ok = make_operand_map(&ctx->maps.w13_shared, ctx->shared_recs + lay.w13_codes, dims->d / 2,
+                                  2 * dims->F, dims->L, lay.bytes) &&
+                 make_operand_map(&ctx->maps.w2_shared, ctx->shared_recs + lay.w2_codes, dims->F / 2, dims->d,
+                                  dims->L, lay.bytes);
+        }
+        if (!ok) {
+            delete ctx;
+            return MOE_ERR_UNSUPPORTED;
+        }
+    }
 
     ctx->page_cap = 2 * dims->E + 8;
     const size_t page_bytes = sizeof(HostPage) + sizeof(HostEvent) * ctx->page_cap;
@@ -668,6 +758,17 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
     ctx->tab.stamp = reinterpret_cast<unsigned long long *>(tb + tl.stamp);
     ctx->tab.C = num_slots;
     ctx->flags = flags & ~MOE_CACHE_RESET;
+    if (ctx->wl.xq >= 0) {  // prefill GEMM descriptors of the arena's weight codes
+        if (!make_operand_map(&ctx->maps.w13, a + ctx->lay.w13_codes, D.d / 2, 2 * D.F, num_slots, ctx->lay.bytes) ||
+            !make_operand_map(&ctx->maps.w2, a + ctx->lay.w2_codes, D.F / 2, D.d, num_slots, ctx->lay.bytes)) {
+            ctx->configured = false;
+            return MOE_ERR_UNSUPPORTED;
+        }
+        if (!D.has_shared) {
+            ctx->maps.w13_shared = ctx->maps.w13;
+            ctx->maps.w2_shared = ctx->maps.w2;
+        }
+    }
     if (reset) {
         // finish outstanding work of the old state first
         CK(cudaStreamSynchronize(ctx->xs));

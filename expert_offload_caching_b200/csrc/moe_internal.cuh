@@ -1,6 +1,7 @@
 // Internal definitions shared by the kernels and the C-ABI host code.
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -79,7 +80,15 @@ struct DecodeWs {
     int32_t *cnt;        // [E] rows per expert
     int32_t *fill;       // [E] scatter cursors
     int32_t *jobidx;     // [E] job of an expert, -1 if unused
-    float *h32;          // [T][k+1][F] fp32 h before its activation quantization
+    float *h32;          // grouped rows x F: fp32 h before its activation quantization
+    uint8_t *xq;         // grouped rows x d/2: E2M1 codes of x (NVFP4, per-row scale)
+    uint8_t *xq_scales;  // grouped rows x d/16: E4M3 block scales
+    float *xq_st;        // grouped rows: fp32 row scales
+    uint8_t *hq;         // grouped rows x F/2: E2M1 codes of h
+    uint8_t *hq_scales;  // grouped rows x F/16
+    float *hq_st;        // grouped rows
+    int2 *pairs;         // (job, n tile) pairs of the grouped GEMMs
+    int32_t *n_pairs;
 };
 
 struct RouteArgs {
@@ -104,8 +113,6 @@ struct GemvArgs {
     const int32_t *n_jobs;
     const RowRef *rowrefs;
     int only_job;          // >= 0: process just this job; -1: every hit job (+ shared)
-    int all_jobs;          // with only_job = -1: hit and missed jobs alike (prefill)
-    float *h32_out;        // gate/up: write fp32 h here instead of the fp16 (hi, lo) pair
     int shared_slot;       // gridDim.y index of the shared job, -1 if none
     const uint8_t *arena;
     int64_t rec_bytes;
@@ -125,16 +132,55 @@ struct GemvArgs {
     uint32_t *ticket;
 };
 
+// Grouped W4A4 expert GEMMs of a prefill chunk (tcgen05 block-scaled MMA).
+// Activation rows are in expert-grouped order: the routed rows of job j at
+// [row_off_j, row_off_j + nrows_j) (RowRef gives (t, p)), then the shared
+// expert's rows t at T*k + t.
+struct GroupedGemmArgs {
+    int mode;                 // kGateUp: h = silu(g) * u into h32; kDown: into part
+    const Job *jobs;
+    const int32_t *n_jobs;
+    const int2 *pairs;        // (job, n tile) per tile pair; job == n_jobs: shared expert
+    const int32_t *n_pairs;
+    int m_tiles;              // 128-row tiles of the weight matrix
+    int layer, T, k, d, F;
+    const uint8_t *arena;
+    int64_t rec_bytes;
+    const uint8_t *shared_rec;  // the L shared-expert records, or null
+    RecordLayout lay;
+    const uint8_t *act_scales;  // grouped rows x K/16 E4M3
+    const float *act_st;        // grouped rows: per-row fp32 scale
+    const RowRef *rowrefs;
+    float *h32;               // gate/up output: grouped rows x F
+    float *part;              // down output: [T][k+1][d]
+    HostPage *page;
+};
+// TMA descriptors of the operands: weight codes of the slot arena (3D: byte,
+// row, slot) and of the shared records (3D: byte, row, layer); grouped
+// activation codes (2D: byte, row).
+struct GroupedGemmMaps {
+    CUtensorMap w13, w2, w13_shared, w2_shared, xq, hq;
+};
+
 // launchers (one per .cu)
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s);
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
 cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s);
-cudaError_t launch_quant_x(const __nv_bfloat16 *x, int T, int d, __half *xh, cudaStream_t s);
-cudaError_t launch_quant_h(const float *h32, int T, int k, int F, int has_shared, __half *hh,
-                           cudaStream_t s);
 cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
                            int has_shared, cudaStream_t s);
+cudaError_t launch_quant_x_grouped(const __nv_bfloat16 *x, int T, int k, int d, int has_shared,
+                                   const RowRef *rowrefs, uint8_t *codes, uint8_t *scales, float *st,
+                                   cudaStream_t s);
+cudaError_t launch_quant_h_grouped(const float *h32, int rows, int F, uint8_t *codes, uint8_t *scales,
+                                   float *st, cudaStream_t s);
+int grouped_pairs_cap(int n_jobs, int T, int k, int has_shared);
+cudaError_t launch_tile_plan(const Job *jobs, const int32_t *n_jobs, int T, int has_shared, int2 *pairs,
+                             int32_t *n_pairs, cudaStream_t s);
+cudaError_t launch_grouped_gemm(const GroupedGemmMaps &maps, const GroupedGemmArgs &a, int pairs_cap,
+                                cudaStream_t s);
+bool make_operand_map(CUtensorMap *out, const void *base, int64_t row_bytes, int64_t rows, int64_t count,
+                      int64_t matrix_stride);
 
 }  // namespace moe

@@ -160,7 +160,8 @@ MOE_API size_t moe_arena_bytes(const moe_dims *dims, int64_t num_slots);
  *   compute_stream, copy_stream: cudaStream_t handles (NULL = legacy stream not
  *              accepted: pass real streams); work is issued on them only.
  * Shapes handled: d and F multiples of 64, 1 <= k <= 32, k <= E <= 1024,
- * 1 <= max_rows <= 4096; else MOE_ERR_UNSUPPORTED. */
+ * 1 <= max_rows <= 4096, and with max_rows > 32 (prefill) d >= 256 and
+ * F >= 256; else MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t host_pool_bytes,
                           const void *router_w, const void *shared_recs, void *workspace,
                           size_t workspace_bytes, void *compute_stream, void *copy_stream,
@@ -190,8 +191,11 @@ MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_a
  * expert) and multiplied against the NVFP4 weights (W4A4); the lookup batch is
  * the layer's distinct experts, and with MOE_CACHE_PREFETCH_NEXT a second
  * batch of all experts of layer + 1 follows, whose misses are copied while
- * this layer computes (the next call for layer + 1 waits for them).  The trace
- * lists the routed entries, then the prefetch entries (prefetch = 1, layer + 1). */
+ * this layer computes (the next call for layer + 1 waits for them; records
+ * with consecutive pool indices and slots go in one copy).  The expert FFNs
+ * of a prefill call run as grouped block-scaled NVFP4 GEMMs on the tensor
+ * cores (rows grouped by expert, fp32 accumulation).  The trace lists the
+ * routed entries, then the prefetch entries (prefetch = 1, layer + 1). */
 MOE_API moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
                              moe_layer_trace *trace);
 
