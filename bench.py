@@ -34,6 +34,7 @@ import synth  # noqa: E402
 from synth import problem as sp  # noqa: E402
 
 METRIC = "MoE decode tok/s at batch 1; % of HBM+H2D roofline; expert miss rate"
+H2D_SM = {}  # SM-driven H2D rates measured by open_stack
 DISTINCT_RECORDS = 32  # generated records; the rest of the pool repeats them (same bytes moved)
 PREFILL_ROWS = 4096     # rows of one prefill chunk
 STREAMS = 16            # concurrent decode streams
@@ -59,6 +60,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="override L (small profiling cases)")
     ap.add_argument("--slots", type=int, default=0, help="override the HBM cache slots")
     ap.add_argument("--pool-records", type=int, default=0, help="override the host pool records")
+    ap.add_argument("--policy", default="lru", choices=["lru", "static"],
+                    help="cache policy: the global LRU (default) or the static per-layer split")
     ap.add_argument("--warm", action="store_true",
                     help="warm up on the timed inputs and keep the cache (all-hit runs)")
     a = ap.parse_args()
@@ -69,18 +72,34 @@ def parse():
     return a
 
 
-def dist_setup(n):
+def dist_setup(n, backend: str = "nccl"):
+    """One process per GPU (torchrun env).  Replicas only: the process group
+    carries the barriers and the max/sum over ranks, no data-path collective.
+    backend "gloo" runs the same logic on host tensors (CPU tests)."""
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                             device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                                 device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
+
+
+def _reduce_device():
+    return "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+
+
+def replica_pool_records(L: int, E: int, world: int) -> int:
+    """Host-pool records per replica: the whole pool alone, else an aliased share
+    (expert (l, e) -> record (l*E + e) mod P) so that the host RAM holds about one pool."""
+    return L * E if world == 1 else max(DISTINCT_RECORDS, (L * E) // world)
 
 
 def barrier(world):
@@ -91,7 +110,7 @@ def barrier(world):
 def max_over_ranks(v: float, world: int) -> float:
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -99,7 +118,7 @@ def max_over_ranks(v: float, world: int) -> float:
 def sum_over_ranks(v: float, world: int) -> float:
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
     return float(t.item())
 
@@ -291,7 +310,7 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
     rb = synth.record_bytes(shape.d, shape.F)
     # one replica per rank; with several ranks on one host the pools alias so
     # that the host RAM holds about one full pool in total
-    P = L * E if world == 1 else max(DISTINCT_RECORDS, (L * E) // world)
+    P = replica_pool_records(L, E, world)
     if args.pool_records:
         P = min(args.pool_records, L * E)
     pool = sp.RegisteredPool(shape, P, distinct=DISTINCT_RECORDS)
@@ -300,7 +319,8 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
     dims = abi.make_dims(L, E, shape.k, shape.d, shape.F, shape.shared, True, max_rows,
                          0 if P == L * E else P)
     stack = LayerStack(dims, pool.tensor, sp.to_device(Wr), sp.to_device(shared),
-                       shape.cache_slots, prefetch=prefetch)
+                       shape.cache_slots, prefetch=prefetch,
+                       static_split=getattr(args, "policy", "lru") == "static")
 
     # H2D bandwidth of this machine, measured now (the roofline's PCIe term)
     nb = 1 << 30
@@ -308,6 +328,14 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
     dbuf = torch.empty(nb, dtype=torch.uint8, device="cuda")
     h2d = abi.moe_measure_h2d(dbuf, hbuf, nb, 0, 10, stack.copy)
     h2d_rec = abi.moe_measure_h2d(dbuf, hbuf, (nb // rb) * rb, rb, 5, stack.copy)
+    # the same through SM loads of mapped host memory (a device-initiated fetch)
+    global H2D_SM
+    try:
+        H2D_SM = {"h2d_sm_gbs": abi.moe_measure_h2d_sm(dbuf, hbuf, nb, 0, 5, stack.copy),
+                  "h2d_sm_record_gbs": abi.moe_measure_h2d_sm(dbuf, hbuf, (nb // rb) * rb, rb, 3,
+                                                              stack.copy)}
+    except abi.MoeError as e:
+        H2D_SM = {"h2d_sm_gbs": None, "h2d_sm_note": str(e)}
     del dbuf, hbuf
     return stack, pool, P, rb, Wr, shared, h2d, h2d_rec
 
@@ -406,6 +434,7 @@ def bench_decode(args, shape, rank, world, local):
                    for i in range(abi.MOE_K_COUNT) if kst.kernel_launches[i]}
     route_phases = {n: round(v / max(st.forward_calls, 1), 3)
                     for n, v in zip(abi.ROUTE_PHASES, st.route_phase_us)}
+    host_phases = host_us_per_call(st)
     launches = int(st.forward_calls * 3 + 2 * st.misses)  # route, hit gate/up, hit down; 2 per miss
 
     # end to end: host buffers through moe_layer_forward_host
@@ -437,9 +466,9 @@ def bench_decode(args, shape, rank, world, local):
                        "l2": "inputs larger than L2 (each step reads "
                              f"{k * L * rb / 1e9:.2f} GB of expert records)",
                        "cold_cache": True, "parallelism": f"replicas x{world}",
-                       "pool_distinct_records": DISTINCT_RECORDS},
+                       "pool_distinct_records": DISTINCT_RECORDS, "policy": args.policy},
             "miss_rate": st.misses / max(st.lookups, 1),
-            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec,
+            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec, **H2D_SM,
             "layer_roofline": {"t_roof_s": t_roof, "t_measured_s": el,
                                "frac": t_roof / el, "frac_at_8tbs": t_roof_8tb / el,
                                "hbm_term_s": hit_bytes / (hbm_peak * 1e9),
@@ -447,6 +476,7 @@ def bench_decode(args, shape, rank, world, local):
                                "bw_hbm_gbs": hbm_peak, "bw_h2d_gbs": h2d,
                                "hit_bytes": hit_bytes, "miss_bytes": miss_bytes},
             "roofline": roof, "kernels": kernels, "route_phase_us_per_call": route_phases,
+            "host_us_per_call": host_phases,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk,
         }
@@ -454,6 +484,13 @@ def bench_decode(args, shape, rank, world, local):
     stack.close()
     pool.close()
 
+
+
+def host_us_per_call(st):
+    """Host time per forward call: inside the call, waiting for the miss list, issuing after it."""
+    n = max(st.forward_calls, 1)
+    return {k: round(v / n, 2) for k, v in zip(("in_call", "wait_miss_list", "issue_after_list"),
+                                                st.host_us)}
 
 
 def kernel_table(kst):
@@ -607,7 +644,7 @@ def bench_prefill(args, shape, rank, world, local):
                        "pool_distinct_records": DISTINCT_RECORDS},
             "miss_rate": st.misses / max(st.lookups, 1),
             "prefetch_miss_rate": st.prefetch_misses / max(st.prefetch_lookups, 1),
-            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec,
+            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec, **H2D_SM,
             "layer_roofline": {"t_roof_s": t_roof, "t_measured_s": el, "frac": t_roof / el,
                                "hbm_term_s": hit_bytes / (hbm_peak * 1e9),
                                "h2d_term_s": miss_bytes / (h2d * 1e9),
@@ -615,6 +652,7 @@ def bench_prefill(args, shape, rank, world, local):
                                "hit_bytes": hit_bytes, "miss_bytes": miss_bytes,
                                "h2d_achieved_gbs": miss_bytes / el / 1e9},
             "expert_tflop": (flops_gu + flops_dn) / 1e12,
+            "host_us_per_call": host_us_per_call(st),
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches, "clocks": clk,
         }
@@ -713,7 +751,8 @@ def bench_concurrent(args, shape, rank, world, local):
                        "pool_distinct_records": DISTINCT_RECORDS},
             "miss_rate": st.misses / max(st.lookups, 1),
             "experts_per_layer_step": st.lookups / max(st.forward_calls, 1),
-            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec,
+            "host_us_per_call": host_us_per_call(st),
+            "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec, **H2D_SM,
             "layer_roofline": {"t_roof_s": t_roof, "t_measured_s": el, "frac": t_roof / el,
                                "hbm_term_s": hit_bytes / (hbm_peak * 1e9),
                                "h2d_term_s": miss_bytes / (h2d * 1e9),

@@ -12,6 +12,7 @@ from . import build as _build
 MOE_OK, MOE_ERR_ARG, MOE_ERR_CUDA, MOE_ERR_NOT_PINNED = 0, 1, 2, 3
 MOE_ERR_CAPACITY, MOE_ERR_TIMEOUT, MOE_ERR_STATE, MOE_ERR_UNSUPPORTED = 4, 5, 6, 7
 MOE_CACHE_RESET, MOE_CACHE_PREFETCH_NEXT = 1, 2
+MOE_CACHE_STATIC_SPLIT = 4
 MOE_K_ROUTE, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE = 0, 1, 2, 3
 MOE_K_PREFILL_ROUTE, MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_COUNT = 4, 5, 6, 7
 KERNEL_NAMES = ["route_lookup", "gate_up", "down", "combine", "prefill_route", "prefill_gate_up",
@@ -46,7 +47,8 @@ class moe_stats(ctypes.Structure):
                 ("kernel_launches", ctypes.c_int64 * MOE_K_COUNT),
                 ("kernel_ms", ctypes.c_double * MOE_K_COUNT),
                 ("kernel_bytes", ctypes.c_double * MOE_K_COUNT),
-                ("route_phase_us", ctypes.c_double * 8)]
+                ("route_phase_us", ctypes.c_double * 8),
+                ("host_us", ctypes.c_double * 3)]
 
 
 class moe_split(ctypes.Structure):
@@ -58,7 +60,7 @@ class moe_split(ctypes.Structure):
 EXPORTS = ["moe_record_bytes", "moe_record_layout", "moe_workspace_bytes", "moe_arena_bytes",
            "moe_layer_init", "cache_configure", "moe_layer_forward", "moe_layer_forward_host",
            "moe_get_routing", "moe_cache_export", "moe_get_stats", "moe_set_timing",
-           "moe_set_wait_limit", "moe_debug_inject", "plan_split", "moe_measure_h2d",
+           "moe_set_wait_limit", "moe_debug_inject", "plan_split", "moe_measure_h2d", "moe_measure_h2d_sm",
            "moe_route_noalloc", "moe_status_str", "moe_last_error", "moe_layer_destroy"]
 
 _lib = None
@@ -110,6 +112,8 @@ def lib():
         L.plan_split.argtypes = [i32, dbl, dbl, dbl, dbl, ctypes.POINTER(moe_split)]
         L.moe_measure_h2d.restype = ctypes.c_int
         L.moe_measure_h2d.argtypes = [vp, vp, sz, sz, i32, vp, ctypes.POINTER(dbl)]
+        L.moe_measure_h2d_sm.restype = ctypes.c_int
+        L.moe_measure_h2d_sm.argtypes = [vp, vp, sz, sz, i32, vp, ctypes.POINTER(dbl)]
         L.moe_route_noalloc.restype = ctypes.c_int
         L.moe_route_noalloc.argtypes = [vp, vp, i32, i32, i32, i32, i32, vp, vp, vp]
         L.moe_status_str.restype = ctypes.c_char_p
@@ -244,6 +248,15 @@ def moe_measure_h2d(dev_buf, host_buf, nbytes: int, chunk_bytes: int = 0, reps: 
     gbs = ctypes.c_double()
     _check(lib().moe_measure_h2d(_ptr(dev_buf), _ptr(host_buf), nbytes, chunk_bytes, reps,
                                  _stream(stream), ctypes.byref(gbs)), "moe_measure_h2d")
+    return gbs.value
+
+
+def moe_measure_h2d_sm(dev_buf, host_buf, nbytes: int, chunk_bytes: int = 0, reps: int = 10,
+                       stream=None) -> float:
+    """moe_measure_h2d with the copy done by an SM kernel reading mapped host memory."""
+    gbs = ctypes.c_double()
+    _check(lib().moe_measure_h2d_sm(_ptr(dev_buf), _ptr(host_buf), nbytes, chunk_bytes, reps,
+                                    _stream(stream), ctypes.byref(gbs)), "moe_measure_h2d_sm")
     return gbs.value
 
 

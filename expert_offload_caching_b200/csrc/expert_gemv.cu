@@ -9,12 +9,12 @@
 //
 // Decode is HBM-bound (a few rows, weights read once) and latency-bound when
 // one expert is processed alone.  So:
-//   * one CTA per 16-row weight tile; the tile's rows are contiguous in the
-//     record, so the CTA stages the whole tile into shared memory with 16-byte
-//     asynchronous copies (cp.async.cg, L1 bypassed) issued all at once.  No
-//     registers hold data in flight, and with ~26-41 KB per CTA several CTAs
-//     per SM keep ~200 KB per SM of HBM reads outstanding;
-//   * the 4 warps split the tile's K-steps of 256 elements;
+//   * one CTA per 16-row weight tile and group of experts; the tile's rows are
+//     contiguous in each record, so the CTA stages a whole tile into shared
+//     memory with 16-byte asynchronous copies (cp.async.cg, L1 bypassed)
+//     issued all at once, the next expert's tile while it computes the current
+//     one.  No registers hold data in flight;
+//   * the warps split the tile's K-steps of 256 elements;
 //   * E2M1 codes are decoded in registers with cvt.rn.f16x2.e2m1x2 (2 per op),
 //     then multiplied by the E4M3 block scale (cvt.rn.f16x2.e4m3x2); the
 //     product of an E2M1 and an E4M3 value is exact in fp16;
@@ -27,8 +27,9 @@
 //   * K-split partial sums are reduced in shared memory in a fixed order;
 //   * the gate/up launch prefetches the expert's down-projection bytes into
 //     L2 (prefetch.global.L2), so the down launch reads L2;
-//   * the last down launch of a layer also does the combine: its last CTA
-//     (threadfence + ticket, no waiting) sums the partials in ascending id.
+//   * the last down launch of a layer also does the combine, per 16-row tile:
+//     the tile's last CTA (threadfence + per-tile ticket, no waiting) sums its
+//     rows' partials in ascending id.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -76,6 +77,8 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 }
 
 constexpr int kMaxSteps = 16;  // K <= 4096: at most 16 K-steps of 256, one per warp
+constexpr int kMaxJobsPerCta = 32;
+constexpr int kCtaTarget = 8 * 148;  // CTAs per launch the expert grouping aims for
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
@@ -136,21 +139,29 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
     }
 }
 
-// One CTA per 16-row weight tile; each warp owns spw consecutive K-steps of 256
-// elements (spw = ceil(K-steps / warps)).  The tile's rows are contiguous in
-// the record; all threads stage it into shared memory with 16-byte cp.async
-// copies (the whole tile in flight at once), each warp computes its steps, and
-// warp 0 sums the warps' partials in a fixed order.  Dynamic shared memory:
-// 16*K/2 code bytes + K scale bytes + the partials (warps x NG x 512 bytes).
+// One CTA per (16-row weight tile, group of up to jobs_per_cta experts): the CTA
+// walks its experts in ascending id (the shared expert last), staging expert
+// i + 1's tile into the second shared-memory buffer (16-byte cp.async copies,
+// the whole tile in flight) while it computes expert i.  Each warp owns spw
+// consecutive K-steps of 256 elements; warp 0 sums the warps' partials in a
+// fixed order.  Dynamic shared memory: 2 x (16*K/2 code bytes + K scale
+// bytes) + the partials (warps x NG x 512 bytes).
 //
 // Launched with programmatic stream serialization: gate/up waits for the
 // route kernel before reading anything (job list, activations); the down
-// projection reads the job list (complete, two launches back), stages its W2
-// tile, and only then waits for gate/up's h.  Both release their dependents
-// early; every dependent waits before writing shared buffers.
+// projection reads the job list (complete, two launches back), stages its
+// first W2 tile, and only then waits for gate/up's h.  Every CTA executes the
+// wait, so a launch completes only after its predecessor.
+//
+// Combine (down launches with a.combine): the CTA that finishes a tile last
+// (per-tile ticket; the only CTA when the launch has one group) sums that
+// tile's 16 output rows over the layer's experts in ascending id, plus the
+// shared expert, for every row t.
 template <int NG>
 __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_job[kMaxJobsPerCta];  // job index, or -1: the shared expert
+    __shared__ int s_n, s_last;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, q = lane & 3;
     const bool gate_up = a.mode == kGateUp;
@@ -158,62 +169,81 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
     if (gate_up) pdl_wait();  // job list and x come from the previous launch
     pdl_launch_dependents();
 
-    // ---- which expert (job) this CTA serves
-    const uint8_t *rec = nullptr;
-    int nrows = 0, row_off = 0;
-    bool shared = false, work = true;
-    if (a.only_job < 0 && (int)blockIdx.y == a.shared_slot) {
-        rec = a.shared_rec;
-        nrows = a.T;
-        shared = true;
-    } else {
-        // L2 reads (ld.global.cg): the down launch reads these before its PDL
-        // wait, and an SM's L1 may still hold lines of an older launch
-        const int jy = a.only_job >= 0 ? a.only_job : (int)blockIdx.y;
-        if (jy >= __ldcg(a.n_jobs)) {
-            work = false;
-        } else {
-            const int4 j0 = __ldcg(reinterpret_cast<const int4 *>(&a.jobs[jy]));  // expert, slot, hit, nrows
-            const int row_off_j = __ldcg(&a.jobs[jy].row_off);
-            if (a.only_job < 0 && !j0.z) {
-                work = false;
-            } else {
-                rec = a.arena + (int64_t)j0.y * a.rec_bytes;
-                nrows = j0.w;
-                row_off = row_off_j;
-            }
+    // ---- this CTA's experts: launch slots [y*J, y*J + J) -- hit jobs, and the
+    // shared expert at slot shared_slot -- or the one job only_job.  L2 reads
+    // (ld.global.cg): the down launch reads the job list before its PDL wait,
+    // and an SM's L1 may still hold lines of an older launch.
+    if (warp == 0) {
+        int mine = -2;
+        if (a.only_job >= 0) {
+            if (lane == 0 && blockIdx.y == 0) mine = a.only_job;
+        } else if (lane < a.jobs_per_cta) {
+            const int slot = (int)blockIdx.y * a.jobs_per_cta + lane;
+            if (slot == a.shared_slot) mine = -1;
+            else if (slot < __ldcg(a.n_jobs) && __ldcg(&a.jobs[slot].hit)) mine = slot;
         }
+        const unsigned ball = __ballot_sync(0xffffffffu, mine != -2);
+        if (mine != -2) s_job[__popc(ball & ((1u << lane) - 1u))] = mine;
+        if (lane == 0) s_n = __popc(ball);
     }
+    __syncthreads();
+    const int njobs = s_n;
 
     const int K = gate_up ? a.d : a.F;
-    const int tiles = gate_up ? (a.F >> 3) : (a.d >> 4);
     const int tile = blockIdx.x;
-    if (work && tile < tiles) {
-        const int NCH = K >> 6;
-        const int nwarps = (int)(blockDim.x >> 5);
-        const int nsteps = (NCH + 3) >> 2;
-        const int spw = (nsteps + nwarps - 1) / nwarps;
-        const uint32_t code_bytes = 16u * (uint32_t)(K >> 1), scale_bytes = (uint32_t)K;
-        uint8_t *s_codes = smem, *s_scales = smem + code_bytes;
-        float(*red)[NG][4][32] = reinterpret_cast<float(*)[NG][4][32]>(smem + code_bytes + scale_bytes);
+    const int NCH = K >> 6;
+    const int nwarps = (int)(blockDim.x >> 5);
+    const int nsteps = (NCH + 3) >> 2;
+    const int spw = (nsteps + nwarps - 1) / nwarps;
+    const uint32_t code_bytes = 16u * (uint32_t)(K >> 1), scale_bytes = (uint32_t)K;
+    const uint32_t buf_bytes = code_bytes + scale_bytes;
+    const int nbuf = a.jobs_per_cta > 1 ? 2 : 1;  // a second buffer only when the CTA has several experts
+    float(*red)[NG][4][32] = reinterpret_cast<float(*)[NG][4][32]>(smem + nbuf * buf_bytes);
+
+    auto record = [&](int jid) -> const uint8_t * {
+        return jid < 0 ? a.shared_rec : a.arena + (int64_t)__ldcg(&a.jobs[jid].slot) * a.rec_bytes;
+    };
+    // stage expert i of the list into buffer i & 1 (one cp.async group)
+    auto stage = [&](int i) {
+        const uint8_t *rec = record(s_job[i]);
+        uint8_t *dst = smem + (i & (nbuf - 1)) * buf_bytes;
         const uint8_t *codes = rec + (gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)tile * code_bytes;
         const uint8_t *scales = rec + (gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)tile * scale_bytes;
-        // stage the tile: every thread issues its 16-byte pieces, then waits for its own
-        const uint32_t n16c = code_bytes >> 4, n16s = scale_bytes >> 4;
-        for (uint32_t i = threadIdx.x; i < n16c; i += blockDim.x) cp_async16(s_codes + 16 * i, codes + 16 * i);
-        for (uint32_t i = threadIdx.x; i < n16s; i += blockDim.x) cp_async16(s_scales + 16 * i, scales + 16 * i);
-        if (gate_up) {  // this expert's down projection -> L2 for the down launch
+        for (uint32_t o = threadIdx.x; o < (code_bytes >> 4); o += blockDim.x) cp_async16(dst + 16 * o, codes + 16 * o);
+        for (uint32_t o = threadIdx.x; o < (scale_bytes >> 4); o += blockDim.x)
+            cp_async16(dst + code_bytes + 16 * o, scales + 16 * o);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (gate_up) {  // this expert's down projection -> L2 for the down launch (a 1/tiles slice)
             const uint32_t total = (uint32_t)(a.lay.bytes - a.lay.w2_codes);
             const uint32_t per = ((total / gridDim.x) + 127u) & ~127u;
             const uint32_t off = per * blockIdx.x;
             if (off < total) prefetch_l2_range(rec + a.lay.w2_codes + off, per < total - off ? per : total - off);
         }
-        const float *ts = reinterpret_cast<const float *>(rec + a.lay.tscales);
-        // tile-local rows of this thread: gate_up 2g (gate) / 2g+1 (up); down g / g+8
-        const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
-        if (!gate_up) pdl_wait();  // h comes from the gate/up launch; W2 is already in flight
-        cp_async_wait_all();
+    };
+
+    if (!gate_up) {
+        if (njobs > 0) stage(0);  // W2 does not depend on the gate/up launch
+        pdl_wait();               // h does
+    } else if (njobs > 0) {
+        stage(0);
+    }
+    // tile-local rows of this thread: gate_up 2g (gate) / 2g+1 (up); down g / g+8
+    const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
+    for (int i = 0; i < njobs; ++i) {
+        if (i + 1 < njobs) {
+            stage(i + 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
         __syncthreads();
+        const int jid = s_job[i];
+        const bool shared = jid < 0;
+        const uint8_t *rec = record(jid);
+        const int nrows = shared ? a.T : __ldcg(&a.jobs[jid].nrows);
+        const int row_off = shared ? 0 : __ldcg(&a.jobs[jid].row_off);
+        const uint8_t *s_codes = smem + (i & (nbuf - 1)) * buf_bytes, *s_scales = s_codes + code_bytes;
+        const float *ts = reinterpret_cast<const float *>(rec + a.lay.tscales);
         for (int r0 = 0; r0 < nrows; r0 += 4 * NG) {
             // mma column n = g carries activation row r0 + 4*grp + g/2, the hi (g
             // even) or lo (g odd) fp16 part.
@@ -239,8 +269,8 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
             for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) acc[grp][j] = 0.f;
-            for (int i = 0; i < spw; ++i) {  // this warp's K-steps (uniform across the warp)
-                const int c = 4 * (warp * spw + i) + q;
+            for (int st = 0; st < spw; ++st) {  // this warp's K-steps (uniform across the warp)
+                const int c = 4 * (warp * spw + st) + q;
                 const bool cv = c < NCH;  // ragged K tail: some lanes of the quad feed zeros
                 const int cc = cv ? c : 0;
                 const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
@@ -279,39 +309,40 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
                         a.hh_out[sel * 2 * a.F + j] = hi;
                         a.hh_out[sel * 2 * a.F + a.F + j] = lo;
                     } else {
-                        const int i = 16 * tile + g;
-                        a.part_out[sel * a.d + i] = ts[2] * v0;
-                        a.part_out[sel * a.d + i + 8] = ts[2] * v1;
+                        const int o = 16 * tile + g;
+                        a.part_out[sel * a.d + o] = ts[2] * v0;
+                        a.part_out[sel * a.d + o + 8] = ts[2] * v1;
                     }
                 }
             }
-            __syncthreads();
+            __syncthreads();  // red reused; after the last row group, the buffer is free
         }
     }
 
-    if (a.combine) {  // the launch's last CTA sums the partials of the layer
-        __shared__ int s_last;
+    if (a.combine && !gate_up) {
         __syncthreads();
-        if (threadIdx.x == 0) {
-            __threadfence();
-            const unsigned int total = gridDim.x * gridDim.y;
-            s_last = (atomicAdd(a.ticket, 1u) == total - 1);
+        bool last = true;
+        if (gridDim.y > 1) {
+            if (threadIdx.x == 0) {
+                __threadfence();
+                s_last = atomicAdd(&a.tile_ticket[tile], 1u) == gridDim.y - 1;
+            }
+            __syncthreads();
+            last = s_last;
+            if (last) __threadfence();
         }
-        __syncthreads();
-        if (s_last) {
-            __threadfence();
-            if (a.combine == 1 || *a.n_misses == 0) {
-                const int n = a.T * a.d;
-                for (int i = threadIdx.x; i < n; i += blockDim.x) {
-                    const int t = i / a.d, c = i - t * a.d;
-                    const float *pr = a.part_out + (size_t)t * (a.k + 1) * a.d + c;
-                    float s = 0.f;
-                    for (int p = 0; p < a.k; ++p) s = fmaf(a.gates[t * a.k + p], pr[(size_t)p * a.d], s);
-                    if (a.shared_rec) s += pr[(size_t)a.k * a.d];
-                    a.y[i] = s;
+        if (last) {
+            if (a.combine == 1 || __ldcg(a.n_misses) == 0) {
+                for (int e = threadIdx.x; e < 16 * a.T; e += blockDim.x) {
+                    const int t = e >> 4, o = 16 * tile + (e & 15);
+                    const float *pr = a.part_out + (size_t)t * (a.k + 1) * a.d + o;
+                    float sum = 0.f;
+                    for (int p = 0; p < a.k; ++p) sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                    if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
+                    a.y[(size_t)t * a.d + o] = sum;
                 }
             }
-            if (threadIdx.x == 0) *a.ticket = 0u;
+            if (gridDim.y > 1 && threadIdx.x == 0) a.tile_ticket[tile] = 0u;
         }
     }
 }
@@ -340,16 +371,29 @@ cudaError_t launch_ng(const GemvArgs &a, dim3 grid, int threads, size_t smem, cu
 
 }  // namespace
 
-cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s) {
+cudaError_t launch_gemv(const GemvArgs &a_in, int slots, cudaStream_t s) {
+    GemvArgs a = a_in;
     const int K = a.mode == kGateUp ? a.d : a.F;
     const int tiles = a.mode == kGateUp ? a.F / 8 : a.d / 16;
     const int nsteps = (K / 64 + 3) / 4;
-    if (nsteps < 1 || nsteps > kMaxSteps) return cudaErrorInvalidValue;
+    if (nsteps < 1 || nsteps > kMaxSteps || slots < 1) return cudaErrorInvalidValue;
     const int spw = nsteps >= 8 ? 2 : 1;  // 2 K-steps per warp for long rows: smaller CTAs, more per SM
     const int warps = (nsteps + spw - 1) / spw;
-    const dim3 grid(tiles, grid_y);
+    // expert groups per tile: about kCtaTarget CTAs (several per SM, so staging
+    // latencies overlap across CTAs), at most 32 experts per CTA
+    int gy = 1;
+    if (a.only_job < 0) {
+        gy = (kCtaTarget + tiles - 1) / tiles;
+        if (gy > slots) gy = slots;
+        if ((slots + gy - 1) / gy > kMaxJobsPerCta) gy = (slots + kMaxJobsPerCta - 1) / kMaxJobsPerCta;
+        a.jobs_per_cta = (slots + gy - 1) / gy;
+    } else {
+        a.jobs_per_cta = 1;
+    }
+    const dim3 grid(tiles, gy);
     const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
-    const size_t smem = 16 * (size_t)(K / 2) + (size_t)K + (size_t)warps * ng * 4 * 32 * sizeof(float);
+    const size_t buf = 16 * (size_t)(K / 2) + (size_t)K;  // one expert's tile: codes + scales
+    const size_t smem = (a.jobs_per_cta > 1 ? 2 : 1) * buf + (size_t)warps * ng * 4 * 32 * sizeof(float);
     if (smem > 96 * 1024) return cudaErrorInvalidValue;
     if (ng == 1) return launch_ng<1>(a, grid, warps * 32, smem, s);
     return launch_ng<2>(a, grid, warps * 32, smem, s);

@@ -85,7 +85,7 @@ WsLayout ws_layout(const moe_dims *d) {
     w.n_jobs = take(4);
     w.n_misses = take(4);
     w.ticket = take(4);
-    w.ticket2 = take(4);
+    w.ticket2 = take(4 * kMaxTiles);
     w.rowrefs = take(T * k * (int64_t)sizeof(RowRef));
     w.xh = take(Td * 2 * dd * 2);
     w.hh = take(Td * (k + 1) * 2 * F * 2);
@@ -171,6 +171,7 @@ struct moe_ctx {
     // injection and limits
     int64_t inj_copy_fail_at = 0, inj_drop_publish = 0;
     double wait_limit = 60.0;
+    std::chrono::steady_clock::time_point issue_t0;  // end of the last miss-list wait
 };
 
 namespace {
@@ -256,7 +257,7 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
     g.n_misses = ctx->dws.n_misses;
     g.gates = ctx->dws.gates;
     g.y = nullptr;
-    g.ticket = ctx->dws.ticket2;
+    g.tile_ticket = ctx->dws.ticket2;
     return g;
 }
 
@@ -278,6 +279,15 @@ moe_status device_error(moe_ctx *ctx) {
 // Bounded host wait for the device's miss list (sequence number `seq`).
 moe_status wait_miss_list(moe_ctx *ctx, uint32_t seq) {
     const auto t0 = std::chrono::steady_clock::now();
+    struct Account {  // time spent here, and the start of the issue phase that follows
+        moe_ctx *c;
+        std::chrono::steady_clock::time_point a;
+        ~Account() {
+            const auto now = std::chrono::steady_clock::now();
+            c->stats.host_us[1] += std::chrono::duration<double, std::micro>(now - a).count();
+            c->issue_t0 = now;
+        }
+    } account{ctx, t0};
     uint64_t spins = 0;
     while (ctx->page_h->seq != seq) {
         _mm_pause();
@@ -427,6 +437,8 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     ctx->stats.misses += nev - hits;
     ctx->stats.evictions += evictions;
     ctx->stats.forward_calls += 1;
+    ctx->stats.host_us[2] +=
+        std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - ctx->issue_t0).count();
     fill_trace(ctx, layer, nev, nev, trace);
     ctx->last_T = T;
     return MOE_OK;
@@ -597,6 +609,8 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     ctx->stats.prefetch_lookups += nev - n;
     ctx->stats.prefetch_misses += npm;
     ctx->stats.forward_calls += 1;
+    ctx->stats.host_us[2] +=
+        std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - ctx->issue_t0).count();
     fill_trace(ctx, layer, n, nev, trace);
     ctx->last_T = T;
     return MOE_OK;
@@ -726,7 +740,7 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
         }
     }
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket2, 0, 4, ctx->cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket2, 0, 4 * kMaxTiles, ctx->cs);
     if (e != cudaSuccess) {
         st = cuda_fail(ctx, e, "moe_layer_init");
         moe_layer_destroy(ctx);
@@ -745,8 +759,13 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
     if ((flags & MOE_CACHE_PREFETCH_NEXT) && num_slots < 2ll * D.E) return MOE_ERR_CAPACITY;
     if (num_slots > 65536) return MOE_ERR_UNSUPPORTED;
     if (arena_bytes < moe_arena_bytes(&D, num_slots)) return MOE_ERR_ARG;
+    const bool stat = (flags & MOE_CACHE_STATIC_SPLIT) != 0;
+    if (stat && (flags & MOE_CACHE_PREFETCH_NEXT)) return MOE_ERR_ARG;
     const bool reset = (flags & MOE_CACHE_RESET) || !ctx->configured || ctx->arena != slot_arena ||
-                       ctx->C != num_slots;
+                       ctx->C != num_slots || ((ctx->flags ^ flags) & MOE_CACHE_STATIC_SPLIT);
+    // static split: the resident experts per layer, after `need` scratch slots
+    int64_t per_layer = stat ? (num_slots - need) / D.L : 0;
+    if (per_layer > D.E) per_layer = D.E;
     uint8_t *a = static_cast<uint8_t *>(slot_arena);
     ctx->arena = a;
     ctx->C = num_slots;
@@ -757,6 +776,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
     ctx->tab.owner = reinterpret_cast<int32_t *>(tb + tl.owner);
     ctx->tab.stamp = reinterpret_cast<unsigned long long *>(tb + tl.stamp);
     ctx->tab.C = num_slots;
+    ctx->tab.scratch_base = stat ? (int32_t)(D.L * per_layer) : -1;
     ctx->flags = flags & ~MOE_CACHE_RESET;
     if (ctx->wl.xq >= 0) {  // prefill GEMM descriptors of the arena's weight codes
         if (!make_operand_map(&ctx->maps.w13, a + ctx->lay.w13_codes, D.d / 2, 2 * D.F, num_slots, ctx->lay.bytes) ||
@@ -773,15 +793,47 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         // finish outstanding work of the old state first
         CK(cudaStreamSynchronize(ctx->xs));
         CK(cudaStreamSynchronize(ctx->cs));
-        CK(launch_table_reset(ctx->tab, (int64_t)D.L * D.E, ctx->cs));
+        if (stat) {
+            CK(launch_table_static(ctx->tab, D.L, D.E, (int)per_layer, ctx->cs));
+        } else {
+            CK(launch_table_reset(ctx->tab, (int64_t)D.L * D.E, ctx->cs));
+        }
         CK(cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs));
-        CK(cudaMemsetAsync(ctx->dws.ticket2, 0, 4, ctx->cs));
+        CK(cudaMemsetAsync(ctx->dws.ticket2, 0, 4 * kMaxTiles, ctx->cs));
         ctx->pending.clear();
         ctx->page_h->error = 0;
         std::fill(ctx->pf_pending.begin(), ctx->pf_pending.end(), 0);
         memset(&ctx->stats, 0, sizeof ctx->stats);
         ctx->state = MOE_OK;
         ctx->err.clear();
+        if (stat && per_layer > 0) {
+            // fill the resident set (layer l's experts 0 .. per_layer-1 in consecutive
+            // slots), merging records consecutive in both the pool and the arena;
+            // the compute stream waits for the fill
+            int64_t run_src = -1, run_dst = -1, run_n = 0;
+            auto flush = [&]() -> cudaError_t {
+                if (run_n == 0) return cudaSuccess;
+                const cudaError_t e = cudaMemcpyAsync(a + run_dst * ctx->lay.bytes, ctx->pool + run_src * ctx->lay.bytes,
+                                                      run_n * ctx->lay.bytes, cudaMemcpyHostToDevice, ctx->xs);
+                run_n = 0;
+                return e;
+            };
+            for (int l = 0; l < D.L; ++l)
+                for (int64_t e = 0; e < per_layer; ++e) {
+                    const int64_t src = ((int64_t)l * D.E + e) % ctx->P, dst = l * per_layer + e;
+                    if (run_n > 0 && src == run_src + run_n && dst == run_dst + run_n) {
+                        ++run_n;
+                        continue;
+                    }
+                    CK(flush());
+                    run_src = src;
+                    run_dst = dst;
+                    run_n = 1;
+                }
+            CK(flush());
+            CK(cudaEventRecord(ctx->ev_routed, ctx->xs));
+            CK(cudaStreamWaitEvent(ctx->cs, ctx->ev_routed, 0));
+        }
     }
     ctx->configured = true;
     return MOE_OK;
@@ -794,8 +846,11 @@ moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t
     if (!ctx->configured) return MOE_ERR_STATE;
     const moe_dims &D = ctx->dims;
     if (layer < 0 || layer >= D.L || T < 1 || T > D.max_rows || !x || !y) return MOE_ERR_ARG;
-    if (T <= kDecodeMaxRows) return forward_decode(ctx, layer, x, T, y, trace);
-    return forward_prefill(ctx, layer, x, T, y, trace);
+    const auto t0 = std::chrono::steady_clock::now();
+    const moe_status st = T <= kDecodeMaxRows ? forward_decode(ctx, layer, x, T, y, trace)
+                                              : forward_prefill(ctx, layer, x, T, y, trace);
+    ctx->stats.host_us[0] += std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+    return st;
 }
 
 moe_status moe_layer_forward_host(moe_ctx *ctx, int32_t layer, const void *x_host, int32_t T,
@@ -916,6 +971,61 @@ moe_status moe_measure_h2d(void *dev_buf, const void *host_buf, size_t bytes, si
                                static_cast<const uint8_t *>(host_buf) + o, n,
                                cudaMemcpyHostToDevice, s));
         }
+        CK(cudaEventRecord(b, s));
+        CK(cudaEventSynchronize(b));
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, a, b));
+        const double rate = (double)bytes / (ms * 1e-3) / 1e9;
+        if (rate > best) best = rate;
+    }
+    cudaEventDestroy(a);
+    cudaEventDestroy(b);
+    *gbs = best;
+    return MOE_OK;
+}
+
+// SM-driven copy from mapped page-locked host memory: every thread streams
+// 16-byte loads (4 in flight) over PCIe and stores them to device memory.
+__global__ void h2d_sm_copy_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, size_t n16) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n16; i += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldcv(src + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[i + u * stride] = v[u];
+    }
+    for (; i < n16; i += stride) dst[i] = __ldcv(src + i);
+}
+
+moe_status moe_measure_h2d_sm(void *dev_buf, const void *host_buf, size_t bytes, size_t chunk_bytes,
+                              int32_t reps, void *stream, double *gbs) {
+    moe_ctx *ctx = nullptr;
+    if (!dev_buf || !host_buf || !bytes || reps < 1 || !stream || !gbs) return MOE_ERR_ARG;
+    const size_t chunk = chunk_bytes ? chunk_bytes : bytes;
+    if ((bytes & 15) || (chunk & 15) || (reinterpret_cast<uintptr_t>(dev_buf) & 15) ||
+        (reinterpret_cast<uintptr_t>(host_buf) & 15))
+        return MOE_ERR_ARG;
+    void *src = nullptr;
+    if (cudaHostGetDevicePointer(&src, const_cast<void *>(host_buf), 0) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_NOT_PINNED;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t a, b;
+    CK(cudaEventCreate(&a));
+    CK(cudaEventCreate(&b));
+    double best = 0.0;
+    for (int r = 0; r < reps; ++r) {
+        CK(cudaEventRecord(a, s));
+        for (size_t o = 0; o < bytes; o += chunk) {
+            const size_t n = bytes - o < chunk ? bytes - o : chunk;
+            h2d_sm_copy_kernel<<<296, 512, 0, s>>>(
+                reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(src) + o),
+                reinterpret_cast<uint4 *>(static_cast<uint8_t *>(dev_buf) + o), n / 16);
+        }
+        CK(cudaGetLastError());
         CK(cudaEventRecord(b, s));
         CK(cudaEventSynchronize(b));
         float ms = 0.f;

@@ -11,6 +11,7 @@ namespace moe {
 constexpr int kDecodeMaxRows = 32;  // T <= this takes the GEMV (decode) path
 constexpr int kMaxK = 32;
 constexpr int kMaxE = 1024;
+constexpr int kMaxTiles = 512;  // GEMV tiles per launch: max(d / 16, F / 8) with d, F <= 4096
 
 // Record sections (byte offsets), computed once per context.
 struct RecordLayout {
@@ -33,6 +34,10 @@ struct Table {
     int32_t *owner;             // [C] key in slot or -1
     unsigned long long *stamp;  // [C]
     int64_t C;
+    // static per-layer split (scratch_base >= 0): map holds the fixed resident
+    // set and never changes; the m-th miss of a batch goes to slot
+    // scratch_base + m, reused by every batch
+    int32_t scratch_base;
 };
 
 // One distinct expert of a lookup batch, in ascending expert order.
@@ -75,7 +80,7 @@ struct DecodeWs {
     __half *hh;          // [maxT][k+1][2][F] fp16 hi/lo split of h
     float *part;         // [maxT][k+1][d] per-selection expert outputs (p = k: shared)
     uint32_t *ticket;    // last-CTA counter of the route kernel
-    uint32_t *ticket2;   // last-CTA counter of the combining down launch
+    uint32_t *ticket2;   // [kMaxTiles] per-tile counters of the combining down launch
     // prefill only (T > 32)
     int32_t *cnt;        // [E] rows per expert
     int32_t *fill;       // [E] scatter cursors
@@ -113,6 +118,7 @@ struct GemvArgs {
     const int32_t *n_jobs;
     const RowRef *rowrefs;
     int only_job;          // >= 0: process just this job; -1: every hit job (+ shared)
+    int jobs_per_cta;      // job slots per CTA (set by launch_gemv)
     int shared_slot;       // gridDim.y index of the shared job, -1 if none
     const uint8_t *arena;
     int64_t rec_bytes;
@@ -129,7 +135,7 @@ struct GemvArgs {
     const int32_t *n_misses;
     const float *gates;
     float *y;
-    uint32_t *ticket;
+    uint32_t *tile_ticket;  // [tiles] per-tile counters of the combining launch, kept at 0
 };
 
 // Grouped W4A4 expert GEMMs of a prefill chunk (tcgen05 block-scaled MMA).
@@ -164,8 +170,10 @@ struct GroupedGemmMaps {
 
 // launchers (one per .cu)
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
-cudaError_t launch_gemv(const GemvArgs &a, int grid_y, cudaStream_t s);
+// slots: job slots of the launch (max jobs + shared expert), 1 with only_job
+cudaError_t launch_gemv(const GemvArgs &a, int slots, cudaStream_t s);
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
+cudaError_t launch_table_static(Table t, int L, int E, int per_layer, cudaStream_t s);
 cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,

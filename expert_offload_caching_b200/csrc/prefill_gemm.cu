@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_full + 8 * s, 32);  // the producer warp's lanes (one with the tx count)
+            mbar_init(bar_full + 8 * s, 33);  // lane 0's tx-count arrive + all 32 lanes after their scales
             mbar_init(bar_empty + 8 * s, 1);  // tcgen05.commit of the MMA thread
         }
         mbar_init(bar_done, 1);
@@ -280,7 +280,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---- producer: scale factors by the lanes, operand tiles by TMA
+        // ---- producer: operand tiles by TMA, scale factors by the lanes.  The
+        // scale words of stage it + 1 are loaded into registers while stage it
+        // is handed over, so their latency overlaps the wait for a free stage.
+        uint32_t wa[4][kStepsPerStage], wb[4][kStepsPerStage];
+        auto load_sf = [&](int itl) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                // row m = lane + 32c of the tile; its 4 scales of a K step are one word
+                const int wrow = mt * kBM + lane + 32 * c;
+                const int n = n0 + lane + 32 * c;
+                const uint32_t *pw = reinterpret_cast<const uint32_t *>(wsf + (int64_t)wrow * sf_pitch);
+                const uint32_t *pb =
+                    reinterpret_cast<const uint32_t *>(a.act_scales + (int64_t)(row_off + n) * sf_pitch);
+#pragma unroll
+                for (int i = 0; i < kStepsPerStage; ++i) {
+                    const int ks = itl * kStepsPerStage + i;
+                    wa[c][i] = (wrow < rows_w && ks < ksteps) ? __ldg(pw + ks) : 0u;
+                    wb[c][i] = (n < nrows && ks < ksteps) ? __ldg(pb + ks) : 0u;
+                }
+            }
+        };
+        load_sf(0);
         int it = 0;
         for (; it < nkb; ++it) {
             const int s = it % kStages, r = it / kStages;
@@ -290,38 +311,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (lane == 0) { gemm_fail(a, 41, it); *s_fail = 1; }
                 break;
             }
-#pragma unroll 1
-            for (int i = 0; i < kStepsPerStage; ++i) {
-                const int ks = it * kStepsPerStage + i;
-                if (ks >= ksteps) break;
-                uint32_t *sfa = reinterpret_cast<uint32_t *>(sm + kOffSfA + (s * kStepsPerStage + i) * kSfAtom);
-                uint32_t *sfb = reinterpret_cast<uint32_t *>(sm + kOffSfB + (s * kStepsPerStage + i) * kSfAtom);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    // atom word of row m = lane + 32c: 16 B per lane row, 4 B per row quarter
-                    const int wrow = mt * kBM + lane + 32 * c;
-                    uint32_t w = 0u;
-                    if (wrow < rows_w)
-                        w = __ldg(reinterpret_cast<const uint32_t *>(wsf + (int64_t)wrow * sf_pitch) + ks);
-                    sfa[lane * 4 + c] = w;
-                    const int n = n0 + lane + 32 * c;
-                    uint32_t b = 0u;
-                    if (n < nrows)
-                        b = __ldg(reinterpret_cast<const uint32_t *>(a.act_scales +
-                                                                     (int64_t)(row_off + n) * sf_pitch) + ks);
-                    sfb[lane * 4 + c] = b;
-                }
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
             if (lane == 0) {
                 mbar_arrive_tx(bar_full + 8 * s, 2 * kTileBytes);
                 const uint32_t da = base + kOffA + s * kTileBytes, db = base + kOffB + s * kTileBytes;
                 tma_load_3d(da, shared ? &tm_ws : &tm_w, bar_full + 8 * s, it * kStageKBytes, mt * kBM, zc);
                 tma_load_2d(db, &tm_act, bar_full + 8 * s, it * kStageKBytes, row_off + n0);
-            } else {
-                mbar_arrive(bar_full + 8 * s);
             }
+            // scale-factor atoms: lane row holds rows lane, lane + 32, lane + 64, lane + 96
+#pragma unroll
+            for (int i = 0; i < kStepsPerStage; ++i) {
+                uint4 *sfa = reinterpret_cast<uint4 *>(sm + kOffSfA + (s * kStepsPerStage + i) * kSfAtom);
+                uint4 *sfb = reinterpret_cast<uint4 *>(sm + kOffSfB + (s * kStepsPerStage + i) * kSfAtom);
+                sfa[lane] = make_uint4(wa[0][i], wa[1][i], wa[2][i], wa[3][i]);
+                sfb[lane] = make_uint4(wb[0][i], wb[1][i], wb[2][i], wb[3][i]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(bar_full + 8 * s);
+            if (it + 1 < nkb) load_sf(it + 1);
         }
         // on failure: let the stages already issued land before the CTA exits
         if (it < nkb && lane == 0) {

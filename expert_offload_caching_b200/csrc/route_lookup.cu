@@ -232,6 +232,30 @@ __device__ void lookup_batch(const Table &tab, int layer, int E, int n, LookupSm
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int64_t keybase = (int64_t)layer * E;
     const int C = (int)tab.C;
+    if (tab.scratch_base >= 0) {  // static split: resident set fixed, misses to scratch slots
+        for (int j = threadIdx.x; j < n; j += blockDim.x) sm.slot[j] = tab.map[keybase + sm.exp[j]];
+        __syncthreads();
+        if (threadIdx.x == 0 && t_read) *t_read = global_ns();
+        if (warp == 0) {
+            int hc = 0, mc = 0;
+            for (int j0 = 0; j0 < n; j0 += 32) {
+                const int j = j0 + lane;
+                const bool valid = j < n, hit = valid && sm.slot[j] >= 0;
+                const unsigned hm = __ballot_sync(0xffffffffu, hit);
+                const unsigned mm = __ballot_sync(0xffffffffu, valid && !hit);
+                if (valid && !hit) {
+                    const int m = mc + __popc(mm & ((1u << lane) - 1u));
+                    sm.slot[j] = -2 - (tab.scratch_base + m);
+                }
+                if (valid) sm.evict[j] = -1;
+                hc += __popc(hm);
+                mc += __popc(mm);
+            }
+            if (lane == 0) { sm.nhit = hc; sm.nmiss = mc; }
+        }
+        __syncthreads();
+        return;
+    }
     for (int i = threadIdx.x; i < kMaxSlotBits / 32; i += blockDim.x) sm.hitmap[i] = 0u;
     for (int j = threadIdx.x; j < n; j += blockDim.x) sm.slot[j] = tab.map[keybase + sm.exp[j]];
     if (threadIdx.x == 0) { sm.clock = tab.hdr->clock; sm.nf = tab.hdr->next_free; }
@@ -471,7 +495,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
         t_table = global_ns();
     }
 
-    // ---- publish: one 16-byte record per entry, the counts, phase times, then the flag
+    // ---- publish: one 16-byte record per entry, the counts and phase times,
+    // then the flag with one system-scope release store (cumulative: the
+    // warp's writes, ordered before it by the warp barrier, land first)
     if (warp == 0) {
         publish_events(a.page, 0, sm, njobs, 0);
         if (lane == 0) {
@@ -484,15 +510,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
             a.page->phase_ns[3] = (uint32_t)(t_jobs - t_topk);
             a.page->phase_ns[4] = (uint32_t)(t_read - t_jobs);
             a.page->phase_ns[5] = (uint32_t)(t_table - t_read);
-        }
-        __threadfence_system();
-        __syncwarp();
-        if (lane == 0) {
-            const unsigned long long t_pub = global_ns();
-            a.page->phase_ns[6] = (uint32_t)(t_pub - t_table);
+            a.page->phase_ns[6] = (uint32_t)(global_ns() - t_table);
             a.page->phase_ns[7] = (uint32_t)(t_start - t_entry);  // launch-to-start: PDL wait
-            __threadfence_system();
-            if (a.publish) a.page->seq = a.seq;
+        }
+        __syncwarp();
+        if (lane == 0 && a.publish) {
+            const uint32_t v = a.seq;
+            asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(&a.page->seq), "r"(v) : "memory");
         }
     }
     __syncthreads();
@@ -697,6 +721,27 @@ __global__ void table_reset_kernel(Table t, int64_t nkeys) {
     }
 }
 
+// Static per-layer split: expert e < per_layer of layer l resident in slot
+// l*per_layer + e; every other key absent; the scratch slots unowned.
+__global__ void table_static_kernel(Table t, int L, int E, int per_layer) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t nkeys = (int64_t)L * E;
+    for (int64_t j = i; j < nkeys; j += stride) {
+        const int l = (int)(j / E), e = (int)(j - (int64_t)l * E);
+        t.map[j] = e < per_layer ? l * per_layer + e : -1;
+    }
+    for (int64_t j = i; j < t.C; j += stride) {
+        const bool resident = j < (int64_t)L * per_layer;
+        t.owner[j] = resident ? (int)((j / per_layer) * E + j % per_layer) : -1;
+        t.stamp[j] = 0ull;
+    }
+    if (i == 0) {
+        t.hdr->clock = 0ull;
+        t.hdr->next_free = L * per_layer;
+    }
+}
+
 template <int NV>
 cudaError_t launch_nv(const RouteArgs &a, int grid, cudaStream_t s) {
     static bool configured = false;  // allow up to 64 KB of dynamic smem for the x chunk
@@ -759,6 +804,11 @@ cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s) {
 
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s) {
     table_reset_kernel<<<256, 256, 0, s>>>(t, nkeys);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_table_static(Table t, int L, int E, int per_layer, cudaStream_t s) {
+    table_static_kernel<<<256, 256, 0, s>>>(t, L, E, per_layer);
     return cudaGetLastError();
 }
 

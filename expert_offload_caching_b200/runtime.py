@@ -22,7 +22,7 @@ class LayerStack:
 
     def __init__(self, dims: abi.moe_dims, host_pool: torch.Tensor, router_w: torch.Tensor,
                  shared: torch.Tensor | None, num_slots: int, *, prefetch: bool = False,
-                 device: str | torch.device = "cuda"):
+                 static_split: bool = False, device: str | torch.device = "cuda"):
         if not torch.cuda.is_available():
             raise RuntimeError("LayerStack needs a CUDA device")
         self.dims = dims
@@ -38,7 +38,8 @@ class LayerStack:
         torch.cuda.synchronize(self.device)
         self.ctx = abi.moe_layer_init(dims, host_pool, host_pool.numel(), router_w, shared,
                                       self.ws, self.ws.numel(), self.compute, self.copy)
-        self.flags = abi.MOE_CACHE_PREFETCH_NEXT if prefetch else 0
+        self.flags = ((abi.MOE_CACHE_PREFETCH_NEXT if prefetch else 0) |
+                      (abi.MOE_CACHE_STATIC_SPLIT if static_split else 0))
         self.reset()
 
     def reset(self) -> None:

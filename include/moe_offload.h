@@ -121,6 +121,10 @@ typedef struct {
      * miss list; [7] launch to start (waiting for the previous layer; the
      * kernel is launched early).  Device %globaltimer. */
     double route_phase_us[8];
+    /* host side, summed over forward calls (steady clock): [0] time inside the
+     * calls, [1] of which waiting for the device's miss list, [2] of which
+     * issuing the copies and launches that follow it */
+    double host_us[3];
 } moe_stats;
 
 /* Hybrid split plan (ai-hardware-zukan "GPUに載らない分をどう間に合わせるか";
@@ -137,6 +141,15 @@ typedef struct {
 /* cache_configure flags */
 #define MOE_CACHE_RESET 1u          /* empty the cache (cold start), zero the counters */
 #define MOE_CACHE_PREFETCH_NEXT 2u  /* prefill: stream layer l+1's experts during layer l */
+/* The pages' comparison policy (ai-hardware-zukan.com, "GPUに載らない分をどう間に合わせるか":
+ * experts split over the layers statically, without looking at the routing):
+ * with R = min(k * max_rows, E) scratch slots, each layer keeps its experts
+ * 0 .. s-1 resident, s = min((num_slots - R) / L, E), in slots l*s .. l*s+s-1,
+ * copied in at the reset (before the next call's kernels); every other
+ * selected expert is a miss, copied on each use into scratch slot L*s + m (m:
+ * its rank among the batch's misses, ascending id), and nothing is evicted.
+ * Not with MOE_CACHE_PREFETCH_NEXT (MOE_ERR_ARG).  Changing the policy resets. */
+#define MOE_CACHE_STATIC_SPLIT 4u
 
 /* Bytes of one expert record; 0 if dims are invalid. */
 MOE_API size_t moe_record_bytes(const moe_dims *dims);
@@ -246,6 +259,16 @@ MOE_API moe_status plan_split(int32_t m, double B_P, double B_H, double threshol
  * back-to-back copies of chunk_bytes each (record-sized copies). */
 MOE_API moe_status moe_measure_h2d(void *dev_buf, const void *host_buf, size_t bytes, size_t chunk_bytes,
                            int32_t reps, void *stream, double *gbs);
+
+/* The same measurement with the copy done by the SMs instead of a copy engine:
+ * a kernel reads host_buf through its mapped device address with 16-byte loads
+ * and writes dev_buf (one launch per chunk).  This is the transfer rate a
+ * device-initiated miss fetch would get.  bytes, chunk_bytes and both
+ * addresses must be multiples of 16 (MOE_ERR_ARG); MOE_ERR_NOT_PINNED when
+ * host_buf has no device mapping.  No counterpart on the pages: it measures
+ * the alternative to their copy-engine transfers. */
+MOE_API moe_status moe_measure_h2d_sm(void *dev_buf, const void *host_buf, size_t bytes, size_t chunk_bytes,
+                              int32_t reps, void *stream, double *gbs);
 
 /* Router logits, softmax and top-k for T rows with no workspace (the routing
  * part of moe_layer_forward: same selection, gates and ascending id order).

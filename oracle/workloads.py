@@ -106,3 +106,29 @@ def prefill_trace(idx: np.ndarray, L: int, E: int, C: int, prefetch: bool = True
             for e, s, h, v in lru.batch(l + 1, np.arange(E, dtype=np.int32)):
                 events.append((1, l + 1, e, s, h, v))
     return events, lru
+
+
+def static_split_trace(idx: np.ndarray, L: int, E: int, C: int, scratch: int):
+    """The static per-layer split (ai-hardware-zukan.com, "GPUに載らない分をどう間に合わせるか":
+    the comparison policy that splits the expert cache over the layers without
+    looking at the routing), as the C ABI's MOE_CACHE_STATIC_SPLIT defines it:
+    s = min((C - scratch) // L, E) experts per layer are resident -- layer l's
+    experts 0 .. s-1 in slots l*s .. l*s+s-1 -- and never change; in each lookup
+    batch (the distinct experts over the rows, ascending) an expert e < s is a
+    hit in slot l*s + e, any other is the m-th miss of the batch and goes to
+    scratch slot L*s + m; nothing is evicted.
+
+    idx: [T, L, rows, k].  Returns events [(t, layer, expert, slot, hit, evicted)]."""
+    s = min((C - scratch) // L, E)
+    events = []
+    for t in range(idx.shape[0]):
+        for l in range(L):
+            m = 0
+            for e in np.unique(idx[t, l].ravel()):
+                e = int(e)
+                if e < s:
+                    events.append((t, l, e, l * s + e, 1, -1))
+                else:
+                    events.append((t, l, e, L * s + m, 0, -1))
+                    m += 1
+    return events

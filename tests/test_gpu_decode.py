@@ -211,3 +211,60 @@ def test_h2d_measurement():
     with pytest.raises(abi.MoeError) as ei:
         abi.moe_measure_h2d(d, np.zeros(16, np.uint8), 16, 0, 1, s)
     assert ei.value.status == abi.MOE_ERR_NOT_PINNED
+
+
+def test_h2d_sm_measurement_copies_the_bytes():
+    n = 64 << 20
+    h = torch.randint(0, 256, (n,), dtype=torch.uint8).pin_memory()
+    d = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    gbs = abi.moe_measure_h2d_sm(d, h, n, 0, 1, s)
+    s.synchronize()
+    assert torch.equal(d.cpu(), h)
+    d.zero_()
+    torch.cuda.synchronize()
+    gbs_rec = abi.moe_measure_h2d_sm(d, h, n - 4096, synth.record_bytes(2048, 768), 1, s)
+    s.synchronize()
+    assert torch.equal(d[:n - 4096].cpu(), h[:n - 4096]) and int(d[n - 4096:].sum()) == 0
+    assert 1.0 < gbs < 200.0 and 1.0 < gbs_rec < 200.0
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_measure_h2d_sm(d, h, 24, 0, 1, s)  # not a multiple of 16
+    assert ei.value.status == abi.MOE_ERR_ARG
+
+
+@pytest.mark.parametrize("S", [1, 5])
+def test_static_split_policy_trace_and_outputs(S):
+    """The static per-layer split: fixed resident experts per layer, misses into
+    scratch slots; events bit-exact against the oracle's simulator, the resident
+    slots hold their records, outputs within the bar."""
+    from oracle.workloads import static_split_trace
+    from expert_offload_caching_b200.runtime import LayerStack
+    R = min(S * MID.k, MID.E)
+    C = 3 * MID.L + R + 2  # 3 resident experts per layer (2 slots left over)
+    pb = DecodeProblem(MID, T=6, streams=S, C=C, stream0=200)
+    st = LayerStack(pb.dims(), pb.pool, sp.to_device(pb.Wr), sp.to_device(pb.shared), C,
+                    static_split=True)
+    run = pb.run(stack=st, routing=True)
+    idx, gates = pb.oracle_routing()
+    np.testing.assert_array_equal(run.idx, idx)
+    assert run.events == static_split_trace(idx, MID.L, MID.E, C, R)
+    m, o = run.table[0], run.table[1]
+    for l in range(MID.L):
+        for e in range(MID.E):
+            assert m[l * MID.E + e] == (l * 3 + e if e < 3 else -1)
+    assert all(o[s] == (s // 3) * MID.E + s % 3 for s in range(3 * MID.L))
+    assert all(o[s] == -1 for s in range(3 * MID.L, C))
+    pb.check_slots(st, o)
+    y = run.y.cpu().numpy()
+    for t in range(pb.T):
+        for l in range(MID.L):
+            assert rel_l2(y[t, l], pb.oracle_y(t, l)) <= REL_L2_MAX
+    hits = sum(ev[4] for ev in run.events)
+    assert run.stats.hits == hits and run.stats.misses == len(run.events) - hits > 0
+    assert run.stats.evictions == 0
+    with pytest.raises(abi.MoeError) as ei:  # no next-layer prefetch with the static split
+        abi.cache_configure(st.ctx, C, st.arena, st.arena.numel(),
+                            abi.MOE_CACHE_RESET | abi.MOE_CACHE_STATIC_SPLIT | abi.MOE_CACHE_PREFETCH_NEXT)
+    assert ei.value.status == abi.MOE_ERR_ARG
+    st.close()

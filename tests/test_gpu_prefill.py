@@ -147,3 +147,23 @@ def test_prefill_full_chunk_qwen_shaped_two_layers():
     events, idx, gates, y = pb.run(st)
     rows = np.random.default_rng(3).choice(4096, 24, replace=False)
     _check(pb, st, events, idx, gates, y, True, rows=np.sort(rows))
+
+
+def test_prefill_static_split_policy():
+    """A prefill chunk under the static per-layer split (no prefetch): routed
+    misses into scratch slots, events bit-exact, outputs within the bar."""
+    from oracle.workloads import static_split_trace
+    T, R = 200, PF.E  # the largest batch: every expert of a layer
+    C = 10 * PF.L + R
+    pb = PrefillProblem(PF, T=T, C=C)
+    sh = PF
+    dims = abi.make_dims(sh.L, sh.E, sh.k, sh.d, sh.F, sh.shared, True, T, 0)
+    st = LayerStack(dims, pb.pool, sp.to_device(pb.Wr), sp.to_device(pb.shared), C, static_split=True)
+    events, idx, gates, y = pb.run(st)
+    want_idx = np.stack([oracle.route(pb.Wr[l], pb.x[l], sh.k)[0] for l in range(sh.L)])
+    np.testing.assert_array_equal(idx, want_idx)
+    want = static_split_trace(want_idx[None], sh.L, sh.E, C, R)
+    assert events == want
+    for l in range(sh.L):
+        assert rel_l2(y[l], pb.oracle_y(l, np.arange(T))) <= REL_L2_MAX
+    st.close()

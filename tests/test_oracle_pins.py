@@ -257,6 +257,40 @@ def test_lru_hand_trace():
     assert (misses, hits) == (7, 5)
 
 
+def test_static_split_hand_trace():
+    """The static per-layer split against the hand-worked trace (golden)."""
+    from oracle.workloads import static_split_trace
+    rows = _rows("static_split_hand_trace.txt")
+    idx = np.zeros((2, 2, 2, 2), dtype=np.int32)
+    want = []
+    for r in rows:
+        t, l = int(r[0]), int(r[1])
+        idx[t, l] = [[int(v) for v in row.split(",")] for row in r[2].split("|")]
+        want += [(t, l) + tuple(int(v) for v in ev.split(":")) + (-1,) for ev in r[4:]]
+    assert static_split_trace(idx, 2, 8, 8, 4) == want
+
+
+def test_static_split_miss_rate_closed_form():
+    """Every expert of every layer used once per step: the hits are exactly the s
+    resident experts per layer, so the miss rate is 1 - s/E; no slot outside
+    [0, C) and no resident slot is ever given to a miss."""
+    from oracle.workloads import static_split_trace
+    L, E, C, R = 3, 40, 50, 10
+    s = (C - R) // L  # 13
+    idx = np.tile(np.arange(E, dtype=np.int32), (2, L, 1, 1))  # [T=2, L, rows=1, k=E]
+    ev = static_split_trace(idx, L, E, C, R + E)  # scratch for a whole-E batch
+    s2 = min((C - (R + E)) // L, E)
+    assert s2 == 0 and all(h == 0 for *_, h, _v in ev)
+    ev = static_split_trace(idx, L, E, C + E, R + E)
+    s3 = (C + E - R - E) // L
+    assert s3 == s
+    hits = sum(e[4] for e in ev)
+    assert hits == 2 * L * s and len(ev) == 2 * L * E
+    assert all(0 <= e[3] < C + E for e in ev)
+    assert all(e[3] >= L * s for e in ev if not e[4])
+    assert abs((1 - hits / len(ev)) - (1 - s / E)) < 1e-12
+
+
 class _DictLRU:
     """Brute-force LRU for the cross-check: an ordered dict of resident keys."""
 
