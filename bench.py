@@ -209,7 +209,9 @@ def timed(stack, x, y, L, world, host=False):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stack.compute)
+    torch.cuda.nvtx.range_push("timed")  # lets a profiler select the timed region's launches
     run_tokens(stack, x, y, L, host)
+    torch.cuda.nvtx.range_pop()
     e1.record(stack.compute)
     torch.cuda.synchronize()
     barrier(world)
@@ -563,7 +565,9 @@ def bench_prefill(args, shape, rank, world, local):
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stack.compute)
+            torch.cuda.nvtx.range_push("timed")
             run_chunk(stack, xs, ys, L, host)
+            torch.cuda.nvtx.range_pop()
             e1.record(stack.compute)
             torch.cuda.synchronize()
             total += e0.elapsed_time(e1) * 1e-3

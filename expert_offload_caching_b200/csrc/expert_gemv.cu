@@ -77,8 +77,9 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 }
 
 constexpr int kMaxSteps = 16;  // K <= 4096: at most 16 K-steps of 256, one per warp
-constexpr int kMaxJobsPerCta = 32;
-constexpr int kCtaTarget = 8 * 148;  // CTAs per launch the expert grouping aims for
+constexpr int kGStages = 3;                           // tiles in flight per CTA
+constexpr int kMaxSlots = kMaxK * kDecodeMaxRows + 1;  // job slots of a launch (+ shared)
+constexpr int kSmCount = 148;
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
@@ -139,29 +140,32 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
     }
 }
 
-// One CTA per (16-row weight tile, group of up to jobs_per_cta experts): the CTA
-// walks its experts in ascending id (the shared expert last), staging expert
-// i + 1's tile into the second shared-memory buffer (16-byte cp.async copies,
-// the whole tile in flight) while it computes expert i.  Each warp owns spw
-// consecutive K-steps of 256 elements; warp 0 sums the warps' partials in a
-// fixed order.  Dynamic shared memory: 2 x (16*K/2 code bytes + K scale
-// bytes) + the partials (warps x NG x 512 bytes).
+// Persistent schedule: the launch's work items are (expert, 16-row weight
+// tile) pairs -- the valid experts of the launch in ascending id (hit jobs, or
+// the one job only_job), then the shared expert -- numbered expert-major; CTA b
+// takes items b, b + G, b + 2G, ... (G = gridDim.x, a few CTAs per SM).  Each
+// CTA streams its items through a kGStages-deep ring of shared-memory buffers
+// (16-byte cp.async copies of the whole tile, one group per item), so the
+// loads of the next items are in flight while it computes the current one.
+// Each warp owns spw consecutive K-steps of 256 elements; warp 0 sums the
+// warps' partials in a fixed order.  Dynamic shared memory: kGStages x (16*K/2
+// code bytes + K scale bytes) + the partials (warps x NG x 512 bytes).
 //
 // Launched with programmatic stream serialization: gate/up waits for the
 // route kernel before reading anything (job list, activations); the down
 // projection reads the job list (complete, two launches back), stages its
-// first W2 tile, and only then waits for gate/up's h.  Every CTA executes the
+// first W2 tiles, and only then waits for gate/up's h.  Every CTA executes the
 // wait, so a launch completes only after its predecessor.
 //
-// Combine (down launches with a.combine): the CTA that finishes a tile last
-// (per-tile ticket; the only CTA when the launch has one group) sums that
+// Combine (down launches with a.combine): the CTA that completes the last
+// expert of a tile (per-tile ticket counting the launch's experts) sums that
 // tile's 16 output rows over the layer's experts in ascending id, plus the
 // shared expert, for every row t.
 template <int NG>
 __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_job[kMaxJobsPerCta];  // job index, or -1: the shared expert
-    __shared__ int s_n, s_last;
+    __shared__ int s_valid[kMaxSlots];  // job index per valid expert, -1: the shared expert
+    __shared__ int s_nvalid, s_last;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, q = lane & 3;
     const bool gate_up = a.mode == kGateUp;
@@ -169,80 +173,89 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
     if (gate_up) pdl_wait();  // job list and x come from the previous launch
     pdl_launch_dependents();
 
-    // ---- this CTA's experts: launch slots [y*J, y*J + J) -- hit jobs, and the
-    // shared expert at slot shared_slot -- or the one job only_job.  L2 reads
-    // (ld.global.cg): the down launch reads the job list before its PDL wait,
-    // and an SM's L1 may still hold lines of an older launch.
+    // ---- the launch's valid experts.  L2 reads (ld.global.cg): the down launch
+    // reads the job list before its PDL wait, and an SM's L1 may still hold
+    // lines of an older launch.
     if (warp == 0) {
-        int mine = -2;
+        int cnt = 0;
         if (a.only_job >= 0) {
-            if (lane == 0 && blockIdx.y == 0) mine = a.only_job;
-        } else if (lane < a.jobs_per_cta) {
-            const int slot = (int)blockIdx.y * a.jobs_per_cta + lane;
-            if (slot == a.shared_slot) mine = -1;
-            else if (slot < __ldcg(a.n_jobs) && __ldcg(&a.jobs[slot].hit)) mine = slot;
+            if (lane == 0) s_valid[0] = a.only_job;
+            cnt = 1;
+        } else {
+            const int nj = __ldcg(a.n_jobs);
+            for (int b = 0; b < a.slots; b += 32) {
+                const int slot = b + lane;
+                int v = -2;
+                if (slot < a.slots) {
+                    if (slot == a.shared_slot) v = -1;
+                    else if (slot < nj && __ldcg(&a.jobs[slot].hit)) v = slot;
+                }
+                const unsigned ball = __ballot_sync(0xffffffffu, v != -2);
+                if (v != -2) s_valid[cnt + __popc(ball & ((1u << lane) - 1u))] = v;
+                cnt += __popc(ball);
+            }
         }
-        const unsigned ball = __ballot_sync(0xffffffffu, mine != -2);
-        if (mine != -2) s_job[__popc(ball & ((1u << lane) - 1u))] = mine;
-        if (lane == 0) s_n = __popc(ball);
+        if (lane == 0) s_nvalid = cnt;
     }
     __syncthreads();
-    const int njobs = s_n;
+    const int nvalid = s_nvalid;
 
     const int K = gate_up ? a.d : a.F;
-    const int tile = blockIdx.x;
+    const int tiles = gate_up ? (a.F >> 3) : (a.d >> 4);
+    const int nitems = nvalid * tiles;
+    const int G = (int)gridDim.x;
+    const int n_my = (int)blockIdx.x < nitems ? (nitems - 1 - (int)blockIdx.x) / G + 1 : 0;
     const int NCH = K >> 6;
     const int nwarps = (int)(blockDim.x >> 5);
     const int nsteps = (NCH + 3) >> 2;
     const int spw = (nsteps + nwarps - 1) / nwarps;
     const uint32_t code_bytes = 16u * (uint32_t)(K >> 1), scale_bytes = (uint32_t)K;
     const uint32_t buf_bytes = code_bytes + scale_bytes;
-    const int nbuf = a.jobs_per_cta > 1 ? 2 : 1;  // a second buffer only when the CTA has several experts
-    float(*red)[NG][4][32] = reinterpret_cast<float(*)[NG][4][32]>(smem + nbuf * buf_bytes);
+    float(*red)[NG][4][32] = reinterpret_cast<float(*)[NG][4][32]>(smem + kGStages * buf_bytes);
 
     auto record = [&](int jid) -> const uint8_t * {
         return jid < 0 ? a.shared_rec : a.arena + (int64_t)__ldcg(&a.jobs[jid].slot) * a.rec_bytes;
     };
-    // stage expert i of the list into buffer i & 1 (one cp.async group)
-    auto stage = [&](int i) {
-        const uint8_t *rec = record(s_job[i]);
-        uint8_t *dst = smem + (i & (nbuf - 1)) * buf_bytes;
-        const uint8_t *codes = rec + (gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)tile * code_bytes;
-        const uint8_t *scales = rec + (gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)tile * scale_bytes;
-        for (uint32_t o = threadIdx.x; o < (code_bytes >> 4); o += blockDim.x) cp_async16(dst + 16 * o, codes + 16 * o);
-        for (uint32_t o = threadIdx.x; o < (scale_bytes >> 4); o += blockDim.x)
-            cp_async16(dst + code_bytes + 16 * o, scales + 16 * o);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        if (gate_up) {  // this expert's down projection -> L2 for the down launch (a 1/tiles slice)
-            const uint32_t total = (uint32_t)(a.lay.bytes - a.lay.w2_codes);
-            const uint32_t per = ((total / gridDim.x) + 127u) & ~127u;
-            const uint32_t off = per * blockIdx.x;
-            if (off < total) prefetch_l2_range(rec + a.lay.w2_codes + off, per < total - off ? per : total - off);
+    // stage this CTA's j-th item into buffer j % kGStages; always one cp.async group
+    auto stage = [&](int j) {
+        if (j < n_my) {
+            const int item = (int)blockIdx.x + j * G;
+            const int jid = s_valid[item / tiles], tile = item - (item / tiles) * tiles;
+            const uint8_t *rec = record(jid);
+            uint8_t *dst = smem + (j % kGStages) * buf_bytes;
+            const uint8_t *codes = rec + (gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)tile * code_bytes;
+            const uint8_t *scales =
+                rec + (gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)tile * scale_bytes;
+            for (uint32_t o = threadIdx.x; o < (code_bytes >> 4); o += blockDim.x)
+                cp_async16(dst + 16 * o, codes + 16 * o);
+            for (uint32_t o = threadIdx.x; o < (scale_bytes >> 4); o += blockDim.x)
+                cp_async16(dst + code_bytes + 16 * o, scales + 16 * o);
+            if (gate_up) {  // this expert's down projection -> L2 for the down launch (a 1/tiles slice)
+                const uint32_t total = (uint32_t)(a.lay.bytes - a.lay.w2_codes);
+                const uint32_t per = ((total / tiles) + 127u) & ~127u;
+                const uint32_t off = per * tile;
+                if (off < total)
+                    prefetch_l2_range(rec + a.lay.w2_codes + off, per < total - off ? per : total - off);
+            }
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
-    if (!gate_up) {
-        if (njobs > 0) stage(0);  // W2 does not depend on the gate/up launch
-        pdl_wait();               // h does
-    } else if (njobs > 0) {
-        stage(0);
-    }
+    for (int j = 0; j < kGStages - 1; ++j) stage(j);
+    if (!gate_up) pdl_wait();  // h comes from the gate/up launch; W2 tiles already in flight
     // tile-local rows of this thread: gate_up 2g (gate) / 2g+1 (up); down g / g+8
     const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
-    for (int i = 0; i < njobs; ++i) {
-        if (i + 1 < njobs) {
-            stage(i + 1);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
+    for (int j = 0; j < n_my; ++j) {
+        stage(j + kGStages - 1);
+        asm volatile("cp.async.wait_group %0;" ::"n"(kGStages - 1) : "memory");
         __syncthreads();
-        const int jid = s_job[i];
+        const int item = (int)blockIdx.x + j * G;
+        const int jid = s_valid[item / tiles], tile = item - (item / tiles) * tiles;
         const bool shared = jid < 0;
         const uint8_t *rec = record(jid);
         const int nrows = shared ? a.T : __ldcg(&a.jobs[jid].nrows);
         const int row_off = shared ? 0 : __ldcg(&a.jobs[jid].row_off);
-        const uint8_t *s_codes = smem + (i & (nbuf - 1)) * buf_bytes, *s_scales = s_codes + code_bytes;
+        const uint8_t *s_codes = smem + (j % kGStages) * buf_bytes, *s_scales = s_codes + code_bytes;
         const float *ts = reinterpret_cast<const float *>(rec + a.lay.tscales);
         for (int r0 = 0; r0 < nrows; r0 += 4 * NG) {
             // mma column n = g carries activation row r0 + 4*grp + g/2, the hi (g
@@ -268,7 +281,7 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
 #pragma unroll
             for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[grp][j] = 0.f;
+                for (int i = 0; i < 4; ++i) acc[grp][i] = 0.f;
             for (int st = 0; st < spw; ++st) {  // this warp's K-steps (uniform across the warp)
                 const int c = 4 * (warp * spw + st) + q;
                 const bool cv = c < NCH;  // ragged K tail: some lanes of the quad feed zeros
@@ -282,14 +295,14 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
 #pragma unroll
             for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) red[warp][grp][j][lane] = acc[grp][j];
+                for (int i = 0; i < 4; ++i) red[warp][grp][i][lane] = acc[grp][i];
             __syncthreads();
             if (warp == 0) {
                 for (int w = 1; w < nwarps; ++w)
 #pragma unroll
                     for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) acc[grp][j] += red[w][grp][j][lane];
+                        for (int i = 0; i < 4; ++i) acc[grp][i] += red[w][grp][i][lane];
 #pragma unroll
                 for (int grp = 0; grp < NG; ++grp) {
                     const int r = r0 + 4 * grp + q;  // this thread's results: activation row q
@@ -303,11 +316,11 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
                     if (gate_up) {
                         const float gt = ts[0] * v0, up = ts[1] * v1;
                         const float h = gt / (1.0f + expf(-gt)) * up;
-                        const int j = 8 * tile + g;
+                        const int o = 8 * tile + g;
                         const __half hi = __float2half_rn(h);
                         const __half lo = __float2half_rn(h - __half2float(hi));
-                        a.hh_out[sel * 2 * a.F + j] = hi;
-                        a.hh_out[sel * 2 * a.F + a.F + j] = lo;
+                        a.hh_out[sel * 2 * a.F + o] = hi;
+                        a.hh_out[sel * 2 * a.F + a.F + o] = lo;
                     } else {
                         const int o = 16 * tile + g;
                         a.part_out[sel * a.d + o] = ts[2] * v0;
@@ -317,47 +330,58 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
             }
             __syncthreads();  // red reused; after the last row group, the buffer is free
         }
-    }
 
-    if (a.combine && !gate_up) {
-        __syncthreads();
-        bool last = true;
-        if (gridDim.y > 1) {
+        if (a.combine && !gate_up) {  // the tile's last expert: combine its rows
             if (threadIdx.x == 0) {
                 __threadfence();
-                s_last = atomicAdd(&a.tile_ticket[tile], 1u) == gridDim.y - 1;
+                s_last = atomicAdd(&a.tile_ticket[tile], 1u) == (unsigned)(nvalid - 1);
             }
             __syncthreads();
-            last = s_last;
-            if (last) __threadfence();
-        }
-        if (last) {
-            if (a.combine == 1 || __ldcg(a.n_misses) == 0) {
-                for (int e = threadIdx.x; e < 16 * a.T; e += blockDim.x) {
-                    const int t = e >> 4, o = 16 * tile + (e & 15);
-                    const float *pr = a.part_out + (size_t)t * (a.k + 1) * a.d + o;
-                    float sum = 0.f;
-                    for (int p = 0; p < a.k; ++p) sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
-                    if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
-                    a.y[(size_t)t * a.d + o] = sum;
+            if (s_last) {
+                __threadfence();
+                if (a.combine == 1 || __ldcg(a.n_misses) == 0) {
+                    for (int e = threadIdx.x; e < 16 * a.T; e += blockDim.x) {
+                        const int t = e >> 4, o = 16 * tile + (e & 15);
+                        const float *pr = a.part_out + (size_t)t * (a.k + 1) * a.d + o;
+                        float sum = 0.f;
+                        for (int p = 0; p < a.k; ++p)
+                            sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                        if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
+                        a.y[(size_t)t * a.d + o] = sum;
+                    }
                 }
+                if (threadIdx.x == 0) a.tile_ticket[tile] = 0u;
             }
-            if (gridDim.y > 1 && threadIdx.x == 0) a.tile_ticket[tile] = 0u;
+            __syncthreads();
         }
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");  // no copy outlives the CTA
 }
 
 template <int NG>
-cudaError_t launch_ng(const GemvArgs &a, dim3 grid, int threads, size_t smem, cudaStream_t s) {
+cudaError_t launch_ng(const GemvArgs &a, int tiles, int threads, size_t smem, cudaStream_t s) {
     static bool configured = false;  // per instantiation: allow > 48 KB of dynamic smem
+    static int sms = 0;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<NG>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+        if (e != cudaSuccess) return e;
+        int dev = 0;
+        e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         configured = true;
     }
+    // persistent grid: as many CTAs as fit at once (at most 4 per SM), no more than the items
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_gemv_kernel<NG>, threads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    if (per_sm > 4) per_sm = 4;
+    int grid = sms * per_sm;
+    if (grid > a.slots * tiles) grid = a.slots * tiles;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
+    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -376,27 +400,17 @@ cudaError_t launch_gemv(const GemvArgs &a_in, int slots, cudaStream_t s) {
     const int K = a.mode == kGateUp ? a.d : a.F;
     const int tiles = a.mode == kGateUp ? a.F / 8 : a.d / 16;
     const int nsteps = (K / 64 + 3) / 4;
-    if (nsteps < 1 || nsteps > kMaxSteps || slots < 1) return cudaErrorInvalidValue;
+    if (nsteps < 1 || nsteps > kMaxSteps || slots < 1 || slots > kMaxSlots || tiles > kMaxTiles)
+        return cudaErrorInvalidValue;
+    a.slots = a.only_job >= 0 ? 1 : slots;
     const int spw = nsteps >= 8 ? 2 : 1;  // 2 K-steps per warp for long rows: smaller CTAs, more per SM
     const int warps = (nsteps + spw - 1) / spw;
-    // expert groups per tile: about kCtaTarget CTAs (several per SM, so staging
-    // latencies overlap across CTAs), at most 32 experts per CTA
-    int gy = 1;
-    if (a.only_job < 0) {
-        gy = (kCtaTarget + tiles - 1) / tiles;
-        if (gy > slots) gy = slots;
-        if ((slots + gy - 1) / gy > kMaxJobsPerCta) gy = (slots + kMaxJobsPerCta - 1) / kMaxJobsPerCta;
-        a.jobs_per_cta = (slots + gy - 1) / gy;
-    } else {
-        a.jobs_per_cta = 1;
-    }
-    const dim3 grid(tiles, gy);
     const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
-    const size_t buf = 16 * (size_t)(K / 2) + (size_t)K;  // one expert's tile: codes + scales
-    const size_t smem = (a.jobs_per_cta > 1 ? 2 : 1) * buf + (size_t)warps * ng * 4 * 32 * sizeof(float);
-    if (smem > 96 * 1024) return cudaErrorInvalidValue;
-    if (ng == 1) return launch_ng<1>(a, grid, warps * 32, smem, s);
-    return launch_ng<2>(a, grid, warps * 32, smem, s);
+    const size_t buf = 16 * (size_t)(K / 2) + (size_t)K;  // one tile: codes + scales
+    const size_t smem = kGStages * buf + (size_t)warps * ng * 4 * 32 * sizeof(float);
+    if (smem > 160 * 1024) return cudaErrorInvalidValue;
+    if (ng == 1) return launch_ng<1>(a, tiles, warps * 32, smem, s);
+    return launch_ng<2>(a, tiles, warps * 32, smem, s);
 }
 
 }  // namespace moe

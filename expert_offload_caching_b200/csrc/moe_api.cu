@@ -475,7 +475,13 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     CK(cudaMemsetAsync(ctx->dws.cnt, 0, (size_t)D.E * 4, ctx->cs));
     TimedLaunch tr;
     time_begin(ctx, tr, MOE_K_PREFILL_ROUTE);
-    CK(launch_prefill_route(ra, ctx->cs));
+    CUtensorMap tm_x;  // logits on the tensor cores when x's rows can be TMA boxes
+    if (make_operand_map(&tm_x, x, 2 * (int64_t)D.d, T, 0, 0)) {
+        CK(launch_router_gemm(tm_x, ctx->maps.router, ctx->dws.z, T, D.E, D.d, layer, ctx->page_d, ctx->cs));
+        CK(launch_prefill_select(ra, ctx->cs));
+    } else {
+        CK(launch_prefill_route(ra, ctx->cs));
+    }
     time_end(ctx, tr, (double)D.E * D.d * 2 + (double)T * D.d * 2);
     CK(launch_prefill_scatter(ra, ctx->cs));
     CK(launch_tile_plan(ctx->dws.jobs, ctx->dws.n_jobs, T, D.has_shared, ctx->dws.pairs, ctx->dws.n_pairs,
@@ -704,7 +710,9 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
         ctx->dws.n_pairs = reinterpret_cast<int32_t *>(w + L.n_pairs);
         const int64_t R = (int64_t)dims->max_rows * (dims->k + 1);
         bool ok = make_operand_map(&ctx->maps.xq, ctx->dws.xq, dims->d / 2, R, 0, 0) &&
-                  make_operand_map(&ctx->maps.hq, ctx->dws.hq, dims->F / 2, R, 0, 0);
+                  make_operand_map(&ctx->maps.hq, ctx->dws.hq, dims->F / 2, R, 0, 0) &&
+                  make_operand_map(&ctx->maps.router, router_w, 2 * (int64_t)dims->d, dims->E, dims->L,
+                                   2 * (int64_t)dims->E * dims->d);
         if (ok && dims->has_shared) {
             ok = make_operand_map(&ctx->maps.w13_shared, ctx->shared_recs + lay.w13_codes, dims->d / 2,
                                   2 * dims->F, dims->L, lay.bytes) &&
@@ -753,14 +761,14 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
 moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, size_t arena_bytes,
                            uint32_t flags) {
     if (!ctx || !slot_arena || num_slots <= 0) return MOE_ERR_ARG;
+    const bool stat = (flags & MOE_CACHE_STATIC_SPLIT) != 0;
+    if (stat && (flags & MOE_CACHE_PREFETCH_NEXT)) return MOE_ERR_ARG;
     const moe_dims &D = ctx->dims;
     const int64_t need = max_jobs(&D, D.max_rows);
     if (num_slots < need) return MOE_ERR_CAPACITY;
     if ((flags & MOE_CACHE_PREFETCH_NEXT) && num_slots < 2ll * D.E) return MOE_ERR_CAPACITY;
     if (num_slots > 65536) return MOE_ERR_UNSUPPORTED;
     if (arena_bytes < moe_arena_bytes(&D, num_slots)) return MOE_ERR_ARG;
-    const bool stat = (flags & MOE_CACHE_STATIC_SPLIT) != 0;
-    if (stat && (flags & MOE_CACHE_PREFETCH_NEXT)) return MOE_ERR_ARG;
     const bool reset = (flags & MOE_CACHE_RESET) || !ctx->configured || ctx->arena != slot_arena ||
                        ctx->C != num_slots || ((ctx->flags ^ flags) & MOE_CACHE_STATIC_SPLIT);
     // static split: the resident experts per layer, after `need` scratch slots

@@ -118,7 +118,7 @@ struct GemvArgs {
     const int32_t *n_jobs;
     const RowRef *rowrefs;
     int only_job;          // >= 0: process just this job; -1: every hit job (+ shared)
-    int jobs_per_cta;      // job slots per CTA (set by launch_gemv)
+    int slots;             // job slots of the launch, shared expert included (set by launch_gemv)
     int shared_slot;       // gridDim.y index of the shared job, -1 if none
     const uint8_t *arena;
     int64_t rec_bytes;
@@ -166,6 +166,7 @@ struct GroupedGemmArgs {
 // activation codes (2D: byte, row).
 struct GroupedGemmMaps {
     CUtensorMap w13, w2, w13_shared, w2_shared, xq, hq;
+    CUtensorMap router;  // router weights (3D: byte, expert row, layer) for the logits GEMM
 };
 
 // launchers (one per .cu)
@@ -176,6 +177,7 @@ cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
 cudaError_t launch_table_static(Table t, int L, int E, int per_layer, cudaStream_t s);
 cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_select(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
                            int has_shared, cudaStream_t s);
 cudaError_t launch_quant_x_grouped(const __nv_bfloat16 *x, int T, int k, int d, int has_shared,
@@ -188,6 +190,8 @@ cudaError_t launch_tile_plan(const Job *jobs, const int32_t *n_jobs, int T, int 
                              int32_t *n_pairs, cudaStream_t s);
 cudaError_t launch_grouped_gemm(const GroupedGemmMaps &maps, const GroupedGemmArgs &a, int pairs_cap,
                                 cudaStream_t s);
+cudaError_t launch_router_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, float *z, int T, int E, int d,
+                               int layer, HostPage *page, cudaStream_t s);
 bool make_operand_map(CUtensorMap *out, const void *base, int64_t row_bytes, int64_t rows, int64_t count,
                       int64_t matrix_stride);
 

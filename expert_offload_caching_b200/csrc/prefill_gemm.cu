@@ -463,7 +463,164 @@ __global__ void __launch_bounds__(1024) tile_plan_kernel(const Job *jobs, const 
     if (j == 0) *n_pairs = s_total + nsh;
 }
 
+// ---- router logits of a prefill chunk: z = x W_r^T on the tensor cores
+// (tcgen05.mma kind::f16, bf16 x bf16 -> fp32 in tensor memory).  One CTA per
+// 128 rows x 128 experts; K (d) streamed through a 4-deep ring of TMA boxes
+// (128 bytes = 64 bf16 of K, 128-byte swizzle; 4 MMAs of K = 16 per box).
+// The products are exact in fp32; only the summation order differs from an
+// fp32 FMA chain.
+constexpr int kRStages = 4;
+constexpr uint32_t kROffBar = 2 * kRStages * kTileBytes;
+constexpr uint32_t kRSmemBytes = kROffBar + 128 + 1024;
+
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t"
+        "}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+        : "memory");
+}
+// Instruction descriptor: bf16 x bf16 -> fp32, K-major A and B, M = 128, N.
+__device__ __forceinline__ uint32_t idesc_bf16(int N) {
+    return (1u << 4)                          // D format fp32
+           | (1u << 7)                        // A format bf16
+           | (1u << 10)                       // B format bf16
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(kBM >> 4) << 24);    // M / 16
+}
+
+__device__ void router_fail(HostPage *page, int code, int stage) {
+    page->diag[1] = 20;
+    page->diag[2] = (int)(blockIdx.x + 1000 * blockIdx.y);
+    page->diag[3] = stage;
+    page->diag[4] = (int)threadIdx.x;
+    __threadfence_system();
+    page->error = code;
+    __threadfence_system();
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                       float *z, int T, int E, int d, int layer, HostPage *page) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kBM, e0 = blockIdx.y * kBM;
+    const int nkb = (2 * d + kStageKBytes - 1) / kStageKBytes;
+    extern __shared__ uint8_t dsm_raw[];
+    const uint32_t raw = saddr(dsm_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *sm = dsm_raw + (base - raw);
+    const uint32_t bar_full = base + kROffBar, bar_empty = bar_full + 8 * kRStages,
+                   bar_done = bar_empty + 8 * kRStages;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sm + kROffBar + 8 * (2 * kRStages + 1));
+    volatile int32_t *s_fail = reinterpret_cast<volatile int32_t *>(sm + kROffBar + 8 * (2 * kRStages + 1) + 4);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_done, 1);
+        *s_fail = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc(base + kROffBar + 8 * (2 * kRStages + 1), 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {  // TMA producer
+            int it = 0;
+            for (; it < nkb; ++it) {
+                const int s = it % kRStages, r = it / kRStages;
+                if (r > 0 && !mbar_wait(bar_empty + 8 * s, (r - 1) & 1)) {
+                    router_fail(page, 51, it);
+                    *s_fail = 1;
+                    break;
+                }
+                mbar_arrive_tx(bar_full + 8 * s, 2 * kTileBytes);
+                tma_load_2d(base + s * kTileBytes, &tm_x, bar_full + 8 * s, it * kStageKBytes, t0);
+                tma_load_3d(base + (kRStages + s) * kTileBytes, &tm_w, bar_full + 8 * s, it * kStageKBytes, e0,
+                            layer);
+            }
+            if (it < nkb)  // let the stages already issued land before the CTA exits
+                for (int j = it - 1; j >= 0 && j >= it - kRStages; --j)
+                    mbar_wait(bar_full + 8 * (j % kRStages), (j / kRStages) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {  // MMA issue
+            const uint32_t idesc = idesc_bf16(kBM);
+            for (int it = 0; it < nkb; ++it) {
+                const int s = it % kRStages, r = it / kRStages;
+                if (!mbar_wait(bar_full + 8 * s, r & 1)) {
+                    router_fail(page, 52, it);
+                    *s_fail = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t da = base + s * kTileBytes, db = base + (kRStages + s) * kTileBytes;
+                const int steps = min(4, (2 * d - it * kStageKBytes) / 32);  // K = 16 bf16 = 32 bytes each
+                for (int i = 0; i < steps; ++i)
+                    tc_mma_bf16(tmem, desc_sw128(da + 32 * i), desc_sw128(db + 32 * i), idesc, (it | i) != 0);
+                tc_commit(bar_empty + 8 * s);
+            }
+            tc_commit(bar_done);
+        }
+        __syncwarp();
+    } else {  // epilogue: lane = row of x, columns = experts
+        bool ok = mbar_wait(bar_done, 0);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && lane == 0) { router_fail(page, 53, nkb); *s_fail = 1; }
+        tc_fence_after();
+        if (ok && !*s_fail) {
+            const int q = warp & 3;
+            const int t = t0 + q * 32 + lane;
+            const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+            for (int c0 = 0; c0 < kBM && e0 + c0 < E; c0 += 16) {
+                float v[16];
+                tmem_ld16(trow + (uint32_t)c0, v);
+                if (t < T) {
+                    float *zr = z + (size_t)t * E + e0 + c0;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (e0 + c0 + i < E) zr[i] = v[i];
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_router_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, float *z, int T, int E, int d,
+                               int layer, HostPage *page, cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kRSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const dim3 grid((T + kBM - 1) / kBM, (E + kBM - 1) / kBM);
+    router_gemm_kernel<<<grid, kGemmThreads, kRSmemBytes, s>>>(tm_x, tm_w, z, T, E, d, layer, page);
+    return cudaGetLastError();
+}
+
+
 
 int grouped_pairs_cap(int n_jobs, int T, int k, int has_shared) {
     return n_jobs + (T * k + kBN - 1) / kBN + (has_shared ? (T + kBN - 1) / kBN : 0);

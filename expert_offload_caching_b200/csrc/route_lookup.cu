@@ -783,6 +783,16 @@ cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
+// Prefill selection on logits already in ws.z: top-k + counts, then the
+// lookup CTA.  The caller zeroes ws.cnt first.
+cudaError_t launch_prefill_select(const RouteArgs &a, cudaStream_t s) {
+    prefill_topk_kernel<<<(a.T + kRouteThreads / 32 - 1) / (kRouteThreads / 32), kRouteThreads, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    prefill_lookup_kernel<<<1, kRouteThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 // Prefill routing: logits, top-k + counts, then the lookup CTA (which
 // publishes the miss and prefetch lists).  The caller zeroes ws.cnt first.
 cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s) {
