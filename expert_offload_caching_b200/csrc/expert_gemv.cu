@@ -78,6 +78,7 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 constexpr int kMaxSteps = 16;  // K <= 4096: at most 16 K-steps of 256, one per warp
 constexpr int kGStages = 3;                           // tiles in flight per CTA
+constexpr int kMaxGemvWarps = 12;                     // two CTAs of up to 12 warps per SM
 constexpr int kMaxSlots = kMaxK * kDecodeMaxRows + 1;  // job slots of a launch (+ shared)
 constexpr int kSmCount = 148;
 
@@ -162,7 +163,7 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
 // tile's 16 output rows over the layer's experts in ascending id, plus the
 // shared expert, for every row t.
 template <int NG>
-__global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kMaxGemvWarps * 32, 2) expert_gemv_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_valid[kMaxSlots];  // job index per valid expert, -1: the shared expert
     __shared__ int s_nvalid, s_last;
@@ -403,7 +404,8 @@ cudaError_t launch_gemv(const GemvArgs &a_in, int slots, cudaStream_t s) {
     if (nsteps < 1 || nsteps > kMaxSteps || slots < 1 || slots > kMaxSlots || tiles > kMaxTiles)
         return cudaErrorInvalidValue;
     a.slots = a.only_job >= 0 ? 1 : slots;
-    const int spw = nsteps >= 8 ? 2 : 1;  // 2 K-steps per warp for long rows: smaller CTAs, more per SM
+    // one K-step of 256 per warp (two when that would exceed kMaxGemvWarps warps)
+    const int spw = (nsteps + kMaxGemvWarps - 1) / kMaxGemvWarps;
     const int warps = (nsteps + spw - 1) / spw;
     const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
     const size_t buf = 16 * (size_t)(K / 2) + (size_t)K;  // one tile: codes + scales

@@ -144,25 +144,29 @@ __device__ void split_x(const RouteArgs &a) {
 
 // Softmax + top-k of row t by one warp; writes idx/gates of the row in ascending
 // id and returns the expert selected by this lane (lanes < k), else -1.
-__device__ int topk_row(const RouteArgs &a, int t) {
+// NVE: 32-wide chunks of the row held in registers (E <= 32 * NVE).
+template <int NVE>
+__device__ int topk_row_n(const RouteArgs &a, int t) {
     const int lane = threadIdx.x & 31;
     const float *z = a.ws.z + (size_t)t * a.E;
     const int nv = (a.E + 31) >> 5;
-    float v[kMaxE / 32];
+    float v[NVE];
 #pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j) {
+    for (int j = 0; j < NVE; ++j) {
         const int e = lane + 32 * j;
         v[j] = (j < nv && e < a.E) ? z[e] : -INFINITY;
     }
     float m = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j) m = fmaxf(m, v[j]);
+    for (int j = 0; j < NVE; ++j) m = fmaxf(m, v[j]);
     m = warp_max(m);
-    float sall = 0.f;
+    float sall = 0.f;  // the full softmax denominator (only without renormalisation)
+    if (!a.renorm) {
 #pragma unroll
-    for (int j = 0; j < kMaxE / 32; ++j)
-        if (lane + 32 * j < a.E) sall += expf(v[j] - m);
-    sall = warp_sum(sall);
+        for (int j = 0; j < NVE; ++j)
+            if (lane + 32 * j < a.E) sall += expf(v[j] - m);
+        sall = warp_sum(sall);
+    }
 
     int my_idx = 0x7fffffff;
     float my_val = -INFINITY;
@@ -170,7 +174,7 @@ __device__ int topk_row(const RouteArgs &a, int t) {
         float bv = -INFINITY;
         int bi = 0x7fffffff;
 #pragma unroll
-        for (int j = 0; j < kMaxE / 32; ++j) {
+        for (int j = 0; j < NVE; ++j) {
             const int e = lane + 32 * j;
             if (e < a.E && v[j] > bv) { bv = v[j]; bi = e; }
         }
@@ -183,7 +187,7 @@ __device__ int topk_row(const RouteArgs &a, int t) {
         if (lane == s) { my_idx = bi; my_val = bv; }
         const int owner = bi & 31, slotj = bi >> 5;
 #pragma unroll
-        for (int j = 0; j < kMaxE / 32; ++j)
+        for (int j = 0; j < NVE; ++j)
             if (lane == owner && j == slotj) v[j] = -INFINITY;
     }
     const float top = __shfl_sync(0xffffffffu, my_val, 0);
@@ -201,6 +205,14 @@ __device__ int topk_row(const RouteArgs &a, int t) {
         a.ws.gates[t * a.k + rank] = g;
     }
     return lane < a.k ? my_idx : -1;
+}
+
+__device__ int topk_row(const RouteArgs &a, int t) {
+    const int nv = (a.E + 31) >> 5;
+    if (nv <= 4) return topk_row_n<4>(a, t);
+    if (nv <= 8) return topk_row_n<8>(a, t);
+    if (nv <= 16) return topk_row_n<16>(a, t);
+    return topk_row_n<kMaxE / 32>(a, t);
 }
 
 constexpr int kLookupMax = kMaxK * kDecodeMaxRows;  // entries of one lookup batch (>= kMaxE)
