@@ -399,12 +399,8 @@ def bench_decode(args, shape, rank, world, local):
         before = abi.moe_get_stats(stack.ctx)
         abi.moe_set_timing(stack.ctx, True)
         timed(stack, x, y, L, world)
-        kst = abi.moe_get_stats(stack.ctx)
+        kst = stats_delta(abi.moe_get_stats(stack.ctx), before)
         abi.moe_set_timing(stack.ctx, False)
-        for i in range(abi.MOE_K_COUNT):
-            kst.kernel_launches[i] -= before.kernel_launches[i]
-            kst.kernel_ms[i] -= before.kernel_ms[i]
-            kst.kernel_bytes[i] -= before.kernel_bytes[i]
     el_max = max_over_ranks(el, world)
     tokens_total = sum_over_ranks(float(args.steps), world)
     value = tokens_total / el_max
@@ -416,24 +412,11 @@ def bench_decode(args, shape, rank, world, local):
     t_roof = max(hit_bytes / (hbm_peak * 1e9), miss_bytes / (h2d * 1e9))
     t_roof_8tb = max(hit_bytes / 8000e9, miss_bytes / (h2d * 1e9))
 
-    # dominant kernel by device time (from the timed pass with per-kernel events)
+    # dominant kernel by device time (from the timed pass with per-kernel timing)
     roof, kernels = None, {}
     if kst is not None:
-        ms = list(kst.kernel_ms)
-        dom = int(np.argmax(ms))
-        if kst.kernel_launches[dom] > 0 and ms[dom] > 0:
-            achieved = kst.kernel_bytes[dom] / (ms[dom] * 1e-3) / 1e9
-            roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "hbm", "achieved": achieved,
-                    "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                    "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
-                    "launches": int(kst.kernel_launches[dom]),
-                    "avg_launch_us": ms[dom] * 1e3 / kst.kernel_launches[dom],
-                    "bytes_per_launch": kst.kernel_bytes[dom] / kst.kernel_launches[dom]}
-        kernels = {abi.KERNEL_NAMES[i]: {"launches": int(kst.kernel_launches[i]),
-                                         "ms": round(kst.kernel_ms[i], 3),
-                                         "GBps": (kst.kernel_bytes[i] / (kst.kernel_ms[i] * 1e-3) / 1e9
-                                                  if kst.kernel_ms[i] > 0 else None)}
-                   for i in range(abi.MOE_K_COUNT) if kst.kernel_launches[i]}
+        roof = hbm_roofline(kst, hbm_peak, peak_kind)
+        kernels = kernel_table(kst)
     route_phases = {n: round(v / max(st.forward_calls, 1), 3)
                     for n, v in zip(abi.ROUTE_PHASES, st.route_phase_us)}
     host_phases = host_us_per_call(st)
@@ -495,13 +478,44 @@ def host_us_per_call(st):
                                                 st.host_us)}
 
 
+def kernel_ms(kst, i):
+    """Device time of kernel class i: the summed device spans (first CTA start after
+    its dependency wait to last CTA end) where the class is instrumented, else the
+    CUDA-event time around the launches (which also counts launch latency and any
+    wait for the host or for the previous kernel)."""
+    return kst.kernel_span_ms[i] if kst.kernel_span_ms[i] > 0 else kst.kernel_ms[i]
+
+
 def kernel_table(kst):
     from expert_offload_caching_b200 import abi
-    return {abi.KERNEL_NAMES[i]: {"launches": int(kst.kernel_launches[i]),
-                                  "ms": round(kst.kernel_ms[i], 3),
-                                  "GBps": (kst.kernel_bytes[i] / (kst.kernel_ms[i] * 1e-3) / 1e9
-                                           if kst.kernel_ms[i] > 0 else None)}
-            for i in range(abi.MOE_K_COUNT) if kst.kernel_launches[i]}
+    out = {}
+    for i in range(abi.MOE_K_COUNT):
+        if not kst.kernel_launches[i]:
+            continue
+        t = kernel_ms(kst, i)
+        out[abi.KERNEL_NAMES[i]] = {
+            "launches": int(kst.kernel_launches[i]), "ms": round(t, 3),
+            "ms_events": round(kst.kernel_ms[i], 3),
+            "timing": "device span" if kst.kernel_span_ms[i] > 0 else "events",
+            "GBps": kst.kernel_bytes[i] / (t * 1e-3) / 1e9 if t > 0 else None}
+    return out
+
+
+def hbm_roofline(kst, hbm_peak, peak_kind):
+    """roofline object of the dominant (most device time) HBM-bound kernel class."""
+    from expert_offload_caching_b200 import abi
+    times = [kernel_ms(kst, i) for i in range(abi.MOE_K_COUNT)]
+    dom = int(np.argmax(times))
+    if not kst.kernel_launches[dom] or times[dom] <= 0:
+        return None
+    achieved = kst.kernel_bytes[dom] / (times[dom] * 1e-3) / 1e9
+    return {"kernel": abi.KERNEL_NAMES[dom], "bound": "hbm", "achieved": achieved,
+            "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+            "peak_kind": f"{peak_kind} hbm_gbs (burst copy)", "traffic": None,
+            "timing": "device span" if kst.kernel_span_ms[dom] > 0 else "events",
+            "launches": int(kst.kernel_launches[dom]),
+            "avg_launch_us": times[dom] * 1e3 / kst.kernel_launches[dom],
+            "bytes_per_launch": kst.kernel_bytes[dom] / kst.kernel_launches[dom]}
 
 
 def stats_combine(a, b, sign):
@@ -600,21 +614,22 @@ def bench_prefill(args, shape, rank, world, local):
         kernels = kernel_table(kst)
         tpeak, tkind = measured_fp4_peak()
         i_gu, i_dn = abi.KERNEL_NAMES.index("prefill_gate_up"), abi.KERNEL_NAMES.index("prefill_down")
-        dom, fl = (i_gu, flops_gu) if kst.kernel_ms[i_gu] >= kst.kernel_ms[i_dn] else (i_dn, flops_dn)
-        if kst.kernel_launches[dom] and kst.kernel_ms[dom] > 0:
-            achieved = fl / (kst.kernel_ms[dom] * 1e-3) / 1e12
+        dom, fl = (i_gu, flops_gu) if kernel_ms(kst, i_gu) >= kernel_ms(kst, i_dn) else (i_dn, flops_dn)
+        if kst.kernel_launches[dom] and kernel_ms(kst, dom) > 0:
+            achieved = fl / (kernel_ms(kst, dom) * 1e-3) / 1e12
             roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "tensor", "achieved": achieved,
                     "peak": tpeak, "unit": "TFLOP/s", "frac": achieved / tpeak,
                     "peak_kind": tkind, "traffic": None,
                     "launches": int(kst.kernel_launches[dom]),
-                    "avg_launch_us": kst.kernel_ms[dom] * 1e3 / kst.kernel_launches[dom],
+                    "avg_launch_us": kernel_ms(kst, dom) * 1e3 / kst.kernel_launches[dom],
+                    "timing": "device span" if kst.kernel_span_ms[dom] > 0 else "events",
                     "flops_per_launch": fl / kst.kernel_launches[dom],
                     "note": "tcgen05.mma kind::mxf4nvf4 block16 (E2M1 x E2M1, E4M3 scales), "
                             "TMA-fed, fp32 accumulation in tensor memory"}
         for name, f in (("prefill_gate_up", flops_gu), ("prefill_down", flops_dn)):
             i = abi.KERNEL_NAMES.index(name)
-            if kst.kernel_ms[i] > 0 and name in kernels:
-                kernels[name]["TFLOPs"] = f / (kst.kernel_ms[i] * 1e-3) / 1e12
+            if kernel_ms(kst, i) > 0 and name in kernels:
+                kernels[name]["TFLOPs"] = f / (kernel_ms(kst, i) * 1e-3) / 1e12
 
     e2e = None
     if not args.no_e2e:
@@ -712,16 +727,7 @@ def bench_concurrent(args, shape, rank, world, local):
     roof, kernels = None, {}
     if kst is not None:
         kernels = kernel_table(kst)
-        ms = list(kst.kernel_ms)
-        dom = int(np.argmax(ms))
-        if kst.kernel_launches[dom] > 0 and ms[dom] > 0:
-            achieved = kst.kernel_bytes[dom] / (ms[dom] * 1e-3) / 1e9
-            roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "hbm", "achieved": achieved,
-                    "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                    "peak_kind": f"{peak_kind} hbm_gbs", "traffic": None,
-                    "launches": int(kst.kernel_launches[dom]),
-                    "avg_launch_us": ms[dom] * 1e3 / kst.kernel_launches[dom],
-                    "bytes_per_launch": kst.kernel_bytes[dom] / kst.kernel_launches[dom]}
+        roof = hbm_roofline(kst, hbm_peak, peak_kind)
 
     e2e = None
     if not args.no_e2e:

@@ -48,7 +48,8 @@ class moe_stats(ctypes.Structure):
                 ("kernel_ms", ctypes.c_double * MOE_K_COUNT),
                 ("kernel_bytes", ctypes.c_double * MOE_K_COUNT),
                 ("route_phase_us", ctypes.c_double * 8),
-                ("host_us", ctypes.c_double * 3)]
+                ("host_us", ctypes.c_double * 3),
+                ("kernel_span_ms", ctypes.c_double * MOE_K_COUNT)]
 
 
 class moe_split(ctypes.Structure):

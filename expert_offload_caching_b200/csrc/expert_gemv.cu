@@ -78,7 +78,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 constexpr int kMaxSteps = 16;  // K <= 4096: at most 16 K-steps of 256, one per warp
 constexpr int kGStages = 3;                           // tiles in flight per CTA
-constexpr int kMaxGemvWarps = 12;                     // two CTAs of up to 12 warps per SM
 constexpr int kMaxSlots = kMaxK * kDecodeMaxRows + 1;  // job slots of a launch (+ shared)
 constexpr int kSmCount = 148;
 
@@ -150,7 +149,8 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
 // loads of the next items are in flight while it computes the current one.
 // Each warp owns spw consecutive K-steps of 256 elements; warp 0 sums the
 // warps' partials in a fixed order.  Dynamic shared memory: kGStages x (16*K/2
-// code bytes + K scale bytes) + the partials (warps x NG x 512 bytes).
+// code bytes + K scale bytes) + two buffers of partials (warps x NG x 512
+// bytes each), used in turn, so two barriers per item suffice.
 //
 // Launched with programmatic stream serialization: gate/up waits for the
 // route kernel before reading anything (job list, activations); the down
@@ -163,7 +163,7 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
 // tile's 16 output rows over the layer's experts in ascending id, plus the
 // shared expert, for every row t.
 template <int NG>
-__global__ void __launch_bounds__(kMaxGemvWarps * 32, 2) expert_gemv_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_valid[kMaxSlots];  // job index per valid expert, -1: the shared expert
     __shared__ int s_nvalid, s_last;
@@ -171,7 +171,10 @@ __global__ void __launch_bounds__(kMaxGemvWarps * 32, 2) expert_gemv_kernel(Gemv
     const int g = lane >> 2, q = lane & 3;
     const bool gate_up = a.mode == kGateUp;
 
-    if (gate_up) pdl_wait();  // job list and x come from the previous launch
+    if (gate_up) {
+        pdl_wait();  // job list and x come from the previous launch
+        if (threadIdx.x == 0) span_mark(a.span, 0);
+    }
     pdl_launch_dependents();
 
     // ---- the launch's valid experts.  L2 reads (ld.global.cg): the down launch
@@ -243,13 +246,18 @@ __global__ void __launch_bounds__(kMaxGemvWarps * 32, 2) expert_gemv_kernel(Gemv
     };
 
     for (int j = 0; j < kGStages - 1; ++j) stage(j);
-    if (!gate_up) pdl_wait();  // h comes from the gate/up launch; W2 tiles already in flight
+    if (!gate_up) {
+        pdl_wait();  // h comes from the gate/up launch; W2 tiles already in flight
+        if (threadIdx.x == 0) span_mark(a.span, 0);
+    }
     // tile-local rows of this thread: gate_up 2g (gate) / 2g+1 (up); down g / g+8
     const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
+    int rr = 0;  // row-group counter: the partials buffer alternates, so warp 0's
+                 // epilogue of one group overlaps the other warps' next group
     for (int j = 0; j < n_my; ++j) {
-        stage(j + kGStages - 1);
-        asm volatile("cp.async.wait_group %0;" ::"n"(kGStages - 1) : "memory");
-        __syncthreads();
+        asm volatile("cp.async.wait_group %0;" ::"n"(kGStages - 2) : "memory");  // item j landed
+        __syncthreads();  // ... for every thread; and every thread is done with item j - 1
+        stage(j + kGStages - 1);  // into item j - 1's buffer
         const int item = (int)blockIdx.x + j * G;
         const int jid = s_valid[item / tiles], tile = item - (item / tiles) * tiles;
         const bool shared = jid < 0;
@@ -293,17 +301,19 @@ __global__ void __launch_bounds__(kMaxGemvWarps * 32, 2) expert_gemv_kernel(Gemv
                              col, colv, ngrp, acc);
             }
             // ---- reduce the warps' partial sums (fixed order), then the epilogue
+            float(*rb)[NG][4][32] = red + (rr & 1) * nwarps;
+            ++rr;
 #pragma unroll
             for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) red[warp][grp][i][lane] = acc[grp][i];
+                for (int i = 0; i < 4; ++i) rb[warp][grp][i][lane] = acc[grp][i];
             __syncthreads();
             if (warp == 0) {
                 for (int w = 1; w < nwarps; ++w)
 #pragma unroll
                     for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[grp][i] += red[w][grp][i][lane];
+                        for (int i = 0; i < 4; ++i) acc[grp][i] += rb[w][grp][i][lane];
 #pragma unroll
                 for (int grp = 0; grp < NG; ++grp) {
                     const int r = r0 + 4 * grp + q;  // this thread's results: activation row q
@@ -329,10 +339,10 @@ __global__ void __launch_bounds__(kMaxGemvWarps * 32, 2) expert_gemv_kernel(Gemv
                     }
                 }
             }
-            __syncthreads();  // red reused; after the last row group, the buffer is free
         }
 
         if (a.combine && !gate_up) {  // the tile's last expert: combine its rows
+            __syncthreads();  // warp 0's partials of this item are written
             if (threadIdx.x == 0) {
                 __threadfence();
                 s_last = atomicAdd(&a.tile_ticket[tile], 1u) == (unsigned)(nvalid - 1);
@@ -357,6 +367,10 @@ __global__ void __launch_bounds__(kMaxGemvWarps * 32, 2) expert_gemv_kernel(Gemv
         }
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");  // no copy outlives the CTA
+    if (a.span) {
+        __syncthreads();
+        if (threadIdx.x == 0) span_mark(a.span, 1);
+    }
 }
 
 template <int NG>
@@ -404,12 +418,11 @@ cudaError_t launch_gemv(const GemvArgs &a_in, int slots, cudaStream_t s) {
     if (nsteps < 1 || nsteps > kMaxSteps || slots < 1 || slots > kMaxSlots || tiles > kMaxTiles)
         return cudaErrorInvalidValue;
     a.slots = a.only_job >= 0 ? 1 : slots;
-    // one K-step of 256 per warp (two when that would exceed kMaxGemvWarps warps)
-    const int spw = (nsteps + kMaxGemvWarps - 1) / kMaxGemvWarps;
+    const int spw = nsteps >= 8 ? 2 : 1;  // 2 K-steps per warp for long rows: smaller CTAs, more per SM
     const int warps = (nsteps + spw - 1) / spw;
     const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
     const size_t buf = 16 * (size_t)(K / 2) + (size_t)K;  // one tile: codes + scales
-    const size_t smem = kGStages * buf + (size_t)warps * ng * 4 * 32 * sizeof(float);
+    const size_t smem = kGStages * buf + 2 * (size_t)warps * ng * 4 * 32 * sizeof(float);
     if (smem > 160 * 1024) return cudaErrorInvalidValue;
     if (ng == 1) return launch_ng<1>(a, tiles, warps * 32, smem, s);
     return launch_ng<2>(a, tiles, warps * 32, smem, s);

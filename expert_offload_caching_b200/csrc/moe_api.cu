@@ -127,6 +127,7 @@ struct TimedLaunch {
     int cls;
     cudaEvent_t a, b;
     double bytes;
+    int64_t slot;  // device span slot, -1 if the kernel is not instrumented
 };
 
 }  // namespace
@@ -172,6 +173,9 @@ struct moe_ctx {
     int64_t inj_copy_fail_at = 0, inj_drop_publish = 0;
     double wait_limit = 60.0;
     std::chrono::steady_clock::time_point issue_t0;  // end of the last miss-list wait
+    // device spans of timed launches: [slot][2] = {min start, min ~end}, all ones when free
+    unsigned long long *kspan = nullptr;
+    int64_t kspan_cap = 0, kspan_used = 0;
 };
 
 namespace {
@@ -203,9 +207,28 @@ void time_begin(moe_ctx *ctx, TimedLaunch &tl, int cls) {
     tl.cls = cls;
     tl.a = tl.b = nullptr;
     tl.bytes = 0;
+    tl.slot = -1;
     if (!ctx->timing) return;
     tl.a = pool_event(ctx);
     cudaEventRecord(tl.a, ctx->cs);
+}
+// A span slot for an instrumented launch (null when timing is off or the
+// slots cannot be had); the kernel records into it.
+unsigned long long *time_span(moe_ctx *ctx, TimedLaunch &tl) {
+    if (!ctx->timing || !tl.a) return nullptr;
+    if (!ctx->kspan) {
+        const int64_t cap = 1 << 18;
+        if (cudaMalloc(&ctx->kspan, cap * 2 * sizeof(unsigned long long)) != cudaSuccess ||
+            cudaMemset(ctx->kspan, 0xff, cap * 2 * sizeof(unsigned long long)) != cudaSuccess) {
+            cudaGetLastError();
+            ctx->kspan = nullptr;
+            return nullptr;
+        }
+        ctx->kspan_cap = cap;
+    }
+    if (ctx->kspan_used == ctx->kspan_cap) return nullptr;  // full until the next resolve
+    tl.slot = ctx->kspan_used++;
+    return ctx->kspan + 2 * tl.slot;
 }
 // Returns the index of the pending record, or -1 when timing is off.
 long time_end(moe_ctx *ctx, TimedLaunch &tl, double bytes) {
@@ -219,12 +242,24 @@ long time_end(moe_ctx *ctx, TimedLaunch &tl, double bytes) {
 moe_status resolve_timing(moe_ctx *ctx) {
     if (ctx->pending.empty()) return MOE_OK;
     CK(cudaStreamSynchronize(ctx->cs));
+    std::vector<unsigned long long> sp;
+    if (ctx->kspan && ctx->kspan_used > 0) {
+        sp.resize(2 * ctx->kspan_used);
+        CK(cudaMemcpy(sp.data(), ctx->kspan, sp.size() * sizeof(unsigned long long), cudaMemcpyDeviceToHost));
+        CK(cudaMemset(ctx->kspan, 0xff, sp.size() * sizeof(unsigned long long)));
+        ctx->kspan_used = 0;
+    }
     for (auto &t : ctx->pending) {
         float ms = 0.f;
         CK(cudaEventElapsedTime(&ms, t.a, t.b));
         ctx->stats.kernel_ms[t.cls] += ms;
         ctx->stats.kernel_launches[t.cls] += 1;
         ctx->stats.kernel_bytes[t.cls] += t.bytes;
+        if (t.slot >= 0 && 2 * t.slot + 1 < (int64_t)sp.size()) {
+            const unsigned long long start = sp[2 * t.slot], end = ~sp[2 * t.slot + 1];
+            if (start != ~0ull && sp[2 * t.slot + 1] != ~0ull && end >= start)
+                ctx->stats.kernel_span_ms[t.cls] += (double)(end - start) * 1e-6;
+        }
         ctx->ev_pool.push_back(t.a);
         ctx->ev_pool.push_back(t.b);
     }
@@ -353,6 +388,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     }
     TimedLaunch tl;
     time_begin(ctx, tl, MOE_K_ROUTE);
+    ra.span = time_span(ctx, tl);
     CK(launch_route_lookup(ra, ctx->cs));
     time_end(ctx, tl, (double)D.E * D.d * 2 + (double)T * D.d * 2);
 
@@ -361,11 +397,14 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     const int grid_y = nj + (D.has_shared ? 1 : 0);
     TimedLaunch tg, td;
     time_begin(ctx, tg, MOE_K_GATEUP);
-    CK(launch_gemv(gemv_args(ctx, layer, T, kGateUp, -1), grid_y, ctx->cs));
+    GemvArgs hg = gemv_args(ctx, layer, T, kGateUp, -1);
+    hg.span = time_span(ctx, tg);
+    CK(launch_gemv(hg, grid_y, ctx->cs));
     const long ig = time_end(ctx, tg, 0);
     time_begin(ctx, td, MOE_K_DOWN);
     GemvArgs hd = gemv_args(ctx, layer, T, kDown, -1, 2);  // combines when nothing missed
     hd.y = y;
+    hd.span = time_span(ctx, td);
     CK(launch_gemv(hd, grid_y, ctx->cs));
     const long id = time_end(ctx, td, 0);
 
@@ -415,12 +454,15 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j], 0));
         TimedLaunch mg, md;
         time_begin(ctx, mg, MOE_K_GATEUP);
-        CK(launch_gemv(gemv_args(ctx, layer, T, kGateUp, j), 1, ctx->cs));
+        GemvArgs mg_args = gemv_args(ctx, layer, T, kGateUp, j);
+        mg_args.span = time_span(ctx, mg);
+        CK(launch_gemv(mg_args, 1, ctx->cs));
         time_end(ctx, mg, w13_bytes(ctx) + (double)T * D.d * 2);
         CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j + 1], 0));
         time_begin(ctx, md, MOE_K_DOWN);
         GemvArgs md_args = gemv_args(ctx, layer, T, kDown, j, j == last_miss ? 1 : 0);
         md_args.y = y;
+        md_args.span = time_span(ctx, md);
         CK(launch_gemv(md_args, 1, ctx->cs));
         time_end(ctx, md, w2_bytes(ctx) + (double)T * D.F * 4);
     }
@@ -586,6 +628,7 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     gu.page = ctx->page_d;
     TimedLaunch tg;
     time_begin(ctx, tg, MOE_K_PREFILL_GATEUP);
+    gu.span = time_span(ctx, tg);
     CK(launch_grouped_gemm(ctx->maps, gu, cap, ctx->cs));
     time_end(ctx, tg, grid_y * w13_bytes(ctx));
     const int grouped_rows = T * D.k + (D.has_shared ? T : 0);
@@ -598,6 +641,7 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     dn.act_st = ctx->dws.hq_st;
     TimedLaunch td;
     time_begin(ctx, td, MOE_K_PREFILL_DOWN);
+    dn.span = time_span(ctx, td);
     CK(launch_grouped_gemm(ctx->maps, dn, cap, ctx->cs));
     time_end(ctx, td, grid_y * w2_bytes(ctx));
     CK(launch_combine(ctx->dws.part, ctx->dws.gates, y, T, D.k, D.d, D.has_shared, ctx->cs));
@@ -808,7 +852,14 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         }
         CK(cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs));
         CK(cudaMemsetAsync(ctx->dws.ticket2, 0, 4 * kMaxTiles, ctx->cs));
+        for (auto &t : ctx->pending) {  // timing records of the old state
+            ctx->ev_pool.push_back(t.a);
+            ctx->ev_pool.push_back(t.b);
+        }
         ctx->pending.clear();
+        if (ctx->kspan && ctx->kspan_used > 0)
+            CK(cudaMemset(ctx->kspan, 0xff, 2 * ctx->kspan_used * sizeof(unsigned long long)));
+        ctx->kspan_used = 0;
         ctx->page_h->error = 0;
         std::fill(ctx->pf_pending.begin(), ctx->pf_pending.end(), 0);
         memset(&ctx->stats, 0, sizeof ctx->stats);
@@ -867,6 +918,17 @@ moe_status moe_layer_forward_host(moe_ctx *ctx, int32_t layer, const void *x_hos
     if (ctx->state != MOE_OK || !ctx->configured) return MOE_ERR_STATE;
     const moe_dims &D = ctx->dims;
     if (layer < 0 || layer >= D.L || T < 1 || T > D.max_rows || !x_host || !y_host) return MOE_ERR_ARG;
+    if (T <= kDecodeMaxRows) {
+        // decode: the kernels read x and write y through the buffers' mapped device
+        // addresses (a few KB over PCIe, no copy launches); unmapped or unaligned
+        // buffers take the copy path below
+        void *xm = nullptr, *ym = nullptr;
+        if (((reinterpret_cast<uintptr_t>(x_host) | reinterpret_cast<uintptr_t>(y_host)) & 15) == 0 &&
+            cudaHostGetDevicePointer(&xm, const_cast<void *>(x_host), 0) == cudaSuccess &&
+            cudaHostGetDevicePointer(&ym, y_host, 0) == cudaSuccess)
+            return moe_layer_forward(ctx, layer, xm, T, static_cast<float *>(ym), trace);
+        cudaGetLastError();
+    }
     void *xd = ctx->ws + ctx->wl.xstage;
     float *yd = reinterpret_cast<float *>(ctx->ws + ctx->wl.ystage);
     CK(cudaMemcpyAsync(xd, x_host, (size_t)T * D.d * 2, cudaMemcpyHostToDevice, ctx->cs));
@@ -1078,6 +1140,7 @@ void moe_layer_destroy(moe_ctx *ctx) {
         if (e) cudaEventDestroy(e);
     if (ctx->ev_routed) cudaEventDestroy(ctx->ev_routed);
     if (ctx->page_h) cudaFreeHost(ctx->page_h);
+    if (ctx->kspan) cudaFree(ctx->kspan);
     delete ctx;
 }
 

@@ -108,6 +108,7 @@ struct RouteArgs {
     HostPage *page;          // device alias of the mapped page
     uint32_t seq;
     int publish;
+    unsigned long long *span;  // launch timing slot (see span_mark), or null
 };
 
 enum GemvMode { kGateUp = 0, kDown = 1 };
@@ -136,6 +137,7 @@ struct GemvArgs {
     const float *gates;
     float *y;
     uint32_t *tile_ticket;  // [tiles] per-tile counters of the combining launch, kept at 0
+    unsigned long long *span;  // launch timing slot (see span_mark), or null
 };
 
 // Grouped W4A4 expert GEMMs of a prefill chunk (tcgen05 block-scaled MMA).
@@ -160,6 +162,7 @@ struct GroupedGemmArgs {
     float *h32;               // gate/up output: grouped rows x F
     float *part;              // down output: [T][k+1][d]
     HostPage *page;
+    unsigned long long *span;  // launch timing slot (see span_mark), or null
 };
 // TMA descriptors of the operands: weight codes of the slot arena (3D: byte,
 // row, slot) and of the shared records (3D: byte, row, layer); grouped
@@ -168,6 +171,15 @@ struct GroupedGemmMaps {
     CUtensorMap w13, w2, w13_shared, w2_shared, xq, hq;
     CUtensorMap router;  // router weights (3D: byte, expert row, layer) for the logits GEMM
 };
+
+// Launch timing: slot[0] = min over CTAs of the start time, slot[1] = min of
+// ~end (so both start at all ones and take atomicMin); one thread per CTA.
+__device__ __forceinline__ void span_mark(unsigned long long *slot, int which) {
+    if (slot == nullptr) return;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    atomicMin(slot + which, which ? ~t : t);
+}
 
 // launchers (one per .cu)
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);

@@ -278,6 +278,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) span_mark(a.span, 0);
 
     if (warp == 0) {
         // ---- producer: operand tiles by TMA, scale factors by the lanes.  The
@@ -425,6 +426,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (threadIdx.x == 0) span_mark(a.span, 1);
 }
 
 // (job, n tile) pairs of the layer: a block-wide exclusive scan over the jobs

@@ -97,6 +97,19 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
         const uint4 *xg = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.d);
         for (int i = threadIdx.x; i < nr * nvec; i += blockDim.x) xs[i] = __ldg(xg + i);
         __syncthreads();
+        // the chunk's x as fp16 (hi, lo) pairs for the expert GEMVs (hi + lo == x
+        // for |x| < 65504: bf16 needs no lo in the normal fp16 range, lo keeps what
+        // fp16 subnormals would drop), each element by one thread of the grid
+        // from the staged copy
+        const __nv_bfloat16 *xsb = reinterpret_cast<const __nv_bfloat16 *>(xs);
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nr * a.d; i += gridDim.x * blockDim.x) {
+            const int t = t0 + i / a.d, c = i - (i / a.d) * a.d;
+            const float v = __bfloat162float(xsb[i]);
+            const __half hi = __float2half_rn(v);
+            const __half lo = __float2half_rn(v - __half2float(hi));
+            a.ws.xh[(size_t)t * 2 * a.d + c] = hi;
+            a.ws.xh[(size_t)t * 2 * a.d + a.d + c] = lo;
+        }
         if (has_row) {
             for (int r0 = 0; r0 < nr; r0 += 4) {
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -125,20 +138,6 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
             }
         }
         __syncthreads();
-    }
-}
-
-// x -> (hi, lo) fp16 pair with hi + lo == x for |x| < 65504 (bf16 needs no lo
-// in the normal fp16 range; lo keeps what fp16 subnormals would drop).
-__device__ void split_x(const RouteArgs &a) {
-    const int n = a.T * a.d;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-        const int t = i / a.d, c = i - t * a.d;
-        const float v = __bfloat162float(a.x[i]);
-        const __half hi = __float2half_rn(v);
-        const __half lo = __float2half_rn(v - __half2float(hi));
-        a.ws.xh[(size_t)t * 2 * a.d + c] = hi;
-        a.ws.xh[(size_t)t * 2 * a.d + a.d + c] = lo;
     }
 }
 
@@ -408,8 +407,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     pdl_wait();
     pdl_launch_dependents();
     const unsigned long long t_start = global_ns();  // phases are timed from here
+    if (threadIdx.x == 0) span_mark(a.span, 0);
     router_logits<NV>(a, w, e_row, has_row, xs, rows_per_chunk);
-    split_x(a);
 
     __shared__ int s_last;
     __syncthreads();
@@ -546,6 +545,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     if (threadIdx.x == 0) {
         *a.ws.n_jobs = njobs;
         *a.ws.ticket = 0u;
+    }
+    if (a.span) {
+        __syncthreads();
+        if (threadIdx.x == 0) span_mark(a.span, 1);
     }
 }
 

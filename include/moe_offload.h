@@ -33,9 +33,10 @@
  *
  * Conventions: all functions return a moe_status and never throw; pointers
  * documented as "device" must be device memory of the current CUDA device;
- * the library never allocates device memory -- the caller passes every
- * device buffer.  The library owns only its context, a few CUDA events and
- * one small mapped pinned page for the device-to-host miss list.
+ * the library allocates no device memory on the step's path -- the caller
+ * passes every device buffer.  The library owns its context, a few CUDA
+ * events, one small mapped pinned page for the device-to-host miss list, and
+ * (only once moe_set_timing enables timing) a 4 MB device buffer of timing slots.
  */
 #ifndef MOE_OFFLOAD_H
 #define MOE_OFFLOAD_H
@@ -125,6 +126,10 @@ typedef struct {
      * calls, [1] of which waiting for the device's miss list, [2] of which
      * issuing the copies and launches that follow it */
     double host_us[3];
+    /* with timing on, per kernel class: summed device spans of the launches,
+     * from the first CTA's start (after its wait on the previous kernel) to the
+     * last CTA's end (%globaltimer); 0 for classes not instrumented */
+    double kernel_span_ms[MOE_K_COUNT];
 } moe_stats;
 
 /* Hybrid split plan (ai-hardware-zukan "GPUに載らない分をどう間に合わせるか";
@@ -213,8 +218,12 @@ MOE_API moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x,
                              moe_layer_trace *trace);
 
 /* Same step with HOST buffers: x_host bf16 [T][d] and y_host fp32 [T][d]
- * (page-locked for asynchronous copies).  The copies run on compute_stream
- * through the workspace; y_host is valid after compute_stream synchronises. */
+ * (page-locked).  Decode (T <= 32) with both buffers mapped into the device
+ * address space (cudaHostGetDevicePointer succeeds; true for page-locked
+ * memory on systems with unified addressing) and 16-byte aligned: the kernels
+ * read x and write y in place over PCIe, with no copies.  Otherwise the copies
+ * run on compute_stream through the workspace.  y_host is valid after
+ * compute_stream synchronises. */
 MOE_API moe_status moe_layer_forward_host(moe_ctx *ctx, int32_t layer, const void *x_host, int32_t T,
                                   float *y_host, moe_layer_trace *trace);
 
@@ -231,7 +240,10 @@ MOE_API moe_status moe_cache_export(moe_ctx *ctx, int32_t *map, int32_t *owner, 
 /* Counters; resolves pending kernel timings (synchronises compute_stream if timing is on). */
 MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
 
-/* Per-kernel-class CUDA-event timing on (1) or off (0). */
+/* Per-kernel-class timing on (1) or off (0): CUDA events around every launch
+ * on compute_stream, and device spans (%globaltimer, kernel_span_ms) for the
+ * route, expert GEMV and prefill GEMM kernels.  The first enable allocates a
+ * 4 MB device buffer of span slots, freed by moe_layer_destroy. */
 MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
 
 /* Longest host wait for the device miss list, in seconds (default 60). */

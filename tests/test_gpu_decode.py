@@ -268,3 +268,24 @@ def test_static_split_policy_trace_and_outputs(S):
                             abi.MOE_CACHE_RESET | abi.MOE_CACHE_STATIC_SPLIT | abi.MOE_CACHE_PREFETCH_NEXT)
     assert ei.value.status == abi.MOE_ERR_ARG
     st.close()
+
+
+def test_host_io_unaligned_buffers_take_the_copy_path():
+    """Decode with host buffers: aligned pinned buffers are read and written in
+    place (mapped), unaligned ones go through staging copies; same results."""
+    pb = DecodeProblem(MID, T=3)
+    a = pb.run()
+    st = pb.stack()
+    sh = MID
+    n = pb.T * sh.L * sh.d
+    xh = torch.empty(n + 8, dtype=torch.int16).pin_memory()
+    yh = torch.empty(pb.T * sh.L * sh.d + 4, dtype=torch.float32).pin_memory()
+    xv = xh[1:1 + n].view(pb.T, sh.L, 1, sh.d)  # 2 bytes off the allocation's alignment
+    yv = yh[1:1 + pb.T * sh.L * sh.d].view(pb.T, sh.L, 1, sh.d)
+    xv.copy_(torch.from_numpy(pb.x.view(np.int16)))
+    for t in range(pb.T):
+        for l in range(sh.L):
+            st.forward_host(l, xv[t, l], yv[t, l])
+    st.synchronize()
+    assert torch.equal(yv.cuda(), a.y)
+    st.close()
