@@ -22,7 +22,10 @@ def test_tile_copies_inside_record_and_aligned(shape):
             ("down", shape.F, shape.d // 16, off[2], off[3], off[5])):
         code_bytes, scale_bytes = 16 * (K // 2), K
         assert code_bytes % 16 == 0 and scale_bytes % 16 == 0
-        assert code_bytes + scale_bytes <= 96 * 1024  # dynamic shared memory limit set at launch
+        nsteps = (K // 64 + 3) // 4
+        warps = (nsteps + (2 if nsteps >= 8 else 1) - 1) // (2 if nsteps >= 8 else 1)
+        smem = 3 * (code_bytes + scale_bytes) + 2 * warps * 2 * 512  # ring + two partials buffers (NG 2)
+        assert smem <= 160 * 1024  # dynamic shared memory limit set at launch
         for t in range(tiles):
             c0, s0 = codes0 + t * code_bytes, scales0 + t * scale_bytes
             assert c0 % 16 == 0 and s0 % 16 == 0
@@ -54,3 +57,75 @@ def test_router_rows_fit_the_register_tile(shape):
     grid = (shape.E + 7) // 8
     per = ((total // grid) + 127) & ~127
     assert per * (grid - 1) < total
+
+
+@pytest.mark.parametrize("nitems,G", [(1440, 296), (720, 296), (360, 296), (5, 296), (296, 296),
+                                      (4 * 2560, 148), (1, 1), (7, 3)])
+def test_persistent_gemv_items_cover_each_item_once(nitems, G):
+    """CTA b takes items b, b + G, ...: its count is (nitems - 1 - b) // G + 1 when b < nitems."""
+    seen = []
+    for b in range(min(G, nitems)):
+        n_my = (nitems - 1 - b) // G + 1 if b < nitems else 0
+        seen += [b + j * G for j in range(n_my)]
+    assert sorted(seen) == list(range(nitems))
+
+
+@pytest.mark.parametrize("nvalid,tiles", [(4, 360), (4, 180), (11, 96), (1, 360), (138, 128)])
+def test_combine_ticket_reaches_the_count_once_per_tile(nvalid, tiles):
+    """Expert-major items: each tile receives one ticket per valid expert, so the
+    count nvalid - 1 is reached exactly once per tile, after all its partials."""
+    tickets = [0] * tiles
+    combined = []
+    for item in range(nvalid * tiles):  # any completion order gives the same counts
+        t = item % tiles
+        if tickets[t] == nvalid - 1:
+            combined.append(t)
+        tickets[t] += 1
+    assert sorted(combined) == list(range(tiles))
+
+
+PREFILL = [s for s in SHAPES if s.d >= 256 and s.F >= 256]
+
+
+@pytest.mark.parametrize("shape", PREFILL, ids=lambda s: s.name)
+def test_grouped_gemm_boxes_and_scale_words_inside_their_tensors(shape):
+    """The tcgen05 grouped GEMM: TMA boxes of 128 bytes x 128 rows start on
+    16-byte x coordinates inside each operand's row; the scale words a CTA loads
+    lie inside the record's scale section (weights) or the grouped rows
+    (activations); tensor-memory columns and shared memory fit."""
+    dims = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, shape.shared)
+    off = abi.moe_record_layout(dims)
+    assert 128 + 3 * 4 * 8 <= 256  # accumulator + scale-factor columns of one CTA
+    smem = 2 * 3 * 128 * 128 + 2 * 3 * 4 * 512 + 128 + 1024
+    assert smem <= 113 * 1024  # two CTAs per SM
+    for K, rows_w, sf0, sf_end in ((shape.d, 2 * shape.F, off[1], off[2]),
+                                   (shape.F, shape.d, off[3], off[5])):
+        ksteps, nkb = K // 64, (K // 64 + 3) // 4
+        m_tiles = (rows_w + 127) // 128
+        assert (K // 2) % 16 == 0 and K // 2 >= 128
+        for it in range(nkb):
+            x = it * 128
+            assert x % 16 == 0 and x < K // 2  # box start inside the row (the tail is zero-filled)
+        pitch = K // 16
+        assert pitch % 4 == 0
+        last_word = (rows_w - 1) * pitch + 4 * (ksteps - 1) + 4
+        assert sf0 + last_word <= sf_end
+        assert m_tiles * 128 >= rows_w
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_grouped_gemm_pair_capacity_bounds_the_tile_plan(seed):
+    """sum over jobs of ceil(rows / 128), plus the shared expert's tiles, never
+    exceeds the capacity the host sizes the grid and buffers with."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    T, k = int(rng.integers(33, 4097)), int(rng.integers(1, 33))
+    E = int(rng.integers(k, 1025))
+    sel = np.stack([rng.choice(E, k, replace=False) for _ in range(min(T, 64))])
+    sel = np.concatenate([sel] * (T // len(sel)) + [sel[:T % len(sel)]])
+    counts = np.bincount(sel.ravel(), minlength=E)
+    jobs = counts[counts > 0]
+    for shared in (0, 1):
+        need = int(np.sum((jobs + 127) // 128)) + (shared * ((T + 127) // 128))
+        cap = len(jobs) + (T * k + 127) // 128 + (shared * ((T + 127) // 128))
+        assert need <= cap
