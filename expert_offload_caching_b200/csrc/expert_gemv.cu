@@ -9,11 +9,11 @@
 //
 // Decode is HBM-bound (a few rows, weights read once) and latency-bound when
 // one expert is processed alone.  So:
-//   * one CTA per 16-row weight tile and group of experts; the tile's rows are
-//     contiguous in each record, so the CTA stages a whole tile into shared
-//     memory with 16-byte asynchronous copies (cp.async.cg, L1 bypassed)
-//     issued all at once, the next expert's tile while it computes the current
-//     one.  No registers hold data in flight;
+//   * a persistent grid walks the launch's (expert, 16-row weight tile) items;
+//     a tile's rows are contiguous in the record, so a CTA stages whole tiles
+//     into a 3-deep ring of shared-memory buffers with 16-byte asynchronous
+//     copies (cp.async.cg, L1 bypassed), the next two tiles in flight while it
+//     computes the current one.  No registers hold data in flight;
 //   * the warps split the tile's K-steps of 256 elements;
 //   * E2M1 codes are decoded in registers with cvt.rn.f16x2.e2m1x2 (2 per op),
 //     then multiplied by the E4M3 block scale (cvt.rn.f16x2.e4m3x2); the

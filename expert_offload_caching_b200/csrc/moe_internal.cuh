@@ -131,7 +131,8 @@ struct GemvArgs {
     float *part_out;
     HostPage *page;        // device alias of the mapped page (error word + diagnostics)
     // combine (down launches only): 1 = always, 2 = only if the lookup had no
-    // miss; performed by the last CTA of the launch
+    // miss; performed per 16-row output tile by the CTA that completes the
+    // tile's last expert
     int combine;
     const int32_t *n_misses;
     const float *gates;
