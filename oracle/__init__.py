@@ -83,6 +83,12 @@ def lib():
         L.orc_lru_batch.argtypes = [vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, vp]
         L.orc_plan_split.restype = ctypes.c_int
         L.orc_plan_split.argtypes = [ctypes.c_int, dbl, dbl, dbl, dbl, ip, ip, ip, dp, dp]
+        L.orc_e8m0.restype = dbl
+        L.orc_e8m0.argtypes = [ctypes.c_int]
+        L.orc_mx_record_layout.argtypes = [ctypes.c_int, ctypes.c_int, vp]
+        L.orc_dequant_matrix_mx.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
+        L.orc_expert_mx_w4a16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_expert_bf16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp]
         _lib = L
     return _lib
 
@@ -169,6 +175,39 @@ def expert_w4a16(rec: np.ndarray, d: int, F: int, x: np.ndarray):
 def expert_w4a4(rec: np.ndarray, d: int, F: int, x: np.ndarray) -> np.ndarray:
     y = np.empty(d, dtype=np.float64)
     lib().orc_expert_w4a4(_p(np.ascontiguousarray(rec)), d, F,
+                          _p(np.ascontiguousarray(x, dtype=np.uint16)), _p(y))
+    return y
+
+
+def e8m0(code: int) -> float:
+    return lib().orc_e8m0(int(code))
+
+
+def mx_record_layout(d: int, F: int) -> tuple[int, ...]:
+    off = np.zeros(5, dtype=np.int64)
+    lib().orc_mx_record_layout(d, F, _p(off))
+    return tuple(int(v) for v in off)
+
+
+def dequant_matrix_mx(rec: np.ndarray, d: int, F: int, which: int) -> np.ndarray:
+    """Dequantised matrix of an MXFP4 record: 0 gate [F, d], 1 up [F, d], 2 down [d, F]."""
+    out = np.empty((F, d) if which < 2 else (d, F), dtype=np.float64)
+    lib().orc_dequant_matrix_mx(_p(np.ascontiguousarray(rec)), d, F, which, _p(out))
+    return out
+
+
+def expert_mx_w4a16(rec: np.ndarray, d: int, F: int, x: np.ndarray) -> np.ndarray:
+    """One expert over an MXFP4 record on one bf16 row, fp64."""
+    y = np.empty(d, dtype=np.float64)
+    lib().orc_expert_mx_w4a16(_p(np.ascontiguousarray(rec)), d, F,
+                              _p(np.ascontiguousarray(x, dtype=np.uint16)), _p(y))
+    return y
+
+
+def expert_bf16(rec: np.ndarray, d: int, F: int, x: np.ndarray) -> np.ndarray:
+    """One expert over a BF16 record (W13 rows interleaved, then W2) on one bf16 row, fp64."""
+    y = np.empty(d, dtype=np.float64)
+    lib().orc_expert_bf16(_p(np.ascontiguousarray(rec, dtype=np.uint16)), d, F,
                           _p(np.ascontiguousarray(x, dtype=np.uint16)), _p(y))
     return y
 

@@ -208,6 +208,96 @@ EXPORT void orc_expert_w4a16(const uint8_t *rec, int d, int F, const uint16_t *x
     free(xv);
 }
 
+/* ------------------------------------------- MXFP4 and BF16 expert records -- */
+/* The formats the pages name for other checkpoints (florigen, "NVFP4で約135GBまで縮める":
+ * shared experts kept in BF16; pages' model tables: gpt-oss and DeepSeek-V4
+ * routed experts in MXFP4).  MXFP4 as the OCP microscaling formats define it:
+ * E2M1 elements, one E8M0 scale per 32 consecutive elements, no tensor scale. */
+
+/* E8M0: an 8-bit biased exponent, value 2^(code - 127); code 255 is NaN. */
+EXPORT double orc_e8m0(int code) {
+    if (code == 255) return NAN;
+    return ldexp(1.0, code - 127);
+}
+
+/* MXFP4 record offsets: [0] W13 codes [2F x d/2] (row 2j = gate_j, 2j+1 = up_j),
+ * [1] W13 E8M0 scales [2F x d/32], [2] W2 codes [d x F/2], [3] W2 scales
+ * [d x F/32]; [4] record size; every section on a 256-byte boundary. */
+EXPORT void orc_mx_record_layout(int d, int F, int64_t *off) {
+    int64_t w13_rows = 2 * (int64_t)F, w2_rows = d;
+    off[0] = 0;
+    off[1] = off[0] + up256(w13_rows * d / 2);
+    off[2] = off[1] + up256(w13_rows * d / 32);
+    off[3] = off[2] + up256(w2_rows * F / 2);
+    off[4] = off[3] + up256(w2_rows * F / 32);
+}
+
+static double dq_mx(const uint8_t *codes, const uint8_t *scales, int64_t K, int64_t r, int64_t k) {
+    uint8_t byte = codes[r * (K / 2) + k / 2];
+    int code = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+    return orc_e2m1(code) * orc_e8m0(scales[r * (K / 32) + k / 32]);
+}
+
+/* Full dequantised matrix of an MXFP4 record: which = 0 gate [F x d], 1 up, 2 down [d x F]. */
+EXPORT void orc_dequant_matrix_mx(const uint8_t *rec, int d, int F, int which, double *out) {
+    int64_t off[5];
+    orc_mx_record_layout(d, F, off);
+    if (which < 2) {
+        for (int64_t j = 0; j < F; ++j)
+            for (int64_t k = 0; k < d; ++k) out[j * d + k] = dq_mx(rec + off[0], rec + off[1], d, 2 * j + which, k);
+    } else {
+        for (int64_t i = 0; i < d; ++i)
+            for (int64_t j = 0; j < F; ++j) out[i * F + j] = dq_mx(rec + off[2], rec + off[3], F, i, j);
+    }
+}
+
+/* W4A16 expert over an MXFP4 record, in fp64 (same SwiGLU as expert_from_f64). */
+EXPORT void orc_expert_mx_w4a16(const uint8_t *rec, int d, int F, const uint16_t *x, double *y) {
+    int64_t off[5];
+    orc_mx_record_layout(d, F, off);
+    double *h = (double *)malloc(sizeof(double) * F);
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < F; ++j) {
+        double g = 0.0, u = 0.0;
+        for (int64_t K = 0; K < d; ++K) {
+            const double xv = bf16_val(x[K]);
+            g += dq_mx(rec + off[0], rec + off[1], d, 2 * j, K) * xv;
+            u += dq_mx(rec + off[0], rec + off[1], d, 2 * j + 1, K) * xv;
+        }
+        h[j] = silu(g) * u;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < F; ++j) acc += dq_mx(rec + off[2], rec + off[3], F, i, j) * h[j];
+        y[i] = acc;
+    }
+    free(h);
+}
+
+/* Expert over a BF16 record (W13 [2F x d], rows interleaved gate/up, then W2 [d x F]), fp64. */
+EXPORT void orc_expert_bf16(const uint16_t *rec, int d, int F, const uint16_t *x, double *y) {
+    const uint16_t *w13 = rec, *w2 = rec + 2 * (int64_t)F * d;
+    double *h = (double *)malloc(sizeof(double) * F);
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < F; ++j) {
+        double g = 0.0, u = 0.0;
+        for (int64_t K = 0; K < d; ++K) {
+            const double xv = bf16_val(x[K]);
+            g += bf16_val(w13[(2 * j) * d + K]) * xv;
+            u += bf16_val(w13[(2 * j + 1) * d + K]) * xv;
+        }
+        h[j] = silu(g) * u;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < F; ++j) acc += bf16_val(w2[i * (int64_t)F + j]) * h[j];
+        y[i] = acc;
+    }
+    free(h);
+}
+
 /* ------------------------------------------- NVFP4 activation quantizer -- */
 /* fp32, round-to-nearest-even, in this order:
  *   s_t = amax(row) / 2688 (1 if amax = 0); r = amax(block) / (6 s_t);

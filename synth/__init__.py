@@ -1,8 +1,8 @@
 """Seeded synthetic inputs for the per-layer routed-expert step.
 
-Inputs only: SplitMix64 counter-based draws, Box-Muller normals, NVFP4 encoding
-of the synthetic expert weights, bf16 rounding and the AR(1) hidden-state
-recurrence.  None of the step's own arithmetic lives here; both the CPU oracle
+Inputs only: SplitMix64 counter-based draws, Box-Muller normals, NVFP4 (and
+MXFP4 / BF16) encoding of the synthetic expert weights, bf16 rounding and the
+AR(1) hidden-state recurrence.  None of the step's own arithmetic lives here; both the CPU oracle
 (``oracle/``) and the CUDA path read the bytes this module writes.
 
 Workload recipes (shapes from the FreeToken pages' models; weights N(0, 0.02)):
@@ -59,6 +59,10 @@ def lib():
         L.synth_expert_matrix_f32.argtypes = [u64, i32, i32, i32, i32, i32, i32, dbl, vp]
         L.synth_replicate_records.argtypes = [vp, i64, i64, i64]
         L.synth_prefill_rows_bf16.argtypes = [u64, i32, i32, i32, vp]
+        L.synth_mx_record_layout.argtypes = [i32, i32, vp]
+        L.synth_mx_encode.argtypes = [vp, i64, i64, vp, vp]
+        L.synth_expert_record_mx.argtypes = [u64, i32, i32, i32, i32, i32, dbl, vp]
+        L.synth_expert_record_bf16.argtypes = [u64, i32, i32, i32, i32, i32, dbl, vp]
         _lib = L
     return _lib
 
@@ -120,6 +124,41 @@ def expert_matrix_f32(layer: int, expert: int, m: int, d: int, F: int, *, seed: 
     lib().synth_expert_matrix_f32(seed, purpose, layer, 0 if shared else expert, m, d, F, sigma,
                                   _p(out))
     return out.reshape((F, d) if m < 2 else (d, F))
+
+
+def mx_record_layout(d: int, F: int) -> tuple[int, int, int, int, int]:
+    """MXFP4 record: (w13 codes, w13 E8M0 scales, w2 codes, w2 scales, total) byte offsets."""
+    off = np.zeros(5, dtype=np.int64)
+    lib().synth_mx_record_layout(d, F, _p(off))
+    return tuple(int(v) for v in off)
+
+
+def mx_encode(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP4 codes [rows, K/2] and E8M0 scales [rows, K/32] of an fp32 [rows, K] matrix."""
+    w = np.ascontiguousarray(np.atleast_2d(w), dtype=np.float32)
+    rows, K = w.shape
+    codes = np.empty((rows, K // 2), dtype=np.uint8)
+    scales = np.empty((rows, K // 32), dtype=np.uint8)
+    lib().synth_mx_encode(_p(w), rows, K, _p(codes), _p(scales))
+    return codes, scales
+
+
+def expert_record_mx(layer: int, expert: int, d: int, F: int, *, seed: int = MASTER_SEED,
+                     shared: bool = False, sigma: float = 0.02) -> np.ndarray:
+    """The MXFP4 record (E2M1, one E8M0 scale per 32) of the same draws as expert_record."""
+    out = np.empty(mx_record_layout(d, F)[4], dtype=np.uint8)
+    purpose = PURPOSE_SHARED if shared else PURPOSE_EXPERT
+    lib().synth_expert_record_mx(seed, purpose, layer, 0 if shared else expert, d, F, sigma, _p(out))
+    return out
+
+
+def expert_record_bf16(layer: int, expert: int, d: int, F: int, *, seed: int = MASTER_SEED,
+                       shared: bool = True, sigma: float = 0.02) -> np.ndarray:
+    """A BF16 record of the same draws: W13 [2F x d] (rows interleaved gate/up), then W2 [d x F]."""
+    out = np.empty(3 * d * F, dtype=np.uint16)
+    purpose = PURPOSE_SHARED if shared else PURPOSE_EXPERT
+    lib().synth_expert_record_bf16(seed, purpose, layer, 0 if shared else expert, d, F, sigma, _p(out))
+    return out
 
 
 def replicate_records(ptr: int, rec_bytes: int, n_src: int, n_dst: int) -> None:

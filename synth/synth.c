@@ -220,6 +220,102 @@ EXPORT void synth_expert_record(uint64_t seed, int32_t purpose, int32_t layer, i
     free(w);
 }
 
+/* ------------------------------------------------------- MXFP4 encode -- */
+/* MXFP4 (OCP Microscaling formats: E2M1 elements, one E8M0 scale 2^(c - 127)
+ * per 32 consecutive elements, no tensor scale).  Per block: shared exponent
+ * e = floor(log2(amax)) - 2 (2 = the largest E2M1 exponent), clamped to
+ * [-127, 127]; scale code e + 127; element code E2M1(x / 2^e), RNE, saturating
+ * to 6.  An all-zero block gets scale code 0 and zero codes. */
+static void encode_matrix_mx(const float *w, int64_t rows, int64_t K, int64_t row_mul,
+                             int64_t row_add, uint8_t *codes, uint8_t *scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t orow = r * row_mul + row_add;
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const float *blk = w + r * K + b * 32;
+            float amax = 0.0f;
+            for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(blk[j]));
+            int e = -127;
+            if (amax > 0.0f) {
+                int ex;
+                frexpf(amax, &ex); /* amax = m * 2^ex, m in [0.5, 1): floor(log2 amax) = ex - 1 */
+                e = ex - 1 - 2;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            scales[orow * (K / 32) + b] = (uint8_t)(e + 127);
+            uint8_t *cb = codes + orow * (K / 2) + b * 16;
+            for (int j = 0; j < 16; ++j) {
+                uint8_t lo = 0, hi = 0;
+                if (amax > 0.0f) {
+                    lo = e2m1_encode(ldexpf(blk[2 * j], -e));
+                    hi = e2m1_encode(ldexpf(blk[2 * j + 1], -e));
+                }
+                cb[j] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+}
+
+/* MXFP4 codes and scales of a row-major [rows x K] fp32 matrix (K a multiple of 32). */
+EXPORT void synth_mx_encode(const float *w, int64_t rows, int64_t K, uint8_t *codes, uint8_t *scales) {
+    build_tables();
+    encode_matrix_mx(w, rows, K, 1, 0, codes, scales);
+}
+
+/* Section offsets of one MXFP4 record: [w13 codes, w13 scales, w2 codes, w2 scales, total];
+ * the same row order as the NVFP4 record (W13 row 2j = gate_j, 2j+1 = up_j). */
+EXPORT void synth_mx_record_layout(int32_t d, int32_t F, int64_t *off) {
+    int64_t dd = d, ff = F;
+    off[0] = 0;
+    off[1] = off[0] + align256(2 * ff * dd / 2);
+    off[2] = off[1] + align256(2 * ff * dd / 32);
+    off[3] = off[2] + align256(dd * ff / 2);
+    off[4] = off[3] + align256(dd * ff / 32);
+}
+
+/* The MXFP4 record of the same fp32 draws as synth_expert_record. */
+EXPORT void synth_expert_record_mx(uint64_t seed, int32_t purpose, int32_t layer, int32_t expert,
+                                   int32_t d, int32_t F, double sigma, uint8_t *rec) {
+    build_tables();
+    int64_t off[5];
+    synth_mx_record_layout(d, F, off);
+    memset(rec, 0, (size_t)off[4]);
+    int64_t n = (int64_t)F * d;
+    float *w = (float *)malloc((size_t)n * sizeof(float));
+    for (int m = 0; m < 3; ++m) {
+        uint64_t key = synth_key(seed, (uint64_t)purpose, (uint64_t)layer, (uint64_t)expert,
+                                 (uint64_t)m, 0);
+        synth_normals_f32(key, n, sigma, w);
+        if (m < 2)
+            encode_matrix_mx(w, F, d, 2, m, rec + off[0], rec + off[1]);
+        else
+            encode_matrix_mx(w, d, F, 1, 0, rec + off[2], rec + off[3]);
+    }
+    free(w);
+}
+
+/* A BF16 expert record of the same fp32 draws (the checkpoints keep shared
+ * experts in BF16): W13 [2F x d] (row 2j = gate_j, 2j+1 = up_j), then W2 [d x F],
+ * bf16 RNE; 2 * 3dF bytes. */
+EXPORT void synth_expert_record_bf16(uint64_t seed, int32_t purpose, int32_t layer, int32_t expert,
+                                     int32_t d, int32_t F, double sigma, uint16_t *rec) {
+    int64_t n = (int64_t)F * d;
+    float *w = (float *)malloc((size_t)n * sizeof(float));
+    for (int m = 0; m < 3; ++m) {
+        uint64_t key = synth_key(seed, (uint64_t)purpose, (uint64_t)layer, (uint64_t)expert,
+                                 (uint64_t)m, 0);
+        synth_normals_f32(key, n, sigma, w);
+        if (m < 2) {
+            for (int64_t j = 0; j < F; ++j)
+                for (int64_t i = 0; i < d; ++i) rec[(2 * j + m) * d + i] = f32_to_bf16_rne(w[j * d + i]);
+        } else {
+            for (int64_t i = 0; i < n; ++i) rec[2 * n + i] = f32_to_bf16_rne(w[i]);
+        }
+    }
+    free(w);
+}
+
 /* The fp32 draws behind matrix m of a record (for checking the encoding). */
 EXPORT void synth_expert_matrix_f32(uint64_t seed, int32_t purpose, int32_t layer,
                                     int32_t expert, int32_t m, int32_t d, int32_t F,

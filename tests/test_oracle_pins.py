@@ -468,3 +468,103 @@ def test_layer_record_index_uses_layer_and_expert():
         r = (2 * s.E + idx[t, 0]) % P
         np.testing.assert_array_equal(y[t], oracle.expert_w4a16(pool[r * rb:(r + 1) * rb],
                                                                 s.d, s.F, x[t])[0])
+
+
+# ------------------------------------------------- MXFP4 and BF16 records --
+def test_e8m0_golden_points():
+    for c, v in _rows("e8m0_points.txt"):
+        got = oracle.e8m0(int(c, 16))
+        if v == "nan":
+            assert math.isnan(got)
+        else:
+            assert got == float(v), (c, got, v)
+
+
+def _mx_tiny_record(codes_row, scale):
+    """An MXFP4 record of d = 32, F = 32 whose gate row 0 holds the given 32 codes."""
+    d, F = 32, 32
+    off = oracle.mx_record_layout(d, F)
+    rec = np.zeros(off[4], dtype=np.uint8)
+    packed = [codes_row[2 * i] | (codes_row[2 * i + 1] << 4) for i in range(16)]
+    rec[off[0]:off[0] + 16] = packed  # W13 row 0 (gate_0)
+    rec[off[1]] = scale               # its one scale byte
+    return rec, d, F
+
+
+def test_mxfp4_worked_block_decodes_by_hand():
+    rows = _rows("mxfp4_worked_block.txt")
+    scale = int(rows[0][1], 16)
+    codes = [0] * 32
+    want = np.zeros(32)
+    for r in rows[1:]:
+        codes[int(r[0])] = int(r[2], 16)
+        want[int(r[0])] = float(r[3])
+    rec, d, F = _mx_tiny_record(codes, scale)
+    got = oracle.dequant_matrix_mx(rec, d, F, 0)[0]
+    np.testing.assert_array_equal(got, want)
+
+
+def test_mxfp4_encoder_reproduces_the_worked_block():
+    """The input generator's MXFP4 encoder gives the hand-derived codes and scale."""
+    rows = _rows("mxfp4_worked_block.txt")
+    x = np.zeros(32, dtype=np.float32)
+    want = np.zeros(32, dtype=np.int64)
+    for r in rows[1:]:
+        x[int(r[0])] = float(r[1])
+        want[int(r[0])] = int(r[2], 16)
+    codes, scales = synth.mx_encode(x)
+    got = np.empty(32, dtype=np.int64)
+    got[0::2], got[1::2] = codes[0] & 0xF, codes[0] >> 4
+    np.testing.assert_array_equal(got, want)
+    assert scales[0, 0] == int(rows[0][1], 16)
+
+
+def test_mxfp4_records_decode_like_an_independent_numpy_decode():
+    d, F = 256, 128
+    rec = synth.expert_record_mx(1, 7, d, F)
+    off = oracle.mx_record_layout(d, F)
+    assert off == synth.mx_record_layout(d, F)
+    tab = np.array([E2M1_GOLDEN[c] for c in range(16)])
+
+    def decode(codes, scales, rows, K):
+        c = codes.reshape(rows, K // 2)
+        v = np.empty((rows, K))
+        v[:, 0::2] = tab[c & 0xF]
+        v[:, 1::2] = tab[c >> 4]
+        sc = 2.0 ** (scales.reshape(rows, K // 32).astype(np.float64) - 127)
+        return v * np.repeat(sc, 32, axis=1)
+
+    w13 = decode(rec[off[0]:off[0] + F * d], rec[off[1]:off[1] + F * d // 16], 2 * F, d)
+    w2 = decode(rec[off[2]:off[2] + d * F // 2], rec[off[3]:off[3] + d * F // 32], d, F)
+    np.testing.assert_array_equal(oracle.dequant_matrix_mx(rec, d, F, 0), w13[0::2])
+    np.testing.assert_array_equal(oracle.dequant_matrix_mx(rec, d, F, 1), w13[1::2])
+    np.testing.assert_array_equal(oracle.dequant_matrix_mx(rec, d, F, 2), w2)
+    # the encoding error bound of the scale rule: X = 2^e <= amax/4 per block; an element
+    # within 6X is off by at most X (half the widest E2M1 gap), a clamped one by < 2X
+    for m, W in ((0, w13[0::2]), (1, w13[1::2]), (2, w2)):
+        w = synth.expert_matrix_f32(1, 7, m, d, F).astype(np.float64)
+        blocks = np.abs(w).reshape(-1, 32)
+        X = 2.0 ** (np.floor(np.log2(blocks.max(axis=1))) - 2)
+        err = np.abs(W - w).reshape(-1, 32)
+        assert np.all(err <= 2 * X[:, None] + 1e-12)
+        inside = blocks <= 6 * X[:, None]
+        assert np.all(err[inside] <= np.broadcast_to(X[:, None], err.shape)[inside] + 1e-12)
+
+
+def test_mxfp4_and_bf16_experts_match_dense_numpy():
+    d, F = 256, 128
+    x = _bf16_bits(np.random.default_rng(5).standard_normal(d))
+    xv = _bf16_val(x)
+    silu = lambda v: v * expit(v)  # noqa: E731
+    rec = synth.expert_record_mx(2, 3, d, F)
+    g, u = oracle.dequant_matrix_mx(rec, d, F, 0) @ xv, oracle.dequant_matrix_mx(rec, d, F, 1) @ xv
+    want = oracle.dequant_matrix_mx(rec, d, F, 2) @ (silu(g) * u)
+    np.testing.assert_allclose(oracle.expert_mx_w4a16(rec, d, F, x), want, rtol=1e-12, atol=1e-15)
+    b = synth.expert_record_bf16(2, 0, d, F)
+    w13 = _bf16_val(b[:2 * F * d]).reshape(2 * F, d)
+    w2 = _bf16_val(b[2 * F * d:]).reshape(d, F)
+    h = silu(w13[0::2] @ xv) * (w13[1::2] @ xv)
+    np.testing.assert_allclose(oracle.expert_bf16(b, d, F, x), w2 @ h, rtol=1e-12, atol=1e-15)
+    # the BF16 record holds the same draws as the NVFP4 shared record, rounded to bf16
+    gate = synth.expert_matrix_f32(2, 0, 0, d, F, shared=True)
+    np.testing.assert_array_equal(b[:2 * F * d].reshape(2 * F, d)[0::2], _bf16_bits(gate))
