@@ -91,6 +91,14 @@ def test_init_argument_checks_without_device():
     with pytest.raises(abi.MoeError) as ei:
         abi.moe_layer_init(too_many_k, fake, 1 << 30, fake, None, fake, 1 << 30, fake, fake)
     assert ei.value.status == abi.MOE_ERR_UNSUPPORTED
+    narrow_prefill = abi.make_dims(2, 16, 2, 192, 512, max_rows=64)  # prefill needs d, F >= 256
+    with pytest.raises(abi.MoeError) as ei:
+        abi.moe_layer_init(narrow_prefill, fake, 1 << 30, fake, None, fake, 1 << 30, fake, fake)
+    assert ei.value.status == abi.MOE_ERR_UNSUPPORTED
+    narrow_decode = abi.make_dims(2, 16, 2, 192, 512, max_rows=32)  # decode only: accepted shape
+    with pytest.raises(abi.MoeError) as ei:  # ... and then the unpinned fake pool is refused
+        abi.moe_layer_init(narrow_decode, fake, 1 << 30, fake, None, fake, 1 << 40, fake, fake)
+    assert ei.value.status != abi.MOE_ERR_UNSUPPORTED
     shared_missing = abi.make_dims(2, 16, 2, 256, 512, has_shared=True, max_rows=1)
     with pytest.raises(abi.MoeError) as ei:
         abi.moe_layer_init(shared_missing, fake, 1 << 30, fake, None, fake, 1 << 30, fake, fake)
