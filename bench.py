@@ -194,8 +194,12 @@ def make_inputs(shape, T, stream0):
     return sp.decode_inputs(shape, T, 1, stream0=stream0)
 
 
-def run_tokens(stack, x, y, L, host=False):
+def run_tokens(stack, x, y, L, host=False, mark=None):
+    """Tokens t = 0.. through all L layers; mark = (t0, event): the event is
+    recorded on the compute stream before token t0."""
     for t in range(x.shape[0]):
+        if mark is not None and t == mark[0]:
+            mark[1].record(stack.compute)
         for l in range(L):
             if host:
                 stack.forward_host(l, x[t, l], y[t, l])
@@ -203,18 +207,28 @@ def run_tokens(stack, x, y, L, host=False):
                 stack.forward(l, x[t, l], y[t, l])
 
 
+LAST_STEADY = {}  # steady-window time of the last timed() call: {"t0": first token, "s": seconds}
+
+
 def timed(stack, x, y, L, world, host=False):
+    """Device seconds of all tokens; also records the steady window (tokens from
+    T/4 on, after the cold cache has filled) in LAST_STEADY."""
     barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
+    eq = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    t0 = x.shape[0] // 4
     e0.record(stack.compute)
     torch.cuda.nvtx.range_push("timed")  # lets a profiler select the timed region's launches
-    run_tokens(stack, x, y, L, host)
+    run_tokens(stack, x, y, L, host, mark=(t0, eq) if t0 > 0 else None)
     torch.cuda.nvtx.range_pop()
     e1.record(stack.compute)
     torch.cuda.synchronize()
     barrier(world)
+    LAST_STEADY.clear()
+    if t0 > 0:
+        LAST_STEADY.update(t0=t0, s=eq.elapsed_time(e1) * 1e-3)
     return e0.elapsed_time(e1) * 1e-3
 
 
@@ -383,6 +397,7 @@ def bench_decode(args, shape, rank, world, local):
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
     el = timed(stack, x, y, L, world)
+    steady = dict(LAST_STEADY)
     clk = clocks.stop()
     st = abi.moe_get_stats(stack.ctx)
     if args.warm:  # counters of the timed region only
@@ -404,6 +419,11 @@ def bench_decode(args, shape, rank, world, local):
     el_max = max_over_ranks(el, world)
     tokens_total = sum_over_ranks(float(args.steps), world)
     value = tokens_total / el_max
+    steady_line = None
+    if steady:  # tokens T/4 .. T-1, after the cold cache has filled (every rank takes part)
+        s_max = max_over_ranks(steady["s"], world)
+        steady_line = {"from_token": steady["t0"], "unit": "tok/s",
+                       "value": sum_over_ranks(float(args.steps - steady["t0"]), world) / s_max}
 
     # roofline of the step (the benchmark spec): max(hit bytes / HBM BW, miss bytes / H2D BW)
     hbm_peak, peak_kind = measured_peaks()
@@ -452,7 +472,7 @@ def bench_decode(args, shape, rank, world, local):
                              f"{k * L * rb / 1e9:.2f} GB of expert records)",
                        "cold_cache": True, "parallelism": f"replicas x{world}",
                        "pool_distinct_records": DISTINCT_RECORDS, "policy": args.policy},
-            "miss_rate": st.misses / max(st.lookups, 1),
+            "miss_rate": st.misses / max(st.lookups, 1), "steady_window": steady_line,
             "h2d_gbs": h2d, "h2d_record_gbs": h2d_rec, **H2D_SM,
             "layer_roofline": {"t_roof_s": t_roof, "t_measured_s": el,
                                "frac": t_roof / el, "frac_at_8tbs": t_roof_8tb / el,
