@@ -89,6 +89,9 @@ def lib():
         L.orc_dequant_matrix_mx.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
         L.orc_expert_mx_w4a16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp]
         L.orc_expert_bf16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_moe_layer_fmt.argtypes = [vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -212,20 +215,31 @@ def expert_bf16(rec: np.ndarray, d: int, F: int, x: np.ndarray) -> np.ndarray:
     return y
 
 
+FMT_NVFP4, FMT_MXFP4, FMT_BF16 = 0, 1, 2
+
+
 def moe_layer(pool: np.ndarray, P: int, layer: int, E: int, d: int, F: int, k: int,
               Wr_layer: np.ndarray, shared_rec: np.ndarray | None, x: np.ndarray,
-              w4a4: bool = False, renorm: bool = True):
-    """One layer on T independent rows: (idx [T,k], gates [T,k], y [T,d] fp64)."""
+              w4a4: bool = False, renorm: bool = True, fmt: int = FMT_NVFP4,
+              shared_fmt: int | None = None):
+    """One layer on T independent rows: (idx [T,k], gates [T,k], y [T,d] fp64).
+
+    fmt: the routed records' format (NVFP4 or MXFP4); shared_fmt: the shared
+    record's (None: the routed format; or BF16)."""
     x = np.ascontiguousarray(np.atleast_2d(x), dtype=np.uint16)
     T = x.shape[0]
+    sf = fmt if shared_fmt is None else shared_fmt
     idx = np.empty((T, k), dtype=np.int32)
     gates = np.empty((T, k), dtype=np.float64)
     y = np.empty((T, d), dtype=np.float64)
-    rc = lib().orc_moe_layer(_p(pool), P, layer, E, d, F, k, int(renorm),
-                             _p(np.ascontiguousarray(Wr_layer, dtype=np.uint16)),
-                             _p(shared_rec), _p(x), T, int(w4a4), _p(idx), _p(gates), _p(y))
+    if shared_rec is not None:
+        shared_rec = np.ascontiguousarray(shared_rec).view(np.uint8)
+    rc = lib().orc_moe_layer_fmt(_p(pool), P, layer, E, d, F, k, int(renorm),
+                                 _p(np.ascontiguousarray(Wr_layer, dtype=np.uint16)),
+                                 _p(shared_rec), _p(x), T, int(w4a4), fmt, sf, _p(idx), _p(gates),
+                                 _p(y))
     if rc:
-        raise ValueError("orc_moe_layer: bad arguments")
+        raise ValueError("orc_moe_layer_fmt: bad arguments")
     return idx, gates, y
 
 

@@ -423,16 +423,29 @@ static const uint8_t *pool_record(const uint8_t *pool, int64_t P, int64_t rec_by
     return pool + (((int64_t)layer * E + e) % P) * rec_bytes;
 }
 
+/* One expert on one bf16 row in the record's format: 0 NVFP4 (W4A16, or W4A4
+ * with w4a4), 1 MXFP4 (W4A16), 2 BF16. */
+static void expert_fmt(const uint8_t *rec, int fmt, int w4a4, int d, int F, const uint16_t *x, double *y) {
+    if (fmt == 1) orc_expert_mx_w4a16(rec, d, F, x, y);
+    else if (fmt == 2) orc_expert_bf16((const uint16_t *)rec, d, F, x, y);
+    else if (w4a4) orc_expert_w4a4(rec, d, F, x, y);
+    else orc_expert_w4a16(rec, d, F, x, y, NULL);
+}
+
 /* One MoE layer on T independent rows: route, then
  * y = sum over selected e in ascending id of g_e * E_e(x) + S(x).
- * w4a4 = 0: decode path (W4A16); 1: prefill path (W4A4).
- * shared_rec may be NULL (no shared expert). */
-EXPORT int orc_moe_layer(const uint8_t *pool, int64_t P, int layer, int E, int d, int F, int k,
-                         int renorm, const uint16_t *Wr_layer, const uint8_t *shared_rec,
-                         const uint16_t *x, int T, int w4a4, int32_t *idx, double *gates,
-                         double *y) {
+ * fmt: the routed records' format (0 NVFP4, 1 MXFP4); shared_fmt: the shared
+ * record's (0, 1 or 2 BF16).  w4a4 = 0: decode path (W4A16); 1: prefill path
+ * (W4A4, NVFP4 records only).  shared_rec may be NULL (no shared expert). */
+EXPORT int orc_moe_layer_fmt(const uint8_t *pool, int64_t P, int layer, int E, int d, int F, int k,
+                             int renorm, const uint16_t *Wr_layer, const uint8_t *shared_rec,
+                             const uint16_t *x, int T, int w4a4, int fmt, int shared_fmt, int32_t *idx,
+                             double *gates, double *y) {
+    if (fmt < 0 || fmt > 1 || shared_fmt < 0 || shared_fmt > 2 || (w4a4 && (fmt || shared_fmt))) return 1;
     int64_t off[6];
-    orc_record_layout(d, F, off);
+    if (fmt == 1) orc_mx_record_layout(d, F, off);
+    else orc_record_layout(d, F, off);
+    const int64_t rec_bytes = fmt == 1 ? off[4] : off[5];
     int rc = orc_route(Wr_layer, x, T, E, d, k, renorm, idx, gates, NULL, NULL);
     if (rc) return rc;
     double *ye = (double *)malloc(sizeof(double) * d);
@@ -442,20 +455,26 @@ EXPORT int orc_moe_layer(const uint8_t *pool, int64_t P, int layer, int E, int d
         for (int i = 0; i < d; ++i) yr[i] = 0.0;
         for (int j = 0; j < k; ++j) {
             int e = idx[(int64_t)t * k + j];
-            const uint8_t *rec = pool_record(pool, P, off[5], layer, E, e);
-            if (w4a4) orc_expert_w4a4(rec, d, F, xr, ye);
-            else orc_expert_w4a16(rec, d, F, xr, ye, NULL);
+            expert_fmt(pool_record(pool, P, rec_bytes, layer, E, e), fmt, w4a4, d, F, xr, ye);
             double g = gates[(int64_t)t * k + j];
             for (int i = 0; i < d; ++i) yr[i] += g * ye[i];
         }
         if (shared_rec) {
-            if (w4a4) orc_expert_w4a4(shared_rec, d, F, xr, ye);
-            else orc_expert_w4a16(shared_rec, d, F, xr, ye, NULL);
+            expert_fmt(shared_rec, shared_fmt, w4a4, d, F, xr, ye);
             for (int i = 0; i < d; ++i) yr[i] += ye[i];
         }
     }
     free(ye);
     return 0;
+}
+
+/* The layer with NVFP4 records throughout. */
+EXPORT int orc_moe_layer(const uint8_t *pool, int64_t P, int layer, int E, int d, int F, int k,
+                         int renorm, const uint16_t *Wr_layer, const uint8_t *shared_rec,
+                         const uint16_t *x, int T, int w4a4, int32_t *idx, double *gates,
+                         double *y) {
+    return orc_moe_layer_fmt(pool, P, layer, E, d, F, k, renorm, Wr_layer, shared_rec, x, T, w4a4, 0, 0,
+                             idx, gates, y);
 }
 
 /* --------------------------------------------------------- LRU simulator -- */

@@ -568,3 +568,52 @@ def test_mxfp4_and_bf16_experts_match_dense_numpy():
     # the BF16 record holds the same draws as the NVFP4 shared record, rounded to bf16
     gate = synth.expert_matrix_f32(2, 0, 0, d, F, shared=True)
     np.testing.assert_array_equal(b[:2 * F * d].reshape(2 * F, d)[0::2], _bf16_bits(gate))
+
+
+def test_layer_with_mxfp4_records_and_bf16_shared_matches_numpy():
+    """The layer over MXFP4 routed records (pool indexed by MXFP4 record size)
+    and an MXFP4 or BF16 shared record, against a numpy composition that
+    decodes the records itself."""
+    d, F, E, k, L = 256, 128, 6, 2, 2
+    tab = np.array([E2M1_GOLDEN[c] for c in range(16)])
+    off = synth.mx_record_layout(d, F)
+
+    def mx(rec, which):
+        lo, hi = (off[0], off[1]) if which < 2 else (off[2], off[3])
+        rows, K = (2 * F, d) if which < 2 else (d, F)
+        c = rec[lo:lo + rows * K // 2].reshape(rows, K // 2)
+        v = np.empty((rows, K))
+        v[:, 0::2], v[:, 1::2] = tab[c & 0xF], tab[c >> 4]
+        v *= np.repeat(2.0 ** (rec[hi:hi + rows * K // 32].reshape(rows, K // 32) - 127.0), 32, axis=1)
+        return v if which == 2 else v[which::2]
+
+    silu = lambda v: v * expit(v)  # noqa: E731
+
+    def expert_mx(rec, xv):
+        return mx(rec, 2) @ (silu(mx(rec, 0) @ xv) * (mx(rec, 1) @ xv))
+
+    def expert_bf(b, xv):
+        w13 = _bf16_val(b[:2 * F * d]).reshape(2 * F, d)
+        return _bf16_val(b[2 * F * d:]).reshape(d, F) @ (silu(w13[0::2] @ xv) * (w13[1::2] @ xv))
+
+    pool = np.concatenate([synth.expert_record_mx(l, e, d, F) for l in range(L) for e in range(E)])
+    rb = off[4]
+    Wr = synth.router_bf16(1, E, d)
+    x = _bf16_bits(np.random.default_rng(11).normal(0, 1, (3, d)))
+    shared_mx = synth.expert_record_mx(1, 0, d, F, shared=True)
+    shared_bf = synth.expert_record_bf16(1, 0, d, F)
+    for P in (L * E, 5):  # record of (layer, e) is (layer*E + e) mod P
+        for srec, sfmt, sfun in ((None, None, None), (shared_mx, oracle.FMT_MXFP4, expert_mx),
+                                 (shared_bf, oracle.FMT_BF16, expert_bf)):
+            idx, g, y = oracle.moe_layer(pool[:P * rb], P, 1, E, d, F, k, Wr, srec, x,
+                                         fmt=oracle.FMT_MXFP4, shared_fmt=sfmt)
+            i2, g2, _, _ = oracle.route(Wr, x, k)
+            np.testing.assert_array_equal(idx, i2)
+            for t in range(3):
+                xv = _bf16_val(x[t])
+                want = sum(g[t, j] * expert_mx(pool[((E + idx[t, j]) % P) * rb:][:rb], xv) for j in range(k))
+                if srec is not None:
+                    want = want + sfun(srec, xv)
+                np.testing.assert_allclose(y[t], want, rtol=1e-11, atol=1e-14)
+    with pytest.raises(ValueError):  # W4A4 is the NVFP4 prefill path only
+        oracle.moe_layer(pool, L * E, 1, E, d, F, k, Wr, None, x, w4a4=True, fmt=oracle.FMT_MXFP4)
