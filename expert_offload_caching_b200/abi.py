@@ -13,6 +13,7 @@ MOE_OK, MOE_ERR_ARG, MOE_ERR_CUDA, MOE_ERR_NOT_PINNED = 0, 1, 2, 3
 MOE_ERR_CAPACITY, MOE_ERR_TIMEOUT, MOE_ERR_STATE, MOE_ERR_UNSUPPORTED = 4, 5, 6, 7
 MOE_CACHE_RESET, MOE_CACHE_PREFETCH_NEXT = 1, 2
 MOE_CACHE_STATIC_SPLIT = 4
+MOE_FMT_NVFP4, MOE_FMT_MXFP4, MOE_FMT_BF16 = 0, 1, 2
 MOE_K_ROUTE, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE = 0, 1, 2, 3
 MOE_K_PREFILL_ROUTE, MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_COUNT = 4, 5, 6, 7
 KERNEL_NAMES = ["route_lookup", "gate_up", "down", "combine", "prefill_route", "prefill_gate_up",
@@ -25,7 +26,8 @@ class moe_dims(ctypes.Structure):
     _fields_ = [("L", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("F", ctypes.c_int32), ("has_shared", ctypes.c_int32),
                 ("renormalize", ctypes.c_int32), ("max_rows", ctypes.c_int32),
-                ("pool_records", ctypes.c_int64)]
+                ("pool_records", ctypes.c_int64), ("weight_format", ctypes.c_int32),
+                ("shared_format", ctypes.c_int32)]
 
 
 class moe_cache_event(ctypes.Structure):
@@ -58,7 +60,7 @@ class moe_split(ctypes.Structure):
                 ("t_finish", ctypes.c_double)]
 
 
-EXPORTS = ["moe_record_bytes", "moe_record_layout", "moe_workspace_bytes", "moe_arena_bytes",
+EXPORTS = ["moe_record_bytes", "moe_shared_record_bytes", "moe_record_layout", "moe_workspace_bytes", "moe_arena_bytes",
            "moe_layer_init", "cache_configure", "moe_layer_forward", "moe_layer_forward_host",
            "moe_get_routing", "moe_cache_export", "moe_get_stats", "moe_set_timing",
            "moe_set_wait_limit", "moe_debug_inject", "plan_split", "moe_measure_h2d", "moe_measure_h2d_sm",
@@ -82,6 +84,8 @@ def lib():
         D = ctypes.POINTER(moe_dims)
         L.moe_record_bytes.restype = sz
         L.moe_record_bytes.argtypes = [D]
+        L.moe_shared_record_bytes.restype = sz
+        L.moe_shared_record_bytes.argtypes = [D]
         L.moe_record_layout.restype = ctypes.c_int
         L.moe_record_layout.argtypes = [D, vp]
         L.moe_workspace_bytes.restype = sz
@@ -158,12 +162,20 @@ def _check(rc: int, where: str, ctx=None):
         raise MoeError(rc, where, detail)
 
 
-def make_dims(L, E, k, d, F, has_shared=False, renormalize=True, max_rows=1, pool_records=0):
-    return moe_dims(L, E, k, d, F, int(has_shared), int(renormalize), max_rows, pool_records)
+def make_dims(L, E, k, d, F, has_shared=False, renormalize=True, max_rows=1, pool_records=0,
+              weight_format=MOE_FMT_NVFP4, shared_format=None):
+    """shared_format None: the routed format."""
+    sf = weight_format if shared_format is None else shared_format
+    return moe_dims(L, E, k, d, F, int(has_shared), int(renormalize), max_rows, pool_records,
+                    weight_format, sf)
 
 
 def moe_record_bytes(dims: moe_dims) -> int:
     return lib().moe_record_bytes(ctypes.byref(dims))
+
+
+def moe_shared_record_bytes(dims: moe_dims) -> int:
+    return lib().moe_shared_record_bytes(ctypes.byref(dims))
 
 
 def moe_record_layout(dims: moe_dims) -> tuple[int, ...]:

@@ -24,6 +24,12 @@
 //     against fp32 FMAs.  The dot product is order-free: the mma's logical k
 //     positions are mapped onto each thread's own 64-element chunk, and the
 //     activations are loaded at the same positions;
+//   * MXFP4 records (E8M0 scale 2^(c-127) per 32 elements, no tensor scale):
+//     the scale spans far more than fp16 does, so per K-step and row the
+//     quad's largest scale code c_max is factored out: the mma sees
+//     e2m1 * 2^(c - c_max + 12) (exact in fp16 while c >= c_max - 35; the
+//     +12 keeps those weights normal and below 6 * 2^12), and the step's
+//     fp32 result is multiplied by 2^(c_max - 139) before it is accumulated;
 //   * K-split partial sums are reduced in shared memory in a fixed order;
 //   * the gate/up launch prefetches the expert's down-projection bytes into
 //     L2 (prefetch.global.L2), so the down launch reads L2;
@@ -74,6 +80,81 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 2^diff + kMxBias as an fp16 pair (diff <= 0: an E8M0 code minus the largest
+// code of its K-step; 0 below the fp16 range).
+constexpr int kMxBias = 12;
+__device__ __forceinline__ __half2 mx_pow2_h2(int diff) {
+    const int e = diff + kMxBias;  // <= 12
+    uint32_t bits = e >= -14 ? (uint32_t)(e + 15) << 10 : (e >= -24 ? 1u << (e + 24) : 0u);
+    bits |= bits << 16;
+    return *reinterpret_cast<__half2 *>(&bits);
+}
+// 2^(code - 127 - kMxBias) in fp32 (code 255, E8M0's NaN: NaN).
+__device__ __forceinline__ float mx_factor(int code) {
+    if (code == 255) return __int_as_float(0x7fc00000);
+    const int b = code - kMxBias;  // the fp32 biased exponent
+    return __int_as_float(b >= 1 ? b << 23 : 1 << (b + 22));
+}
+
+// MXFP4 K-step of one thread: as step_mma, with sa / sb holding the two E8M0
+// codes (blocks of 32) of the thread's chunk of rows rA / rB.  The mma
+// accumulates into a zeroed step sum, which is scaled by 2^(c_max - 139) per
+// row (c_max over the quad's chunks, so over the whole mma row) and added.
+template <int NG>
+__device__ __forceinline__ void step_mma_mx(const uint8_t *cA, const uint8_t *cB, uint32_t sa, uint32_t sb,
+                                            int c, bool cv, const __half *const (&col)[NG],
+                                            const bool (&colv)[NG], int ngrp, float (&acc)[NG][4]) {
+    const int a0 = sa & 0xff, a1 = (sa >> 8) & 0xff, b0 = sb & 0xff, b1 = (sb >> 8) & 0xff;
+    int ma = max(a0, a1), mb = max(b0, b1);
+    ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+    ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+    mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+    mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+    const __half2 sAv[2] = {mx_pow2_h2(a0 - ma), mx_pow2_h2(a1 - ma)};
+    const __half2 sBv[2] = {mx_pow2_h2(b0 - mb), mx_pow2_h2(b1 - mb)};
+    float stp[NG][4];
+#pragma unroll
+    for (int grp = 0; grp < NG; ++grp)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) stp[grp][i] = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 qa = cv ? *reinterpret_cast<const uint4 *>(cA + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint4 qb = cv ? *reinterpret_cast<const uint4 *>(cB + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+        const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int w = 4 * h + u;  // 8 codes: elements 8w .. 8w+7 of the chunk, block w / 4
+            uint32_t fa[4], fb[4];
+            e2m1x8_to_f16(wa[u], fa);
+            e2m1x8_to_f16(wb[u], fb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                fa[j] = hmul2u(fa[j], sAv[w >> 2]);
+                fb[j] = hmul2u(fb[j], sBv[w >> 2]);
+            }
+#pragma unroll
+            for (int grp = 0; grp < NG; ++grp) {
+                if (grp < ngrp) {
+                    uint4 bv = make_uint4(0, 0, 0, 0);
+                    if (colv[grp] && cv) bv = __ldg(reinterpret_cast<const uint4 *>(col[grp] + 64 * c + 8 * w));
+                    mma16816(stp[grp], fa[0], fb[0], fa[1], fb[1], bv.x, bv.y);
+                    mma16816(stp[grp], fa[2], fb[2], fa[3], fb[3], bv.z, bv.w);
+                }
+            }
+        }
+    }
+    const float fA = mx_factor(ma), fB = mx_factor(mb);
+#pragma unroll
+    for (int grp = 0; grp < NG; ++grp) {  // d0, d1: row rA; d2, d3: row rB
+        acc[grp][0] = fmaf(stp[grp][0], fA, acc[grp][0]);
+        acc[grp][1] = fmaf(stp[grp][1], fA, acc[grp][1]);
+        acc[grp][2] = fmaf(stp[grp][2], fB, acc[grp][2]);
+        acc[grp][3] = fmaf(stp[grp][3], fB, acc[grp][3]);
+    }
 }
 
 constexpr int kMaxSteps = 16;  // K <= 4096: at most 16 K-steps of 256, one per warp
@@ -162,7 +243,7 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
 // expert of a tile (per-tile ticket counting the launch's experts) sums that
 // tile's 16 output rows over the layer's experts in ascending id, plus the
 // shared expert, for every row t.
-template <int NG>
+template <int NG, int FMT>
 __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_valid[kMaxSlots];  // job index per valid expert, -1: the shared expert
@@ -213,7 +294,8 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
     const int nwarps = (int)(blockDim.x >> 5);
     const int nsteps = (NCH + 3) >> 2;
     const int spw = (nsteps + nwarps - 1) / nwarps;
-    const uint32_t code_bytes = 16u * (uint32_t)(K >> 1), scale_bytes = (uint32_t)K;
+    constexpr bool kMx = FMT == kFmtMxfp4;
+    const uint32_t code_bytes = 16u * (uint32_t)(K >> 1), scale_bytes = kMx ? (uint32_t)(K >> 1) : (uint32_t)K;
     const uint32_t buf_bytes = code_bytes + scale_bytes;
     float(*red)[NG][4][32] = reinterpret_cast<float(*)[NG][4][32]>(smem + kGStages * buf_bytes);
 
@@ -265,7 +347,8 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
         const int nrows = shared ? a.T : __ldcg(&a.jobs[jid].nrows);
         const int row_off = shared ? 0 : __ldcg(&a.jobs[jid].row_off);
         const uint8_t *s_codes = smem + (j % kGStages) * buf_bytes, *s_scales = s_codes + code_bytes;
-        const float *ts = reinterpret_cast<const float *>(rec + a.lay.tscales);
+        // tensor scales (gate, up, down): NVFP4 only
+        const float *ts = kMx ? nullptr : reinterpret_cast<const float *>(rec + a.lay.tscales);
         for (int r0 = 0; r0 < nrows; r0 += 4 * NG) {
             // mma column n = g carries activation row r0 + 4*grp + g/2, the hi (g
             // even) or lo (g odd) fp16 part.
@@ -295,10 +378,17 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
                 const int c = 4 * (warp * spw + st) + q;
                 const bool cv = c < NCH;  // ragged K tail: some lanes of the quad feed zeros
                 const int cc = cv ? c : 0;
-                const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
-                const uint32_t sb = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rB * (K >> 4) + 4 * c) : 0u;
-                step_mma<NG>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc, sa, sb, cc, cv,
-                             col, colv, ngrp, acc);
+                if constexpr (kMx) {  // two E8M0 codes per row and chunk
+                    const uint32_t sa = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rA * (K >> 5) + 2 * c) : 0u;
+                    const uint32_t sb = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rB * (K >> 5) + 2 * c) : 0u;
+                    step_mma_mx<NG>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc, sa, sb, cc,
+                                    cv, col, colv, ngrp, acc);
+                } else {
+                    const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
+                    const uint32_t sb = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rB * (K >> 4) + 4 * c) : 0u;
+                    step_mma<NG>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc, sa, sb, cc,
+                                 cv, col, colv, ngrp, acc);
+                }
             }
             // ---- reduce the warps' partial sums (fixed order), then the epilogue
             float(*rb)[NG][4][32] = red + (rr & 1) * nwarps;
@@ -325,7 +415,7 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
                     const float v1 = acc[grp][2] + acc[grp][3];  // tile row rB
                     const size_t sel = (size_t)t * (a.k + 1) + p;
                     if (gate_up) {
-                        const float gt = ts[0] * v0, up = ts[1] * v1;
+                        const float gt = kMx ? v0 : ts[0] * v0, up = kMx ? v1 : ts[1] * v1;
                         const float h = gt / (1.0f + expf(-gt)) * up;
                         const int o = 8 * tile + g;
                         const __half hi = __float2half_rn(h);
@@ -334,8 +424,9 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
                         a.hh_out[sel * 2 * a.F + a.F + o] = lo;
                     } else {
                         const int o = 16 * tile + g;
-                        a.part_out[sel * a.d + o] = ts[2] * v0;
-                        a.part_out[sel * a.d + o + 8] = ts[2] * v1;
+                        const float sd = kMx ? 1.0f : ts[2];
+                        a.part_out[sel * a.d + o] = sd * v0;
+                        a.part_out[sel * a.d + o + 8] = sd * v1;
                     }
                 }
             }
@@ -373,12 +464,12 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
     }
 }
 
-template <int NG>
+template <int NG, int FMT>
 cudaError_t launch_ng(const GemvArgs &a, int tiles, int threads, size_t smem, cudaStream_t s) {
     static bool configured = false;  // per instantiation: allow > 48 KB of dynamic smem
     static int sms = 0;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<NG>,
+        cudaError_t e = cudaFuncSetAttribute(expert_gemv_kernel<NG, FMT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
         if (e != cudaSuccess) return e;
         int dev = 0;
@@ -389,7 +480,7 @@ cudaError_t launch_ng(const GemvArgs &a, int tiles, int threads, size_t smem, cu
     }
     // persistent grid: as many CTAs as fit at once (at most 4 per SM), no more than the items
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_gemv_kernel<NG>, threads, smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_gemv_kernel<NG, FMT>, threads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     if (per_sm > 4) per_sm = 4;
@@ -405,7 +496,7 @@ cudaError_t launch_ng(const GemvArgs &a, int tiles, int threads, size_t smem, cu
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, expert_gemv_kernel<NG>, a);
+    return cudaLaunchKernelEx(&cfg, expert_gemv_kernel<NG, FMT>, a);
 }
 
 }  // namespace
@@ -421,11 +512,17 @@ cudaError_t launch_gemv(const GemvArgs &a_in, int slots, cudaStream_t s) {
     const int spw = nsteps >= 8 ? 2 : 1;  // 2 K-steps per warp for long rows: smaller CTAs, more per SM
     const int warps = (nsteps + spw - 1) / spw;
     const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
-    const size_t buf = 16 * (size_t)(K / 2) + (size_t)K;  // one tile: codes + scales
+    const bool mx = a.lay.fmt == kFmtMxfp4;
+    if (!mx && a.lay.fmt != kFmtNvfp4) return cudaErrorInvalidValue;
+    const size_t buf = 16 * (size_t)(K / 2) + (size_t)(mx ? K / 2 : K);  // one tile: codes + scales
     const size_t smem = kGStages * buf + 2 * (size_t)warps * ng * 4 * 32 * sizeof(float);
     if (smem > 160 * 1024) return cudaErrorInvalidValue;
-    if (ng == 1) return launch_ng<1>(a, tiles, warps * 32, smem, s);
-    return launch_ng<2>(a, tiles, warps * 32, smem, s);
+    if (mx) {
+        if (ng == 1) return launch_ng<1, kFmtMxfp4>(a, tiles, warps * 32, smem, s);
+        return launch_ng<2, kFmtMxfp4>(a, tiles, warps * 32, smem, s);
+    }
+    if (ng == 1) return launch_ng<1, kFmtNvfp4>(a, tiles, warps * 32, smem, s);
+    return launch_ng<2, kFmtNvfp4>(a, tiles, warps * 32, smem, s);
 }
 
 }  // namespace moe

@@ -26,6 +26,8 @@
 #include "moe_internal.cuh"
 
 using namespace moe;
+static_assert(kFmtNvfp4 == MOE_FMT_NVFP4 && kFmtMxfp4 == MOE_FMT_MXFP4 && kFmtBf16 == MOE_FMT_BF16,
+              "record format values");
 
 namespace {
 
@@ -33,27 +35,50 @@ inline int64_t up256(int64_t x) { return (x + 255) / 256 * 256; }
 
 bool dims_valid(const moe_dims *d) {
     return d && d->L > 0 && d->E > 0 && d->k > 0 && d->k <= d->E && d->d > 0 && d->F > 0 &&
-           d->max_rows > 0 && d->pool_records >= 0;
+           d->max_rows > 0 && d->pool_records >= 0 &&
+           (d->weight_format == MOE_FMT_NVFP4 || d->weight_format == MOE_FMT_MXFP4) &&
+           (!d->has_shared || d->shared_format == d->weight_format || d->shared_format == MOE_FMT_BF16);
 }
+// The shared experts' format (the routed one when there are none).
+int shared_fmt(const moe_dims *d) { return d->has_shared ? d->shared_format : d->weight_format; }
 bool dims_supported(const moe_dims *d) {
     return d->d % 64 == 0 && d->F % 64 == 0 && d->d <= 4096 && d->F <= 4096 && d->k <= kMaxK &&
            d->E <= kMaxE &&
            d->max_rows <= 4096 && (int64_t)d->L * d->E < (1ll << 31) &&
-           // prefill GEMM operands: TMA boxes of 128 bytes of a row
-           (d->max_rows <= kDecodeMaxRows || (d->d >= 256 && d->F >= 256));
+           // prefill GEMM operands: TMA boxes of 128 bytes of a row; NVFP4 block scales
+           (d->max_rows <= kDecodeMaxRows || (d->d >= 256 && d->F >= 256 && d->weight_format == MOE_FMT_NVFP4 &&
+                                              shared_fmt(d) == MOE_FMT_NVFP4));
 }
 
-RecordLayout layout_of(const moe_dims *d) {
+// Section offsets of a record of format fmt (the header's MOE_FMT_* layouts).
+RecordLayout layout_fmt(const moe_dims *d, int fmt) {
     RecordLayout r;
     const int64_t dd = d->d, ff = d->F;
-    r.tscales = 0;  // head: the gate/up half (tensor scales + W13) is a contiguous prefix
-    r.w13_codes = up256(12);
-    r.w13_scales = r.w13_codes + up256(2 * ff * dd / 2);
-    r.w2_codes = r.w13_scales + up256(2 * ff * dd / 16);
-    r.w2_scales = r.w2_codes + up256(dd * ff / 2);
-    r.bytes = r.w2_scales + up256(dd * ff / 16);
+    r.fmt = fmt;
+    if (fmt == MOE_FMT_BF16) {  // W13 then W2, bf16, unpadded
+        r.tscales = r.w13_scales = r.w2_scales = -1;
+        r.w13_codes = 0;
+        r.w2_codes = 2 * (2 * ff * dd);
+        r.bytes = r.w2_codes + 2 * (dd * ff);
+    } else if (fmt == MOE_FMT_MXFP4) {  // E8M0 scale per 32, no tensor scales
+        r.tscales = -1;
+        r.w13_codes = 0;
+        r.w13_scales = r.w13_codes + up256(2 * ff * dd / 2);
+        r.w2_codes = r.w13_scales + up256(2 * ff * dd / 32);
+        r.w2_scales = r.w2_codes + up256(dd * ff / 2);
+        r.bytes = r.w2_scales + up256(dd * ff / 32);
+    } else {
+        r.tscales = 0;  // head: the gate/up half (tensor scales + W13) is a contiguous prefix
+        r.w13_codes = up256(12);
+        r.w13_scales = r.w13_codes + up256(2 * ff * dd / 2);
+        r.w2_codes = r.w13_scales + up256(2 * ff * dd / 16);
+        r.w2_scales = r.w2_codes + up256(dd * ff / 2);
+        r.bytes = r.w2_scales + up256(dd * ff / 16);
+    }
     return r;
 }
+RecordLayout layout_of(const moe_dims *d) { return layout_fmt(d, d->weight_format); }
+RecordLayout shared_layout_of(const moe_dims *d) { return layout_fmt(d, shared_fmt(d)); }
 
 int max_jobs(const moe_dims *d, int T) {
     int64_t n = (int64_t)T * d->k;
@@ -134,7 +159,8 @@ struct TimedLaunch {
 
 struct moe_ctx {
     moe_dims dims;
-    RecordLayout lay;
+    RecordLayout lay;   // routed records
+    RecordLayout slay;  // shared-expert records
     int64_t P = 0;
     const uint8_t *pool = nullptr;
     const __nv_bfloat16 *router_w = nullptr;
@@ -267,6 +293,10 @@ moe_status resolve_timing(moe_ctx *ctx) {
     return MOE_OK;
 }
 
+bool shared_separate(const moe_ctx *ctx) {
+    return ctx->dims.has_shared && ctx->slay.fmt != ctx->lay.fmt;
+}
+
 GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int combine = 0) {
     const moe_dims &D = ctx->dims;
     GemvArgs g{};
@@ -275,10 +305,13 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
     g.n_jobs = ctx->dws.n_jobs;
     g.rowrefs = ctx->dws.rowrefs;
     g.only_job = only_job;
-    g.shared_slot = (only_job < 0 && D.has_shared) ? max_jobs(&D, T) : -1;
+    // the shared expert is an item of the routed launches when it has their
+    // format; a BF16 shared expert runs in its own launches (its partial is
+    // still summed by the combine: shared_rec non-null)
+    g.shared_slot = (only_job < 0 && D.has_shared && !shared_separate(ctx)) ? max_jobs(&D, T) : -1;
     g.arena = ctx->arena;
     g.rec_bytes = ctx->lay.bytes;
-    g.shared_rec = D.has_shared ? ctx->shared_recs + (int64_t)layer * ctx->lay.bytes : nullptr;
+    g.shared_rec = D.has_shared ? ctx->shared_recs + (int64_t)layer * ctx->slay.bytes : nullptr;
     g.T = T;
     g.k = D.k;
     g.d = D.d;
@@ -296,8 +329,12 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
     return g;
 }
 
-double w13_bytes(const moe_ctx *c) { return (double)(c->lay.w2_codes - c->lay.w13_codes) + 8.0; }
-double w2_bytes(const moe_ctx *c) { return (double)(c->lay.bytes - c->lay.w2_codes) + 4.0; }
+double w13_bytes(const moe_ctx *c) {
+    return (double)(c->lay.w2_codes - c->lay.w13_codes) + (c->lay.tscales >= 0 ? 8.0 : 0.0);
+}
+double w2_bytes(const moe_ctx *c) {
+    return (double)(c->lay.bytes - c->lay.w2_codes) + (c->lay.tscales >= 0 ? 4.0 : 0.0);
+}
 
 // A kernel reported a failed self-check through the mapped page (error word
 // and a diagnostic record: check code, kernel mode, block, tile, sizes).
@@ -392,9 +429,23 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     CK(launch_route_lookup(ra, ctx->cs));
     time_end(ctx, tl, (double)D.E * D.d * 2 + (double)T * D.d * 2);
 
-    // hit experts and the shared expert, before the miss list is known
     const int nj = max_jobs(&D, T);
-    const int grid_y = nj + (D.has_shared ? 1 : 0);
+    if (shared_separate(ctx)) {  // BF16 shared expert: its own two launches
+        TimedLaunch sg, sd;
+        const uint8_t *rec = ctx->shared_recs + (int64_t)layer * ctx->slay.bytes;
+        const int64_t sel0 = D.k, sel_stride = D.k + 1;  // selection p = k of row t
+        time_begin(ctx, sg, MOE_K_GATEUP);
+        CK(launch_shared_bf16(kGateUp, rec, D.d, D.F, T, ctx->dws.xh, ctx->dws.hh, ctx->dws.part, sel0, sel_stride,
+                              ctx->cs));
+        time_end(ctx, sg, 2.0 * 2 * D.F * D.d + (double)T * D.d * 2);
+        time_begin(ctx, sd, MOE_K_DOWN);
+        CK(launch_shared_bf16(kDown, rec, D.d, D.F, T, ctx->dws.xh, ctx->dws.hh, ctx->dws.part, sel0, sel_stride,
+                              ctx->cs));
+        time_end(ctx, sd, 2.0 * D.d * D.F + (double)T * D.F * 4);
+    }
+    // hit experts and the shared expert, before the miss list is known
+    const int in_launch_shared = (D.has_shared && !shared_separate(ctx)) ? 1 : 0;
+    const int grid_y = nj + in_launch_shared;
     TimedLaunch tg, td;
     time_begin(ctx, tg, MOE_K_GATEUP);
     GemvArgs hg = gemv_args(ctx, layer, T, kGateUp, -1);
@@ -422,7 +473,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         if (!(ev[j].flags & 1)) last_miss = j;
     }
     if (ig >= 0 && id >= 0) {  // algorithmic bytes of the two hit launches, now known
-        const int nexp = n_hit_jobs + (D.has_shared ? 1 : 0);
+        const int nexp = n_hit_jobs + in_launch_shared;
         ctx->pending[ig].bytes = nexp * w13_bytes(ctx) + (double)T * D.d * 2;
         ctx->pending[id].bytes = nexp * w2_bytes(ctx) + (double)T * D.F * 4;
     }
@@ -675,6 +726,11 @@ size_t moe_record_bytes(const moe_dims *dims) {
     return (size_t)layout_of(dims).bytes;
 }
 
+size_t moe_shared_record_bytes(const moe_dims *dims) {
+    if (!dims_valid(dims)) return 0;
+    return (size_t)shared_layout_of(dims).bytes;
+}
+
 moe_status moe_record_layout(const moe_dims *dims, int64_t off[6]) {
     if (!dims_valid(dims) || !off) return MOE_ERR_ARG;
     RecordLayout r = layout_of(dims);
@@ -716,6 +772,7 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     moe_ctx *ctx = new moe_ctx();
     ctx->dims = *dims;
     ctx->lay = lay;
+    ctx->slay = shared_layout_of(dims);
     ctx->P = P;
     ctx->pool = static_cast<const uint8_t *>(host_pool);
     ctx->router_w = static_cast<const __nv_bfloat16 *>(router_w);
@@ -759,9 +816,9 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
                                    2 * (int64_t)dims->E * dims->d);
         if (ok && dims->has_shared) {
             ok = make_operand_map(&ctx->maps.w13_shared, ctx->shared_recs + lay.w13_codes, dims->d / 2,
-                                  2 * dims->F, dims->L, lay.bytes) &&
+                                  2 * dims->F, dims->L, ctx->slay.bytes) &&
                  make_operand_map(&ctx->maps.w2_shared, ctx->shared_recs + lay.w2_codes, dims->F / 2, dims->d,
-                                  dims->L, lay.bytes);
+                                  dims->L, ctx->slay.bytes);
         }
         if (!ok) {
             delete ctx;

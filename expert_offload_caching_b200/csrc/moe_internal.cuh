@@ -13,9 +13,14 @@ constexpr int kMaxK = 32;
 constexpr int kMaxE = 1024;
 constexpr int kMaxTiles = 512;  // GEMV tiles per launch: max(d / 16, F / 8) with d, F <= 4096
 
-// Record sections (byte offsets), computed once per context.
+// Record formats (the values of the C ABI's MOE_FMT_* constants).
+constexpr int kFmtNvfp4 = 0, kFmtMxfp4 = 1, kFmtBf16 = 2;
+
+// Record sections (byte offsets, -1 for a section the format lacks), computed
+// once per context; fmt is the record format (MOE_FMT_NVFP4 / MXFP4 / BF16).
 struct RecordLayout {
     int64_t w13_codes, w13_scales, w2_codes, w2_scales, tscales, bytes;
+    int32_t fmt;
 };
 
 // Device cache table, in the slot arena after the slots.  The least recently
@@ -186,6 +191,12 @@ __device__ __forceinline__ void span_mark(unsigned long long *slot, int which) {
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
 // slots: job slots of the launch (max jobs + shared expert), 1 with only_job
 cudaError_t launch_gemv(const GemvArgs &a, int slots, cudaStream_t s);
+// BF16 shared expert of a decode call (T <= 32 rows; x as DecodeWs::xh):
+// kGateUp writes h = silu(W1 x) * (W3 x) as fp16 (hi, lo) into hh at selection
+// sel0 + t * sel_stride (layout of DecodeWs::hh); kDown reads that h and
+// writes W2 h into part at the same selection.
+cudaError_t launch_shared_bf16(int mode, const uint8_t *rec, int d, int F, int T, const __half *xh,
+                               __half *hh, float *part, int64_t sel0, int64_t sel_stride, cudaStream_t s);
 cudaError_t launch_table_reset(Table t, int64_t nkeys, cudaStream_t s);
 cudaError_t launch_table_static(Table t, int L, int E, int per_layer, cudaStream_t s);
 cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s);

@@ -17,7 +17,7 @@ class LayerStack:
 
     host_pool: page-locked uint8 tensor of P expert records (the pinned host pool).
     router_w: device tensor, bf16 [L, E, d] (or its uint16 bit pattern).
-    shared: device uint8 tensor of L shared-expert records, or None.
+    shared: device uint8 tensor of L shared-expert records (abi.moe_shared_record_bytes each), or None.
     """
 
     def __init__(self, dims: abi.moe_dims, host_pool: torch.Tensor, router_w: torch.Tensor,

@@ -19,8 +19,9 @@
  * For prefill chunks, the next layer's experts are streamed in while the
  * current layer computes (holude.com "長いプロンプトとエージェント処理も意識している").
  *
- * Expert record (one contiguous block per (layer, expert); moe_record_layout
- * returns the offsets off[0..5] of the sections named below):
+ * Expert record (one contiguous block per (layer, expert)) in the default
+ * format, NVFP4 (other formats: MOE_FMT_* below); moe_record_layout returns
+ * the offsets off[0..5] of the sections named below:
  *   off[4] 3 fp32 tensor scales: gate, up, down (at the record head)
  *   off[0] W13 codes  [2F x d/2] bytes; row 2j = gate_j, row 2j+1 = up_j; E2M1,
  *                     two per byte, element 2i in the low nibble
@@ -72,14 +73,33 @@ typedef enum {
  * the softmax renormalised over the selected k (1) or the plain softmax probabilities (0).
  * max_rows: largest T passed to moe_layer_forward.
  * pool_records: P, the records in the host pool; expert (l, e) is record (l*E + e) mod P;
- * 0 means P = L*E. */
+ * 0 means P = L*E.
+ * weight_format: MOE_FMT_NVFP4 (0) or MOE_FMT_MXFP4, the routed experts' records.
+ * shared_format: the shared experts' records (has_shared): the routed
+ *   format or MOE_FMT_BF16.  Zeros (both NVFP4) keep the default layout. */
 typedef struct {
     int32_t L, E, k, d, F;
     int32_t has_shared;
     int32_t renormalize;
     int32_t max_rows;
     int64_t pool_records;
+    int32_t weight_format;
+    int32_t shared_format;
 } moe_dims;
+
+/* Record formats.  NVFP4: the layout below.  MXFP4 (OCP microscaling; the
+ * pages' model tables list gpt-oss and DeepSeek-V4 routed experts in MXFP4):
+ * E2M1 codes as in NVFP4, one E8M0 scale byte 2^(c - 127) per 32 consecutive
+ * elements of a row (c = 255: NaN), no tensor scales; sections off[0] W13
+ * codes [2F x d/2], off[1] W13 scales [2F x d/32], off[2] W2 codes [d x F/2],
+ * off[3] W2 scales [d x F/32], 256-byte aligned, off[4] = -1, off[5] total.
+ * BF16 (shared experts only; florigen.ai "NVFP4で約135GBまで縮める" keeps
+ * them in BF16): W13 [2F x d] bf16 (row 2j = gate_j, 2j+1 = up_j) at 0, then
+ * W2 [d x F] at 4Fd bytes; 6Fd bytes.  MXFP4 and BF16 run on the decode path
+ * only (max_rows <= 32, else MOE_ERR_UNSUPPORTED). */
+#define MOE_FMT_NVFP4 0
+#define MOE_FMT_MXFP4 1
+#define MOE_FMT_BF16 2
 
 typedef struct moe_ctx moe_ctx; /* opaque, library-owned host state */
 
@@ -156,10 +176,14 @@ typedef struct {
  * Not with MOE_CACHE_PREFETCH_NEXT (MOE_ERR_ARG).  Changing the policy resets. */
 #define MOE_CACHE_STATIC_SPLIT 4u
 
-/* Bytes of one expert record; 0 if dims are invalid. */
+/* Bytes of one routed expert record (weight_format); 0 if dims are invalid. */
 MOE_API size_t moe_record_bytes(const moe_dims *dims);
 
-/* Section offsets of one record into off[6] (see the layout above). */
+/* Bytes of one shared-expert record (shared_format); 0 if dims are invalid. */
+MOE_API size_t moe_shared_record_bytes(const moe_dims *dims);
+
+/* Section offsets of one routed record into off[6] (see the layouts above;
+ * -1 for a section the format does not have). */
 MOE_API moe_status moe_record_layout(const moe_dims *dims, int64_t off[6]);
 
 /* Device workspace bytes moe_layer_init needs for these dims (caller-owned). */
@@ -173,13 +197,16 @@ MOE_API size_t moe_arena_bytes(const moe_dims *dims, int64_t num_slots);
  *              (else MOE_ERR_NOT_PINNED); read by DMA only; caller-owned, must
  *              outlive the context; host_pool_bytes >= P * record bytes.
  *   router_w:  device, bf16 [L][E][d] router weights.
- *   shared_recs: device, L shared-expert records back to back (has_shared), else NULL.
+ *   shared_recs: device, L shared-expert records (moe_shared_record_bytes each)
+ *              back to back (has_shared), else NULL.
  *   workspace: device, >= moe_workspace_bytes(dims), caller-owned.
  *   compute_stream, copy_stream: cudaStream_t handles (NULL = legacy stream not
  *              accepted: pass real streams); work is issued on them only.
  * Shapes handled: d and F multiples of 64, 1 <= k <= 32, k <= E <= 1024,
- * 1 <= max_rows <= 4096, and with max_rows > 32 (prefill) d >= 256 and
- * F >= 256; else MOE_ERR_UNSUPPORTED. */
+ * 1 <= max_rows <= 4096, and with max_rows > 32 (prefill) d >= 256,
+ * F >= 256 and NVFP4 records only; else MOE_ERR_UNSUPPORTED.  MOE_ERR_ARG for
+ * an unknown format, a BF16 routed format, or (has_shared) a shared format
+ * that is neither the routed one nor BF16. */
 MOE_API moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t host_pool_bytes,
                           const void *router_w, const void *shared_recs, void *workspace,
                           size_t workspace_bytes, void *compute_stream, void *copy_stream,
@@ -203,7 +230,8 @@ MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_a
  * compute_stream reaches that point.  The call waits (host side, bounded) for
  * the device's miss list; on timeout it returns MOE_ERR_TIMEOUT and the
  * context is in MOE_ERR_STATE until a reset.  T <= 32 takes the decode path
- * (W4A16: bf16 activations against NVFP4 weights).  Larger T takes the
+ * (W4A16: bf16 activations against NVFP4 or MXFP4 weights; a BF16 shared
+ * expert runs in its own two launches before the routed ones).  Larger T takes the
  * prefill path: the activations are quantized to NVFP4 per row (E2M1 values,
  * E4M3 scale per 16, one fp32 scale per row: x per token, h per token and
  * expert) and multiplied against the NVFP4 weights (W4A4); the lookup batch is

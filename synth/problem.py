@@ -14,8 +14,20 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (LayerShape, MASTER_SEED, decode_hidden_bf16, expert_record, expert_record_into,
-               record_bytes, replicate_records, router_bf16)
+from . import (LayerShape, MASTER_SEED, decode_hidden_bf16, expert_record, expert_record_bf16,
+               expert_record_into, expert_record_mx, mx_record_layout, record_bytes, replicate_records,
+               router_bf16)
+
+# record formats (the values of the library's MOE_FMT_* constants)
+FMT_NVFP4, FMT_MXFP4, FMT_BF16 = 0, 1, 2
+
+
+def format_record_bytes(fmt: int, d: int, F: int) -> int:
+    if fmt == FMT_MXFP4:
+        return mx_record_layout(d, F)[4]
+    if fmt == FMT_BF16:
+        return 6 * d * F
+    return record_bytes(d, F)
 
 
 def pinned_pool(shape: LayerShape, P: int | None = None, distinct: int | None = None,
@@ -30,6 +42,36 @@ def pinned_pool(shape: LayerShape, P: int | None = None, distinct: int | None = 
     if distinct < P:
         replicate_records(base, rb, distinct, P)
     return pool
+
+
+def pinned_pool_fmt(shape: LayerShape, fmt: int, P: int | None = None, distinct: int | None = None,
+                    seed: int = MASTER_SEED) -> torch.Tensor:
+    """pinned_pool with the records in NVFP4 or MXFP4 (same draws)."""
+    if fmt == FMT_NVFP4:
+        return pinned_pool(shape, P, distinct, seed)
+    P = shape.L * shape.E if P is None else P
+    distinct = P if distinct is None else min(distinct, P)
+    rb = format_record_bytes(fmt, shape.d, shape.F)
+    pool = torch.empty(P * rb, dtype=torch.uint8, pin_memory=True)
+    arr = pool.numpy()
+    for i in range(distinct):
+        arr[i * rb:(i + 1) * rb] = expert_record_mx(i // shape.E, i % shape.E, shape.d, shape.F, seed=seed)
+    if distinct < P:
+        replicate_records(pool.data_ptr(), rb, distinct, P)
+    return pool
+
+
+def shared_records_fmt(shape: LayerShape, fmt: int, seed: int = MASTER_SEED) -> np.ndarray | None:
+    """The L shared-expert records (uint8) in NVFP4, MXFP4 or BF16 (same draws)."""
+    if not shape.shared:
+        return None
+    if fmt == FMT_NVFP4:
+        return shared_records(shape, seed)
+    if fmt == FMT_MXFP4:
+        return np.concatenate([expert_record_mx(l, 0, shape.d, shape.F, shared=True, seed=seed)
+                               for l in range(shape.L)])
+    return np.concatenate([expert_record_bf16(l, 0, shape.d, shape.F, shared=True, seed=seed).view(np.uint8)
+                           for l in range(shape.L)])
 
 
 def router_weights(shape: LayerShape, seed: int = MASTER_SEED) -> np.ndarray:

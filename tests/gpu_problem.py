@@ -36,14 +36,18 @@ class DecodeRun:
 
 class DecodeProblem:
     def __init__(self, shape: synth.LayerShape, T: int, streams: int = 1, P: int | None = None,
-                 distinct: int | None = None, C: int | None = None, stream0: int = 0):
+                 distinct: int | None = None, C: int | None = None, stream0: int = 0,
+                 fmt: int = sp.FMT_NVFP4, shared_fmt: int | None = None):
         self.shape, self.T, self.S = shape, T, streams
+        self.fmt = fmt
+        self.shared_fmt = fmt if shared_fmt is None else shared_fmt
         self.P = shape.L * shape.E if P is None else P
         self.C = shape.cache_slots if C is None else C
-        self.rb = synth.record_bytes(shape.d, shape.F)
+        self.rb = sp.format_record_bytes(fmt, shape.d, shape.F)
+        self.srb = sp.format_record_bytes(self.shared_fmt, shape.d, shape.F)
         self.Wr = sp.router_weights(shape)
-        self.shared = sp.shared_records(shape)
-        self.pool = sp.pinned_pool(shape, self.P, distinct)
+        self.shared = sp.shared_records_fmt(shape, self.shared_fmt)
+        self.pool = sp.pinned_pool_fmt(shape, fmt, self.P, distinct)
         self.pool_np = self.pool.numpy()
         x = np.empty((T, shape.L, streams, shape.d), dtype=np.uint16)
         for s in range(streams):
@@ -68,15 +72,16 @@ class DecodeProblem:
 
     def oracle_y(self, t: int, l: int) -> np.ndarray:
         sh = self.shape
-        shared = None if self.shared is None else self.shared[l * self.rb:(l + 1) * self.rb]
+        shared = None if self.shared is None else self.shared[l * self.srb:(l + 1) * self.srb]
         return oracle.moe_layer(self.pool_np, self.P, l, sh.E, sh.d, sh.F, sh.k, self.Wr[l],
-                                shared, self.x[t, l])[2]
+                                shared, self.x[t, l], fmt=self.fmt, shared_fmt=self.shared_fmt)[2]
 
     # ------------------------------------------------------------- GPU --
     def dims(self):
         sh = self.shape
         return abi.make_dims(sh.L, sh.E, sh.k, sh.d, sh.F, sh.shared, True, self.S,
-                             0 if self.P == sh.L * sh.E else self.P)
+                             0 if self.P == sh.L * sh.E else self.P, weight_format=self.fmt,
+                             shared_format=self.shared_fmt)
 
     def stack(self) -> LayerStack:
         return LayerStack(self.dims(), self.pool, sp.to_device(self.Wr),

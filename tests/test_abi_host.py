@@ -105,3 +105,50 @@ def test_init_argument_checks_without_device():
     assert ei.value.status == abi.MOE_ERR_ARG
     assert abi.moe_record_bytes(abi.make_dims(0, 16, 2, 256, 512)) == 0
     assert abi.moe_status_str(abi.MOE_ERR_TIMEOUT) == "timed out waiting for the device"
+
+
+@pytest.mark.parametrize("shape", list(synth.SHAPES.values()), ids=lambda s: s.name)
+def test_mxfp4_and_bf16_record_layouts(shape):
+    """MXFP4 routed records and BF16 shared records: the ABI's offsets and sizes
+    agree with the oracle's and the generator's layouts."""
+    d = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, True,
+                      weight_format=abi.MOE_FMT_MXFP4)
+    off = oracle.mx_record_layout(shape.d, shape.F)
+    assert synth.mx_record_layout(shape.d, shape.F) == off
+    assert abi.moe_record_layout(d) == (off[0], off[1], off[2], off[3], -1, off[4])
+    assert abi.moe_record_bytes(d) == off[4]
+    assert abi.moe_shared_record_bytes(d) == off[4]  # shared format = routed format
+    for wf in (abi.MOE_FMT_NVFP4, abi.MOE_FMT_MXFP4):
+        db = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, True,
+                           weight_format=wf, shared_format=abi.MOE_FMT_BF16)
+        assert abi.moe_shared_record_bytes(db) == 2 * 3 * shape.d * shape.F
+        assert synth.expert_record_bf16(0, 0, shape.d, shape.F).nbytes == 6 * shape.d * shape.F
+    nv = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, True)
+    assert abi.moe_shared_record_bytes(nv) == abi.moe_record_bytes(nv)
+
+
+def test_format_argument_checks_without_device():
+    fake = 0x1000
+    bad = [abi.make_dims(2, 16, 2, 256, 512, weight_format=abi.MOE_FMT_BF16),  # BF16 routed
+           abi.make_dims(2, 16, 2, 256, 512, weight_format=7),
+           abi.make_dims(2, 16, 2, 256, 512, True, weight_format=abi.MOE_FMT_MXFP4,
+                         shared_format=abi.MOE_FMT_NVFP4)]  # shared neither routed nor BF16
+    for d in bad:
+        assert abi.moe_record_bytes(d) == 0 and abi.moe_shared_record_bytes(d) == 0
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_layer_init(d, fake, 1 << 30, fake, fake, fake, 1 << 30, fake, fake)
+        assert ei.value.status == abi.MOE_ERR_ARG
+    # no shared expert: the shared format is not looked at
+    ok = abi.make_dims(2, 16, 2, 256, 512, False, weight_format=abi.MOE_FMT_MXFP4,
+                       shared_format=abi.MOE_FMT_NVFP4)
+    assert abi.moe_record_bytes(ok) == oracle.mx_record_layout(256, 512)[4]
+    # MXFP4 and BF16 records run on the decode path only
+    for wf, sf in ((abi.MOE_FMT_MXFP4, None), (abi.MOE_FMT_NVFP4, abi.MOE_FMT_BF16)):
+        pre = abi.make_dims(2, 16, 2, 256, 512, True, max_rows=64, weight_format=wf, shared_format=sf)
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_layer_init(pre, fake, 1 << 30, fake, fake, fake, 1 << 40, fake, fake)
+        assert ei.value.status == abi.MOE_ERR_UNSUPPORTED
+        dec = abi.make_dims(2, 16, 2, 256, 512, True, max_rows=32, weight_format=wf, shared_format=sf)
+        with pytest.raises(abi.MoeError) as ei:  # accepted shape; then the fake pool is refused
+            abi.moe_layer_init(dec, fake, 1 << 30, fake, fake, fake, 1 << 40, fake, fake)
+        assert ei.value.status == abi.MOE_ERR_NOT_PINNED
