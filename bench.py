@@ -425,7 +425,7 @@ def bench_decode(args, shape, rank, world, local):
         steady_line = {"from_token": steady["t0"], "unit": "tok/s",
                        "value": sum_over_ranks(float(args.steps - steady["t0"]), world) / s_max}
 
-    # roofline of the step (the benchmark spec): max(hit bytes / HBM BW, miss bytes / H2D BW)
+    # roofline of the step: max(hit bytes / HBM BW, miss bytes / H2D BW)
     hbm_peak, peak_kind = measured_peaks()
     hit_bytes = (st.hits + (st.forward_calls if shape.shared else 0)) * rb
     miss_bytes = st.misses * rb
