@@ -160,7 +160,6 @@ __device__ __forceinline__ void step_mma_mx(const uint8_t *cA, const uint8_t *cB
 constexpr int kMaxSteps = 16;  // K <= 4096: at most 16 K-steps of 256, one per warp
 constexpr int kGStages = 3;                           // tiles in flight per CTA
 constexpr int kMaxSlots = kMaxK * kDecodeMaxRows + 1;  // job slots of a launch (+ shared)
-constexpr int kSmCount = 148;
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
@@ -174,9 +173,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
                  : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // One K-step of one thread: 32 code bytes of each of its two tile rows (from
