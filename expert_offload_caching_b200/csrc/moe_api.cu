@@ -537,7 +537,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     return MOE_OK;
 }
 
-// One layer of a prefill chunk (T > 32 rows): W4A4 through the expert GEMV,
+// One layer of a prefill chunk (T > 32 rows): W4A4 grouped tensor-core GEMMs,
 // with the next layer's experts prefetched when MOE_CACHE_PREFETCH_NEXT is set.
 moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
                            moe_layer_trace *trace) {
@@ -966,6 +966,9 @@ moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t
     const moe_status st = T <= kDecodeMaxRows ? forward_decode(ctx, layer, x, T, y, trace)
                                               : forward_prefill(ctx, layer, x, T, y, trace);
     ctx->stats.host_us[0] += std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - t0).count();
+    // a failure after the lookup may leave slots assigned whose copies were
+    // never issued: nothing may run on this cache until a reset
+    if (st != MOE_OK) ctx->state = MOE_ERR_STATE;
     return st;
 }
 

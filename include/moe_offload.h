@@ -241,7 +241,11 @@ MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_a
  * with consecutive pool indices and slots go in one copy).  The expert FFNs
  * of a prefill call run as grouped block-scaled NVFP4 GEMMs on the tensor
  * cores (rows grouped by expert, fp32 accumulation).  The trace lists the
- * routed entries, then the prefetch entries (prefetch = 1, layer + 1). */
+ * routed entries, then the prefetch entries (prefetch = 1, layer + 1).
+ * Any failure after the argument checks (MOE_ERR_CUDA, MOE_ERR_TIMEOUT, a
+ * failed device check) leaves the context in MOE_ERR_STATE until
+ * cache_configure(..., MOE_CACHE_RESET): the lookup may have assigned slots
+ * whose copies were not issued. */
 MOE_API moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
                              moe_layer_trace *trace);
 
