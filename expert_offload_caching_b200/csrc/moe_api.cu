@@ -899,6 +899,9 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         }
     }
     if (reset) {
+        // unusable until the reset below completes (a failed step returns with
+        // configured = false, so forward calls refuse to run on a half-reset table)
+        ctx->configured = false;
         // finish outstanding work of the old state first
         CK(cudaStreamSynchronize(ctx->xs));
         CK(cudaStreamSynchronize(ctx->cs));
