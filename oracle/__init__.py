@@ -89,6 +89,8 @@ def lib():
         L.orc_dequant_matrix_mx.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
         L.orc_expert_mx_w4a16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp]
         L.orc_expert_bf16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp]
+        L.orc_mx_quantize.argtypes = [vp, ctypes.c_int64, vp, vp]
+        L.orc_expert_mx_w4a4.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, vp]
         L.orc_moe_layer_fmt.argtypes = [vp, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp]
@@ -204,6 +206,23 @@ def expert_mx_w4a16(rec: np.ndarray, d: int, F: int, x: np.ndarray) -> np.ndarra
     y = np.empty(d, dtype=np.float64)
     lib().orc_expert_mx_w4a16(_p(np.ascontiguousarray(rec)), d, F,
                               _p(np.ascontiguousarray(x, dtype=np.uint16)), _p(y))
+    return y
+
+
+def mx_quantize(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP4 codes (n/2 bytes) and E8M0 scales (n/32) of fp32 values (OCP rule)."""
+    x = np.ascontiguousarray(x, dtype=np.float32).ravel()
+    codes = np.empty(x.size // 2, dtype=np.uint8)
+    scales = np.empty(x.size // 32, dtype=np.uint8)
+    lib().orc_mx_quantize(_p(x), x.size, _p(codes), _p(scales))
+    return codes, scales
+
+
+def expert_mx_w4a4(rec: np.ndarray, d: int, F: int, x: np.ndarray) -> np.ndarray:
+    """One expert over an MXFP4 record on one bf16 row, activations MXFP4-quantized (prefill)."""
+    y = np.empty(d, dtype=np.float64)
+    lib().orc_expert_mx_w4a4(_p(np.ascontiguousarray(rec)), d, F,
+                             _p(np.ascontiguousarray(x, dtype=np.uint16)), _p(y))
     return y
 
 

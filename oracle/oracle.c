@@ -416,6 +416,82 @@ EXPORT void orc_expert_w4a4(const uint8_t *rec, int d, int F, const uint16_t *x,
     free(xf); free(xc); free(xs); free(xv); free(hf); free(hc); free(hs);
 }
 
+/* ------------------------------------------ MXFP4 activation quantizer -- */
+/* OCP microscaling, per block of 32 consecutive values: shared exponent
+ * e = floor(log2(amax)) - 2 (2 = the largest E2M1 exponent), clamped to
+ * [-127, 127], stored as the E8M0 code e + 127; element code = E2M1 of
+ * x / 2^e, RNE, saturating to +-6.  An all-zero block gets code 0 and zero
+ * elements.  Every step is exact in fp32 (amax, the exponent, the division by
+ * a power of two), so the codes do not depend on the precision it runs in.
+ * n a multiple of 32; codes n/2 bytes (element 2i in the low nibble), scales n/32. */
+EXPORT void orc_mx_quantize(const float *x, int64_t n, uint8_t *codes, uint8_t *scales) {
+    for (int64_t b = 0; b < n / 32; ++b) {
+        const float *blk = x + b * 32;
+        float amax = 0.0f;
+        for (int j = 0; j < 32; ++j) {
+            float a = fabsf(blk[j]);
+            if (a > amax) amax = a;
+        }
+        int e = -127;
+        if (amax > 0.0f) {
+            int ex;
+            frexpf(amax, &ex); /* amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1 */
+            e = ex - 1 - 2;
+            if (e < -127) e = -127;
+            if (e > 127) e = 127;
+        }
+        scales[b] = (uint8_t)(e + 127);
+        for (int j = 0; j < 16; ++j) {
+            int lo = 0, hi = 0;
+            if (amax > 0.0f) {
+                lo = orc_e2m1_rne(ldexpf(blk[2 * j], -e));
+                hi = orc_e2m1_rne(ldexpf(blk[2 * j + 1], -e));
+            }
+            codes[b * 16 + j] = (uint8_t)(lo | (hi << 4));
+        }
+    }
+}
+
+static double dq_act_mx(const uint8_t *codes, const uint8_t *scales, int64_t i) {
+    int code = (i % 2 == 0) ? (codes[i / 2] & 0xF) : (codes[i / 2] >> 4);
+    return orc_e2m1(code) * orc_e8m0(scales[i / 32]);
+}
+
+/* W4A4 expert over an MXFP4 record for one row (the prefill path with MXFP4
+ * records): x is MXFP4-quantized per block of 32, the products are taken in
+ * fp64, h is rounded to fp32 and MXFP4-quantized before the down projection
+ * (the same steps as the NVFP4 W4A4 expert, with E8M0 block scales and no
+ * row scale). */
+EXPORT void orc_expert_mx_w4a4(const uint8_t *rec, int d, int F, const uint16_t *x, double *y) {
+    int64_t off[5];
+    orc_mx_record_layout(d, F, off);
+    float *xf = (float *)malloc(sizeof(float) * d);
+    uint8_t *xc = (uint8_t *)malloc((size_t)d / 2), *xs = (uint8_t *)malloc((size_t)d / 32);
+    double *xv = (double *)malloc(sizeof(double) * d);
+    for (int K = 0; K < d; ++K) xf[K] = (float)bf16_val(x[K]);
+    orc_mx_quantize(xf, d, xc, xs);
+    for (int K = 0; K < d; ++K) xv[K] = dq_act_mx(xc, xs, K);
+    float *hf = (float *)malloc(sizeof(float) * F);
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < F; ++j) {
+        double g = 0.0, u = 0.0;
+        for (int64_t K = 0; K < d; ++K) {
+            g += dq_mx(rec + off[0], rec + off[1], d, 2 * j, K) * xv[K];
+            u += dq_mx(rec + off[0], rec + off[1], d, 2 * j + 1, K) * xv[K];
+        }
+        hf[j] = (float)(silu(g) * u);
+    }
+    uint8_t *hc = (uint8_t *)malloc((size_t)F / 2), *hs = (uint8_t *)malloc((size_t)F / 32);
+    orc_mx_quantize(hf, F, hc, hs);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int64_t j = 0; j < F; ++j) acc += dq_mx(rec + off[2], rec + off[3], F, i, j) * dq_act_mx(hc, hs, j);
+        y[i] = acc;
+    }
+    free(xf); free(xc); free(xs); free(xv); free(hf); free(hc); free(hs);
+}
+
 /* ------------------------------------------------------------ one layer -- */
 /* Record of (layer, expert) in a host pool of P records: index (layer*E + expert) mod P. */
 static const uint8_t *pool_record(const uint8_t *pool, int64_t P, int64_t rec_bytes, int layer,
@@ -423,10 +499,11 @@ static const uint8_t *pool_record(const uint8_t *pool, int64_t P, int64_t rec_by
     return pool + (((int64_t)layer * E + e) % P) * rec_bytes;
 }
 
-/* One expert on one bf16 row in the record's format: 0 NVFP4 (W4A16, or W4A4
- * with w4a4), 1 MXFP4 (W4A16), 2 BF16. */
+/* One expert on one bf16 row in the record's format: 0 NVFP4, 1 MXFP4 (W4A16,
+ * or W4A4 with w4a4), 2 BF16 (weights and activations as they are, both paths). */
 static void expert_fmt(const uint8_t *rec, int fmt, int w4a4, int d, int F, const uint16_t *x, double *y) {
-    if (fmt == 1) orc_expert_mx_w4a16(rec, d, F, x, y);
+    if (fmt == 1 && w4a4) orc_expert_mx_w4a4(rec, d, F, x, y);
+    else if (fmt == 1) orc_expert_mx_w4a16(rec, d, F, x, y);
     else if (fmt == 2) orc_expert_bf16((const uint16_t *)rec, d, F, x, y);
     else if (w4a4) orc_expert_w4a4(rec, d, F, x, y);
     else orc_expert_w4a16(rec, d, F, x, y, NULL);
@@ -436,12 +513,13 @@ static void expert_fmt(const uint8_t *rec, int fmt, int w4a4, int d, int F, cons
  * y = sum over selected e in ascending id of g_e * E_e(x) + S(x).
  * fmt: the routed records' format (0 NVFP4, 1 MXFP4); shared_fmt: the shared
  * record's (0, 1 or 2 BF16).  w4a4 = 0: decode path (W4A16); 1: prefill path
- * (W4A4, NVFP4 records only).  shared_rec may be NULL (no shared expert). */
+ * (W4A4: NVFP4 or MXFP4 activations to match the records; a BF16 shared
+ * expert is not quantized).  shared_rec may be NULL (no shared expert). */
 EXPORT int orc_moe_layer_fmt(const uint8_t *pool, int64_t P, int layer, int E, int d, int F, int k,
                              int renorm, const uint16_t *Wr_layer, const uint8_t *shared_rec,
                              const uint16_t *x, int T, int w4a4, int fmt, int shared_fmt, int32_t *idx,
                              double *gates, double *y) {
-    if (fmt < 0 || fmt > 1 || shared_fmt < 0 || shared_fmt > 2 || (w4a4 && (fmt || shared_fmt))) return 1;
+    if (fmt < 0 || fmt > 1 || shared_fmt < 0 || shared_fmt > 2 || (shared_fmt != fmt && shared_fmt != 2)) return 1;
     int64_t off[6];
     if (fmt == 1) orc_mx_record_layout(d, F, off);
     else orc_record_layout(d, F, off);

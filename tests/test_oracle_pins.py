@@ -615,5 +615,91 @@ def test_layer_with_mxfp4_records_and_bf16_shared_matches_numpy():
                 if srec is not None:
                     want = want + sfun(srec, xv)
                 np.testing.assert_allclose(y[t], want, rtol=1e-11, atol=1e-14)
-    with pytest.raises(ValueError):  # W4A4 is the NVFP4 prefill path only
-        oracle.moe_layer(pool, L * E, 1, E, d, F, k, Wr, None, x, w4a4=True, fmt=oracle.FMT_MXFP4)
+    with pytest.raises(ValueError):  # a shared record neither in the routed format nor BF16
+        oracle.moe_layer(pool, L * E, 1, E, d, F, k, Wr, shared_mx, x, fmt=oracle.FMT_MXFP4,
+                         shared_fmt=oracle.FMT_NVFP4)
+    # the prefill path (W4A4): MXFP4 activations for MXFP4 records, a BF16 shared
+    # expert unquantized
+    for srec, sfmt, sfun in ((shared_mx, oracle.FMT_MXFP4, oracle.expert_mx_w4a4),
+                             (shared_bf, oracle.FMT_BF16, oracle.expert_bf16)):
+        idx, g, y = oracle.moe_layer(pool, L * E, 1, E, d, F, k, Wr, srec, x, w4a4=True,
+                                     fmt=oracle.FMT_MXFP4, shared_fmt=sfmt)
+        for t in range(3):
+            want = sum(g[t, j] * oracle.expert_mx_w4a4(pool[(E + idx[t, j]) * rb:][:rb], d, F, x[t])
+                       for j in range(k))
+            np.testing.assert_allclose(y[t], want + sfun(srec, d, F, x[t]), rtol=1e-11, atol=1e-14)
+
+
+# ------------------------------------------- MXFP4 activations (prefill) --
+def test_mx_quantizer_reproduces_the_worked_block():
+    """The oracle's MXFP4 activation quantizer gives the hand-derived codes and scale."""
+    rows = _rows("mxfp4_worked_block.txt")
+    x = np.zeros(32, dtype=np.float32)
+    want = np.zeros(32, dtype=np.int64)
+    for r in rows[1:]:
+        x[int(r[0])] = float(r[1])
+        want[int(r[0])] = int(r[2], 16)
+    codes, scales = oracle.mx_quantize(x)
+    got = np.empty(32, dtype=np.int64)
+    got[0::2], got[1::2] = codes & 0xF, codes >> 4
+    np.testing.assert_array_equal(got, want)
+    assert scales[0] == int(rows[0][1], 16)
+
+
+def test_mx_quantizer_matches_the_generators_encoder():
+    """Two implementations of the OCP rule (the oracle's and the input
+    generator's, no shared code) agree bit for bit, including zero blocks,
+    -0, fp32 subnormals, huge values and exact E2M1 midpoints."""
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-30, 30, (64, 1)))).astype(np.float32)
+    x[0, :32] = 0.0
+    x[1, :32] = -0.0
+    x[2, :32] = np.float32(1e-42) * rng.integers(1, 100, 32)
+    x[3, :32] = np.float32(3e38) * rng.uniform(-1, 1, 32)
+    x[4, :32] = np.array([4.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0] * 4, dtype=np.float32)
+    codes, scales = oracle.mx_quantize(x)
+    c2, s2 = synth.mx_encode(x)
+    np.testing.assert_array_equal(codes, c2.ravel())
+    np.testing.assert_array_equal(scales, s2.ravel())
+
+
+def test_mx_quantizer_round_trip_of_representable_blocks():
+    """A block of E2M1 values times 2^e whose largest magnitude is 4 or 6 times
+    2^e quantizes to itself (codes and scale 127 + e)."""
+    rng = np.random.default_rng(32)
+    for e in (-127, -60, -3, 0, 5, 120):
+        for top in (6, 7):  # a 4 or a 6 in the block: amax in [4, 8) * 2^e
+            codes = rng.integers(0, 16, 32)
+            codes[rng.integers(32)] = top
+            vals = np.array([E2M1_GOLDEN[c] for c in codes]) * 2.0 ** e
+            q, s = oracle.mx_quantize(vals.astype(np.float32))
+            got = np.empty(32, dtype=np.int64)
+            got[0::2], got[1::2] = q & 0xF, q >> 4
+            assert s[0] == 127 + e
+            np.testing.assert_array_equal(np.array([E2M1_GOLDEN[c] for c in got]),
+                                          np.array([E2M1_GOLDEN[c] for c in codes]))
+
+
+def test_mx_w4a4_expert_matches_its_steps_in_numpy():
+    """The MXFP4 prefill expert: x quantized per block of 32, fp64 products,
+    h rounded to fp32 and quantized, then the down projection."""
+    d, F = 256, 128
+    rec = synth.expert_record_mx(3, 5, d, F)
+    x = _bf16_bits(np.random.default_rng(33).normal(0, 1, d))
+    tab = np.array([E2M1_GOLDEN[c] for c in range(16)])
+
+    def deq(codes, scales):
+        v = np.empty(codes.size * 2)
+        v[0::2], v[1::2] = tab[codes & 0xF], tab[codes >> 4]
+        return v * np.repeat(2.0 ** (scales.astype(np.float64) - 127), 32)
+
+    silu = lambda v: v * expit(v)  # noqa: E731
+    xv = deq(*oracle.mx_quantize(_bf16_val(x).astype(np.float32)))
+    g = oracle.dequant_matrix_mx(rec, d, F, 0) @ xv
+    u = oracle.dequant_matrix_mx(rec, d, F, 1) @ xv
+    hv = deq(*oracle.mx_quantize((silu(g) * u).astype(np.float32)))
+    want = oracle.dequant_matrix_mx(rec, d, F, 2) @ hv
+    np.testing.assert_allclose(oracle.expert_mx_w4a4(rec, d, F, x), want, rtol=1e-11, atol=1e-14)
+    # and the quantization costs what 4-bit activations cost, no more
+    exact = oracle.expert_mx_w4a16(rec, d, F, x)
+    assert 0 < np.linalg.norm(want - exact) / np.linalg.norm(exact) < 0.3
