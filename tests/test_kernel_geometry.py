@@ -129,3 +129,49 @@ def test_grouped_gemm_pair_capacity_bounds_the_tile_plan(seed):
         need = int(np.sum((jobs + 127) // 128)) + (shared * ((T + 127) // 128))
         cap = len(jobs) + (T * k + 127) // 128 + (shared * ((T + 127) // 128))
         assert need <= cap
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: s.name)
+def test_mxfp4_tile_copies_and_scale_reads(shape):
+    """The GEMV's MXFP4 instantiation: a 16-row tile stages 16 * K/2 code bytes
+    and 16 * K/32 = K/2 scale bytes; both copies lie inside their record
+    sections on 16-byte boundaries; a thread's two E8M0 bytes of chunk c of
+    tile row r (a 16-bit read at r * K/32 + 2c) are aligned and inside the
+    staged scales; shared memory fits."""
+    dims = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, shape.shared,
+                         weight_format=abi.MOE_FMT_MXFP4)
+    off = abi.moe_record_layout(dims)
+    assert off[4] == -1 and all(o % 256 == 0 for i, o in enumerate(off) if i != 4)
+    for K, tiles, codes0, scales0, end in ((shape.d, shape.F // 8, off[0], off[1], off[2]),
+                                           (shape.F, shape.d // 16, off[2], off[3], off[5])):
+        code_bytes, scale_bytes = 16 * (K // 2), K // 2
+        assert code_bytes % 16 == 0 and scale_bytes % 16 == 0
+        nsteps = (K // 64 + 3) // 4
+        spw = 2 if nsteps >= 8 else 1
+        warps = (nsteps + spw - 1) // spw
+        assert 3 * (code_bytes + scale_bytes) + 2 * warps * 2 * 512 <= 160 * 1024
+        for t in (0, tiles - 1):
+            assert (codes0 + t * code_bytes) % 16 == 0 and (scales0 + t * scale_bytes) % 16 == 0
+            assert codes0 + (t + 1) * code_bytes <= scales0
+            assert scales0 + (t + 1) * scale_bytes <= end
+        nch = K // 64
+        for r in (0, 7, 8, 15):
+            for c in (0, nch - 1):
+                o = r * (K // 32) + 2 * c
+                assert o % 2 == 0 and o + 2 <= scale_bytes
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: s.name)
+def test_bf16_shared_reads_inside_record(shape):
+    """The BF16 shared-expert GEMV: warp j of gate/up reads W13 rows 2j, 2j+1 in
+    16-byte chunks, warp i of down reads W2 rows 2i, 2i+1; all inside the 6dF
+    bytes of the record and 16-byte aligned (the record's pitch keeps them)."""
+    d, F = shape.d, shape.F
+    dims = abi.make_dims(shape.L, shape.E, shape.k, d, F, True, shared_format=abi.MOE_FMT_BF16)
+    rb = abi.moe_shared_record_bytes(dims)
+    assert rb == 6 * d * F and rb % 16 == 0
+    for K, rows, base in ((d, 2 * F, 0), (F, d, 4 * F * d)):
+        nch = K // 8
+        last_row = base + (rows - 1) * K * 2
+        assert base % 16 == 0 and (K * 2) % 16 == 0
+        assert last_row + 16 * (nch - 1) + 16 <= (4 * F * d if base == 0 else rb)
