@@ -175,3 +175,55 @@ def test_bf16_shared_reads_inside_record(shape):
         last_row = base + (rows - 1) * K * 2
         assert base % 16 == 0 and (K * 2) % 16 == 0
         assert last_row + 16 * (nch - 1) + 16 <= (4 * F * d if base == 0 else rb)
+
+
+def test_mxfp4_step_factoring_keeps_products_exact():
+    """(Imports the oracle: test infrastructure.)  A numpy model of the MXFP4 GEMV's arithmetic (per 256-value K-step and
+    row: the largest E8M0 code c_max factored out, weights e2m1 * 2^(c - c_max
+    + 12) rounded to fp16, activations as fp16 (hi, lo), fp32 step sums scaled
+    by 2^(c_max - 139)) against the oracle's fp64 expert, on scales spread by
+    25 codes inside a step with some blocks 80+ codes below: the products stay
+    exact, so only fp32 summation separates the two."""
+    import numpy as np
+    import oracle
+    import synth
+
+    d, F = 320, 192
+    rng = np.random.default_rng(41)
+    rec = synth.expert_record_mx(0, 3, d, F).copy()
+    off = synth.mx_record_layout(d, F)
+    for start, n in ((off[1], 2 * F * d // 32), (off[3], d * F // 32)):
+        c = rng.integers(99, 125, n)
+        tiny = rng.random(n) < 0.02
+        c[tiny] = rng.integers(20, 41, int(tiny.sum()))
+        rec[start:start + n] = c.astype(np.uint8)
+    tab = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, 0, -.5, -1, -1.5, -2, -3, -4, -6])
+
+    def gemv(codes, scales, K, act):
+        v = np.empty((codes.shape[0], K))
+        v[:, 0::2], v[:, 1::2] = tab[codes & 0xF], tab[codes >> 4]
+        hi = act.astype(np.float16)
+        lo = (act - hi.astype(np.float32)).astype(np.float16)
+        out = np.zeros(codes.shape[0], np.float32)
+        for k0 in range(0, K, 256):
+            k1 = min(K, k0 + 256)
+            sc = scales[:, k0 // 32:(k1 + 31) // 32].astype(np.int64)
+            cmax = sc.max(axis=1)
+            w = (v[:, k0:k1] * np.exp2(np.repeat(sc - cmax[:, None], 32, axis=1)[:, :k1 - k0] + 12.0))
+            w16 = w.astype(np.float16).astype(np.float64)
+            assert np.array_equal(w16[np.abs(w) >= 2.0 ** -24], w[np.abs(w) >= 2.0 ** -24])  # exact
+            stp = (w16 @ hi[k0:k1].astype(np.float64) + w16 @ lo[k0:k1].astype(np.float64)).astype(np.float32)
+            out = out + stp * np.exp2(cmax - 139.0).astype(np.float32)
+        return out
+
+    x = synth.to_bf16(rng.normal(0, 1, d).astype(np.float32))
+    xf = synth.bf16_to_f32(x).astype(np.float32)
+    c13 = rec[off[0]:off[0] + F * d].reshape(2 * F, d // 2)
+    s13 = rec[off[1]:off[1] + 2 * F * d // 32].reshape(2 * F, d // 32)
+    gu = gemv(c13, s13, d, xf)
+    g, u = gu[0::2], gu[1::2]
+    h = (g / (1 + np.exp(-g)) * u).astype(np.float32)
+    y = gemv(rec[off[2]:off[2] + d * F // 2].reshape(d, F // 2),
+             rec[off[3]:off[3] + d * F // 32].reshape(d, F // 32), F, h)
+    want = oracle.expert_mx_w4a16(rec, d, F, x)
+    assert np.linalg.norm(y - want) / np.linalg.norm(want) < 1e-6
