@@ -152,3 +152,44 @@ def test_format_argument_checks_without_device():
         with pytest.raises(abi.MoeError) as ei:  # accepted shape; then the fake pool is refused
             abi.moe_layer_init(dec, fake, 1 << 30, fake, fake, fake, 1 << 40, fake, fake)
         assert ei.value.status == abi.MOE_ERR_NOT_PINNED
+
+
+def test_size_queries_and_init_checks_over_random_dims():
+    """Random dims, valid and not: the size queries return 0 exactly for
+    invalid dims, grow with the slot count, and cover the layout; init with
+    fake pointers answers ARG, UNSUPPORTED or NOT_PINNED (never touching them)."""
+    rng = np.random.default_rng(51)
+    fake = 0x1000
+    seen = set()
+    for _ in range(400):
+        L = int(rng.choice([0, 1, 2, 48, 64]))
+        E = int(rng.choice([0, 1, 16, 256, 512, 1024, 2048]))
+        k = int(rng.choice([0, 1, 4, 10, 32, 33]))
+        d = int(rng.choice([0, 64, 192, 250, 2048, 2880, 4096, 8192]))
+        F = int(rng.choice([0, 64, 768, 2880, 4096, 5000]))
+        rows = int(rng.choice([0, 1, 32, 33, 4096, 5000]))
+        wf = int(rng.choice([0, 1, 2, 3]))
+        sf = int(rng.choice([0, 1, 2]))
+        sh = bool(rng.integers(2))
+        dims = abi.make_dims(L, E, k, d, F, sh, True, rows, 0, weight_format=wf, shared_format=sf)
+        valid = (L > 0 and E > 0 and 0 < k <= E and d > 0 and F > 0 and rows > 0 and wf in (0, 1)
+                 and (not sh or sf in (wf, 2)))
+        rb = abi.moe_record_bytes(dims)
+        assert (rb > 0) == valid
+        if not valid:
+            assert abi.moe_workspace_bytes(dims) == 0 and abi.moe_arena_bytes(dims, 8) == 0
+            with pytest.raises(abi.MoeError) as ei:
+                abi.moe_layer_init(dims, fake, 1 << 40, fake, fake, fake, 1 << 40, fake, fake)
+            assert ei.value.status == abi.MOE_ERR_ARG
+            seen.add("arg")
+            continue
+        off = abi.moe_record_layout(dims)
+        assert off[5] == rb and max(off[:5]) < rb
+        assert abi.moe_workspace_bytes(dims) > 0
+        a8, a16 = abi.moe_arena_bytes(dims, 8), abi.moe_arena_bytes(dims, 16)
+        assert a16 - a8 >= 8 * rb
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_layer_init(dims, fake, 1 << 50, fake, fake, fake, 1 << 50, fake, fake)
+        assert ei.value.status in (abi.MOE_ERR_UNSUPPORTED, abi.MOE_ERR_NOT_PINNED)
+        seen.add(ei.value.status)
+    assert seen >= {"arg", abi.MOE_ERR_UNSUPPORTED, abi.MOE_ERR_NOT_PINNED}
