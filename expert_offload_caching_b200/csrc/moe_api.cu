@@ -965,6 +965,8 @@ moe_status moe_layer_forward(moe_ctx *ctx, int32_t layer, const void *x, int32_t
     if (!ctx->configured) return MOE_ERR_STATE;
     const moe_dims &D = ctx->dims;
     if (layer < 0 || layer >= D.L || T < 1 || T > D.max_rows || !x || !y) return MOE_ERR_ARG;
+    // x rows are read as 16-byte vectors (and as TMA boxes in prefill); y as floats
+    if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(y) & 3)) return MOE_ERR_ARG;
     const auto t0 = std::chrono::steady_clock::now();
     const moe_status st = T <= kDecodeMaxRows ? forward_decode(ctx, layer, x, T, y, trace)
                                               : forward_prefill(ctx, layer, x, T, y, trace);

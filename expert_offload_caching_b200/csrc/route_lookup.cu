@@ -79,6 +79,22 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// A selected id outside [0, E) (the selection is total, so this is a broken
+// invariant, not an input case): record it in the mapped page; the caller
+// skips the access and the host turns the error word into MOE_ERR_CUDA.
+constexpr int kCheckExpertRange = 30;
+__device__ void route_fail(HostPage *page, int mode, int e, int E) {
+    page->diag[1] = mode;
+    page->diag[2] = (int)blockIdx.x;
+    page->diag[3] = 0;
+    page->diag[4] = (int)threadIdx.x;
+    page->diag[5] = e;
+    page->diag[6] = E;
+    __threadfence_system();
+    page->error = kCheckExpertRange;
+    __threadfence_system();
+}
+
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -144,16 +160,23 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
 // Softmax + top-k of row t by one warp; writes idx/gates of the row in ascending
 // id and returns the expert selected by this lane (lanes < k), else -1.
 // NVE: 32-wide chunks of the row held in registers (E <= 32 * NVE).
+// The order is total: a NaN logit counts as -inf, equal values go to the lower
+// id, and a picked entry is masked out by a bit (not by overwriting its value),
+// so k distinct ids in [0, E) come out whatever the logits hold.
 template <int NVE>
 __device__ int topk_row_n(const RouteArgs &a, int t) {
     const int lane = threadIdx.x & 31;
     const float *z = a.ws.z + (size_t)t * a.E;
     const int nv = (a.E + 31) >> 5;
     float v[NVE];
+    uint32_t avail = 0u;  // bit j: entry lane + 32 j is a real expert not yet picked
 #pragma unroll
     for (int j = 0; j < NVE; ++j) {
         const int e = lane + 32 * j;
-        v[j] = (j < nv && e < a.E) ? z[e] : -INFINITY;
+        const bool real = j < nv && e < a.E;
+        const float zv = real ? z[e] : -INFINITY;
+        v[j] = zv != zv ? -INFINITY : zv;
+        if (real) avail |= 1u << j;
     }
     float m = -INFINITY;
 #pragma unroll
@@ -171,12 +194,10 @@ __device__ int topk_row_n(const RouteArgs &a, int t) {
     float my_val = -INFINITY;
     for (int s = 0; s < a.k; ++s) {
         float bv = -INFINITY;
-        int bi = 0x7fffffff;
+        int bi = 0x7fffffff;  // lane-local candidates are visited in ascending id
 #pragma unroll
-        for (int j = 0; j < NVE; ++j) {
-            const int e = lane + 32 * j;
-            if (e < a.E && v[j] > bv) { bv = v[j]; bi = e; }
-        }
+        for (int j = 0; j < NVE; ++j)
+            if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = lane + 32 * j; }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -184,10 +205,7 @@ __device__ int topk_row_n(const RouteArgs &a, int t) {
             if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
         }
         if (lane == s) { my_idx = bi; my_val = bv; }
-        const int owner = bi & 31, slotj = bi >> 5;
-#pragma unroll
-        for (int j = 0; j < NVE; ++j)
-            if (lane == owner && j == slotj) v[j] = -INFINITY;
+        if (bi < a.E && lane == (bi & 31)) avail &= ~(1u << (bi >> 5));
     }
     const float top = __shfl_sync(0xffffffffu, my_val, 0);
     float g;
@@ -442,7 +460,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
         const int e = a.ws.idx[i];
         s_idx[i] = e;
-        atomicOr(&s_bits[e >> 5], 1u << (e & 31));
+        if ((unsigned)e < (unsigned)a.E) atomicOr(&s_bits[e >> 5], 1u << (e & 31));
+        else route_fail(a.page, 1, e, a.E);
     }
     __syncthreads();
     if (warp == 0) {
@@ -613,7 +632,8 @@ __global__ void __launch_bounds__(kRouteThreads) prefill_topk_kernel(RouteArgs a
     const int t = blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5);
     if (t >= a.T) return;
     const int e = topk_row(a, t);
-    if (e >= 0) atomicAdd(&a.ws.cnt[e], 1);
+    if ((unsigned)e < (unsigned)a.E) atomicAdd(&a.ws.cnt[e], 1);
+    else if ((threadIdx.x & 31) < a.k) route_fail(a.page, 2, e, a.E);
 }
 
 __global__ void __launch_bounds__(kRouteThreads) prefill_lookup_kernel(RouteArgs a) {
@@ -698,7 +718,9 @@ __global__ void prefill_scatter_kernel(RouteArgs a) {
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= a.T * a.k) return;
     const int e = a.ws.idx[i];
+    if ((unsigned)e >= (unsigned)a.E) { route_fail(a.page, 3, e, a.E); return; }
     const int j = a.ws.jobidx[e];
+    if (j < 0) { route_fail(a.page, 4, e, a.E); return; }
     const int pos = a.ws.jobs[j].row_off + atomicAdd(&a.ws.fill[e], 1);
     a.ws.rowrefs[pos].t = (int16_t)(i / a.k);
     a.ws.rowrefs[pos].p = (int16_t)(i % a.k);

@@ -19,8 +19,8 @@
 //
 // What it computes matches the routing part of moe_layer_forward: z = W_r x
 // (bf16 inputs, fp32 accumulation), p = softmax(z), the k largest logits with
-// ties to the lower id, gates renormalised over the k (or the plain softmax
-// probabilities), ids in ascending order.
+// ties to the lower id and NaN logits counted as -inf, gates renormalised over
+// the k (or the plain softmax probabilities), ids in ascending order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -98,13 +98,15 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
     if (!s_last) return;
     __threadfence();
 
+    // a NaN logit counts as -inf (selection and softmax), as in moe_layer_forward
     for (int t = warp; t < T; t += nw) {
         const float *zr = z + (size_t)t * E;
+        auto zval = [&](int e) { const float v = zr[e]; return v != v ? -INFINITY : v; };
         float m = -INFINITY;
-        for (int e = lane; e < E; e += 32) m = fmaxf(m, zr[e]);
+        for (int e = lane; e < E; e += 32) m = fmaxf(m, zval(e));
         m = na_warp_max(m);
         float sall = 0.f;
-        for (int e = lane; e < E; e += 32) sall += expf(zr[e] - m);
+        for (int e = lane; e < E; e += 32) sall += expf(zval(e) - m);
         sall = na_warp_sum(sall);
         // selection s: the largest logit below the previous pick in (value desc, id asc) order
         float pv = INFINITY;
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
             float bv = -INFINITY;
             int bi = 0x7fffffff;
             for (int e = lane; e < E; e += 32) {
-                const float v = zr[e];
+                const float v = zval(e);
                 const bool after_prev = v < pv || (v == pv && e > pi);
                 if (after_prev && (v > bv || (v == bv && e < bi))) { bv = v; bi = e; }
             }
@@ -173,6 +175,8 @@ extern "C" MOE_API moe_status moe_route_noalloc(const void *router_w, const void
         return MOE_ERR_ARG;
     // sizes beyond the built-in scratch (and the kernel's shapes) are refused
     if (T > kNaMaxRows || E > kNaMaxE || k > kNaMaxK || d % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    // rows are read as 16-byte vectors: both operands must start on a 16-byte boundary
+    if (((uintptr_t)router_w | (uintptr_t)x) & 15u) return MOE_ERR_ARG;
     void *scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

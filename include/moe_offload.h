@@ -192,7 +192,9 @@ MOE_API size_t moe_workspace_bytes(const moe_dims *dims);
 /* Device bytes of a slot arena of num_slots slots plus its cache table. */
 MOE_API size_t moe_arena_bytes(const moe_dims *dims, int64_t num_slots);
 
-/* Create a context.
+/* Create a context: the layer stack's routers, shared experts and the pinned
+ * host pool that every miss is copied from (pirouter.ai "32 GB に 65 GB が載る仕組み":
+ * the expert pool lives in page-locked host RAM that the GPU reads by DMA).
  *   host_pool: P expert records back to back, page-locked host memory
  *              (else MOE_ERR_NOT_PINNED); read by DMA only; caller-owned, must
  *              outlive the context; host_pool_bytes >= P * record bytes.
@@ -214,7 +216,10 @@ MOE_API moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, s
 
 /* Attach the HBM slot arena (device, >= moe_arena_bytes(dims, num_slots),
  * caller-owned) holding num_slots expert slots and the cache table, and set
- * flags.  MOE_CACHE_RESET (required the first time and after an error) empties
+ * flags.  One slot holds one (layer, expert) record and the slots form one LRU
+ * cache shared by all layers (ai-hardware-zukan "GPUに載らない分をどう間に合わせるか":
+ * the cache unit is the (layer, expert) pair, replaced least-recently-used;
+ * gaming-st.com "技術的背景": one global expert cache across the layers).  MOE_CACHE_RESET (required the first time and after an error) empties
  * the cache on the compute stream.  MOE_ERR_CAPACITY if num_slots < k * max_rows
  * distinct experts could need (min(k*max_rows, E)), or, with
  * MOE_CACHE_PREFETCH_NEXT, num_slots < 2*E; MOE_ERR_UNSUPPORTED above 65536 slots.
@@ -224,7 +229,12 @@ MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_a
                            uint32_t flags);
 
 /* One MoE layer on T rows (1 <= T <= max_rows), stream-ordered on compute_stream.
- *   x: device, bf16 [T][d] hidden states; y: device, fp32 [T][d] output.
+ *   x: device, bf16 [T][d] hidden states, 16-byte aligned; y: device, fp32
+ *      [T][d] output, 4-byte aligned (else MOE_ERR_ARG, before any work).
+ * Selection order: logits descending, equal logits to the lower id, a NaN
+ * logit counted as -inf (in the softmax too), so k distinct ids in [0, E)
+ * always come out; non-finite inputs give non-finite gates and outputs, not
+ * a fault.
  *   trace: optional host struct filled with the cache events (NULL = none).
  * Returns after the layer's copies and kernels are issued; y is valid when
  * compute_stream reaches that point.  The call waits (host side, bounded) for
@@ -315,7 +325,8 @@ MOE_API moe_status moe_measure_h2d_sm(void *dev_buf, const void *host_buf, size_
                               int32_t reps, void *stream, double *gbs);
 
 /* Router logits, softmax and top-k for T rows with no workspace (the routing
- * part of moe_layer_forward: same selection, gates and ascending id order).
+ * part of moe_layer_forward: same selection rule -- NaN logits as -inf, ties
+ * to the lower id -- gates and ascending id order).
  * The FreeToken pages have no counterpart: this serves callers that cannot
  * allocate device memory when they run -- e.g. a host framework that owns the
  * whole device memory pool and passes only inputs and outputs, or a process
@@ -327,7 +338,8 @@ MOE_API moe_status moe_measure_h2d_sm(void *dev_buf, const void *host_buf, size_
  * each call clears the counter it needs at zero, and calls that overlap on
  * the GPU race -- serialise them.  The first call on a device looks up the
  * array's address with that device current; make it before any stream capture.
- *   router_w: device bf16 [E][d]; x: device bf16 [T][d];
+ *   router_w: device bf16 [E][d]; x: device bf16 [T][d]; both 16-byte aligned
+ *             (MOE_ERR_ARG otherwise, before anything is launched);
  *   idx: device int32 [T][k] out (ascending per row); gates: device fp32 [T][k] out;
  *   stream: cudaStream_t the work is issued on (stream-ordered, returns at once).
  * Limits: T <= 32, E <= 1024, k <= 32, d a multiple of 64; larger sizes return

@@ -114,6 +114,11 @@ EXPORT void orc_dequant_matrix(const uint8_t *rec, int d, int F, int which, doub
  * products), softmax over all E, the k largest logits (ties: lower id),
  * gates renormalised over the selection when renorm != 0.  Output ids are in
  * ascending order.  gap[t] = z_(k) - z_(k+1) (+inf when k == E).
+ * Non-finite logits (the pages say nothing about them; reading taken): a NaN
+ * logit is replaced by -inf before the selection and the softmax, so the
+ * order (value descending, id ascending) is total and k distinct ids in
+ * [0, E) always come out; gates follow IEEE arithmetic on those values (NaN
+ * when the largest logit is +inf or every logit is -inf).
  * Returns 0, or -1 on bad arguments. */
 EXPORT int orc_route(const uint16_t *Wr, const uint16_t *x, int T, int E, int d, int k,
                      int renorm, int32_t *idx, double *gates, double *logits, double *gap) {
@@ -128,7 +133,7 @@ EXPORT int orc_route(const uint16_t *Wr, const uint16_t *x, int T, int E, int d,
             double acc = 0.0;
             const uint16_t *w = Wr + (int64_t)e * d;
             for (int K = 0; K < d; ++K) acc += bf16_val(w[K]) * bf16_val(xr[K]);
-            z[e] = acc;
+            z[e] = isnan(acc) ? -INFINITY : acc;
         }
         /* selection: repeatedly take the largest remaining logit, lower id on ties */
         for (int j = 0; j < k; ++j) {

@@ -289,3 +289,49 @@ def test_host_io_unaligned_buffers_take_the_copy_path():
     st.synchronize()
     assert torch.equal(yv.cuda(), a.y)
     st.close()
+
+
+def test_non_finite_rows_select_valid_experts_like_the_oracle():
+    """Rows holding -inf, NaN and +inf through the whole decode step: the
+    selection rule (NaN logits as -inf, ties to the lower id) gives valid ids,
+    equal to the oracle's; the cache trace and table follow the oracle's LRU;
+    finite rows keep their outputs, non-finite rows give non-finite outputs
+    (no fault, no out-of-range index)."""
+    pb = DecodeProblem(MID, T=4)
+    bad = {(1, 0, 3): -np.inf, (2, 1, 5): np.nan, (3, 2, 0): np.inf}
+    for (t, l, c), v in bad.items():
+        pb.x[t, l, 0, c] = synth.to_bf16(np.array([v], np.float32))[0]
+    run = pb.run(routing=True)
+    idx, gates = pb.oracle_routing()
+    np.testing.assert_array_equal(run.idx, idx)
+    assert run.idx.min() >= 0 and run.idx.max() < MID.E
+    np.testing.assert_allclose(run.gates, gates, rtol=2e-5, atol=1e-7)  # NaN where the oracle has NaN
+    want_events, lru = pb.oracle_trace(idx)
+    assert run.events == want_events
+    m, o, s, c = lru.state()
+    np.testing.assert_array_equal(run.table[0], m)
+    np.testing.assert_array_equal(run.table[1], o)
+    np.testing.assert_array_equal(run.table[2], s)
+    y = run.y.cpu().numpy()
+    for t in range(pb.T):
+        for l in range(MID.L):
+            if (t, l) in {(k[0], k[1]) for k in bad}:
+                assert not np.isfinite(y[t, l]).all()
+            else:
+                assert rel_l2(y[t, l], pb.oracle_y(t, l)) <= REL_L2_MAX
+
+
+def test_forward_rejects_unaligned_activations_before_launching():
+    pb = DecodeProblem(synth.TINY, T=1)
+    st = pb.stack()
+    d = synth.TINY.d
+    xs = torch.zeros(d + 8, dtype=torch.uint16, device="cuda")
+    ys = torch.zeros(d + 4, dtype=torch.float32, device="cuda")
+    for xv, yv in [(xs[1:1 + d], ys[:d]), (xs[:d], ys.view(torch.uint8)[1:1 + 4 * d])]:
+        with pytest.raises(abi.MoeError) as ei:
+            abi.moe_layer_forward(st.ctx, 0, xv, 1, yv, None)
+        assert ei.value.status == abi.MOE_ERR_ARG
+    # nothing ran: the context is usable and the cache still cold
+    run = pb.run(stack=st)
+    assert run.stats.lookups == len(run.events) > 0
+    st.close()

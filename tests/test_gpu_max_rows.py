@@ -1,8 +1,6 @@
 """The decode path at its largest row count (T = 32 rows per call: the union
 lookup of 32 x k selections, four 8-row passes of the GEMV's mma columns,
-four 8-row passes of the BF16 shared expert) against the oracle.
-
-(Named to run after the other GPU tests.)"""
+four 8-row passes of the BF16 shared expert) against the oracle."""
 import pytest
 
 from synth import problem as sp

@@ -2,9 +2,7 @@
 far apart inside one K-step (the GEMV factors out each step's largest code),
 blocks far below their step's largest (their contribution falls under fp16),
 and a NaN scale (code 255), which the OCP definition propagates to every
-output of the expert.
-
-(Named to run after the other GPU tests.)"""
+output of the expert."""
 import numpy as np
 import pytest
 

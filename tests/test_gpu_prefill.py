@@ -84,9 +84,19 @@ def _check(pb, st, events, idx, gates, y, prefetch, rows=None):
     assert clock == wc
     rows = np.arange(pb.T) if rows is None else rows
     for l in range(sh.L):
-        err = rel_l2(y[l][rows], pb.oracle_y(l, rows))
-        assert err <= REL_L2_MAX, (l, err)
+        _check_rows(y[l][rows], pb.oracle_y(l, rows), l)
     return lru
+
+
+def _check_rows(got, want, l):
+    """Each row on its own within the bar (one bad row among hundreds must not
+    hide in a layer-wide norm).  The median row is also held to 1e-5, far under
+    the bar: a systematic error would lift it, while a rare E2M1 rounding that
+    the fp32 summation order flips at a midpoint moves single rows only."""
+    errs = np.array([rel_l2(g, w) for g, w in zip(got, want)])
+    worst = int(np.argmax(errs))
+    assert errs[worst] <= REL_L2_MAX, (l, worst, errs[worst])
+    assert np.median(errs) < 1e-5, (l, float(np.median(errs)))
 
 
 @pytest.mark.parametrize("prefetch", [True, False])
@@ -165,5 +175,5 @@ def test_prefill_static_split_policy():
     want = static_split_trace(want_idx[None], sh.L, sh.E, C, R)
     assert events == want
     for l in range(sh.L):
-        assert rel_l2(y[l], pb.oracle_y(l, np.arange(T))) <= REL_L2_MAX
+        _check_rows(y[l], pb.oracle_y(l, np.arange(T)), l)
     st.close()

@@ -173,6 +173,29 @@ def test_topk_ties_go_to_lower_id():
     assert tuple(idx[0]) == (1, 2) and gap[0] == 0.0
 
 
+def test_non_finite_logits_rank_as_minus_infinity():
+    """Hand-worked selections with non-finite inputs: NaN logits rank as -inf,
+    equal values go to the lower id, and k distinct ids in [0, E) come out."""
+    E, d = 8, 16
+    Wr = np.zeros((E, d), dtype=np.float32)
+    Wr[:, 1:] = 0.25
+    Wr[:, 0] = [1, 1, -1, 1, 0, -1, 1, 1]  # x_0 = -inf: experts 2 and 5 go to +inf, 4 to NaN
+    x = np.ones((3, d), dtype=np.float32)
+    x[0, 0] = -np.inf
+    x[1, 0] = np.nan                       # every logit NaN
+    x[2, 0] = np.inf                       # +inf except 2, 5 (-inf) and 4 (NaN)
+    idx, gates, z, _ = oracle.route(_bf16_bits(Wr), _bf16_bits(x), 3)
+    assert tuple(idx[0]) == (0, 2, 5)      # the two +inf, then the lowest -inf
+    assert tuple(idx[1]) == (0, 1, 2)      # all -inf: the lowest ids
+    assert tuple(idx[2]) == (0, 1, 3)      # five +inf: the lowest three
+    assert z[0, 4] == -np.inf and np.all(z[1] == -np.inf)
+    assert np.all(np.isnan(gates))         # inf - inf in every softmax
+    # a finite row beside them is untouched
+    x2 = np.ones((1, d), dtype=np.float32)
+    i2, g2, z2, _ = oracle.route(_bf16_bits(Wr), _bf16_bits(x2), 3)
+    assert np.all(np.isfinite(g2)) and abs(g2.sum() - 1.0) < 1e-12
+
+
 # --------------------------------------------------------- expert FFN --
 def test_expert_one_hot_input_closed_form():
     d, F = 128, 256
@@ -435,6 +458,66 @@ def test_w4a4_one_hot_row():
     np.testing.assert_allclose(y, W2 @ hq, rtol=1e-9, atol=1e-12)
     # and the quantized h is within NVFP4's error of h
     assert np.linalg.norm(hq - h) / np.linalg.norm(h) < 0.15
+
+
+def _e2m1_rne_independent(v):
+    """E2M1 code of fp32 values by nearest grid point, ties to the even
+    mantissa (even index), |v| > 6 saturating; sign bit from the sign."""
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    dist = np.abs(a[:, None] - grid[None, :])
+    best = dist.min(axis=1, keepdims=True)
+    cand = dist == best
+    even = cand & (np.arange(8) % 2 == 0)[None, :]
+    m = np.where(even.any(axis=1), even.argmax(axis=1), cand.argmax(axis=1))
+    return np.where(np.signbit(np.asarray(v, dtype=np.float32)), 8, 0) | m
+
+
+def _nvfp4_act_dequant_independent(v):
+    """Per-row NVFP4 activation quantization written from the definition, in
+    fp32 with RNE: s_t = amax / 2688, per 16 values the E4M3 scale of
+    amax_b / (6 s_t) (torch's RNE cast), codes E2M1(v / (scale s_t)); returns
+    the dequantised values in fp64."""
+    v = np.asarray(v, dtype=np.float32)
+    amax = np.float32(np.abs(v).max())
+    s_t = np.float32(amax / np.float32(2688.0)) if amax > 0 else np.float32(1.0)
+    out = np.empty(v.size, dtype=np.float64)
+    for b in range(v.size // 16):
+        blk = v[16 * b:16 * b + 16]
+        r = np.float32(np.abs(blk).max() / np.float32(np.float32(6.0) * s_t))
+        sb = torch.tensor([min(float(r), 448.0)], dtype=torch.float32).to(torch.float8_e4m3fn)
+        sval = np.float32(sb.double().item())
+        if sval == 0:
+            out[16 * b:16 * b + 16] = 0.0
+            continue
+        denom = np.float32(sval * s_t)
+        codes = _e2m1_rne_independent((blk / denom).astype(np.float32))
+        out[16 * b:16 * b + 16] = np.array([E2M1_GOLDEN[int(c)] for c in codes]) * float(sval) * float(s_t)
+    return out
+
+
+def test_w4a4_expert_matches_its_steps_in_numpy():
+    """The NVFP4 prefill expert on dense rows: x quantized per block of 16 with
+    one fp32 row scale, fp64 products against independently decoded weights, h
+    rounded to fp32 and quantized the same way, then the down projection.
+    Block magnitudes spread over several decades, so every block has its own
+    scale and a wrong block size or an unquantized operand moves the result
+    far beyond the tolerance."""
+    d, F = 256, 128
+    rec = synth.expert_record(1, 7, d, F)
+    W1, W3, W2 = _matrices_independent(rec, d, F)
+    rng = np.random.default_rng(44)
+    for trial in range(3):
+        spread = np.repeat(10.0 ** rng.uniform(-3, 1, d // 16), 16)
+        x = _bf16_bits(rng.normal(0, 1, d) * spread)
+        xq = _nvfp4_act_dequant_independent(_bf16_val(x).astype(np.float32))
+        g, u = W1 @ xq, W3 @ xq
+        h = (g * expit(g) * u).astype(np.float32)
+        want = W2 @ _nvfp4_act_dequant_independent(h)
+        got = oracle.expert_w4a4(rec, d, F, x)
+        np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-14 * np.abs(want).max())
+        exact = oracle.expert_w4a16(rec, d, F, x)[0]
+        assert 1e-4 < np.linalg.norm(got - exact) / np.linalg.norm(exact) < 0.3
 
 
 # ----------------------------------------------------- generator sanity --
