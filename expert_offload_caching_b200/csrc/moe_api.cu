@@ -88,7 +88,7 @@ int max_jobs(const moe_dims *d, int T) {
 // Workspace carve-up (offsets from the caller's base).  Row buffers are sized
 // for the largest call (max_rows); the prefill buffers exist when max_rows > 32.
 struct WsLayout {
-    int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, rowrefs, xh, hh, part, cnt, fill,
+    int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, lk, rowrefs, xh, hh, part, cnt, fill,
         jobidx, h32, xq, xq_scales, xq_st, hq, hq_scales, hq_st, pairs, n_pairs, xstage, ystage, total;
 };
 int pairs_capacity(const moe_dims *d) {
@@ -111,6 +111,7 @@ WsLayout ws_layout(const moe_dims *d) {
     w.n_misses = take(4);
     w.ticket = take(4);
     w.ticket2 = take(4 * kMaxTiles);
+    w.lk = take(4 * (4 + 3 * (int64_t)kMaxSlots));  // layer kernel: queue[2], release, pad, done_a, flags
     w.rowrefs = take(T * k * (int64_t)sizeof(RowRef));
     w.xh = take(Td * 2 * dd * 2);
     w.hh = take(Td * (k + 1) * 2 * F * 2);
@@ -196,7 +197,11 @@ struct moe_ctx {
     std::vector<cudaEvent_t> ev_pool;
     std::vector<TimedLaunch> pending;
     // injection and limits
-    int64_t inj_copy_fail_at = 0, inj_drop_publish = 0;
+    int64_t inj_copy_fail_at = 0, inj_drop_publish = 0, inj_drop_flags = 0;
+    // decode: the persistent layer kernel (one launch per layer, misses gated
+    // by flags the copy stream writes), when stream memory writes work here;
+    // else a launch per miss, gated by events
+    bool fused = false;
     double wait_limit = 60.0;
     std::chrono::steady_clock::time_point issue_t0;  // end of the last miss-list wait
     // device spans of timed launches: [slot][2] = {min start, min ~end}, all ones when free
@@ -217,6 +222,31 @@ moe_status cuda_fail(moe_ctx *c, cudaError_t e, const char *what) {
         cudaError_t e_ = (call);                                    \
         if (e_ != cudaSuccess) return cuda_fail(ctx, e_, #call);    \
     } while (0)
+
+// cuStreamWriteValue32 (driver API, through the runtime's entry-point query):
+// a 32-bit store to device memory executed in stream order, after the
+// stream's earlier work (the default flags include a memory barrier, so the
+// bytes of an earlier copy are visible before the value).
+typedef CUresult (*StreamWriteFn)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+StreamWriteFn stream_write_fn() {
+    static const StreamWriteFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuStreamWriteValue32", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<StreamWriteFn>(p);
+        cudaGetLastError();
+        return static_cast<StreamWriteFn>(nullptr);
+    }();
+    return fn;
+}
+cudaError_t stream_write(cudaStream_t s, uint32_t *addr, uint32_t value) {
+    const StreamWriteFn fn = stream_write_fn();
+    if (!fn) return cudaErrorNotSupported;
+    return fn(reinterpret_cast<CUstream>(s), reinterpret_cast<CUdeviceptr>(addr), value, 0) == CUDA_SUCCESS
+               ? cudaSuccess
+               : cudaErrorNotSupported;
+}
 
 cudaEvent_t pool_event(moe_ctx *ctx) {
     if (!ctx->ev_pool.empty()) {
@@ -393,6 +423,27 @@ void fill_trace(moe_ctx *ctx, int32_t layer, int nrouted, int nev, moe_layer_tra
     }
 }
 
+// Counters and trace of a decode call whose miss list (nev entries) is in the page.
+moe_status finish_decode(moe_ctx *ctx, int32_t layer, int32_t T, int nev, moe_layer_trace *trace) {
+    const HostEvent *ev = ctx->page_h->ev;
+    int64_t hits = 0, evictions = 0;
+    for (int j = 0; j < nev; ++j) {
+        hits += ev[j].flags & 1;
+        evictions += ev[j].evicted >= 0;
+    }
+    for (int i = 0; i < 8; ++i) ctx->stats.route_phase_us[i] += ctx->page_h->phase_ns[i] * 1e-3;
+    ctx->stats.lookups += nev;
+    ctx->stats.hits += hits;
+    ctx->stats.misses += nev - hits;
+    ctx->stats.evictions += evictions;
+    ctx->stats.forward_calls += 1;
+    ctx->stats.host_us[2] +=
+        std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - ctx->issue_t0).count();
+    fill_trace(ctx, layer, nev, nev, trace);
+    ctx->last_T = T;
+    return MOE_OK;
+}
+
 moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T, float *y,
                           moe_layer_trace *trace) {
     const moe_dims &D = ctx->dims;
@@ -443,8 +494,91 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
                               ctx->cs));
         time_end(ctx, sd, 2.0 * D.d * D.F + (double)T * D.F * 4);
     }
-    // hit experts and the shared expert, before the miss list is known
     const int in_launch_shared = (D.has_shared && !shared_separate(ctx)) ? 1 : 0;
+    if (ctx->fused) {
+        // one launch for every expert GEMV of the layer: the hit and shared
+        // experts at once, each miss when the copy stream flags its halves
+        LayerArgs la{};
+        la.jobs = ctx->dws.jobs;
+        la.n_jobs = ctx->dws.n_jobs;
+        la.rowrefs = ctx->dws.rowrefs;
+        la.arena = ctx->arena;
+        la.rec_bytes = ctx->lay.bytes;
+        la.shared_rec = D.has_shared ? ctx->shared_recs + (int64_t)layer * ctx->slay.bytes : nullptr;
+        la.shared_item = in_launch_shared;
+        la.T = T;
+        la.k = D.k;
+        la.d = D.d;
+        la.F = D.F;
+        la.lay = ctx->lay;
+        la.xh = ctx->dws.xh;
+        la.hh = ctx->dws.hh;
+        la.part = ctx->dws.part;
+        la.gates = ctx->dws.gates;
+        la.y = y;
+        la.tile_ticket = ctx->dws.ticket2;
+        la.done_a = ctx->dws.lk_done_a;
+        la.queue = ctx->dws.lk_queue;
+        la.miss_flag = ctx->dws.lk_flags;
+        la.release = ctx->dws.lk_release;
+        la.seq = seq;
+        la.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 30.0) * 1e9);
+        la.page = ctx->page_d;
+        TimedLaunch tk, th;
+        time_begin(ctx, tk, MOE_K_LAYER);
+        la.span = time_span(ctx, tk);
+        time_begin(ctx, th, MOE_K_LAYER_HITS);
+        la.span_hit = time_span(ctx, th);
+        CK(launch_expert_layer(la, ctx->cs));
+        const long ik = time_end(ctx, tk, 0);
+        const long ih = time_end(ctx, th, 0);
+        // every way out before the last flag is written releases the kernel's waits
+        struct Release {
+            moe_ctx *c;
+            uint32_t seq;
+            bool armed = true;
+            ~Release() {
+                if (armed) stream_write(c->xs, c->dws.lk_release, seq);
+            }
+        } rel{ctx, seq};
+        {
+            const moe_status ws_ = wait_miss_list(ctx, seq);
+            if (ws_ != MOE_OK) return ws_;
+        }
+        if (ctx->page_h->error) return device_error(ctx);
+        const int nev = ctx->page_h->n_events;
+        const HostEvent *ev = ctx->page_h->ev;
+        int n_hit_jobs = 0;
+        for (int j = 0; j < nev; ++j) n_hit_jobs += ev[j].flags & 1;
+        const double rec = w13_bytes(ctx) + w2_bytes(ctx);
+        if (ik >= 0) ctx->pending[ik].bytes = (nev + in_launch_shared) * rec + (double)T * D.d * 2;
+        if (ih >= 0) ctx->pending[ih].bytes = (n_hit_jobs + in_launch_shared) * rec + (double)T * D.d * 2;
+        // misses: the gate/up prefix, its flag, the W2 half, its flag
+        const int64_t split = ctx->lay.w2_codes;
+        for (int j = 0; j < nev; ++j) {
+            if (ev[j].flags & 1) continue;
+            if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
+                ctx->state = MOE_ERR_STATE;
+                ctx->err = "injected failure of an H2D copy issue";
+                return MOE_ERR_CUDA;
+            }
+            const int64_t rec_idx = ((int64_t)layer * D.E + ev[j].expert) % ctx->P;
+            uint8_t *dst = ctx->arena + (int64_t)ev[j].slot * ctx->lay.bytes;
+            const uint8_t *src = ctx->pool + rec_idx * ctx->lay.bytes;
+            const bool flags = !(ctx->inj_drop_flags > 0 && (--ctx->inj_drop_flags, true));
+            CK(cudaMemcpyAsync(dst, src, split, cudaMemcpyHostToDevice, ctx->xs));
+            if (flags) CK(stream_write(ctx->xs, ctx->dws.lk_flags + 2 * j, seq));
+            CK(cudaMemcpyAsync(dst + split, src + split, ctx->lay.bytes - split, cudaMemcpyHostToDevice, ctx->xs));
+            if (flags) CK(stream_write(ctx->xs, ctx->dws.lk_flags + 2 * j + 1, seq));
+            else rel.armed = false;  // injected: the kernel's own wait limit must end it
+            ctx->stats.h2d_copies += 1;
+            ctx->stats.h2d_bytes += ctx->lay.bytes;
+        }
+        rel.armed = false;
+        return finish_decode(ctx, layer, T, nev, trace);
+    }
+
+    // hit experts and the shared expert, before the miss list is known
     const int grid_y = nj + in_launch_shared;
     TimedLaunch tg, td;
     time_begin(ctx, tg, MOE_K_GATEUP);
@@ -518,23 +652,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         time_end(ctx, md, w2_bytes(ctx) + (double)T * D.F * 4);
     }
 
-    // trace and counters
-    int64_t hits = 0, evictions = 0;
-    for (int j = 0; j < nev; ++j) {
-        hits += ev[j].flags & 1;
-        evictions += ev[j].evicted >= 0;
-    }
-    for (int i = 0; i < 8; ++i) ctx->stats.route_phase_us[i] += ctx->page_h->phase_ns[i] * 1e-3;
-    ctx->stats.lookups += nev;
-    ctx->stats.hits += hits;
-    ctx->stats.misses += nev - hits;
-    ctx->stats.evictions += evictions;
-    ctx->stats.forward_calls += 1;
-    ctx->stats.host_us[2] +=
-        std::chrono::duration<double, std::micro>(std::chrono::steady_clock::now() - ctx->issue_t0).count();
-    fill_trace(ctx, layer, nev, nev, trace);
-    ctx->last_T = T;
-    return MOE_OK;
+    return finish_decode(ctx, layer, T, nev, trace);
 }
 
 // One layer of a prefill chunk (T > 32 rows): W4A4 grouped tensor-core GEMMs,
@@ -792,6 +910,10 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     ctx->dws.n_misses = reinterpret_cast<int32_t *>(w + L.n_misses);
     ctx->dws.ticket = reinterpret_cast<uint32_t *>(w + L.ticket);
     ctx->dws.ticket2 = reinterpret_cast<uint32_t *>(w + L.ticket2);
+    ctx->dws.lk_queue = reinterpret_cast<uint32_t *>(w + L.lk);
+    ctx->dws.lk_release = ctx->dws.lk_queue + 2;
+    ctx->dws.lk_done_a = ctx->dws.lk_queue + 4;
+    ctx->dws.lk_flags = ctx->dws.lk_done_a + kMaxSlots;
     ctx->dws.rowrefs = reinterpret_cast<RowRef *>(w + L.rowrefs);
     ctx->dws.xh = reinterpret_cast<__half *>(w + L.xh);
     ctx->dws.hh = reinterpret_cast<__half *>(w + L.hh);
@@ -850,6 +972,15 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     }
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs);
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket2, 0, 4 * kMaxTiles, ctx->cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.lk_queue, 0, 4 * (4 + 3 * (size_t)kMaxSlots), ctx->cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->cs);
+    // the persistent layer kernel needs stream memory writes on the copy stream:
+    // one trial write (of the value already there) decides
+    if (e == cudaSuccess) {
+        ctx->fused = stream_write(ctx->xs, ctx->dws.lk_release, 0u) == cudaSuccess &&
+                     cudaStreamSynchronize(ctx->xs) == cudaSuccess;
+        cudaGetLastError();
+    }
     if (e != cudaSuccess) {
         st = cuda_fail(ctx, e, "moe_layer_init");
         moe_layer_destroy(ctx);
@@ -912,6 +1043,10 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         }
         CK(cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs));
         CK(cudaMemsetAsync(ctx->dws.ticket2, 0, 4 * kMaxTiles, ctx->cs));
+        // layer-kernel counters (flags and the release word keep their values:
+        // they are compared with sequence numbers that only grow)
+        CK(cudaMemsetAsync(ctx->dws.lk_queue, 0, 8, ctx->cs));
+        CK(cudaMemsetAsync(ctx->dws.lk_done_a, 0, 4 * (size_t)kMaxSlots, ctx->cs));
         for (auto &t : ctx->pending) {  // timing records of the old state
             ctx->ev_pool.push_back(t.a);
             ctx->ev_pool.push_back(t.b);
@@ -1057,9 +1192,13 @@ moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds) {
 
 moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
     if (!ctx || n < 0) return MOE_ERR_ARG;
-    if (what == 0) { ctx->inj_copy_fail_at = 0; ctx->inj_drop_publish = 0; }
+    if (what == 0) { ctx->inj_copy_fail_at = 0; ctx->inj_drop_publish = 0; ctx->inj_drop_flags = 0; }
     else if (what == 1) ctx->inj_copy_fail_at = n;
     else if (what == 2) ctx->inj_drop_publish = n;
+    else if (what == 3) {  // decode path: 0 = a launch per miss, 1 = the layer kernel
+        if (n == 1 && stream_write(ctx->xs, ctx->dws.lk_release, 0u) != cudaSuccess) return MOE_ERR_UNSUPPORTED;
+        ctx->fused = n == 1;
+    } else if (what == 4) ctx->inj_drop_flags = n;
     else return MOE_ERR_ARG;
     return MOE_OK;
 }

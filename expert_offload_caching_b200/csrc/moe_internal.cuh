@@ -12,6 +12,7 @@ constexpr int kDecodeMaxRows = 32;  // T <= this takes the GEMV (decode) path
 constexpr int kMaxK = 32;
 constexpr int kMaxE = 1024;
 constexpr int kMaxTiles = 512;  // GEMV tiles per launch: max(d / 16, F / 8) with d, F <= 4096
+constexpr int kMaxSlots = kMaxK * kDecodeMaxRows + 1;  // experts of one decode layer (+ shared)
 
 // Record formats (the values of the C ABI's MOE_FMT_* constants).
 constexpr int kFmtNvfp4 = 0, kFmtMxfp4 = 1, kFmtBf16 = 2;
@@ -86,6 +87,11 @@ struct DecodeWs {
     float *part;         // [maxT][k+1][d] per-selection expert outputs (p = k: shared)
     uint32_t *ticket;    // last-CTA counter of the route kernel
     uint32_t *ticket2;   // [kMaxTiles] per-tile counters of the combining down launch
+    // persistent layer kernel (see LayerArgs)
+    uint32_t *lk_queue;    // [2]
+    uint32_t *lk_release;  // [1]
+    uint32_t *lk_done_a;   // [kMaxSlots]
+    uint32_t *lk_flags;    // [2 * kMaxSlots]
     // prefill only (T > 32)
     int32_t *cnt;        // [E] rows per expert
     int32_t *fill;       // [E] scatter cursors
@@ -146,6 +152,41 @@ struct GemvArgs {
     unsigned long long *span;  // launch timing slot (see span_mark), or null
 };
 
+// Persistent decode layer kernel (all expert GEMVs of one layer, misses as
+// their copies land).  Counters in the workspace, zero between launches (the
+// kernel's last CTA resets them): queue[0] next item, queue[1] CTAs done,
+// done_a[job] gate/up tiles completed (slot kMaxSlots - 1: the shared expert),
+// tile_ticket[d / 16] experts completed per output tile.  miss_flag[2 j] /
+// [2 j + 1]: the call's sequence number once job j's gate/up prefix / W2 half
+// is in its slot (written by the copy stream); release: the host gives up the
+// call (>= seq), every wait ends.
+struct LayerArgs {
+    const Job *jobs;
+    const int32_t *n_jobs;
+    const RowRef *rowrefs;
+    const uint8_t *arena;
+    int64_t rec_bytes;
+    const uint8_t *shared_rec;  // this layer's shared record (any format), or null
+    int shared_item;            // 1: the shared expert is an item of the launch (routed format)
+    int T, k, d, F;
+    RecordLayout lay;
+    const __half *xh;           // [T][2][d] x as fp16 (hi, lo)
+    __half *hh;                 // [T][k+1][2][F]
+    float *part;                // [T][k+1][d]
+    const float *gates;         // [T][k]
+    float *y;                   // [T][d]
+    uint32_t *tile_ticket;
+    uint32_t *done_a;
+    uint32_t *queue;
+    const uint32_t *miss_flag;
+    const uint32_t *release;
+    uint32_t seq;
+    unsigned long long wait_ns;  // bound of every wait, from the kernel's start
+    HostPage *page;
+    unsigned long long *span;      // launch timing slot, or null
+    unsigned long long *span_hit;  // [start, end of the last hit/shared item], or null
+};
+
 // Grouped W4A4 expert GEMMs of a prefill chunk (tcgen05 block-scaled MMA).
 // Activation rows are in expert-grouped order: the routed rows of job j at
 // [row_off_j, row_off_j + nrows_j) (RowRef gives (t, p)), then the shared
@@ -191,6 +232,7 @@ __device__ __forceinline__ void span_mark(unsigned long long *slot, int which) {
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
 // slots: job slots of the launch (max jobs + shared expert), 1 with only_job
 cudaError_t launch_gemv(const GemvArgs &a, int slots, cudaStream_t s);
+cudaError_t launch_expert_layer(const LayerArgs &a, cudaStream_t s);
 // BF16 shared expert of a decode call (T <= 32 rows; x as DecodeWs::xh):
 // kGateUp writes h = silu(W1 x) * (W3 x) as fp16 (hi, lo) into hh at selection
 // sel0 + t * sel_stride (layout of DecodeWs::hh); kDown reads that h and

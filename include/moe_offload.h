@@ -124,8 +124,13 @@ typedef struct {
 /* Cumulative counters since the last MOE_CACHE_RESET.
  * lookups/hits/misses count routed lookups (each distinct (layer, expert) of a
  * batch once); prefetch_* count next-layer prefetch entries separately. */
+/* Kernel classes of the timing counters.  MOE_K_LAYER: the decode layer
+ * kernel (every expert GEMV of a layer in one launch, misses as their copies
+ * land); MOE_K_LAYER_HITS: the same launches up to the end of their last
+ * resident-expert item (hit and shared experts: the part bounded by HBM, not
+ * by the copies). */
 enum { MOE_K_ROUTE = 0, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE, MOE_K_PREFILL_ROUTE,
-       MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_COUNT };
+       MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_LAYER, MOE_K_LAYER_HITS, MOE_K_COUNT };
 typedef struct {
     int64_t lookups, hits, misses, evictions;
     int64_t prefetch_lookups, prefetch_misses;
@@ -288,13 +293,21 @@ MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
  * 4 MB device buffer of span slots, freed by moe_layer_destroy. */
 MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
 
-/* Longest host wait for the device miss list, in seconds (default 60). */
+/* Longest wait, in seconds (default 60): the host's wait for the device miss
+ * list, and (capped at 30 s, counted from the kernel's start) every wait of the
+ * decode layer kernel for a miss's copy or for another CTA's tiles; a device
+ * wait that runs out records a failed check (MOE_ERR_CUDA at the next call). */
 MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
 
-/* Host-side fault injection for tests.  what = 1: the n-th H2D copy issue
- * (counted from now, 1-based) fails with MOE_ERR_CUDA before it is issued;
- * what = 2: the next n lookups do not publish their miss list, so the host
- * wait runs out (MOE_ERR_TIMEOUT); what = 0 clears both. */
+/* Host-side fault injection and path selection for tests.  what = 1: the n-th
+ * H2D copy issue (counted from now, 1-based) fails with MOE_ERR_CUDA before it
+ * is issued; what = 2: the next n lookups do not publish their miss list, so
+ * the host wait runs out (MOE_ERR_TIMEOUT); what = 4: the next n misses are
+ * copied without their completion flags, so the decode layer kernel's bounded
+ * wait runs out (a failed device check, reported by the next call); what = 3:
+ * decode runs the layer kernel (n = 1; the default where stream memory writes
+ * work, MOE_ERR_UNSUPPORTED elsewhere) or a gate/up and a down launch per miss,
+ * gated by copy events (n = 0); what = 0 clears 1, 2 and 4. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Hybrid split: m missing experts, PCIe bandwidth B_P, host expert-processing

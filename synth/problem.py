@@ -109,16 +109,20 @@ class RegisteredPool:
     ``tensor`` is a uint8 view; call ``close()`` (or drop the object) to unpin."""
 
     def __init__(self, shape: LayerShape, P: int | None = None, distinct: int | None = None,
-                 seed: int = MASTER_SEED):
+                 seed: int = MASTER_SEED, fmt: int = FMT_NVFP4):
         P = shape.L * shape.E if P is None else P
         distinct = P if distinct is None else min(distinct, P)
-        rb = record_bytes(shape.d, shape.F)
+        rb = format_record_bytes(fmt, shape.d, shape.F)
         self.nbytes = P * rb
         self.array = np.empty(self.nbytes, dtype=np.uint8)
         base = self.array.ctypes.data
         for i in range(distinct):
-            expert_record_into(base + i * rb, i // shape.E, i % shape.E, shape.d, shape.F,
-                               seed=seed)
+            if fmt == FMT_NVFP4:
+                expert_record_into(base + i * rb, i // shape.E, i % shape.E, shape.d, shape.F,
+                                   seed=seed)
+            else:
+                self.array[i * rb:(i + 1) * rb] = expert_record_mx(i // shape.E, i % shape.E, shape.d,
+                                                                   shape.F, seed=seed)
         if distinct < P:
             replicate_records(base, rb, distinct, P)
         rc = torch.cuda.cudart().cudaHostRegister(base, self.nbytes, 0)

@@ -335,3 +335,45 @@ def test_forward_rejects_unaligned_activations_before_launching():
     run = pb.run(stack=st)
     assert run.stats.lookups == len(run.events) > 0
     st.close()
+
+
+def test_per_miss_launch_path_matches_the_oracle():
+    """The decode path without the layer kernel (a gate/up and a down launch per
+    miss, gated by copy events; what the library runs where stream memory writes
+    are unavailable): same trace, table, slots and outputs."""
+    pb = DecodeProblem(MID, T=12)
+    st = pb.stack()
+    abi.moe_debug_inject(st.ctx, 3, 0)
+    run = pb.run(stack=st, routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(st, run.table[1])
+    abi.moe_debug_inject(st.ctx, 3, 1)  # back to the layer kernel on the same cache
+    st.close()
+
+
+def test_layer_kernel_flag_wait_runs_out_then_reset_recovers():
+    """A miss whose copy flags are never written: the layer kernel's bounded wait
+    runs out (limit 0.3 s), the kernel records the failed check in the mapped
+    page and returns; the next call reports it (MOE_ERR_CUDA, device check 40 or
+    41), a reset brings the context back, and a full run matches the oracle."""
+    import time
+    pb = DecodeProblem(synth.TINY, T=8)
+    st = pb.stack()
+    abi.moe_set_wait_limit(st.ctx, 0.3)
+    abi.moe_debug_inject(st.ctx, 4, 1)  # the next miss: copies issued, flags not written
+    x = torch.from_numpy(pb.x[:, 0]).cuda()
+    y = torch.zeros((pb.T, 1, pb.shape.d), device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    st.forward(0, x[0], y[0])  # cold cache: every selected expert misses
+    st.synchronize()
+    assert time.perf_counter() - t0 < 10.0
+    with pytest.raises(abi.MoeError) as ei:
+        st.forward(0, x[1], y[1])
+    assert ei.value.status == abi.MOE_ERR_CUDA
+    msg = abi.moe_last_error(st.ctx)
+    assert "device check 40" in msg or "device check 41" in msg, msg
+    st.reset()
+    abi.moe_set_wait_limit(st.ctx, 60.0)
+    _check_run(pb, pb.run(stack=st))
+    st.close()
