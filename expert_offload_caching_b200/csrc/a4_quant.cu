@@ -1,4 +1,4 @@
-// NVFP4 activation quantizer (the W4A4 prefill path) and the prefill combine.
+// NVFP4 and MXFP4 activation quantizers (the W4A4 prefill path) and the prefill combine.
 //
 // The routed experts of the checkpoint are W4A4 NVFP4 (florigen.ai,
 // "NVFP4で約135GBまで縮める"): activations are quantized like the weights --
@@ -77,28 +77,76 @@ __device__ void quant_row_codes(LoadFn load, int n, uint8_t *codes, uint8_t *sca
     if (lane == 0) *st = s_t;
 }
 
+// MXFP4 activations (OCP microscaling; the W4A4 path over MXFP4 records): one
+// E8M0 scale 2^e per 32 values, e = floor(log2 amax(block)) - 2 clamped to
+// [-127, 127] (-127 for an all-zero block), codes E2M1(v * 2^-e), RNE and
+// saturating, no row scale.  Multiplying by the power of two 2^-e is exact
+// (or, below fp32's normal range, correctly rounded like the oracle's ldexpf),
+// so every decision is the oracle's.
+__device__ __forceinline__ int mx_exponent(float amax) {
+    const uint32_t eb = (__float_as_uint(amax) >> 23) & 0xffu;
+    if (amax == 0.f || eb == 0u) return -127;  // zero or subnormal: floor(log2) - 2 < -127
+    const int e = (int)eb - 127 - 2;
+    return e > 127 ? 127 : e;
+}
+__device__ __forceinline__ float pow2f(int e) {  // 2^e for e in [-149, 127], exact
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
+}
+template <typename LoadFn>
+__device__ void quant_row_codes_mx(LoadFn load, int n, uint8_t *codes, uint8_t *scales) {
+    const int lane = threadIdx.x & 31;
+    for (int b = lane; b < n / 32; b += 32) {
+        float v[32];
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            v[j] = load(32 * b + j);
+            amax = fmaxf(amax, fabsf(v[j]));
+        }
+        const int e = mx_exponent(amax);
+        const float inv = pow2f(-e);
+        uint32_t word[4] = {0u, 0u, 0u, 0u};
+        if (amax > 0.f) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                uint16_t c;
+                asm("{\n\t.reg .b8 c8;\n\t"
+                    "cvt.rn.satfinite.e2m1x2.f32 c8, %2, %1;\n\t"
+                    "cvt.u16.u8 %0, c8;\n\t}"
+                    : "=h"(c)
+                    : "f"(v[j] * inv), "f"(v[j + 1] * inv));
+                word[j >> 3] |= (uint32_t)(c & 0xffu) << (4 * (j & 7));
+            }
+        }
+        *reinterpret_cast<uint4 *>(codes + 16 * b) = make_uint4(word[0], word[1], word[2], word[3]);
+        scales[b] = (uint8_t)(e + 127);
+    }
+}
+
 // Grouped rows of x for the tensor-core GEMMs: row g < T*k is token
 // rowrefs[g].t, row T*k + t (shared expert) is token t; one warp per row.
 __global__ void quant_x_grouped_kernel(const __nv_bfloat16 *__restrict__ x, int T, int k, int d,
                                        int has_shared, const RowRef *__restrict__ rowrefs,
-                                       uint8_t *codes, uint8_t *scales, float *st) {
+                                       uint8_t *codes, uint8_t *scales, float *st, int mx) {
     const int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int tk = T * k;
     if (g >= tk + (has_shared ? T : 0)) return;
     const int t = g < tk ? rowrefs[g].t : g - tk;
     const __nv_bfloat16 *row = x + (size_t)t * d;
-    quant_row_codes([&](int i) { return __bfloat162float(row[i]); }, d, codes + (size_t)g * (d / 2),
-                    scales + (size_t)g * (d / 16), st + g);
+    auto load = [&](int i) { return __bfloat162float(row[i]); };
+    if (mx) quant_row_codes_mx(load, d, codes + (size_t)g * (d / 2), scales + (size_t)g * (d / 32));
+    else quant_row_codes(load, d, codes + (size_t)g * (d / 2), scales + (size_t)g * (d / 16), st + g);
 }
 
 // Grouped h rows (fp32 [rows][F]) -> NVFP4 codes, scales, row scales; one warp per row.
 __global__ void quant_h_grouped_kernel(const float *__restrict__ h32, int rows, int F, uint8_t *codes,
-                                       uint8_t *scales, float *st) {
+                                       uint8_t *scales, float *st, int mx) {
     const int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (g >= rows) return;
     const float *row = h32 + (size_t)g * F;
-    quant_row_codes([&](int i) { return row[i]; }, F, codes + (size_t)g * (F / 2),
-                    scales + (size_t)g * (F / 16), st + g);
+    auto load = [&](int i) { return row[i]; };
+    if (mx) quant_row_codes_mx(load, F, codes + (size_t)g * (F / 2), scales + (size_t)g * (F / 32));
+    else quant_row_codes(load, F, codes + (size_t)g * (F / 2), scales + (size_t)g * (F / 16), st + g);
 }
 
 // y[t] = sum over p < k of gates[t][p] * part[t][p] (+ part[t][k], the shared expert)
@@ -114,23 +162,41 @@ __global__ void combine_kernel(const float *__restrict__ part, const float *__re
     y[i] = acc;
 }
 
+__global__ void swiglu_split_kernel(const float *__restrict__ sg, int T, int F, uint16_t *__restrict__ hs) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= (int64_t)T * F) return;
+    const int t = (int)(i / F), j = (int)(i - (int64_t)t * F);
+    const float gt = sg[(size_t)t * 2 * F + 2 * j], up = sg[(size_t)t * 2 * F + 2 * j + 1];
+    const float h = gt / (1.0f + expf(-gt)) * up;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
+    hs[(size_t)t * 2 * F + j] = __bfloat16_as_ushort(hi);
+    hs[(size_t)t * 2 * F + F + j] = __bfloat16_as_ushort(lo);
+}
+
 }  // namespace
+
+cudaError_t launch_swiglu_split(const float *sg, int T, int F, uint16_t *hs, cudaStream_t s) {
+    const int64_t n = (int64_t)T * F;
+    swiglu_split_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sg, T, F, hs);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quant_x_grouped(const __nv_bfloat16 *x, int T, int k, int d, int has_shared,
                                    const RowRef *rowrefs, uint8_t *codes, uint8_t *scales, float *st,
-                                   cudaStream_t s) {
+                                   int mx, cudaStream_t s) {
     const int rows = T * k + (has_shared ? T : 0);
     const int warps_per_cta = 8;
     quant_x_grouped_kernel<<<(rows + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(
-        x, T, k, d, has_shared, rowrefs, codes, scales, st);
+        x, T, k, d, has_shared, rowrefs, codes, scales, st, mx);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quant_h_grouped(const float *h32, int rows, int F, uint8_t *codes, uint8_t *scales,
-                                   float *st, cudaStream_t s) {
+                                   float *st, int mx, cudaStream_t s) {
     const int warps_per_cta = 8;
     quant_h_grouped_kernel<<<(rows + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(
-        h32, rows, F, codes, scales, st);
+        h32, rows, F, codes, scales, st, mx);
     return cudaGetLastError();
 }
 

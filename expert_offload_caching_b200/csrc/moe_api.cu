@@ -45,9 +45,8 @@ bool dims_supported(const moe_dims *d) {
     return d->d % 64 == 0 && d->F % 64 == 0 && d->d <= 4096 && d->F <= 4096 && d->k <= kMaxK &&
            d->E <= kMaxE &&
            d->max_rows <= 4096 && (int64_t)d->L * d->E < (1ll << 31) &&
-           // prefill GEMM operands: TMA boxes of 128 bytes of a row; NVFP4 block scales
-           (d->max_rows <= kDecodeMaxRows || (d->d >= 256 && d->F >= 256 && d->weight_format == MOE_FMT_NVFP4 &&
-                                              shared_fmt(d) == MOE_FMT_NVFP4));
+           // prefill GEMM operands: TMA boxes of 128 bytes of a row
+           (d->max_rows <= kDecodeMaxRows || (d->d >= 256 && d->F >= 256));
 }
 
 // Section offsets of a record of format fmt (the header's MOE_FMT_* layouts).
@@ -89,7 +88,7 @@ int max_jobs(const moe_dims *d, int T) {
 // for the largest call (max_rows); the prefill buffers exist when max_rows > 32.
 struct WsLayout {
     int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, lk, rowrefs, xh, hh, part, cnt, fill,
-        jobidx, h32, xq, xq_scales, xq_st, hq, hq_scales, hq_st, pairs, n_pairs, xstage, ystage, total;
+        jobidx, h32, xq, xq_scales, xq_st, hq, hq_scales, hq_st, pairs, n_pairs, sg, hs, xstage, ystage, total;
 };
 int pairs_capacity(const moe_dims *d) {
     return grouped_pairs_cap(d->E, d->max_rows, d->k, d->has_shared ? 1 : 0);
@@ -128,6 +127,11 @@ WsLayout ws_layout(const moe_dims *d) {
     w.hq_st = prefill ? take(R * 4) : -1;
     w.pairs = prefill ? take((int64_t)pairs_capacity(d) * 8) : -1;
     w.n_pairs = prefill ? take(4) : -1;
+    // a BF16 shared expert on the prefill path: its gate/up outputs [T][2F] fp32
+    // and h as bf16 (hi, lo) halves [T][2F]
+    const bool sbf = prefill && d->has_shared && d->shared_format == MOE_FMT_BF16;
+    w.sg = sbf ? take(T * 2 * F * 4) : -1;
+    w.hs = sbf ? take(T * 2 * F * 2) : -1;
     w.xstage = take(T * dd * 2);
     w.ystage = take(T * dd * 4);
     w.total = o;
@@ -204,6 +208,9 @@ struct moe_ctx {
     bool fused = false;
     double wait_limit = 60.0;
     std::chrono::steady_clock::time_point issue_t0;  // end of the last miss-list wait
+    // prefill with a BF16 shared expert: its gate/up outputs and bf16 (hi, lo) h
+    float *dws_sg = nullptr;
+    uint16_t *dws_hs = nullptr;
     // device spans of timed launches: [slot][2] = {min start, min ~end}, all ones when free
     unsigned long long *kspan = nullptr;
     int64_t kspan_cap = 0, kspan_used = 0;
@@ -683,11 +690,18 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
         ra.publish = 0;
         --ctx->inj_drop_publish;
     }
+    // the shared expert is a job of the grouped GEMMs when it has the routed
+    // format; a BF16 one runs as two bf16 GEMMs of its own
+    const bool sep = shared_separate(ctx);
+    const int grouped_shared = (D.has_shared && !sep) ? 1 : 0;
+    const bool mx = ctx->lay.fmt == kFmtMxfp4;
     CK(cudaMemsetAsync(ctx->dws.cnt, 0, (size_t)D.E * 4, ctx->cs));
     TimedLaunch tr;
     time_begin(ctx, tr, MOE_K_PREFILL_ROUTE);
     CUtensorMap tm_x;  // logits on the tensor cores when x's rows can be TMA boxes
-    if (make_operand_map(&tm_x, x, 2 * (int64_t)D.d, T, 0, 0)) {
+    const bool x_map = make_operand_map(&tm_x, x, 2 * (int64_t)D.d, T, 0, 0);
+    if (sep && !x_map) return MOE_ERR_UNSUPPORTED;  // (x is 16-byte aligned and d a multiple of 64: not reached)
+    if (x_map) {
         CK(launch_router_gemm(tm_x, ctx->maps.router, ctx->dws.z, T, D.E, D.d, layer, ctx->page_d, ctx->cs));
         CK(launch_prefill_select(ra, ctx->cs));
     } else {
@@ -695,10 +709,10 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     }
     time_end(ctx, tr, (double)D.E * D.d * 2 + (double)T * D.d * 2);
     CK(launch_prefill_scatter(ra, ctx->cs));
-    CK(launch_tile_plan(ctx->dws.jobs, ctx->dws.n_jobs, T, D.has_shared, ctx->dws.pairs, ctx->dws.n_pairs,
+    CK(launch_tile_plan(ctx->dws.jobs, ctx->dws.n_jobs, T, grouped_shared, ctx->dws.pairs, ctx->dws.n_pairs,
                         ctx->cs));
-    CK(launch_quant_x_grouped(ra.x, T, D.k, D.d, D.has_shared, ctx->dws.rowrefs, ctx->dws.xq,
-                              ctx->dws.xq_scales, ctx->dws.xq_st, ctx->cs));
+    CK(launch_quant_x_grouped(ra.x, T, D.k, D.d, grouped_shared, ctx->dws.rowrefs, ctx->dws.xq,
+                              ctx->dws.xq_scales, ctx->dws.xq_st, mx ? 1 : 0, ctx->cs));
 
     const moe_status ws_ = wait_miss_list(ctx, seq);
     if (ws_ != MOE_OK) return ws_;
@@ -771,8 +785,8 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
 
     // experts: grouped tensor-core GEMMs -- gate/up (+SwiGLU, fp32 h), h
     // quantized per row, down -- then the gate-weighted combine
-    const int grid_y = n + (D.has_shared ? 1 : 0);
-    const int cap = grouped_pairs_cap(n, T, D.k, D.has_shared);
+    const int grid_y = n + grouped_shared;
+    const int cap = grouped_pairs_cap(n, T, D.k, grouped_shared);
     GroupedGemmArgs gu{};
     gu.mode = kGateUp;
     gu.jobs = ctx->dws.jobs;
@@ -787,7 +801,7 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     gu.F = D.F;
     gu.arena = ctx->arena;
     gu.rec_bytes = ctx->lay.bytes;
-    gu.shared_rec = D.has_shared ? ctx->shared_recs : nullptr;
+    gu.shared_rec = grouped_shared ? ctx->shared_recs : nullptr;
     gu.lay = ctx->lay;
     gu.act_scales = ctx->dws.xq_scales;
     gu.act_st = ctx->dws.xq_st;
@@ -800,9 +814,9 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     gu.span = time_span(ctx, tg);
     CK(launch_grouped_gemm(ctx->maps, gu, cap, ctx->cs));
     time_end(ctx, tg, grid_y * w13_bytes(ctx));
-    const int grouped_rows = T * D.k + (D.has_shared ? T : 0);
+    const int grouped_rows = T * D.k + (grouped_shared ? T : 0);
     CK(launch_quant_h_grouped(ctx->dws.h32, grouped_rows, D.F, ctx->dws.hq, ctx->dws.hq_scales,
-                              ctx->dws.hq_st, ctx->cs));
+                              ctx->dws.hq_st, mx ? 1 : 0, ctx->cs));
     GroupedGemmArgs dn = gu;
     dn.mode = kDown;
     dn.m_tiles = (D.d + 127) / 128;
@@ -813,6 +827,18 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     dn.span = time_span(ctx, td);
     CK(launch_grouped_gemm(ctx->maps, dn, cap, ctx->cs));
     time_end(ctx, td, grid_y * w2_bytes(ctx));
+    if (sep) {  // BF16 shared expert: [g u] = x W13^T, h = silu(g) u as bf16 (hi, lo), W2 h into part[t][k]
+        TimedLaunch sg_t, sd_t;
+        time_begin(ctx, sg_t, MOE_K_PREFILL_GATEUP);
+        CK(launch_bf16_gemm(tm_x, ctx->maps.w13_sbf, ctx->dws_sg, 2 * (int64_t)D.F, T, 2 * D.F, 2 * D.d, 0, layer,
+                            ctx->page_d, ctx->cs));
+        time_end(ctx, sg_t, 2.0 * 2 * D.F * D.d + (double)T * D.d * 2);
+        CK(launch_swiglu_split(ctx->dws_sg, T, D.F, ctx->dws_hs, ctx->cs));
+        time_begin(ctx, sd_t, MOE_K_PREFILL_DOWN);
+        CK(launch_bf16_gemm(ctx->maps.hs, ctx->maps.w2_sbf, ctx->dws.part + (int64_t)D.k * D.d,
+                            (int64_t)(D.k + 1) * D.d, T, D.d, 4 * D.F, 2 * D.F, layer, ctx->page_d, ctx->cs));
+        time_end(ctx, sd_t, 2.0 * D.d * D.F + (double)T * D.F * 4);
+    }
     CK(launch_combine(ctx->dws.part, ctx->dws.gates, y, T, D.k, D.d, D.has_shared, ctx->cs));
 
     int64_t hits = 0, evictions = 0, pf_evict = 0;
@@ -936,11 +962,19 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
                   make_operand_map(&ctx->maps.hq, ctx->dws.hq, dims->F / 2, R, 0, 0) &&
                   make_operand_map(&ctx->maps.router, router_w, 2 * (int64_t)dims->d, dims->E, dims->L,
                                    2 * (int64_t)dims->E * dims->d);
-        if (ok && dims->has_shared) {
+        if (ok && dims->has_shared && ctx->slay.fmt == lay.fmt) {  // the shared expert as a grouped-GEMM job
             ok = make_operand_map(&ctx->maps.w13_shared, ctx->shared_recs + lay.w13_codes, dims->d / 2,
                                   2 * dims->F, dims->L, ctx->slay.bytes) &&
                  make_operand_map(&ctx->maps.w2_shared, ctx->shared_recs + lay.w2_codes, dims->F / 2, dims->d,
                                   dims->L, ctx->slay.bytes);
+        } else if (ok && dims->has_shared) {  // a BF16 shared expert: two bf16 GEMMs of its own
+            ctx->dws_sg = reinterpret_cast<float *>(w + L.sg);
+            ctx->dws_hs = reinterpret_cast<uint16_t *>(w + L.hs);
+            ok = make_operand_map(&ctx->maps.w13_sbf, ctx->shared_recs + ctx->slay.w13_codes, 2 * (int64_t)dims->d,
+                                  2 * dims->F, dims->L, ctx->slay.bytes) &&
+                 make_operand_map(&ctx->maps.w2_sbf, ctx->shared_recs + ctx->slay.w2_codes, 2 * (int64_t)dims->F,
+                                  dims->d, dims->L, ctx->slay.bytes) &&
+                 make_operand_map(&ctx->maps.hs, ctx->dws_hs, 4 * (int64_t)dims->F, dims->max_rows, 0, 0);
         }
         if (!ok) {
             delete ctx;
@@ -1024,7 +1058,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
             ctx->configured = false;
             return MOE_ERR_UNSUPPORTED;
         }
-        if (!D.has_shared) {
+        if (!D.has_shared || shared_separate(ctx)) {  // no shared job in the grouped GEMMs
             ctx->maps.w13_shared = ctx->maps.w13;
             ctx->maps.w2_shared = ctx->maps.w2;
         }

@@ -217,6 +217,8 @@ struct GroupedGemmArgs {
 struct GroupedGemmMaps {
     CUtensorMap w13, w2, w13_shared, w2_shared, xq, hq;
     CUtensorMap router;  // router weights (3D: byte, expert row, layer) for the logits GEMM
+    // a BF16 shared expert: W13 and W2 of the L records (3D), and its h as bf16 (hi, lo) halves (2D)
+    CUtensorMap w13_sbf, w2_sbf, hs;
 };
 
 // Launch timing: slot[0] = min over CTAs of the start time, slot[1] = min of
@@ -246,11 +248,12 @@ cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_select(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
                            int has_shared, cudaStream_t s);
+// mx = 0: NVFP4 (E4M3 per 16 + fp32 row scale st); mx = 1: MXFP4 (E8M0 per 32, st unused)
 cudaError_t launch_quant_x_grouped(const __nv_bfloat16 *x, int T, int k, int d, int has_shared,
                                    const RowRef *rowrefs, uint8_t *codes, uint8_t *scales, float *st,
-                                   cudaStream_t s);
+                                   int mx, cudaStream_t s);
 cudaError_t launch_quant_h_grouped(const float *h32, int rows, int F, uint8_t *codes, uint8_t *scales,
-                                   float *st, cudaStream_t s);
+                                   float *st, int mx, cudaStream_t s);
 int grouped_pairs_cap(int n_jobs, int T, int k, int has_shared);
 cudaError_t launch_tile_plan(const Job *jobs, const int32_t *n_jobs, int T, int has_shared, int2 *pairs,
                              int32_t *n_pairs, cudaStream_t s);
@@ -258,6 +261,15 @@ cudaError_t launch_grouped_gemm(const GroupedGemmMaps &maps, const GroupedGemmAr
                                 cudaStream_t s);
 cudaError_t launch_router_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, float *z, int T, int E, int d,
                                int layer, HostPage *page, cudaStream_t s);
+// out[t * out_stride + n] = sum_K A[t][K] B[n][K] (bf16, fp32 accumulation) for
+// t < M, n < N; kbytes of K per A row; B's K coordinate modulo wrap bytes (0: none);
+// zb: B's matrix in its 3D map.  kbytes and wrap multiples of 128.
+cudaError_t launch_bf16_gemm(const CUtensorMap &tm_a, const CUtensorMap &tm_b, float *out, int64_t out_stride,
+                             int M, int N, int kbytes, int wrap, int zb, HostPage *page, cudaStream_t s);
+// h = silu(g) * u from the gate/up GEMM's [T][2F] output (gate_j in column 2j,
+// up_j in 2j + 1), written as bf16 halves: hs[t][j] = bf16(h), hs[t][F + j] =
+// bf16(h - that), so that hi + lo keeps about 16 bits of h.
+cudaError_t launch_swiglu_split(const float *sg, int T, int F, uint16_t *hs, cudaStream_t s);
 bool make_operand_map(CUtensorMap *out, const void *base, int64_t row_bytes, int64_t rows, int64_t count,
                       int64_t matrix_stride);
 

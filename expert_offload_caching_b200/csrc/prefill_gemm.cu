@@ -154,6 +154,20 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");
 }
+// MXFP4 x MXFP4: E2M1 with one UE8M0 scale per 32 values on each side (OCP
+// microscaling); per MMA (K = 64) each row has two scales, in the low two bytes
+// of its 32-bit scale-factor column (scale-factor id 0).
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+        "}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
 // arrive on the mbarrier once every tcgen05 operation issued so far by this thread is done
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -216,9 +230,14 @@ __device__ void gemm_fail(const GroupedGemmArgs &a, int code, int stage) {
     __threadfence_system();
 }
 
+// FMT: the records' format.  NVFP4: E4M3 scales per 16 (kind::mxf4nvf4
+// block16), per-matrix and per-row fp32 scales in the epilogue.  MXFP4: E8M0
+// scales per 32 (kind::mxf4 block32), nothing else to apply.
+template <int FMT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_ws,
                         const __grid_constant__ CUtensorMap tm_act, const GroupedGemmArgs a) {
+    constexpr bool kMx = FMT == kFmtMxfp4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int pair = (int)blockIdx.x / a.m_tiles, mt = (int)blockIdx.x % a.m_tiles;
     if (pair >= *a.n_pairs) return;  // grid sized for the worst case
@@ -247,9 +266,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int rows_w = gate_up ? 2 * a.F : a.d;
     const int ksteps = K >> 6;
     const int nkb = (ksteps + kStepsPerStage - 1) / kStepsPerStage;
-    const int sf_pitch = K >> 4;  // scale bytes per row, weights and activations alike
+    const int sf_pitch = kMx ? K >> 5 : K >> 4;  // scale bytes per row, weights and activations alike
     const uint8_t *wsf = rec + (gate_up ? a.lay.w13_scales : a.lay.w2_scales);
-    const float *tsc = reinterpret_cast<const float *>(rec + a.lay.tscales);
+    const float *tsc = kMx ? nullptr : reinterpret_cast<const float *>(rec + a.lay.tscales);
 
     extern __shared__ uint8_t dsm_raw[];
     const uint32_t raw = saddr(dsm_raw);
@@ -291,14 +310,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 // row m = lane + 32c of the tile; its 4 scales of a K step are one word
                 const int wrow = mt * kBM + lane + 32 * c;
                 const int n = n0 + lane + 32 * c;
-                const uint32_t *pw = reinterpret_cast<const uint32_t *>(wsf + (int64_t)wrow * sf_pitch);
-                const uint32_t *pb =
-                    reinterpret_cast<const uint32_t *>(a.act_scales + (int64_t)(row_off + n) * sf_pitch);
+                const uint8_t *pw = wsf + (int64_t)wrow * sf_pitch;
+                const uint8_t *pb = a.act_scales + (int64_t)(row_off + n) * sf_pitch;
 #pragma unroll
                 for (int i = 0; i < kStepsPerStage; ++i) {
                     const int ks = itl * kStepsPerStage + i;
-                    wa[c][i] = (wrow < rows_w && ks < ksteps) ? __ldg(pw + ks) : 0u;
-                    wb[c][i] = (n < nrows && ks < ksteps) ? __ldg(pb + ks) : 0u;
+                    if constexpr (kMx) {  // two E8M0 bytes, as bytes 0-1 (and again 2-3) of the word
+                        const uint32_t va = (wrow < rows_w && ks < ksteps)
+                                                ? __ldg(reinterpret_cast<const uint16_t *>(pw) + ks) : 0u;
+                        const uint32_t vb = (n < nrows && ks < ksteps)
+                                                ? __ldg(reinterpret_cast<const uint16_t *>(pb) + ks) : 0u;
+                        wa[c][i] = va | (va << 16);
+                        wb[c][i] = vb | (vb << 16);
+                    } else {
+                        wa[c][i] = (wrow < rows_w && ks < ksteps) ? __ldg(reinterpret_cast<const uint32_t *>(pw) + ks) : 0u;
+                        wb[c][i] = (n < nrows && ks < ksteps) ? __ldg(reinterpret_cast<const uint32_t *>(pb) + ks) : 0u;
+                    }
                 }
             }
         };
@@ -338,7 +365,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ---- MMA issue, one thread
         if (lane == 0) {
-            const uint32_t idesc = idesc_nvf4(N);
+            const uint32_t idesc = idesc_nvf4(N) | (kMx ? (1u << 23) : 0u);  // bit 23: UE8M0 scales
             for (int it = 0; it < nkb; ++it) {
                 const int s = it % kStages, r = it / kStages;
                 if (!mbar_wait(bar_full + 8 * s, r & 1)) {
@@ -355,8 +382,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t t_sfb = t_sfa + 4;
                     tc_cp_sf(t_sfa, desc_sf(base + kOffSfA + (s * kStepsPerStage + i) * kSfAtom));
                     tc_cp_sf(t_sfb, desc_sf(base + kOffSfB + (s * kStepsPerStage + i) * kSfAtom));
-                    tc_mma_nvf4(tmem, desc_sw128(da + 32 * i), desc_sw128(db + 32 * i), idesc, t_sfa, t_sfb,
-                                (it | i) != 0 ? 1u : 0u);
+                    if constexpr (kMx)
+                        tc_mma_mxf4(tmem, desc_sw128(da + 32 * i), desc_sw128(db + 32 * i), idesc, t_sfa, t_sfb,
+                                    (it | i) != 0 ? 1u : 0u);
+                    else
+                        tc_mma_nvf4(tmem, desc_sw128(da + 32 * i), desc_sw128(db + 32 * i), idesc, t_sfa, t_sfb,
+                                    (it | i) != 0 ? 1u : 0u);
                 }
                 tc_commit(bar_empty + 8 * s);
             }
@@ -375,7 +406,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int wrow = mt * kBM + m;
             const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
             if (gate_up) {
-                const float ts_g = tsc[0], ts_u = tsc[1];
+                const float ts_g = kMx ? 1.0f : tsc[0], ts_u = kMx ? 1.0f : tsc[1];
                 for (int c0 = 0; c0 < N; c0 += 16) {
                     float v[16];
                     tmem_ld16(trow + (uint32_t)c0, v);
@@ -385,7 +416,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const int n = c0 + cc;
                         if ((lane & 1) == 0 && n < nvalid && wrow < rows_w) {
                             const int g = row_off + n0 + n;
-                            const float st = a.act_st[g];
+                            const float st = kMx ? 1.0f : a.act_st[g];
                             const float gt = v[cc] * ts_g * st;   // row 2j: gate_j
                             const float up = other * ts_u * st;   // row 2j + 1: up_j
                             a.h32[(int64_t)g * a.F + (wrow >> 1)] = gt / (1.0f + expf(-gt)) * up;
@@ -393,7 +424,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             } else {
-                const float ts_d = tsc[2];
+                const float ts_d = kMx ? 1.0f : tsc[2];
                 const int tk = a.T * a.k;
                 for (int c0 = 0; c0 < N; c0 += 16) {
                     float v[16];
@@ -412,7 +443,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 t = g - tk;
                                 p = a.k;
                             }
-                            a.part[((int64_t)t * (a.k + 1) + p) * a.d + wrow] = v[cc] * ts_d * a.act_st[g];
+                            a.part[((int64_t)t * (a.k + 1) + p) * a.d + wrow] =
+                                v[cc] * ts_d * (kMx ? 1.0f : a.act_st[g]);
                         }
                     }
                 }
@@ -465,12 +497,15 @@ __global__ void __launch_bounds__(1024) tile_plan_kernel(const Job *jobs, const 
     if (j == 0) *n_pairs = s_total + nsh;
 }
 
-// ---- router logits of a prefill chunk: z = x W_r^T on the tensor cores
-// (tcgen05.mma kind::f16, bf16 x bf16 -> fp32 in tensor memory).  One CTA per
-// 128 rows x 128 experts; K (d) streamed through a 4-deep ring of TMA boxes
-// (128 bytes = 64 bf16 of K, 128-byte swizzle; 4 MMAs of K = 16 per box).
-// The products are exact in fp32; only the summation order differs from an
-// fp32 FMA chain.
+// ---- bf16 x bf16 -> fp32 GEMM on the tensor cores (tcgen05.mma kind::f16,
+// accumulators in tensor memory): out[t][n] = sum_K A[t][K] B[n][K], A and B
+// K-major bf16 (TMA boxes of 128 bytes = 64 values of K, 128-byte swizzle,
+// 4 MMAs of K = 16 per box, a 4-deep ring).  One CTA per 128 rows of A x 128
+// rows of B.  The products are exact in fp32; only the summation order
+// differs from an fp32 FMA chain.  Uses: the router logits of a prefill chunk
+// (A = x, B = W_r of the layer) and a BF16 shared expert (A = x, B = W13; then
+// A = h as bf16 (hi, lo) halves, B = W2 with K wrapped: K positions j and F + j
+// both read W2's column j, so hi and lo meet W2 in one accumulation).
 constexpr int kRStages = 4;
 constexpr uint32_t kROffBar = 2 * kRStages * kTileBytes;
 constexpr uint32_t kRSmemBytes = kROffBar + 128 + 1024;
@@ -504,12 +539,14 @@ __device__ void router_fail(HostPage *page, int code, int stage) {
     __threadfence_system();
 }
 
+// kbytes: bytes of K per row of A; wrap: B's K coordinate is taken modulo wrap
+// bytes (0: no wrap); zb: B's matrix index (layer) in its 3D map.
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                       float *z, int T, int E, int d, int layer, HostPage *page) {
+    bf16_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                     float *z, int64_t z_stride, int T, int E, int kbytes, int wrap, int layer, HostPage *page) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * kBM, e0 = blockIdx.y * kBM;
-    const int nkb = (2 * d + kStageKBytes - 1) / kStageKBytes;
+    const int nkb = (kbytes + kStageKBytes - 1) / kStageKBytes;
     extern __shared__ uint8_t dsm_raw[];
     const uint32_t raw = saddr(dsm_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -549,7 +586,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 mbar_arrive_tx(bar_full + 8 * s, 2 * kTileBytes);
                 tma_load_2d(base + s * kTileBytes, &tm_x, bar_full + 8 * s, it * kStageKBytes, t0);
-                tma_load_3d(base + (kRStages + s) * kTileBytes, &tm_w, bar_full + 8 * s, it * kStageKBytes, e0,
+                const int kb = it * kStageKBytes;
+                tma_load_3d(base + (kRStages + s) * kTileBytes, &tm_w, bar_full + 8 * s, wrap ? kb % wrap : kb, e0,
                             layer);
             }
             if (it < nkb)  // let the stages already issued land before the CTA exits
@@ -569,7 +607,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t da = base + s * kTileBytes, db = base + (kRStages + s) * kTileBytes;
-                const int steps = min(4, (2 * d - it * kStageKBytes) / 32);  // K = 16 bf16 = 32 bytes each
+                const int steps = min(4, (kbytes - it * kStageKBytes) / 32);  // K = 16 bf16 = 32 bytes each
                 for (int i = 0; i < steps; ++i)
                     tc_mma_bf16(tmem, desc_sw128(da + 32 * i), desc_sw128(db + 32 * i), idesc, (it | i) != 0);
                 tc_commit(bar_empty + 8 * s);
@@ -590,7 +628,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 float v[16];
                 tmem_ld16(trow + (uint32_t)c0, v);
                 if (t < T) {
-                    float *zr = z + (size_t)t * E + e0 + c0;
+                    float *zr = z + (size_t)t * z_stride + e0 + c0;
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         if (e0 + c0 + i < E) zr[i] = v[i];
@@ -608,18 +646,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_router_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, float *z, int T, int E, int d,
-                               int layer, HostPage *page, cudaStream_t s) {
+cudaError_t launch_bf16_gemm(const CUtensorMap &tm_a, const CUtensorMap &tm_b, float *out, int64_t out_stride,
+                             int M, int N, int kbytes, int wrap, int zb, HostPage *page, cudaStream_t s) {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(bf16_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kRSmemBytes);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const dim3 grid((T + kBM - 1) / kBM, (E + kBM - 1) / kBM);
-    router_gemm_kernel<<<grid, kGemmThreads, kRSmemBytes, s>>>(tm_x, tm_w, z, T, E, d, layer, page);
+    if ((kbytes % kStageKBytes) || (wrap % kStageKBytes)) return cudaErrorInvalidValue;  // whole TMA boxes
+    const dim3 grid((M + kBM - 1) / kBM, (N + kBM - 1) / kBM);
+    bf16_gemm_kernel<<<grid, kGemmThreads, kRSmemBytes, s>>>(tm_a, tm_b, out, out_stride, M, N, kbytes, wrap, zb,
+                                                             page);
     return cudaGetLastError();
+}
+
+cudaError_t launch_router_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, float *z, int T, int E, int d,
+                               int layer, HostPage *page, cudaStream_t s) {
+    return launch_bf16_gemm(tm_x, tm_w, z, E, T, E, 2 * d, 0, layer, page, s);
 }
 
 
@@ -638,8 +683,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemmMaps &maps, const GroupedGemmAr
                                 cudaStream_t s) {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kFmtNvfp4>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(grouped_gemm_kernel<kFmtMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -648,7 +696,12 @@ cudaError_t launch_grouped_gemm(const GroupedGemmMaps &maps, const GroupedGemmAr
     const CUtensorMap &act = a.mode == kGateUp ? maps.xq : maps.hq;
     const unsigned grid = (unsigned)pairs_cap * (unsigned)a.m_tiles;
     if (grid == 0) return cudaSuccess;
-    grouped_gemm_kernel<<<grid, kGemmThreads, kSmemBytes, s>>>(w, ws, act, a);
+    if (a.lay.fmt == kFmtMxfp4)
+        grouped_gemm_kernel<kFmtMxfp4><<<grid, kGemmThreads, kSmemBytes, s>>>(w, ws, act, a);
+    else if (a.lay.fmt == kFmtNvfp4)
+        grouped_gemm_kernel<kFmtNvfp4><<<grid, kGemmThreads, kSmemBytes, s>>>(w, ws, act, a);
+    else
+        return cudaErrorInvalidValue;
     return cudaGetLastError();
 }
 

@@ -95,8 +95,10 @@ typedef struct {
  * off[3] W2 scales [d x F/32], 256-byte aligned, off[4] = -1, off[5] total.
  * BF16 (shared experts only; florigen.ai "NVFP4で約135GBまで縮める" keeps
  * them in BF16): W13 [2F x d] bf16 (row 2j = gate_j, 2j+1 = up_j) at 0, then
- * W2 [d x F] at 4Fd bytes; 6Fd bytes.  MXFP4 and BF16 run on the decode path
- * only (max_rows <= 32, else MOE_ERR_UNSUPPORTED). */
+ * W2 [d x F] at 4Fd bytes; 6Fd bytes.  On the prefill path MXFP4 experts are
+ * W4A4 with MXFP4 activations (OCP: E8M0 scale 2^e per 32 values, e =
+ * floor(log2 amax) - 2, E2M1 codes, no row scale) and a BF16 shared expert is
+ * not quantized (bf16 GEMMs, fp32 accumulation, h carried as bf16 (hi, lo)). */
 #define MOE_FMT_NVFP4 0
 #define MOE_FMT_MXFP4 1
 #define MOE_FMT_BF16 2
@@ -210,8 +212,8 @@ MOE_API size_t moe_arena_bytes(const moe_dims *dims, int64_t num_slots);
  *   compute_stream, copy_stream: cudaStream_t handles (NULL = legacy stream not
  *              accepted: pass real streams); work is issued on them only.
  * Shapes handled: d and F multiples of 64, 1 <= k <= 32, k <= E <= 1024,
- * 1 <= max_rows <= 4096, and with max_rows > 32 (prefill) d >= 256,
- * F >= 256 and NVFP4 records only; else MOE_ERR_UNSUPPORTED.  MOE_ERR_ARG for
+ * 1 <= max_rows <= 4096, and with max_rows > 32 (prefill) d >= 256 and
+ * F >= 256; else MOE_ERR_UNSUPPORTED.  MOE_ERR_ARG for
  * an unknown format, a BF16 routed format, or (has_shared) a shared format
  * that is neither the routed one nor BF16. */
 MOE_API moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t host_pool_bytes,
@@ -246,16 +248,21 @@ MOE_API moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_a
  * the device's miss list; on timeout it returns MOE_ERR_TIMEOUT and the
  * context is in MOE_ERR_STATE until a reset.  T <= 32 takes the decode path
  * (W4A16: bf16 activations against NVFP4 or MXFP4 weights; a BF16 shared
- * expert runs in its own two launches before the routed ones).  Larger T takes the
- * prefill path: the activations are quantized to NVFP4 per row (E2M1 values,
- * E4M3 scale per 16, one fp32 scale per row: x per token, h per token and
- * expert) and multiplied against the NVFP4 weights (W4A4); the lookup batch is
+ * expert runs in its own two launches before the routed ones; where stream
+ * memory writes work, every expert GEMV of the layer runs in one persistent
+ * launch that starts each miss when the copy stream flags its record, else
+ * each miss gets its own launches gated by copy events).  Larger T takes the
+ * prefill path: the activations are quantized like the weights -- NVFP4 per
+ * row (E2M1 values, E4M3 scale per 16, one fp32 scale per row: x per token, h
+ * per token and expert), or MXFP4 (E8M0 per 32) for MXFP4 records -- and
+ * multiplied against the weights (W4A4); the lookup batch is
  * the layer's distinct experts, and with MOE_CACHE_PREFETCH_NEXT a second
  * batch of all experts of layer + 1 follows, whose misses are copied while
  * this layer computes (the next call for layer + 1 waits for them; records
  * with consecutive pool indices and slots go in one copy).  The expert FFNs
- * of a prefill call run as grouped block-scaled NVFP4 GEMMs on the tensor
- * cores (rows grouped by expert, fp32 accumulation).  The trace lists the
+ * of a prefill call run as grouped block-scaled FP4 GEMMs on the tensor cores
+ * (rows grouped by expert, fp32 accumulation); a BF16 shared expert as two
+ * bf16 GEMMs.  The trace lists the
  * routed entries, then the prefetch entries (prefetch = 1, layer + 1).
  * Any failure after the argument checks (MOE_ERR_CUDA, MOE_ERR_TIMEOUT, a
  * failed device check) leaves the context in MOE_ERR_STATE until

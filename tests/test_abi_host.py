@@ -142,16 +142,15 @@ def test_format_argument_checks_without_device():
     ok = abi.make_dims(2, 16, 2, 256, 512, False, weight_format=abi.MOE_FMT_MXFP4,
                        shared_format=abi.MOE_FMT_NVFP4)
     assert abi.moe_record_bytes(ok) == oracle.mx_record_layout(256, 512)[4]
-    # MXFP4 and BF16 records run on the decode path only
-    for wf, sf in ((abi.MOE_FMT_MXFP4, None), (abi.MOE_FMT_NVFP4, abi.MOE_FMT_BF16)):
-        pre = abi.make_dims(2, 16, 2, 256, 512, True, max_rows=64, weight_format=wf, shared_format=sf)
-        with pytest.raises(abi.MoeError) as ei:
-            abi.moe_layer_init(pre, fake, 1 << 30, fake, fake, fake, 1 << 40, fake, fake)
-        assert ei.value.status == abi.MOE_ERR_UNSUPPORTED
-        dec = abi.make_dims(2, 16, 2, 256, 512, True, max_rows=32, weight_format=wf, shared_format=sf)
-        with pytest.raises(abi.MoeError) as ei:  # accepted shape; then the fake pool is refused
-            abi.moe_layer_init(dec, fake, 1 << 30, fake, fake, fake, 1 << 40, fake, fake)
-        assert ei.value.status == abi.MOE_ERR_NOT_PINNED
+    # MXFP4 and BF16 records run on the decode and the prefill paths
+    for wf, sf in ((abi.MOE_FMT_MXFP4, None), (abi.MOE_FMT_NVFP4, abi.MOE_FMT_BF16),
+                   (abi.MOE_FMT_MXFP4, abi.MOE_FMT_BF16)):
+        for rows in (32, 64):
+            dims = abi.make_dims(2, 16, 2, 256, 512, True, max_rows=rows, weight_format=wf,
+                                 shared_format=sf)
+            with pytest.raises(abi.MoeError) as ei:  # accepted shape; then the fake pool is refused
+                abi.moe_layer_init(dims, fake, 1 << 30, fake, fake, fake, 1 << 40, fake, fake)
+            assert ei.value.status == abi.MOE_ERR_NOT_PINNED
 
 
 def test_size_queries_and_init_checks_over_random_dims():

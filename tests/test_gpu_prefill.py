@@ -24,20 +24,24 @@ PF = synth.LayerShape("pf-mid", L=3, E=40, k=5, d=960, F=320, shared=True, token
 
 
 class PrefillProblem:
-    def __init__(self, shape, T, P=None, C=None, distinct=None):
+    def __init__(self, shape, T, P=None, C=None, distinct=None, fmt=sp.FMT_NVFP4, shared_fmt=None):
         self.shape, self.T = shape, T
+        self.fmt = fmt
+        self.shared_fmt = fmt if shared_fmt is None else shared_fmt
         self.P = shape.L * shape.E if P is None else P
         self.C = shape.cache_slots if C is None else C
-        self.rb = synth.record_bytes(shape.d, shape.F)
+        self.rb = sp.format_record_bytes(fmt, shape.d, shape.F)
+        self.srb = sp.format_record_bytes(self.shared_fmt, shape.d, shape.F)
         self.Wr = sp.router_weights(shape)
-        self.shared = sp.shared_records(shape)
-        self.pool = sp.pinned_pool(shape, self.P, distinct)
+        self.shared = sp.shared_records_fmt(shape, self.shared_fmt)
+        self.pool = sp.pinned_pool_fmt(shape, fmt, self.P, distinct)
         self.x = np.stack([conditioned_prefill(self.Wr[l], shape.k, l, T)[0] for l in range(shape.L)])
 
     def stack(self, prefetch, max_rows=None):
         sh = self.shape
         dims = abi.make_dims(sh.L, sh.E, sh.k, sh.d, sh.F, sh.shared, True, max_rows or self.T,
-                             0 if self.P == sh.L * sh.E else self.P)
+                             0 if self.P == sh.L * sh.E else self.P, weight_format=self.fmt,
+                             shared_format=self.shared_fmt)
         return LayerStack(dims, self.pool, sp.to_device(self.Wr), sp.to_device(self.shared), self.C,
                           prefetch=prefetch)
 
@@ -58,9 +62,10 @@ class PrefillProblem:
 
     def oracle_y(self, l, rows):
         sh = self.shape
-        shared = None if self.shared is None else self.shared[l * self.rb:(l + 1) * self.rb]
+        shared = None if self.shared is None else self.shared[l * self.srb:(l + 1) * self.srb]
         return oracle.moe_layer(self.pool.numpy(), self.P, l, sh.E, sh.d, sh.F, sh.k, self.Wr[l],
-                                shared, self.x[l][rows], w4a4=True)[2]
+                                shared, self.x[l][rows], w4a4=True, fmt=self.fmt,
+                                shared_fmt=self.shared_fmt)[2]
 
 
 def _check(pb, st, events, idx, gates, y, prefetch, rows=None):
@@ -138,7 +143,7 @@ def test_prefill_then_concurrent_decode_continues_the_cache():
     want, _ = decode_trace(didx, sh.L, sh.E, pb.C, lru=lru)
     assert got == want
     ydn = yd.cpu().numpy()
-    shared = [pb.shared[l * pb.rb:(l + 1) * pb.rb] for l in range(sh.L)]
+    shared = [pb.shared[l * pb.srb:(l + 1) * pb.srb] for l in range(sh.L)]
     for t in range(steps):
         for l in range(sh.L):
             want_y = oracle.moe_layer(pb.pool.numpy(), pb.P, l, sh.E, sh.d, sh.F, sh.k, pb.Wr[l],
@@ -176,4 +181,35 @@ def test_prefill_static_split_policy():
     assert events == want
     for l in range(sh.L):
         _check_rows(y[l], pb.oracle_y(l, np.arange(T)), l)
+    st.close()
+
+
+@pytest.mark.parametrize("fmt,shared_fmt", [(sp.FMT_MXFP4, None), (sp.FMT_MXFP4, sp.FMT_BF16),
+                                            (sp.FMT_NVFP4, sp.FMT_BF16)],
+                         ids=["mxfp4", "mxfp4+bf16-shared", "nvfp4+bf16-shared"])
+def test_prefill_record_formats(fmt, shared_fmt):
+    """Prefill over MXFP4 routed records (W4A4 with MXFP4 activations: E8M0 per
+    32, kind::mxf4 block32 tensor-core GEMMs) and with a BF16 shared expert (two
+    bf16 tensor-core GEMMs, h as bf16 (hi, lo) halves); ragged K tails of the
+    mid shape, prefetch on; bit-exact routing, trace, table; every row within
+    the bar against the oracle's W4A4 layer of those formats."""
+    pb = PrefillProblem(PF, T=200, fmt=fmt, shared_fmt=shared_fmt)
+    st = pb.stack(True)
+    events, idx, gates, y = pb.run(st)
+    _check(pb, st, events, idx, gates, y, True)
+    st.close()
+
+
+def test_prefill_mxfp4_full_chunk_gpt_oss_shaped_two_layers():
+    """The 4096-row chunk on gpt-oss-120b-shaped MXFP4 layers (128 experts,
+    top-4, d = F = 2880: 45 K-steps of 64, a ragged stage), two layers with
+    prefetch; sampled rows."""
+    full = synth.GPT_OSS
+    sh = synth.LayerShape(full.name, L=2, E=full.E, k=full.k, d=full.d, F=full.F, shared=False,
+                          tokens=0, cache_slots=2 * full.E)
+    pb = PrefillProblem(sh, T=4096, P=61, fmt=sp.FMT_MXFP4)
+    st = pb.stack(True)
+    events, idx, gates, y = pb.run(st)
+    rows = np.sort(np.random.default_rng(4).choice(4096, 16, replace=False))
+    _check(pb, st, events, idx, gates, y, True, rows=rows)
     st.close()
