@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_layer_kernel(LayerArgs 
     const int nwarps = (int)(blockDim.x >> 5);
     float(*red)[NG][4][32] = reinterpret_cast<float(*)[NG][4][32]>(smem + S * buf_bytes);
 
-    // issue the copies of the j-th claimed item into buffer j % S (no commit)
+    // issue the copies of the j-th claimed item into buffer j % S (no commit);
+    // weights are read once per layer: evict-first in L2
+    const uint64_t ef = evict_first_policy();
     auto issue = [&](int i, int j) {
         const Item it = decode(i);
         const int K = it.gate_up ? a.d : a.F;
@@ -176,9 +178,10 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_layer_kernel(LayerArgs 
         uint8_t *dst = smem + (j % S) * buf_bytes;
         const uint8_t *codes = rec + (it.gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)it.tile * code_bytes;
         const uint8_t *scales = rec + (it.gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)it.tile * scale_bytes;
-        for (uint32_t o = threadIdx.x; o < (code_bytes >> 4); o += blockDim.x) cp_async16(dst + 16 * o, codes + 16 * o);
+        for (uint32_t o = threadIdx.x; o < (code_bytes >> 4); o += blockDim.x)
+            cp_async16_ef(dst + 16 * o, codes + 16 * o, ef);
         for (uint32_t o = threadIdx.x; o < (scale_bytes >> 4); o += blockDim.x)
-            cp_async16(dst + code_bytes + 16 * o, scales + 16 * o);
+            cp_async16_ef(dst + code_bytes + 16 * o, scales + 16 * o, ef);
         if (it.gate_up && it.miss < 0) {  // a resident expert's down projection -> L2 (a 1/nA slice)
             const uint32_t tot = (uint32_t)(a.lay.bytes - a.lay.w2_codes);
             const uint32_t sl = ((tot / nA) + 127u) & ~127u;

@@ -529,7 +529,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         la.miss_flag = ctx->dws.lk_flags;
         la.release = ctx->dws.lk_release;
         la.seq = seq;
-        la.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 30.0) * 1e9);
+        la.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 5.0) * 1e9);
         la.page = ctx->page_d;
         TimedLaunch tk, th;
         time_begin(ctx, tk, MOE_K_LAYER);

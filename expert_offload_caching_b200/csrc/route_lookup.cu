@@ -457,62 +457,79 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     __syncthreads();
     if (threadIdx.x == 0) t_topk = global_ns();
     const int nsel = a.T * a.k;
-    for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
-        const int e = a.ws.idx[i];
-        s_idx[i] = e;
-        if ((unsigned)e < (unsigned)a.E) atomicOr(&s_bits[e >> 5], 1u << (e & 31));
-        else route_fail(a.page, 1, e, a.E);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const int c = __popc(s_bits[lane]);
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
+    if (a.T == 1) {
+        // one row: its k ids are already distinct and ascending -- they are the
+        // jobs, one row each, in selection order
+        for (int j = threadIdx.x; j < a.k; j += blockDim.x) {
+            int e = a.ws.idx[j];
+            if ((unsigned)e >= (unsigned)a.E) { route_fail(a.page, 1, e, a.E); e = 0; }
+            s_exp[j] = e;
+            s_cnt[j] = 1;
+            s_off[j] = j;
+            a.ws.rowrefs[j].t = 0;
+            a.ws.rowrefs[j].p = (int16_t)j;
         }
-        s_base[lane] = incl - c;
-        if (lane == 31) s_njobs = incl;
-    }
-    __syncthreads();
-    const int njobs = s_njobs;
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-        const uint32_t w = s_bits[e >> 5];
-        if (w & (1u << (e & 31))) s_exp[s_base[e >> 5] + __popc(w & ((1u << (e & 31)) - 1u))] = e;
-    }
-    __syncthreads();
-    for (int j = threadIdx.x; j < njobs; j += blockDim.x) {
-        int c = 0;
-        for (int i = 0; i < nsel; ++i) c += (s_idx[i] == s_exp[j]);
-        s_cnt[j] = c;
-    }
-    __syncthreads();
-    if (warp == 0) {  // exclusive scan of the counts, 32 at a time
-        int carry = 0;
-        for (int j0 = 0; j0 < njobs; j0 += 32) {
-            const int j = j0 + lane;
-            const int c = j < njobs ? s_cnt[j] : 0;
+        if (threadIdx.x == 0) s_njobs = a.k;
+        __syncthreads();
+    } else {
+        for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
+            const int e = a.ws.idx[i];
+            s_idx[i] = e;
+            if ((unsigned)e < (unsigned)a.E) atomicOr(&s_bits[e >> 5], 1u << (e & 31));
+            else route_fail(a.page, 1, e, a.E);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const int c = __popc(s_bits[lane]);
             int incl = c;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += y;
             }
-            if (j < njobs) s_off[j] = carry + incl - c;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
+            s_base[lane] = incl - c;
+            if (lane == 31) s_njobs = incl;
         }
-    }
-    __syncthreads();
-    for (int j = threadIdx.x; j < njobs; j += blockDim.x) {
-        int pos = s_off[j];
-        for (int i = 0; i < nsel; ++i)
-            if (s_idx[i] == s_exp[j]) {
-                a.ws.rowrefs[pos].t = (int16_t)(i / a.k);
-                a.ws.rowrefs[pos].p = (int16_t)(i % a.k);
-                ++pos;
+        __syncthreads();
+        const int nj = s_njobs;
+        for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+            const uint32_t w = s_bits[e >> 5];
+            if (w & (1u << (e & 31))) s_exp[s_base[e >> 5] + __popc(w & ((1u << (e & 31)) - 1u))] = e;
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < nj; j += blockDim.x) {
+            int c = 0;
+            for (int i = 0; i < nsel; ++i) c += (s_idx[i] == s_exp[j]);
+            s_cnt[j] = c;
+        }
+        __syncthreads();
+        if (warp == 0) {  // exclusive scan of the counts, 32 at a time
+            int carry = 0;
+            for (int j0 = 0; j0 < nj; j0 += 32) {
+                const int j = j0 + lane;
+                const int c = j < nj ? s_cnt[j] : 0;
+                int incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                if (j < nj) s_off[j] = carry + incl - c;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
             }
-    }
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < nj; j += blockDim.x) {
+            int pos = s_off[j];
+            for (int i = 0; i < nsel; ++i)
+                if (s_idx[i] == s_exp[j]) {
+                    a.ws.rowrefs[pos].t = (int16_t)(i / a.k);
+                    a.ws.rowrefs[pos].p = (int16_t)(i % a.k);
+                    ++pos;
+                }
+        }
+    }  // T > 1
+    const int njobs = s_njobs;
 
     __syncthreads();
     if (threadIdx.x == 0) t_jobs = global_ns();

@@ -301,7 +301,7 @@ MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
 MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
 
 /* Longest wait, in seconds (default 60): the host's wait for the device miss
- * list, and (capped at 30 s, counted from the kernel's start) every wait of the
+ * list, and (capped at 5 s, counted from the kernel's start) every wait of the
  * decode layer kernel for a miss's copy or for another CTA's tiles; a device
  * wait that runs out records a failed check (MOE_ERR_CUDA at the next call). */
 MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
