@@ -201,7 +201,7 @@ struct moe_ctx {
     std::vector<cudaEvent_t> ev_pool;
     std::vector<TimedLaunch> pending;
     // injection and limits
-    int64_t inj_copy_fail_at = 0, inj_drop_publish = 0, inj_drop_flags = 0;
+    int64_t inj_copy_fail_at = 0, inj_drop_publish = 0, inj_drop_flags = 0, inj_gemm_skip = 0;
     // decode: the persistent layer kernel (one launch per layer, misses gated
     // by flags the copy stream writes), when stream memory writes work here;
     // else a launch per miss, gated by events
@@ -809,6 +809,12 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     gu.h32 = ctx->dws.h32;
     gu.part = ctx->dws.part;
     gu.page = ctx->page_d;
+    gu.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 4.0) * 1e9);
+    gu.inj_skip = 0;
+    if (ctx->inj_gemm_skip > 0) {
+        --ctx->inj_gemm_skip;
+        gu.inj_skip = 1;
+    }
     TimedLaunch tg;
     time_begin(ctx, tg, MOE_K_PREFILL_GATEUP);
     gu.span = time_span(ctx, tg);
@@ -818,6 +824,7 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     CK(launch_quant_h_grouped(ctx->dws.h32, grouped_rows, D.F, ctx->dws.hq, ctx->dws.hq_scales,
                               ctx->dws.hq_st, mx ? 1 : 0, ctx->cs));
     GroupedGemmArgs dn = gu;
+    dn.inj_skip = 0;
     dn.mode = kDown;
     dn.m_tiles = (D.d + 127) / 128;
     dn.act_scales = ctx->dws.hq_scales;
@@ -1226,13 +1233,19 @@ moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds) {
 
 moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
     if (!ctx || n < 0) return MOE_ERR_ARG;
-    if (what == 0) { ctx->inj_copy_fail_at = 0; ctx->inj_drop_publish = 0; ctx->inj_drop_flags = 0; }
+    if (what == 0) {
+        ctx->inj_copy_fail_at = 0;
+        ctx->inj_drop_publish = 0;
+        ctx->inj_drop_flags = 0;
+        ctx->inj_gemm_skip = 0;
+    }
     else if (what == 1) ctx->inj_copy_fail_at = n;
     else if (what == 2) ctx->inj_drop_publish = n;
     else if (what == 3) {  // decode path: 0 = a launch per miss, 1 = the layer kernel
         if (n == 1 && stream_write(ctx->xs, ctx->dws.lk_release, 0u) != cudaSuccess) return MOE_ERR_UNSUPPORTED;
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;
+    else if (what == 5) ctx->inj_gemm_skip = n;
     else return MOE_ERR_ARG;
     return MOE_OK;
 }

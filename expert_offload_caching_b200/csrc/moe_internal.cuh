@@ -210,6 +210,8 @@ struct GroupedGemmArgs {
     float *part;              // down output: [T][k+1][d]
     HostPage *page;
     unsigned long long *span;  // launch timing slot (see span_mark), or null
+    unsigned long long wait_ns;  // bound of each mbarrier wait
+    int inj_skip;             // test injection: block 0 does not issue its first stage's copies
 };
 // TMA descriptors of the operands: weight codes of the slot arena (3D: byte,
 // row, slot) and of the shared records (3D: byte, row, layer); grouped

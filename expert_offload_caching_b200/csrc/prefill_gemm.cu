@@ -55,7 +55,6 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment of the base to
 // columns of A scales and 4 of B scales.
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemSf = 128;
-constexpr uint64_t kWaitNs = 4000000000ull;  // 4 s per wait
 
 static_assert(kTmemSf + kStages * kStepsPerStage * 8 <= kTmemCols, "tensor memory columns");
 static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
@@ -80,8 +79,8 @@ __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
-// Wait for the phase of the given parity to complete; false after kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of the given parity to complete; false after limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t done;
@@ -95,7 +94,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
         if (done) return true;
         if (i == 0) {
             t0 = gtimer();
-        } else if ((i & 15) == 0 && gtimer() - t0 > kWaitNs) {
+        } else if ((i & 15) == 0 && gtimer() - t0 > limit_ns) {
             return false;
         }
     }
@@ -333,7 +332,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int it = 0;
         for (; it < nkb; ++it) {
             const int s = it % kStages, r = it / kStages;
-            bool ok = r == 0 || mbar_wait(bar_empty + 8 * s, (r - 1) & 1);
+            bool ok = r == 0 || mbar_wait(bar_empty + 8 * s, (r - 1) & 1, a.wait_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 if (lane == 0) { gemm_fail(a, 41, it); *s_fail = 1; }
@@ -342,8 +341,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (lane == 0) {
                 mbar_arrive_tx(bar_full + 8 * s, 2 * kTileBytes);
                 const uint32_t da = base + kOffA + s * kTileBytes, db = base + kOffB + s * kTileBytes;
-                tma_load_3d(da, shared ? &tm_ws : &tm_w, bar_full + 8 * s, it * kStageKBytes, mt * kBM, zc);
-                tma_load_2d(db, &tm_act, bar_full + 8 * s, it * kStageKBytes, row_off + n0);
+                // test injection: block 0 never issues its first stage's copies, so
+                // that stage's wait runs out (the wind-down path below is exercised)
+                if (!(a.inj_skip && blockIdx.x == 0 && it == 0)) {
+                    tma_load_3d(da, shared ? &tm_ws : &tm_w, bar_full + 8 * s, it * kStageKBytes, mt * kBM, zc);
+                    tma_load_2d(db, &tm_act, bar_full + 8 * s, it * kStageKBytes, row_off + n0);
+                }
             }
             // scale-factor atoms: lane row holds rows lane, lane + 32, lane + 64, lane + 96
 #pragma unroll
@@ -360,7 +363,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // on failure: let the stages already issued land before the CTA exits
         if (it < nkb && lane == 0) {
             for (int j = it - 1; j >= 0 && j >= it - kStages; --j)
-                mbar_wait(bar_full + 8 * (j % kStages), (j / kStages) & 1);
+                mbar_wait(bar_full + 8 * (j % kStages), (j / kStages) & 1, a.wait_ns);
         }
     } else if (warp == 1) {
         // ---- MMA issue, one thread
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t idesc = idesc_nvf4(N) | (kMx ? (1u << 23) : 0u);  // bit 23: UE8M0 scales
             for (int it = 0; it < nkb; ++it) {
                 const int s = it % kStages, r = it / kStages;
-                if (!mbar_wait(bar_full + 8 * s, r & 1)) {
+                if (!mbar_wait(bar_full + 8 * s, r & 1, a.wait_ns)) {
                     gemm_fail(a, 42, it);
                     *s_fail = 1;
                     break;
@@ -396,7 +399,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else {
         // ---- epilogue: warp w reads lanes [32 (w % 4), +32) of the accumulator
-        bool ok = mbar_wait(bar_done, 0);
+        bool ok = mbar_wait(bar_done, 0, a.wait_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok && lane == 0) { gemm_fail(a, 43, nkb); *s_fail = 1; }
         tc_fence_after();
@@ -507,6 +510,7 @@ __global__ void __launch_bounds__(1024) tile_plan_kernel(const Job *jobs, const 
 // A = h as bf16 (hi, lo) halves, B = W2 with K wrapped: K positions j and F + j
 // both read W2's column j, so hi and lo meet W2 in one accumulation).
 constexpr int kRStages = 4;
+constexpr uint64_t kRWaitNs = 4000000000ull;  // 4 s per wait
 constexpr uint32_t kROffBar = 2 * kRStages * kTileBytes;
 constexpr uint32_t kRSmemBytes = kROffBar + 128 + 1024;
 
@@ -579,7 +583,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int it = 0;
             for (; it < nkb; ++it) {
                 const int s = it % kRStages, r = it / kRStages;
-                if (r > 0 && !mbar_wait(bar_empty + 8 * s, (r - 1) & 1)) {
+                if (r > 0 && !mbar_wait(bar_empty + 8 * s, (r - 1) & 1, kRWaitNs)) {
                     router_fail(page, 51, it);
                     *s_fail = 1;
                     break;
@@ -592,7 +596,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             if (it < nkb)  // let the stages already issued land before the CTA exits
                 for (int j = it - 1; j >= 0 && j >= it - kRStages; --j)
-                    mbar_wait(bar_full + 8 * (j % kRStages), (j / kRStages) & 1);
+                    mbar_wait(bar_full + 8 * (j % kRStages), (j / kRStages) & 1, kRWaitNs);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -600,7 +604,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t idesc = idesc_bf16(kBM);
             for (int it = 0; it < nkb; ++it) {
                 const int s = it % kRStages, r = it / kRStages;
-                if (!mbar_wait(bar_full + 8 * s, r & 1)) {
+                if (!mbar_wait(bar_full + 8 * s, r & 1, kRWaitNs)) {
                     router_fail(page, 52, it);
                     *s_fail = 1;
                     break;
@@ -616,7 +620,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else {  // epilogue: lane = row of x, columns = experts
-        bool ok = mbar_wait(bar_done, 0);
+        bool ok = mbar_wait(bar_done, 0, kRWaitNs);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok && lane == 0) { router_fail(page, 53, nkb); *s_fail = 1; }
         tc_fence_after();

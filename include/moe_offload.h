@@ -301,8 +301,9 @@ MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
 MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
 
 /* Longest wait, in seconds (default 60): the host's wait for the device miss
- * list, and (capped at 5 s, counted from the kernel's start) every wait of the
- * decode layer kernel for a miss's copy or for another CTA's tiles; a device
+ * list; (capped at 5 s, counted from the kernel's start) every wait of the
+ * decode layer kernel for a miss's copy or for another CTA's tiles; and
+ * (capped at 4 s) each mbarrier wait of the prefill expert GEMMs.  A device
  * wait that runs out records a failed check (MOE_ERR_CUDA at the next call). */
 MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
 
@@ -311,10 +312,14 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * is issued; what = 2: the next n lookups do not publish their miss list, so
  * the host wait runs out (MOE_ERR_TIMEOUT); what = 4: the next n misses are
  * copied without their completion flags, so the decode layer kernel's bounded
- * wait runs out (a failed device check, reported by the next call); what = 3:
+ * wait runs out (a failed device check, reported by the next call); what = 5:
+ * in the next n prefill calls, one CTA of the gate/up expert GEMM does not
+ * issue its first stage's tensor copies, so its bounded mbarrier waits run out
+ * (the CTA records the check, frees its tensor memory and returns; the next
+ * call reports MOE_ERR_CUDA); what = 3:
  * decode runs the layer kernel (n = 1; the default where stream memory writes
  * work, MOE_ERR_UNSUPPORTED elsewhere) or a gate/up and a down launch per miss,
- * gated by copy events (n = 0); what = 0 clears 1, 2 and 4. */
+ * gated by copy events (n = 0); what = 0 clears 1, 2, 4 and 5. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Hybrid split: m missing experts, PCIe bandwidth B_P, host expert-processing

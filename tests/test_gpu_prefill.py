@@ -213,3 +213,34 @@ def test_prefill_mxfp4_full_chunk_gpt_oss_shaped_two_layers():
     rows = np.sort(np.random.default_rng(4).choice(4096, 16, replace=False))
     _check(pb, st, events, idx, gates, y, True, rows=rows)
     st.close()
+
+
+def test_gemm_wait_limit_runs_out_then_reset_recovers():
+    """One CTA of a prefill gate/up GEMM never issues its first stage's tensor
+    copies (host-set injection) and the mbarrier wait limit is 50 ms: that
+    CTA's waits run out, it records the failed check in the mapped page, frees
+    its tensor memory and returns.  The next call reports MOE_ERR_CUDA with the
+    check; after a reset the whole chunk runs clean against the oracle (tensor
+    memory of that SM was given back, or later CTAs could not allocate it)."""
+    import time
+    pb = PrefillProblem(PF, T=200)
+    st = pb.stack(True)
+    abi.moe_set_wait_limit(st.ctx, 0.05)
+    abi.moe_debug_inject(st.ctx, 5, 1)
+    xd = torch.from_numpy(pb.x).cuda()
+    y = torch.zeros((PF.L, pb.T, PF.d), device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    st.forward(0, xd[0], y[0])
+    st.synchronize()
+    assert time.perf_counter() - t0 < 10.0
+    with pytest.raises(abi.MoeError) as ei:
+        st.forward(1, xd[1], y[1])
+    assert ei.value.status == abi.MOE_ERR_CUDA
+    msg = abi.moe_last_error(st.ctx)
+    assert any(f"device check {c}" in msg for c in (41, 42, 43)), msg
+    st.reset()
+    abi.moe_set_wait_limit(st.ctx, 60.0)
+    events, idx, gates, y2 = pb.run(st)
+    _check(pb, st, events, idx, gates, y2, True)
+    st.close()
