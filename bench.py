@@ -72,6 +72,9 @@ def parse():
                     help="routed expert records (decode): NVFP4 (default) or MXFP4")
     ap.add_argument("--shared-format", default="same", choices=["same", "bf16"],
                     help="shared expert records: the routed format (default) or BF16")
+    ap.add_argument("--ep", action="store_true",
+                    help="decode with N > 1: expert parallelism (rank r serves experts e %% N == r, its "
+                         "own cache; the partial outputs all-reduced per layer) instead of replicas")
     a = ap.parse_args()
     d_steps, d_warm, d_cfg = MODE_DEFAULTS[a.mode]
     a.steps = d_steps if a.steps is None else a.steps
@@ -108,6 +111,23 @@ def replica_pool_records(L: int, E: int, world: int) -> int:
     """Host-pool records per replica: the whole pool alone, else an aliased share
     (expert (l, e) -> record (l*E + e) mod P) so that the host RAM holds about one pool."""
     return L * E if world == 1 else max(DISTINCT_RECORDS, (L * E) // world)
+
+
+def ep_owned(e, rank: int, world: int) -> bool:
+    """Expert parallelism: rank r serves the routed experts e with e % world == r."""
+    return e % world == rank
+
+
+def ep_reduce(y, world: int, stream=None) -> None:
+    """Sum the ranks' partial layer outputs in place (expert parallelism): an
+    all-reduce, ordered on the library's compute stream on GPUs."""
+    if world == 1:
+        return
+    if stream is not None:
+        with torch.cuda.stream(stream):
+            torch.distributed.all_reduce(y)
+    else:
+        torch.distributed.all_reduce(y)
 
 
 def barrier(world):
@@ -202,9 +222,11 @@ def make_inputs(shape, T, stream0):
     return sp.decode_inputs(shape, T, 1, stream0=stream0)
 
 
-def run_tokens(stack, x, y, L, host=False, mark=None):
+def run_tokens(stack, x, y, L, host=False, mark=None, ep_world=1):
     """Tokens t = 0.. through all L layers; mark = (t0, event): the event is
-    recorded on the compute stream before token t0."""
+    recorded on the compute stream before token t0.  ep_world > 1: expert
+    parallelism, each layer's partial output summed over the ranks before the
+    next layer runs."""
     for t in range(x.shape[0]):
         if mark is not None and t == mark[0]:
             mark[1].record(stack.compute)
@@ -213,12 +235,14 @@ def run_tokens(stack, x, y, L, host=False, mark=None):
                 stack.forward_host(l, x[t, l], y[t, l])
             else:
                 stack.forward(l, x[t, l], y[t, l])
+            if ep_world > 1:
+                ep_reduce(y[t, l], ep_world, None if host else stack.compute)
 
 
 LAST_STEADY = {}  # steady-window time of the last timed() call: {"t0": first token, "s": seconds}
 
 
-def timed(stack, x, y, L, world, host=False):
+def timed(stack, x, y, L, world, host=False, ep_world=1):
     """Device seconds of all tokens; also records the steady window (tokens from
     T/4 on, after the cold cache has filled) in LAST_STEADY."""
     barrier(world)
@@ -229,7 +253,7 @@ def timed(stack, x, y, L, world, host=False):
     t0 = x.shape[0] // 4
     e0.record(stack.compute)
     torch.cuda.nvtx.range_push("timed")  # lets a profiler select the timed region's launches
-    run_tokens(stack, x, y, L, host, mark=(t0, eq) if t0 > 0 else None)
+    run_tokens(stack, x, y, L, host, mark=(t0, eq) if t0 > 0 else None, ep_world=ep_world)
     torch.cuda.nvtx.range_pop()
     e1.record(stack.compute)
     torch.cuda.synchronize()
@@ -415,9 +439,11 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
     shared = sp.shared_records_fmt(shape, sfmt)
     dims = abi.make_dims(L, E, shape.k, shape.d, shape.F, shape.shared, True, max_rows,
                          0 if P == L * E else P, weight_format=fmt, shared_format=sfmt)
+    rank = int(os.environ.get("RANK", 0))
+    shard = (rank, world) if getattr(args, "ep", False) and world > 1 else (0, 1)
     stack = LayerStack(dims, pool.tensor, sp.to_device(Wr), sp.to_device(shared),
                        shape.cache_slots, prefetch=prefetch,
-                       static_split=getattr(args, "policy", "lru") == "static")
+                       static_split=getattr(args, "policy", "lru") == "static", shard=shard)
 
     # H2D bandwidth of this machine, measured now (the roofline's PCIe term)
     nb = 1 << 30
@@ -458,26 +484,28 @@ def bench_decode(args, shape, rank, world, local):
     from expert_offload_caching_b200 import abi
     L, E, k, d, F = shape.L, shape.E, shape.k, shape.d, shape.F
     stack, pool, P, rb, Wr, shared, h2d, h2d_rec = open_stack(args, shape, world, 1)
-
-    x_warm = torch.from_numpy(make_inputs(shape, max(args.warmup, 1), 1000 + rank)).cuda()
-    x = torch.from_numpy(make_inputs(shape, args.steps, rank)).cuda()
+    # expert parallelism: every rank runs the same tokens (one model over N GPUs)
+    ep = args.ep and world > 1
+    epw = world if ep else 1
+    x_warm = torch.from_numpy(make_inputs(shape, max(args.warmup, 1), 1000 + (0 if ep else rank))).cuda()
+    x = torch.from_numpy(make_inputs(shape, args.steps, 0 if ep else rank)).cuda()
     y = torch.empty((args.steps, L, 1, d), dtype=torch.float32, device="cuda")
     yw = torch.empty((x_warm.shape[0], L, 1, d), dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
 
     # warm-up on other inputs, then a cold cache
     if args.warm:
-        run_tokens(stack, x, y, L)
+        run_tokens(stack, x, y, L, ep_world=epw)
         stack.synchronize()
         abi.moe_get_stats(stack.ctx)
         base = abi.moe_get_stats(stack.ctx)
     else:
-        run_tokens(stack, x_warm[:args.warmup], yw, L)
+        run_tokens(stack, x_warm[:args.warmup], yw, L, ep_world=epw)
         stack.synchronize()
         stack.reset()
     clocks = ClockSampler(local if world > 1 else 0)
     clocks.start()
-    el = timed(stack, x, y, L, world)
+    el = timed(stack, x, y, L, world, ep_world=epw)
     steady = dict(LAST_STEADY)
     clk = clocks.stop()
     st = abi.moe_get_stats(stack.ctx)
@@ -494,21 +522,23 @@ def bench_decode(args, shape, rank, world, local):
             stack.reset()
         before = abi.moe_get_stats(stack.ctx)
         abi.moe_set_timing(stack.ctx, True)
-        timed(stack, x, y, L, world)
+        timed(stack, x, y, L, world, ep_world=epw)
         kst = stats_delta(abi.moe_get_stats(stack.ctx), before)
         abi.moe_set_timing(stack.ctx, False)
     el_max = max_over_ranks(el, world)
-    tokens_total = sum_over_ranks(float(args.steps), world)
+    # replicas: every rank's own tokens; expert parallelism: the same tokens on all ranks
+    tokens_total = float(args.steps) if ep else sum_over_ranks(float(args.steps), world)
     value = tokens_total / el_max
     steady_line = None
     if steady:  # tokens T/4 .. T-1, after the cold cache has filled (every rank takes part)
         s_max = max_over_ranks(steady["s"], world)
+        steady_tok = float(args.steps - steady["t0"])
         steady_line = {"from_token": steady["t0"], "unit": "tok/s",
-                       "value": sum_over_ranks(float(args.steps - steady["t0"]), world) / s_max}
+                       "value": (steady_tok if ep else sum_over_ranks(steady_tok, world)) / s_max}
 
     # end to end: host buffers through moe_layer_forward_host
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not ep:  # (with expert parallelism the partials are reduced on the device)
         stack.reset()
         xh = x.cpu().pin_memory()
         yh = torch.empty((args.steps, L, 1, d), dtype=torch.float32).pin_memory()
@@ -557,7 +587,7 @@ def bench_decode(args, shape, rank, world, local):
         line = {
             "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el_max / args.steps * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if ep else "weak", "vs_baseline": None,
             "dtype": f"{fname[fmt].lower()} x bf16 -> f32 (w4a16)", "data": "synthetic",
             "warm_cache": bool(args.warm),
             "config": {"workload": f"{shape.name} decode: {L} layers x {E} experts, top-{k}"
@@ -568,7 +598,9 @@ def bench_decode(args, shape, rank, world, local):
                                    f"({P * rb / 1e9:.1f} GB; {args.pool_note})",
                        "l2": "inputs larger than L2 (each step reads "
                              f"{k * L * rb / 1e9:.2f} GB of expert records)",
-                       "cold_cache": not args.warm, "parallelism": f"replicas x{world}",
+                       "cold_cache": not args.warm,
+                       "parallelism": (f"expert parallel x{world} (experts e % {world} per rank, "
+                                       f"partial outputs all-reduced per layer)") if ep else f"replicas x{world}",
                        "pool_distinct_records": DISTINCT_RECORDS, "policy": args.policy},
             "miss_rate": counts["misses"] / max(counts["lookups"], 1),
             "counts": {"source": source, **counts,

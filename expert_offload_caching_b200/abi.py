@@ -64,7 +64,8 @@ class moe_split(ctypes.Structure):
 EXPORTS = ["moe_record_bytes", "moe_shared_record_bytes", "moe_record_layout", "moe_workspace_bytes", "moe_arena_bytes",
            "moe_layer_init", "cache_configure", "moe_layer_forward", "moe_layer_forward_host",
            "moe_get_routing", "moe_cache_export", "moe_get_stats", "moe_set_timing",
-           "moe_set_wait_limit", "moe_debug_inject", "plan_split", "moe_measure_h2d", "moe_measure_h2d_sm",
+           "moe_set_wait_limit", "moe_set_expert_shard", "moe_debug_inject", "plan_split", "moe_measure_h2d",
+           "moe_measure_h2d_sm",
            "moe_route_noalloc", "moe_status_str", "moe_last_error", "moe_layer_destroy"]
 
 _lib = None
@@ -112,6 +113,8 @@ def lib():
         L.moe_set_timing.argtypes = [vp, i32]
         L.moe_set_wait_limit.restype = ctypes.c_int
         L.moe_set_wait_limit.argtypes = [vp, dbl]
+        L.moe_set_expert_shard.restype = ctypes.c_int
+        L.moe_set_expert_shard.argtypes = [vp, i32, i32]
         L.moe_debug_inject.restype = ctypes.c_int
         L.moe_debug_inject.argtypes = [vp, i32, i64]
         L.plan_split.restype = ctypes.c_int
@@ -244,6 +247,10 @@ def moe_set_timing(ctx: int, enable: bool) -> None:
 
 def moe_set_wait_limit(ctx: int, seconds: float) -> None:
     _check(lib().moe_set_wait_limit(ctx, seconds), "moe_set_wait_limit", ctx)
+
+
+def moe_set_expert_shard(ctx: int, rank: int, size: int) -> None:
+    _check(lib().moe_set_expert_shard(ctx, rank, size), "moe_set_expert_shard", ctx)
 
 
 def moe_debug_inject(ctx: int, what: int, n: int) -> None:

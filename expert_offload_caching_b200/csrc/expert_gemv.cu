@@ -270,7 +270,8 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_gemv_kernel(GemvArgs a)
                         const float *pr = a.part_out + (size_t)t * (a.k + 1) * a.d + o;
                         float sum = 0.f;
                         for (int p = 0; p < a.k; ++p)
-                            sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                            if (a.ep_size == 1 || a.idx[t * a.k + p] % a.ep_size == a.ep_rank)
+                                sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
                         if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
                         a.y[(size_t)t * a.d + o] = sum;
                     }

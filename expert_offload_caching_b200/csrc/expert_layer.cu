@@ -139,6 +139,15 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_layer_kernel(LayerArgs 
     __syncthreads();
     const int H = s_nhit, M = s_nmiss;
     const int nA = a.F >> 3, nB = a.d >> 4, per = nA + nB;
+    if (H + M == 0 && blockIdx.x == 0) {
+        // a shard of an expert-parallel layer that owns none of the selected
+        // experts (and no resident shared expert): its partial output is the
+        // shared expert's (computed by earlier launches) or zero
+        for (int e = threadIdx.x; e < a.T * a.d; e += blockDim.x) {
+            const int t = e / a.d, o = e - t * a.d;
+            a.y[e] = a.shared_rec ? __ldcg(a.part + ((size_t)t * (a.k + 1) + a.k) * a.d + o) : 0.f;
+        }
+    }
     const int total = (H + M) * per, hit_items = H * per;
     auto decode = [&](int i) -> Item {
         Item it;
@@ -364,7 +373,9 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_layer_kernel(LayerArgs 
                     const int t = e >> 4, o = 16 * it.tile + (e & 15);
                     const float *pr = a.part + (size_t)t * (a.k + 1) * a.d + o;
                     float sum = 0.f;
-                    for (int p = 0; p < a.k; ++p) sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                    for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
+                        if (a.ep_size == 1 || a.idx[t * a.k + p] % a.ep_size == a.ep_rank)
+                            sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
                     if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
                     a.y[(size_t)t * a.d + o] = sum;
                 }

@@ -206,6 +206,9 @@ struct moe_ctx {
     // by flags the copy stream writes), when stream memory writes work here;
     // else a launch per miss, gated by events
     bool fused = false;
+    // expert parallelism: the routed experts e with e % ep_size == ep_rank; the
+    // shared expert on rank 0; y is this rank's partial sum
+    int32_t ep_rank = 0, ep_size = 1;
     double wait_limit = 60.0;
     std::chrono::steady_clock::time_point issue_t0;  // end of the last miss-list wait
     // prefill with a BF16 shared expert: its gate/up outputs and bf16 (hi, lo) h
@@ -333,6 +336,8 @@ moe_status resolve_timing(moe_ctx *ctx) {
 bool shared_separate(const moe_ctx *ctx) {
     return ctx->dims.has_shared && ctx->slay.fmt != ctx->lay.fmt;
 }
+// This context computes the shared expert (with expert parallelism: rank 0 only).
+bool shared_here(const moe_ctx *ctx) { return ctx->dims.has_shared && ctx->ep_rank == 0; }
 
 GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int combine = 0) {
     const moe_dims &D = ctx->dims;
@@ -345,10 +350,10 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
     // the shared expert is an item of the routed launches when it has their
     // format; a BF16 shared expert runs in its own launches (its partial is
     // still summed by the combine: shared_rec non-null)
-    g.shared_slot = (only_job < 0 && D.has_shared && !shared_separate(ctx)) ? max_jobs(&D, T) : -1;
+    g.shared_slot = (only_job < 0 && shared_here(ctx) && !shared_separate(ctx)) ? max_jobs(&D, T) : -1;
     g.arena = ctx->arena;
     g.rec_bytes = ctx->lay.bytes;
-    g.shared_rec = D.has_shared ? ctx->shared_recs + (int64_t)layer * ctx->slay.bytes : nullptr;
+    g.shared_rec = shared_here(ctx) ? ctx->shared_recs + (int64_t)layer * ctx->slay.bytes : nullptr;
     g.T = T;
     g.k = D.k;
     g.d = D.d;
@@ -363,6 +368,9 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
     g.gates = ctx->dws.gates;
     g.y = nullptr;
     g.tile_ticket = ctx->dws.ticket2;
+    g.idx = ctx->dws.idx;
+    g.ep_rank = ctx->ep_rank;
+    g.ep_size = ctx->ep_size;
     return g;
 }
 
@@ -473,6 +481,8 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     ra.page = ctx->page_d;
     ra.seq = seq;
     ra.publish = 1;
+    ra.ep_rank = ctx->ep_rank;
+    ra.ep_size = ctx->ep_size;
     if (ctx->inj_drop_publish > 0) {
         ra.publish = 0;
         --ctx->inj_drop_publish;
@@ -488,7 +498,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     time_end(ctx, tl, (double)D.E * D.d * 2 + (double)T * D.d * 2);
 
     const int nj = max_jobs(&D, T);
-    if (shared_separate(ctx)) {  // BF16 shared expert: its own two launches
+    if (shared_separate(ctx) && shared_here(ctx)) {  // BF16 shared expert: its own two launches
         TimedLaunch sg, sd;
         const uint8_t *rec = ctx->shared_recs + (int64_t)layer * ctx->slay.bytes;
         const int64_t sel0 = D.k, sel_stride = D.k + 1;  // selection p = k of row t
@@ -501,7 +511,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
                               ctx->cs));
         time_end(ctx, sd, 2.0 * D.d * D.F + (double)T * D.F * 4);
     }
-    const int in_launch_shared = (D.has_shared && !shared_separate(ctx)) ? 1 : 0;
+    const int in_launch_shared = (shared_here(ctx) && !shared_separate(ctx)) ? 1 : 0;
     if (ctx->fused) {
         // one launch for every expert GEMV of the layer: the hit and shared
         // experts at once, each miss when the copy stream flags its halves
@@ -511,7 +521,7 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         la.rowrefs = ctx->dws.rowrefs;
         la.arena = ctx->arena;
         la.rec_bytes = ctx->lay.bytes;
-        la.shared_rec = D.has_shared ? ctx->shared_recs + (int64_t)layer * ctx->slay.bytes : nullptr;
+        la.shared_rec = shared_here(ctx) ? ctx->shared_recs + (int64_t)layer * ctx->slay.bytes : nullptr;
         la.shared_item = in_launch_shared;
         la.T = T;
         la.k = D.k;
@@ -531,6 +541,9 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         la.seq = seq;
         la.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 5.0) * 1e9);
         la.page = ctx->page_d;
+        la.idx = ctx->dws.idx;
+        la.ep_rank = ctx->ep_rank;
+        la.ep_size = ctx->ep_size;
         TimedLaunch tk, th;
         time_begin(ctx, tk, MOE_K_LAYER);
         la.span = time_span(ctx, tk);
@@ -686,6 +699,8 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     ra.page = ctx->page_d;
     ra.seq = seq;
     ra.publish = 1;
+    ra.ep_rank = 0;  // (expert parallelism is a decode-path feature)
+    ra.ep_size = 1;
     if (ctx->inj_drop_publish > 0) {
         ra.publish = 0;
         --ctx->inj_drop_publish;
@@ -1036,6 +1051,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
     if (!ctx || !slot_arena || num_slots <= 0) return MOE_ERR_ARG;
     const bool stat = (flags & MOE_CACHE_STATIC_SPLIT) != 0;
     if (stat && (flags & MOE_CACHE_PREFETCH_NEXT)) return MOE_ERR_ARG;
+    if (stat && ctx->ep_size > 1) return MOE_ERR_UNSUPPORTED;
     const moe_dims &D = ctx->dims;
     const int64_t need = max_jobs(&D, D.max_rows);
     if (num_slots < need) return MOE_ERR_CAPACITY;
@@ -1225,6 +1241,16 @@ moe_status moe_set_timing(moe_ctx *ctx, int32_t enable) {
     return MOE_OK;
 }
 
+moe_status moe_set_expert_shard(moe_ctx *ctx, int32_t rank, int32_t size) {
+    if (!ctx || size < 1 || rank < 0 || rank >= size || size > ctx->dims.E) return MOE_ERR_ARG;
+    if (size > 1 && (ctx->dims.max_rows > kDecodeMaxRows || !ctx->fused || (ctx->flags & MOE_CACHE_STATIC_SPLIT)))
+        return MOE_ERR_UNSUPPORTED;
+    if (rank != ctx->ep_rank || size != ctx->ep_size) ctx->configured = false;  // a new cache: reset first
+    ctx->ep_rank = rank;
+    ctx->ep_size = size;
+    return MOE_OK;
+}
+
 moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds) {
     if (!ctx || !(seconds > 0)) return MOE_ERR_ARG;
     ctx->wait_limit = seconds;
@@ -1242,6 +1268,7 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
     else if (what == 1) ctx->inj_copy_fail_at = n;
     else if (what == 2) ctx->inj_drop_publish = n;
     else if (what == 3) {  // decode path: 0 = a launch per miss, 1 = the layer kernel
+        if (n == 0 && ctx->ep_size > 1) return MOE_ERR_UNSUPPORTED;
         if (n == 1 && stream_write(ctx->xs, ctx->dws.lk_release, 0u) != cudaSuccess) return MOE_ERR_UNSUPPORTED;
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;

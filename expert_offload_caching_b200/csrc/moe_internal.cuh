@@ -120,6 +120,8 @@ struct RouteArgs {
     uint32_t seq;
     int publish;
     unsigned long long *span;  // launch timing slot (see span_mark), or null
+    // expert parallelism: this context serves the experts e with e % ep_size == ep_rank
+    int ep_rank, ep_size;
 };
 
 enum GemvMode { kGateUp = 0, kDown = 1 };
@@ -150,6 +152,8 @@ struct GemvArgs {
     float *y;
     uint32_t *tile_ticket;  // [tiles] per-tile counters of the combining launch, kept at 0
     unsigned long long *span;  // launch timing slot (see span_mark), or null
+    const int32_t *idx;     // [T][k] selected experts: the combine takes the owned ones only
+    int ep_rank, ep_size;
 };
 
 // Persistent decode layer kernel (all expert GEMVs of one layer, misses as
@@ -185,6 +189,8 @@ struct LayerArgs {
     HostPage *page;
     unsigned long long *span;      // launch timing slot, or null
     unsigned long long *span_hit;  // [start, end of the last hit/shared item], or null
+    const int32_t *idx;            // [T][k] selected experts: the combine takes the owned ones only
+    int ep_rank, ep_size;
 };
 
 // Grouped W4A4 expert GEMMs of a prefill chunk (tcgen05 block-scaled MMA).

@@ -458,25 +458,30 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     if (threadIdx.x == 0) t_topk = global_ns();
     const int nsel = a.T * a.k;
     if (a.T == 1) {
-        // one row: its k ids are already distinct and ascending -- they are the
-        // jobs, one row each, in selection order
-        for (int j = threadIdx.x; j < a.k; j += blockDim.x) {
-            int e = a.ws.idx[j];
-            if ((unsigned)e >= (unsigned)a.E) { route_fail(a.page, 1, e, a.E); e = 0; }
-            s_exp[j] = e;
-            s_cnt[j] = 1;
-            s_off[j] = j;
-            a.ws.rowrefs[j].t = 0;
-            a.ws.rowrefs[j].p = (int16_t)j;
+        // one row: its k ids are already distinct and ascending -- they (the
+        // owned ones, with expert parallelism) are the jobs, one row each
+        if (warp == 0) {
+            int e = lane < a.k ? a.ws.idx[lane] : 0;
+            if (lane < a.k && (unsigned)e >= (unsigned)a.E) { route_fail(a.page, 1, e, a.E); e = 0; }
+            const bool own = lane < a.k && e % a.ep_size == a.ep_rank;
+            const unsigned ob = __ballot_sync(0xffffffffu, own);
+            const int pos = __popc(ob & ((1u << lane) - 1u));
+            if (own) {
+                s_exp[pos] = e;
+                s_cnt[pos] = 1;
+                s_off[pos] = pos;
+                a.ws.rowrefs[pos].t = 0;
+                a.ws.rowrefs[pos].p = (int16_t)lane;
+            }
+            if (lane == 0) s_njobs = __popc(ob);
         }
-        if (threadIdx.x == 0) s_njobs = a.k;
         __syncthreads();
     } else {
         for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
             const int e = a.ws.idx[i];
             s_idx[i] = e;
-            if ((unsigned)e < (unsigned)a.E) atomicOr(&s_bits[e >> 5], 1u << (e & 31));
-            else route_fail(a.page, 1, e, a.E);
+            if ((unsigned)e >= (unsigned)a.E) route_fail(a.page, 1, e, a.E);
+            else if (e % a.ep_size == a.ep_rank) atomicOr(&s_bits[e >> 5], 1u << (e & 31));
         }
         __syncthreads();
         if (warp == 0) {

@@ -22,7 +22,8 @@ class LayerStack:
 
     def __init__(self, dims: abi.moe_dims, host_pool: torch.Tensor, router_w: torch.Tensor,
                  shared: torch.Tensor | None, num_slots: int, *, prefetch: bool = False,
-                 static_split: bool = False, device: str | torch.device = "cuda"):
+                 static_split: bool = False, shard: tuple[int, int] = (0, 1),
+                 device: str | torch.device = "cuda"):
         if not torch.cuda.is_available():
             raise RuntimeError("LayerStack needs a CUDA device")
         self.dims = dims
@@ -40,6 +41,8 @@ class LayerStack:
                                       self.ws, self.ws.numel(), self.compute, self.copy)
         self.flags = ((abi.MOE_CACHE_PREFETCH_NEXT if prefetch else 0) |
                       (abi.MOE_CACHE_STATIC_SPLIT if static_split else 0))
+        if shard != (0, 1):  # expert parallelism: this stack serves experts e % size == rank
+            abi.moe_set_expert_shard(self.ctx, shard[0], shard[1])
         self.reset()
 
     def reset(self) -> None:

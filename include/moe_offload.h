@@ -300,6 +300,23 @@ MOE_API moe_status moe_get_stats(moe_ctx *ctx, moe_stats *out);
  * 4 MB device buffer of span slots, freed by moe_layer_destroy. */
 MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
 
+/* Expert parallelism over several GPUs (one context per GPU; the pages'
+ * engine offloads to host RAM from one GPU -- ai-hardware-zukan
+ * "GPUに載らない分をどう間に合わせるか" -- and this spreads the cache and the
+ * PCIe links over G of them): this context serves the routed experts e with
+ * e mod size == rank -- its cache holds and its lookups count only those --
+ * and the shared expert only when rank == 0; moe_layer_forward then writes
+ * to y this rank's partial sum over its experts of the selected ones (zero if
+ * it owns none), and the layer's output is the sum of the partials over the
+ * ranks, which the caller forms (e.g. an all-reduce on compute_stream).  Every
+ * rank computes the same routing from the same x (moe_get_routing returns all
+ * k).  size = 1 (the default) is the whole layer.  A change needs
+ * cache_configure(..., MOE_CACHE_RESET) before the next call (MOE_ERR_STATE
+ * until then).  MOE_ERR_ARG unless 0 <= rank < size <= E; MOE_ERR_UNSUPPORTED
+ * for size > 1 with max_rows > 32, the static split, or without the decode
+ * layer kernel (stream memory writes unavailable). */
+MOE_API moe_status moe_set_expert_shard(moe_ctx *ctx, int32_t rank, int32_t size);
+
 /* Longest wait, in seconds (default 60): the host's wait for the device miss
  * list; (capped at 5 s, counted from the kernel's start) every wait of the
  * decode layer kernel for a miss's copy or for another CTA's tiles; and

@@ -74,19 +74,24 @@ def conditioned_prefill(Wr: np.ndarray, k: int, layer: int, T: int,
                                                  int(attempt[t]), d, seed=seed))
 
 
-def decode_trace(idx: np.ndarray, L: int, E: int, C: int, lru: LRU | None = None):
+def decode_trace(idx: np.ndarray, L: int, E: int, C: int, lru: LRU | None = None,
+                 shard: tuple[int, int] = (0, 1)):
     """Replay decode lookups through the oracle LRU.
 
     idx: [T, L, rows, k] selected experts per (token step, layer, row).  One
     lookup batch per (step, layer): the distinct experts over the rows, in
-    ascending id.  Returns (events [(t, layer, expert, slot, hit, evicted)], lru).
+    ascending id -- with shard = (rank, size), only those with e % size == rank
+    (the cache of one rank of an expert-parallel layer).
+    Returns (events [(t, layer, expert, slot, hit, evicted)], lru).
     """
     lru = LRU(L, E, C) if lru is None else lru
     events = []
     T = idx.shape[0]
+    rank, size = shard
     for t in range(T):
         for l in range(L):
             batch = np.unique(idx[t, l].ravel())
+            batch = batch[batch % size == rank]
             for e, s, h, v in lru.batch(l, batch):
                 events.append((t, l, e, s, h, v))
     return events, lru
