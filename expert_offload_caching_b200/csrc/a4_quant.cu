@@ -127,10 +127,11 @@ __device__ void quant_row_codes_mx(LoadFn load, int n, uint8_t *codes, uint8_t *
 // rowrefs[g].t, row T*k + t (shared expert) is token t; one warp per row.
 __global__ void quant_x_grouped_kernel(const __nv_bfloat16 *__restrict__ x, int T, int k, int d,
                                        int has_shared, const RowRef *__restrict__ rowrefs,
-                                       uint8_t *codes, uint8_t *scales, float *st, int mx) {
+                                       const int32_t *__restrict__ n_routed, uint8_t *codes, uint8_t *scales,
+                                       float *st, int mx) {
     const int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int tk = T * k;
-    if (g >= tk + (has_shared ? T : 0)) return;
+    if (g >= tk + (has_shared ? T : 0) || (g < tk && g >= *n_routed)) return;
     const int t = g < tk ? rowrefs[g].t : g - tk;
     const __nv_bfloat16 *row = x + (size_t)t * d;
     auto load = [&](int i) { return __bfloat162float(row[i]); };
@@ -139,25 +140,30 @@ __global__ void quant_x_grouped_kernel(const __nv_bfloat16 *__restrict__ x, int 
 }
 
 // Grouped h rows (fp32 [rows][F]) -> NVFP4 codes, scales, row scales; one warp per row.
-__global__ void quant_h_grouped_kernel(const float *__restrict__ h32, int rows, int F, uint8_t *codes,
+__global__ void quant_h_grouped_kernel(const float *__restrict__ h32, int T, int k, int has_shared,
+                                       const int32_t *__restrict__ n_routed, int F, uint8_t *codes,
                                        uint8_t *scales, float *st, int mx) {
     const int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (g >= rows) return;
+    const int tk = T * k;
+    if (g >= tk + (has_shared ? T : 0) || (g < tk && g >= *n_routed)) return;
     const float *row = h32 + (size_t)g * F;
     auto load = [&](int i) { return row[i]; };
     if (mx) quant_row_codes_mx(load, F, codes + (size_t)g * (F / 2), scales + (size_t)g * (F / 32));
     else quant_row_codes(load, F, codes + (size_t)g * (F / 2), scales + (size_t)g * (F / 16), st + g);
 }
 
-// y[t] = sum over p < k of gates[t][p] * part[t][p] (+ part[t][k], the shared expert)
+// y[t] = sum over p < k of gates[t][p] * part[t][p] (+ part[t][k], the shared expert); with
+// expert parallelism only the selections this rank owns
 __global__ void combine_kernel(const float *__restrict__ part, const float *__restrict__ gates,
+                               const int32_t *__restrict__ idx, int ep_rank, int ep_size,
                                float *__restrict__ y, int T, int k, int d, int has_shared) {
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= (int64_t)T * d) return;
     const int t = (int)(i / d), c = (int)(i - (int64_t)t * d);
     const float *pr = part + (size_t)t * (k + 1) * d + c;
     float acc = 0.f;
-    for (int p = 0; p < k; ++p) acc = fmaf(gates[t * k + p], pr[(size_t)p * d], acc);
+    for (int p = 0; p < k; ++p)
+        if (ep_size == 1 || idx[t * k + p] % ep_size == ep_rank) acc = fmaf(gates[t * k + p], pr[(size_t)p * d], acc);
     if (has_shared) acc += pr[(size_t)k * d];
     y[i] = acc;
 }
@@ -183,27 +189,29 @@ cudaError_t launch_swiglu_split(const float *sg, int T, int F, uint16_t *hs, cud
 }
 
 cudaError_t launch_quant_x_grouped(const __nv_bfloat16 *x, int T, int k, int d, int has_shared,
-                                   const RowRef *rowrefs, uint8_t *codes, uint8_t *scales, float *st,
-                                   int mx, cudaStream_t s) {
+                                   const RowRef *rowrefs, const int32_t *n_routed, uint8_t *codes,
+                                   uint8_t *scales, float *st, int mx, cudaStream_t s) {
     const int rows = T * k + (has_shared ? T : 0);
     const int warps_per_cta = 8;
     quant_x_grouped_kernel<<<(rows + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(
-        x, T, k, d, has_shared, rowrefs, codes, scales, st, mx);
+        x, T, k, d, has_shared, rowrefs, n_routed, codes, scales, st, mx);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quant_h_grouped(const float *h32, int rows, int F, uint8_t *codes, uint8_t *scales,
-                                   float *st, int mx, cudaStream_t s) {
+cudaError_t launch_quant_h_grouped(const float *h32, int T, int k, int has_shared, const int32_t *n_routed,
+                                   int F, uint8_t *codes, uint8_t *scales, float *st, int mx, cudaStream_t s) {
+    const int rows = T * k + (has_shared ? T : 0);
     const int warps_per_cta = 8;
     quant_h_grouped_kernel<<<(rows + warps_per_cta - 1) / warps_per_cta, warps_per_cta * 32, 0, s>>>(
-        h32, rows, F, codes, scales, st, mx);
+        h32, T, k, has_shared, n_routed, F, codes, scales, st, mx);
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
-                           int has_shared, cudaStream_t s) {
+cudaError_t launch_combine(const float *part, const float *gates, const int32_t *idx, int ep_rank, int ep_size,
+                           float *y, int T, int k, int d, int has_shared, cudaStream_t s) {
     const int64_t n = (int64_t)T * d;
-    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, gates, y, T, k, d, has_shared);
+    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, gates, idx, ep_rank, ep_size, y, T, k, d,
+                                                               has_shared);
     return cudaGetLastError();
 }
 

@@ -88,7 +88,8 @@ int max_jobs(const moe_dims *d, int T) {
 // for the largest call (max_rows); the prefill buffers exist when max_rows > 32.
 struct WsLayout {
     int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, lk, rowrefs, xh, hh, part, cnt, fill,
-        jobidx, h32, xq, xq_scales, xq_st, hq, hq_scales, hq_st, pairs, n_pairs, sg, hs, xstage, ystage, total;
+        jobidx, h32, xq, xq_scales, xq_st, hq, hq_scales, hq_st, pairs, n_pairs, n_grouped, sg, hs, xstage, ystage,
+        total;
 };
 int pairs_capacity(const moe_dims *d) {
     return grouped_pairs_cap(d->E, d->max_rows, d->k, d->has_shared ? 1 : 0);
@@ -127,6 +128,7 @@ WsLayout ws_layout(const moe_dims *d) {
     w.hq_st = prefill ? take(R * 4) : -1;
     w.pairs = prefill ? take((int64_t)pairs_capacity(d) * 8) : -1;
     w.n_pairs = prefill ? take(4) : -1;
+    w.n_grouped = prefill ? take(4) : -1;
     // a BF16 shared expert on the prefill path: its gate/up outputs [T][2F] fp32
     // and h as bf16 (hi, lo) halves [T][2F]
     const bool sbf = prefill && d->has_shared && d->shared_format == MOE_FMT_BF16;
@@ -699,16 +701,16 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     ra.page = ctx->page_d;
     ra.seq = seq;
     ra.publish = 1;
-    ra.ep_rank = 0;  // (expert parallelism is a decode-path feature)
-    ra.ep_size = 1;
+    ra.ep_rank = ctx->ep_rank;
+    ra.ep_size = ctx->ep_size;
     if (ctx->inj_drop_publish > 0) {
         ra.publish = 0;
         --ctx->inj_drop_publish;
     }
     // the shared expert is a job of the grouped GEMMs when it has the routed
     // format; a BF16 one runs as two bf16 GEMMs of its own
-    const bool sep = shared_separate(ctx);
-    const int grouped_shared = (D.has_shared && !sep) ? 1 : 0;
+    const bool sep = shared_separate(ctx) && shared_here(ctx);
+    const int grouped_shared = (shared_here(ctx) && !shared_separate(ctx)) ? 1 : 0;
     const bool mx = ctx->lay.fmt == kFmtMxfp4;
     CK(cudaMemsetAsync(ctx->dws.cnt, 0, (size_t)D.E * 4, ctx->cs));
     TimedLaunch tr;
@@ -726,7 +728,7 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     CK(launch_prefill_scatter(ra, ctx->cs));
     CK(launch_tile_plan(ctx->dws.jobs, ctx->dws.n_jobs, T, grouped_shared, ctx->dws.pairs, ctx->dws.n_pairs,
                         ctx->cs));
-    CK(launch_quant_x_grouped(ra.x, T, D.k, D.d, grouped_shared, ctx->dws.rowrefs, ctx->dws.xq,
+    CK(launch_quant_x_grouped(ra.x, T, D.k, D.d, grouped_shared, ctx->dws.rowrefs, ctx->dws.n_grouped, ctx->dws.xq,
                               ctx->dws.xq_scales, ctx->dws.xq_st, mx ? 1 : 0, ctx->cs));
 
     const moe_status ws_ = wait_miss_list(ctx, seq);
@@ -835,9 +837,8 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
     gu.span = time_span(ctx, tg);
     CK(launch_grouped_gemm(ctx->maps, gu, cap, ctx->cs));
     time_end(ctx, tg, grid_y * w13_bytes(ctx));
-    const int grouped_rows = T * D.k + (grouped_shared ? T : 0);
-    CK(launch_quant_h_grouped(ctx->dws.h32, grouped_rows, D.F, ctx->dws.hq, ctx->dws.hq_scales,
-                              ctx->dws.hq_st, mx ? 1 : 0, ctx->cs));
+    CK(launch_quant_h_grouped(ctx->dws.h32, T, D.k, grouped_shared, ctx->dws.n_grouped, D.F, ctx->dws.hq,
+                              ctx->dws.hq_scales, ctx->dws.hq_st, mx ? 1 : 0, ctx->cs));
     GroupedGemmArgs dn = gu;
     dn.inj_skip = 0;
     dn.mode = kDown;
@@ -861,7 +862,8 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
                             (int64_t)(D.k + 1) * D.d, T, D.d, 4 * D.F, 2 * D.F, layer, ctx->page_d, ctx->cs));
         time_end(ctx, sd_t, 2.0 * D.d * D.F + (double)T * D.F * 4);
     }
-    CK(launch_combine(ctx->dws.part, ctx->dws.gates, y, T, D.k, D.d, D.has_shared, ctx->cs));
+    CK(launch_combine(ctx->dws.part, ctx->dws.gates, ctx->dws.idx, ctx->ep_rank, ctx->ep_size, y, T, D.k, D.d,
+                      shared_here(ctx) ? 1 : 0, ctx->cs));
 
     int64_t hits = 0, evictions = 0, pf_evict = 0;
     for (int j = 0; j < n; ++j) {  // (npm: prefetch misses counted above)
@@ -979,6 +981,7 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
         ctx->dws.hq_st = reinterpret_cast<float *>(w + L.hq_st);
         ctx->dws.pairs = reinterpret_cast<int2 *>(w + L.pairs);
         ctx->dws.n_pairs = reinterpret_cast<int32_t *>(w + L.n_pairs);
+        ctx->dws.n_grouped = reinterpret_cast<int32_t *>(w + L.n_grouped);
         const int64_t R = (int64_t)dims->max_rows * (dims->k + 1);
         bool ok = make_operand_map(&ctx->maps.xq, ctx->dws.xq, dims->d / 2, R, 0, 0) &&
                   make_operand_map(&ctx->maps.hq, ctx->dws.hq, dims->F / 2, R, 0, 0) &&
@@ -1243,8 +1246,7 @@ moe_status moe_set_timing(moe_ctx *ctx, int32_t enable) {
 
 moe_status moe_set_expert_shard(moe_ctx *ctx, int32_t rank, int32_t size) {
     if (!ctx || size < 1 || rank < 0 || rank >= size || size > ctx->dims.E) return MOE_ERR_ARG;
-    if (size > 1 && (ctx->dims.max_rows > kDecodeMaxRows || !ctx->fused || (ctx->flags & MOE_CACHE_STATIC_SPLIT)))
-        return MOE_ERR_UNSUPPORTED;
+    if (size > 1 && (!ctx->fused || (ctx->flags & MOE_CACHE_STATIC_SPLIT))) return MOE_ERR_UNSUPPORTED;
     if (rank != ctx->ep_rank || size != ctx->ep_size) ctx->configured = false;  // a new cache: reset first
     ctx->ep_rank = rank;
     ctx->ep_size = size;

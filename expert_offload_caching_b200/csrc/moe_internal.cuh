@@ -105,6 +105,7 @@ struct DecodeWs {
     float *hq_st;        // grouped rows
     int2 *pairs;         // (job, n tile) pairs of the grouped GEMMs
     int32_t *n_pairs;
+    int32_t *n_grouped;  // routed grouped rows of the chunk (all T*k, or the owned ones with expert parallelism)
 };
 
 struct RouteArgs {
@@ -254,14 +255,16 @@ cudaError_t launch_table_static(Table t, int L, int E, int per_layer, cudaStream
 cudaError_t launch_prefill_route(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_scatter(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_select(const RouteArgs &a, cudaStream_t s);
-cudaError_t launch_combine(const float *part, const float *gates, float *y, int T, int k, int d,
-                           int has_shared, cudaStream_t s);
-// mx = 0: NVFP4 (E4M3 per 16 + fp32 row scale st); mx = 1: MXFP4 (E8M0 per 32, st unused)
+// y[t] = sum of the owned selections' gated partials (all with ep_size 1) + the shared one
+cudaError_t launch_combine(const float *part, const float *gates, const int32_t *idx, int ep_rank, int ep_size,
+                           float *y, int T, int k, int d, int has_shared, cudaStream_t s);
+// mx = 0: NVFP4 (E4M3 per 16 + fp32 row scale st); mx = 1: MXFP4 (E8M0 per 32, st unused).
+// Grouped rows: the routed ones [0, *n_routed) of [0, T*k), then (has_shared) T*k + t.
 cudaError_t launch_quant_x_grouped(const __nv_bfloat16 *x, int T, int k, int d, int has_shared,
-                                   const RowRef *rowrefs, uint8_t *codes, uint8_t *scales, float *st,
-                                   int mx, cudaStream_t s);
-cudaError_t launch_quant_h_grouped(const float *h32, int rows, int F, uint8_t *codes, uint8_t *scales,
-                                   float *st, int mx, cudaStream_t s);
+                                   const RowRef *rowrefs, const int32_t *n_routed, uint8_t *codes,
+                                   uint8_t *scales, float *st, int mx, cudaStream_t s);
+cudaError_t launch_quant_h_grouped(const float *h32, int T, int k, int has_shared, const int32_t *n_routed,
+                                   int F, uint8_t *codes, uint8_t *scales, float *st, int mx, cudaStream_t s);
 int grouped_pairs_cap(int n_jobs, int T, int k, int has_shared);
 cudaError_t launch_tile_plan(const Job *jobs, const int32_t *n_jobs, int T, int has_shared, int2 *pairs,
                              int32_t *n_pairs, cudaStream_t s);

@@ -654,8 +654,11 @@ __global__ void __launch_bounds__(kRouteThreads) prefill_topk_kernel(RouteArgs a
     const int t = blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5);
     if (t >= a.T) return;
     const int e = topk_row(a, t);
-    if ((unsigned)e < (unsigned)a.E) atomicAdd(&a.ws.cnt[e], 1);
-    else if ((threadIdx.x & 31) < a.k) route_fail(a.page, 2, e, a.E);
+    if ((unsigned)e < (unsigned)a.E) {
+        if (e % a.ep_size == a.ep_rank) atomicAdd(&a.ws.cnt[e], 1);  // (this rank's experts)
+    } else if ((threadIdx.x & 31) < a.k) {
+        route_fail(a.page, 2, e, a.E);
+    }
 }
 
 __global__ void __launch_bounds__(kRouteThreads) prefill_lookup_kernel(RouteArgs a) {
@@ -688,7 +691,10 @@ __global__ void __launch_bounds__(kRouteThreads) prefill_lookup_kernel(RouteArgs
             if (j < nj) s_off[j] = carry + incl - c;
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) s_n = nj;
+        if (lane == 0) {
+            s_n = nj;
+            *a.ws.n_grouped = nj > 0 ? carry : 0;  // routed grouped rows (carry: their total)
+        }
     }
     __syncthreads();
     const int n = s_n;
@@ -712,12 +718,22 @@ __global__ void __launch_bounds__(kRouteThreads) prefill_lookup_kernel(RouteArgs
     }
     __syncthreads();  // the routed batch is consumed before the prefetch batch reuses sm
     int npf = 0, pf_miss = 0;
-    if (a.prefetch && a.layer + 1 < a.L) {
-        for (int e = threadIdx.x; e < a.E; e += blockDim.x) sm.exp[e] = e;
+    if (a.prefetch && a.layer + 1 < a.L) {  // all of the next layer's experts (this rank's)
+        if (warp == 0) {
+            int c = 0;
+            for (int e0 = 0; e0 < a.E; e0 += 32) {
+                const int e = e0 + lane;
+                const bool own = e < a.E && e % a.ep_size == a.ep_rank;
+                const unsigned ob = __ballot_sync(0xffffffffu, own);
+                if (own) sm.exp[c + __popc(ob & ((1u << lane) - 1u))] = e;
+                c += __popc(ob);
+            }
+            if (lane == 0) s_n = c;
+        }
         __syncthreads();
-        lookup_batch(a.tab, a.layer + 1, a.E, a.E, sm, nullptr);
-        if (warp == 0) publish_events(a.page, n, sm, a.E, 1);
-        npf = a.E;
+        npf = s_n;
+        lookup_batch(a.tab, a.layer + 1, a.E, npf, sm, nullptr);
+        if (warp == 0) publish_events(a.page, n, sm, npf, 1);
         pf_miss = sm.nmiss;
     }
     if (warp == 0) {
@@ -741,6 +757,7 @@ __global__ void prefill_scatter_kernel(RouteArgs a) {
     if (i >= a.T * a.k) return;
     const int e = a.ws.idx[i];
     if ((unsigned)e >= (unsigned)a.E) { route_fail(a.page, 3, e, a.E); return; }
+    if (e % a.ep_size != a.ep_rank) return;  // another rank's expert
     const int j = a.ws.jobidx[e];
     if (j < 0) { route_fail(a.page, 4, e, a.E); return; }
     const int pos = a.ws.jobs[j].row_off + atomicAdd(&a.ws.fill[e], 1);

@@ -312,9 +312,11 @@ MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
  * rank computes the same routing from the same x (moe_get_routing returns all
  * k).  size = 1 (the default) is the whole layer.  A change needs
  * cache_configure(..., MOE_CACHE_RESET) before the next call (MOE_ERR_STATE
- * until then).  MOE_ERR_ARG unless 0 <= rank < size <= E; MOE_ERR_UNSUPPORTED
- * for size > 1 with max_rows > 32, the static split, or without the decode
- * layer kernel (stream memory writes unavailable). */
+ * until then).  Prefill chunks likewise: the lookup and prefetch batches, the
+ * grouped GEMMs and the combine cover this rank's experts only.  MOE_ERR_ARG
+ * unless 0 <= rank < size <= E; MOE_ERR_UNSUPPORTED for size > 1 with the
+ * static split or without the decode layer kernel (stream memory writes
+ * unavailable). */
 MOE_API moe_status moe_set_expert_shard(moe_ctx *ctx, int32_t rank, int32_t size);
 
 /* Longest wait, in seconds (default 60): the host's wait for the device miss

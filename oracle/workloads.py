@@ -98,17 +98,21 @@ def decode_trace(idx: np.ndarray, L: int, E: int, C: int, lru: LRU | None = None
 
 
 def prefill_trace(idx: np.ndarray, L: int, E: int, C: int, prefetch: bool = True,
-                  lru: LRU | None = None):
+                  lru: LRU | None = None, shard: tuple[int, int] = (0, 1)):
     """Replay a prefill chunk: idx [L, T, k].  Per layer one routed batch (the
     distinct experts of all rows, ascending), then, with prefetch, one batch of
-    all E experts of the next layer.  Events carry a kind: 0 routed, 1 prefetch."""
+    all E experts of the next layer -- with shard = (rank, size), only the
+    experts e % size == rank in both.  Events carry a kind: 0 routed, 1 prefetch."""
     lru = LRU(L, E, C) if lru is None else lru
     events = []
+    rank, size = shard
     for l in range(L):
-        for e, s, h, v in lru.batch(l, np.unique(idx[l].ravel())):
+        batch = np.unique(idx[l].ravel())
+        for e, s, h, v in lru.batch(l, batch[batch % size == rank]):
             events.append((0, l, e, s, h, v))
         if prefetch and l + 1 < L:
-            for e, s, h, v in lru.batch(l + 1, np.arange(E, dtype=np.int32)):
+            allx = np.arange(E, dtype=np.int32)
+            for e, s, h, v in lru.batch(l + 1, allx[allx % size == rank]):
                 events.append((1, l + 1, e, s, h, v))
     return events, lru
 

@@ -94,3 +94,42 @@ def test_shard_argument_checks():
     st.forward(0, x, y)
     st.synchronize()
     st.close()
+
+
+@pytest.mark.parametrize("fmt,shared_fmt", [(sp.FMT_NVFP4, None), (sp.FMT_MXFP4, sp.FMT_BF16)],
+                         ids=["nvfp4", "mxfp4+bf16-shared"])
+def test_prefill_shards_sum_to_the_layer(fmt, shared_fmt):
+    """A prefill chunk under expert parallelism (2 ranks, prefetch on): each
+    rank's routed and prefetch batches hold its own experts only (trace and
+    table equal the oracle's LRU over them), the grouped GEMMs run over its
+    rows only, and the partials sum to the oracle's W4A4 layer row by row."""
+    from oracle.workloads import prefill_trace
+    from tests.test_gpu_prefill import PF, PrefillProblem
+    import oracle
+    pb = PrefillProblem(PF, T=200, fmt=fmt, shared_fmt=shared_fmt)
+    total = None
+    want_idx = np.stack([oracle.route(pb.Wr[l], pb.x[l], PF.k)[0] for l in range(PF.L)])
+    for rank in range(2):
+        sh = PF
+        dims = abi.make_dims(sh.L, sh.E, sh.k, sh.d, sh.F, sh.shared, True, pb.T, 0, weight_format=fmt,
+                             shared_format=pb.shared_fmt)
+        st = LayerStack(dims, pb.pool, sp.to_device(pb.Wr), sp.to_device(pb.shared), pb.C, prefetch=True,
+                        shard=(rank, 2))
+        events, idx, gates, y = pb.run(st)
+        np.testing.assert_array_equal(idx, want_idx)
+        want_ev, lru = prefill_trace(want_idx, sh.L, sh.E, pb.C, prefetch=True, shard=(rank, 2))
+        assert events == want_ev
+        m = np.empty(sh.L * sh.E, np.int32)
+        o = np.empty(pb.C, np.int32)
+        s_ = np.empty(pb.C, np.uint64)
+        clock = abi.moe_cache_export(st.ctx, m, o, s_)
+        wm, wo, ws, wc = lru.state()
+        np.testing.assert_array_equal(m, wm)
+        np.testing.assert_array_equal(o, wo)
+        assert clock == wc
+        total = y if total is None else total + y
+        st.close()
+    for l in range(PF.L):
+        want = pb.oracle_y(l, np.arange(pb.T))
+        for r in range(pb.T):
+            assert rel_l2(total[l][r], want[r]) <= REL_L2_MAX, (l, r)

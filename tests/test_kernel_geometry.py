@@ -227,3 +227,60 @@ def test_mxfp4_step_factoring_keeps_products_exact():
              rec[off[3]:off[3] + d * F // 32].reshape(d, F // 32), F, h)
     want = oracle.expert_mx_w4a16(rec, d, F, x)
     assert np.linalg.norm(y - want) / np.linalg.norm(want) < 1e-6
+
+
+# ------------------------------------------------------- decode layer kernel --
+def _layer_decode(i, H, M, nA, nB):
+    """Mirror of the layer kernel's queue decode: (expert slot, gate_up, tile, miss)."""
+    per = nA + nB
+    if i < H * nA:
+        return (i // nA, 1, i % nA, -1)
+    if i < H * per:
+        j = i - H * nA
+        return (j // nB, 0, j % nB, -1)
+    j = i - H * per
+    m, r = divmod(j, per)
+    return (H + m, 1 if r < nA else 0, r if r < nA else r - nA, m)
+
+
+@pytest.mark.parametrize("H,M", [(1, 0), (0, 3), (7, 0), (4, 2), (11, 10), (1, 32)])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: s.name)
+def test_layer_queue_covers_every_tile_once_in_dependency_order(shape, H, M):
+    """Every (expert, phase, tile) once; each down tile after all gate/up tiles of
+    its expert (so a waiting CTA only waits on tiles held by running CTAs); the
+    misses in the order the host copies them, each miss's gate/up before its down."""
+    nA, nB = shape.F // 8, shape.d // 16
+    total = (H + M) * (nA + nB)
+    seen = {}
+    for i in range(total):
+        key = _layer_decode(i, H, M, nA, nB)
+        assert key[:3] not in seen
+        seen[key[:3]] = i
+    assert len(seen) == total
+    for (x, gu, t), i in seen.items():
+        if not gu:
+            assert all(seen[(x, 1, a)] < i for a in range(nA))
+    firsts = [min(i for (x, gu, t), i in seen.items() if x == H + m) for m in range(M)]
+    assert firsts == sorted(firsts)
+    assert all(_layer_decode(i, H, M, nA, nB)[3] == -1 for i in range(H * (nA + nB)))
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: s.name)
+@pytest.mark.parametrize("mx", [False, True])
+def test_layer_kernel_ring_fits_and_keeps_two_ctas_per_sm_where_it_can(shape, mx):
+    """The launcher's choice: a 3-tile ring when two CTAs still fit an SM (227 KB of
+    shared memory, ~5 KB static per CTA), else 2; the ring covers the longer K."""
+    Kmax = max(shape.d, shape.F)
+    nsteps = (Kmax // 64 + 3) // 4
+    spw = 2 if nsteps >= 8 else 1
+    warps = (nsteps + spw - 1) // spw
+    buf = 16 * (Kmax // 2) + (Kmax // 2 if mx else Kmax)
+    for ng in (1, 2):
+        red = 2 * warps * ng * 4 * 32 * 4
+        smem3 = 3 * buf + red
+        S = 3 if 2 * (smem3 + 6 * 1024) <= 227 * 1024 else 2
+        smem = S * buf + red
+        assert smem <= 200 * 1024
+        assert buf % 16 == 0  # every stage starts on a cp.async boundary
+        if S == 2:
+            assert 2 * buf + red + 6 * 1024 <= 227 * 1024  # one CTA fits with room for the static part
