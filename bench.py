@@ -803,16 +803,29 @@ def bench_prefill(args, shape, rank, world, local):
         i_gu, i_dn = abi.KERNEL_NAMES.index("prefill_gate_up"), abi.KERNEL_NAMES.index("prefill_down")
         dom, fl = (i_gu, flops_gu) if kernel_ms(kst, i_gu) >= kernel_ms(kst, i_dn) else (i_dn, flops_dn)
         if kst.kernel_launches[dom] and kernel_ms(kst, dom) > 0:
-            achieved = fl / (kernel_ms(kst, dom) * 1e-3) / 1e12
-            roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "tensor", "achieved": achieved,
-                    "peak": tpeak, "unit": "TFLOP/s", "frac": achieved / tpeak,
-                    "peak_kind": tkind, "traffic": None,
+            # the binding roof of the grouped GEMM: its FLOPs against the FP4 tensor peak, or
+            # the expert weights it streams (each read once per layer) against HBM -- with
+            # about k*T/E rows per expert its arithmetic intensity sits below the ridge point
+            span = kernel_ms(kst, dom) * 1e-3
+            wbytes = kst.kernel_bytes[dom]
+            tflops, gbs = fl / span / 1e12, wbytes / span / 1e9
+            hbm_bound = wbytes / (hbm_peak * 1e9) > fl / (tpeak * 1e12)
+            roof = {"kernel": abi.KERNEL_NAMES[dom], "bound": "hbm" if hbm_bound else "tensor",
+                    "achieved": gbs if hbm_bound else tflops,
+                    "peak": hbm_peak if hbm_bound else tpeak, "unit": "GB/s" if hbm_bound else "TFLOP/s",
+                    "frac": gbs / hbm_peak if hbm_bound else tflops / tpeak,
+                    "peak_kind": f"{peak_kind} hbm_gbs (burst copy)" if hbm_bound else tkind,
+                    "traffic": None,
+                    "tensor_tflops": tflops, "tensor_frac": tflops / tpeak, "tensor_peak": tpeak,
+                    "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak,
+                    "flop_per_weight_byte": fl / max(wbytes, 1.0),
                     "launches": int(kst.kernel_launches[dom]),
                     "avg_launch_us": kernel_ms(kst, dom) * 1e3 / kst.kernel_launches[dom],
                     "timing": "device span" if kst.kernel_span_ms[dom] > 0 else "events",
                     "flops_per_launch": fl / kst.kernel_launches[dom],
-                    "note": "tcgen05.mma kind::mxf4nvf4 block16 (E2M1 x E2M1, E4M3 scales), "
-                            "TMA-fed, fp32 accumulation in tensor memory"}
+                    "bytes_per_launch": wbytes / kst.kernel_launches[dom],
+                    "note": "grouped tcgen05.mma block-scaled FP4 (E2M1 x E2M1), TMA-fed, fp32 "
+                            "accumulation in tensor memory"}
         for name, f in (("prefill_gate_up", flops_gu), ("prefill_down", flops_dn)):
             i = abi.KERNEL_NAMES.index(name)
             if kernel_ms(kst, i) > 0 and name in kernels:
@@ -830,8 +843,10 @@ def bench_prefill(args, shape, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_rows(shape, pool.array, P, Wr, shared, x, rows=64, w4a4=True)
     if rank == 0:
-        # route, scatter, quant x, gate/up, quant h, down, combine per layer
-        launches = int(st.forward_calls * 7)
+        # per layer: logits GEMM, top-k, lookup, scatter, tile plan, quant x, gate/up GEMM,
+        # quant h, down GEMM, combine (+ a BF16 shared expert's GEMM, SwiGLU split, GEMM)
+        bf16_shared = shape.shared and formats(args)[1] == sp.FMT_BF16
+        launches = int(st.forward_calls * (10 + (3 if bf16_shared else 0)))
         line = {
             "metric": "MoE prefill tok/s (4096-row chunk, cold cache, next-layer prefetch); "
                       "% of HBM+H2D roofline",
