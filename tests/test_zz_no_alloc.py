@@ -23,6 +23,9 @@ MID = synth.LayerShape("mid", L=3, E=40, k=5, d=960, F=320, shared=True, tokens=
 
 
 def _noalloc(Wr_d, x_d, T, E, d, k, renorm, stream):
+    """One call on `stream`.  The caller keeps Wr_d and x_d alive until the stream
+    has synchronised: the kernel reads them there, after this returns, and the
+    caching allocator may hand a freed block to the next allocation at once."""
     idx_d = torch.full((T, k), -1, dtype=torch.int32, device="cuda")
     gates_d = torch.full((T, k), -1.0, dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
@@ -68,10 +71,11 @@ def test_noalloc_full_scratch_matches_the_oracle():
     xa = conditioned_prefill(Wr, k, 0, T)[0]
     xb = conditioned_prefill(Wr, k, 1, T)[0]
     Wr_d = torch.from_numpy(Wr).cuda()
+    xs_d = [torch.from_numpy(xa).cuda(), torch.from_numpy(xb).cuda()]
     stream = torch.cuda.Stream()
     got = []
-    for x, renorm in [(xa, True), (xb, False)]:
-        got.append((x, renorm) + _noalloc(Wr_d, torch.from_numpy(x).cuda(), T, E, d, k, renorm, stream))
+    for x, x_d, renorm in [(xa, xs_d[0], True), (xb, xs_d[1], False)]:
+        got.append((x, renorm) + _noalloc(Wr_d, x_d, T, E, d, k, renorm, stream))
     stream.synchronize()
     for x, renorm, idx_d, gates_d in got:
         want_idx, want_g, _, _ = oracle.route(Wr, x, k, renorm=renorm)
@@ -87,13 +91,13 @@ def test_noalloc_ragged_expert_count_after_a_larger_call():
     stream = torch.cuda.Stream()
     Wbig = synth.router_bf16(2, 1024, 256)
     xbig = conditioned_prefill(Wbig, 32, 2, 32)[0]
-    _noalloc(torch.from_numpy(Wbig).cuda(), torch.from_numpy(xbig).cuda(), 32, 1024, 256, 32, True,
-             stream)
+    big_d = (torch.from_numpy(Wbig).cuda(), torch.from_numpy(xbig).cuda())
+    _noalloc(big_d[0], big_d[1], 32, 1024, 256, 32, True, stream)
     E, d, k, T = 1000, 192, 7, 5
     Wr = synth.router_bf16(3, E, d)
     x = conditioned_prefill(Wr, k, 3, T)[0]
-    idx_d, gates_d = _noalloc(torch.from_numpy(Wr).cuda(), torch.from_numpy(x).cuda(), T, E, d, k,
-                              True, stream)
+    small_d = (torch.from_numpy(Wr).cuda(), torch.from_numpy(x).cuda())
+    idx_d, gates_d = _noalloc(small_d[0], small_d[1], T, E, d, k, True, stream)
     stream.synchronize()
     want_idx, want_g, _, _ = oracle.route(Wr, x, k)
     np.testing.assert_array_equal(idx_d.cpu().numpy(), want_idx)
@@ -111,8 +115,8 @@ def test_noalloc_non_finite_rows_follow_the_selection_rule():
     x[1, 7] = synth.to_bf16(np.array([np.nan], np.float32))[0]
     x[2, 0] = synth.to_bf16(np.array([np.inf], np.float32))[0]
     stream = torch.cuda.Stream()
-    idx_d, gates_d = _noalloc(torch.from_numpy(Wr).cuda(), torch.from_numpy(x).cuda(), 4, E, d, k,
-                              True, stream)
+    in_d = (torch.from_numpy(Wr).cuda(), torch.from_numpy(x).cuda())
+    idx_d, gates_d = _noalloc(in_d[0], in_d[1], 4, E, d, k, True, stream)
     stream.synchronize()
     want_idx, want_g, _, _ = oracle.route(Wr, x, k)
     got_idx = idx_d.cpu().numpy()
