@@ -72,6 +72,9 @@ def parse():
                     help="routed expert records (decode): NVFP4 (default) or MXFP4")
     ap.add_argument("--shared-format", default="same", choices=["same", "bf16"],
                     help="shared expert records: the routed format (default) or BF16")
+    ap.add_argument("--per-miss-launches", action="store_true",
+                    help="decode without the layer kernel: a gate/up and a down launch per miss, "
+                         "gated by copy events (the path where stream memory writes are unavailable)")
     ap.add_argument("--ep", action="store_true",
                     help="decode with N > 1: expert parallelism (rank r serves experts e %% N == r, its "
                          "own cache; the partial outputs all-reduced per layer) instead of replicas")
@@ -444,6 +447,8 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
     stack = LayerStack(dims, pool.tensor, sp.to_device(Wr), sp.to_device(shared),
                        shape.cache_slots, prefetch=prefetch,
                        static_split=getattr(args, "policy", "lru") == "static", shard=shard)
+    if getattr(args, "per_miss_launches", False):
+        abi.moe_debug_inject(stack.ctx, 3, 0)
 
     # H2D bandwidth of this machine, measured now (the roofline's PCIe term)
     nb = 1 << 30
@@ -601,7 +606,8 @@ def bench_decode(args, shape, rank, world, local):
                        "cold_cache": not args.warm,
                        "parallelism": (f"expert parallel x{world} (experts e % {world} per rank, "
                                        f"partial outputs all-reduced per layer)") if ep else f"replicas x{world}",
-                       "pool_distinct_records": DISTINCT_RECORDS, "policy": args.policy},
+                       "pool_distinct_records": DISTINCT_RECORDS, "policy": args.policy,
+                       "expert_kernels": "a launch per miss" if args.per_miss_launches else "layer kernel"},
             "miss_rate": counts["misses"] / max(counts["lookups"], 1),
             "counts": {"source": source, **counts,
                        "gpu_counters_match": all(gpu_counts[f] == counts[f] for f in counts)},
