@@ -355,31 +355,37 @@ __global__ void __launch_bounds__(kMaxSteps * 32) expert_layer_kernel(LayerArgs 
                 }
             }
         }
-        __syncthreads();  // warp 0's outputs of this item are written
-        if (gate_up) {
-            if (threadIdx.x == 0) {
-                __threadfence();
-                atomicAdd(a.done_a + it.job, 1u);
-            }
-        } else {  // the tile's last expert combines its rows
-            if (threadIdx.x == 0) {
-                __threadfence();
-                s_last = atomicAdd(&a.tile_ticket[it.tile], 1u) == (unsigned)(H + M - 1);
-            }
-            __syncthreads();
-            if (s_last) {
-                __threadfence();
-                for (int e = threadIdx.x; e < 16 * a.T; e += blockDim.x) {
-                    const int t = e >> 4, o = 16 * it.tile + (e & 15);
-                    const float *pr = a.part + (size_t)t * (a.k + 1) * a.d + o;
-                    float sum = 0.f;
-                    for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
-                        if (a.ep_size == 1 || a.idx[t * a.k + p] % a.ep_size == a.ep_rank)
-                            sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
-                    if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
-                    a.y[(size_t)t * a.d + o] = sum;
+        // warp 0 wrote this item's outputs; it also publishes them (the other warps
+        // wait for it at the next item's barrier): a warp barrier orders its lanes'
+        // stores before lane 0's fence and counter update
+        if (warp == 0) {
+            __syncwarp();
+            if (gate_up) {
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(a.done_a + it.job, 1u);
                 }
-                if (threadIdx.x == 0) a.tile_ticket[it.tile] = 0u;
+            } else {  // the tile's last expert combines its rows
+                int last = 0;
+                if (lane == 0) {
+                    __threadfence();
+                    last = atomicAdd(&a.tile_ticket[it.tile], 1u) == (unsigned)(H + M - 1);
+                }
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence();
+                    for (int e = lane; e < 16 * a.T; e += 32) {
+                        const int t = e >> 4, o = 16 * it.tile + (e & 15);
+                        const float *pr = a.part + (size_t)t * (a.k + 1) * a.d + o;
+                        float sum = 0.f;
+                        for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
+                            if (a.ep_size == 1 || a.idx[t * a.k + p] % a.ep_size == a.ep_rank)
+                                sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                        if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
+                        a.y[(size_t)t * a.d + o] = sum;
+                    }
+                    if (lane == 0) a.tile_ticket[it.tile] = 0u;
+                }
             }
         }
         if (threadIdx.x == 0 && i < hit_items) span_mark(a.span_hit, 1);
