@@ -17,8 +17,8 @@
 //   hit and shared experts: all gate/up tiles, then all down tiles;
 //   then per miss, in the order the host copies them (ascending expert id):
 //   its gate/up tiles, then its down tiles.
-// CTAs reserve items with an atomic counter, a few consecutive ones at a time,
-// and stage the next ones while they compute the current one (cp.async ring).  A down tile needs all of its
+// CTAs claim items with an atomic counter and stage the next ones while they
+// compute the current one (3-deep cp.async ring).  A down tile needs all of its
 // expert's gate/up tiles (h): those come earlier in the queue, so they are
 // already held by running CTAs, which wait on nothing but copy flags -- the
 // smallest unfinished item can always proceed, so the schedule cannot
@@ -40,7 +40,6 @@ namespace {
 using namespace gemv;
 
 constexpr int kSharedJob = kMaxSlots - 1;  // done_a slot of the shared expert
-constexpr int kClaim = 4;                   // queue items reserved per atomic
 
 // Error codes written to HostPage::error by this kernel.
 constexpr int kErrFlagWait = 40;   // a miss's copy flag did not arrive in time
@@ -92,7 +91,7 @@ struct Item {
 // S: tiles in flight per CTA (the shared-memory ring); 2 where 3 would keep
 // two CTAs from sharing an SM.
 template <int NG, int FMT, int S>
-__global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerArgs a) {
+__global__ void __launch_bounds__(kMaxSteps * 32) expert_layer_kernel(LayerArgs a) {
     constexpr int kRing = S + 1;  // claimed-item slots: one more than the tiles in flight
     extern __shared__ __align__(128) uint8_t smem[];
     // the launch's experts: hits (ascending job index, then the shared expert)
@@ -139,42 +138,6 @@ __global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerAr
     }
     __syncthreads();
     const int H = s_nhit, M = s_nmiss;
-    // per-job metadata in shared memory, read once here instead of from global
-    // memory in every item: slot, rows, first row, the tensor scales of a
-    // resident record (a miss's are read after its flag), and the row refs
-    const int cap = a.job_cap;  // jobs of the launch + 1 (the shared expert's entry: cap - 1)
-    int *m_slot = reinterpret_cast<int *>(smem + a.meta_off);
-    int *m_rows = m_slot + cap, *m_off = m_rows + cap;
-    float *m_ts = reinterpret_cast<float *>(m_off + cap);  // [cap][3]
-    RowRef *m_rr = reinterpret_cast<RowRef *>(m_ts + 3 * cap);  // [T * k]
-    {
-        const int nj = H + M - (a.shared_item ? 1 : 0);
-        for (int j = threadIdx.x; j < nj; j += blockDim.x) {
-            const int slot = __ldcg(&a.jobs[j].slot);
-            m_slot[j] = slot;
-            m_rows[j] = __ldcg(&a.jobs[j].nrows);
-            m_off[j] = __ldcg(&a.jobs[j].row_off);
-            if (!kMx && __ldcg(&a.jobs[j].hit)) {
-                const float *t = reinterpret_cast<const float *>(a.arena + (int64_t)slot * a.rec_bytes + a.lay.tscales);
-                m_ts[3 * j] = t[0];
-                m_ts[3 * j + 1] = t[1];
-                m_ts[3 * j + 2] = t[2];
-            }
-        }
-        if (threadIdx.x == 0 && a.shared_item) {
-            m_rows[cap - 1] = a.T;
-            m_off[cap - 1] = 0;
-            if (!kMx) {
-                const float *t = reinterpret_cast<const float *>(a.shared_rec + a.lay.tscales);
-                m_ts[3 * (cap - 1)] = t[0];
-                m_ts[3 * (cap - 1) + 1] = t[1];
-                m_ts[3 * (cap - 1) + 2] = t[2];
-            }
-        }
-        for (int i = threadIdx.x; i < a.T * a.k; i += blockDim.x) m_rr[i] = a.rowrefs[i];
-    }
-    __syncthreads();
-    auto ci = [&](int job) { return job == kSharedJob ? cap - 1 : job; };
     const int nA = a.F >> 3, nB = a.d >> 4, per = nA + nB;
     if (H + M == 0 && blockIdx.x == 0) {
         // a shard of an expert-parallel layer that owns none of the selected
@@ -201,7 +164,7 @@ __global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerAr
         return it;
     };
     auto record = [&](int job) -> const uint8_t * {
-        return job == kSharedJob ? a.shared_rec : a.arena + (int64_t)m_slot[job] * a.rec_bytes;
+        return job == kSharedJob ? a.shared_rec : a.arena + (int64_t)__ldcg(&a.jobs[job].slot) * a.rec_bytes;
     };
     auto flag_of = [&](const Item &it) -> const uint32_t * {  // null: resident, nothing to wait for
         return it.miss < 0 ? nullptr : a.miss_flag + 2 * it.job + (it.gate_up ? 0 : 1);
@@ -236,17 +199,9 @@ __global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerAr
         }
     };
     // claim (thread 0): the next queue item into ring slot j % kRing, and
-    // whether its record is already resident (else its copies wait for compute
-    // time).  Items are reserved kClaim at a time (one atomic round trip per
-    // kClaim items); a CTA still takes its items in increasing order.
-    int next_i = 0, left = 0;  // (thread 0) the rest of the current reservation
+    // whether its record is already resident (else its copies wait for compute time)
     auto claim = [&](int j) {
-        if (left == 0) {
-            next_i = (int)atomicAdd(a.queue, (unsigned)kClaim);
-            left = kClaim;
-        }
-        const int i = next_i++;
-        --left;
+        const int i = (int)atomicAdd(a.queue, 1u);
         s_item[j % kRing] = i;
         int def = 0;
         if (i < total) {
@@ -307,12 +262,10 @@ __global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerAr
         const int NCH = K >> 6, nsteps = (NCH + 3) >> 2, spw = (nsteps + nwarps - 1) / nwarps;
         const uint32_t code_bytes = 16u * (uint32_t)(K >> 1);
         const uint8_t *rec = record(it.job);
-        const int nrows = m_rows[ci(it.job)];
-        const int row_off = m_off[ci(it.job)];
+        const int nrows = shared ? a.T : __ldcg(&a.jobs[it.job].nrows);
+        const int row_off = shared ? 0 : __ldcg(&a.jobs[it.job].row_off);
         const uint8_t *s_codes = smem + (j % S) * buf_bytes, *s_scales = s_codes + code_bytes;
-        // tensor scales: cached for a resident record; a miss's from its slot (landed)
-        const float *ts = kMx ? nullptr
-                              : (it.miss < 0 ? m_ts + 3 * ci(it.job) : reinterpret_cast<const float *>(rec + a.lay.tscales));
+        const float *ts = kMx ? nullptr : reinterpret_cast<const float *>(rec + a.lay.tscales);
         const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
         const __half *act = gate_up ? a.xh : a.hh;
         for (int r0 = 0; r0 < nrows; r0 += 4 * NG) {
@@ -328,7 +281,7 @@ __global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerAr
                 if (colv[grp]) {
                     int t, p;
                     if (shared) { t = r; p = a.k; }
-                    else { const RowRef rf = m_rr[row_off + r]; t = rf.t; p = rf.p; }
+                    else { const RowRef rf = a.rowrefs[row_off + r]; t = rf.t; p = rf.p; }
                     col[grp] = gate_up ? act + (size_t)t * 2 * a.d + (g & 1) * a.d
                                        : act + (size_t)(t * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
                 }
@@ -381,7 +334,7 @@ __global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerAr
                     if (r >= nrows) continue;
                     int t, p;
                     if (shared) { t = r; p = a.k; }
-                    else { const RowRef rf = m_rr[row_off + r]; t = rf.t; p = rf.p; }
+                    else { const RowRef rf = a.rowrefs[row_off + r]; t = rf.t; p = rf.p; }
                     const float v0 = acc[grp][0] + acc[grp][1];
                     const float v1 = acc[grp][2] + acc[grp][3];
                     const size_t sel = (size_t)t * (a.k + 1) + p;
@@ -402,37 +355,31 @@ __global__ void __launch_bounds__(kMaxSteps * 32, 1) expert_layer_kernel(LayerAr
                 }
             }
         }
-        // warp 0 wrote this item's outputs; it also publishes them (the other warps
-        // wait for it at the next item's barrier): a warp barrier orders its lanes'
-        // stores before lane 0's fence and counter update
-        if (warp == 0) {
-            __syncwarp();
-            if (gate_up) {
-                if (lane == 0) {
-                    __threadfence();
-                    atomicAdd(a.done_a + it.job, 1u);
+        __syncthreads();  // warp 0's outputs of this item are written
+        if (gate_up) {
+            if (threadIdx.x == 0) {
+                __threadfence();
+                atomicAdd(a.done_a + it.job, 1u);
+            }
+        } else {  // the tile's last expert combines its rows
+            if (threadIdx.x == 0) {
+                __threadfence();
+                s_last = atomicAdd(&a.tile_ticket[it.tile], 1u) == (unsigned)(H + M - 1);
+            }
+            __syncthreads();
+            if (s_last) {
+                __threadfence();
+                for (int e = threadIdx.x; e < 16 * a.T; e += blockDim.x) {
+                    const int t = e >> 4, o = 16 * it.tile + (e & 15);
+                    const float *pr = a.part + (size_t)t * (a.k + 1) * a.d + o;
+                    float sum = 0.f;
+                    for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
+                        if (a.ep_size == 1 || a.idx[t * a.k + p] % a.ep_size == a.ep_rank)
+                            sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                    if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
+                    a.y[(size_t)t * a.d + o] = sum;
                 }
-            } else {  // the tile's last expert combines its rows
-                int last = 0;
-                if (lane == 0) {
-                    __threadfence();
-                    last = atomicAdd(&a.tile_ticket[it.tile], 1u) == (unsigned)(H + M - 1);
-                }
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {
-                    __threadfence();
-                    for (int e = lane; e < 16 * a.T; e += 32) {
-                        const int t = e >> 4, o = 16 * it.tile + (e & 15);
-                        const float *pr = a.part + (size_t)t * (a.k + 1) * a.d + o;
-                        float sum = 0.f;
-                        for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
-                            if (a.ep_size == 1 || a.idx[t * a.k + p] % a.ep_size == a.ep_rank)
-                                sum = fmaf(a.gates[t * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
-                        if (a.shared_rec) sum += __ldcg(pr + (size_t)a.k * a.d);
-                        a.y[(size_t)t * a.d + o] = sum;
-                    }
-                    if (lane == 0) a.tile_ticket[it.tile] = 0u;
-                }
+                if (threadIdx.x == 0) a.tile_ticket[it.tile] = 0u;
             }
         }
         if (threadIdx.x == 0 && i < hit_items) span_mark(a.span_hit, 1);
@@ -491,17 +438,12 @@ cudaError_t launch_layer_ng(const LayerArgs &a, int threads, size_t smem, cudaSt
 }
 
 template <int NG, int FMT>
-cudaError_t launch_layer_fmt(const LayerArgs &a, int threads, size_t buf, size_t red, size_t meta, cudaStream_t st) {
+cudaError_t launch_layer_fmt(const LayerArgs &a, int threads, size_t buf, size_t red, cudaStream_t st) {
     // 3 tiles in flight unless that keeps a second CTA off the SM (227 KB of
     // shared memory per SM, of which ~5 KB static per CTA)
-    LayerArgs b = a;
-    const size_t smem3 = 3 * buf + red + meta;
-    if (2 * (smem3 + 6 * 1024) <= 227 * 1024) {
-        b.meta_off = (unsigned)(3 * buf + red);
-        return launch_layer_ng<NG, FMT, 3>(b, threads, smem3, st);
-    }
-    b.meta_off = (unsigned)(2 * buf + red);
-    return launch_layer_ng<NG, FMT, 2>(b, threads, 2 * buf + red + meta, st);
+    const size_t smem3 = 3 * buf + red;
+    if (2 * (smem3 + 6 * 1024) <= 227 * 1024) return launch_layer_ng<NG, FMT, 3>(a, threads, smem3, st);
+    return launch_layer_ng<NG, FMT, 2>(a, threads, 2 * buf + red, st);
 }
 
 }  // namespace
@@ -517,16 +459,14 @@ cudaError_t launch_expert_layer(const LayerArgs &a, cudaStream_t s) {
     if (!mx && a.lay.fmt != kFmtNvfp4) return cudaErrorInvalidValue;
     const size_t buf = 16 * (size_t)(Kmax / 2) + (size_t)(mx ? Kmax / 2 : Kmax);
     const size_t red = 2 * (size_t)warps * ng * 4 * 32 * sizeof(float);
-    // metadata cache: slot, rows, first row, 3 tensor scales per job; the row refs
-    const size_t meta = ((size_t)a.job_cap * 24 + (size_t)a.T * a.k * sizeof(RowRef) + 15) & ~(size_t)15;
-    if (a.job_cap < 1 || a.job_cap > kMaxSlots || 2 * buf + red + meta > 200 * 1024) return cudaErrorInvalidValue;
+    if (2 * buf + red > 200 * 1024) return cudaErrorInvalidValue;
     const int threads = warps * 32;
     if (mx) {
-        if (ng == 1) return launch_layer_fmt<1, kFmtMxfp4>(a, threads, buf, red, meta, s);
-        return launch_layer_fmt<2, kFmtMxfp4>(a, threads, buf, red, meta, s);
+        if (ng == 1) return launch_layer_fmt<1, kFmtMxfp4>(a, threads, buf, red, s);
+        return launch_layer_fmt<2, kFmtMxfp4>(a, threads, buf, red, s);
     }
-    if (ng == 1) return launch_layer_fmt<1, kFmtNvfp4>(a, threads, buf, red, meta, s);
-    return launch_layer_fmt<2, kFmtNvfp4>(a, threads, buf, red, meta, s);
+    if (ng == 1) return launch_layer_fmt<1, kFmtNvfp4>(a, threads, buf, red, s);
+    return launch_layer_fmt<2, kFmtNvfp4>(a, threads, buf, red, s);
 }
 
 }  // namespace moe

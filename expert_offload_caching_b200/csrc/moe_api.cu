@@ -546,7 +546,6 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         la.idx = ctx->dws.idx;
         la.ep_rank = ctx->ep_rank;
         la.ep_size = ctx->ep_size;
-        la.job_cap = max_jobs(&D, T) + 1;
         TimedLaunch tk, th;
         time_begin(ctx, tk, MOE_K_LAYER);
         la.span = time_span(ctx, tk);

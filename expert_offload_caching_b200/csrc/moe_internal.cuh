@@ -192,8 +192,6 @@ struct LayerArgs {
     unsigned long long *span_hit;  // [start, end of the last hit/shared item], or null
     const int32_t *idx;            // [T][k] selected experts: the combine takes the owned ones only
     int ep_rank, ep_size;
-    int job_cap;                   // jobs of the launch at most + 1 (sizes the metadata cache)
-    unsigned meta_off;             // byte offset of the metadata cache in dynamic shared memory
 };
 
 // Grouped W4A4 expert GEMMs of a prefill chunk (tcgen05 block-scaled MMA).

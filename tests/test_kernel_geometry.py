@@ -269,22 +269,18 @@ def test_layer_queue_covers_every_tile_once_in_dependency_order(shape, H, M):
 @pytest.mark.parametrize("mx", [False, True])
 def test_layer_kernel_ring_fits_and_keeps_two_ctas_per_sm_where_it_can(shape, mx):
     """The launcher's choice: a 3-tile ring when two CTAs still fit an SM (227 KB of
-    shared memory, ~5 KB static per CTA), else 2; the ring covers the longer K, and
-    the per-job metadata cache follows it."""
+    shared memory, ~5 KB static per CTA), else 2; the ring covers the longer K."""
     Kmax = max(shape.d, shape.F)
     nsteps = (Kmax // 64 + 3) // 4
     spw = 2 if nsteps >= 8 else 1
     warps = (nsteps + spw - 1) // spw
     buf = 16 * (Kmax // 2) + (Kmax // 2 if mx else Kmax)
-    for T in (1, 16, 32):
-        ng = 1 if T <= 4 else 2
+    for ng in (1, 2):
         red = 2 * warps * ng * 4 * 32 * 4
-        cap = min(T * shape.k, shape.E) + 1  # the metadata cache: per job 24 bytes, + the row refs
-        meta = (cap * 24 + T * shape.k * 4 + 15) & ~15
-        smem3 = 3 * buf + red + meta
+        smem3 = 3 * buf + red
         S = 3 if 2 * (smem3 + 6 * 1024) <= 227 * 1024 else 2
-        smem = S * buf + red + meta
+        smem = S * buf + red
         assert smem <= 200 * 1024
-        assert buf % 16 == 0 and (S * buf + red) % 16 == 0  # stages and cache on 16-byte boundaries
+        assert buf % 16 == 0  # every stage starts on a cp.async boundary
         if S == 2:
             assert smem + 6 * 1024 <= 227 * 1024  # one CTA fits with room for the static part
