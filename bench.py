@@ -72,9 +72,15 @@ def parse():
                     help="routed expert records (decode): NVFP4 (default) or MXFP4")
     ap.add_argument("--shared-format", default="same", choices=["same", "bf16"],
                     help="shared expert records: the routed format (default) or BF16")
-    ap.add_argument("--per-miss-launches", action="store_true",
-                    help="decode without the layer kernel: a gate/up and a down launch per miss, "
-                         "gated by copy events (the path where stream memory writes are unavailable)")
+    ap.add_argument("--layer-kernel", action="store_true",
+                    help="decode through the persistent layer kernel (one launch per layer, misses gated "
+                         "by copy flags) instead of the default launches (hit experts, then a gate/up and "
+                         "a down launch per miss, gated by copy events)")
+    ap.add_argument("--split-k", action="store_true",
+                    help="the default decode launches with the split-K expert kernels instead of the "
+                         "streaming ones")
+    ap.add_argument("--copy-streams", type=int, default=0, choices=[0, 1, 2],
+                    help="decode misses on 1 or 2 copy streams (0: the library's default)")
     ap.add_argument("--ep", action="store_true",
                     help="decode with N > 1: expert parallelism (rank r serves experts e %% N == r, its "
                          "own cache; the partial outputs all-reduced per layer) instead of replicas")
@@ -447,8 +453,12 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
     stack = LayerStack(dims, pool.tensor, sp.to_device(Wr), sp.to_device(shared),
                        shape.cache_slots, prefetch=prefetch,
                        static_split=getattr(args, "policy", "lru") == "static", shard=shard)
-    if getattr(args, "per_miss_launches", False):
-        abi.moe_debug_inject(stack.ctx, 3, 0)
+    if getattr(args, "layer_kernel", False):
+        abi.moe_debug_inject(stack.ctx, 3, 1)
+    if getattr(args, "split_k", False):
+        abi.moe_debug_inject(stack.ctx, 7, 0)
+    if getattr(args, "copy_streams", 0):
+        abi.moe_debug_inject(stack.ctx, 6, args.copy_streams)
 
     # H2D bandwidth of this machine, measured now (the roofline's PCIe term)
     nb = 1 << 30
@@ -466,6 +476,13 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
         H2D_SM = {"h2d_sm_gbs": None, "h2d_sm_note": str(e)}
     del dbuf, hbuf
     return stack, pool, P, rb, Wr, shared, h2d, h2d_rec
+
+
+def expert_kernels_label(args) -> str:
+    if getattr(args, "layer_kernel", False):
+        return "persistent layer kernel (misses gated by copy flags)"
+    kind = "split-K" if getattr(args, "split_k", False) else "streaming"
+    return f"{kind} expert kernels: one launch for the hit experts, a gate/up and a down launch per miss"
 
 
 def main():
@@ -607,7 +624,8 @@ def bench_decode(args, shape, rank, world, local):
                        "parallelism": (f"expert parallel x{world} (experts e % {world} per rank, "
                                        f"partial outputs all-reduced per layer)") if ep else f"replicas x{world}",
                        "pool_distinct_records": DISTINCT_RECORDS, "policy": args.policy,
-                       "expert_kernels": "a launch per miss" if args.per_miss_launches else "layer kernel"},
+                       "expert_kernels": expert_kernels_label(args),
+                       "copy_streams": args.copy_streams or "default"},
             "miss_rate": counts["misses"] / max(counts["lookups"], 1),
             "counts": {"source": source, **counts,
                        "gpu_counters_match": all(gpu_counts[f] == counts[f] for f in counts)},
@@ -683,7 +701,7 @@ TRAFFIC_RATIO = {
 
 # Kernel classes whose device time is not bounded by HBM: the whole decode layer
 # kernel waits for the PCIe copies of the misses (its HBM-bound part, the
-# resident experts, is the class expert_layer_hits).
+# resident experts, is the class expert_hits).
 NOT_HBM_BOUND = {"expert_layer"}
 
 

@@ -1,0 +1,567 @@
+// Streaming expert GEMVs for decode (W4A16 over NVFP4 / MXFP4 records):
+// gate/up with fused SwiGLU, down, and the gate-weighted combine.
+//
+// The arithmetic is the routed expert of the FreeToken pages (florigen.ai
+// "NVFP4で約135GBまで縮める": NVFP4 routed experts; ai-hardware-zukan
+// "GPUに載らない分をどう間に合わせるか": MXFP4 checkpoints):
+//   h_j = silu(g_j) * u_j,  g = W1 x, u = W3 x;   y_e = W2 h;
+//   y = sum over selected e (ascending id) of gate_e * y_e + y_shared.
+//
+// Decode reads each weight once for 1-32 activation rows, so the launch is
+// bound by how many weight bytes are in flight, not by math.  Design:
+//   * one CTA per SM; warp 0's lane 0 is the producer: it walks the CTA's
+//     work items (a few consecutive 16-row weight tiles of one expert, whose
+//     codes and scales are contiguous in the record) and moves each with two
+//     1-D bulk copies (cp.async.bulk, completion counted on the stage's
+//     mbarrier, L2 evict-first) into a ring of shared-memory stages; it waits
+//     for a stage's previous item to be released before reusing it;
+//   * consumer warps (warps 1..C) take the CTA's items in turn (item l: warp
+//     1 + l mod C, stage l mod S, with S a multiple of C, so each stage serves
+//     one warp and its uses are waited on in order); a warp
+//     computes every tile of its item over the whole K by itself, so there is
+//     no cross-warp reduction and no CTA barrier per item: it waits on the
+//     stage's full barrier, runs the K-steps (E2M1 decoded in registers,
+//     block scales applied in fp16, mma.sync m16n8k16 with fp32 accumulation:
+//     the K-step code of gemv_inner.cuh), releases the stage, and writes its
+//     outputs;
+//   * phase 3 launches run an expert's down tiles in the same launch as its
+//     gate/up tiles: every CTA's items are gate/up items first, so a down item
+//     waits (bounded) only for gate/up items that never wait -- deadlock-free
+//     with every CTA resident (one per SM);
+//   * combine: a down launch with combine set has the warp that completes the
+//     last expert of a 16-row output tile (per-tile ticket) sum the tile's rows
+//     over the layer's selected experts in ascending id, plus the shared
+//     expert's partial.
+// Every wait is bounded (globaltimer, the launch's wait_ns); a wait that runs
+// out writes the mapped page's error word, the CTA stops, and no bulk copy
+// outlives it.
+#include "gemv_inner.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace gemv;
+
+constexpr int kStMaxStages = 8;
+constexpr int kStMaxConsumers = 7;             // + the producer warp: 256 threads
+constexpr int kErrStreamFull = 42;             // a stage's copy did not land in time
+constexpr int kErrStreamEmpty = 43;            // a stage was not released in time
+constexpr int kErrStreamDep = 44;              // a down item's gate/up tiles did not complete in time
+constexpr int kErrStreamSize = 45;             // more experts than the metadata area holds
+
+struct ExpMeta {            // one expert of the launch (dynamic shared memory)
+    const uint8_t *rec;     // its record (slot in the arena, or the shared record)
+    int nrows, row_off;     // rows using it, first row ref
+    float ts[3];            // NVFP4 tensor scales (gate, up, down)
+    int job;                // job index, -1: the shared expert
+};
+static_assert(sizeof(ExpMeta) == 32, "metadata stride");
+
+__device__ __forceinline__ unsigned long long st_now() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ uint32_t st_ld_acquire(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void st_mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void st_mbar_expect(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool st_mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// Wait for the phase of the given parity; false when the deadline passes or
+// the CTA is stopping.
+__device__ __forceinline__ bool st_mbar_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline,
+                                             volatile int *stop) {
+    for (uint32_t i = 0;; ++i) {
+        if (st_mbar_test(bar, parity)) return true;
+        if ((i & 31u) == 31u && (*stop || st_now() > deadline)) return false;
+    }
+}
+// 1-D bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completion counted on bar; L2 evict-first (read once).
+__device__ __forceinline__ void st_bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ void st_fail(const GemvArgs &a, int code, int item, int what) {
+    HostPage *pg = a.page;
+    pg->diag[1] = 31;  // kernel: expert_stream
+    pg->diag[2] = (int)blockIdx.x;
+    pg->diag[3] = item;
+    pg->diag[4] = what;
+    pg->diag[5] = a.phase;
+    __threadfence_system();
+    pg->error = code;
+    __threadfence_system();
+}
+
+// A work item: expert e (launch-local), gate/up (else down), tiles
+// [tile0, tile0 + nt).  Items are numbered gate/up first (expert-major), then
+// down (phase 3).
+struct StItem {
+    int e, gate_up, tile0, nt;
+};
+__device__ __forceinline__ StItem st_item(int g, int phase, int nexp, int nA, int nB, int iA, int iB, int tpa,
+                                          int tpb) {
+    StItem it;
+    const int gA = (phase & 1) ? nexp * iA : 0;
+    if (g < gA) {
+        it.e = g / iA;
+        it.tile0 = (g - it.e * iA) * tpa;
+        it.nt = min(tpa, nA - it.tile0);
+        it.gate_up = 1;
+    } else {
+        g -= gA;
+        it.e = g / iB;
+        it.tile0 = (g - it.e * iB) * tpb;
+        it.nt = min(tpb, nB - it.tile0);
+        it.gate_up = 0;
+    }
+    return it;
+}
+
+template <int NG, int FMT>
+__global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_kernel(GemvArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t s_full[kStMaxStages], s_empty[kStMaxStages];
+    __shared__ int s_nexp, s_last;
+    __shared__ volatile int s_stop;
+    constexpr bool kMx = FMT == kFmtMxfp4;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int NS = a.ns, C = a.nc;
+    ExpMeta *meta = reinterpret_cast<ExpMeta *>(smem + a.meta_off);
+    RowRef *rrs = reinterpret_cast<RowRef *>(smem + a.rr_off);
+
+    pdl_wait();  // the job list, x and the row refs come from the route kernel; h from gate/up
+    const unsigned long long deadline = st_now() + a.wait_ns;
+    if (threadIdx.x == 0) {
+        span_mark(a.span, 0);
+        s_stop = 0;
+        for (int s = 0; s < NS; ++s) {
+            st_mbar_init(&s_full[s], 1);   // the producer's expect-tx arrive (+ the bytes)
+            st_mbar_init(&s_empty[s], 1);  // the consumer that used the stage
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    pdl_launch_dependents();
+
+    // ---- the launch's experts: hit jobs in ascending job index, then the
+    // shared expert; or the one job only_job
+    if (warp == 0) {
+        int cnt = 0;
+        if (a.only_job >= 0) {
+            if (lane == 0) meta[0].job = a.only_job;
+            cnt = 1;
+        } else {
+            const int nj = __ldcg(a.n_jobs);
+            for (int b = 0; b < nj; b += 32) {
+                const int j = b + lane;
+                const bool hit = j < nj && __ldcg(&a.jobs[j].hit);
+                const unsigned ball = __ballot_sync(0xffffffffu, hit);
+                const int pos = cnt + __popc(ball & ((1u << lane) - 1u));
+                if (hit && pos < a.exp_cap) meta[pos].job = j;
+                cnt += __popc(ball);
+            }
+            if (a.shared_item) {
+                if (lane == 0 && cnt < a.exp_cap) meta[cnt].job = -1;
+                ++cnt;
+            }
+        }
+        if (lane == 0) {
+            if (cnt > a.exp_cap) {  // cannot happen with the host's sizing; refuse rather than overrun
+                st_fail(a, kErrStreamSize, cnt, a.exp_cap);
+                s_stop = 1;
+                cnt = 0;
+            }
+            s_nexp = cnt;
+        }
+    }
+    __syncthreads();
+    const int nexp = s_nexp;
+    for (int e = threadIdx.x; e < nexp; e += blockDim.x) {
+        ExpMeta &m = meta[e];
+        const int j = m.job;
+        if (j < 0) {
+            m.rec = a.shared_rec;
+            m.nrows = a.T;
+            m.row_off = 0;
+        } else {
+            m.rec = a.arena + (int64_t)__ldcg(&a.jobs[j].slot) * a.rec_bytes;
+            m.nrows = __ldcg(&a.jobs[j].nrows);
+            m.row_off = __ldcg(&a.jobs[j].row_off);
+        }
+        if (!kMx) {
+            const float *t = reinterpret_cast<const float *>(m.rec + a.lay.tscales);
+            m.ts[0] = t[0];
+            m.ts[1] = t[1];
+            m.ts[2] = t[2];
+        }
+    }
+    for (int i = threadIdx.x; i < a.T * a.k; i += blockDim.x) {
+        const RowRef r = a.rowrefs[i];
+        rrs[i] = r;
+    }
+    __syncthreads();
+
+    // ---- item geometry
+    const int nA = a.F >> 3, nB = a.d >> 4;  // tiles per expert: 8 gate/up row pairs, 16 down rows
+    const int iA = (nA + a.tpa - 1) / a.tpa, iB = (nB + a.tpb - 1) / a.tpb;
+    const int total = nexp * (((a.phase & 1) ? iA : 0) + ((a.phase & 2) ? iB : 0));
+    const int G = (int)gridDim.x;
+    const int n_my = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / G + 1 : 0;
+    const uint32_t cbA = 8u * (uint32_t)a.d, sbA = kMx ? (uint32_t)(a.d >> 1) : (uint32_t)a.d;
+    const uint32_t cbB = 8u * (uint32_t)a.F, sbB = kMx ? (uint32_t)(a.F >> 1) : (uint32_t)a.F;
+
+    if (nexp == 0 && a.combine && blockIdx.x == 0 && (a.combine == 1 || __ldcg(a.n_misses) == 0)) {
+        // nothing of this layer is computed here (an expert-parallel shard that
+        // owns none of the selected experts): its partial output is the shared
+        // expert's (computed by earlier launches) or zero
+        for (int i = threadIdx.x; i < a.T * a.d; i += blockDim.x) {
+            const int t = i / a.d, o = i - t * a.d;
+            a.y[i] = a.shared_part ? __ldcg(a.part_out + ((size_t)t * (a.k + 1) + a.k) * a.d + o) : 0.f;
+        }
+    }
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol = evict_first_policy();
+            int issued = 0;
+            for (int l = 0; l < n_my; ++l) {
+                const int s = l % NS, n = l / NS;
+                if (n > 0 && !st_mbar_wait(&s_empty[s], (n - 1) & 1, deadline, &s_stop)) {
+                    if (!s_stop) st_fail(a, kErrStreamEmpty, l, s);
+                    s_stop = 1;
+                    break;
+                }
+                const StItem it = st_item((int)blockIdx.x + l * G, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
+                const uint32_t cb = it.gate_up ? cbA : cbB, sb = it.gate_up ? sbA : sbB;
+                const uint8_t *rec = meta[it.e].rec;
+                const uint8_t *codes = rec + (it.gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)it.tile0 * cb;
+                const uint8_t *scales = rec + (it.gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)it.tile0 * sb;
+                uint8_t *dst = smem + (size_t)s * a.stage_bytes;
+                st_mbar_expect(&s_full[s], (uint32_t)it.nt * (cb + sb));
+                st_bulk_g2s(dst, codes, (uint32_t)it.nt * cb, &s_full[s], pol);
+                st_bulk_g2s(dst + (size_t)it.nt * cb, scales, (uint32_t)it.nt * sb, &s_full[s], pol);
+                issued = l + 1;
+            }
+            // no copy outlives the CTA: the last item issued into each stage has landed
+            const unsigned long long drain = st_now() + 1000000000ull;
+            volatile int never = 0;
+            for (int l = issued > NS ? issued - NS : 0; l < issued; ++l)
+                st_mbar_wait(&s_full[l % NS], (l / NS) & 1, drain, &never);
+        }
+    } else if (warp <= C) {
+        // ---------------------------------------------------------- consumers
+        const int g = lane >> 2, q = lane & 3;
+        for (int l = warp - 1; l < n_my; l += C) {
+            const int s = l % NS, n = l / NS;
+            // lane 0 waits (bounded); the verdict is the warp's, so the lanes stay
+            // converged for mma.sync; then every lane observes the completed phase
+            int ok = 1;
+            if (lane == 0) {
+                ok = st_mbar_wait(&s_full[s], n & 1, deadline, &s_stop);
+                if (!ok && !s_stop) st_fail(a, kErrStreamFull, l, s);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+                s_stop = 1;
+                break;
+            }
+            for (uint32_t i = 0; i < (1u << 20) && !st_mbar_test(&s_full[s], n & 1); ++i) {
+            }
+            const int gi = (int)blockIdx.x + l * G;
+            const StItem it = st_item(gi, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
+            const bool gate_up = it.gate_up;
+            const ExpMeta m = meta[it.e];
+            const bool shared = m.job < 0;
+            if (!gate_up && a.phase == 3) {  // h: every gate/up tile of this expert
+                int ok = 1;
+                if (lane == 0) {
+                    unsigned ns_ = 32;
+                    for (uint32_t i = 0;; ++i) {
+                        if (st_ld_acquire(a.done + it.e) >= (uint32_t)nA) break;
+                        if ((i & 7u) == 7u && (s_stop || st_now() > deadline)) {
+                            if (!s_stop) st_fail(a, kErrStreamDep, gi, it.e);
+                            s_stop = 1;
+                            ok = 0;
+                            break;
+                        }
+                        __nanosleep(ns_);
+                        if (ns_ < 512) ns_ <<= 1;
+                    }
+                    __threadfence();
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
+            const int K = gate_up ? a.d : a.F;
+            const int NCH = K >> 6, nsteps = (NCH + 3) >> 2;
+            const uint32_t cb = gate_up ? cbA : cbB, sb = gate_up ? sbA : sbB;
+            const uint8_t *stage = smem + (size_t)s * a.stage_bytes;
+            const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
+            const __half *act = gate_up ? a.act : a.hh_out;
+            bool released = false;
+            for (int t = 0; t < it.nt; ++t) {
+                const int tile = it.tile0 + t;
+                const uint8_t *s_codes = stage + (size_t)t * cb;
+                const uint8_t *s_scales = stage + (size_t)it.nt * cb + (size_t)t * sb;
+                for (int r0 = 0; r0 < m.nrows; r0 += 4 * NG) {
+                    // mma column n = g carries activation row r0 + 4*grp + g/2, its
+                    // hi (g even) or lo (g odd) fp16 part
+                    const __half *col[NG];
+                    bool colv[NG];
+                    int ngrp = 0;
+#pragma unroll
+                    for (int grp = 0; grp < NG; ++grp) {
+                        const int r = r0 + 4 * grp + (g >> 1);
+                        colv[grp] = r < m.nrows;
+                        col[grp] = act;
+                        if (r0 + 4 * grp < m.nrows) ngrp = grp + 1;
+                        if (colv[grp]) {
+                            int tr, p;
+                            if (shared) { tr = r; p = a.k; }
+                            else { const RowRef rf = rrs[m.row_off + r]; tr = rf.t; p = rf.p; }
+                            col[grp] = gate_up ? act + (size_t)tr * 2 * a.d + (g & 1) * a.d
+                                               : act + (size_t)(tr * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
+                        }
+                    }
+                    float acc[NG][4];
+#pragma unroll
+                    for (int grp = 0; grp < NG; ++grp)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) acc[grp][u] = 0.f;
+                    for (int st = 0; st < nsteps; ++st) {
+                        const int c = 4 * st + q;
+                        const bool cv = c < NCH;  // ragged K tail: this lane feeds zeros
+                        const int cc = cv ? c : 0;
+                        if constexpr (kMx) {
+                            const uint32_t sa = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rA * (K >> 5) + 2 * c) : 0u;
+                            const uint32_t sbv = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rB * (K >> 5) + 2 * c) : 0u;
+                            if (gate_up)
+                                step_mma_mx<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                       sa, sbv, cc, cv, col, colv, ngrp, acc);
+                            else
+                                step_mma_mx<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                      sa, sbv, cc, cv, col, colv, ngrp, acc);
+                        } else {
+                            const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
+                            const uint32_t sbv = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rB * (K >> 4) + 4 * c) : 0u;
+                            if (gate_up)
+                                step_mma<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                    sa, sbv, cc, cv, col, colv, ngrp, acc);
+                            else
+                                step_mma<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                   sa, sbv, cc, cv, col, colv, ngrp, acc);
+                        }
+                    }
+                    if (t == it.nt - 1 && r0 + 4 * NG >= m.nrows) {
+                        // the stage's last read by this warp: hand it back to the producer
+                        __syncwarp();
+                        if (lane == 0) st_mbar_arrive(&s_empty[s]);
+                        released = true;
+                    }
+                    // each lane's results: activation row r0 + 4*grp + q; tile rows rA (d0, d1), rB (d2, d3)
+#pragma unroll
+                    for (int grp = 0; grp < NG; ++grp) {
+                        const int r = r0 + 4 * grp + q;
+                        if (r >= m.nrows) continue;
+                        int tr, p;
+                        if (shared) { tr = r; p = a.k; }
+                        else { const RowRef rf = rrs[m.row_off + r]; tr = rf.t; p = rf.p; }
+                        const float v0 = acc[grp][0] + acc[grp][1];
+                        const float v1 = acc[grp][2] + acc[grp][3];
+                        const size_t sel = (size_t)tr * (a.k + 1) + p;
+                        if (gate_up) {
+                            const float gt = kMx ? v0 : m.ts[0] * v0, up = kMx ? v1 : m.ts[1] * v1;
+                            const float h = gt / (1.0f + expf(-gt)) * up;
+                            const int o = 8 * tile + g;
+                            const __half hi = __float2half_rn(h);
+                            const __half lo = __float2half_rn(h - __half2float(hi));
+                            a.hh_out[sel * 2 * a.F + o] = hi;
+                            a.hh_out[sel * 2 * a.F + a.F + o] = lo;
+                        } else {
+                            const int o = 16 * tile + g;
+                            const float sd = kMx ? 1.0f : m.ts[2];
+                            a.part_out[sel * a.d + o] = sd * v0;
+                            a.part_out[sel * a.d + o + 8] = sd * v1;
+                        }
+                    }
+                }
+                if (!gate_up && a.combine) {  // the tile's last expert: combine its rows
+                    __syncwarp();
+                    int last = 0;
+                    if (lane == 0) {
+                        __threadfence();
+                        last = atomicAdd(&a.tile_ticket[tile], 1u) == (unsigned)(nexp - 1);
+                    }
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    if (last) {
+                        __threadfence();
+                        if (a.combine == 1 || __ldcg(a.n_misses) == 0) {
+                            for (int i = lane; i < 16 * a.T; i += 32) {
+                                const int tr = i >> 4, o = 16 * tile + (i & 15);
+                                const float *pr = a.part_out + (size_t)tr * (a.k + 1) * a.d + o;
+                                float sum = 0.f;
+                                for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
+                                    if (a.ep_size == 1 || a.idx[tr * a.k + p] % a.ep_size == a.ep_rank)
+                                        sum = fmaf(a.gates[tr * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                                if (a.shared_part) sum += __ldcg(pr + (size_t)a.k * a.d);
+                                a.y[(size_t)tr * a.d + o] = sum;
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) a.tile_ticket[tile] = 0u;
+                    }
+                }
+            }
+            if (!released) {  // (an expert without rows: nothing read)
+                __syncwarp();
+                if (lane == 0) st_mbar_arrive(&s_empty[s]);
+            }
+            if (gate_up && a.phase == 3) {  // publish this item's h tiles
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(a.done + it.e, (unsigned)it.nt);
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (a.phase == 3) {  // the last CTA out resets the launch's gate/up counters
+        if (threadIdx.x == 0) {
+            __threadfence();
+            s_last = atomicAdd(a.exit_ticket, 1u) == gridDim.x - 1;
+        }
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            for (int e = threadIdx.x; e < nexp; e += blockDim.x) a.done[e] = 0u;
+            if (threadIdx.x == 0) *a.exit_ticket = 0u;
+        }
+    }
+    if (threadIdx.x == 0) span_mark(a.span, 1);
+}
+
+template <int NG, int FMT>
+cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) {
+    static bool configured = false;  // per instantiation: allow the large dynamic shared memory
+    if (!configured) {
+        const cudaError_t e = cudaFuncSetAttribute(expert_stream_kernel<NG, FMT>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 210 * 1024);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * (a.nc + 1));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, expert_stream_kernel<NG, FMT>, a);
+}
+
+}  // namespace
+
+cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
+    GemvArgs a = a_in;
+    const bool mx = a.lay.fmt == kFmtMxfp4;
+    if (!mx && a.lay.fmt != kFmtNvfp4) return cudaErrorInvalidValue;
+    if (a.phase < 1 || a.phase > 3 || max_exp < 1 || max_exp > kMaxSlots) return cudaErrorInvalidValue;
+    if (a.d % 64 || a.F % 64 || a.d < 64 || a.F < 64 || a.d / 64 > 4 * kMaxSteps || a.F / 64 > 4 * kMaxSteps)
+        return cudaErrorInvalidValue;
+    if (a.phase == 3 && (a.done == nullptr || a.exit_ticket == nullptr)) return cudaErrorInvalidValue;
+    // bulk copies start on 16-byte boundaries: record bases and section offsets
+    const uintptr_t al = reinterpret_cast<uintptr_t>(a.arena) | reinterpret_cast<uintptr_t>(a.shared_rec) |
+                         (uintptr_t)a.rec_bytes | (uintptr_t)a.lay.w13_codes | (uintptr_t)a.lay.w13_scales |
+                         (uintptr_t)a.lay.w2_codes | (uintptr_t)a.lay.w2_scales;
+    if (al & 15) return cudaErrorInvalidValue;
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
+    // stage = the larger tile (codes + scales), at least 16 KB; several
+    // consecutive tiles of one expert per item where they fit
+    const size_t tA = 8 * (size_t)a.d + (mx ? a.d / 2 : a.d), tB = 8 * (size_t)a.F + (mx ? a.F / 2 : a.F);
+    size_t sb = tA > tB ? tA : tB;
+    if (sb < 16 * 1024) sb = 16 * 1024;
+    sb = (sb + 127) & ~(size_t)127;
+    const int nA = a.F / 8, nB = a.d / 16;
+    // items: enough of them that every SM's consumers get a few
+    const int64_t want = 3 * (int64_t)sms;
+    auto per_item = [&](size_t tile_bytes, int tiles_per_exp, int phases_exp) {
+        int tp = (int)(sb / tile_bytes);
+        const int64_t tiles = (int64_t)tiles_per_exp * phases_exp;
+        while (tp > 1 && tiles / tp < want) --tp;
+        return tp < 1 ? 1 : tp;
+    };
+    a.tpa = per_item(tA, nA, max_exp);
+    a.tpb = per_item(tB, nB, max_exp);
+    const size_t meta = (size_t)max_exp * sizeof(ExpMeta);
+    const size_t rr = (((size_t)a.T * a.k * sizeof(RowRef)) + 15) & ~(size_t)15;
+    const size_t budget = 200 * 1024;
+    if (meta + rr + 2 * sb > budget) return cudaErrorInvalidValue;
+    int ns = (int)((budget - meta - rr) / sb);
+    if (ns > kStMaxStages) ns = kStMaxStages;
+    // stages per consumer warp: two (one loads while the other is computed)
+    // where six or more fit, else one; the stage count is a multiple of the
+    // consumer count, so a stage always serves the same warp and its phases are
+    // consumed in order (a parity wait can then not see an older phase)
+    int nc = ns >= 6 ? ns / 2 : ns;
+    if (nc > 4 && ns >= 6) nc = 4;
+    a.nc = nc;
+    a.ns = ns = (ns >= 6 ? 2 : 1) * nc;
+    a.stage_bytes = (uint32_t)sb;
+    a.meta_off = (uint32_t)(ns * sb);
+    a.rr_off = (uint32_t)(ns * sb + meta);
+    a.exp_cap = max_exp;
+    const size_t smem = ns * sb + meta + rr;
+    const int iA = (nA + a.tpa - 1) / a.tpa, iB = (nB + a.tpb - 1) / a.tpb;
+    const int64_t items = (int64_t)max_exp * (((a.phase & 1) ? iA : 0) + ((a.phase & 2) ? iB : 0));
+    const int grid = (int)(items < sms ? items : sms);
+    const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
+    if (mx) {
+        if (ng == 1) return launch_st<1, kFmtMxfp4>(a, grid, smem, s);
+        return launch_st<2, kFmtMxfp4>(a, grid, smem, s);
+    }
+    if (ng == 1) return launch_st<1, kFmtNvfp4>(a, grid, smem, s);
+    return launch_st<2, kFmtNvfp4>(a, grid, smem, s);
+}
+
+}  // namespace moe

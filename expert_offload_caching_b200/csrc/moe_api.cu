@@ -86,6 +86,7 @@ int max_jobs(const moe_dims *d, int T) {
 
 // Workspace carve-up (offsets from the caller's base).  Row buffers are sized
 // for the largest call (max_rows); the prefill buffers exist when max_rows > 32.
+constexpr int64_t kLkWords = 4 + 4 * (int64_t)kMaxSlots + 4;
 struct WsLayout {
     int64_t z, idx, gates, jobs, n_jobs, n_misses, ticket, ticket2, lk, rowrefs, xh, hh, part, cnt, fill,
         jobidx, h32, xq, xq_scales, xq_st, hq, hq_scales, hq_st, pairs, n_pairs, n_grouped, sg, hs, xstage, ystage,
@@ -111,7 +112,8 @@ WsLayout ws_layout(const moe_dims *d) {
     w.n_misses = take(4);
     w.ticket = take(4);
     w.ticket2 = take(4 * kMaxTiles);
-    w.lk = take(4 * (4 + 3 * (int64_t)kMaxSlots));  // layer kernel: queue[2], release, pad, done_a, flags
+    // layer kernel: queue[2], release, pad, done_a, flags; streaming kernel: done, exit (+3 pad)
+    w.lk = take(4 * (kLkWords));
     w.rowrefs = take(T * k * (int64_t)sizeof(RowRef));
     w.xh = take(Td * 2 * dd * 2);
     w.hh = take(Td * (k + 1) * 2 * F * 2);
@@ -176,6 +178,18 @@ struct moe_ctx {
     WsLayout wl;
     DecodeWs dws;
     cudaStream_t cs = nullptr, xs = nullptr;
+    // decode misses alternate between the caller's copy stream and one of the
+    // library's own (copy_streams = 2), so one copy's start-up overlaps the
+    // other's transfer; xs2 starts after xs's earlier work (ev_xs_tail) and xs
+    // waits for xs2 at the end of each call, so the caller's copy stream still
+    // covers every copy
+    cudaStream_t xs2 = nullptr;
+    cudaEvent_t ev_xs_tail = nullptr, ev_xs2_tail = nullptr;
+    int copy_streams = 1;
+    // decode expert kernels of the per-miss path: 1 = streaming (bulk-copy ring,
+    // a warp per tile; the hit experts' gate/up and down in one launch), 0 = the
+    // split-K kernel (expert_gemv.cu)
+    int gemv_kind = 1;
     // cache
     uint8_t *arena = nullptr;
     int64_t C = 0;
@@ -204,10 +218,12 @@ struct moe_ctx {
     std::vector<TimedLaunch> pending;
     // injection and limits
     int64_t inj_copy_fail_at = 0, inj_drop_publish = 0, inj_drop_flags = 0, inj_gemm_skip = 0;
-    // decode: the persistent layer kernel (one launch per layer, misses gated
-    // by flags the copy stream writes), when stream memory writes work here;
-    // else a launch per miss, gated by events
-    bool fused = false;
+    // decode: a launch for the hit experts and a gate/up and a down launch per
+    // miss, gated by copy events (the default; measured faster: a stream memory
+    // write between copies idles the copy engine longer than an event record),
+    // or the persistent layer kernel (one launch per layer, misses gated by
+    // flags the copy stream writes; where stream memory writes work: fused_ok)
+    bool fused = false, fused_ok = false;
     // expert parallelism: the routed experts e with e % ep_size == ep_rank; the
     // shared expert on rank 0; y is this rank's partial sum
     int32_t ep_rank = 0, ep_size = 1;
@@ -258,6 +274,28 @@ cudaError_t stream_write(cudaStream_t s, uint32_t *addr, uint32_t value) {
     return fn(reinterpret_cast<CUstream>(s), reinterpret_cast<CUdeviceptr>(addr), value, 0) == CUDA_SUCCESS
                ? cudaSuccess
                : cudaErrorNotSupported;
+}
+// The copy stream of a call's m-th miss (0-based): every other one on the
+// library's second copy stream when two are enabled; xs2's first copy of the
+// call is ordered after xs's work of earlier calls.
+cudaError_t miss_stream(moe_ctx *ctx, int m, bool *used2, cudaStream_t *out) {
+    *out = ctx->xs;
+    if (ctx->copy_streams < 2 || !(m & 1)) return cudaSuccess;
+    *out = ctx->xs2;
+    if (*used2) return cudaSuccess;
+    *used2 = true;
+    return cudaStreamWaitEvent(ctx->xs2, ctx->ev_xs_tail, 0);
+}
+// End of a call's copies: the caller's copy stream waits for xs2's, and marks
+// where the next call's xs2 copies may start.
+cudaError_t copy_tail(moe_ctx *ctx, bool used2) {
+    cudaError_t e = cudaSuccess;
+    if (used2) {
+        e = cudaEventRecord(ctx->ev_xs2_tail, ctx->xs2);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(ctx->xs, ctx->ev_xs2_tail, 0);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ctx->ev_xs_tail, ctx->xs);
+    return e;
 }
 
 cudaEvent_t pool_event(moe_ctx *ctx) {
@@ -373,6 +411,20 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
     g.idx = ctx->dws.idx;
     g.ep_rank = ctx->ep_rank;
     g.ep_size = ctx->ep_size;
+    return g;
+}
+
+// Arguments of a streaming-kernel launch (expert_stream.cu): phase 1 gate/up,
+// 2 down, 3 both (the hit experts); only_job >= 0: that miss alone.
+GemvArgs stream_args(moe_ctx *ctx, int layer, int T, int phase, int only_job, int combine) {
+    GemvArgs g = gemv_args(ctx, layer, T, phase == 2 ? kDown : kGateUp, only_job, combine);
+    g.act = ctx->dws.xh;
+    g.phase = phase;
+    g.shared_item = (only_job < 0 && shared_here(ctx) && !shared_separate(ctx)) ? 1 : 0;
+    g.shared_part = shared_here(ctx) ? 1 : 0;
+    g.done = ctx->dws.st_done;
+    g.exit_ticket = ctx->dws.st_exit;
+    g.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 5.0) * 1e9);
     return g;
 }
 
@@ -577,6 +629,8 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         if (ih >= 0) ctx->pending[ih].bytes = (n_hit_jobs + in_launch_shared) * rec + (double)T * D.d * 2;
         // misses: the gate/up prefix, its flag, the W2 half, its flag
         const int64_t split = ctx->lay.w2_codes;
+        int mo = 0;
+        bool used2 = false;
         for (int j = 0; j < nev; ++j) {
             if (ev[j].flags & 1) continue;
             if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
@@ -588,32 +642,47 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
             uint8_t *dst = ctx->arena + (int64_t)ev[j].slot * ctx->lay.bytes;
             const uint8_t *src = ctx->pool + rec_idx * ctx->lay.bytes;
             const bool flags = !(ctx->inj_drop_flags > 0 && (--ctx->inj_drop_flags, true));
-            CK(cudaMemcpyAsync(dst, src, split, cudaMemcpyHostToDevice, ctx->xs));
-            if (flags) CK(stream_write(ctx->xs, ctx->dws.lk_flags + 2 * j, seq));
-            CK(cudaMemcpyAsync(dst + split, src + split, ctx->lay.bytes - split, cudaMemcpyHostToDevice, ctx->xs));
-            if (flags) CK(stream_write(ctx->xs, ctx->dws.lk_flags + 2 * j + 1, seq));
+            cudaStream_t s;
+            CK(miss_stream(ctx, mo++, &used2, &s));
+            CK(cudaMemcpyAsync(dst, src, split, cudaMemcpyHostToDevice, s));
+            if (flags) CK(stream_write(s, ctx->dws.lk_flags + 2 * j, seq));
+            CK(cudaMemcpyAsync(dst + split, src + split, ctx->lay.bytes - split, cudaMemcpyHostToDevice, s));
+            if (flags) CK(stream_write(s, ctx->dws.lk_flags + 2 * j + 1, seq));
             else rel.armed = false;  // injected: the kernel's own wait limit must end it
             ctx->stats.h2d_copies += 1;
             ctx->stats.h2d_bytes += ctx->lay.bytes;
         }
+        if (mo > 0) CK(copy_tail(ctx, used2));
         rel.armed = false;
         return finish_decode(ctx, layer, T, nev, trace);
     }
 
     // hit experts and the shared expert, before the miss list is known
     const int grid_y = nj + in_launch_shared;
-    TimedLaunch tg, td;
-    time_begin(ctx, tg, MOE_K_GATEUP);
-    GemvArgs hg = gemv_args(ctx, layer, T, kGateUp, -1);
-    hg.span = time_span(ctx, tg);
-    CK(launch_gemv(hg, grid_y, ctx->cs));
-    const long ig = time_end(ctx, tg, 0);
-    time_begin(ctx, td, MOE_K_DOWN);
-    GemvArgs hd = gemv_args(ctx, layer, T, kDown, -1, 2);  // combines when nothing missed
-    hd.y = y;
-    hd.span = time_span(ctx, td);
-    CK(launch_gemv(hd, grid_y, ctx->cs));
-    const long id = time_end(ctx, td, 0);
+    const bool stream = ctx->gemv_kind == 1;
+    long ig = -1, id = -1, ih = -1;
+    if (stream) {  // one launch: their gate/up tiles, then their down tiles (+ combine if nothing missed)
+        TimedLaunch th;
+        time_begin(ctx, th, MOE_K_LAYER_HITS);
+        GemvArgs ha = stream_args(ctx, layer, T, 3, -1, 2);
+        ha.y = y;
+        ha.span = time_span(ctx, th);
+        CK(launch_stream(ha, grid_y, ctx->cs));
+        ih = time_end(ctx, th, 0);
+    } else {
+        TimedLaunch tg, td;
+        time_begin(ctx, tg, MOE_K_GATEUP);
+        GemvArgs hg = gemv_args(ctx, layer, T, kGateUp, -1);
+        hg.span = time_span(ctx, tg);
+        CK(launch_gemv(hg, grid_y, ctx->cs));
+        ig = time_end(ctx, tg, 0);
+        time_begin(ctx, td, MOE_K_DOWN);
+        GemvArgs hd = gemv_args(ctx, layer, T, kDown, -1, 2);  // combines when nothing missed
+        hd.y = y;
+        hd.span = time_span(ctx, td);
+        CK(launch_gemv(hd, grid_y, ctx->cs));
+        id = time_end(ctx, td, 0);
+    }
 
     // bounded host wait for the device's miss list
     {
@@ -628,16 +697,19 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         n_hit_jobs += ev[j].flags & 1;
         if (!(ev[j].flags & 1)) last_miss = j;
     }
-    if (ig >= 0 && id >= 0) {  // algorithmic bytes of the two hit launches, now known
+    {  // algorithmic bytes of the hit launches, now known
         const int nexp = n_hit_jobs + in_launch_shared;
-        ctx->pending[ig].bytes = nexp * w13_bytes(ctx) + (double)T * D.d * 2;
-        ctx->pending[id].bytes = nexp * w2_bytes(ctx) + (double)T * D.F * 4;
+        if (ig >= 0) ctx->pending[ig].bytes = nexp * w13_bytes(ctx) + (double)T * D.d * 2;
+        if (id >= 0) ctx->pending[id].bytes = nexp * w2_bytes(ctx) + (double)T * D.F * 4;
+        if (ih >= 0) ctx->pending[ih].bytes = nexp * (w13_bytes(ctx) + w2_bytes(ctx)) + (double)T * D.d * 2;
     }
 
     // misses: each record in two copies on the copy stream -- the gate/up half
     // (tensor scales + W13, a prefix of the record) and the down half -- with an
     // event after each, so a miss's gate/up runs while its down half streams in
     const int64_t split = ctx->lay.w2_codes;
+    int mo = 0;
+    bool used2 = false;
     for (int j = 0; j < nev; ++j) {
         if (ev[j].flags & 1) continue;
         if (ctx->inj_copy_fail_at > 0 && --ctx->inj_copy_fail_at == 0) {
@@ -648,29 +720,32 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         const int64_t rec_idx = ((int64_t)layer * D.E + ev[j].expert) % ctx->P;
         uint8_t *dst = ctx->arena + (int64_t)ev[j].slot * ctx->lay.bytes;
         const uint8_t *src = ctx->pool + rec_idx * ctx->lay.bytes;
-        CK(cudaMemcpyAsync(dst, src, split, cudaMemcpyHostToDevice, ctx->xs));
-        CK(cudaEventRecord(ctx->miss_ev[2 * j], ctx->xs));
-        CK(cudaMemcpyAsync(dst + split, src + split, ctx->lay.bytes - split, cudaMemcpyHostToDevice,
-                           ctx->xs));
-        CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], ctx->xs));
+        cudaStream_t s;
+        CK(miss_stream(ctx, mo++, &used2, &s));
+        CK(cudaMemcpyAsync(dst, src, split, cudaMemcpyHostToDevice, s));
+        CK(cudaEventRecord(ctx->miss_ev[2 * j], s));
+        CK(cudaMemcpyAsync(dst + split, src + split, ctx->lay.bytes - split, cudaMemcpyHostToDevice, s));
+        CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], s));
         ctx->stats.h2d_copies += 1;
         ctx->stats.h2d_bytes += ctx->lay.bytes;
     }
+    if (mo > 0) CK(copy_tail(ctx, used2));
     for (int j = 0; j < nev; ++j) {
         if (ev[j].flags & 1) continue;
         CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j], 0));
         TimedLaunch mg, md;
         time_begin(ctx, mg, MOE_K_GATEUP);
-        GemvArgs mg_args = gemv_args(ctx, layer, T, kGateUp, j);
+        GemvArgs mg_args = stream ? stream_args(ctx, layer, T, 1, j, 0) : gemv_args(ctx, layer, T, kGateUp, j);
         mg_args.span = time_span(ctx, mg);
-        CK(launch_gemv(mg_args, 1, ctx->cs));
+        CK(stream ? launch_stream(mg_args, 1, ctx->cs) : launch_gemv(mg_args, 1, ctx->cs));
         time_end(ctx, mg, w13_bytes(ctx) + (double)T * D.d * 2);
         CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j + 1], 0));
         time_begin(ctx, md, MOE_K_DOWN);
-        GemvArgs md_args = gemv_args(ctx, layer, T, kDown, j, j == last_miss ? 1 : 0);
+        const int comb = j == last_miss ? 1 : 0;
+        GemvArgs md_args = stream ? stream_args(ctx, layer, T, 2, j, comb) : gemv_args(ctx, layer, T, kDown, j, comb);
         md_args.y = y;
         md_args.span = time_span(ctx, md);
-        CK(launch_gemv(md_args, 1, ctx->cs));
+        CK(stream ? launch_stream(md_args, 1, ctx->cs) : launch_gemv(md_args, 1, ctx->cs));
         time_end(ctx, md, w2_bytes(ctx) + (double)T * D.F * 4);
     }
 
@@ -799,6 +874,7 @@ moe_status forward_prefill(moe_ctx *ctx, int32_t layer, const void *x, int32_t T
         CK(cudaEventRecord(ctx->ev_pf[layer + 1], ctx->xs));
         ctx->pf_pending[layer + 1] = 1;
     }
+    if (nrm + npm > 0) CK(copy_tail(ctx, false));
 
     // experts: grouped tensor-core GEMMs -- gate/up (+SwiGLU, fp32 h), h
     // quantized per row, down -- then the gate-weighted combine
@@ -964,6 +1040,8 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     ctx->dws.lk_release = ctx->dws.lk_queue + 2;
     ctx->dws.lk_done_a = ctx->dws.lk_queue + 4;
     ctx->dws.lk_flags = ctx->dws.lk_done_a + kMaxSlots;
+    ctx->dws.st_done = ctx->dws.lk_flags + 2 * kMaxSlots;
+    ctx->dws.st_exit = ctx->dws.st_done + kMaxSlots;
     ctx->dws.rowrefs = reinterpret_cast<RowRef *>(w + L.rowrefs);
     ctx->dws.xh = reinterpret_cast<__half *>(w + L.xh);
     ctx->dws.hh = reinterpret_cast<__half *>(w + L.hh);
@@ -1021,6 +1099,10 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
         }
     }
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_routed, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_xs_tail, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ctx->ev_xs2_tail, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&ctx->xs2, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventRecord(ctx->ev_xs_tail, ctx->xs);
     if (e == cudaSuccess) {
         ctx->ev_pf.resize(dims->L, nullptr);
         ctx->pf_pending.assign(dims->L, 0);
@@ -1031,13 +1113,13 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     }
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket, 0, 4, ctx->cs);
     if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.ticket2, 0, 4 * kMaxTiles, ctx->cs);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.lk_queue, 0, 4 * (4 + 3 * (size_t)kMaxSlots), ctx->cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ctx->dws.lk_queue, 0, 4 * (size_t)kLkWords, ctx->cs);
     if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->cs);
     // the persistent layer kernel needs stream memory writes on the copy stream:
     // one trial write (of the value already there) decides
     if (e == cudaSuccess) {
-        ctx->fused = stream_write(ctx->xs, ctx->dws.lk_release, 0u) == cudaSuccess &&
-                     cudaStreamSynchronize(ctx->xs) == cudaSuccess;
+        ctx->fused_ok = stream_write(ctx->xs, ctx->dws.lk_release, 0u) == cudaSuccess &&
+                        cudaStreamSynchronize(ctx->xs) == cudaSuccess;
         cudaGetLastError();
     }
     if (e != cudaSuccess) {
@@ -1094,6 +1176,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         // configured = false, so forward calls refuse to run on a half-reset table)
         ctx->configured = false;
         // finish outstanding work of the old state first
+        CK(cudaStreamSynchronize(ctx->xs2));
         CK(cudaStreamSynchronize(ctx->xs));
         CK(cudaStreamSynchronize(ctx->cs));
         if (stat) {
@@ -1107,6 +1190,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
         // they are compared with sequence numbers that only grow)
         CK(cudaMemsetAsync(ctx->dws.lk_queue, 0, 8, ctx->cs));
         CK(cudaMemsetAsync(ctx->dws.lk_done_a, 0, 4 * (size_t)kMaxSlots, ctx->cs));
+        CK(cudaMemsetAsync(ctx->dws.st_done, 0, 4 * ((size_t)kMaxSlots + 1), ctx->cs));
         for (auto &t : ctx->pending) {  // timing records of the old state
             ctx->ev_pool.push_back(t.a);
             ctx->ev_pool.push_back(t.b);
@@ -1147,6 +1231,7 @@ moe_status cache_configure(moe_ctx *ctx, int64_t num_slots, void *slot_arena, si
             CK(flush());
             CK(cudaEventRecord(ctx->ev_routed, ctx->xs));
             CK(cudaStreamWaitEvent(ctx->cs, ctx->ev_routed, 0));
+            CK(copy_tail(ctx, false));
         }
     }
     ctx->configured = true;
@@ -1246,7 +1331,10 @@ moe_status moe_set_timing(moe_ctx *ctx, int32_t enable) {
 
 moe_status moe_set_expert_shard(moe_ctx *ctx, int32_t rank, int32_t size) {
     if (!ctx || size < 1 || rank < 0 || rank >= size || size > ctx->dims.E) return MOE_ERR_ARG;
-    if (size > 1 && (!ctx->fused || (ctx->flags & MOE_CACHE_STATIC_SPLIT))) return MOE_ERR_UNSUPPORTED;
+    // (a shard may own none of a layer's experts: the layer kernel and the
+    // streaming kernels write its zero / shared-only partial output)
+    if (size > 1 && ((!ctx->fused && ctx->gemv_kind != 1) || (ctx->flags & MOE_CACHE_STATIC_SPLIT)))
+        return MOE_ERR_UNSUPPORTED;
     if (rank != ctx->ep_rank || size != ctx->ep_size) ctx->configured = false;  // a new cache: reset first
     ctx->ep_rank = rank;
     ctx->ep_size = size;
@@ -1270,10 +1358,18 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
     else if (what == 1) ctx->inj_copy_fail_at = n;
     else if (what == 2) ctx->inj_drop_publish = n;
     else if (what == 3) {  // decode path: 0 = a launch per miss, 1 = the layer kernel
-        if (n == 0 && ctx->ep_size > 1) return MOE_ERR_UNSUPPORTED;
-        if (n == 1 && stream_write(ctx->xs, ctx->dws.lk_release, 0u) != cudaSuccess) return MOE_ERR_UNSUPPORTED;
+        if (n == 0 && ctx->ep_size > 1 && ctx->gemv_kind != 1) return MOE_ERR_UNSUPPORTED;
+        if (n == 1 && !ctx->fused_ok) return MOE_ERR_UNSUPPORTED;
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;
+    else if (what == 7) {  // per-miss path expert kernels: 1 streaming, 0 split-K
+        if (n < 0 || n > 1) return MOE_ERR_ARG;
+        if (n == 0 && ctx->ep_size > 1 && !ctx->fused) return MOE_ERR_UNSUPPORTED;
+        ctx->gemv_kind = (int)n;
+    } else if (what == 6) {  // decode misses on 1 or 2 copy streams
+        if (n < 1 || n > 2) return MOE_ERR_ARG;
+        ctx->copy_streams = (int)n;
+    }
     else if (what == 5) ctx->inj_gemm_skip = n;
     else return MOE_ERR_ARG;
     return MOE_OK;
@@ -1409,6 +1505,12 @@ void moe_layer_destroy(moe_ctx *ctx) {
     if (!ctx) return;
     if (ctx->cs) cudaStreamSynchronize(ctx->cs);
     if (ctx->xs) cudaStreamSynchronize(ctx->xs);
+    if (ctx->xs2) {
+        cudaStreamSynchronize(ctx->xs2);
+        cudaStreamDestroy(ctx->xs2);
+    }
+    if (ctx->ev_xs_tail) cudaEventDestroy(ctx->ev_xs_tail);
+    if (ctx->ev_xs2_tail) cudaEventDestroy(ctx->ev_xs2_tail);
     for (auto &t : ctx->pending) {
         if (t.a) cudaEventDestroy(t.a);
         if (t.b) cudaEventDestroy(t.b);

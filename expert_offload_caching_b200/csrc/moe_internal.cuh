@@ -92,6 +92,9 @@ struct DecodeWs {
     uint32_t *lk_release;  // [1]
     uint32_t *lk_done_a;   // [kMaxSlots]
     uint32_t *lk_flags;    // [2 * kMaxSlots]
+    // streaming expert kernel, phase 3: gate/up tiles done per launch expert; CTAs out
+    uint32_t *st_done;     // [kMaxSlots]
+    uint32_t *st_exit;     // [1]
     // prefill only (T > 32)
     int32_t *cnt;        // [E] rows per expert
     int32_t *fill;       // [E] scatter cursors
@@ -155,6 +158,20 @@ struct GemvArgs {
     unsigned long long *span;  // launch timing slot (see span_mark), or null
     const int32_t *idx;     // [T][k] selected experts: the combine takes the owned ones only
     int ep_rank, ep_size;
+    // streaming kernel (expert_stream.cu): phase 1 = gate/up, 2 = down, 3 =
+    // gate/up then down of the same experts in one launch (down items wait on
+    // done[expert] == F / 8 gate/up tiles); the shared expert is an expert of the
+    // launch when shared_item; y gets the shared partial when shared_part
+    int phase = 0;
+    int shared_item = 0, shared_part = 0;
+    uint32_t *done = nullptr;        // [kMaxSlots] phase 3: gate/up tiles completed per launch expert
+    uint32_t *exit_ticket = nullptr; // phase 3: CTAs finished (the last one resets done)
+    unsigned long long wait_ns = 0;  // every wait of the kernel ends by then (from its start)
+    // set by launch_stream
+    int tpa = 0, tpb = 0;            // weight tiles per work item (gate/up, down)
+    int ns = 0, nc = 0;              // shared-memory stages, consumer warps
+    uint32_t stage_bytes = 0, meta_off = 0, rr_off = 0;
+    int exp_cap = 0;                 // experts the metadata area holds
 };
 
 // Persistent decode layer kernel (all expert GEMVs of one layer, misses as
@@ -242,6 +259,9 @@ __device__ __forceinline__ void span_mark(unsigned long long *slot, int which) {
 // launchers (one per .cu)
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s);
 // slots: job slots of the launch (max jobs + shared expert), 1 with only_job
+// Streaming expert GEMVs (expert_stream.cu): max_exp = the launch's largest
+// possible expert count (hit jobs + shared, or 1 with only_job).
+cudaError_t launch_stream(const GemvArgs &a, int max_exp, cudaStream_t s);
 cudaError_t launch_gemv(const GemvArgs &a, int slots, cudaStream_t s);
 cudaError_t launch_expert_layer(const LayerArgs &a, cudaStream_t s);
 // BF16 shared expert of a decode call (T <= 32 rows; x as DecodeWs::xh):

@@ -126,11 +126,13 @@ typedef struct {
 /* Cumulative counters since the last MOE_CACHE_RESET.
  * lookups/hits/misses count routed lookups (each distinct (layer, expert) of a
  * batch once); prefetch_* count next-layer prefetch entries separately. */
-/* Kernel classes of the timing counters.  MOE_K_LAYER: the decode layer
- * kernel (every expert GEMV of a layer in one launch, misses as their copies
- * land); MOE_K_LAYER_HITS: the same launches up to the end of their last
- * resident-expert item (hit and shared experts: the part bounded by HBM, not
- * by the copies). */
+/* Kernel classes of the timing counters.  MOE_K_GATEUP / MOE_K_DOWN: the
+ * per-miss launches (and, with the split-K kernels, the hit launches);
+ * MOE_K_LAYER: the decode layer kernel (every expert GEMV of a layer in one
+ * launch, misses as their copies land); MOE_K_LAYER_HITS: the hit and shared
+ * experts' gate/up and down -- the default path's hit launch, or the layer
+ * kernel up to the end of its last resident-expert item (the part bounded by
+ * HBM, not by the copies). */
 enum { MOE_K_ROUTE = 0, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE, MOE_K_PREFILL_ROUTE,
        MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_LAYER, MOE_K_LAYER_HITS, MOE_K_COUNT };
 typedef struct {
@@ -315,8 +317,8 @@ MOE_API moe_status moe_set_timing(moe_ctx *ctx, int32_t enable);
  * until then).  Prefill chunks likewise: the lookup and prefetch batches, the
  * grouped GEMMs and the combine cover this rank's experts only.  MOE_ERR_ARG
  * unless 0 <= rank < size <= E; MOE_ERR_UNSUPPORTED for size > 1 with the
- * static split or without the decode layer kernel (stream memory writes
- * unavailable). */
+ * static split, or with the split-K per-miss kernels selected (debug option
+ * what = 7, n = 0) and no decode layer kernel. */
 MOE_API moe_status moe_set_expert_shard(moe_ctx *ctx, int32_t rank, int32_t size);
 
 /* Longest wait, in seconds (default 60): the host's wait for the device miss
@@ -336,9 +338,17 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * issue its first stage's tensor copies, so its bounded mbarrier waits run out
  * (the CTA records the check, frees its tensor memory and returns; the next
  * call reports MOE_ERR_CUDA); what = 3:
- * decode runs the layer kernel (n = 1; the default where stream memory writes
- * work, MOE_ERR_UNSUPPORTED elsewhere) or a gate/up and a down launch per miss,
- * gated by copy events (n = 0); what = 0 clears 1, 2, 4 and 5. */
+ * decode runs the persistent layer kernel (n = 1; MOE_ERR_UNSUPPORTED where
+ * stream memory writes do not work) or, the default, a launch for the hit
+ * experts and a gate/up and a down launch per miss, gated by copy events
+ * (n = 0); what = 6: decode misses go on n copy
+ * streams (1: the caller's copy stream; 2: every other miss on a second copy
+ * stream the library owns, so that one copy's start-up overlaps another's
+ * transfer; the caller's copy stream still waits for it at the end of each
+ * call); what = 7: the per-miss path's expert kernels are the streaming
+ * kernels (n = 1, the default: bulk-copied tiles, a warp per tile, the hit
+ * experts' gate/up and down in one launch) or the split-K kernels (n = 0);
+ * what = 0 clears 1, 2, 4 and 5. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Hybrid split: m missing experts, PCIe bandwidth B_P, host expert-processing

@@ -337,17 +337,47 @@ def test_forward_rejects_unaligned_activations_before_launching():
     st.close()
 
 
-def test_per_miss_launch_path_matches_the_oracle():
-    """The decode path without the layer kernel (a gate/up and a down launch per
-    miss, gated by copy events; what the library runs where stream memory writes
-    are unavailable): same trace, table, slots and outputs."""
+def test_layer_kernel_path_matches_the_oracle():
+    """The persistent layer kernel (one launch per layer, misses gated by copy
+    flags) instead of the default launches: same trace, table, slots and
+    outputs; then back to the default on the same cache."""
     pb = DecodeProblem(MID, T=12)
     st = pb.stack()
-    abi.moe_debug_inject(st.ctx, 3, 0)
+    abi.moe_debug_inject(st.ctx, 3, 1)
     run = pb.run(stack=st, routing=True)
     assert _check_run(pb, run) < 1e-5
     pb.check_slots(st, run.table[1])
-    abi.moe_debug_inject(st.ctx, 3, 1)  # back to the layer kernel on the same cache
+    abi.moe_debug_inject(st.ctx, 3, 0)
+    st.close()
+
+
+@pytest.mark.parametrize("T", [1, 5])
+def test_split_k_per_miss_kernels_match_the_oracle(T):
+    """The per-miss path with the split-K expert kernels (expert_gemv.cu)
+    instead of the streaming ones: same trace, table, slots and outputs."""
+    pb = DecodeProblem(MID, T=12, streams=T)
+    st = pb.stack()
+    abi.moe_debug_inject(st.ctx, 7, 0)
+    run = pb.run(stack=st, routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(st, run.table[1])
+    st.close()
+
+
+@pytest.mark.parametrize("path", [1, 0], ids=["layer-kernel", "per-miss"])
+def test_two_copy_streams_match_the_oracle(path):
+    """Misses alternating between the caller's copy stream and the library's
+    second one, on both decode paths: same trace, table, slots and outputs.
+    Several misses per call (12 rows, cold cache), so both streams carry copies
+    in the same call; the cache then persists across calls."""
+    pb = DecodeProblem(MID, T=12)
+    st = pb.stack()
+    abi.moe_debug_inject(st.ctx, 3, path)
+    abi.moe_debug_inject(st.ctx, 6, 2)
+    run = pb.run(stack=st, routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(st, run.table[1])
+    assert run.stats.misses >= 2 * pb.T // 3  # the calls held several misses each
     st.close()
 
 
@@ -359,6 +389,7 @@ def test_layer_kernel_flag_wait_runs_out_then_reset_recovers():
     import time
     pb = DecodeProblem(synth.TINY, T=8)
     st = pb.stack()
+    abi.moe_debug_inject(st.ctx, 3, 1)  # the layer kernel
     abi.moe_set_wait_limit(st.ctx, 0.3)
     abi.moe_debug_inject(st.ctx, 4, 1)  # the next miss: copies issued, flags not written
     x = torch.from_numpy(pb.x[:, 0]).cuda()

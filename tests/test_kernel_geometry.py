@@ -284,3 +284,113 @@ def test_layer_kernel_ring_fits_and_keeps_two_ctas_per_sm_where_it_can(shape, mx
         assert buf % 16 == 0  # every stage starts on a cp.async boundary
         if S == 2:
             assert smem + 6 * 1024 <= 227 * 1024  # one CTA fits with room for the static part
+
+
+# ------------------------------------------------ streaming expert kernel --
+def _stream_launch(d, F, T, k, max_exp, mx, sms=148):
+    """launch_stream's sizing, restated: stage bytes, tiles per item (gate/up,
+    down), stages, consumer warps, metadata and row-ref offsets, grid."""
+    tA = 8 * d + (d // 2 if mx else d)
+    tB = 8 * F + (F // 2 if mx else F)
+    sb = max(tA, tB, 16 * 1024)
+    sb = (sb + 127) & ~127
+    nA, nB = F // 8, d // 16
+    want = 3 * sms
+
+    def per_item(tile_bytes, tiles_per_exp):
+        tp = sb // tile_bytes
+        tiles = tiles_per_exp * max_exp
+        while tp > 1 and tiles // tp < want:
+            tp -= 1
+        return max(tp, 1)
+
+    tpa, tpb = per_item(tA, nA), per_item(tB, nB)
+    meta = max_exp * 32
+    rr = (T * k * 4 + 15) & ~15
+    budget = 200 * 1024
+    assert meta + rr + 2 * sb <= budget
+    ns = min((budget - meta - rr) // sb, 8)
+    nc = ns // 2 if ns >= 6 else ns
+    if nc > 4 and ns >= 6:
+        nc = 4
+    ns = (2 if ns >= 6 else 1) * nc
+    return dict(sb=sb, tpa=tpa, tpb=tpb, ns=ns, nc=nc, meta_off=ns * sb, rr_off=ns * sb + meta,
+                smem=ns * sb + meta + rr, nA=nA, nB=nB, cbA=8 * d, sbA=d // 2 if mx else d,
+                cbB=8 * F, sbB=F // 2 if mx else F)
+
+
+def _stream_items(L, nexp, phase):
+    """st_item over a launch: (expert, gate_up, tile0, nt) in global item order."""
+    iA = -(-L["nA"] // L["tpa"])
+    iB = -(-L["nB"] // L["tpb"])
+    total = nexp * ((iA if phase & 1 else 0) + (iB if phase & 2 else 0))
+    gA = nexp * iA if phase & 1 else 0
+    out = []
+    for g in range(total):
+        if g < gA:
+            e, j = divmod(g, iA)
+            t0 = j * L["tpa"]
+            out.append((e, 1, t0, min(L["tpa"], L["nA"] - t0)))
+        else:
+            e, j = divmod(g - gA, iB)
+            t0 = j * L["tpb"]
+            out.append((e, 0, t0, min(L["tpb"], L["nB"] - t0)))
+    return out
+
+
+@pytest.mark.parametrize("mx", [False, True], ids=["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: s.name)
+def test_stream_items_fit_their_stage_and_stay_in_the_record(shape, mx):
+    fmt = abi.MOE_FMT_MXFP4 if mx else abi.MOE_FMT_NVFP4
+    dims = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, shape.shared, weight_format=fmt)
+    off = abi.moe_record_layout(dims)  # w13 codes, w13 scales, w2 codes, w2 scales, tensor scales, bytes
+    for T in (1, 4, 16, 32):
+        max_exp = min(T * shape.k, shape.E) + 1
+        L = _stream_launch(shape.d, shape.F, T, shape.k, max_exp, mx)
+        assert 2 <= L["ns"] <= 8 and 2 <= L["nc"] <= 7
+        # each stage serves one consumer warp: the uses of a stage are waited on in order
+        assert L["ns"] % L["nc"] == 0
+        for l in range(64):
+            assert (l % L["ns"]) % L["nc"] == l % L["nc"]
+        assert L["smem"] <= 200 * 1024 and L["meta_off"] % 128 == 0 and L["rr_off"] % 8 == 0
+        for phase in (1, 2, 3):
+            nexp = min(max_exp, 3)
+            items = _stream_items(L, nexp, phase)
+            seen = set()
+            first_down = None
+            for n, (e, gu, t0, nt) in enumerate(items):
+                assert nt >= 1
+                cb, sb = (L["cbA"], L["sbA"]) if gu else (L["cbB"], L["sbB"])
+                codes0, scales0, end = (off[0], off[1], off[2]) if gu else (off[2], off[3], off[5])
+                # the stage: codes of nt tiles, then their scales
+                assert nt * (cb + sb) <= L["sb"]
+                assert (nt * cb) % 16 == 0 and (nt * sb) % 16 == 0
+                # the two bulk copies: 16-byte aligned, inside their record section
+                c0, s0 = codes0 + t0 * cb, scales0 + t0 * sb
+                assert c0 % 16 == 0 and s0 % 16 == 0
+                assert c0 + nt * cb <= scales0 and s0 + nt * sb <= end
+                for t in range(t0, t0 + nt):
+                    assert (e, gu, t) not in seen
+                    seen.add((e, gu, t))
+                if not gu and first_down is None:
+                    first_down = n
+                if gu:  # gate/up items precede every down item (phase 3's dependency order)
+                    assert first_down is None
+            want = set()
+            for e in range(nexp):
+                if phase & 1:
+                    want |= {(e, 1, t) for t in range(L["nA"])}
+                if phase & 2:
+                    want |= {(e, 0, t) for t in range(L["nB"])}
+            assert seen == want
+
+
+def test_stream_k_step_reads_stay_inside_the_tile():
+    """The K-step's shared-memory reads (rows rA/rB <= 15, chunk c < K/64, 32 code
+    bytes and 4 (NVFP4) or 2 (MXFP4) scale bytes per row and chunk) end at the
+    tile's code and scale sizes exactly."""
+    for K in (256, 320, 768, 960, 2048, 2880, 4096):
+        nch = K // 64
+        assert 15 * (K // 2) + 32 * (nch - 1) + 32 == 8 * K
+        assert 15 * (K // 16) + 4 * (nch - 1) + 4 == K
+        assert 15 * (K // 32) + 2 * (nch - 1) + 2 == K // 2
