@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             const uint64_t pol = evict_first_policy();
-            int issued = 0;
+            int issued = 0, skipped = -1;
             for (int l = 0; l < n_my; ++l) {
                 const int s = l % NS, n = l / NS;
                 if (n > 0 && !st_mbar_wait(&s_empty[s], (n - 1) & 1, deadline, &s_stop)) {
@@ -267,16 +267,20 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
                 const uint8_t *codes = rec + (it.gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)it.tile0 * cb;
                 const uint8_t *scales = rec + (it.gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)it.tile0 * sb;
                 uint8_t *dst = smem + (size_t)s * a.stage_bytes;
+                issued = l + 1;
+                if (a.inj_skip && blockIdx.x == 0 && l == 0) {  // test injection: this stage never fills
+                    skipped = 0;
+                    continue;
+                }
                 st_mbar_expect(&s_full[s], (uint32_t)it.nt * (cb + sb));
                 st_bulk_g2s(dst, codes, (uint32_t)it.nt * cb, &s_full[s], pol);
                 st_bulk_g2s(dst + (size_t)it.nt * cb, scales, (uint32_t)it.nt * sb, &s_full[s], pol);
-                issued = l + 1;
             }
             // no copy outlives the CTA: the last item issued into each stage has landed
             const unsigned long long drain = st_now() + 1000000000ull;
             volatile int never = 0;
             for (int l = issued > NS ? issued - NS : 0; l < issued; ++l)
-                st_mbar_wait(&s_full[l % NS], (l / NS) & 1, drain, &never);
+                if (l != skipped) st_mbar_wait(&s_full[l % NS], (l / NS) & 1, drain, &never);
         }
     } else if (warp <= C) {
         // ---------------------------------------------------------- consumers

@@ -217,7 +217,7 @@ struct moe_ctx {
     std::vector<cudaEvent_t> ev_pool;
     std::vector<TimedLaunch> pending;
     // injection and limits
-    int64_t inj_copy_fail_at = 0, inj_drop_publish = 0, inj_drop_flags = 0, inj_gemm_skip = 0;
+    int64_t inj_copy_fail_at = 0, inj_drop_publish = 0, inj_drop_flags = 0, inj_gemm_skip = 0, inj_stream_skip = 0;
     // decode: a launch for the hit experts and a gate/up and a down launch per
     // miss, gated by copy events (the default; measured faster: a stream memory
     // write between copies idles the copy engine longer than an event record),
@@ -425,6 +425,10 @@ GemvArgs stream_args(moe_ctx *ctx, int layer, int T, int phase, int only_job, in
     g.done = ctx->dws.st_done;
     g.exit_ticket = ctx->dws.st_exit;
     g.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 5.0) * 1e9);
+    if (ctx->inj_stream_skip > 0) {
+        g.inj_skip = 1;
+        --ctx->inj_stream_skip;
+    }
     return g;
 }
 
@@ -1354,6 +1358,7 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
         ctx->inj_drop_publish = 0;
         ctx->inj_drop_flags = 0;
         ctx->inj_gemm_skip = 0;
+        ctx->inj_stream_skip = 0;
     }
     else if (what == 1) ctx->inj_copy_fail_at = n;
     else if (what == 2) ctx->inj_drop_publish = n;
@@ -1362,6 +1367,7 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
         if (n == 1 && !ctx->fused_ok) return MOE_ERR_UNSUPPORTED;
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;
+    else if (what == 8) ctx->inj_stream_skip = n;
     else if (what == 7) {  // per-miss path expert kernels: 1 streaming, 0 split-K
         if (n < 0 || n > 1) return MOE_ERR_ARG;
         if (n == 0 && ctx->ep_size > 1 && !ctx->fused) return MOE_ERR_UNSUPPORTED;

@@ -172,6 +172,7 @@ struct GemvArgs {
     int ns = 0, nc = 0;              // shared-memory stages, consumer warps
     uint32_t stage_bytes = 0, meta_off = 0, rr_off = 0;
     int exp_cap = 0;                 // experts the metadata area holds
+    int inj_skip = 0;                // test injection: CTA 0 issues no copies for its first item
 };
 
 // Persistent decode layer kernel (all expert GEMVs of one layer, misses as

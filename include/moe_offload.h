@@ -348,7 +348,10 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * call); what = 7: the per-miss path's expert kernels are the streaming
  * kernels (n = 1, the default: bulk-copied tiles, a warp per tile, the hit
  * experts' gate/up and down in one launch) or the split-K kernels (n = 0);
- * what = 0 clears 1, 2, 4 and 5. */
+ * what = 8: in the next n streaming-kernel launches, CTA 0 issues no copies
+ * for its first work item, so a consumer's bounded wait runs out (the CTA
+ * records the check, lets its other copies land and returns; the next call
+ * reports MOE_ERR_CUDA); what = 0 clears 1, 2, 4, 5 and 8. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Hybrid split: m missing experts, PCIe bandwidth B_P, host expert-processing

@@ -355,7 +355,7 @@ def test_layer_kernel_path_matches_the_oracle():
 def test_split_k_per_miss_kernels_match_the_oracle(T):
     """The per-miss path with the split-K expert kernels (expert_gemv.cu)
     instead of the streaming ones: same trace, table, slots and outputs."""
-    pb = DecodeProblem(MID, T=12, streams=T)
+    pb = DecodeProblem(MID, T=12, streams=T, C=min(T * MID.k, MID.E) + 6)
     st = pb.stack()
     abi.moe_debug_inject(st.ctx, 7, 0)
     run = pb.run(stack=st, routing=True)
@@ -378,6 +378,37 @@ def test_two_copy_streams_match_the_oracle(path):
     assert _check_run(pb, run) < 1e-5
     pb.check_slots(st, run.table[1])
     assert run.stats.misses >= 2 * pb.T // 3  # the calls held several misses each
+    st.close()
+
+
+def test_streaming_kernel_wait_runs_out_then_reset_recovers():
+    """CTA 0 of the next streaming launches issues no copies for its first work
+    item: the consumer's bounded wait on that stage runs out (limit 0.3 s), the
+    CTA records the failed check in the mapped page, lets its other copies land
+    and returns -- nothing hangs, the context stays usable.  The next call
+    reports it (MOE_ERR_CUDA, device check 42-44), a reset brings the context
+    back, and a full run matches the oracle."""
+    import time
+    pb = DecodeProblem(synth.TINY, T=8)
+    st = pb.stack()
+    abi.moe_set_wait_limit(st.ctx, 0.3)
+    abi.moe_debug_inject(st.ctx, 8, 3)  # the next three streaming launches
+    x = torch.from_numpy(pb.x[:, 0]).cuda()
+    y = torch.zeros((pb.T, 1, pb.shape.d), device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    st.forward(0, x[0], y[0])
+    st.synchronize()
+    assert time.perf_counter() - t0 < 10.0
+    with pytest.raises(abi.MoeError) as ei:
+        st.forward(0, x[1], y[1])
+    assert ei.value.status == abi.MOE_ERR_CUDA
+    msg = abi.moe_last_error(st.ctx)
+    assert any(f"device check {c}" in msg for c in (42, 43, 44)), msg
+    abi.moe_debug_inject(st.ctx, 0, 0)
+    st.reset()
+    abi.moe_set_wait_limit(st.ctx, 60.0)
+    _check_run(pb, pb.run(stack=st))
     st.close()
 
 
