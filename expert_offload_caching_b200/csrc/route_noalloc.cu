@@ -98,27 +98,39 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
     if (!s_last) return;
     __threadfence();
 
-    // a NaN logit counts as -inf (selection and softmax), as in moe_layer_forward
+    // a NaN logit counts as -inf (selection and softmax), as in moe_layer_forward.
+    // A row lives in registers (entry lane + 32 j in v[j]); a picked entry is
+    // masked out by its bit, so each pick is the largest remaining logit in
+    // (value desc, id asc) order and k distinct ids in [0, E) come out.
+    constexpr int kNv = kNaMaxE / 32;
     for (int t = warp; t < T; t += nw) {
         const float *zr = z + (size_t)t * E;
-        auto zval = [&](int e) { const float v = zr[e]; return v != v ? -INFINITY : v; };
+        float v[kNv];
+        uint32_t avail = 0u;
         float m = -INFINITY;
-        for (int e = lane; e < E; e += 32) m = fmaxf(m, zval(e));
+#pragma unroll
+        for (int j = 0; j < kNv; ++j) {
+            const int e = lane + 32 * j;
+            const float zv = e < E ? __ldcg(zr + e) : -INFINITY;
+            v[j] = zv != zv ? -INFINITY : zv;
+            if (e < E) avail |= 1u << j;
+            m = fmaxf(m, v[j]);
+        }
         m = na_warp_max(m);
         float sall = 0.f;
-        for (int e = lane; e < E; e += 32) sall += expf(zval(e) - m);
+#pragma unroll
+        for (int j = 0; j < kNv; ++j)
+            if ((avail >> j) & 1u) sall += expf(v[j] - m);
         sall = na_warp_sum(sall);
-        // selection s: the largest logit below the previous pick in (value desc, id asc) order
-        float pv = INFINITY;
-        int pi = -1, my_idx = 0x7fffffff;
+        int my_idx = 0x7fffffff;
         float my_val = -INFINITY;
         for (int s = 0; s < k; ++s) {
             float bv = -INFINITY;
             int bi = 0x7fffffff;
-            for (int e = lane; e < E; e += 32) {
-                const float v = zval(e);
-                const bool after_prev = v < pv || (v == pv && e > pi);
-                if (after_prev && (v > bv || (v == bv && e < bi))) { bv = v; bi = e; }
+#pragma unroll
+            for (int j = 0; j < kNv; ++j) {  // ascending ids within the lane: keep the first of equal values
+                const int e = lane + 32 * j;
+                if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = e; }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -126,9 +138,8 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
                 const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
                 if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
             }
+            if (bi != 0x7fffffff && (bi & 31) == lane) avail &= ~(1u << (bi >> 5));
             if (lane == s) { my_idx = bi; my_val = bv; }
-            pv = bv;
-            pi = bi;
         }
         const float top = __shfl_sync(0xffffffffu, my_val, 0);
         float g;
