@@ -55,8 +55,10 @@ struct ExpMeta {            // one expert of the launch (dynamic shared memory)
     int nrows, row_off;     // rows using it, first row ref
     float ts[3];            // NVFP4 tensor scales (gate, up, down)
     int job;                // job index, -1: the shared expert
+    int cnt;                // phase 3: gate/up tiles of it this CTA completed
+    int pad;
 };
-static_assert(sizeof(ExpMeta) == 32, "metadata stride");
+static_assert(sizeof(ExpMeta) == 40, "metadata stride");
 
 __device__ __forceinline__ unsigned long long st_now() {
     unsigned long long t;
@@ -217,6 +219,7 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
             m.nrows = __ldcg(&a.jobs[j].nrows);
             m.row_off = __ldcg(&a.jobs[j].row_off);
         }
+        m.cnt = 0;
         if (!kMx) {
             const float *t = reinterpret_cast<const float *>(m.rec + a.lay.tscales);
             m.ts[0] = t[0];
@@ -239,7 +242,10 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
     const uint32_t cbA = 8u * (uint32_t)a.d, sbA = kMx ? (uint32_t)(a.d >> 1) : (uint32_t)a.d;
     const uint32_t cbB = 8u * (uint32_t)a.F, sbB = kMx ? (uint32_t)(a.F >> 1) : (uint32_t)a.F;
 
-    if (nexp == 0 && a.combine && blockIdx.x == 0 && (a.combine == 1 || __ldcg(a.n_misses) == 0)) {
+    // combine here: always (1), or (2) only if the lookup had no miss (the
+    // route kernel, complete, wrote the count)
+    const bool combine = a.combine == 1 || (a.combine == 2 && __ldcg(a.n_misses) == 0);
+    if (nexp == 0 && combine && blockIdx.x == 0) {
         // nothing of this layer is computed here (an expert-parallel shard that
         // owns none of the selected experts): its partial output is the shared
         // expert's (computed by earlier launches) or zero
@@ -285,8 +291,26 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
     } else if (warp <= C) {
         // ---------------------------------------------------------- consumers
         const int g = lane >> 2, q = lane & 3;
+        // phase 3: gate/up tiles this CTA completed, per launch expert, published
+        // once, when every consumer warp has passed its last gate/up item
+        bool published = a.phase != 3;
+        auto publish = [&]() {
+            // (named barrier 1: the consumer warps only; it orders their h writes
+            // before the fence of the warp that publishes)
+            asm volatile("barrier.sync 1, %0;" ::"r"(32 * C) : "memory");
+            if (warp == 1) {
+                __threadfence();
+                for (int e = lane; e < nexp; e += 32)
+                    if (meta[e].cnt) atomicAdd(a.done + e, (unsigned)meta[e].cnt);
+            }
+            published = true;
+        };
         for (int l = warp - 1; l < n_my; l += C) {
             const int s = l % NS, n = l / NS;
+            const int gi = (int)blockIdx.x + l * G;
+            const StItem it = st_item(gi, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
+            const bool gate_up = it.gate_up;
+            if (!gate_up && !published) publish();
             // lane 0 waits (bounded); the verdict is the warp's, so the lanes stay
             // converged for mma.sync; then every lane observes the completed phase
             int ok = 1;
@@ -301,13 +325,10 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
             }
             for (uint32_t i = 0; i < (1u << 20) && !st_mbar_test(&s_full[s], n & 1); ++i) {
             }
-            const int gi = (int)blockIdx.x + l * G;
-            const StItem it = st_item(gi, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
-            const bool gate_up = it.gate_up;
             const ExpMeta m = meta[it.e];
             const bool shared = m.job < 0;
             if (!gate_up && a.phase == 3) {  // h: every gate/up tile of this expert
-                int ok = 1;
+                ok = 1;
                 if (lane == 0) {
                     unsigned ns_ = 32;
                     for (uint32_t i = 0;; ++i) {
@@ -357,12 +378,16 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
                                                : act + (size_t)(tr * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
                         }
                     }
-                    float acc[NG][4];
+                    // four accumulator sets (step parity x chunk half): four short
+                    // mma dependency chains instead of one long one
+                    float acc[4][NG][4];
 #pragma unroll
-                    for (int grp = 0; grp < NG; ++grp)
+                    for (int z = 0; z < 4; ++z)
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) acc[grp][u] = 0.f;
-                    for (int st = 0; st < nsteps; ++st) {
+                        for (int grp = 0; grp < NG; ++grp)
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) acc[z][grp][u] = 0.f;
+                    auto kstep = [&](int st, float(&a0)[NG][4], float(&a1)[NG][4]) {
                         const int c = 4 * st + q;
                         const bool cv = c < NCH;  // ragged K tail: this lane feeds zeros
                         const int cc = cv ? c : 0;
@@ -370,21 +395,25 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
                             const uint32_t sa = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rA * (K >> 5) + 2 * c) : 0u;
                             const uint32_t sbv = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rB * (K >> 5) + 2 * c) : 0u;
                             if (gate_up)
-                                step_mma_mx<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
-                                                       sa, sbv, cc, cv, col, colv, ngrp, acc);
+                                step_mma_mx_x2<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                          sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                             else
-                                step_mma_mx<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
-                                                      sa, sbv, cc, cv, col, colv, ngrp, acc);
+                                step_mma_mx_x2<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                         sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                         } else {
                             const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
                             const uint32_t sbv = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rB * (K >> 4) + 4 * c) : 0u;
                             if (gate_up)
-                                step_mma<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
-                                                    sa, sbv, cc, cv, col, colv, ngrp, acc);
+                                step_mma_x2<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                       sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                             else
-                                step_mma<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
-                                                   sa, sbv, cc, cv, col, colv, ngrp, acc);
+                                step_mma_x2<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                      sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                         }
+                    };
+                    for (int st = 0; st < nsteps; st += 2) {
+                        kstep(st, acc[0], acc[1]);
+                        if (st + 1 < nsteps) kstep(st + 1, acc[2], acc[3]);
                     }
                     if (t == it.nt - 1 && r0 + 4 * NG >= m.nrows) {
                         // the stage's last read by this warp: hand it back to the producer
@@ -400,8 +429,11 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
                         int tr, p;
                         if (shared) { tr = r; p = a.k; }
                         else { const RowRef rf = rrs[m.row_off + r]; tr = rf.t; p = rf.p; }
-                        const float v0 = acc[grp][0] + acc[grp][1];
-                        const float v1 = acc[grp][2] + acc[grp][3];
+                        float d4[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) d4[u] = (acc[0][grp][u] + acc[1][grp][u]) + (acc[2][grp][u] + acc[3][grp][u]);
+                        const float v0 = d4[0] + d4[1];
+                        const float v1 = d4[2] + d4[3];
                         const size_t sel = (size_t)tr * (a.k + 1) + p;
                         if (gate_up) {
                             const float gt = kMx ? v0 : m.ts[0] * v0, up = kMx ? v1 : m.ts[1] * v1;
@@ -419,45 +451,47 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
                         }
                     }
                 }
-                if (!gate_up && a.combine) {  // the tile's last expert: combine its rows
-                    __syncwarp();
-                    int last = 0;
-                    if (lane == 0) {
-                        __threadfence();
-                        last = atomicAdd(&a.tile_ticket[tile], 1u) == (unsigned)(nexp - 1);
-                    }
-                    last = __shfl_sync(0xffffffffu, last, 0);
-                    if (last) {
-                        __threadfence();
-                        if (a.combine == 1 || __ldcg(a.n_misses) == 0) {
-                            for (int i = lane; i < 16 * a.T; i += 32) {
-                                const int tr = i >> 4, o = 16 * tile + (i & 15);
-                                const float *pr = a.part_out + (size_t)tr * (a.k + 1) * a.d + o;
-                                float sum = 0.f;
-                                for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
-                                    if (a.ep_size == 1 || a.idx[tr * a.k + p] % a.ep_size == a.ep_rank)
-                                        sum = fmaf(a.gates[tr * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
-                                if (a.shared_part) sum += __ldcg(pr + (size_t)a.k * a.d);
-                                a.y[(size_t)tr * a.d + o] = sum;
-                            }
-                        }
-                        __syncwarp();
-                        if (lane == 0) a.tile_ticket[tile] = 0u;
-                    }
-                }
             }
             if (!released) {  // (an expert without rows: nothing read)
                 __syncwarp();
                 if (lane == 0) st_mbar_arrive(&s_empty[s]);
             }
-            if (gate_up && a.phase == 3) {  // publish this item's h tiles
+            if (gate_up && a.phase == 3 && lane == 0) atomicAdd(&meta[it.e].cnt, it.nt);  // (shared memory)
+            if (!gate_up && combine) {
+                // the item's tiles whose last expert this is: their rows are combined here.
+                // One expert in the launch: every tile (earlier launches completed the rest).
+                uint32_t last = it.nt >= 32 ? 0xffffffffu : ((1u << it.nt) - 1u);
                 __syncwarp();
-                if (lane == 0) {
-                    __threadfence();
-                    atomicAdd(a.done + it.e, (unsigned)it.nt);
+                if (nexp > 1) {
+                    uint32_t mine = 0u;
+                    if (lane == 0) {
+                        __threadfence();
+                        for (int t = 0; t < it.nt; ++t)
+                            if (atomicAdd(&a.tile_ticket[it.tile0 + t], 1u) == (unsigned)(nexp - 1)) mine |= 1u << t;
+                    }
+                    last = __shfl_sync(0xffffffffu, mine, 0);
+                    if (last) __threadfence();
+                }
+                for (int t = 0; t < it.nt; ++t) {
+                    if (!((last >> t) & 1u)) continue;
+                    const int tile = it.tile0 + t;
+                    for (int i = lane; i < 16 * a.T; i += 32) {
+                        const int tr = i >> 4, o = 16 * tile + (i & 15);
+                        const float *pr = a.part_out + (size_t)tr * (a.k + 1) * a.d + o;
+                        float sum = 0.f;
+                        for (int p = 0; p < a.k; ++p)  // (with expert parallelism: the owned experts)
+                            if (a.ep_size == 1 || a.idx[tr * a.k + p] % a.ep_size == a.ep_rank)
+                                sum = fmaf(a.gates[tr * a.k + p], __ldcg(pr + (size_t)p * a.d), sum);
+                        if (a.shared_part) sum += __ldcg(pr + (size_t)a.k * a.d);
+                        a.y[(size_t)tr * a.d + o] = sum;
+                    }
+                    if (nexp > 1 && lane == 0) a.tile_ticket[tile] = 0u;
                 }
             }
         }
+        // every consumer warp passes the barrier exactly once, on error paths too
+        // (a consumer without down items, or one that stopped, arrives here)
+        if (!published) publish();
     }
 
     __syncthreads();

@@ -203,5 +203,108 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
     }
 }
 
+// step_mma / step_mma_mx with two accumulator sets: the first 32 codes of the
+// chunk (h = 0) go into acc0, the last 32 (h = 1) into acc1, so the mma
+// dependency chain is half as long (the dot product is order-free).
+template <int NG, bool kCg = false>
+__device__ __forceinline__ void step_mma_x2(const uint8_t *cA, const uint8_t *cB, uint32_t sa, uint32_t sb, int c,
+                                            bool cv, const __half *const (&col)[NG], const bool (&colv)[NG], int ngrp,
+                                            float (&acc0)[NG][4], float (&acc1)[NG][4]) {
+    const __half2 a01 = e4m3x2_to_h2(sa & 0xffffu), a23 = e4m3x2_to_h2(sa >> 16);
+    const __half2 b01 = e4m3x2_to_h2(sb & 0xffffu), b23 = e4m3x2_to_h2(sb >> 16);
+    const __half2 sAv[4] = {__low2half2(a01), __high2half2(a01), __low2half2(a23), __high2half2(a23)};
+    const __half2 sBv[4] = {__low2half2(b01), __high2half2(b01), __low2half2(b23), __high2half2(b23)};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float(&acc)[NG][4] = h == 0 ? acc0 : acc1;
+        const uint4 qa = cv ? *reinterpret_cast<const uint4 *>(cA + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint4 qb = cv ? *reinterpret_cast<const uint4 *>(cB + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+        const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int w = 4 * h + u;
+            uint32_t fa[4], fb[4];
+            e2m1x8_to_f16(wa[u], fa);
+            e2m1x8_to_f16(wb[u], fb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                fa[j] = hmul2u(fa[j], sAv[w >> 1]);
+                fb[j] = hmul2u(fb[j], sBv[w >> 1]);
+            }
+#pragma unroll
+            for (int grp = 0; grp < NG; ++grp) {
+                if (grp < ngrp) {
+                    uint4 bv = make_uint4(0, 0, 0, 0);
+                    if (colv[grp] && cv) bv = ld_act<kCg>(col[grp] + 64 * c + 8 * w);
+                    mma16816(acc[grp], fa[0], fb[0], fa[1], fb[1], bv.x, bv.y);
+                    mma16816(acc[grp], fa[2], fb[2], fa[3], fb[3], bv.z, bv.w);
+                }
+            }
+        }
+    }
+}
+
+template <int NG, bool kCg = false>
+__device__ __forceinline__ void step_mma_mx_x2(const uint8_t *cA, const uint8_t *cB, uint32_t sa, uint32_t sb, int c,
+                                               bool cv, const __half *const (&col)[NG], const bool (&colv)[NG],
+                                               int ngrp, float (&acc0)[NG][4], float (&acc1)[NG][4]) {
+    const int a0 = sa & 0xff, a1 = (sa >> 8) & 0xff, b0 = sb & 0xff, b1 = (sb >> 8) & 0xff;
+    int ma = max(a0, a1), mb = max(b0, b1);
+    ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+    ma = max(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+    mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+    mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+    const __half2 sAv[2] = {mx_pow2_h2(a0 - ma), mx_pow2_h2(a1 - ma)};
+    const __half2 sBv[2] = {mx_pow2_h2(b0 - mb), mx_pow2_h2(b1 - mb)};
+    float stp[2][NG][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int grp = 0; grp < NG; ++grp)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) stp[h][grp][i] = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint4 qa = cv ? *reinterpret_cast<const uint4 *>(cA + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint4 qb = cv ? *reinterpret_cast<const uint4 *>(cB + 16 * h) : make_uint4(0, 0, 0, 0);
+        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+        const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int w = 4 * h + u;  // block w / 4 == h
+            uint32_t fa[4], fb[4];
+            e2m1x8_to_f16(wa[u], fa);
+            e2m1x8_to_f16(wb[u], fb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                fa[j] = hmul2u(fa[j], sAv[h]);
+                fb[j] = hmul2u(fb[j], sBv[h]);
+            }
+#pragma unroll
+            for (int grp = 0; grp < NG; ++grp) {
+                if (grp < ngrp) {
+                    uint4 bv = make_uint4(0, 0, 0, 0);
+                    if (colv[grp] && cv) bv = ld_act<kCg>(col[grp] + 64 * c + 8 * w);
+                    mma16816(stp[h][grp], fa[0], fb[0], fa[1], fb[1], bv.x, bv.y);
+                    mma16816(stp[h][grp], fa[2], fb[2], fa[3], fb[3], bv.z, bv.w);
+                }
+            }
+        }
+    }
+    const float fA = mx_factor(ma), fB = mx_factor(mb);
+#pragma unroll
+    for (int grp = 0; grp < NG; ++grp) {  // d0, d1: row rA; d2, d3: row rB
+        acc0[grp][0] = fmaf(stp[0][grp][0], fA, acc0[grp][0]);
+        acc0[grp][1] = fmaf(stp[0][grp][1], fA, acc0[grp][1]);
+        acc0[grp][2] = fmaf(stp[0][grp][2], fB, acc0[grp][2]);
+        acc0[grp][3] = fmaf(stp[0][grp][3], fB, acc0[grp][3]);
+        acc1[grp][0] = fmaf(stp[1][grp][0], fA, acc1[grp][0]);
+        acc1[grp][1] = fmaf(stp[1][grp][1], fA, acc1[grp][1]);
+        acc1[grp][2] = fmaf(stp[1][grp][2], fB, acc1[grp][2]);
+        acc1[grp][3] = fmaf(stp[1][grp][3], fB, acc1[grp][3]);
+    }
+}
+
 }  // namespace gemv
 }  // namespace moe

@@ -305,7 +305,7 @@ def _stream_launch(d, F, T, k, max_exp, mx, sms=148):
         return max(tp, 1)
 
     tpa, tpb = per_item(tA, nA), per_item(tB, nB)
-    meta = max_exp * 32
+    meta = max_exp * 40
     rr = (T * k * 4 + 15) & ~15
     budget = 200 * 1024
     assert meta + rr + 2 * sb <= budget
