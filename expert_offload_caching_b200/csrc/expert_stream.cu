@@ -44,7 +44,7 @@ namespace {
 using namespace gemv;
 
 constexpr int kStMaxStages = 8;
-constexpr int kStMaxConsumers = 7;             // + the producer warp: 256 threads
+constexpr int kStMaxPairs = 5;                 // consumer warp pairs; + the producer warp: 352 threads
 constexpr int kErrStreamFull = 42;             // a stage's copy did not land in time
 constexpr int kErrStreamEmpty = 43;            // a stage was not released in time
 constexpr int kErrStreamDep = 44;              // a down item's gate/up tiles did not complete in time
@@ -149,10 +149,12 @@ __device__ __forceinline__ StItem st_item(int g, int phase, int nexp, int nA, in
 }
 
 template <int NG, int FMT>
-__global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kStMaxStages], s_empty[kStMaxStages];
     __shared__ int s_nexp, s_last;
+    __shared__ int s_pair_ok[kStMaxPairs];
+    __shared__ float s_red[kStMaxPairs * 2 * 2 * 4 * 32];  // [pair][buffer][NG <= 2][4][32] partials of member 1
     __shared__ volatile int s_stop;
     constexpr bool kMx = FMT == kFmtMxfp4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -288,72 +290,78 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
             for (int l = issued > NS ? issued - NS : 0; l < issued; ++l)
                 if (l != skipped) st_mbar_wait(&s_full[l % NS], (l / NS) & 1, drain, &never);
         }
-    } else if (warp <= C) {
+    } else if (warp <= 2 * C) {
         // ---------------------------------------------------------- consumers
+        // warp pairs: pair gq takes the CTA's items gq, gq + C, ... (stage l mod S,
+        // S a multiple of C); member 0 the first half of each tile's K-steps,
+        // member 1 the second; member 1's partial sums meet member 0's through
+        // shared memory at the pair's named barrier (2 + gq, 64 threads)
+        const int cw = warp - 1, gq = cw >> 1, mp = cw & 1;
         const int g = lane >> 2, q = lane & 3;
+        const uint32_t pair_bar = 2u + (uint32_t)gq;
+        auto pair_sync = [&]() { asm volatile("barrier.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
+        int rbuf = 0;  // partials double buffer, flipped per row group
         // phase 3: gate/up tiles this CTA completed, per launch expert, published
         // once, when every consumer warp has passed its last gate/up item
         bool published = a.phase != 3;
         auto publish = [&]() {
-            // (named barrier 1: the consumer warps only; it orders their h writes
+            // (named barrier 1: every consumer warp; it orders their h writes
             // before the fence of the warp that publishes)
-            asm volatile("barrier.sync 1, %0;" ::"r"(32 * C) : "memory");
-            if (warp == 1) {
+            asm volatile("barrier.sync 1, %0;" ::"r"(64 * C) : "memory");
+            if (cw == 0) {
                 __threadfence();
                 for (int e = lane; e < nexp; e += 32)
                     if (meta[e].cnt) atomicAdd(a.done + e, (unsigned)meta[e].cnt);
             }
             published = true;
         };
-        for (int l = warp - 1; l < n_my; l += C) {
+        for (int l = gq; l < n_my; l += C) {
             const int s = l % NS, n = l / NS;
             const int gi = (int)blockIdx.x + l * G;
             const StItem it = st_item(gi, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
             const bool gate_up = it.gate_up;
             if (!gate_up && !published) publish();
-            // lane 0 waits (bounded); the verdict is the warp's, so the lanes stay
-            // converged for mma.sync; then every lane observes the completed phase
-            int ok = 1;
-            if (lane == 0) {
-                ok = st_mbar_wait(&s_full[s], n & 1, deadline, &s_stop);
-                if (!ok && !s_stop) st_fail(a, kErrStreamFull, l, s);
+            // member 0 takes the waits (bounded) and hands the verdict to member 1
+            // at the pair barrier, so both break or proceed together
+            if (mp == 0) {
+                int ok = 1;
+                if (lane == 0) {
+                    ok = st_mbar_wait(&s_full[s], n & 1, deadline, &s_stop);
+                    if (!ok && !s_stop) st_fail(a, kErrStreamFull, l, s);
+                    if (ok && !gate_up && a.phase == 3) {  // h: every gate/up tile of this expert
+                        unsigned ns_ = 32;
+                        for (uint32_t i = 0;; ++i) {
+                            if (st_ld_acquire(a.done + it.e) >= (uint32_t)nA) break;
+                            if ((i & 7u) == 7u && (s_stop || st_now() > deadline)) {
+                                if (!s_stop) st_fail(a, kErrStreamDep, gi, it.e);
+                                ok = 0;
+                                break;
+                            }
+                            __nanosleep(ns_);
+                            if (ns_ < 512) ns_ <<= 1;
+                        }
+                        __threadfence();
+                    }
+                    if (!ok) s_stop = 1;
+                    s_pair_ok[gq] = ok;
+                }
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) {
-                s_stop = 1;
-                break;
-            }
+            pair_sync();
+            const int ok = s_pair_ok[gq];
+            if (!ok) break;
+            // every lane observes the completed phase (it has: member 0 saw it)
             for (uint32_t i = 0; i < (1u << 20) && !st_mbar_test(&s_full[s], n & 1); ++i) {
             }
             const ExpMeta m = meta[it.e];
             const bool shared = m.job < 0;
-            if (!gate_up && a.phase == 3) {  // h: every gate/up tile of this expert
-                ok = 1;
-                if (lane == 0) {
-                    unsigned ns_ = 32;
-                    for (uint32_t i = 0;; ++i) {
-                        if (st_ld_acquire(a.done + it.e) >= (uint32_t)nA) break;
-                        if ((i & 7u) == 7u && (s_stop || st_now() > deadline)) {
-                            if (!s_stop) st_fail(a, kErrStreamDep, gi, it.e);
-                            s_stop = 1;
-                            ok = 0;
-                            break;
-                        }
-                        __nanosleep(ns_);
-                        if (ns_ < 512) ns_ <<= 1;
-                    }
-                    __threadfence();
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-            }
             const int K = gate_up ? a.d : a.F;
             const int NCH = K >> 6, nsteps = (NCH + 3) >> 2;
+            const int half = (nsteps + 1) >> 1;
+            const int st0 = mp ? half : 0, st1 = mp ? nsteps : half;
             const uint32_t cb = gate_up ? cbA : cbB, sb = gate_up ? sbA : sbB;
             const uint8_t *stage = smem + (size_t)s * a.stage_bytes;
             const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
             const __half *act = gate_up ? a.act : a.hh_out;
-            bool released = false;
             for (int t = 0; t < it.nt; ++t) {
                 const int tile = it.tile0 + t;
                 const uint8_t *s_codes = stage + (size_t)t * cb;
@@ -411,29 +419,41 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
                                                       sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                         }
                     };
-                    for (int st = 0; st < nsteps; st += 2) {
+                    for (int st = st0; st < st1; st += 2) {
                         kstep(st, acc[0], acc[1]);
-                        if (st + 1 < nsteps) kstep(st + 1, acc[2], acc[3]);
+                        if (st + 1 < st1) kstep(st + 1, acc[2], acc[3]);
                     }
-                    if (t == it.nt - 1 && r0 + 4 * NG >= m.nrows) {
-                        // the stage's last read by this warp: hand it back to the producer
-                        __syncwarp();
-                        if (lane == 0) st_mbar_arrive(&s_empty[s]);
-                        released = true;
+                    float d4[NG][4];
+#pragma unroll
+                    for (int grp = 0; grp < NG; ++grp)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            d4[grp][u] = (acc[0][grp][u] + acc[1][grp][u]) + (acc[2][grp][u] + acc[3][grp][u]);
+                    float(*rb)[4][32] = reinterpret_cast<float(*)[4][32]>(s_red + (gq * 2 + rbuf) * (2 * 4 * 32));
+                    rbuf ^= 1;
+                    if (mp == 1) {
+#pragma unroll
+                        for (int grp = 0; grp < NG; ++grp)
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) rb[grp][u][lane] = d4[grp][u];
                     }
-                    // each lane's results: activation row r0 + 4*grp + q; tile rows rA (d0, d1), rB (d2, d3)
+                    pair_sync();  // member 1's partials are in shared memory; both are done with the stage's rows
+                    if (t == it.nt - 1 && r0 + 4 * NG >= m.nrows && mp == 0 && lane == 0)
+                        st_mbar_arrive(&s_empty[s]);  // the pair's last read of the stage: hand it back
+                    if (mp == 1) continue;
+                    // member 0: each lane's results -- activation row r0 + 4*grp + q; tile
+                    // rows rA (d0, d1), rB (d2, d3)
 #pragma unroll
                     for (int grp = 0; grp < NG; ++grp) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) d4[grp][u] += rb[grp][u][lane];
                         const int r = r0 + 4 * grp + q;
                         if (r >= m.nrows) continue;
                         int tr, p;
                         if (shared) { tr = r; p = a.k; }
                         else { const RowRef rf = rrs[m.row_off + r]; tr = rf.t; p = rf.p; }
-                        float d4[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) d4[u] = (acc[0][grp][u] + acc[1][grp][u]) + (acc[2][grp][u] + acc[3][grp][u]);
-                        const float v0 = d4[0] + d4[1];
-                        const float v1 = d4[2] + d4[3];
+                        const float v0 = d4[grp][0] + d4[grp][1];
+                        const float v1 = d4[grp][2] + d4[grp][3];
                         const size_t sel = (size_t)tr * (a.k + 1) + p;
                         if (gate_up) {
                             const float gt = kMx ? v0 : m.ts[0] * v0, up = kMx ? v1 : m.ts[1] * v1;
@@ -452,10 +472,8 @@ __global__ void __launch_bounds__(32 * (kStMaxConsumers + 1), 1) expert_stream_k
                     }
                 }
             }
-            if (!released) {  // (an expert without rows: nothing read)
-                __syncwarp();
-                if (lane == 0) st_mbar_arrive(&s_empty[s]);
-            }
+            if (m.nrows <= 0 && mp == 0 && lane == 0) st_mbar_arrive(&s_empty[s]);  // (an expert without rows)
+            if (mp == 1) continue;  // member 0 publishes and combines
             if (gate_up && a.phase == 3 && lane == 0) atomicAdd(&meta[it.e].cnt, it.nt);  // (shared memory)
             if (!gate_up && combine) {
                 // the item's tiles whose last expert this is: their rows are combined here.
@@ -521,7 +539,7 @@ cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) 
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(32 * (a.nc + 1));
+    cfg.blockDim = dim3(32 * (2 * a.nc + 1));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
@@ -581,8 +599,9 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
     // where six or more fit, else one; the stage count is a multiple of the
     // consumer count, so a stage always serves the same warp and its phases are
     // consumed in order (a parity wait can then not see an older phase)
-    int nc = ns >= 6 ? ns / 2 : ns;
+    int nc = ns >= 6 ? ns / 2 : ns;  // warp pairs
     if (nc > 4 && ns >= 6) nc = 4;
+    if (nc > kStMaxPairs) nc = kStMaxPairs;
     a.nc = nc;
     a.ns = ns = (ns >= 6 ? 2 : 1) * nc;
     a.stage_bytes = (uint32_t)sb;
