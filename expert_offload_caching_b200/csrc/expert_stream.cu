@@ -44,7 +44,10 @@ namespace {
 using namespace gemv;
 
 constexpr int kStMaxStages = 8;
-constexpr int kStMaxPairs = 5;                 // consumer warp pairs; + the producer warp: 352 threads
+constexpr int kStMaxGroups = 5;                // consumer warp groups (P warps each) + the producer warp
+// (with the producer, 16 or 11 warps: at most four per SM sub-partition, so
+// up to 128 registers per thread for groups of three)
+__host__ __device__ constexpr int st_max_groups(int P) { return kStMaxGroups; }
 constexpr int kErrStreamFull = 42;             // a stage's copy did not land in time
 constexpr int kErrStreamEmpty = 43;            // a stage was not released in time
 constexpr int kErrStreamDep = 44;              // a down item's gate/up tiles did not complete in time
@@ -148,13 +151,13 @@ __device__ __forceinline__ StItem st_item(int g, int phase, int nexp, int nA, in
     return it;
 }
 
-template <int NG, int FMT>
-__global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_kernel(GemvArgs a) {
+template <int NG, int FMT, int P>
+__global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_stream_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kStMaxStages], s_empty[kStMaxStages];
     __shared__ int s_nexp, s_last;
-    __shared__ int s_pair_ok[kStMaxPairs];
-    __shared__ float s_red[kStMaxPairs * 2 * 2 * 4 * 32];  // [pair][buffer][NG <= 2][4][32] partials of member 1
+    __shared__ int s_pair_ok[st_max_groups(P)];
+    __shared__ float s_red[st_max_groups(P) * 2 * (P - 1) * NG * 4 * 32];  // [group][buffer][member 1..P-1][NG][4][32]
     __shared__ volatile int s_stop;
     constexpr bool kMx = FMT == kFmtMxfp4;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -290,16 +293,16 @@ __global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_k
             for (int l = issued > NS ? issued - NS : 0; l < issued; ++l)
                 if (l != skipped) st_mbar_wait(&s_full[l % NS], (l / NS) & 1, drain, &never);
         }
-    } else if (warp <= 2 * C) {
+    } else if (warp <= P * C) {
         // ---------------------------------------------------------- consumers
-        // warp pairs: pair gq takes the CTA's items gq, gq + C, ... (stage l mod S,
-        // S a multiple of C); member 0 the first half of each tile's K-steps,
-        // member 1 the second; member 1's partial sums meet member 0's through
-        // shared memory at the pair's named barrier (2 + gq, 64 threads)
-        const int cw = warp - 1, gq = cw >> 1, mp = cw & 1;
+        // warp groups of P: group gq takes the CTA's items gq, gq + C, ... (stage
+        // l mod S, S a multiple of C); member mp takes the mp-th P-th of each
+        // tile's K-steps; members 1..P-1 leave their partial sums in shared memory
+        // for member 0 at the group's named barrier (2 + gq, 32 P threads)
+        const int cw = warp - 1, gq = cw / P, mp = cw % P;
         const int g = lane >> 2, q = lane & 3;
         const uint32_t pair_bar = 2u + (uint32_t)gq;
-        auto pair_sync = [&]() { asm volatile("barrier.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
+        auto pair_sync = [&]() { asm volatile("barrier.sync %0, %1;" ::"r"(pair_bar), "r"(32 * P) : "memory"); };
         int rbuf = 0;  // partials double buffer, flipped per row group
         // phase 3: gate/up tiles this CTA completed, per launch expert, published
         // once, when every consumer warp has passed its last gate/up item
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_k
         auto publish = [&]() {
             // (named barrier 1: every consumer warp; it orders their h writes
             // before the fence of the warp that publishes)
-            asm volatile("barrier.sync 1, %0;" ::"r"(64 * C) : "memory");
+            asm volatile("barrier.sync 1, %0;" ::"r"(32 * P * C) : "memory");
             if (cw == 0) {
                 __threadfence();
                 for (int e = lane; e < nexp; e += 32)
@@ -356,8 +359,7 @@ __global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_k
             const bool shared = m.job < 0;
             const int K = gate_up ? a.d : a.F;
             const int NCH = K >> 6, nsteps = (NCH + 3) >> 2;
-            const int half = (nsteps + 1) >> 1;
-            const int st0 = mp ? half : 0, st1 = mp ? nsteps : half;
+            const int st0 = mp * nsteps / P, st1 = (mp + 1) * nsteps / P;
             const uint32_t cb = gate_up ? cbA : cbB, sb = gate_up ? sbA : sbB;
             const uint8_t *stage = smem + (size_t)s * a.stage_bytes;
             const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
@@ -386,11 +388,12 @@ __global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_k
                                                : act + (size_t)(tr * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
                         }
                     }
-                    // four accumulator sets (step parity x chunk half): four short
-                    // mma dependency chains instead of one long one
-                    float acc[4][NG][4];
+                    // accumulator sets: chunk half (x step parity with pairs, whose
+                    // members run more steps each): short mma dependency chains
+                    constexpr int kChains = P >= 3 ? 2 : 4;
+                    float acc[kChains][NG][4];
 #pragma unroll
-                    for (int z = 0; z < 4; ++z)
+                    for (int z = 0; z < kChains; ++z)
 #pragma unroll
                         for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
@@ -419,34 +422,45 @@ __global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_k
                                                       sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                         }
                     };
-                    for (int st = st0; st < st1; st += 2) {
-                        kstep(st, acc[0], acc[1]);
-                        if (st + 1 < st1) kstep(st + 1, acc[2], acc[3]);
+                    if constexpr (kChains == 4) {
+                        for (int st = st0; st < st1; st += 2) {
+                            kstep(st, acc[0], acc[1]);
+                            if (st + 1 < st1) kstep(st + 1, acc[kChains - 2], acc[kChains - 1]);
+                        }
+                    } else {
+                        for (int st = st0; st < st1; ++st) kstep(st, acc[0], acc[1]);
                     }
                     float d4[NG][4];
 #pragma unroll
                     for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            d4[grp][u] = (acc[0][grp][u] + acc[1][grp][u]) + (acc[2][grp][u] + acc[3][grp][u]);
-                    float(*rb)[4][32] = reinterpret_cast<float(*)[4][32]>(s_red + (gq * 2 + rbuf) * (2 * 4 * 32));
+                        for (int u = 0; u < 4; ++u) {
+                            float v = acc[0][grp][u] + acc[1][grp][u];
+                            if constexpr (kChains == 4) v += acc[kChains - 2][grp][u] + acc[kChains - 1][grp][u];
+                            d4[grp][u] = v;
+                        }
+                    float *rbase = s_red + (size_t)(gq * 2 + rbuf) * (P - 1) * NG * 128;  // this row group's buffer
                     rbuf ^= 1;
-                    if (mp == 1) {
+                    if (mp > 0) {
+                        float(*rb)[4][32] = reinterpret_cast<float(*)[4][32]>(rbase + (mp - 1) * NG * 128);
 #pragma unroll
                         for (int grp = 0; grp < NG; ++grp)
 #pragma unroll
                             for (int u = 0; u < 4; ++u) rb[grp][u][lane] = d4[grp][u];
                     }
-                    pair_sync();  // member 1's partials are in shared memory; both are done with the stage's rows
+                    pair_sync();  // the members' partials are in shared memory; all are done with the stage's rows
                     if (t == it.nt - 1 && r0 + 4 * NG >= m.nrows && mp == 0 && lane == 0)
-                        st_mbar_arrive(&s_empty[s]);  // the pair's last read of the stage: hand it back
-                    if (mp == 1) continue;
+                        st_mbar_arrive(&s_empty[s]);  // the group's last read of the stage: hand it back
+                    if (mp > 0) continue;
                     // member 0: each lane's results -- activation row r0 + 4*grp + q; tile
                     // rows rA (d0, d1), rB (d2, d3)
 #pragma unroll
                     for (int grp = 0; grp < NG; ++grp) {
+                        for (int j = 1; j < P; ++j) {  // members in order: a fixed summation order
+                            const float(*rb)[4][32] = reinterpret_cast<const float(*)[4][32]>(rbase + (j - 1) * NG * 128);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) d4[grp][u] += rb[grp][u][lane];
+                            for (int u = 0; u < 4; ++u) d4[grp][u] += rb[grp][u][lane];
+                        }
                         const int r = r0 + 4 * grp + q;
                         if (r >= m.nrows) continue;
                         int tr, p;
@@ -473,7 +487,7 @@ __global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_k
                 }
             }
             if (m.nrows <= 0 && mp == 0 && lane == 0) st_mbar_arrive(&s_empty[s]);  // (an expert without rows)
-            if (mp == 1) continue;  // member 0 publishes and combines
+            if (mp > 0) continue;  // member 0 publishes and combines
             if (gate_up && a.phase == 3 && lane == 0) atomicAdd(&meta[it.e].cnt, it.nt);  // (shared memory)
             if (!gate_up && combine) {
                 // the item's tiles whose last expert this is: their rows are combined here.
@@ -528,18 +542,18 @@ __global__ void __launch_bounds__(32 * (2 * kStMaxPairs + 1), 1) expert_stream_k
     if (threadIdx.x == 0) span_mark(a.span, 1);
 }
 
-template <int NG, int FMT>
+template <int NG, int FMT, int P>
 cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) {
     static bool configured = false;  // per instantiation: allow the large dynamic shared memory
     if (!configured) {
-        const cudaError_t e = cudaFuncSetAttribute(expert_stream_kernel<NG, FMT>,
+        const cudaError_t e = cudaFuncSetAttribute(expert_stream_kernel<NG, FMT, P>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 210 * 1024);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(32 * (2 * a.nc + 1));
+    cfg.blockDim = dim3(32 * (P * a.nc + 1));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
@@ -547,7 +561,7 @@ cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) 
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, expert_stream_kernel<NG, FMT>, a);
+    return cudaLaunchKernelEx(&cfg, expert_stream_kernel<NG, FMT, P>, a);
 }
 
 }  // namespace
@@ -599,11 +613,14 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
     // where six or more fit, else one; the stage count is a multiple of the
     // consumer count, so a stage always serves the same warp and its phases are
     // consumed in order (a parity wait can then not see an older phase)
-    int nc = ns >= 6 ? ns / 2 : ns;  // warp pairs
-    if (nc > 4 && ns >= 6) nc = 4;
-    if (nc > kStMaxPairs) nc = kStMaxPairs;
+    // consumer warp groups: P = 3 warps each for up to 4 activation rows per
+    // pass (NG 1), 2 otherwise; a group serves two stages (one loads while the
+    // other is computed) where the stages allow, else one
+    const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
+    const int gmax = kStMaxGroups;
+    int nc = ns >= 2 * gmax ? gmax : (ns >= 6 ? ns / 2 : (ns < gmax ? ns : gmax));
     a.nc = nc;
-    a.ns = ns = (ns >= 6 ? 2 : 1) * nc;
+    a.ns = ns = (ns >= 2 * nc ? 2 : 1) * nc;
     a.stage_bytes = (uint32_t)sb;
     a.meta_off = (uint32_t)(ns * sb);
     a.rr_off = (uint32_t)(ns * sb + meta);
@@ -612,13 +629,12 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
     const int iA = (nA + a.tpa - 1) / a.tpa, iB = (nB + a.tpb - 1) / a.tpb;
     const int64_t items = (int64_t)max_exp * (((a.phase & 1) ? iA : 0) + ((a.phase & 2) ? iB : 0));
     const int grid = (int)(items < sms ? items : sms);
-    const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
     if (mx) {
-        if (ng == 1) return launch_st<1, kFmtMxfp4>(a, grid, smem, s);
-        return launch_st<2, kFmtMxfp4>(a, grid, smem, s);
+        if (ng == 1) return launch_st<1, kFmtMxfp4, 3>(a, grid, smem, s);
+        return launch_st<2, kFmtMxfp4, 2>(a, grid, smem, s);
     }
-    if (ng == 1) return launch_st<1, kFmtNvfp4>(a, grid, smem, s);
-    return launch_st<2, kFmtNvfp4>(a, grid, smem, s);
+    if (ng == 1) return launch_st<1, kFmtNvfp4, 3>(a, grid, smem, s);
+    return launch_st<2, kFmtNvfp4, 2>(a, grid, smem, s);
 }
 
 }  // namespace moe
