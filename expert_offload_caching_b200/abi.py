@@ -64,7 +64,8 @@ class moe_split(ctypes.Structure):
 EXPORTS = ["moe_record_bytes", "moe_shared_record_bytes", "moe_record_layout", "moe_workspace_bytes", "moe_arena_bytes",
            "moe_layer_init", "cache_configure", "moe_layer_forward", "moe_layer_forward_host",
            "moe_get_routing", "moe_cache_export", "moe_get_stats", "moe_set_timing",
-           "moe_set_wait_limit", "moe_set_expert_shard", "moe_debug_inject", "plan_split", "moe_measure_h2d",
+           "moe_set_wait_limit", "moe_set_expert_shard", "moe_debug_inject", "moe_debug_trace", "plan_split",
+           "moe_measure_h2d",
            "moe_measure_h2d_sm",
            "moe_route_noalloc", "moe_status_str", "moe_last_error", "moe_layer_destroy"]
 
@@ -117,6 +118,8 @@ def lib():
         L.moe_set_expert_shard.argtypes = [vp, i32, i32]
         L.moe_debug_inject.restype = ctypes.c_int
         L.moe_debug_inject.argtypes = [vp, i32, i64]
+        L.moe_debug_trace.restype = ctypes.c_int
+        L.moe_debug_trace.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), i32]
         L.plan_split.restype = ctypes.c_int
         L.plan_split.argtypes = [i32, dbl, dbl, dbl, dbl, ctypes.POINTER(moe_split)]
         L.moe_measure_h2d.restype = ctypes.c_int
@@ -255,6 +258,13 @@ def moe_set_expert_shard(ctx: int, rank: int, size: int) -> None:
 
 def moe_debug_inject(ctx: int, what: int, n: int) -> None:
     _check(lib().moe_debug_inject(ctx, what, n), "moe_debug_inject", ctx)
+
+
+def moe_debug_trace(ctx: int, n: int = 160 * 32):
+    """The last traced launch's stamps (see moe_debug_inject what = 9) as a list of ints."""
+    buf = (ctypes.c_uint64 * n)()
+    _check(lib().moe_debug_trace(ctx, buf, n), "moe_debug_trace", ctx)
+    return list(buf)
 
 
 def plan_split(m: int, B_P: float, B_H: float, threshold: float = 2.0,

@@ -151,7 +151,8 @@ __device__ __forceinline__ StItem st_item(int g, int phase, int nexp, int nA, in
     return it;
 }
 
-template <int NG, int FMT, int P>
+// kFull: d and F are multiples of 256, so every K-step chunk is in range
+template <int NG, int FMT, int P, bool kFull>
 __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_stream_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kStMaxStages], s_empty[kStMaxStages];
@@ -167,6 +168,11 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
 
     pdl_wait();  // the job list, x and the row refs come from the route kernel; h from gate/up
     const unsigned long long deadline = st_now() + a.wait_ns;
+    // diagnostic trace: slot 0 start, 1 set-up done, 2 gate/up counts published, 3 end;
+    // group 0 / member 0's first 8 items: 4 + 3k stage wait begins, 5 + 3k data in, 6 + 3k sums in
+    unsigned long long *tr = (a.trace && blockIdx.x < kTraceCtas) ? a.trace + (size_t)blockIdx.x * kTraceSlots : nullptr;
+    auto stamp = [&](int slot) { if (tr) tr[slot] = st_now(); };
+    if (threadIdx.x == 0) stamp(0);
     if (threadIdx.x == 0) {
         span_mark(a.span, 0);
         s_stop = 0;
@@ -237,6 +243,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
         rrs[i] = r;
     }
     __syncthreads();
+    if (threadIdx.x == 0) stamp(1);
 
     // ---- item geometry
     const int nA = a.F >> 3, nB = a.d >> 4;  // tiles per expert: 8 gate/up row pairs, 16 down rows
@@ -315,6 +322,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                 __threadfence();
                 for (int e = lane; e < nexp; e += 32)
                     if (meta[e].cnt) atomicAdd(a.done + e, (unsigned)meta[e].cnt);
+                if (lane == 0) stamp(2);
             }
             published = true;
         };
@@ -326,10 +334,13 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
             if (!gate_up && !published) publish();
             // member 0 takes the waits (bounded) and hands the verdict to member 1
             // at the pair barrier, so both break or proceed together
+            const int tk = (gq == 0 && mp == 0 && lane == 0) ? (l / C) : 99;  // traced item ordinal
+            if (tk < 8) stamp(4 + 3 * tk);
             if (mp == 0) {
                 int ok = 1;
                 if (lane == 0) {
                     ok = st_mbar_wait(&s_full[s], n & 1, deadline, &s_stop);
+                    if (tk < 8) stamp(5 + 3 * tk);
                     if (!ok && !s_stop) st_fail(a, kErrStreamFull, l, s);
                     if (ok && !gate_up && a.phase == 3) {  // h: every gate/up tile of this expert
                         unsigned ns_ = 32;
@@ -400,7 +411,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                             for (int u = 0; u < 4; ++u) acc[z][grp][u] = 0.f;
                     auto kstep = [&](int st, float(&a0)[NG][4], float(&a1)[NG][4]) {
                         const int c = 4 * st + q;
-                        const bool cv = c < NCH;  // ragged K tail: this lane feeds zeros
+                        const bool cv = kFull || c < NCH;  // ragged K tail: this lane feeds zeros
                         const int cc = cv ? c : 0;
                         if constexpr (kMx) {
                             const uint32_t sa = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rA * (K >> 5) + 2 * c) : 0u;
@@ -449,6 +460,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                             for (int u = 0; u < 4; ++u) rb[grp][u][lane] = d4[grp][u];
                     }
                     pair_sync();  // the members' partials are in shared memory; all are done with the stage's rows
+                    if (tk < 8) stamp(6 + 3 * tk);
                     if (t == it.nt - 1 && r0 + 4 * NG >= m.nrows && mp == 0 && lane == 0)
                         st_mbar_arrive(&s_empty[s]);  // the group's last read of the stage: hand it back
                     if (mp > 0) continue;
@@ -526,6 +538,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
         if (!published) publish();
     }
 
+    if (threadIdx.x == 32) stamp(3);  // (warp 1: the first consumer warp)
     __syncthreads();
     if (a.phase == 3) {  // the last CTA out resets the launch's gate/up counters
         if (threadIdx.x == 0) {
@@ -542,11 +555,11 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
     if (threadIdx.x == 0) span_mark(a.span, 1);
 }
 
-template <int NG, int FMT, int P>
+template <int NG, int FMT, int P, bool kFull>
 cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) {
     static bool configured = false;  // per instantiation: allow the large dynamic shared memory
     if (!configured) {
-        const cudaError_t e = cudaFuncSetAttribute(expert_stream_kernel<NG, FMT, P>,
+        const cudaError_t e = cudaFuncSetAttribute(expert_stream_kernel<NG, FMT, P, kFull>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 210 * 1024);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -561,7 +574,7 @@ cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) 
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, expert_stream_kernel<NG, FMT, P>, a);
+    return cudaLaunchKernelEx(&cfg, expert_stream_kernel<NG, FMT, P, kFull>, a);
 }
 
 }  // namespace
@@ -629,12 +642,15 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
     const int iA = (nA + a.tpa - 1) / a.tpa, iB = (nB + a.tpb - 1) / a.tpb;
     const int64_t items = (int64_t)max_exp * (((a.phase & 1) ? iA : 0) + ((a.phase & 2) ? iB : 0));
     const int grid = (int)(items < sms ? items : sms);
+    const bool full = a.d % 256 == 0 && a.F % 256 == 0;
     if (mx) {
-        if (ng == 1) return launch_st<1, kFmtMxfp4, 3>(a, grid, smem, s);
-        return launch_st<2, kFmtMxfp4, 2>(a, grid, smem, s);
+        if (ng == 1) return full ? launch_st<1, kFmtMxfp4, 3, true>(a, grid, smem, s)
+                                 : launch_st<1, kFmtMxfp4, 3, false>(a, grid, smem, s);
+        return full ? launch_st<2, kFmtMxfp4, 2, true>(a, grid, smem, s) : launch_st<2, kFmtMxfp4, 2, false>(a, grid, smem, s);
     }
-    if (ng == 1) return launch_st<1, kFmtNvfp4, 3>(a, grid, smem, s);
-    return launch_st<2, kFmtNvfp4, 2>(a, grid, smem, s);
+    if (ng == 1) return full ? launch_st<1, kFmtNvfp4, 3, true>(a, grid, smem, s)
+                             : launch_st<1, kFmtNvfp4, 3, false>(a, grid, smem, s);
+    return full ? launch_st<2, kFmtNvfp4, 2, true>(a, grid, smem, s) : launch_st<2, kFmtNvfp4, 2, false>(a, grid, smem, s);
 }
 
 }  // namespace moe

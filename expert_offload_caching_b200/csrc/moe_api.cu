@@ -190,6 +190,9 @@ struct moe_ctx {
     // a warp per tile; the hit experts' gate/up and down in one launch), 0 = the
     // split-K kernel (expert_gemv.cu)
     int gemv_kind = 1;
+    // diagnostic trace of the next streaming hit launches (moe_debug_inject what = 9)
+    unsigned long long *trace_d = nullptr;
+    int64_t trace_arm = 0;
     // cache
     uint8_t *arena = nullptr;
     int64_t C = 0;
@@ -428,6 +431,12 @@ GemvArgs stream_args(moe_ctx *ctx, int layer, int T, int phase, int only_job, in
     if (ctx->inj_stream_skip > 0) {
         g.inj_skip = 1;
         --ctx->inj_stream_skip;
+    }
+    if (phase == 3 && ctx->trace_arm > 0 && ctx->trace_d) {
+        if (cudaMemsetAsync(ctx->trace_d, 0, sizeof(unsigned long long) * kTraceCtas * kTraceSlots, ctx->cs) ==
+            cudaSuccess)
+            g.trace = ctx->trace_d;
+        --ctx->trace_arm;
     }
     return g;
 }
@@ -1345,6 +1354,16 @@ moe_status moe_set_expert_shard(moe_ctx *ctx, int32_t rank, int32_t size) {
     return MOE_OK;
 }
 
+moe_status moe_debug_trace(moe_ctx *ctx, uint64_t *out, int32_t n) {
+    if (!ctx || !out || n < 0) return MOE_ERR_ARG;
+    if (!ctx->trace_d) return MOE_ERR_STATE;
+    const int64_t total = (int64_t)kTraceCtas * kTraceSlots;
+    const int64_t m = n < total ? n : total;
+    CK(cudaStreamSynchronize(ctx->cs));
+    CK(cudaMemcpy(out, ctx->trace_d, sizeof(unsigned long long) * m, cudaMemcpyDeviceToHost));
+    return MOE_OK;
+}
+
 moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds) {
     if (!ctx || !(seconds > 0)) return MOE_ERR_ARG;
     ctx->wait_limit = seconds;
@@ -1368,6 +1387,15 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;
     else if (what == 8) ctx->inj_stream_skip = n;
+    else if (what == 9) {  // diagnostic: trace the next n streaming hit launches
+        if (!ctx->trace_d &&
+            cudaMalloc(reinterpret_cast<void **>(&ctx->trace_d), sizeof(unsigned long long) * kTraceCtas * kTraceSlots) !=
+                cudaSuccess) {
+            ctx->trace_d = nullptr;
+            return MOE_ERR_CUDA;
+        }
+        ctx->trace_arm = n;
+    }
     else if (what == 7) {  // per-miss path expert kernels: 1 streaming, 0 split-K
         if (n < 0 || n > 1) return MOE_ERR_ARG;
         if (n == 0 && ctx->ep_size > 1 && !ctx->fused) return MOE_ERR_UNSUPPORTED;
@@ -1529,6 +1557,7 @@ void moe_layer_destroy(moe_ctx *ctx) {
     if (ctx->ev_routed) cudaEventDestroy(ctx->ev_routed);
     if (ctx->page_h) cudaFreeHost(ctx->page_h);
     if (ctx->kspan) cudaFree(ctx->kspan);
+    if (ctx->trace_d) cudaFree(ctx->trace_d);
     delete ctx;
 }
 

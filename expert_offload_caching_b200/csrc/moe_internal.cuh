@@ -173,7 +173,10 @@ struct GemvArgs {
     uint32_t stage_bytes = 0, meta_off = 0, rr_off = 0;
     int exp_cap = 0;                 // experts the metadata area holds
     int inj_skip = 0;                // test injection: CTA 0 issues no copies for its first item
+    unsigned long long *trace = nullptr;  // diagnostic: [CTA][kTraceSlots] globaltimer stamps, or null
 };
+constexpr int kTraceSlots = 32;
+constexpr int kTraceCtas = 160;
 
 // Persistent decode layer kernel (all expert GEMVs of one layer, misses as
 // their copies land).  Counters in the workspace, zero between launches (the

@@ -351,8 +351,18 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * what = 8: in the next n streaming-kernel launches, CTA 0 issues no copies
  * for its first work item, so a consumer's bounded wait runs out (the CTA
  * records the check, lets its other copies land and returns; the next call
- * reports MOE_ERR_CUDA); what = 0 clears 1, 2, 4, 5 and 8. */
+ * reports MOE_ERR_CUDA); what = 9: diagnostics -- the next n hit-expert
+ * launches of the streaming kernels record per-CTA %globaltimer stamps (read
+ * them with moe_debug_trace); what = 0 clears 1, 2, 4, 5 and 8. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
+
+/* Diagnostics: copies the first n (<= 160 * 32) stamps of the last traced
+ * launch (see moe_debug_inject what = 9) to out (host, n uint64 values; CTA b's
+ * 32 slots at out[32 b ...]: 0 start, 1 set-up done, 2 gate/up counts published,
+ * 3 end, and for its first consumer group's first 8 items k: 4 + 3k stage wait
+ * begins, 5 + 3k data in, 6 + 3k sums in; 0 = not reached).  Synchronizes the
+ * compute stream.  MOE_ERR_STATE if nothing was traced. */
+MOE_API moe_status moe_debug_trace(moe_ctx *ctx, uint64_t *out, int32_t n);
 
 /* Hybrid split: m missing experts, PCIe bandwidth B_P, host expert-processing
  * bandwidth B_H (bytes/s), auto threshold (2.0 on the pages).  Equal finish
