@@ -151,20 +151,26 @@ __device__ __forceinline__ StItem st_item(int g, int phase, int nexp, int nA, in
     return it;
 }
 
-// kFull: d and F are multiples of 256, so every K-step chunk is in range
-template <int NG, int FMT, int P, bool kFull>
+// kFull: d and F are multiples of 256, so every K-step chunk is in range.
+// kSA: activations from shared memory -- x staged once per CTA, and a down
+// item's h rows copied into its stage by the group after h is complete
+// (T <= 2); else they are read from global memory.
+template <int NG, int FMT, int P, bool kFull, bool kSA>
 __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_stream_kernel(GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kStMaxStages], s_empty[kStMaxStages];
-    __shared__ int s_nexp, s_last;
+    __shared__ __align__(8) uint64_t s_xbar, s_hbar[kStMaxGroups];
+    __shared__ int s_nexp, s_last, s_combine;
     __shared__ int s_pair_ok[st_max_groups(P)];
     __shared__ float s_red[st_max_groups(P) * 2 * (P - 1) * NG * 4 * 32];  // [group][buffer][member 1..P-1][NG][4][32]
     __shared__ volatile int s_stop;
     constexpr bool kMx = FMT == kFmtMxfp4;
+    constexpr int kActA = kSA ? 2 : 0, kActB = kSA ? 2 : 1;  // activation loads: gate/up (x), down (h)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int NS = a.ns, C = a.nc;
     ExpMeta *meta = reinterpret_cast<ExpMeta *>(smem + a.meta_off);
     RowRef *rrs = reinterpret_cast<RowRef *>(smem + a.rr_off);
+    __half *xs = reinterpret_cast<__half *>(smem + a.x_off);  // kSA: [T][2][d] fp16 (hi, lo)
 
     pdl_wait();  // the job list, x and the row refs come from the route kernel; h from gate/up
     const unsigned long long deadline = st_now() + a.wait_ns;
@@ -172,38 +178,76 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
     // group 0 / member 0's first 8 items: 4 + 3k stage wait begins, 5 + 3k data in, 6 + 3k sums in
     unsigned long long *tr = (a.trace && blockIdx.x < kTraceCtas) ? a.trace + (size_t)blockIdx.x * kTraceSlots : nullptr;
     auto stamp = [&](int slot) { if (tr) tr[slot] = st_now(); };
-    if (threadIdx.x == 0) stamp(0);
     if (threadIdx.x == 0) {
+        stamp(0);
         span_mark(a.span, 0);
         s_stop = 0;
         for (int s = 0; s < NS; ++s) {
             st_mbar_init(&s_full[s], 1);   // the producer's expect-tx arrive (+ the bytes)
-            st_mbar_init(&s_empty[s], 1);  // the consumer that used the stage
+            st_mbar_init(&s_empty[s], 1);  // the group that used the stage
         }
+        st_mbar_init(&s_xbar, 1);
+        for (int g = 0; g < C; ++g) st_mbar_init(&s_hbar[g], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (kSA && (a.phase & 1)) {  // x as fp16 (hi, lo) rows, one bulk copy (written by the route kernel, complete)
+            const uint32_t xb = (uint32_t)a.T * 4u * (uint32_t)a.d;
+            st_mbar_expect(&s_xbar, xb);
+            st_bulk_g2s(xs, a.act, xb, &s_xbar, evict_first_policy());
+        }
     }
     pdl_launch_dependents();
 
     // ---- the launch's experts: hit jobs in ascending job index, then the
-    // shared expert; or the one job only_job
+    // shared expert; or the one job only_job.  Each lane reads whole job
+    // records (one L2 round trip after the count).
     if (warp == 0) {
         int cnt = 0;
+        auto put = [&](int pos, int j, const Job &jb) {
+            ExpMeta &m = meta[pos];
+            m.job = j;
+            m.rec = a.arena + (int64_t)jb.slot * a.rec_bytes;
+            m.nrows = jb.nrows;
+            m.row_off = jb.row_off;
+            m.cnt = 0;
+        };
+        auto load_job = [&](int j) {
+            union {
+                Job jb;
+                uint4 v[2];
+            } u;
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.jobs + j);  // 32-byte records
+            u.v[0] = __ldcg(src);
+            u.v[1] = __ldcg(src + 1);
+            return u.jb;
+        };
         if (a.only_job >= 0) {
-            if (lane == 0) meta[0].job = a.only_job;
+            if (lane == 0) put(0, a.only_job, load_job(a.only_job));
             cnt = 1;
         } else {
             const int nj = __ldcg(a.n_jobs);
             for (int b = 0; b < nj; b += 32) {
                 const int j = b + lane;
-                const bool hit = j < nj && __ldcg(&a.jobs[j].hit);
+                Job jb;
+                bool hit = false;
+                if (j < nj) {
+                    jb = load_job(j);
+                    hit = jb.hit != 0;
+                }
                 const unsigned ball = __ballot_sync(0xffffffffu, hit);
                 const int pos = cnt + __popc(ball & ((1u << lane) - 1u));
-                if (hit && pos < a.exp_cap) meta[pos].job = j;
+                if (hit && pos < a.exp_cap) put(pos, j, jb);
                 cnt += __popc(ball);
             }
             if (a.shared_item) {
-                if (lane == 0 && cnt < a.exp_cap) meta[cnt].job = -1;
+                if (lane == 0 && cnt < a.exp_cap) {
+                    ExpMeta &m = meta[cnt];
+                    m.job = -1;
+                    m.rec = a.shared_rec;
+                    m.nrows = a.T;
+                    m.row_off = 0;
+                    m.cnt = 0;
+                }
                 ++cnt;
             }
         }
@@ -215,35 +259,16 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
             }
             s_nexp = cnt;
         }
+    } else if (warp == 1 && lane == 0) {
+        // combine here: always (1), or (2) only if the lookup had no miss (the
+        // route kernel, complete, wrote the count)
+        s_combine = a.combine == 1 || (a.combine == 2 && __ldcg(a.n_misses) == 0);
     }
-    __syncthreads();
-    const int nexp = s_nexp;
-    for (int e = threadIdx.x; e < nexp; e += blockDim.x) {
-        ExpMeta &m = meta[e];
-        const int j = m.job;
-        if (j < 0) {
-            m.rec = a.shared_rec;
-            m.nrows = a.T;
-            m.row_off = 0;
-        } else {
-            m.rec = a.arena + (int64_t)__ldcg(&a.jobs[j].slot) * a.rec_bytes;
-            m.nrows = __ldcg(&a.jobs[j].nrows);
-            m.row_off = __ldcg(&a.jobs[j].row_off);
-        }
-        m.cnt = 0;
-        if (!kMx) {
-            const float *t = reinterpret_cast<const float *>(m.rec + a.lay.tscales);
-            m.ts[0] = t[0];
-            m.ts[1] = t[1];
-            m.ts[2] = t[2];
-        }
-    }
-    for (int i = threadIdx.x; i < a.T * a.k; i += blockDim.x) {
-        const RowRef r = a.rowrefs[i];
-        rrs[i] = r;
-    }
+    for (int i = threadIdx.x; i < a.T * a.k; i += blockDim.x) rrs[i] = a.rowrefs[i];
     __syncthreads();
     if (threadIdx.x == 0) stamp(1);
+    const int nexp = s_nexp;
+    const bool combine = s_combine != 0;
 
     // ---- item geometry
     const int nA = a.F >> 3, nB = a.d >> 4;  // tiles per expert: 8 gate/up row pairs, 16 down rows
@@ -253,10 +278,10 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
     const int n_my = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / G + 1 : 0;
     const uint32_t cbA = 8u * (uint32_t)a.d, sbA = kMx ? (uint32_t)(a.d >> 1) : (uint32_t)a.d;
     const uint32_t cbB = 8u * (uint32_t)a.F, sbB = kMx ? (uint32_t)(a.F >> 1) : (uint32_t)a.F;
+    // stage layout: codes of the item's nt tiles, their scales, 16 bytes of
+    // tensor scales (NVFP4), then (kSA, down items) the expert's h rows
+    auto ts_off = [&](const StItem &it) { return (uint32_t)it.nt * (it.gate_up ? cbA + sbA : cbB + sbB); };
 
-    // combine here: always (1), or (2) only if the lookup had no miss (the
-    // route kernel, complete, wrote the count)
-    const bool combine = a.combine == 1 || (a.combine == 2 && __ldcg(a.n_misses) == 0);
     if (nexp == 0 && combine && blockIdx.x == 0) {
         // nothing of this layer is computed here (an expert-parallel shard that
         // owns none of the selected experts): its partial output is the shared
@@ -290,9 +315,11 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                     skipped = 0;
                     continue;
                 }
-                st_mbar_expect(&s_full[s], (uint32_t)it.nt * (cb + sb));
+                st_mbar_expect(&s_full[s], (uint32_t)it.nt * (cb + sb) + (kMx ? 0u : 16u));
                 st_bulk_g2s(dst, codes, (uint32_t)it.nt * cb, &s_full[s], pol);
                 st_bulk_g2s(dst + (size_t)it.nt * cb, scales, (uint32_t)it.nt * sb, &s_full[s], pol);
+                if (!kMx)  // the record's tensor scales (gate, up, down; 12 of 16 bytes)
+                    st_bulk_g2s(dst + (size_t)it.nt * (cb + sb), rec + a.lay.tscales, 16u, &s_full[s], pol);
             }
             // no copy outlives the CTA: the last item issued into each stage has landed
             const unsigned long long drain = st_now() + 1000000000ull;
@@ -310,7 +337,9 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
         const int g = lane >> 2, q = lane & 3;
         const uint32_t pair_bar = 2u + (uint32_t)gq;
         auto pair_sync = [&]() { asm volatile("barrier.sync %0, %1;" ::"r"(pair_bar), "r"(32 * P) : "memory"); };
-        int rbuf = 0;  // partials double buffer, flipped per row group
+        int rbuf = 0;         // partials double buffer, flipped per row group
+        int hcount = 0;       // kSA: down items of this group so far (the h barrier's phases)
+        bool x_seen = !kSA;   // kSA: this warp has observed x in shared memory
         // phase 3: gate/up tiles this CTA completed, per launch expert, published
         // once, when every consumer warp has passed its last gate/up item
         bool published = a.phase != 3;
@@ -332,16 +361,26 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
             const StItem it = st_item(gi, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
             const bool gate_up = it.gate_up;
             if (!gate_up && !published) publish();
-            // member 0 takes the waits (bounded) and hands the verdict to member 1
-            // at the pair barrier, so both break or proceed together
+            const ExpMeta m = meta[it.e];
+            const bool shared = m.job < 0;
+            uint8_t *stage = smem + (size_t)s * a.stage_bytes;
+            const uint32_t toff = ts_off(it);
             const int tk = (gq == 0 && mp == 0 && lane == 0) ? (l / C) : 99;  // traced item ordinal
             if (tk < 8) stamp(4 + 3 * tk);
+            const bool need_x = kSA && gate_up && !x_seen;
+            const bool need_h = kSA && !gate_up;
+            // member 0 takes the waits (bounded) and hands the verdict to the
+            // other members at the group barrier, so the group breaks or proceeds as one
             if (mp == 0) {
                 int ok = 1;
                 if (lane == 0) {
                     ok = st_mbar_wait(&s_full[s], n & 1, deadline, &s_stop);
-                    if (tk < 8) stamp(5 + 3 * tk);
                     if (!ok && !s_stop) st_fail(a, kErrStreamFull, l, s);
+                    if (tk < 8) stamp(5 + 3 * tk);
+                    if (ok && need_x) {
+                        ok = st_mbar_wait(&s_xbar, 0, deadline, &s_stop);
+                        if (!ok && !s_stop) st_fail(a, kErrStreamFull, l, -1);
+                    }
                     if (ok && !gate_up && a.phase == 3) {  // h: every gate/up tile of this expert
                         unsigned ns_ = 32;
                         for (uint32_t i = 0;; ++i) {
@@ -356,6 +395,25 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                         }
                         __threadfence();
                     }
+                    if (ok && need_h) {
+                        // the expert's h rows (complete: the launch before, or the
+                        // counts above) into the stage, behind the tensor scales;
+                        // the generic-proxy writes of other CTAs are ordered before
+                        // this thread's async-proxy reads
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        const uint32_t hb = 4u * (uint32_t)a.F;
+                        st_mbar_expect(&s_hbar[gq], (uint32_t)m.nrows * hb);
+                        for (int r = 0; r < m.nrows; ++r) {
+                            int tr, p;
+                            if (shared) { tr = r; p = a.k; }
+                            else { const RowRef rf = rrs[m.row_off + r]; tr = rf.t; p = rf.p; }
+                            const size_t sel = (size_t)tr * (a.k + 1) + p;
+                            st_bulk_g2s(stage + toff + 16 + (size_t)r * hb, a.hh_out + sel * 2 * a.F, hb, &s_hbar[gq],
+                                        evict_first_policy());
+                        }
+                        ok = st_mbar_wait(&s_hbar[gq], hcount & 1, deadline, &s_stop);
+                        if (!ok && !s_stop) st_fail(a, kErrStreamFull, l, -2);
+                    }
                     if (!ok) s_stop = 1;
                     s_pair_ok[gq] = ok;
                 }
@@ -363,18 +421,32 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
             pair_sync();
             const int ok = s_pair_ok[gq];
             if (!ok) break;
-            // every lane observes the completed phase (it has: member 0 saw it)
+            // every lane observes the completed phases (member 0 saw them complete)
             for (uint32_t i = 0; i < (1u << 20) && !st_mbar_test(&s_full[s], n & 1); ++i) {
             }
-            const ExpMeta m = meta[it.e];
-            const bool shared = m.job < 0;
+            if (need_x) {
+                for (uint32_t i = 0; i < (1u << 20) && !st_mbar_test(&s_xbar, 0); ++i) {
+                }
+                x_seen = true;
+            }
+            if (need_h) {
+                for (uint32_t i = 0; i < (1u << 20) && !st_mbar_test(&s_hbar[gq], hcount & 1); ++i) {
+                }
+                ++hcount;
+            }
+            float ts0 = 1.f, ts1 = 1.f, ts2 = 1.f;
+            if (!kMx && mp == 0) {  // read before the stage is released
+                const float *tsv = reinterpret_cast<const float *>(stage + toff);
+                ts0 = tsv[0];
+                ts1 = tsv[1];
+                ts2 = tsv[2];
+            }
             const int K = gate_up ? a.d : a.F;
             const int NCH = K >> 6, nsteps = (NCH + 3) >> 2;
             const int st0 = mp * nsteps / P, st1 = (mp + 1) * nsteps / P;
             const uint32_t cb = gate_up ? cbA : cbB, sb = gate_up ? sbA : sbB;
-            const uint8_t *stage = smem + (size_t)s * a.stage_bytes;
             const int rA = gate_up ? 2 * g : g, rB = gate_up ? 2 * g + 1 : g + 8;
-            const __half *act = gate_up ? a.act : a.hh_out;
+            const __half *hs = reinterpret_cast<const __half *>(stage + toff + 16);  // kSA: h rows [r][2][F]
             for (int t = 0; t < it.nt; ++t) {
                 const int tile = it.tile0 + t;
                 const uint8_t *s_codes = stage + (size_t)t * cb;
@@ -389,14 +461,18 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                     for (int grp = 0; grp < NG; ++grp) {
                         const int r = r0 + 4 * grp + (g >> 1);
                         colv[grp] = r < m.nrows;
-                        col[grp] = act;
+                        col[grp] = gate_up ? (kSA ? xs : a.act) : (kSA ? hs : a.hh_out);
                         if (r0 + 4 * grp < m.nrows) ngrp = grp + 1;
                         if (colv[grp]) {
                             int tr, p;
                             if (shared) { tr = r; p = a.k; }
                             else { const RowRef rf = rrs[m.row_off + r]; tr = rf.t; p = rf.p; }
-                            col[grp] = gate_up ? act + (size_t)tr * 2 * a.d + (g & 1) * a.d
-                                               : act + (size_t)(tr * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
+                            if (gate_up)
+                                col[grp] = (kSA ? xs : a.act) + (size_t)tr * 2 * a.d + (g & 1) * a.d;
+                            else if (kSA)
+                                col[grp] = hs + (size_t)r * 2 * a.F + (g & 1) * a.F;
+                            else
+                                col[grp] = a.hh_out + (size_t)(tr * (a.k + 1) + p) * 2 * a.F + (g & 1) * a.F;
                         }
                     }
                     // accumulator sets: chunk half (x step parity with pairs, whose
@@ -417,20 +493,20 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                             const uint32_t sa = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rA * (K >> 5) + 2 * c) : 0u;
                             const uint32_t sbv = cv ? *reinterpret_cast<const uint16_t *>(s_scales + rB * (K >> 5) + 2 * c) : 0u;
                             if (gate_up)
-                                step_mma_mx_x2<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                step_mma_mx_x2<NG, kActA>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
                                                           sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                             else
-                                step_mma_mx_x2<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
-                                                         sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
+                                step_mma_mx_x2<NG, kActB>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                          sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                         } else {
                             const uint32_t sa = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rA * (K >> 4) + 4 * c) : 0u;
                             const uint32_t sbv = cv ? *reinterpret_cast<const uint32_t *>(s_scales + rB * (K >> 4) + 4 * c) : 0u;
                             if (gate_up)
-                                step_mma_x2<NG, false>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                step_mma_x2<NG, kActA>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
                                                        sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                             else
-                                step_mma_x2<NG, true>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
-                                                      sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
+                                step_mma_x2<NG, kActB>(s_codes + rA * (K >> 1) + 32 * cc, s_codes + rB * (K >> 1) + 32 * cc,
+                                                       sa, sbv, cc, cv, col, colv, ngrp, a0, a1);
                         }
                     };
                     if constexpr (kChains == 4) {
@@ -482,7 +558,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                         const float v1 = d4[grp][2] + d4[grp][3];
                         const size_t sel = (size_t)tr * (a.k + 1) + p;
                         if (gate_up) {
-                            const float gt = kMx ? v0 : m.ts[0] * v0, up = kMx ? v1 : m.ts[1] * v1;
+                            const float gt = kMx ? v0 : ts0 * v0, up = kMx ? v1 : ts1 * v1;
                             const float h = gt / (1.0f + expf(-gt)) * up;
                             const int o = 8 * tile + g;
                             const __half hi = __float2half_rn(h);
@@ -491,7 +567,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                             a.hh_out[sel * 2 * a.F + a.F + o] = lo;
                         } else {
                             const int o = 16 * tile + g;
-                            const float sd = kMx ? 1.0f : m.ts[2];
+                            const float sd = kMx ? 1.0f : ts2;
                             a.part_out[sel * a.d + o] = sd * v0;
                             a.part_out[sel * a.d + o + 8] = sd * v1;
                         }
@@ -540,6 +616,10 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
 
     if (threadIdx.x == 32) stamp(3);  // (warp 1: the first consumer warp)
     __syncthreads();
+    if (kSA && (a.phase & 1) && threadIdx.x == 0) {  // no copy outlives the CTA: x has landed
+        volatile int never = 0;
+        st_mbar_wait(&s_xbar, 0, st_now() + 1000000000ull, &never);
+    }
     if (a.phase == 3) {  // the last CTA out resets the launch's gate/up counters
         if (threadIdx.x == 0) {
             __threadfence();
@@ -555,11 +635,11 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
     if (threadIdx.x == 0) span_mark(a.span, 1);
 }
 
-template <int NG, int FMT, int P, bool kFull>
+template <int NG, int FMT, int P, bool kFull, bool kSA>
 cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) {
     static bool configured = false;  // per instantiation: allow the large dynamic shared memory
     if (!configured) {
-        const cudaError_t e = cudaFuncSetAttribute(expert_stream_kernel<NG, FMT, P, kFull>,
+        const cudaError_t e = cudaFuncSetAttribute(expert_stream_kernel<NG, FMT, P, kFull, kSA>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 210 * 1024);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -574,7 +654,13 @@ cudaError_t launch_st(const GemvArgs &a, int grid, size_t smem, cudaStream_t s) 
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, expert_stream_kernel<NG, FMT, P, kFull>, a);
+    return cudaLaunchKernelEx(&cfg, expert_stream_kernel<NG, FMT, P, kFull, kSA>, a);
+}
+
+template <int NG, int FMT, int P>
+cudaError_t launch_st_fs(const GemvArgs &a, int grid, size_t smem, bool full, bool sa, cudaStream_t s) {
+    if (full) return sa ? launch_st<NG, FMT, P, true, true>(a, grid, smem, s) : launch_st<NG, FMT, P, true, false>(a, grid, smem, s);
+    return sa ? launch_st<NG, FMT, P, false, true>(a, grid, smem, s) : launch_st<NG, FMT, P, false, false>(a, grid, smem, s);
 }
 
 }  // namespace
@@ -599,37 +685,42 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
     }
-    // stage = the larger tile (codes + scales), at least 16 KB; several
+    // activations in shared memory for up to 2 rows: x once per CTA, and a
+    // down item's h rows in its stage
+    const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
+    const bool sa = a.T <= 2;
+    const size_t xbytes = sa ? (size_t)a.T * 4 * a.d : 0, hbytes = sa ? (size_t)a.T * 4 * a.F : 0;
+    // stage = the larger item: a tile's codes + scales, 16 bytes of tensor
+    // scales, and for a down item its h rows; at least 16 KB; several
     // consecutive tiles of one expert per item where they fit
     const size_t tA = 8 * (size_t)a.d + (mx ? a.d / 2 : a.d), tB = 8 * (size_t)a.F + (mx ? a.F / 2 : a.F);
-    size_t sb = tA > tB ? tA : tB;
+    size_t sb = tA + 16 > tB + 16 + hbytes ? tA + 16 : tB + 16 + hbytes;
     if (sb < 16 * 1024) sb = 16 * 1024;
     sb = (sb + 127) & ~(size_t)127;
     const int nA = a.F / 8, nB = a.d / 16;
     // items: enough of them that every SM's consumers get a few
     const int64_t want = 3 * (int64_t)sms;
-    auto per_item = [&](size_t tile_bytes, int tiles_per_exp, int phases_exp) {
-        int tp = (int)(sb / tile_bytes);
+    auto per_item = [&](size_t room, size_t tile_bytes, int tiles_per_exp, int phases_exp) {
+        int tp = (int)(room / tile_bytes);
         const int64_t tiles = (int64_t)tiles_per_exp * phases_exp;
         while (tp > 1 && tiles / tp < want) --tp;
         return tp < 1 ? 1 : tp;
     };
-    a.tpa = per_item(tA, nA, max_exp);
-    a.tpb = per_item(tB, nB, max_exp);
-    const size_t meta = (size_t)max_exp * sizeof(ExpMeta);
+    a.tpa = per_item(sb - 16, tA, nA, max_exp);
+    a.tpb = per_item(sb - 16 - hbytes, tB, nB, max_exp);
+    // (areas rounded to 16 bytes: x is a bulk-copy destination)
+    const size_t meta = ((size_t)max_exp * sizeof(ExpMeta) + 15) & ~(size_t)15;
     const size_t rr = (((size_t)a.T * a.k * sizeof(RowRef)) + 15) & ~(size_t)15;
     const size_t budget = 200 * 1024;
-    if (meta + rr + 2 * sb > budget) return cudaErrorInvalidValue;
-    int ns = (int)((budget - meta - rr) / sb);
+    if (meta + rr + xbytes + 2 * sb > budget) return cudaErrorInvalidValue;
+    int ns = (int)((budget - meta - rr - xbytes) / sb);
     if (ns > kStMaxStages) ns = kStMaxStages;
-    // stages per consumer warp: two (one loads while the other is computed)
-    // where six or more fit, else one; the stage count is a multiple of the
-    // consumer count, so a stage always serves the same warp and its phases are
-    // consumed in order (a parity wait can then not see an older phase)
     // consumer warp groups: P = 3 warps each for up to 4 activation rows per
     // pass (NG 1), 2 otherwise; a group serves two stages (one loads while the
-    // other is computed) where the stages allow, else one
-    const int ng = a.T <= 4 ? 1 : 2;  // more rows: passes over the staged tile
+    // other is computed) where the stages allow, else one.  The stage count is
+    // a multiple of the group count, so a stage always serves the same group
+    // and its phases are consumed in order (a parity wait can then not see an
+    // older phase).
     const int gmax = kStMaxGroups;
     int nc = ns >= 2 * gmax ? gmax : (ns >= 6 ? ns / 2 : (ns < gmax ? ns : gmax));
     a.nc = nc;
@@ -637,20 +728,19 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
     a.stage_bytes = (uint32_t)sb;
     a.meta_off = (uint32_t)(ns * sb);
     a.rr_off = (uint32_t)(ns * sb + meta);
+    a.x_off = (uint32_t)(ns * sb + meta + rr);
     a.exp_cap = max_exp;
-    const size_t smem = ns * sb + meta + rr;
+    const size_t smem = ns * sb + meta + rr + xbytes;
     const int iA = (nA + a.tpa - 1) / a.tpa, iB = (nB + a.tpb - 1) / a.tpb;
     const int64_t items = (int64_t)max_exp * (((a.phase & 1) ? iA : 0) + ((a.phase & 2) ? iB : 0));
     const int grid = (int)(items < sms ? items : sms);
     const bool full = a.d % 256 == 0 && a.F % 256 == 0;
     if (mx) {
-        if (ng == 1) return full ? launch_st<1, kFmtMxfp4, 3, true>(a, grid, smem, s)
-                                 : launch_st<1, kFmtMxfp4, 3, false>(a, grid, smem, s);
-        return full ? launch_st<2, kFmtMxfp4, 2, true>(a, grid, smem, s) : launch_st<2, kFmtMxfp4, 2, false>(a, grid, smem, s);
+        if (ng == 1) return launch_st_fs<1, kFmtMxfp4, 3>(a, grid, smem, full, sa, s);
+        return launch_st_fs<2, kFmtMxfp4, 2>(a, grid, smem, full, false, s);
     }
-    if (ng == 1) return full ? launch_st<1, kFmtNvfp4, 3, true>(a, grid, smem, s)
-                             : launch_st<1, kFmtNvfp4, 3, false>(a, grid, smem, s);
-    return full ? launch_st<2, kFmtNvfp4, 2, true>(a, grid, smem, s) : launch_st<2, kFmtNvfp4, 2, false>(a, grid, smem, s);
+    if (ng == 1) return launch_st_fs<1, kFmtNvfp4, 3>(a, grid, smem, full, sa, s);
+    return launch_st_fs<2, kFmtNvfp4, 2>(a, grid, smem, full, false, s);
 }
 
 }  // namespace moe

@@ -203,10 +203,20 @@ __device__ __forceinline__ void step_mma(const uint8_t *cA, const uint8_t *cB, u
     }
 }
 
+// Activation fragment load, three ways: 0 read-only path (data from an earlier
+// kernel), 1 L2 (written by another CTA of this kernel), 2 shared memory (the
+// pointer is into this CTA's shared memory).
+template <int kAct>
+__device__ __forceinline__ uint4 ld_act3(const __half *p) {
+    if constexpr (kAct == 0) return __ldg(reinterpret_cast<const uint4 *>(p));
+    else if constexpr (kAct == 1) return __ldcg(reinterpret_cast<const uint4 *>(p));
+    else return *reinterpret_cast<const uint4 *>(p);
+}
+
 // step_mma / step_mma_mx with two accumulator sets: the first 32 codes of the
 // chunk (h = 0) go into acc0, the last 32 (h = 1) into acc1, so the mma
 // dependency chain is half as long (the dot product is order-free).
-template <int NG, bool kCg = false>
+template <int NG, int kAct = 0>
 __device__ __forceinline__ void step_mma_x2(const uint8_t *cA, const uint8_t *cB, uint32_t sa, uint32_t sb, int c,
                                             bool cv, const __half *const (&col)[NG], const bool (&colv)[NG], int ngrp,
                                             float (&acc0)[NG][4], float (&acc1)[NG][4]) {
@@ -236,7 +246,7 @@ __device__ __forceinline__ void step_mma_x2(const uint8_t *cA, const uint8_t *cB
             for (int grp = 0; grp < NG; ++grp) {
                 if (grp < ngrp) {
                     uint4 bv = make_uint4(0, 0, 0, 0);
-                    if (colv[grp] && cv) bv = ld_act<kCg>(col[grp] + 64 * c + 8 * w);
+                    if (colv[grp] && cv) bv = ld_act3<kAct>(col[grp] + 64 * c + 8 * w);
                     mma16816(acc[grp], fa[0], fb[0], fa[1], fb[1], bv.x, bv.y);
                     mma16816(acc[grp], fa[2], fb[2], fa[3], fb[3], bv.z, bv.w);
                 }
@@ -245,7 +255,7 @@ __device__ __forceinline__ void step_mma_x2(const uint8_t *cA, const uint8_t *cB
     }
 }
 
-template <int NG, bool kCg = false>
+template <int NG, int kAct = 0>
 __device__ __forceinline__ void step_mma_mx_x2(const uint8_t *cA, const uint8_t *cB, uint32_t sa, uint32_t sb, int c,
                                                bool cv, const __half *const (&col)[NG], const bool (&colv)[NG],
                                                int ngrp, float (&acc0)[NG][4], float (&acc1)[NG][4]) {
@@ -285,7 +295,7 @@ __device__ __forceinline__ void step_mma_mx_x2(const uint8_t *cA, const uint8_t 
             for (int grp = 0; grp < NG; ++grp) {
                 if (grp < ngrp) {
                     uint4 bv = make_uint4(0, 0, 0, 0);
-                    if (colv[grp] && cv) bv = ld_act<kCg>(col[grp] + 64 * c + 8 * w);
+                    if (colv[grp] && cv) bv = ld_act3<kAct>(col[grp] + 64 * c + 8 * w);
                     mma16816(stp[h][grp], fa[0], fb[0], fa[1], fb[1], bv.x, bv.y);
                     mma16816(stp[h][grp], fa[2], fb[2], fa[3], fb[3], bv.z, bv.w);
                 }

@@ -170,7 +170,7 @@ struct GemvArgs {
     // set by launch_stream
     int tpa = 0, tpb = 0;            // weight tiles per work item (gate/up, down)
     int ns = 0, nc = 0;              // shared-memory stages, consumer warps
-    uint32_t stage_bytes = 0, meta_off = 0, rr_off = 0;
+    uint32_t stage_bytes = 0, meta_off = 0, rr_off = 0, x_off = 0;
     int exp_cap = 0;                 // experts the metadata area holds
     int inj_skip = 0;                // test injection: CTA 0 issues no copies for its first item
     unsigned long long *trace = nullptr;  // diagnostic: [CTA][kTraceSlots] globaltimer stamps, or null

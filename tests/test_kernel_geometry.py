@@ -289,33 +289,39 @@ def test_layer_kernel_ring_fits_and_keeps_two_ctas_per_sm_where_it_can(shape, mx
 # ------------------------------------------------ streaming expert kernel --
 def _stream_launch(d, F, T, k, max_exp, mx, sms=148):
     """launch_stream's sizing, restated: stage bytes, tiles per item (gate/up,
-    down), stages, consumer warps, metadata and row-ref offsets, grid."""
+    down), stages, consumer groups, metadata, row-ref and x offsets, grid.  A
+    stage holds an item's codes and scales, 16 bytes of tensor scales and, with
+    activations in shared memory (T <= 2), a down item's h rows."""
+    sa = T <= 2
+    xbytes = T * 4 * d if sa else 0
+    hbytes = T * 4 * F if sa else 0
     tA = 8 * d + (d // 2 if mx else d)
     tB = 8 * F + (F // 2 if mx else F)
-    sb = max(tA, tB, 16 * 1024)
+    sb = max(tA + 16, tB + 16 + hbytes, 16 * 1024)
     sb = (sb + 127) & ~127
     nA, nB = F // 8, d // 16
     want = 3 * sms
 
-    def per_item(tile_bytes, tiles_per_exp):
-        tp = sb // tile_bytes
+    def per_item(room, tile_bytes, tiles_per_exp):
+        tp = room // tile_bytes
         tiles = tiles_per_exp * max_exp
         while tp > 1 and tiles // tp < want:
             tp -= 1
         return max(tp, 1)
 
-    tpa, tpb = per_item(tA, nA), per_item(tB, nB)
-    meta = max_exp * 40
+    tpa, tpb = per_item(sb - 16, tA, nA), per_item(sb - 16 - hbytes, tB, nB)
+    meta = (max_exp * 40 + 15) & ~15
     rr = (T * k * 4 + 15) & ~15
     budget = 200 * 1024
-    assert meta + rr + 2 * sb <= budget
-    ns = min((budget - meta - rr) // sb, 8)
-    nc = ns // 2 if ns >= 6 else ns
+    assert meta + rr + xbytes + 2 * sb <= budget
+    ns = min((budget - meta - rr - xbytes) // sb, 8)
+    nc = ns // 2 if ns >= 6 else min(ns, 5)
     if nc > 4 and ns >= 6:
         nc = 4
-    ns = (2 if ns >= 6 else 1) * nc
+    ns = (2 if ns >= 2 * nc else 1) * nc
     return dict(sb=sb, tpa=tpa, tpb=tpb, ns=ns, nc=nc, meta_off=ns * sb, rr_off=ns * sb + meta,
-                smem=ns * sb + meta + rr, nA=nA, nB=nB, cbA=8 * d, sbA=d // 2 if mx else d,
+                x_off=ns * sb + meta + rr, xbytes=xbytes, hbytes=hbytes,
+                smem=ns * sb + meta + rr + xbytes, nA=nA, nB=nB, cbA=8 * d, sbA=d // 2 if mx else d,
                 cbB=8 * F, sbB=F // 2 if mx else F)
 
 
@@ -353,6 +359,7 @@ def test_stream_items_fit_their_stage_and_stay_in_the_record(shape, mx):
         for l in range(64):
             assert (l % L["ns"]) % L["nc"] == l % L["nc"]
         assert L["smem"] <= 200 * 1024 and L["meta_off"] % 128 == 0 and L["rr_off"] % 8 == 0
+        assert L["x_off"] % 16 == 0 and L["xbytes"] % 16 == 0 and (4 * shape.F) % 16 == 0
         for phase in (1, 2, 3):
             nexp = min(max_exp, 3)
             items = _stream_items(L, nexp, phase)
@@ -362,8 +369,10 @@ def test_stream_items_fit_their_stage_and_stay_in_the_record(shape, mx):
                 assert nt >= 1
                 cb, sb = (L["cbA"], L["sbA"]) if gu else (L["cbB"], L["sbB"])
                 codes0, scales0, end = (off[0], off[1], off[2]) if gu else (off[2], off[3], off[5])
-                # the stage: codes of nt tiles, then their scales
-                assert nt * (cb + sb) <= L["sb"]
+                # the stage: codes of nt tiles, their scales, 16 bytes of tensor
+                # scales, then (down items, T <= 2) the expert's h rows
+                assert nt * (cb + sb) + 16 + (0 if gu else L["hbytes"]) <= L["sb"]
+                assert (nt * (cb + sb)) % 16 == 0
                 assert (nt * cb) % 16 == 0 and (nt * sb) % 16 == 0
                 # the two bulk copies: 16-byte aligned, inside their record section
                 c0, s0 = codes0 + t0 * cb, scales0 + t0 * sb
