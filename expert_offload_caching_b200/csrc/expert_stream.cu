@@ -94,18 +94,6 @@ __device__ __forceinline__ bool st_mbar_test(uint64_t *bar, uint32_t parity) {
         : "memory");
     return done != 0;
 }
-// Non-blocking test of the phase of the given parity.
-__device__ __forceinline__ bool st_mbar_probe(uint64_t *bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
-}
 // Wait for the phase of the given parity; false when the deadline passes or
 // the CTA is stopping.
 __device__ __forceinline__ bool st_mbar_wait(uint64_t *bar, uint32_t parity, unsigned long long deadline,
@@ -306,55 +294,38 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        // Each group's items go to its own stages in its own order (item l:
-        // group l mod C, stage l mod S); the producer serves whichever group's
-        // next stage is free, so a slow group does not hold back the others.
         if (lane == 0) {
             const uint64_t pol = evict_first_policy();
-            int next[kStMaxGroups], last_l[kStMaxStages];
-            for (int g = 0; g < C; ++g) next[g] = g;
-            for (int st = 0; st < NS; ++st) last_l[st] = -1;
-            int skipped = -1, left = n_my;
-            for (uint32_t spin = 0; left > 0 && !s_stop;) {
-                bool progress = false;
-                for (int g = 0; g < C; ++g) {
-                    const int l = next[g];
-                    if (l >= n_my) continue;
-                    const int s = l % NS, n = l / NS;
-                    if (n > 0 && !st_mbar_probe(&s_empty[s], (n - 1) & 1)) continue;  // the stage's last use not released yet
-                    const StItem it = st_item((int)blockIdx.x + l * G, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
-                    const uint32_t cb = it.gate_up ? cbA : cbB, sb = it.gate_up ? sbA : sbB;
-                    const uint8_t *rec = meta[it.e].rec;
-                    const uint8_t *codes = rec + (it.gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)it.tile0 * cb;
-                    const uint8_t *scales = rec + (it.gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)it.tile0 * sb;
-                    uint8_t *dst = smem + (size_t)s * a.stage_bytes;
-                    next[g] = l + C;
-                    --left;
-                    progress = true;
-                    last_l[s] = l;
-                    if (a.inj_skip && blockIdx.x == 0 && l == 0) {  // test injection: this stage never fills
-                        skipped = 0;
-                        continue;
-                    }
-                    st_mbar_expect(&s_full[s], (uint32_t)it.nt * (cb + sb) + (kMx ? 0u : 16u));
-                    st_bulk_g2s(dst, codes, (uint32_t)it.nt * cb, &s_full[s], pol);
-                    st_bulk_g2s(dst + (size_t)it.nt * cb, scales, (uint32_t)it.nt * sb, &s_full[s], pol);
-                    if (!kMx)  // the record's tensor scales (gate, up, down; 12 of 16 bytes)
-                        st_bulk_g2s(dst + (size_t)it.nt * (cb + sb), rec + a.lay.tscales, 16u, &s_full[s], pol);
-                }
-                if (progress) {
-                    spin = 0;
-                } else if ((++spin & 31u) == 0u && st_now() > deadline) {  // every pending stage still held
-                    st_fail(a, kErrStreamEmpty, n_my - left, C);
+            int issued = 0, skipped = -1;
+            for (int l = 0; l < n_my; ++l) {
+                const int s = l % NS, n = l / NS;
+                if (n > 0 && !st_mbar_wait(&s_empty[s], (n - 1) & 1, deadline, &s_stop)) {
+                    if (!s_stop) st_fail(a, kErrStreamEmpty, l, s);
                     s_stop = 1;
+                    break;
                 }
+                const StItem it = st_item((int)blockIdx.x + l * G, a.phase, nexp, nA, nB, iA, iB, a.tpa, a.tpb);
+                const uint32_t cb = it.gate_up ? cbA : cbB, sb = it.gate_up ? sbA : sbB;
+                const uint8_t *rec = meta[it.e].rec;
+                const uint8_t *codes = rec + (it.gate_up ? a.lay.w13_codes : a.lay.w2_codes) + (int64_t)it.tile0 * cb;
+                const uint8_t *scales = rec + (it.gate_up ? a.lay.w13_scales : a.lay.w2_scales) + (int64_t)it.tile0 * sb;
+                uint8_t *dst = smem + (size_t)s * a.stage_bytes;
+                issued = l + 1;
+                if (a.inj_skip && blockIdx.x == 0 && l == 0) {  // test injection: this stage never fills
+                    skipped = 0;
+                    continue;
+                }
+                st_mbar_expect(&s_full[s], (uint32_t)it.nt * (cb + sb) + (kMx ? 0u : 16u));
+                st_bulk_g2s(dst, codes, (uint32_t)it.nt * cb, &s_full[s], pol);
+                st_bulk_g2s(dst + (size_t)it.nt * cb, scales, (uint32_t)it.nt * sb, &s_full[s], pol);
+                if (!kMx)  // the record's tensor scales (gate, up, down; 12 of 16 bytes)
+                    st_bulk_g2s(dst + (size_t)it.nt * (cb + sb), rec + a.lay.tscales, 16u, &s_full[s], pol);
             }
             // no copy outlives the CTA: the last item issued into each stage has landed
             const unsigned long long drain = st_now() + 1000000000ull;
             volatile int never = 0;
-            for (int st = 0; st < NS; ++st)
-                if (last_l[st] >= 0 && last_l[st] != skipped)
-                    st_mbar_wait(&s_full[st], (last_l[st] / NS) & 1, drain, &never);
+            for (int l = issued > NS ? issued - NS : 0; l < issued; ++l)
+                if (l != skipped) st_mbar_wait(&s_full[l % NS], (l / NS) & 1, drain, &never);
         }
     } else if (warp <= P * C) {
         // ---------------------------------------------------------- consumers
