@@ -232,133 +232,6 @@ __device__ int topk_row(const RouteArgs &a, int t) {
     return topk_row_n<kMaxE / 32>(a, t);
 }
 
-// Softmax + top-k of one row by every warp of the CTA (the single-row decode
-// step): warp w holds entries lane + 32 (w + nw j) in registers, takes its own
-// k best in the same total order as topk_row_n (NaN as -inf, equal values to
-// the lower id, picked entries masked by a bit), and warp 0 picks the k best of
-// the nw * k candidates -- the row's top k lies among them.  The softmax max
-// and denominator are block reductions.  Same ids as topk_row_n; the gates
-// differ from it only in fp32 summation order.
-constexpr int kTkMaxJ = kMaxE / kRouteThreads;  // entries per lane (E <= 1024, 8 warps)
-struct TopkSmem {
-    float cv[kRouteThreads / 32][kMaxK];
-    int ci[kRouteThreads / 32][kMaxK];
-    float red[kRouteThreads / 32];
-};
-__device__ void topk_row_block(const RouteArgs &a, int t, TopkSmem &sm) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const float *z = a.ws.z + (size_t)t * a.E;
-    float v[kTkMaxJ];
-    uint32_t avail = 0u;
-    float m = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kTkMaxJ; ++j) {
-        const int e = lane + 32 * (warp + nw * j);
-        const bool real = e < a.E;
-        const float zv = real ? __ldcg(z + e) : -INFINITY;
-        v[j] = zv != zv ? -INFINITY : zv;
-        if (real) avail |= 1u << j;
-        m = fmaxf(m, v[j]);
-    }
-    m = warp_max(m);
-    if (lane == 0) sm.red[warp] = m;
-    __syncthreads();
-    m = sm.red[0];
-    for (int w = 1; w < nw; ++w) m = fmaxf(m, sm.red[w]);
-    float sall = 0.f;  // the full softmax denominator (only without renormalisation)
-    if (!a.renorm) {
-        __syncthreads();  // (everyone has read the maxima)
-#pragma unroll
-        for (int j = 0; j < kTkMaxJ; ++j)
-            if ((avail >> j) & 1u) sall += expf(v[j] - m);
-        sall = warp_sum(sall);
-        if (lane == 0) sm.red[warp] = sall;
-        __syncthreads();
-        sall = 0.f;
-        for (int w = 0; w < nw; ++w) sall += sm.red[w];
-    }
-    // this warp's k best
-    for (int s = 0; s < a.k; ++s) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;  // lane-local candidates in ascending id
-#pragma unroll
-        for (int j = 0; j < kTkMaxJ; ++j)
-            if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) {
-                bv = v[j];
-                bi = lane + 32 * (warp + nw * j);
-            }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if (lane == 0) {
-            sm.cv[warp][s] = bv;
-            sm.ci[warp][s] = bi;  // 0x7fffffff: this warp has fewer than k entries
-        }
-        if (bi != 0x7fffffff && ((bi & 31) == lane)) avail &= ~(1u << (((bi >> 5) - warp) / nw));
-    }
-    __syncthreads();
-    if (warp != 0) return;
-    // warp 0: the k best of the nw * k candidates (candidate c = w * k + s)
-    constexpr int kCand = (kRouteThreads / 32) * kMaxK / 32;  // candidates per lane
-    const int ncand = nw * a.k;
-    float cvl[kCand];
-    int cil[kCand];
-    uint32_t cav = 0u;
-#pragma unroll
-    for (int j = 0; j < kCand; ++j) {
-        const int c = lane + 32 * j;
-        cvl[j] = -INFINITY;
-        cil[j] = 0x7fffffff;
-        if (c < ncand) {
-            const int w = c / a.k, s = c - w * a.k;
-            cvl[j] = sm.cv[w][s];
-            cil[j] = sm.ci[w][s];
-            if (cil[j] != 0x7fffffff) cav |= 1u << j;
-        }
-    }
-    int my_idx = 0x7fffffff;
-    float my_val = -INFINITY;
-    for (int s = 0; s < a.k; ++s) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff, bj = -1;
-#pragma unroll
-        for (int j = 0; j < kCand; ++j)
-            if (((cav >> j) & 1u) && (cvl[j] > bv || (cvl[j] == bv && cil[j] < bi) || bj < 0)) {
-                bv = cvl[j];
-                bi = cil[j];
-                bj = j;
-            }
-        int own = lane;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            const int ol = __shfl_xor_sync(0xffffffffu, own, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; own = ol; }
-        }
-        if (lane == s) { my_idx = bi; my_val = bv; }
-        const int wj = __shfl_sync(0xffffffffu, bj, own);  // the winner's slot in its owner lane
-        if (lane == own && wj >= 0) cav &= ~(1u << wj);
-    }
-    const float top = __shfl_sync(0xffffffffu, my_val, 0);
-    float g;
-    if (a.renorm) {
-        const float ex = lane < a.k ? expf(my_val - top) : 0.f;
-        g = ex / warp_sum(ex);
-    } else {
-        g = expf(my_val - m) / sall;
-    }
-    int rank = 0;
-    for (int i = 0; i < a.k; ++i) rank += (__shfl_sync(0xffffffffu, my_idx, i) < my_idx);
-    if (lane < a.k) {
-        a.ws.idx[t * a.k + rank] = my_idx;
-        a.ws.gates[t * a.k + rank] = g;
-    }
-}
-
 constexpr int kLookupMax = kMaxK * kDecodeMaxRows;  // entries of one lookup batch (>= kMaxE)
 
 // Shared memory of one lookup batch.
@@ -569,13 +442,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     if (threadIdx.x == 0) t_elect = global_ns();
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    if (a.T == 1) {  // one row: every warp takes part
-        __shared__ TopkSmem tks;
-        topk_row_block(a, 0, tks);
-        __syncthreads();
-    } else {
-        for (int t = warp; t < a.T; t += nw) topk_row(a, t);
-    }
+    for (int t = warp; t < a.T; t += nw) topk_row(a, t);
 
     // ---- distinct experts of the batch, ascending: a bitmap over E
     __shared__ uint32_t s_bits[kMaxE / 32];
