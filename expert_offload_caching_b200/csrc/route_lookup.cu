@@ -54,6 +54,17 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float *f) {
     }
 }
 
+// Order-preserving 32-bit key of a float (larger key <=> larger value, -0 and
+// +0 equal, -inf the smallest of the values used here; NaN is mapped to -inf
+// before) and back.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 __device__ __forceinline__ uint4 ld_nc16(const void *p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -198,12 +209,12 @@ __device__ int topk_row_n(const RouteArgs &a, int t) {
 #pragma unroll
         for (int j = 0; j < NVE; ++j)
             if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = lane + 32 * j; }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
+        // the warp's largest value (order-preserving integer key, two
+        // single-instruction warp reductions), then the lowest id holding it
+        const uint32_t key = order_key(bv);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0xffffffffu);
+        bv = key_value(kmax);
         if (lane == s) { my_idx = bi; my_val = bv; }
         if (bi < a.E && lane == (bi & 31)) avail &= ~(1u << (bi >> 5));
     }

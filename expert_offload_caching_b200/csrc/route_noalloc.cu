@@ -51,6 +51,15 @@ __device__ __forceinline__ float na_warp_sum(float v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
+// Order-preserving 32-bit key of a float (-0 and +0 equal; NaN is mapped to
+// -inf before) and back.
+__device__ __forceinline__ uint32_t na_key(float v) {
+    const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float na_key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 __device__ __forceinline__ float na_warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -132,12 +141,12 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
                 const int e = lane + 32 * j;
                 if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = e; }
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-            }
+            // the warp's largest value (order-preserving integer key, warp
+            // reductions), then the lowest id holding it
+            const uint32_t key = na_key(bv);
+            const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+            bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0xffffffffu);
+            bv = na_key_value(kmax);
             if (bi != 0x7fffffff && (bi & 31) == lane) avail &= ~(1u << (bi >> 5));
             if (lane == s) { my_idx = bi; my_val = bv; }
         }

@@ -403,3 +403,35 @@ def test_stream_k_step_reads_stay_inside_the_tile():
         assert 15 * (K // 2) + 32 * (nch - 1) + 32 == 8 * K
         assert 15 * (K // 16) + 4 * (nch - 1) + 4 == K
         assert 15 * (K // 32) + 2 * (nch - 1) + 2 == K // 2
+
+
+def test_topk_order_key_preserves_the_selection_order():
+    """The route kernels' warp argmax compares order-preserving 32-bit keys of
+    the logits (a max reduction, then the lowest id holding it): the key must be
+    monotone in the value, give -0 and +0 the same key, keep -inf the smallest,
+    and invert exactly."""
+    import numpy as np
+
+    def key(v):
+        v = np.where(v == 0, np.float32(0), v).astype(np.float32)
+        u = v.view(np.uint32)
+        return np.where(u & np.uint32(0x80000000), ~u, u | np.uint32(0x80000000)).astype(np.uint32)
+
+    def value(k):
+        u = np.where(k & np.uint32(0x80000000), k & np.uint32(0x7fffffff), ~k).astype(np.uint32)
+        return u.view(np.float32)
+
+    rng = np.random.default_rng(7)
+    vals = np.concatenate([
+        np.array([-np.inf, -3.4e38, -1.0, -1e-45, -0.0, 0.0, 1e-45, 1.0, 3.4e38, np.inf], np.float32),
+        rng.standard_normal(4000).astype(np.float32) * np.float32(50),
+        (rng.standard_normal(500) * 1e-40).astype(np.float32)])  # subnormals
+    k = key(vals)
+    order_v = np.argsort(vals, kind="stable")
+    assert np.all(np.diff(k[order_v].astype(np.int64)) >= 0)          # monotone
+    assert key(np.array([-0.0], np.float32))[0] == key(np.array([0.0], np.float32))[0]
+    finite_or_inf = vals[vals == vals]
+    assert key(np.array([-np.inf], np.float32))[0] == key(finite_or_inf).min()
+    back = value(k)
+    same = np.where(vals == 0, np.float32(0), vals)
+    assert np.array_equal(back.view(np.uint32), same.view(np.uint32))  # exact inverse
