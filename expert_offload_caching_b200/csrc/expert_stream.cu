@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
     __shared__ __align__(8) uint64_t s_full[kStMaxStages], s_empty[kStMaxStages];
     __shared__ __align__(8) uint64_t s_xbar, s_hbar[kStMaxGroups];
     __shared__ int s_nexp, s_last, s_combine;
+    __shared__ int s_head_exp, s_head_slot;  // phase 3 with head_bytes: the layer's first miss
     __shared__ int s_pair_ok[st_max_groups(P)];
     __shared__ float s_red[st_max_groups(P) * 2 * (P - 1) * NG * 4 * 32];  // [group][buffer][member 1..P-1][NG][4][32]
     __shared__ volatile int s_stop;
@@ -221,6 +222,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
             u.v[1] = __ldcg(src + 1);
             return u.jb;
         };
+        int head = -1;  // the first miss (lowest job index): its expert and slot
         if (a.only_job >= 0) {
             if (lane == 0) put(0, a.only_job, load_job(a.only_job));
             cnt = 1;
@@ -229,15 +231,27 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
             for (int b = 0; b < nj; b += 32) {
                 const int j = b + lane;
                 Job jb;
-                bool hit = false;
+                bool hit = false, miss = false;
                 if (j < nj) {
                     jb = load_job(j);
                     hit = jb.hit != 0;
+                    miss = !hit;
                 }
                 const unsigned ball = __ballot_sync(0xffffffffu, hit);
                 const int pos = cnt + __popc(ball & ((1u << lane) - 1u));
                 if (hit && pos < a.exp_cap) put(pos, j, jb);
                 cnt += __popc(ball);
+                const unsigned mb = __ballot_sync(0xffffffffu, miss);
+                if (head < 0 && mb) {
+                    const int src = __ffs(mb) - 1;
+                    const int ex = __shfl_sync(0xffffffffu, jb.expert, src);
+                    const int sl = __shfl_sync(0xffffffffu, jb.slot, src);
+                    if (lane == 0) {
+                        s_head_exp = ex;
+                        s_head_slot = sl;
+                    }
+                    head = 1;
+                }
             }
             if (a.shared_item) {
                 if (lane == 0 && cnt < a.exp_cap) {
@@ -251,6 +265,7 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
                 ++cnt;
             }
         }
+        if (lane == 0 && head < 0) s_head_exp = -1;
         if (lane == 0) {
             if (cnt > a.exp_cap) {  // cannot happen with the host's sizing; refuse rather than overrun
                 st_fail(a, kErrStreamSize, cnt, a.exp_cap);
@@ -294,7 +309,27 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        if (lane == 0) {
+        if (lane > 0) {
+            // lanes 1..31 of every CTA: the head of the layer's first miss, from the
+            // page-locked pool over PCIe straight into its slot (16-byte loads, four
+            // in flight per lane); the copy engine moves the rest of the record
+            if (a.phase == 3 && a.head_bytes && s_head_exp >= 0) {
+                const int64_t rec_idx = ((int64_t)a.layer * a.E + s_head_exp) % a.pool_P;
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.pool_d + rec_idx * a.rec_bytes);
+                uint4 *dst = reinterpret_cast<uint4 *>(const_cast<uint8_t *>(a.arena) + (int64_t)s_head_slot * a.rec_bytes);
+                const int64_t n16 = a.head_bytes >> 4, step = (int64_t)gridDim.x * 31;
+                int64_t i = (int64_t)blockIdx.x * 31 + (lane - 1);
+                for (; i + 3 * step < n16; i += 4 * step) {
+                    const uint4 v0 = __ldcv(src + i), v1 = __ldcv(src + i + step), v2 = __ldcv(src + i + 2 * step),
+                                v3 = __ldcv(src + i + 3 * step);
+                    dst[i] = v0;
+                    dst[i + step] = v1;
+                    dst[i + 2 * step] = v2;
+                    dst[i + 3 * step] = v3;
+                }
+                for (; i < n16; i += step) dst[i] = __ldcv(src + i);
+            }
+        } else {
             const uint64_t pol = evict_first_policy();
             int issued = 0, skipped = -1;
             for (int l = 0; l < n_my; ++l) {

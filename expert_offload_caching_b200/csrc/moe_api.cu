@@ -190,6 +190,11 @@ struct moe_ctx {
     // a warp per tile; the hit experts' gate/up and down in one launch), 0 = the
     // split-K kernel (expert_gemv.cu)
     int gemv_kind = 1;
+    // decode: the hit launch's SMs copy the first head_bytes of the layer's first
+    // miss from the pool (pool_d: its device address) while the copy engine
+    // starts on the rest (moe_debug_inject what = 10; 0: off)
+    const uint8_t *pool_d = nullptr;
+    uint32_t head_bytes = 0;
     // diagnostic trace of the next streaming hit launches (moe_debug_inject what = 9)
     unsigned long long *trace_d = nullptr;
     int64_t trace_arm = 0;
@@ -679,6 +684,13 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         time_begin(ctx, th, MOE_K_LAYER_HITS);
         GemvArgs ha = stream_args(ctx, layer, T, 3, -1, 2);
         ha.y = y;
+        if (ctx->head_bytes && ctx->pool_d && !(ctx->flags & MOE_CACHE_STATIC_SPLIT)) {
+            ha.pool_d = ctx->pool_d;
+            ha.pool_P = ctx->P;
+            ha.layer = layer;
+            ha.E = D.E;
+            ha.head_bytes = ctx->head_bytes;
+        }
         ha.span = time_span(ctx, th);
         CK(launch_stream(ha, grid_y, ctx->cs));
         ih = time_end(ctx, th, 0);
@@ -721,6 +733,8 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     // (tensor scales + W13, a prefix of the record) and the down half -- with an
     // event after each, so a miss's gate/up runs while its down half streams in
     const int64_t split = ctx->lay.w2_codes;
+    // the first miss's head came over with the SMs of the hit launch
+    const bool stream_head = stream && ctx->head_bytes && ctx->pool_d && !(ctx->flags & MOE_CACHE_STATIC_SPLIT);
     int mo = 0;
     bool used2 = false;
     for (int j = 0; j < nev; ++j) {
@@ -733,11 +747,13 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         const int64_t rec_idx = ((int64_t)layer * D.E + ev[j].expert) % ctx->P;
         uint8_t *dst = ctx->arena + (int64_t)ev[j].slot * ctx->lay.bytes;
         const uint8_t *src = ctx->pool + rec_idx * ctx->lay.bytes;
+        const int64_t head = (stream_head && mo == 0) ? (int64_t)ctx->head_bytes : 0;
         cudaStream_t s;
         CK(miss_stream(ctx, mo++, &used2, &s));
-        CK(cudaMemcpyAsync(dst, src, split, cudaMemcpyHostToDevice, s));
+        if (head < split) CK(cudaMemcpyAsync(dst + head, src + head, split - head, cudaMemcpyHostToDevice, s));
         CK(cudaEventRecord(ctx->miss_ev[2 * j], s));
-        CK(cudaMemcpyAsync(dst + split, src + split, ctx->lay.bytes - split, cudaMemcpyHostToDevice, s));
+        const int64_t w2 = head > split ? head : split;
+        CK(cudaMemcpyAsync(dst + w2, src + w2, ctx->lay.bytes - w2, cudaMemcpyHostToDevice, s));
         CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], s));
         ctx->stats.h2d_copies += 1;
         ctx->stats.h2d_bytes += ctx->lay.bytes;
@@ -1032,6 +1048,12 @@ moe_status moe_layer_init(const moe_dims *dims, const void *host_pool, size_t ho
     ctx->slay = shared_layout_of(dims);
     ctx->P = P;
     ctx->pool = static_cast<const uint8_t *>(host_pool);
+    {  // the pool's device address (SM reads of the first miss's head); none: the option stays off
+        void *pd = nullptr;
+        if (cudaHostGetDevicePointer(&pd, const_cast<void *>(host_pool), 0) == cudaSuccess)
+            ctx->pool_d = static_cast<const uint8_t *>(pd);
+        cudaGetLastError();
+    }
     ctx->router_w = static_cast<const __nv_bfloat16 *>(router_w);
     ctx->shared_recs = static_cast<const uint8_t *>(shared_recs);
     ctx->ws = static_cast<uint8_t *>(workspace);
@@ -1387,6 +1409,11 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;
     else if (what == 8) ctx->inj_stream_skip = n;
+    else if (what == 10) {  // decode: the SMs copy the first n bytes of a layer's first miss
+        if (n < 0 || (n & 15) || n >= ctx->lay.bytes) return MOE_ERR_ARG;
+        if (n > 0 && !ctx->pool_d) return MOE_ERR_UNSUPPORTED;
+        ctx->head_bytes = (uint32_t)n;
+    }
     else if (what == 9) {  // diagnostic: trace the next n streaming hit launches
         if (!ctx->trace_d &&
             cudaMalloc(reinterpret_cast<void **>(&ctx->trace_d), sizeof(unsigned long long) * kTraceCtas * kTraceSlots) !=

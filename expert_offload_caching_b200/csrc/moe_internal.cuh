@@ -174,6 +174,13 @@ struct GemvArgs {
     int exp_cap = 0;                 // experts the metadata area holds
     int inj_skip = 0;                // test injection: CTA 0 issues no copies for its first item
     unsigned long long *trace = nullptr;  // diagnostic: [CTA][kTraceSlots] globaltimer stamps, or null
+    // phase 3: the first head_bytes of the layer's first miss, copied by the SMs
+    // from the page-locked pool (its device address) into the miss's slot while
+    // the host starts the copy engine on the rest (0: off)
+    const uint8_t *pool_d = nullptr;
+    int64_t pool_P = 0;
+    int layer = 0, E = 0;
+    uint32_t head_bytes = 0;
 };
 constexpr int kTraceSlots = 32;
 constexpr int kTraceCtas = 160;

@@ -353,7 +353,12 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * records the check, lets its other copies land and returns; the next call
  * reports MOE_ERR_CUDA); what = 9: diagnostics -- the next n hit-expert
  * launches of the streaming kernels record per-CTA %globaltimer stamps (read
- * them with moe_debug_trace); what = 0 clears 1, 2, 4, 5 and 8. */
+ * them with moe_debug_trace); what = 10: decode (default path) -- the hit
+ * launch's SMs copy the first n bytes (a multiple of 16, less than a record)
+ * of the layer's first miss from the pool (through its device address) into
+ * the miss's slot, and the copy engine moves only the rest (n = 0: off, the
+ * default; MOE_ERR_UNSUPPORTED if the pool has no device address); what = 0
+ * clears 1, 2, 4, 5 and 8. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Diagnostics: copies the first n (<= 160 * 32) stamps of the last traced

@@ -381,6 +381,24 @@ def test_two_copy_streams_match_the_oracle(path):
     st.close()
 
 
+@pytest.mark.parametrize("frac", [0.1, 0.9], ids=["head-in-gate-up", "head-past-gate-up"])
+def test_sm_head_copy_of_the_first_miss_matches_the_oracle(frac):
+    """The hit launch's SMs copy the head of each layer's first miss from the
+    page-locked pool (through its device address) and the copy engine the rest:
+    the slots are bit-exact and the outputs match the oracle, with the head
+    ending inside the gate/up prefix and past it."""
+    pb = DecodeProblem(MID, T=12)
+    st = pb.stack()
+    rb = synth.record_bytes(MID.d, MID.F)
+    head = int(frac * rb) // 16 * 16
+    abi.moe_debug_inject(st.ctx, 10, head)
+    run = pb.run(stack=st, routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(st, run.table[1])
+    assert run.stats.misses > 0
+    st.close()
+
+
 def test_streaming_kernel_wait_runs_out_then_reset_recovers():
     """CTA 0 of the next streaming launches issues no copies for its first work
     item: the consumer's bounded wait on that stage runs out (limit 0.3 s), the
