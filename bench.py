@@ -81,6 +81,9 @@ def parse():
                          "streaming ones")
     ap.add_argument("--copy-streams", type=int, default=0, choices=[0, 1, 2],
                     help="decode misses on 1 or 2 copy streams (0: the library's default)")
+    ap.add_argument("--head-bytes", type=int, default=0,
+                    help="decode: the hit launch's SMs copy this many bytes of each layer's first miss from "
+                         "the host pool while the copy engine moves the rest (0: off)")
     ap.add_argument("--ep", action="store_true",
                     help="decode with N > 1: expert parallelism (rank r serves experts e %% N == r, its "
                          "own cache; the partial outputs all-reduced per layer) instead of replicas")
@@ -459,6 +462,8 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
         abi.moe_debug_inject(stack.ctx, 7, 0)
     if getattr(args, "copy_streams", 0):
         abi.moe_debug_inject(stack.ctx, 6, args.copy_streams)
+    if getattr(args, "head_bytes", 0):
+        abi.moe_debug_inject(stack.ctx, 10, args.head_bytes)
 
     # H2D bandwidth of this machine, measured now (the roofline's PCIe term)
     nb = 1 << 30
@@ -625,7 +630,8 @@ def bench_decode(args, shape, rank, world, local):
                                        f"partial outputs all-reduced per layer)") if ep else f"replicas x{world}",
                        "pool_distinct_records": DISTINCT_RECORDS, "policy": args.policy,
                        "expert_kernels": expert_kernels_label(args),
-                       "copy_streams": args.copy_streams or "default"},
+                       "copy_streams": args.copy_streams or "default",
+                       "sm_head_bytes": args.head_bytes},
             "miss_rate": counts["misses"] / max(counts["lookups"], 1),
             "counts": {"source": source, **counts,
                        "gpu_counters_match": all(gpu_counts[f] == counts[f] for f in counts)},
