@@ -195,6 +195,9 @@ struct moe_ctx {
     // starts on the rest (moe_debug_inject what = 10; 0: off)
     const uint8_t *pool_d = nullptr;
     uint32_t head_bytes = 0;
+    // decode misses: the gate/up prefix and W2 as two copies (a miss's gate/up
+    // runs while its W2 streams), or the whole record as one (what = 11)
+    bool split_copies = true;
     // diagnostic trace of the next streaming hit launches (moe_debug_inject what = 9)
     unsigned long long *trace_d = nullptr;
     int64_t trace_arm = 0;
@@ -750,11 +753,17 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         const int64_t head = (stream_head && mo == 0) ? (int64_t)ctx->head_bytes : 0;
         cudaStream_t s;
         CK(miss_stream(ctx, mo++, &used2, &s));
-        if (head < split) CK(cudaMemcpyAsync(dst + head, src + head, split - head, cudaMemcpyHostToDevice, s));
-        CK(cudaEventRecord(ctx->miss_ev[2 * j], s));
-        const int64_t w2 = head > split ? head : split;
-        CK(cudaMemcpyAsync(dst + w2, src + w2, ctx->lay.bytes - w2, cudaMemcpyHostToDevice, s));
-        CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], s));
+        if (!ctx->split_copies) {  // one copy; both events after it
+            CK(cudaMemcpyAsync(dst + head, src + head, ctx->lay.bytes - head, cudaMemcpyHostToDevice, s));
+            CK(cudaEventRecord(ctx->miss_ev[2 * j], s));
+            CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], s));
+        } else {
+            if (head < split) CK(cudaMemcpyAsync(dst + head, src + head, split - head, cudaMemcpyHostToDevice, s));
+            CK(cudaEventRecord(ctx->miss_ev[2 * j], s));
+            const int64_t w2 = head > split ? head : split;
+            CK(cudaMemcpyAsync(dst + w2, src + w2, ctx->lay.bytes - w2, cudaMemcpyHostToDevice, s));
+            CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], s));
+        }
         ctx->stats.h2d_copies += 1;
         ctx->stats.h2d_bytes += ctx->lay.bytes;
     }
@@ -1409,7 +1418,10 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;
     else if (what == 8) ctx->inj_stream_skip = n;
-    else if (what == 10) {  // decode: the SMs copy the first n bytes of a layer's first miss
+    else if (what == 11) {  // decode misses: two copies per record (n = 1, default) or one (n = 0)
+        if (n < 0 || n > 1) return MOE_ERR_ARG;
+        ctx->split_copies = n == 1;
+    } else if (what == 10) {  // decode: the SMs copy the first n bytes of a layer's first miss
         if (n < 0 || (n & 15) || n >= ctx->lay.bytes) return MOE_ERR_ARG;
         if (n > 0 && !ctx->pool_d) return MOE_ERR_UNSUPPORTED;
         ctx->head_bytes = (uint32_t)n;

@@ -381,6 +381,18 @@ def test_two_copy_streams_match_the_oracle(path):
     st.close()
 
 
+def test_whole_record_copies_match_the_oracle():
+    """Each missed record as one copy (both of its events after it) instead of
+    the gate/up prefix and W2 as two: same trace, table, slots and outputs."""
+    pb = DecodeProblem(MID, T=12)
+    st = pb.stack()
+    abi.moe_debug_inject(st.ctx, 11, 0)
+    run = pb.run(stack=st, routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(st, run.table[1])
+    st.close()
+
+
 @pytest.mark.parametrize("frac", [0.1, 0.9], ids=["head-in-gate-up", "head-past-gate-up"])
 def test_sm_head_copy_of_the_first_miss_matches_the_oracle(frac):
     """The hit launch's SMs copy the head of each layer's first miss from the
