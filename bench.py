@@ -84,8 +84,8 @@ def parse():
     ap.add_argument("--head-bytes", type=int, default=0,
                     help="decode: the hit launch's SMs copy this many bytes of each layer's first miss from "
                          "the host pool while the copy engine moves the rest (0: off)")
-    ap.add_argument("--whole-record-copies", action="store_true",
-                    help="decode: one copy per missed record instead of two (gate/up prefix, W2)")
+    ap.add_argument("--split-record-copies", action="store_true",
+                    help="decode: two copies per missed record (gate/up prefix, W2) instead of one")
     ap.add_argument("--ep", action="store_true",
                     help="decode with N > 1: expert parallelism (rank r serves experts e %% N == r, its "
                          "own cache; the partial outputs all-reduced per layer) instead of replicas")
@@ -466,8 +466,8 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
         abi.moe_debug_inject(stack.ctx, 6, args.copy_streams)
     if getattr(args, "head_bytes", 0):
         abi.moe_debug_inject(stack.ctx, 10, args.head_bytes)
-    if getattr(args, "whole_record_copies", False):
-        abi.moe_debug_inject(stack.ctx, 11, 0)
+    if getattr(args, "split_record_copies", False):
+        abi.moe_debug_inject(stack.ctx, 11, 1)
 
     # H2D bandwidth of this machine, measured now (the roofline's PCIe term)
     nb = 1 << 30
@@ -636,7 +636,7 @@ def bench_decode(args, shape, rank, world, local):
                        "expert_kernels": expert_kernels_label(args),
                        "copy_streams": args.copy_streams or "default",
                        "sm_head_bytes": args.head_bytes,
-                       "copies_per_miss": 1 if args.whole_record_copies else 2},
+                       "copies_per_miss": 2 if args.split_record_copies else 1},
             "miss_rate": counts["misses"] / max(counts["lookups"], 1),
             "counts": {"source": source, **counts,
                        "gpu_counters_match": all(gpu_counts[f] == counts[f] for f in counts)},

@@ -195,9 +195,10 @@ struct moe_ctx {
     // starts on the rest (moe_debug_inject what = 10; 0: off)
     const uint8_t *pool_d = nullptr;
     uint32_t head_bytes = 0;
-    // decode misses: the gate/up prefix and W2 as two copies (a miss's gate/up
-    // runs while its W2 streams), or the whole record as one (what = 11)
-    bool split_copies = true;
+    // decode misses: the whole record as one copy (the default: fewer copy
+    // start-ups; measured faster or equal), or the gate/up prefix and W2 as two,
+    // so a miss's gate/up runs while its W2 streams (what = 11)
+    bool split_copies = false;
     // diagnostic trace of the next streaming hit launches (moe_debug_inject what = 9)
     unsigned long long *trace_d = nullptr;
     int64_t trace_arm = 0;
@@ -1418,7 +1419,7 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
         ctx->fused = n == 1;
     } else if (what == 4) ctx->inj_drop_flags = n;
     else if (what == 8) ctx->inj_stream_skip = n;
-    else if (what == 11) {  // decode misses: two copies per record (n = 1, default) or one (n = 0)
+    else if (what == 11) {  // decode misses: two copies per record (n = 1) or one (n = 0, default)
         if (n < 0 || n > 1) return MOE_ERR_ARG;
         ctx->split_copies = n == 1;
     } else if (what == 10) {  // decode: the SMs copy the first n bytes of a layer's first miss

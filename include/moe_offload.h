@@ -358,9 +358,9 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * of the layer's first miss from the pool (through its device address) into
  * the miss's slot, and the copy engine moves only the rest (n = 0: off, the
  * default; MOE_ERR_UNSUPPORTED if the pool has no device address); what = 11:
- * decode (default path) copies each missed record as two copies, the gate/up
- * prefix then W2 (n = 1, the default: a miss's gate/up runs while its W2
- * streams), or as one (n = 0); what = 0 clears 1, 2, 4, 5 and 8. */
+ * decode (default path) copies each missed record as one copy (n = 0, the
+ * default) or as two, the gate/up prefix then W2, so a miss's gate/up runs
+ * while its W2 streams (n = 1); what = 0 clears 1, 2, 4, 5 and 8. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Diagnostics: copies the first n (<= 160 * 32) stamps of the last traced

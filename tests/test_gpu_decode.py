@@ -381,12 +381,12 @@ def test_two_copy_streams_match_the_oracle(path):
     st.close()
 
 
-def test_whole_record_copies_match_the_oracle():
-    """Each missed record as one copy (both of its events after it) instead of
-    the gate/up prefix and W2 as two: same trace, table, slots and outputs."""
+def test_split_record_copies_match_the_oracle():
+    """Each missed record as two copies (the gate/up prefix, then W2, each with
+    its event) instead of one: same trace, table, slots and outputs."""
     pb = DecodeProblem(MID, T=12)
     st = pb.stack()
-    abi.moe_debug_inject(st.ctx, 11, 0)
+    abi.moe_debug_inject(st.ctx, 11, 1)
     run = pb.run(stack=st, routing=True)
     assert _check_run(pb, run) < 1e-5
     pb.check_slots(st, run.table[1])
