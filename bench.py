@@ -490,8 +490,11 @@ def open_stack(args, shape, world, max_rows, prefetch=False):
 def expert_kernels_label(args) -> str:
     if getattr(args, "layer_kernel", False):
         return "persistent layer kernel (misses gated by copy flags)"
-    kind = "split-K" if getattr(args, "split_k", False) else "streaming"
-    return f"{kind} expert kernels: one launch for the hit experts, a gate/up and a down launch per miss"
+    if getattr(args, "split_k", False):
+        return "split-K expert kernels: a gate/up and a down launch for the hit experts and per miss"
+    if getattr(args, "split_record_copies", False):
+        return "streaming expert kernels: one launch for the hit experts, a gate/up and a down launch per miss"
+    return "streaming expert kernels: one launch for the hit experts, one per miss (gate/up, then down)"
 
 
 def main():
@@ -661,13 +664,15 @@ def bench_decode(args, shape, rank, world, local):
 
 def launch_count(kst, st):
     """The library's kernel launches in a timed run: counted per class by the
-    timing pass (the same work as the timed run; the hit-phase class is a part of
-    the layer kernel's launches, not launches of its own); without that pass,
-    the per-call structure of the decode path (route + layer kernel)."""
+    timing pass (the same work as the timed run; with the layer kernel, the
+    hit-phase class is a part of its launches, not launches of its own);
+    without that pass, the per-call structure of the decode path (route + hit
+    launch) plus one launch per miss."""
     from expert_offload_caching_b200 import abi
     if kst is not None:
-        return int(sum(kst.kernel_launches[i] for i in range(abi.MOE_K_COUNT) if i != abi.MOE_K_LAYER_HITS))
-    return int(st.forward_calls * 2)
+        part = abi.MOE_K_LAYER_HITS if kst.kernel_launches[abi.MOE_K_LAYER] else -1
+        return int(sum(kst.kernel_launches[i] for i in range(abi.MOE_K_COUNT) if i != part))
+    return int(st.forward_calls * 2 + st.misses)
 
 
 def host_us_per_call(st):

@@ -16,9 +16,9 @@ MOE_CACHE_STATIC_SPLIT = 4
 MOE_FMT_NVFP4, MOE_FMT_MXFP4, MOE_FMT_BF16 = 0, 1, 2
 MOE_K_ROUTE, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE = 0, 1, 2, 3
 MOE_K_PREFILL_ROUTE, MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN = 4, 5, 6
-MOE_K_LAYER, MOE_K_LAYER_HITS, MOE_K_COUNT = 7, 8, 9
+MOE_K_LAYER, MOE_K_LAYER_HITS, MOE_K_MISS, MOE_K_COUNT = 7, 8, 9, 10
 KERNEL_NAMES = ["route_lookup", "gate_up", "down", "combine", "prefill_route", "prefill_gate_up",
-                "prefill_down", "expert_layer", "expert_hits"]
+                "prefill_down", "expert_layer", "expert_hits", "expert_miss"]
 ROUTE_PHASES = ["logits", "elect", "topk", "jobs", "table_read", "select_write", "publish",
                 "wait_previous_layer"]
 

@@ -427,7 +427,8 @@ GemvArgs gemv_args(moe_ctx *ctx, int layer, int T, int mode, int only_job, int c
 }
 
 // Arguments of a streaming-kernel launch (expert_stream.cu): phase 1 gate/up,
-// 2 down, 3 both (the hit experts); only_job >= 0: that miss alone.
+// 2 down, 3 both (the hit experts); only_job >= 0: that miss alone (phase 3:
+// its record has landed whole).
 GemvArgs stream_args(moe_ctx *ctx, int layer, int T, int phase, int only_job, int combine) {
     GemvArgs g = gemv_args(ctx, layer, T, phase == 2 ? kDown : kGateUp, only_job, combine);
     g.act = ctx->dws.xh;
@@ -441,7 +442,7 @@ GemvArgs stream_args(moe_ctx *ctx, int layer, int T, int phase, int only_job, in
         g.inj_skip = 1;
         --ctx->inj_stream_skip;
     }
-    if (phase == 3 && ctx->trace_arm > 0 && ctx->trace_d) {
+    if (phase == 3 && only_job < 0 && ctx->trace_arm > 0 && ctx->trace_d) {
         if (cudaMemsetAsync(ctx->trace_d, 0, sizeof(unsigned long long) * kTraceCtas * kTraceSlots, ctx->cs) ==
             cudaSuccess)
             g.trace = ctx->trace_d;
@@ -733,9 +734,10 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         if (ih >= 0) ctx->pending[ih].bytes = nexp * (w13_bytes(ctx) + w2_bytes(ctx)) + (double)T * D.d * 2;
     }
 
-    // misses: each record in two copies on the copy stream -- the gate/up half
-    // (tensor scales + W13, a prefix of the record) and the down half -- with an
-    // event after each, so a miss's gate/up runs while its down half streams in
+    // misses: each record in one copy on the copy stream, an event after it;
+    // or (split_copies) in two -- the gate/up half (tensor scales + W13, a
+    // prefix of the record) and the down half -- with an event after each, so a
+    // miss's gate/up runs while its down half streams in
     const int64_t split = ctx->lay.w2_codes;
     // the first miss's head came over with the SMs of the hit launch
     const bool stream_head = stream && ctx->head_bytes && ctx->pool_d && !(ctx->flags & MOE_CACHE_STATIC_SPLIT);
@@ -754,10 +756,9 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
         const int64_t head = (stream_head && mo == 0) ? (int64_t)ctx->head_bytes : 0;
         cudaStream_t s;
         CK(miss_stream(ctx, mo++, &used2, &s));
-        if (!ctx->split_copies) {  // one copy; both events after it
+        if (!ctx->split_copies) {  // one copy, one event (both halves)
             CK(cudaMemcpyAsync(dst + head, src + head, ctx->lay.bytes - head, cudaMemcpyHostToDevice, s));
             CK(cudaEventRecord(ctx->miss_ev[2 * j], s));
-            CK(cudaEventRecord(ctx->miss_ev[2 * j + 1], s));
         } else {
             if (head < split) CK(cudaMemcpyAsync(dst + head, src + head, split - head, cudaMemcpyHostToDevice, s));
             CK(cudaEventRecord(ctx->miss_ev[2 * j], s));
@@ -772,15 +773,25 @@ moe_status forward_decode(moe_ctx *ctx, int32_t layer, const void *x, int32_t T,
     for (int j = 0; j < nev; ++j) {
         if (ev[j].flags & 1) continue;
         CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j], 0));
+        const int comb = j == last_miss ? 1 : 0;
+        if (stream && !ctx->split_copies) {  // the whole record is in: one launch, gate/up then down
+            TimedLaunch mm;
+            time_begin(ctx, mm, MOE_K_MISS);
+            GemvArgs ma = stream_args(ctx, layer, T, 3, j, comb);
+            ma.y = y;
+            ma.span = time_span(ctx, mm);
+            CK(launch_stream(ma, 1, ctx->cs));
+            time_end(ctx, mm, w13_bytes(ctx) + w2_bytes(ctx) + (double)T * D.d * 2);
+            continue;
+        }
         TimedLaunch mg, md;
         time_begin(ctx, mg, MOE_K_GATEUP);
         GemvArgs mg_args = stream ? stream_args(ctx, layer, T, 1, j, 0) : gemv_args(ctx, layer, T, kGateUp, j);
         mg_args.span = time_span(ctx, mg);
         CK(stream ? launch_stream(mg_args, 1, ctx->cs) : launch_gemv(mg_args, 1, ctx->cs));
         time_end(ctx, mg, w13_bytes(ctx) + (double)T * D.d * 2);
-        CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j + 1], 0));
+        if (ctx->split_copies) CK(cudaStreamWaitEvent(ctx->cs, ctx->miss_ev[2 * j + 1], 0));
         time_begin(ctx, md, MOE_K_DOWN);
-        const int comb = j == last_miss ? 1 : 0;
         GemvArgs md_args = stream ? stream_args(ctx, layer, T, 2, j, comb) : gemv_args(ctx, layer, T, kDown, j, comb);
         md_args.y = y;
         md_args.span = time_span(ctx, md);

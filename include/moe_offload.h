@@ -127,14 +127,16 @@ typedef struct {
  * lookups/hits/misses count routed lookups (each distinct (layer, expert) of a
  * batch once); prefetch_* count next-layer prefetch entries separately. */
 /* Kernel classes of the timing counters.  MOE_K_GATEUP / MOE_K_DOWN: the
- * per-miss launches (and, with the split-K kernels, the hit launches);
+ * per-miss launches when a missed record comes in two copies (and, with the
+ * split-K kernels, the hit launches); MOE_K_MISS: the default path's one
+ * launch per miss (its gate/up, then its down, after its record landed whole);
  * MOE_K_LAYER: the decode layer kernel (every expert GEMV of a layer in one
  * launch, misses as their copies land); MOE_K_LAYER_HITS: the hit and shared
  * experts' gate/up and down -- the default path's hit launch, or the layer
  * kernel up to the end of its last resident-expert item (the part bounded by
- * HBM, not by the copies). */
+ * HBM, not by the copies; then not a launch of its own). */
 enum { MOE_K_ROUTE = 0, MOE_K_GATEUP, MOE_K_DOWN, MOE_K_COMBINE, MOE_K_PREFILL_ROUTE,
-       MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_LAYER, MOE_K_LAYER_HITS, MOE_K_COUNT };
+       MOE_K_PREFILL_GATEUP, MOE_K_PREFILL_DOWN, MOE_K_LAYER, MOE_K_LAYER_HITS, MOE_K_MISS, MOE_K_COUNT };
 typedef struct {
     int64_t lookups, hits, misses, evictions;
     int64_t prefetch_lookups, prefetch_misses;
@@ -358,9 +360,11 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * of the layer's first miss from the pool (through its device address) into
  * the miss's slot, and the copy engine moves only the rest (n = 0: off, the
  * default; MOE_ERR_UNSUPPORTED if the pool has no device address); what = 11:
- * decode (default path) copies each missed record as one copy (n = 0, the
- * default) or as two, the gate/up prefix then W2, so a miss's gate/up runs
- * while its W2 streams (n = 1); what = 0 clears 1, 2, 4, 5 and 8. */
+ * decode (default path) copies each missed record as one copy and runs the
+ * miss as one launch, gate/up then down (n = 0, the default), or as two
+ * copies, the gate/up prefix then W2, with a gate/up and a down launch, so a
+ * miss's gate/up runs while its W2 streams (n = 1); what = 0 clears 1, 2, 4,
+ * 5 and 8. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Diagnostics: copies the first n (<= 160 * 32) stamps of the last traced

@@ -381,15 +381,43 @@ def test_two_copy_streams_match_the_oracle(path):
     st.close()
 
 
-def test_split_record_copies_match_the_oracle():
-    """Each missed record as two copies (the gate/up prefix, then W2, each with
-    its event) instead of one: same trace, table, slots and outputs."""
+def _launches(st):
+    ks = abi.moe_get_stats(st.ctx)
+    return {n: int(ks.kernel_launches[i]) for i, n in enumerate(abi.KERNEL_NAMES)}
+
+
+def test_one_launch_per_miss_by_default():
+    """Default path: one hit launch per call and one launch per miss (its whole
+    record copied, then gate/up and down in the same launch, the down tiles
+    waiting for the gate/up tiles inside it; the last one combines): outputs,
+    trace, table and slots match the oracle."""
     pb = DecodeProblem(MID, T=12)
     st = pb.stack()
-    abi.moe_debug_inject(st.ctx, 11, 1)
+    abi.moe_set_timing(st.ctx, True)
     run = pb.run(stack=st, routing=True)
     assert _check_run(pb, run) < 1e-5
     pb.check_slots(st, run.table[1])
+    n = _launches(st)
+    calls = pb.T * MID.L
+    assert n["expert_hits"] == calls and n["route_lookup"] == calls
+    assert n["expert_miss"] == run.stats.misses > calls // 2
+    assert n["gate_up"] == n["down"] == 0
+    st.close()
+
+
+def test_split_record_copies_match_the_oracle():
+    """Each missed record as two copies (the gate/up prefix, then W2, each with
+    its event) and a gate/up and a down launch instead of one of each: same
+    trace, table, slots and outputs."""
+    pb = DecodeProblem(MID, T=12)
+    st = pb.stack()
+    abi.moe_debug_inject(st.ctx, 11, 1)
+    abi.moe_set_timing(st.ctx, True)
+    run = pb.run(stack=st, routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(st, run.table[1])
+    n = _launches(st)
+    assert n["gate_up"] == n["down"] == run.stats.misses > 0 and n["expert_miss"] == 0
     st.close()
 
 
