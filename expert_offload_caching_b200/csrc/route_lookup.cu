@@ -170,31 +170,32 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
 
 // Softmax + top-k of row t by one warp; writes idx/gates of the row in ascending
 // id and returns the expert selected by this lane (lanes < k), else -1.
-// NVE: 32-wide chunks of the row held in registers (E <= 32 * NVE).
+// NVE: 32-wide chunks of the row held in registers (E <= 32 * NVE, a power of 2).
 // The order is total: a NaN logit counts as -inf, equal values go to the lower
-// id, and a picked entry is masked out by a bit (not by overwriting its value),
-// so k distinct ids in [0, E) come out whatever the logits hold.
+// id, and a picked entry's key is cleared (a real entry's key is never 0), so
+// k distinct ids in [0, E) come out whatever the logits hold.
 template <int NVE>
 __device__ int topk_row_n(const RouteArgs &a, int t) {
+    static_assert((NVE & (NVE - 1)) == 0, "the lane-local tree wants a power of 2");
     const int lane = threadIdx.x & 31;
     const float *z = a.ws.z + (size_t)t * a.E;
     const int nv = (a.E + 31) >> 5;
     float v[NVE];
-    uint32_t avail = 0u;  // bit j: entry lane + 32 j is a real expert not yet picked
+    uint32_t kk[NVE];  // order keys of the entries still selectable; 0: picked, or no expert
 #pragma unroll
     for (int j = 0; j < NVE; ++j) {
         const int e = lane + 32 * j;
         const bool real = j < nv && e < a.E;
         const float zv = real ? z[e] : -INFINITY;
         v[j] = zv != zv ? -INFINITY : zv;
-        if (real) avail |= 1u << j;
+        kk[j] = real ? order_key(v[j]) : 0u;  // >= key(-inf) = 0x007fffff
     }
-    float m = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < NVE; ++j) m = fmaxf(m, v[j]);
-    m = warp_max(m);
-    float sall = 0.f;  // the full softmax denominator (only without renormalisation)
+    float m = 0.f, sall = 0.f;  // the full softmax's max and denominator (only without renormalisation)
     if (!a.renorm) {
+        m = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < NVE; ++j) m = fmaxf(m, v[j]);
+        m = warp_max(m);
 #pragma unroll
         for (int j = 0; j < NVE; ++j)
             if (lane + 32 * j < a.E) sall += expf(v[j] - m);
@@ -204,19 +205,36 @@ __device__ int topk_row_n(const RouteArgs &a, int t) {
     int my_idx = 0x7fffffff;
     float my_val = -INFINITY;
     for (int s = 0; s < a.k; ++s) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;  // lane-local candidates are visited in ascending id
+        // this lane's largest key, the lowest id among equal ones: pairwise
+        // maxima in a tree (depth log2 NVE), the left (lower id) kept on ties
+        uint32_t tk[NVE];
+        int tj[NVE];
+#pragma unroll
+        for (int j = 0; j < NVE; ++j) {
+            tk[j] = kk[j];
+            tj[j] = j;
+        }
+#pragma unroll
+        for (int w = NVE; w > 1; w >>= 1) {
+#pragma unroll
+            for (int i = 0; i < w / 2; ++i) {
+                const bool r = tk[2 * i + 1] > tk[2 * i];
+                tk[i] = r ? tk[2 * i + 1] : tk[2 * i];
+                tj[i] = r ? tj[2 * i + 1] : tj[2 * i];
+            }
+        }
+        // the warp's largest key (two single-instruction warp reductions), then
+        // the lowest id holding it
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, tk[0]);
+        const int bi = (int)__reduce_min_sync(0xffffffffu, tk[0] == kmax ? (uint32_t)(lane + 32 * tj[0]) : 0xffffffffu);
+        if (lane == s) {
+            my_idx = bi;
+            my_val = key_value(kmax);
+        }
+        const int jsel = (bi < a.E && lane == (bi & 31)) ? (bi >> 5) : -1;
 #pragma unroll
         for (int j = 0; j < NVE; ++j)
-            if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = lane + 32 * j; }
-        // the warp's largest value (order-preserving integer key, two
-        // single-instruction warp reductions), then the lowest id holding it
-        const uint32_t key = order_key(bv);
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-        bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0xffffffffu);
-        bv = key_value(kmax);
-        if (lane == s) { my_idx = bi; my_val = bv; }
-        if (bi < a.E && lane == (bi & 31)) avail &= ~(1u << (bi >> 5));
+            if (j == jsel) kk[j] = 0u;
     }
     const float top = __shfl_sync(0xffffffffu, my_val, 0);
     float g;
@@ -256,8 +274,8 @@ struct LookupSmem {
     uint32_t hitmap[kMaxSlotBits / 32];
     unsigned long long clock, lastv;
     int nf, nhit, nmiss;
-    unsigned long long redv[kRouteThreads / 32];
-    int reds[kRouteThreads / 32];
+    unsigned long long redv[2][kRouteThreads / 32];  // per warp, by round parity
+    int reds[2][kRouteThreads / 32];
 };
 
 // One lookup batch of `layer` over sm.exp[0..n), run by all threads of the CTA.
@@ -327,41 +345,69 @@ __device__ void lookup_batch(const Table &tab, int layer, int E, int n, LookupSm
     const int nhit = sm.nhit, nmiss = sm.nmiss, nf = sm.nf;
     const int nfree = C - nf;
     const int nevict = nmiss > nfree ? nmiss - nfree : 0;
+    // victim candidates of the register tile: stamp << 13 | slot for a used
+    // (stamp > 0), non-hit slot, else ~0 (slots of the tile are < 2^13; stamps
+    // count lookups, far below 2^51); a chosen one is cleared by its thread
+    constexpr int kTileSlots = kRouteThreads * kStampRegs;
+    static_assert(kTileSlots <= (1 << 13) && (kStampRegs & (kStampRegs - 1)) == 0, "tile key layout");
+    unsigned long long sk[kStampRegs];
+#pragma unroll
+    for (int i = 0; i < kStampRegs; ++i) {
+        const int sl = threadIdx.x + kRouteThreads * i;
+        const bool cand = sl < C && sv[i] != 0ull && !(sm.hitmap[sl >> 5] & (1u << (sl & 31)));
+        sk[i] = cand ? (sv[i] << 13) | (unsigned long long)sl : ~0ull;
+    }
     unsigned long long last = 0ull;
     for (int r = 0; r < nevict; ++r) {
+        // this thread's smallest key: pairwise minima in a tree (depth 5)
+        unsigned long long tk[kStampRegs];
+#pragma unroll
+        for (int i = 0; i < kStampRegs; ++i) tk[i] = sk[i];
+#pragma unroll
+        for (int w = kStampRegs; w > 1; w >>= 1) {
+#pragma unroll
+            for (int i = 0; i < w / 2; ++i) tk[i] = tk[2 * i + 1] < tk[2 * i] ? tk[2 * i + 1] : tk[2 * i];
+        }
         unsigned long long bv = ~0ull;
         int bs = -1;
-#pragma unroll
-        for (int i = 0; i < kStampRegs; ++i) {
-            const int sl = threadIdx.x + kRouteThreads * i;
-            if (sl < C && sv[i] > last && sv[i] < bv && !(sm.hitmap[sl >> 5] & (1u << (sl & 31)))) {
-                bv = sv[i];
-                bs = sl;
-            }
+        if (tk[0] != ~0ull) {
+            bv = tk[0] >> 13;
+            bs = (int)(tk[0] & ((1ull << 13) - 1ull));
         }
-        for (int sl = threadIdx.x + kRouteThreads * kStampRegs; sl < C; sl += kRouteThreads) {
+        for (int sl = threadIdx.x + kTileSlots; sl < C; sl += kRouteThreads) {
             const unsigned long long v = tab.stamp[sl];  // caches beyond the register tile
             if (v > last && v < bv && !(sm.hitmap[sl >> 5] & (1u << (sl & 31)))) { bv = v; bs = sl; }
         }
+        // the warp's smallest stamp (stamps are unique: one slot holds it), by
+        // 32-bit warp reductions over its halves
+        const uint32_t hi = __reduce_min_sync(0xffffffffu, (uint32_t)(bv >> 32));
+        const uint32_t lo = __reduce_min_sync(0xffffffffu, (uint32_t)(bv >> 32) == hi ? (uint32_t)bv : ~0u);
+        const unsigned long long wv = ((unsigned long long)hi << 32) | lo;
+        const uint32_t ws = __reduce_min_sync(0xffffffffu, bv == wv ? (uint32_t)bs : ~0u);
+        if (lane == 0) {
+            sm.redv[r & 1][warp] = wv;
+            sm.reds[r & 1][warp] = (int)ws;
+        }
+        __syncthreads();
+        // every thread takes the block's minimum (buffers alternate by round,
+        // so the next round's writes cannot race these reads)
+        unsigned long long mv = sm.redv[r & 1][0];
+        int ms = sm.reds[r & 1][0];
+        for (int w = 1; w < nw; ++w) {
+            const unsigned long long ov = sm.redv[r & 1][w];
+            if (ov < mv) {
+                mv = ov;
+                ms = sm.reds[r & 1][w];
+            }
+        }
+        if (threadIdx.x == 0) sm.victim[r] = ms;
+        last = mv;
+        const int isel = (ms >= 0 && ms < kTileSlots && (ms % kRouteThreads) == (int)threadIdx.x) ? ms / kRouteThreads : -1;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int os = __shfl_xor_sync(0xffffffffu, bs, o);
-            if (ov < bv) { bv = ov; bs = os; }
-        }
-        if (lane == 0) { sm.redv[warp] = bv; sm.reds[warp] = bs; }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            unsigned long long mv = sm.redv[0];
-            int ms = sm.reds[0];
-            for (int w = 1; w < nw; ++w)
-                if (sm.redv[w] < mv) { mv = sm.redv[w]; ms = sm.reds[w]; }
-            sm.victim[r] = ms;
-            sm.lastv = mv;
-        }
-        __syncthreads();
-        last = sm.lastv;
+        for (int i = 0; i < kStampRegs; ++i)
+            if (i == isel) sk[i] = ~0ull;
     }
+    __syncthreads();
     for (int r = threadIdx.x; r < nevict; r += blockDim.x) sm.old[r] = tab.owner[sm.victim[r]];
     __syncthreads();
     const unsigned long long clock = sm.clock;
