@@ -172,8 +172,10 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
 // id and returns the expert selected by this lane (lanes < k), else -1.
 // NVE: 32-wide chunks of the row held in registers (E <= 32 * NVE, a power of 2).
 // The order is total: a NaN logit counts as -inf, equal values go to the lower
-// id, and a picked entry's key is cleared (a real entry's key is never 0), so
-// k distinct ids in [0, E) come out whatever the logits hold.
+// id, and a picked entry's key is cleared to 0 (below every value's key), so k
+// distinct ids in [0, E) come out whatever the logits hold.  Entries past E
+// hold the key of -inf: they lose every tie to a real entry (larger ids), so
+// with k <= E none is picked.
 template <int NVE>
 __device__ int topk_row_n(const RouteArgs &a, int t) {
     static_assert((NVE & (NVE - 1)) == 0, "the lane-local tree wants a power of 2");
@@ -181,14 +183,15 @@ __device__ int topk_row_n(const RouteArgs &a, int t) {
     const float *z = a.ws.z + (size_t)t * a.E;
     const int nv = (a.E + 31) >> 5;
     float v[NVE];
-    uint32_t kk[NVE];  // order keys of the entries still selectable; 0: picked, or no expert
+    uint32_t kk[NVE];  // order keys of the entries still selectable (>= key(-inf) = 0x007fffff); 0: picked
 #pragma unroll
     for (int j = 0; j < NVE; ++j) {
         const int e = lane + 32 * j;
-        const bool real = j < nv && e < a.E;
-        const float zv = real ? z[e] : -INFINITY;
+        const float zv = (j < nv && e < a.E) ? z[e] : -INFINITY;
         v[j] = zv != zv ? -INFINITY : zv;
-        kk[j] = real ? order_key(v[j]) : 0u;  // >= key(-inf) = 0x007fffff
+        // (a key of every entry, not one guarded by the range test: the
+        // guarded form measured twice as slow, its loads no longer overlapped)
+        kk[j] = order_key(v[j]);
     }
     float m = 0.f, sall = 0.f;  // the full softmax's max and denominator (only without renormalisation)
     if (!a.renorm) {
@@ -350,12 +353,15 @@ __device__ void lookup_batch(const Table &tab, int layer, int E, int n, LookupSm
     // count lookups, far below 2^51); a chosen one is cleared by its thread
     constexpr int kTileSlots = kRouteThreads * kStampRegs;
     static_assert(kTileSlots <= (1 << 13) && (kStampRegs & (kStampRegs - 1)) == 0, "tile key layout");
+    // (built only when the batch evicts: it waits for the stamp loads)
     unsigned long long sk[kStampRegs];
+    if (nevict > 0) {
 #pragma unroll
-    for (int i = 0; i < kStampRegs; ++i) {
-        const int sl = threadIdx.x + kRouteThreads * i;
-        const bool cand = sl < C && sv[i] != 0ull && !(sm.hitmap[sl >> 5] & (1u << (sl & 31)));
-        sk[i] = cand ? (sv[i] << 13) | (unsigned long long)sl : ~0ull;
+        for (int i = 0; i < kStampRegs; ++i) {
+            const int sl = threadIdx.x + kRouteThreads * i;
+            const bool cand = sl < C && sv[i] != 0ull && !(sm.hitmap[sl >> 5] & (1u << (sl & 31)));
+            sk[i] = cand ? (sv[i] << 13) | (unsigned long long)sl : ~0ull;
+        }
     }
     unsigned long long last = 0ull;
     for (int r = 0; r < nevict; ++r) {

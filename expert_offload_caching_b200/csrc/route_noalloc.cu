@@ -108,10 +108,11 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
     __threadfence();
 
     // a NaN logit counts as -inf (selection and softmax), as in moe_layer_forward.
-    // A row lives in registers (entry lane + 32 j: order key kk[j], 0 for no
-    // expert and for a picked entry -- a real entry's key is at least that of
-    // -inf), so each pick is the largest remaining logit in (value desc, id
-    // asc) order and k distinct ids in [0, E) come out.
+    // A row lives in registers (entry lane + 32 j: order key kk[j], at least
+    // that of -inf; 0 for a picked entry), so each pick is the largest
+    // remaining logit in (value desc, id asc) order and k distinct ids in
+    // [0, E) come out: entries past E hold the key of -inf and lose every tie
+    // to a real entry (larger ids).
     constexpr int kNv = kNaMaxE / 32;
     static_assert((kNv & (kNv - 1)) == 0, "the lane-local tree wants a power of 2");
     for (int t = warp; t < T; t += nw) {
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
             const int e = lane + 32 * j;
             const float zv = e < E ? __ldcg(zr + e) : -INFINITY;
             v[j] = zv != zv ? -INFINITY : zv;
-            kk[j] = e < E ? na_key(v[j]) : 0u;
+            kk[j] = na_key(v[j]);  // (unguarded: the guarded form kept the loads from overlapping)
             m = fmaxf(m, v[j]);
         }
         m = na_warp_max(m);

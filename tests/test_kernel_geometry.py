@@ -446,10 +446,10 @@ def _order_key(v):
 
 def _warp_tree_topk(z, k, nve):
     """The decode route kernel's selection as the warp runs it: lane l holds
-    entries l + 32 j (j < nve) as order keys (0 for no expert and for picked
-    ones); per round each lane reduces its keys by a tree of pairwise maxima
-    keeping the left side on ties, then the warp takes the largest key and the
-    lowest id holding it."""
+    entries l + 32 j (j < nve) as order keys (entries past E: the key of -inf;
+    picked ones: 0); per round each lane reduces its keys by a tree of pairwise
+    maxima keeping the left side on ties, then the warp takes the largest key
+    and the lowest id holding it."""
     import numpy as np
     E = z.size
     zf = np.where(np.isnan(z), np.float32(-np.inf), z).astype(np.float32)
@@ -457,8 +457,8 @@ def _warp_tree_topk(z, k, nve):
     for j in range(nve):
         for lane in range(32):
             e = lane + 32 * j
-            if e < E:
-                kk[lane, j] = _order_key(zf[e:e + 1])[0]
+            val = zf[e:e + 1] if e < E else np.array([-np.inf], np.float32)
+            kk[lane, j] = _order_key(val)[0]
     out = []
     for _ in range(k):
         tk = kk.copy()
@@ -482,7 +482,8 @@ def test_route_tree_topk_selects_the_largest_with_ties_to_the_lower_id():
     """The lane-local tree plus warp reductions pick the same ids as a plain
     sort by (value descending, id ascending) with NaN as -inf and -0 == +0, on
     rows with many equal values, infinities and NaNs, for E not a multiple of
-    32 and k up to E."""
+    32 and k up to E (rows of -inf included: the entries past E tie with them
+    and must lose)."""
     import numpy as np
     rng = np.random.default_rng(11)
     for E, nve in [(40, 2), (128, 4), (200, 8), (512, 16), (1000, 32)]:
@@ -496,7 +497,9 @@ def test_route_tree_topk_selects_the_largest_with_ties_to_the_lower_id():
                 z[rng.integers(0, E, 2)] = -np.inf
             if trial >= 4:
                 z[rng.integers(0, E, 1)] = np.inf
-            for k in sorted({1, min(10, E), E if E <= 40 else 33}):
+            if trial == 5:
+                z[: E // 2] = -np.inf
+            for k in sorted({1, min(10, E), E if E <= 40 else 33, E}):
                 got = _warp_tree_topk(z, k, nve)
                 zf = np.where(np.isnan(z), np.float32(-np.inf), z)
                 key = _order_key(zf).astype(np.int64)
