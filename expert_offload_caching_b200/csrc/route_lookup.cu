@@ -170,35 +170,31 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
 
 // Softmax + top-k of row t by one warp; writes idx/gates of the row in ascending
 // id and returns the expert selected by this lane (lanes < k), else -1.
-// NVE: 32-wide chunks of the row held in registers (E <= 32 * NVE, a power of 2).
+// NVE: 32-wide chunks of the row held in registers (E <= 32 * NVE).
 // The order is total: a NaN logit counts as -inf, equal values go to the lower
-// id, and a picked entry's key is cleared to 0 (below every value's key), so k
-// distinct ids in [0, E) come out whatever the logits hold.  Entries past E
-// hold the key of -inf: they lose every tie to a real entry (larger ids), so
-// with k <= E none is picked.
+// id, and a picked entry is masked out by a bit (not by overwriting its value),
+// so k distinct ids in [0, E) come out whatever the logits hold.
 template <int NVE>
 __device__ int topk_row_n(const RouteArgs &a, int t) {
-    static_assert((NVE & (NVE - 1)) == 0, "the lane-local tree wants a power of 2");
     const int lane = threadIdx.x & 31;
     const float *z = a.ws.z + (size_t)t * a.E;
     const int nv = (a.E + 31) >> 5;
     float v[NVE];
-    uint32_t kk[NVE];  // order keys of the entries still selectable (>= key(-inf) = 0x007fffff); 0: picked
+    uint32_t avail = 0u;  // bit j: entry lane + 32 j is a real expert not yet picked
 #pragma unroll
     for (int j = 0; j < NVE; ++j) {
         const int e = lane + 32 * j;
-        const float zv = (j < nv && e < a.E) ? z[e] : -INFINITY;
+        const bool real = j < nv && e < a.E;
+        const float zv = real ? z[e] : -INFINITY;
         v[j] = zv != zv ? -INFINITY : zv;
-        // (a key of every entry, not one guarded by the range test: the
-        // guarded form measured twice as slow, its loads no longer overlapped)
-        kk[j] = order_key(v[j]);
+        if (real) avail |= 1u << j;
     }
-    float m = 0.f, sall = 0.f;  // the full softmax's max and denominator (only without renormalisation)
-    if (!a.renorm) {
-        m = -INFINITY;
+    float m = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < NVE; ++j) m = fmaxf(m, v[j]);
-        m = warp_max(m);
+    for (int j = 0; j < NVE; ++j) m = fmaxf(m, v[j]);
+    m = warp_max(m);
+    float sall = 0.f;  // the full softmax denominator (only without renormalisation)
+    if (!a.renorm) {
 #pragma unroll
         for (int j = 0; j < NVE; ++j)
             if (lane + 32 * j < a.E) sall += expf(v[j] - m);
@@ -208,36 +204,19 @@ __device__ int topk_row_n(const RouteArgs &a, int t) {
     int my_idx = 0x7fffffff;
     float my_val = -INFINITY;
     for (int s = 0; s < a.k; ++s) {
-        // this lane's largest key, the lowest id among equal ones: pairwise
-        // maxima in a tree (depth log2 NVE), the left (lower id) kept on ties
-        uint32_t tk[NVE];
-        int tj[NVE];
-#pragma unroll
-        for (int j = 0; j < NVE; ++j) {
-            tk[j] = kk[j];
-            tj[j] = j;
-        }
-#pragma unroll
-        for (int w = NVE; w > 1; w >>= 1) {
-#pragma unroll
-            for (int i = 0; i < w / 2; ++i) {
-                const bool r = tk[2 * i + 1] > tk[2 * i];
-                tk[i] = r ? tk[2 * i + 1] : tk[2 * i];
-                tj[i] = r ? tj[2 * i + 1] : tj[2 * i];
-            }
-        }
-        // the warp's largest key (two single-instruction warp reductions), then
-        // the lowest id holding it
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, tk[0]);
-        const int bi = (int)__reduce_min_sync(0xffffffffu, tk[0] == kmax ? (uint32_t)(lane + 32 * tj[0]) : 0xffffffffu);
-        if (lane == s) {
-            my_idx = bi;
-            my_val = key_value(kmax);
-        }
-        const int jsel = (bi < a.E && lane == (bi & 31)) ? (bi >> 5) : -1;
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;  // lane-local candidates are visited in ascending id
 #pragma unroll
         for (int j = 0; j < NVE; ++j)
-            if (j == jsel) kk[j] = 0u;
+            if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = lane + 32 * j; }
+        // the warp's largest value (order-preserving integer key, two
+        // single-instruction warp reductions), then the lowest id holding it
+        const uint32_t key = order_key(bv);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0xffffffffu);
+        bv = key_value(kmax);
+        if (lane == s) { my_idx = bi; my_val = bv; }
+        if (bi < a.E && lane == (bi & 31)) avail &= ~(1u << (bi >> 5));
     }
     const float top = __shfl_sync(0xffffffffu, my_val, 0);
     float g;

@@ -108,62 +108,47 @@ __global__ void __launch_bounds__(kNaThreads) route_noalloc_kernel(
     __threadfence();
 
     // a NaN logit counts as -inf (selection and softmax), as in moe_layer_forward.
-    // A row lives in registers (entry lane + 32 j: order key kk[j], at least
-    // that of -inf; 0 for a picked entry), so each pick is the largest
-    // remaining logit in (value desc, id asc) order and k distinct ids in
-    // [0, E) come out: entries past E hold the key of -inf and lose every tie
-    // to a real entry (larger ids).
+    // A row lives in registers (entry lane + 32 j in v[j]); a picked entry is
+    // masked out by its bit, so each pick is the largest remaining logit in
+    // (value desc, id asc) order and k distinct ids in [0, E) come out.
     constexpr int kNv = kNaMaxE / 32;
-    static_assert((kNv & (kNv - 1)) == 0, "the lane-local tree wants a power of 2");
     for (int t = warp; t < T; t += nw) {
         const float *zr = z + (size_t)t * E;
         float v[kNv];
-        uint32_t kk[kNv];
+        uint32_t avail = 0u;
         float m = -INFINITY;
 #pragma unroll
         for (int j = 0; j < kNv; ++j) {
             const int e = lane + 32 * j;
             const float zv = e < E ? __ldcg(zr + e) : -INFINITY;
             v[j] = zv != zv ? -INFINITY : zv;
-            kk[j] = na_key(v[j]);  // (unguarded: the guarded form kept the loads from overlapping)
+            if (e < E) avail |= 1u << j;
             m = fmaxf(m, v[j]);
         }
         m = na_warp_max(m);
         float sall = 0.f;
 #pragma unroll
         for (int j = 0; j < kNv; ++j)
-            if (lane + 32 * j < E) sall += expf(v[j] - m);
+            if ((avail >> j) & 1u) sall += expf(v[j] - m);
         sall = na_warp_sum(sall);
         int my_idx = 0x7fffffff;
         float my_val = -INFINITY;
         for (int s = 0; s < k; ++s) {
-            // this lane's largest key, the lowest id among equal ones: pairwise
-            // maxima in a tree, the left (lower id) kept on ties
-            uint32_t tk[kNv];
-            int tj[kNv];
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
 #pragma unroll
-            for (int j = 0; j < kNv; ++j) {
-                tk[j] = kk[j];
-                tj[j] = j;
+            for (int j = 0; j < kNv; ++j) {  // ascending ids within the lane: keep the first of equal values
+                const int e = lane + 32 * j;
+                if (((avail >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) { bv = v[j]; bi = e; }
             }
-#pragma unroll
-            for (int w = kNv; w > 1; w >>= 1) {
-#pragma unroll
-                for (int i = 0; i < w / 2; ++i) {
-                    const bool r = tk[2 * i + 1] > tk[2 * i];
-                    tk[i] = r ? tk[2 * i + 1] : tk[2 * i];
-                    tj[i] = r ? tj[2 * i + 1] : tj[2 * i];
-                }
-            }
-            // the warp's largest key (warp reductions), then the lowest id holding it
-            const uint32_t kmax = __reduce_max_sync(0xffffffffu, tk[0]);
-            const int bi =
-                (int)__reduce_min_sync(0xffffffffu, tk[0] == kmax ? (uint32_t)(lane + 32 * tj[0]) : 0xffffffffu);
-            const int jsel = (bi < E && (bi & 31) == lane) ? (bi >> 5) : -1;
-#pragma unroll
-            for (int j = 0; j < kNv; ++j)
-                if (j == jsel) kk[j] = 0u;
-            if (lane == s) { my_idx = bi; my_val = na_key_value(kmax); }
+            // the warp's largest value (order-preserving integer key, warp
+            // reductions), then the lowest id holding it
+            const uint32_t key = na_key(bv);
+            const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+            bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)bi : 0xffffffffu);
+            bv = na_key_value(kmax);
+            if (bi != 0x7fffffff && (bi & 31) == lane) avail &= ~(1u << (bi >> 5));
+            if (lane == s) { my_idx = bi; my_val = bv; }
         }
         const float top = __shfl_sync(0xffffffffu, my_val, 0);
         float g;

@@ -436,72 +436,3 @@ def test_topk_order_key_preserves_the_selection_order():
     same = np.where(vals == 0, np.float32(0), vals)
     assert np.array_equal(back.view(np.uint32), same.view(np.uint32))  # exact inverse
 
-
-def _order_key(v):
-    import numpy as np
-    v = np.where(v == 0, np.float32(0), v).astype(np.float32)
-    u = v.view(np.uint32)
-    return np.where(u & np.uint32(0x80000000), ~u, u | np.uint32(0x80000000)).astype(np.uint32)
-
-
-def _warp_tree_topk(z, k, nve):
-    """The decode route kernel's selection as the warp runs it: lane l holds
-    entries l + 32 j (j < nve) as order keys (entries past E: the key of -inf;
-    picked ones: 0); per round each lane reduces its keys by a tree of pairwise
-    maxima keeping the left side on ties, then the warp takes the largest key
-    and the lowest id holding it."""
-    import numpy as np
-    E = z.size
-    zf = np.where(np.isnan(z), np.float32(-np.inf), z).astype(np.float32)
-    kk = np.zeros((32, nve), np.uint32)
-    for j in range(nve):
-        for lane in range(32):
-            e = lane + 32 * j
-            val = zf[e:e + 1] if e < E else np.array([-np.inf], np.float32)
-            kk[lane, j] = _order_key(val)[0]
-    out = []
-    for _ in range(k):
-        tk = kk.copy()
-        tj = np.tile(np.arange(nve), (32, 1))
-        w = nve
-        while w > 1:
-            for i in range(w // 2):
-                r = tk[:, 2 * i + 1] > tk[:, 2 * i]
-                tk[:, i] = np.where(r, tk[:, 2 * i + 1], tk[:, 2 * i])
-                tj[:, i] = np.where(r, tj[:, 2 * i + 1], tj[:, 2 * i])
-            w //= 2
-        kmax = tk[:, 0].max()
-        ids = np.where(tk[:, 0] == kmax, np.arange(32) + 32 * tj[:, 0], 2**32 - 1)
-        bi = int(ids.min())
-        out.append(bi)
-        kk[bi & 31, bi >> 5] = 0
-    return out
-
-
-def test_route_tree_topk_selects_the_largest_with_ties_to_the_lower_id():
-    """The lane-local tree plus warp reductions pick the same ids as a plain
-    sort by (value descending, id ascending) with NaN as -inf and -0 == +0, on
-    rows with many equal values, infinities and NaNs, for E not a multiple of
-    32 and k up to E (rows of -inf included: the entries past E tie with them
-    and must lose)."""
-    import numpy as np
-    rng = np.random.default_rng(11)
-    for E, nve in [(40, 2), (128, 4), (200, 8), (512, 16), (1000, 32)]:
-        for trial in range(6):
-            z = rng.integers(-3, 4, E).astype(np.float32)  # many ties
-            if trial % 2:
-                z = rng.standard_normal(E).astype(np.float32)
-            z[rng.integers(0, E, 3)] = np.float32(-0.0)
-            if trial >= 2:
-                z[rng.integers(0, E, 2)] = np.nan
-                z[rng.integers(0, E, 2)] = -np.inf
-            if trial >= 4:
-                z[rng.integers(0, E, 1)] = np.inf
-            if trial == 5:
-                z[: E // 2] = -np.inf
-            for k in sorted({1, min(10, E), E if E <= 40 else 33, E}):
-                got = _warp_tree_topk(z, k, nve)
-                zf = np.where(np.isnan(z), np.float32(-np.inf), z)
-                key = _order_key(zf).astype(np.int64)
-                want = np.lexsort((np.arange(E), -key))[:k]
-                assert got == [int(i) for i in want], (E, trial, k)
