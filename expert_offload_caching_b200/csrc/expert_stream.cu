@@ -307,29 +307,32 @@ __global__ void __launch_bounds__(32 * (P * st_max_groups(P) + 1), 1) expert_str
         }
     }
 
+    if (a.phase == 3 && a.head_bytes && s_head_exp >= 0) {
+        // every thread of every CTA, before its own work: the head of the
+        // layer's first miss, from the page-locked pool over PCIe straight into
+        // its slot (16-byte loads, four in flight per thread: megabytes in
+        // flight over the grid, enough to keep the link busy) while the copy
+        // engine is still starting on the rest of the record.  The launch's own
+        // items wait meanwhile; they are not on the layer's critical path.
+        const int64_t rec_idx = ((int64_t)a.layer * a.E + s_head_exp) % a.pool_P;
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.pool_d + rec_idx * a.rec_bytes);
+        uint4 *dst = reinterpret_cast<uint4 *>(const_cast<uint8_t *>(a.arena) + (int64_t)s_head_slot * a.rec_bytes);
+        const int64_t n16 = a.head_bytes >> 4, step = (int64_t)gridDim.x * blockDim.x;
+        int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        for (; i + 3 * step < n16; i += 4 * step) {
+            const uint4 v0 = __ldcv(src + i), v1 = __ldcv(src + i + step), v2 = __ldcv(src + i + 2 * step),
+                        v3 = __ldcv(src + i + 3 * step);
+            dst[i] = v0;
+            dst[i + step] = v1;
+            dst[i + 2 * step] = v2;
+            dst[i + 3 * step] = v3;
+        }
+        for (; i < n16; i += step) dst[i] = __ldcv(src + i);
+    }
+
     if (warp == 0) {
         // ---------------------------------------------------------- producer
-        if (lane > 0) {
-            // lanes 1..31 of every CTA: the head of the layer's first miss, from the
-            // page-locked pool over PCIe straight into its slot (16-byte loads, four
-            // in flight per lane); the copy engine moves the rest of the record
-            if (a.phase == 3 && a.head_bytes && s_head_exp >= 0) {
-                const int64_t rec_idx = ((int64_t)a.layer * a.E + s_head_exp) % a.pool_P;
-                const uint4 *src = reinterpret_cast<const uint4 *>(a.pool_d + rec_idx * a.rec_bytes);
-                uint4 *dst = reinterpret_cast<uint4 *>(const_cast<uint8_t *>(a.arena) + (int64_t)s_head_slot * a.rec_bytes);
-                const int64_t n16 = a.head_bytes >> 4, step = (int64_t)gridDim.x * 31;
-                int64_t i = (int64_t)blockIdx.x * 31 + (lane - 1);
-                for (; i + 3 * step < n16; i += 4 * step) {
-                    const uint4 v0 = __ldcv(src + i), v1 = __ldcv(src + i + step), v2 = __ldcv(src + i + 2 * step),
-                                v3 = __ldcv(src + i + 3 * step);
-                    dst[i] = v0;
-                    dst[i + step] = v1;
-                    dst[i + 2 * step] = v2;
-                    dst[i + 3 * step] = v3;
-                }
-                for (; i < n16; i += step) dst[i] = __ldcv(src + i);
-            }
-        } else {
+        if (lane == 0) {
             const uint64_t pol = evict_first_policy();
             int issued = 0, skipped = -1;
             for (int l = 0; l < n_my; ++l) {
