@@ -711,7 +711,7 @@ def kernel_table(kst):
 # ratio times its algorithmic bytes (traffic grows with the weight bytes
 # streamed).  A class absent here reports null.
 TRAFFIC_RATIO = {
-    "expert_hits": (1.0391, "profiles/expert_stream_resident_deepseek-shaped.md"),
+    "expert_hits": (1.0476, "profiles/expert_stream_resident_deepseek-shaped.md"),
 }
 
 
