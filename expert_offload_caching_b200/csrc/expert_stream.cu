@@ -46,9 +46,8 @@ using namespace gemv;
 constexpr int kStMaxStages = 8;
 constexpr int kStMaxGroups = 5;                // consumer warp groups (P warps each) + the producer warp
 // (with the producer, 16 or 11 warps: at most four per SM sub-partition, so
-// up to 128 registers per thread for groups of three; groups of five come two
-// to a CTA)
-__host__ __device__ constexpr int st_max_groups(int P) { return P >= 5 ? 2 : kStMaxGroups; }
+// up to 128 registers per thread for groups of three)
+__host__ __device__ constexpr int st_max_groups(int P) { return kStMaxGroups; }
 constexpr int kErrStreamFull = 42;             // a stage's copy did not land in time
 constexpr int kErrStreamEmpty = 43;            // a stage was not released in time
 constexpr int kErrStreamDep = 44;              // a down item's gate/up tiles did not complete in time
@@ -762,11 +761,6 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
     // older phase).
     const int gmax = kStMaxGroups;
     int nc = ns >= 2 * gmax ? gmax : (ns >= 6 ? ns / 2 : (ns < gmax ? ns : gmax));
-    // large tiles (4 or 5 stages fit): two groups of five warps with two stages
-    // each, so a group computes one item while its next one loads, rather than
-    // one stage per group of three that waits for its refill after every item
-    const bool wide = ng == 1 && a.wide_groups && ns >= 4 && ns < 6;
-    if (wide) nc = 2;
     a.nc = nc;
     a.ns = ns = (ns >= 2 * nc ? 2 : 1) * nc;
     a.stage_bytes = (uint32_t)sb;
@@ -780,11 +774,9 @@ cudaError_t launch_stream(const GemvArgs &a_in, int max_exp, cudaStream_t s) {
     const int grid = (int)(items < sms ? items : sms);
     const bool full = a.d % 256 == 0 && a.F % 256 == 0;
     if (mx) {
-        if (wide) return launch_st_fs<1, kFmtMxfp4, 5>(a, grid, smem, full, sa, s);
         if (ng == 1) return launch_st_fs<1, kFmtMxfp4, 3>(a, grid, smem, full, sa, s);
         return launch_st_fs<2, kFmtMxfp4, 2>(a, grid, smem, full, false, s);
     }
-    if (wide) return launch_st_fs<1, kFmtNvfp4, 5>(a, grid, smem, full, sa, s);
     if (ng == 1) return launch_st_fs<1, kFmtNvfp4, 3>(a, grid, smem, full, sa, s);
     return launch_st_fs<2, kFmtNvfp4, 2>(a, grid, smem, full, false, s);
 }

@@ -199,9 +199,6 @@ struct moe_ctx {
     // start-ups; measured faster or equal), or the gate/up prefix and W2 as two,
     // so a miss's gate/up runs while its W2 streams (what = 11)
     bool split_copies = false;
-    // streaming kernels with large tiles: two groups of five warps with two
-    // stages each (1, default) or one stage per group of three (0) (what = 12)
-    int wide_groups = 1;
     // diagnostic trace of the next streaming hit launches (moe_debug_inject what = 9)
     unsigned long long *trace_d = nullptr;
     int64_t trace_arm = 0;
@@ -441,7 +438,6 @@ GemvArgs stream_args(moe_ctx *ctx, int layer, int T, int phase, int only_job, in
     g.done = ctx->dws.st_done;
     g.exit_ticket = ctx->dws.st_exit;
     g.wait_ns = (unsigned long long)(std::min(ctx->wait_limit, 5.0) * 1e9);
-    g.wide_groups = ctx->wide_groups;
     if (ctx->inj_stream_skip > 0) {
         g.inj_skip = 1;
         --ctx->inj_stream_skip;
@@ -1437,9 +1433,6 @@ moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n) {
     else if (what == 11) {  // decode misses: two copies per record (n = 1) or one (n = 0, default)
         if (n < 0 || n > 1) return MOE_ERR_ARG;
         ctx->split_copies = n == 1;
-    } else if (what == 12) {  // streaming kernels, large tiles: groups of five (1, default) or of three (0)
-        if (n < 0 || n > 1) return MOE_ERR_ARG;
-        ctx->wide_groups = n;
     } else if (what == 10) {  // decode: the SMs copy the first n bytes of a layer's first miss
         if (n < 0 || (n & 15) || n >= ctx->lay.bytes) return MOE_ERR_ARG;
         if (n > 0 && !ctx->pool_d) return MOE_ERR_UNSUPPORTED;

@@ -168,9 +168,8 @@ struct GemvArgs {
     uint32_t *exit_ticket = nullptr; // phase 3: CTAs finished (the last one resets done)
     unsigned long long wait_ns = 0;  // every wait of the kernel ends by then (from its start)
     // set by launch_stream
-    int wide_groups = 1;             // (in) large tiles: two groups of five warps, two stages each
     int tpa = 0, tpb = 0;            // weight tiles per work item (gate/up, down)
-    int ns = 0, nc = 0;              // shared-memory stages, consumer warp groups
+    int ns = 0, nc = 0;              // shared-memory stages, consumer warps
     uint32_t stage_bytes = 0, meta_off = 0, rr_off = 0, x_off = 0;
     int exp_cap = 0;                 // experts the metadata area holds
     int inj_skip = 0;                // test injection: CTA 0 issues no copies for its first item

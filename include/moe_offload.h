@@ -363,10 +363,8 @@ MOE_API moe_status moe_set_wait_limit(moe_ctx *ctx, double seconds);
  * decode (default path) copies each missed record as one copy and runs the
  * miss as one launch, gate/up then down (n = 0, the default), or as two
  * copies, the gate/up prefix then W2, with a gate/up and a down launch, so a
- * miss's gate/up runs while its W2 streams (n = 1); what = 12: the streaming
- * kernels, where only 4 or 5 shared-memory stages fit (large tiles), run two
- * groups of five warps with two stages each (n = 1, the default) or one stage
- * per group of three (n = 0); what = 0 clears 1, 2, 4, 5 and 8. */
+ * miss's gate/up runs while its W2 streams (n = 1); what = 0 clears 1, 2, 4,
+ * 5 and 8. */
 MOE_API moe_status moe_debug_inject(moe_ctx *ctx, int32_t what, int64_t n);
 
 /* Diagnostics: copies the first n (<= 160 * 32) stamps of the last traced

@@ -406,26 +406,23 @@ def test_one_launch_per_miss_by_default():
 
 
 # d = 4096: a gate/up tile is 36 KB (NVFP4) or 34 KB (MXFP4), so only 5 stages fit
+# (five groups of three warps, one stage each)
 WIDE = synth.LayerShape("wide", L=2, E=16, k=4, d=4096, F=256, shared=True, tokens=6, cache_slots=10)
 
 
 @pytest.mark.parametrize("fmt", [sp.FMT_NVFP4, sp.FMT_MXFP4], ids=["nvfp4", "mxfp4"])
 @pytest.mark.parametrize("S", [1, 3])
-def test_large_tiles_two_groups_of_five_match_the_oracle(fmt, S):
-    """Large tiles: the streaming kernels run two groups of five warps with two
-    stages each (the hit launch and every miss launch; 1 row with activations
-    in shared memory, 3 rows from global memory); trace, table, slots and
-    outputs match the oracle, as they do with one stage per group of three
-    (moe_debug_inject what = 12, n = 0)."""
-    for wide in (1, 0):
-        pb = DecodeProblem(WIDE, T=6, streams=S, fmt=fmt, C=min(S * WIDE.k, WIDE.E) + 4)
-        st = pb.stack()
-        abi.moe_debug_inject(st.ctx, 12, wide)
-        run = pb.run(stack=st, routing=True)
-        assert _check_run(pb, run) < 1e-5
-        pb.check_slots(st, run.table[1])
-        assert 0 < run.stats.misses < run.stats.lookups
-        st.close()
+def test_large_tiles_match_the_oracle(fmt, S):
+    """Large tiles (one stage per consumer group; 1 row with activations in
+    shared memory, 3 rows from global memory), the hit launch and every miss
+    launch: trace, table, slots and outputs match the oracle."""
+    pb = DecodeProblem(WIDE, T=6, streams=S, fmt=fmt, C=min(S * WIDE.k, WIDE.E) + 4)
+    st = pb.stack()
+    run = pb.run(stack=st, routing=True)
+    assert _check_run(pb, run) < 1e-5
+    pb.check_slots(st, run.table[1])
+    assert 0 < run.stats.misses < run.stats.lookups
+    st.close()
 
 
 def test_split_record_copies_match_the_oracle():

@@ -287,13 +287,11 @@ def test_layer_kernel_ring_fits_and_keeps_two_ctas_per_sm_where_it_can(shape, mx
 
 
 # ------------------------------------------------ streaming expert kernel --
-def _stream_launch(d, F, T, k, max_exp, mx, sms=148, wide=True):
+def _stream_launch(d, F, T, k, max_exp, mx, sms=148):
     """launch_stream's sizing, restated: stage bytes, tiles per item (gate/up,
-    down), stages, consumer groups and their size P, metadata, row-ref and x
-    offsets, grid.  A stage holds an item's codes and scales, 16 bytes of
-    tensor scales and, with activations in shared memory (T <= 2), a down
-    item's h rows.  Where only 4 or 5 stages fit (and up to 4 rows per pass),
-    two groups of five warps take two stages each."""
+    down), stages, consumer groups, metadata, row-ref and x offsets, grid.  A
+    stage holds an item's codes and scales, 16 bytes of tensor scales and, with
+    activations in shared memory (T <= 2), a down item's h rows."""
     sa = T <= 2
     xbytes = T * 4 * d if sa else 0
     hbytes = T * 4 * F if sa else 0
@@ -320,12 +318,8 @@ def _stream_launch(d, F, T, k, max_exp, mx, sms=148, wide=True):
     nc = ns // 2 if ns >= 6 else min(ns, 5)
     if nc > 4 and ns >= 6:
         nc = 4
-    ng = 1 if T <= 4 else 2
-    P = 3 if ng == 1 else 2
-    if wide and ng == 1 and 4 <= ns < 6:
-        nc, P = 2, 5
     ns = (2 if ns >= 2 * nc else 1) * nc
-    return dict(sb=sb, tpa=tpa, tpb=tpb, ns=ns, nc=nc, P=P, meta_off=ns * sb, rr_off=ns * sb + meta,
+    return dict(sb=sb, tpa=tpa, tpb=tpb, ns=ns, nc=nc, meta_off=ns * sb, rr_off=ns * sb + meta,
                 x_off=ns * sb + meta + rr, xbytes=xbytes, hbytes=hbytes,
                 smem=ns * sb + meta + rr + xbytes, nA=nA, nB=nB, cbA=8 * d, sbA=d // 2 if mx else d,
                 cbB=8 * F, sbB=F // 2 if mx else F)
@@ -360,10 +354,6 @@ def test_stream_items_fit_their_stage_and_stay_in_the_record(shape, mx):
         max_exp = min(T * shape.k, shape.E) + 1
         L = _stream_launch(shape.d, shape.F, T, shape.k, max_exp, mx)
         assert 2 <= L["ns"] <= 8 and 2 <= L["nc"] <= 7
-        # the launch's warps (consumers + the producer) and its register share:
-        # groups of five come two to a CTA (11 warps), else at most 16 warps
-        warps = L["P"] * L["nc"] + 1
-        assert warps <= 16 and L["nc"] <= (2 if L["P"] >= 5 else 5)
         # each stage serves one consumer warp: the uses of a stage are waited on in order
         assert L["ns"] % L["nc"] == 0
         for l in range(64):
