@@ -267,13 +267,16 @@ struct LookupSmem {
 // least recently used non-hit slot (the smallest stamps, found by block-wide
 // argmin rounds: stamps are unique, so round r takes the minimum above round
 // r-1's).  Same result as the sequential rule.  *t_read: time after the reads.
+// map_pre: this layer's E map entries already in shared memory, and the header
+// already in sm.clock / sm.nf (read while the top-k ran); or null.
 __device__ void lookup_batch(const Table &tab, int layer, int E, int n, LookupSmem &sm,
-                             unsigned long long *t_read) {
+                             unsigned long long *t_read, const int32_t *map_pre = nullptr) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int64_t keybase = (int64_t)layer * E;
     const int C = (int)tab.C;
     if (tab.scratch_base >= 0) {  // static split: resident set fixed, misses to scratch slots
-        for (int j = threadIdx.x; j < n; j += blockDim.x) sm.slot[j] = tab.map[keybase + sm.exp[j]];
+        for (int j = threadIdx.x; j < n; j += blockDim.x)
+            sm.slot[j] = map_pre ? map_pre[sm.exp[j]] : tab.map[keybase + sm.exp[j]];
         __syncthreads();
         if (threadIdx.x == 0 && t_read) *t_read = global_ns();
         if (warp == 0) {
@@ -297,8 +300,9 @@ __device__ void lookup_batch(const Table &tab, int layer, int E, int n, LookupSm
         return;
     }
     for (int i = threadIdx.x; i < kMaxSlotBits / 32; i += blockDim.x) sm.hitmap[i] = 0u;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) sm.slot[j] = tab.map[keybase + sm.exp[j]];
-    if (threadIdx.x == 0) { sm.clock = tab.hdr->clock; sm.nf = tab.hdr->next_free; }
+    for (int j = threadIdx.x; j < n; j += blockDim.x)
+        sm.slot[j] = map_pre ? map_pre[sm.exp[j]] : tab.map[keybase + sm.exp[j]];
+    if (threadIdx.x == 0 && !map_pre) { sm.clock = tab.hdr->clock; sm.nf = tab.hdr->next_free; }
     unsigned long long sv[kStampRegs];  // this thread's slots tid + 256*i
 #pragma unroll
     for (int i = 0; i < kStampRegs; ++i) {
@@ -484,13 +488,29 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     if (threadIdx.x == 0) t_elect = global_ns();
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    __shared__ LookupSmem sm;
+    // this layer's map entries (behind the x rows in dynamic shared memory) and
+    // the table header, loaded by the warps without a top-k row while the top-k
+    // runs (only this kernel writes the table, and the previous layer's launch
+    // is complete): the lookup then reads them without an L2 round trip
+    int32_t *s_map = reinterpret_cast<int32_t *>(xs + ((size_t)rows_per_chunk * a.d * 2 + 15) / 16);
+    const int tw = a.T < nw ? a.T : nw;  // warps with top-k rows
+    const int64_t keybase = (int64_t)a.layer * a.E;
+    auto preload = [&](int first) {
+        for (int e = (int)threadIdx.x - first; e < a.E; e += (int)blockDim.x - first) s_map[e] = a.tab.map[keybase + e];
+        if ((int)threadIdx.x == first) {
+            sm.clock = a.tab.hdr->clock;
+            sm.nf = a.tab.hdr->next_free;
+        }
+    };
+    if (tw < nw && warp >= tw) preload(32 * tw);
     for (int t = warp; t < a.T; t += nw) topk_row(a, t);
+    if (tw == nw) preload(0);
 
     // ---- distinct experts of the batch, ascending: a bitmap over E
     __shared__ uint32_t s_bits[kMaxE / 32];
     __shared__ int s_base[kMaxE / 32];
     __shared__ int s_njobs;
-    __shared__ LookupSmem sm;
     __shared__ int32_t s_cnt[kMaxK * kDecodeMaxRows];
     __shared__ int32_t s_off[kMaxK * kDecodeMaxRows];
     __shared__ int32_t s_idx[kMaxK * kDecodeMaxRows];
@@ -582,7 +602,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     if (threadIdx.x == 0) t_jobs = global_ns();
 
     // ---- cache lookup: one batch, ascending id
-    lookup_batch(a.tab, a.layer, a.E, njobs, sm, &t_read);
+    lookup_batch(a.tab, a.layer, a.E, njobs, sm, &t_read, s_map);
     const int nmiss = sm.nmiss;
     if (threadIdx.x == 0) {
         *a.ws.n_misses = nmiss;
@@ -862,7 +882,7 @@ __global__ void table_static_kernel(Table t, int L, int E, int per_layer) {
 
 template <int NV>
 cudaError_t launch_nv(const RouteArgs &a, int grid, cudaStream_t s) {
-    static bool configured = false;  // allow up to 64 KB of dynamic smem for the x chunk
+    static bool configured = false;  // allow up to 64 KB of dynamic smem (x chunk + map entries)
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(route_lookup_kernel<NV>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
@@ -872,7 +892,8 @@ cudaError_t launch_nv(const RouteArgs &a, int grid, cudaStream_t s) {
     int rows = (48 * 1024) / (a.d * 2);
     if (rows < 1) rows = 1;
     if (rows > a.T) rows = a.T;
-    const size_t smem = (size_t)rows * a.d * 2;
+    // the x chunk, then (16-byte aligned) the layer's E map entries
+    const size_t smem = (((size_t)rows * a.d * 2 + 15) & ~(size_t)15) + (size_t)a.E * 4;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kRouteThreads);
