@@ -175,7 +175,7 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
 // id, and a picked entry is masked out by a bit (not by overwriting its value),
 // so k distinct ids in [0, E) come out whatever the logits hold.
 template <int NVE>
-__device__ int topk_row_n(const RouteArgs &a, int t) {
+__device__ int topk_row_n(const RouteArgs &a, int t, int32_t *s_out) {
     const int lane = threadIdx.x & 31;
     const float *z = a.ws.z + (size_t)t * a.E;
     const int nv = (a.E + 31) >> 5;
@@ -231,16 +231,18 @@ __device__ int topk_row_n(const RouteArgs &a, int t) {
     if (lane < a.k) {
         a.ws.idx[t * a.k + rank] = my_idx;
         a.ws.gates[t * a.k + rank] = g;
+        if (s_out) s_out[t * a.k + rank] = my_idx;
     }
     return lane < a.k ? my_idx : -1;
 }
 
-__device__ int topk_row(const RouteArgs &a, int t) {
+// s_out: also the row's ids, ascending, in shared memory (or null).
+__device__ int topk_row(const RouteArgs &a, int t, int32_t *s_out = nullptr) {
     const int nv = (a.E + 31) >> 5;
-    if (nv <= 4) return topk_row_n<4>(a, t);
-    if (nv <= 8) return topk_row_n<8>(a, t);
-    if (nv <= 16) return topk_row_n<16>(a, t);
-    return topk_row_n<kMaxE / 32>(a, t);
+    if (nv <= 4) return topk_row_n<4>(a, t, s_out);
+    if (nv <= 8) return topk_row_n<8>(a, t, s_out);
+    if (nv <= 16) return topk_row_n<16>(a, t, s_out);
+    return topk_row_n<kMaxE / 32>(a, t, s_out);
 }
 
 constexpr int kLookupMax = kMaxK * kDecodeMaxRows;  // entries of one lookup batch (>= kMaxE)
@@ -303,11 +305,14 @@ __device__ void lookup_batch(const Table &tab, int layer, int E, int n, LookupSm
     for (int j = threadIdx.x; j < n; j += blockDim.x)
         sm.slot[j] = map_pre ? map_pre[sm.exp[j]] : tab.map[keybase + sm.exp[j]];
     if (threadIdx.x == 0 && !map_pre) { sm.clock = tab.hdr->clock; sm.nf = tab.hdr->next_free; }
-    unsigned long long sv[kStampRegs];  // this thread's slots tid + 256*i
+    // this thread's slots tid + 256 i (past C: slot C - 1's stamp, never used --
+    // the candidate test checks the slot; a select on the loaded value here
+    // would make every thread wait for its loads before the barrier below)
+    unsigned long long sv[kStampRegs];
 #pragma unroll
     for (int i = 0; i < kStampRegs; ++i) {
         const int sl = threadIdx.x + kRouteThreads * i;
-        sv[i] = sl < C ? tab.stamp[sl] : ~0ull;
+        sv[i] = tab.stamp[sl < C ? sl : C - 1];
     }
     __syncthreads();
     if (threadIdx.x == 0 && t_read) *t_read = global_ns();
@@ -503,8 +508,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
             sm.nf = a.tab.hdr->next_free;
         }
     };
+    // the selected ids, ascending per row, also go to shared memory (the job
+    // list reads them there, not back from global memory)
+    __shared__ int32_t s_idx[kMaxK * kDecodeMaxRows];
     if (tw < nw && warp >= tw) preload(32 * tw);
-    for (int t = warp; t < a.T; t += nw) topk_row(a, t);
+    for (int t = warp; t < a.T; t += nw) topk_row(a, t, s_idx);
     if (tw == nw) preload(0);
 
     // ---- distinct experts of the batch, ascending: a bitmap over E
@@ -513,7 +521,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     __shared__ int s_njobs;
     __shared__ int32_t s_cnt[kMaxK * kDecodeMaxRows];
     __shared__ int32_t s_off[kMaxK * kDecodeMaxRows];
-    __shared__ int32_t s_idx[kMaxK * kDecodeMaxRows];
     int32_t *s_exp = sm.exp;
     for (int i = threadIdx.x; i < kMaxE / 32; i += blockDim.x) s_bits[i] = 0u;
     __syncthreads();
@@ -523,7 +530,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
         // one row: its k ids are already distinct and ascending -- they (the
         // owned ones, with expert parallelism) are the jobs, one row each
         if (warp == 0) {
-            int e = lane < a.k ? a.ws.idx[lane] : 0;
+            int e = lane < a.k ? s_idx[lane] : 0;
             if (lane < a.k && (unsigned)e >= (unsigned)a.E) { route_fail(a.page, 1, e, a.E); e = 0; }
             const bool own = lane < a.k && e % a.ep_size == a.ep_rank;
             const unsigned ob = __ballot_sync(0xffffffffu, own);
@@ -540,8 +547,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
         __syncthreads();
     } else {
         for (int i = threadIdx.x; i < nsel; i += blockDim.x) {
-            const int e = a.ws.idx[i];
-            s_idx[i] = e;
+            const int e = s_idx[i];
             if ((unsigned)e >= (unsigned)a.E) route_fail(a.page, 1, e, a.E);
             else if (e % a.ep_size == a.ep_rank) atomicOr(&s_bits[e >> 5], 1u << (e & 31));
         }
