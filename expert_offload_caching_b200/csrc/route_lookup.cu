@@ -111,14 +111,17 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// z[t][e] for this warp's router row e (w: the row, already in registers).
-// x rows are staged in shared memory (xs) a chunk at a time, all loads in
-// flight together.  NV = 16-byte vectors per lane per row (d/256 rounded up).
+// z[t][e] for router row e, split over S consecutive warps of the CTA (warp
+// seg holds the seg-th S-th of the row in registers, w); their partial sums
+// meet in shared memory and are added in segment order.  x rows are staged in
+// shared memory (xs) a chunk at a time, all loads in flight together.  NV =
+// 16-byte vectors per lane of a segment (d/(256 S) rounded up).
 template <int NV>
 __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, bool has_row,
-                              uint4 *xs, int rows_per_chunk) {
-    const int lane = threadIdx.x & 31;
-    const int nvec = a.d >> 3;
+                              uint4 *xs, int rows_per_chunk, int S, int seg) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nvec = a.d >> 3, segv = nvec / S, v0 = seg * segv;
+    __shared__ float s_part[kRouteThreads / 32][4];
     for (int t0 = 0; t0 < a.T; t0 += rows_per_chunk) {
         const int nr = a.T - t0 < rows_per_chunk ? a.T - t0 : rows_per_chunk;
         const uint4 *xg = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.d);
@@ -137,13 +140,14 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
             a.ws.xh[(size_t)t * 2 * a.d + c] = hi;
             a.ws.xh[(size_t)t * 2 * a.d + a.d + c] = lo;
         }
-        if (has_row) {
-            for (int r0 = 0; r0 < nr; r0 += 4) {
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int r0 = 0; r0 < nr; r0 += 4) {  // (the same trip count in every warp of the CTA)
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (has_row) {
 #pragma unroll
                 for (int i = 0; i < NV; ++i) {
-                    const int v = lane + 32 * i;
-                    if (v < nvec) {
+                    const int vl = lane + 32 * i;
+                    if (vl < segv) {
+                        const int v = v0 + vl;
                         float wf[8];
                         bf16x8_to_f32(w[i], wf);
 #pragma unroll
@@ -157,11 +161,26 @@ __device__ void router_logits(const RouteArgs &a, const uint4 (&w)[NV], int e, b
                         }
                     }
                 }
+            }
+            float sum[4];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const float sum = warp_sum(acc[r]);
-                    if (lane == 0 && r0 + r < nr) a.ws.z[(size_t)(t0 + r0 + r) * a.E + e] = sum;
+            for (int r = 0; r < 4; ++r) sum[r] = warp_sum(acc[r]);
+            if (S == 1) {
+                if (has_row && lane == 0)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        if (r0 + r < nr) a.ws.z[(size_t)(t0 + r0 + r) * a.E + e] = sum[r];
+            } else {
+                if (lane == 0)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) s_part[warp][r] = sum[r];
+                __syncthreads();
+                if (has_row && seg == 0 && lane < 4 && r0 + lane < nr) {
+                    float z = 0.f;
+                    for (int q = 0; q < S; ++q) z += s_part[warp + q][lane];
+                    a.ws.z[(size_t)(t0 + r0 + lane) * a.E + e] = z;
                 }
+                __syncthreads();  // s_part is rewritten by the next row group
             }
         }
         __syncthreads();
@@ -447,21 +466,24 @@ __device__ void publish_events(HostPage *page, int base, const LookupSmem &sm, i
 }
 
 template <int NV>
-__global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a, int rows_per_chunk) {
+// split: warps per router row (1, 2, 4 or 8; d/8 divisible by it): more CTAs
+// pull the router's bytes, and each holds fewer of them in flight.
+__global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a, int rows_per_chunk, int split) {
     extern __shared__ __align__(16) uint4 xs[];  // x rows of one chunk (bf16)
     const unsigned long long t_entry = global_ns();  // early: launched before the previous layer ends
     unsigned long long t_logits = 0, t_elect = 0, t_topk = 0, t_jobs = 0, t_read = 0, t_table = 0;
-    // static data first: this warp's router row and the next layer's rows (L2)
-    const int e_row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    // static data first: this warp's segment of its router row and the next layer's rows (L2)
+    const int seg = (int)(threadIdx.x >> 5) % split;
+    const int e_row = blockIdx.x * ((blockDim.x >> 5) / split) + (int)(threadIdx.x >> 5) / split;
     const bool has_row = e_row < a.E;
     uint4 w[NV];
     {
-        const int lane = threadIdx.x & 31, nvec = a.d >> 3;
-        const uint4 *wrow = reinterpret_cast<const uint4 *>(a.Wr + (size_t)(has_row ? e_row : 0) * a.d);
+        const int lane = threadIdx.x & 31, segv = (a.d >> 3) / split;
+        const uint4 *wrow = reinterpret_cast<const uint4 *>(a.Wr + (size_t)(has_row ? e_row : 0) * a.d) + seg * segv;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
             const int v = lane + 32 * i;
-            w[i] = (has_row && v < nvec) ? ld_nc16(wrow + v) : make_uint4(0, 0, 0, 0);
+            w[i] = (has_row && v < segv) ? ld_nc16(wrow + v) : make_uint4(0, 0, 0, 0);
         }
     }
     if (a.Wr_next != nullptr) {  // next layer's router rows -> L2
@@ -477,7 +499,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_lookup_kernel(RouteArgs a
     pdl_launch_dependents();
     const unsigned long long t_start = global_ns();  // phases are timed from here
     if (threadIdx.x == 0) span_mark(a.span, 0);
-    router_logits<NV>(a, w, e_row, has_row, xs, rows_per_chunk);
+    router_logits<NV>(a, w, e_row, has_row, xs, rows_per_chunk, split, seg);
 
     __shared__ int s_last;
     __syncthreads();
@@ -887,7 +909,7 @@ __global__ void table_static_kernel(Table t, int L, int E, int per_layer) {
 }
 
 template <int NV>
-cudaError_t launch_nv(const RouteArgs &a, int grid, cudaStream_t s) {
+cudaError_t launch_nv(const RouteArgs &a, int grid, int split, cudaStream_t s) {
     static bool configured = false;  // allow up to 64 KB of dynamic smem (x chunk + map entries)
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(route_lookup_kernel<NV>,
@@ -910,21 +932,35 @@ cudaError_t launch_nv(const RouteArgs &a, int grid, cudaStream_t s) {
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, route_lookup_kernel<NV>, a, rows);
+    return cudaLaunchKernelEx(&cfg, route_lookup_kernel<NV>, a, rows, split);
 }
 
 }  // namespace
 
 cudaError_t launch_route_lookup(const RouteArgs &a, cudaStream_t s) {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
     const int warps = kRouteThreads / 32;
-    const int grid = (a.E + warps - 1) / warps;  // one router row per warp
-    const int nv = ((a.d >> 3) + 31) >> 5;      // 16-byte vectors per lane per row
-    if (nv <= 1) return launch_nv<1>(a, grid, s);
-    if (nv <= 2) return launch_nv<2>(a, grid, s);
-    if (nv <= 4) return launch_nv<4>(a, grid, s);
-    if (nv <= 8) return launch_nv<8>(a, grid, s);
-    if (nv <= 12) return launch_nv<12>(a, grid, s);
-    if (nv <= 16) return launch_nv<16>(a, grid, s);
+    const int nvec = a.d >> 3;
+    // warps per router row: split while the grid stays within one CTA per SM
+    // and every lane keeps at least one 16-byte vector of its segment
+    int split = 1;
+    while (split < 8 && (int64_t)a.E * 2 * split <= (int64_t)warps * sms && nvec % (2 * split) == 0 &&
+           nvec / (2 * split) >= 32)
+        split *= 2;
+    const int grid = (a.E + warps / split - 1) / (warps / split);
+    const int nv = (nvec / split + 31) >> 5;  // 16-byte vectors per lane per segment
+    if (nv <= 1) return launch_nv<1>(a, grid, split, s);
+    if (nv <= 2) return launch_nv<2>(a, grid, split, s);
+    if (nv <= 4) return launch_nv<4>(a, grid, split, s);
+    if (nv <= 8) return launch_nv<8>(a, grid, split, s);
+    if (nv <= 12) return launch_nv<12>(a, grid, split, s);
+    if (nv <= 16) return launch_nv<16>(a, grid, split, s);
     return cudaErrorInvalidValue;
 }
 
