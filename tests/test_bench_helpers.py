@@ -70,3 +70,28 @@ def test_replica_pool_records():
     assert bench.replica_pool_records(L, E, 1) == L * E
     assert bench.replica_pool_records(L, E, 8) == L * E // 8
     assert bench.replica_pool_records(1, 16, 8) == bench.DISTINCT_RECORDS  # never below the distinct records
+
+
+def test_gpu_launches_count_the_hit_launch_unless_the_layer_kernel_ran():
+    """Default decode path: route + hit launch per call and one launch per miss
+    are all launches of their own; with the layer kernel the hit-phase class is
+    a part of its launches and is not counted again."""
+    default = _stats(kernel_launches=_per_class({abi.MOE_K_ROUTE: 48, abi.MOE_K_LAYER_HITS: 48,
+                                                 abi.MOE_K_MISS: 126}))
+    assert bench.launch_count(default, None) == 48 + 48 + 126
+    layer = _stats(kernel_launches=_per_class({abi.MOE_K_ROUTE: 48, abi.MOE_K_LAYER: 48,
+                                               abi.MOE_K_LAYER_HITS: 48}))
+    assert bench.launch_count(layer, None) == 96
+    split = _stats(kernel_launches=_per_class({abi.MOE_K_ROUTE: 48, abi.MOE_K_LAYER_HITS: 48,
+                                               abi.MOE_K_GATEUP: 126, abi.MOE_K_DOWN: 126}))
+    assert bench.launch_count(split, None) == 48 + 48 + 252
+    # without the timing pass: the default path's structure from the counters
+    st = abi.moe_stats()
+    st.forward_calls, st.misses = 48, 126
+    assert bench.launch_count(None, st) == 2 * 48 + 126
+
+
+def test_kernel_names_cover_every_class():
+    assert len(abi.KERNEL_NAMES) == abi.MOE_K_COUNT
+    assert abi.KERNEL_NAMES[abi.MOE_K_MISS] == "expert_miss"
+    assert abi.KERNEL_NAMES[abi.MOE_K_LAYER_HITS] == "expert_hits"

@@ -436,3 +436,47 @@ def test_topk_order_key_preserves_the_selection_order():
     same = np.where(vals == 0, np.float32(0), vals)
     assert np.array_equal(back.view(np.uint32), same.view(np.uint32))  # exact inverse
 
+
+
+def _route_split(E, d, sms=148, warps=8):
+    """launch_route_lookup's choice, restated: warps per router row (1, 2, 4 or
+    8) while the grid stays within one CTA per SM, the row's 16-byte vectors
+    divide evenly and every lane keeps at least one of its segment."""
+    nvec = d // 8
+    split = 1
+    while split < 8 and E * 2 * split <= warps * sms and nvec % (2 * split) == 0 and nvec // (2 * split) >= 32:
+        split *= 2
+    grid = -(-E // (warps // split))
+    nv = -(-(nvec // split) // 32)
+    return split, grid, nv
+
+
+@pytest.mark.parametrize("E", [1, 2, 8, 40, 100, 128, 256, 512, 1000, 1024])
+@pytest.mark.parametrize("d", [64, 192, 256, 960, 2048, 2880, 4096])
+def test_route_row_split_covers_every_row_and_vector_once(E, d):
+    """Every (row, 16-byte vector) of the router is loaded by exactly one lane
+    of one warp, segments of a row are consecutive warps of one CTA (their
+    partial sums meet in that CTA's shared memory, slots warp .. warp + S - 1),
+    the grid fits one CTA per SM once split, and NV covers a segment."""
+    split, grid, nv = _route_split(E, d)
+    assert split in (1, 2, 4, 8) and nv in range(1, 17)
+    assert split == 1 or grid <= 148
+    nvec = d // 8
+    assert nvec % split == 0
+    segv = nvec // split
+    assert nv * 32 >= segv
+    seen = {}
+    for b in range(grid):
+        for warp in range(8):
+            seg, row = warp % split, b * (8 // split) + warp // split
+            if row >= E:
+                continue
+            assert warp - seg + split <= 8  # the row's warps (its partial-sum slots) lie in the CTA
+            for lane in range(32):
+                for i in range(nv):
+                    v = lane + 32 * i
+                    if v < segv:
+                        key = (row, seg * segv + v)
+                        assert key not in seen
+                        seen[key] = (b, warp, lane)
+    assert len(seen) == E * nvec
