@@ -350,8 +350,9 @@ def test_stream_items_fit_their_stage_and_stay_in_the_record(shape, mx):
     fmt = abi.MOE_FMT_MXFP4 if mx else abi.MOE_FMT_NVFP4
     dims = abi.make_dims(shape.L, shape.E, shape.k, shape.d, shape.F, shape.shared, weight_format=fmt)
     off = abi.moe_record_layout(dims)  # w13 codes, w13 scales, w2 codes, w2 scales, tensor scales, bytes
-    for T in (1, 4, 16, 32):
-        max_exp = min(T * shape.k, shape.E) + 1
+    # the hit launch (every selected expert + the shared one), and a miss's own
+    # launch (one expert: its gate/up, then its down tiles)
+    for T, max_exp in [(T, m) for T in (1, 4, 16, 32) for m in (min(T * shape.k, shape.E) + 1, 1)]:
         L = _stream_launch(shape.d, shape.F, T, shape.k, max_exp, mx)
         assert 2 <= L["ns"] <= 8 and 2 <= L["nc"] <= 7
         # each stage serves one consumer warp: the uses of a stage are waited on in order
